@@ -1,0 +1,232 @@
+/*
+ * csa.h -- C ABI of the CSA / HCA attention hot path (DeepSeek-V4 hybrid attention)
+ * for one NVIDIA B200 (sm_100a).
+ *
+ * Sources, cited by page title and section:
+ *   [P1] 【论文解读】DeepSeek-V4, 一、模型架构 (三) 混合注意力架构：CSA + HCA:
+ *        1(1) 压缩 KV Entries (overlapped compression), 1(2) Lightning Indexer 稀疏选择
+ *        (index score, visibility, top-k), 1(3) Shared Key-Value MQA, 2(1)/2(2) HCA,
+ *        3(1) query / KV RMSNorm, 3(2) partial RoPE and output rotation at -t,
+ *        3(3) sliding window, 3(4) attention sink.
+ *   [P1'] same page, 二、基础设施 (四) FP4 量化感知训练: the indexer's QK path in FP4.
+ *
+ * Conventions shared by every call
+ *   - Every tensor pointer is device memory owned by the caller; the library never
+ *     allocates or frees device memory. Scratch comes from a caller-provided workspace
+ *     whose size csa_workspace_size() returns.
+ *   - Layouts are dense row-major with the shapes given per argument. Pointers must be
+ *     16-byte aligned; c is a multiple of 64 (or exactly 64 for fp32 inputs), 0 <= r <= c,
+ *     r even.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *     and return once the kernels are queued. No host synchronisation happens.
+ *   - Arguments are validated on the host before any launch; on error nothing is
+ *     launched and a status is returned (csa_last_error() gives a one-line reason for
+ *     the calling thread). CSA_ERR_CUDA reports a launch failure seen by
+ *     cudaGetLastError() right after queueing.
+ *   - On the device, top-k indices equal to -1 (or outside [0, N_cap)) are skipped.
+ *     Nothing traps.
+ *   - Positions (q_pos, win_pos0) are int64 device arrays. A query at position t sees the
+ *     compressed entries s < min(floor(t/m), N_cap) ([P1] 1(2)) and the window tokens
+ *     max(t-n_win+1, 0) .. t, its own token included ([P1] 3(3)); the window buffer of
+ *     request b holds token win_pos0[b]+j in row j and must cover those positions.
+ *   - RoPE ([P1] 3(2)): the last r dims, adjacent pairs (2p, 2p+1) of that slice turned by
+ *     pos * rope_base^(-2p/r); compressed entry i sits at position m*i. RMSNorm ([P1] 3(1)):
+ *     x / sqrt(mean(x^2) + rms_eps) * gamma (gamma = 1 when the weight pointer is NULL).
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CSA_OK = 0,
+  CSA_ERR_INVALID_ARG = 1, /* a pointer, size or alignment the call cannot accept */
+  CSA_ERR_UNSUPPORTED = 2, /* a valid shape / dtype combination this build does not implement */
+  CSA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than csa_workspace_size() */
+  CSA_ERR_CUDA = 4         /* the CUDA runtime reported an error while queueing */
+} csa_status;
+
+typedef enum {
+  CSA_F32 = 0,               /* IEEE binary32 */
+  CSA_BF16 = 1,              /* bfloat16 */
+  CSA_FP8_E4M3_ROWSCALE = 2, /* OCP e4m3 codes, one fp32 scale per row (value = code * scale) */
+  CSA_MXFP4 = 3              /* OCP MXFP4: e2m1 pairs per byte (element 2j in the low nibble)
+                                and one e8m0 scale byte per 32 elements */
+} csa_dtype;
+
+/* Method constants, passed by pointer, read on the host during the call only. */
+typedef struct {
+  int32_t m;           /* tokens per compressed entry: 4 (CSA) or m' = 128 (HCA)        */
+  int32_t overlap;     /* 1: CSA a/b overlapped compression; 0: HCA single branch        */
+  int32_t c;           /* head dim of queries and compressed KV rows (512 in the models) */
+  int32_t rope_dims;   /* r: RoPE on the last r dims (64)                                */
+  float rope_base;     /* 10000                                                          */
+  float rms_eps;       /* 1e-6                                                           */
+  float sm_scale;      /* logit scale; <= 0 means 1/sqrt(c)                              */
+  int32_t n_heads;     /* attention query heads H (64 Flash / 128 Pro)                   */
+  int32_t n_idx_heads; /* indexer heads H_I (64)                                         */
+  int32_t d_idx;       /* indexer head dim d_I (128)                                     */
+  int32_t topk;        /* k (512 Flash / 1024 Pro), at most 2048                         */
+  int32_t n_win;       /* sliding window n_win (128)                                     */
+} csa_params;
+
+/* Which call a workspace is sized for (csa_workspace_size's `entry`). */
+typedef enum {
+  CSA_WS_INDEX_TOPK = 1,
+  CSA_WS_TOPK = 2,
+  CSA_WS_SPARSE_MQA = 3,
+  CSA_WS_HCA_MQA = 4,
+  CSA_WS_FORWARD = 5
+} csa_ws_entry;
+
+/*
+ * Stage 1 -- token-level KV compression ([P1] 1(1) overlapped; 2(1) non-overlapped),
+ * optionally finalised with RMSNorm and RoPE at position m*i ([P1] 3(1), 3(2)).
+ *
+ * For each request b and new entry i < n_tok/m, channel j:
+ *   CSA: softmax over the 2m logits Za[b, m*i+r, j] + bias[r, j] and
+ *        Zb[b, m*(i-1)+r, j] + bias[m+r, j] (r < m), weighted sum of Ca / Cb at the same
+ *        tokens. For i = 0 the b-branch reads prev_Cb / prev_Zb [B, m, c] (the last m
+ *        tokens before this chunk); if those are NULL the chunk starts the sequence and the
+ *        b-logits are -inf (values 0).
+ *   HCA (overlap = 0): softmax over the m logits Za[b, m*i+r, j] + bias[r, j], weighted sum
+ *        of Ca; Cb, Zb, prev_* must be NULL.
+ * The entry is written to out_cache[b, first_entry + i, :] ([B, n_cap, c]); with
+ * finalize = 1 it is RMSNorm'd (weight kv_rms_w [c] or NULL) and rotated at position
+ * m*(first_entry + i). n_tok must be a multiple of m and first_entry + n_tok/m <= n_cap.
+ * io: CSA_F32 or CSA_BF16 for every tensor (math is fp32). Ca/Cb/Za/Zb: [B, n_tok, c];
+ * bias: [2m, c] (CSA) or [m, c] (HCA).
+ */
+csa_status csa_compress(const csa_params* p, csa_dtype io, int32_t B, int64_t n_tok,
+                        int64_t first_entry, int64_t n_cap, const void* Ca, const void* Cb,
+                        const void* Za, const void* Zb, const void* bias, const void* prev_Cb,
+                        const void* prev_Zb, const void* kv_rms_w, int32_t finalize,
+                        void* out_cache, void* stream);
+
+/*
+ * Stage 2 -- lightning-indexer scores ([P1] 1(2)):
+ *   I[b,t,s] = sum_h w[b,t,h] * ReLU(qI[b,t,h,:] . KI[b,s,:]),  s < n_vis(b,t),
+ * written to out_scores [B, T, N_cap] fp32. Values at s >= n_vis are left unwritten.
+ * kdt selects the key format and with it the query format:
+ *   CSA_F32:  qI f32 [B,T,H_I,d_I],  KI f32 [B,N_cap,d_I]
+ *   CSA_BF16: qI bf16,               KI bf16
+ *   CSA_FP8_E4M3_ROWSCALE: qI bf16,  KI e4m3 codes [B,N_cap,d_I] + KI_scale f32 [B,N_cap]
+ *   CSA_MXFP4 ([P1'] FP4 QK path): qI [B,T,H_I,d_I/2] bytes + qI_scale [B,T,H_I,d_I/32],
+ *             KI [B,N_cap,d_I/2] bytes + KI_scale [B,N_cap,d_I/32] (e8m0)
+ * w: f32 [B,T,H_I]. q_pos: int64 [B,T]. Scores are fp32 sums of exact products.
+ */
+csa_status csa_index_scores(const csa_params* p, csa_dtype kdt, int32_t B, int32_t T,
+                            int64_t N_cap, const void* qI, const void* qI_scale, const float* w,
+                            const void* KI, const void* KI_scale, const int64_t* q_pos,
+                            float* out_scores, void* stream);
+
+/*
+ * Stage 3 -- top-k selector ([P1] 1(2), C_t^SprsComp): for every (b,t), the indices of the
+ * k largest scores[b,t,s] over s < n_vis(b,t), ordered by (score descending, index
+ * ascending); slots past n_vis hold -1. scores: f32 [B,T,N_cap]; out_idx: int32 [B,T,k].
+ * Deterministic: the result depends only on the scores. -0.0 counts as +0.0.
+ */
+csa_status csa_topk(const csa_params* p, int32_t B, int32_t T, int64_t N_cap,
+                    const float* scores, const int64_t* q_pos, int32_t* out_idx, void* ws,
+                    size_t ws_bytes, void* stream);
+
+/* Stages 2 + 3 in one call. out_scores may be NULL (the scores then live in the workspace). */
+csa_status csa_index_topk(const csa_params* p, csa_dtype kdt, int32_t B, int32_t T,
+                          int64_t N_cap, const void* qI, const void* qI_scale, const float* w,
+                          const void* KI, const void* KI_scale, const int64_t* q_pos,
+                          int32_t* out_idx, float* out_scores, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/*
+ * Stage 4 -- shared-KV MQA over the selected entries plus the window ([P1] 1(3), 3(1)-(4)).
+ * For every (b, t, h): q_hat = RoPE_t(RMSNorm(q[b,t,h,:]) * q_rms_w); the KV rows are
+ * kv_cache[b, idx[b,t,j], :] for every valid j followed by the window rows; key = value;
+ *   o = sum_j e^{z_j} row_j / (sum_j e^{z_j} + e^{sink[h]}),  z_j = sm_scale * q_hat . row_j,
+ * then out[b,t,h,:] = RoPE_{-t}(o). sink may be NULL (no sink). io: CSA_F32 or CSA_BF16 for
+ * q [B,T,H,c], kv_cache [B,N_cap,c], win_kv [B,L_raw,c] and out [B,T,H,c]; q_rms_w [c] or
+ * NULL (same dtype as io). idx: int32 [B,T,k].
+ */
+csa_status csa_sparse_mqa(const csa_params* p, csa_dtype io, int32_t B, int32_t T,
+                          const void* q, const int64_t* q_pos, const void* kv_cache,
+                          int64_t N_cap, const int32_t* idx, const void* win_kv, int64_t L_raw,
+                          const int64_t* win_pos0, const float* sink, const void* q_rms_w,
+                          void* out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * HCA core attention ([P1] 2(2), 3(1)-(4)): as csa_sparse_mqa, with the KV rows being every
+ * visible entry s < min(floor(t/m), N_cap) (m = p->m, e.g. 128) followed by the window.
+ */
+csa_status hca_dense_mqa(const csa_params* p, csa_dtype io, int32_t B, int32_t T,
+                         const void* q, const int64_t* q_pos, const void* kv_cache,
+                         int64_t N_cap, const void* win_kv, int64_t L_raw,
+                         const int64_t* win_pos0, const float* sink, const void* q_rms_w,
+                         void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Inputs of the fused CSA layer call. Pointers as in the stage calls above. */
+typedef struct {
+  /* optional compression of a new chunk into kv_cache (skipped when Ca == NULL) */
+  int64_t n_tok, first_entry;
+  const void *Ca, *Cb, *Za, *Zb, *bias, *prev_Cb, *prev_Zb, *kv_rms_w;
+  /* indexer */
+  csa_dtype idx_dtype;
+  const void *qI, *qI_scale;
+  const float* w;
+  const void *KI, *KI_scale;
+  /* attention */
+  const void* q;
+  const void* q_rms_w;
+  const int64_t* q_pos;
+  void* kv_cache;
+  int64_t N_cap;
+  const void* win_kv;
+  int64_t L_raw;
+  const int64_t* win_pos0;
+  const float* sink;
+  /* outputs */
+  int32_t* out_idx;  /* [B,T,k], required */
+  float* out_scores; /* [B,T,N_cap] or NULL */
+  void* out;         /* [B,T,H,c] */
+} csa_forward_args;
+
+/*
+ * The CSA layer's hot path in one call: [compress the chunk into kv_cache] -> index scores
+ * -> top-k -> sparse MQA, queued on `stream` in that order. io is the dtype of q, KV rows,
+ * chunk inputs and out.
+ */
+csa_status csa_forward(const csa_params* p, csa_dtype io, int32_t B, int32_t T,
+                       const csa_forward_args* a, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Bytes of workspace the call `entry` needs for these sizes (0 if none). Returns 0 and
+ * sets csa_last_error() on invalid sizes. kdt: the indexer key format (for the index calls).
+ */
+size_t csa_workspace_size(const csa_params* p, int32_t entry, csa_dtype kdt, int32_t B,
+                          int32_t T, int64_t N_cap);
+
+/* Static text of a status code. */
+const char* csa_status_string(csa_status s);
+
+/* One-line reason of the last non-OK status returned on the calling thread ("" if none). */
+const char* csa_last_error(void);
+
+/*
+ * Timing hook for measurement. After a call with count > 0, every launch of the
+ * indexer-score kernel records before[i] on the call's stream right before it and after[i]
+ * right after it, i = 0, 1, 2, ... modulo count (cudaEvent_t handles owned by the caller).
+ * count = 0 clears the hook. Not thread-safe; meant for benchmarks.
+ */
+void csa_set_index_timing_events(void* const* before, void* const* after, int32_t count);
+
+/* Library version string. */
+const char* csa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_H_ */

@@ -1,0 +1,427 @@
+// C ABI of libcsa (declared in include/csa.h): host-side validation, workspace layout and
+// dispatch to the stage kernels. Nothing is launched unless every argument checks out.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace {
+
+thread_local char g_err[256] = "";
+
+csa_status fail(csa_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+csa_status ok() {
+  g_err[0] = '\0';
+  return CSA_OK;
+}
+
+csa_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return CSA_OK;
+  return fail(CSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define REQUIRE(cond, ...)                                  \
+  do {                                                      \
+    if (!(cond)) return fail(CSA_ERR_INVALID_ARG, __VA_ARGS__); \
+  } while (0)
+#define REQUIRE_PTR(p) REQUIRE((p) != nullptr && aligned16(p), "%s must be a non-NULL 16-byte aligned device pointer", #p)
+#define OPTIONAL_PTR(p) REQUIRE((p) == nullptr || aligned16(p), "%s must be 16-byte aligned", #p)
+
+constexpr size_t kAlign = 256;
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+csa_status check_params(const csa_params* p) {
+  REQUIRE(p != nullptr, "params is NULL");
+  REQUIRE(p->m >= 1, "m must be >= 1 (got %d)", p->m);
+  REQUIRE(p->c >= 64 && p->c % 64 == 0, "c must be a positive multiple of 64 (got %d)", p->c);
+  REQUIRE(p->rope_dims >= 0 && p->rope_dims <= p->c && p->rope_dims % 2 == 0,
+          "rope_dims must be even and in [0, c] (got %d)", p->rope_dims);
+  REQUIRE(std::isfinite(p->rms_eps) && p->rms_eps >= 0.f, "rms_eps must be finite and >= 0");
+  REQUIRE(std::isfinite(p->rope_base) && p->rope_base > 0.f, "rope_base must be > 0");
+  REQUIRE(std::isfinite(p->sm_scale), "sm_scale must be finite");
+  REQUIRE(p->n_win >= 0, "n_win must be >= 0");
+  return CSA_OK;
+}
+
+csa_status check_attn(const csa_params* p) {
+  REQUIRE(p->n_heads >= 1, "n_heads must be >= 1");
+  REQUIRE(p->n_heads <= 16 || p->n_heads % 16 == 0,
+          "n_heads must be <= 16 or a multiple of 16 (got %d)", p->n_heads);
+  if (p->c > 512) return fail(CSA_ERR_UNSUPPORTED, "attention supports c <= 512 (got %d)", p->c);
+  return CSA_OK;
+}
+
+csa_status check_index(const csa_params* p, csa_dtype kdt) {
+  REQUIRE(p->n_idx_heads >= 1, "n_idx_heads must be >= 1");
+  REQUIRE(p->d_idx >= 32 && p->d_idx % 32 == 0, "d_idx must be a positive multiple of 32");
+  REQUIRE(kdt == CSA_F32 || kdt == CSA_BF16 || kdt == CSA_FP8_E4M3_ROWSCALE || kdt == CSA_MXFP4,
+          "unknown indexer key dtype %d", (int)kdt);
+  const size_t qbytes = (size_t)p->n_idx_heads * p->d_idx * 4 + p->n_idx_heads * 4;
+  if (qbytes > 48 * 1024)
+    return fail(CSA_ERR_UNSUPPORTED, "n_idx_heads * d_idx too large for the indexer (%d x %d)",
+                p->n_idx_heads, p->d_idx);
+  return CSA_OK;
+}
+
+csa_status check_topk(const csa_params* p) {
+  REQUIRE(p->topk >= 1 && p->topk <= csa::kMaxTopk, "topk must be in [1, %d] (got %d)",
+          csa::kMaxTopk, p->topk);
+  return CSA_OK;
+}
+
+csa_status check_sizes(int32_t B, int32_t T, int64_t N_cap) {
+  REQUIRE(B >= 0 && T >= 0, "B and T must be >= 0");
+  REQUIRE(N_cap >= 0 && N_cap <= INT32_MAX, "N_cap must be in [0, 2^31)");
+  REQUIRE((int64_t)B * T <= 65535 * 64, "B*T too large");
+  return CSA_OK;
+}
+
+float eff_scale(const csa_params* p) {
+  return p->sm_scale > 0.f ? p->sm_scale : 1.0f / std::sqrt((float)p->c);
+}
+
+#define TRY(x)                              \
+  do {                                      \
+    csa_status _s = (x);                    \
+    if (_s != CSA_OK) return _s;            \
+  } while (0)
+
+struct TimingHook {
+  std::vector<cudaEvent_t> before, after;
+  size_t next = 0;
+};
+TimingHook g_timing;
+
+csa::MqaArgs make_mqa(const csa_params* p, int32_t B, int32_t T, const void* q,
+                      const int64_t* q_pos, const void* kv, int64_t N_cap, const int32_t* idx,
+                      int k, const void* win, int64_t L_raw, const int64_t* pos0,
+                      const float* sink, const void* q_rms_w, void* out) {
+  csa::MqaArgs a{};
+  a.B = B; a.T = T; a.m = p->m; a.H = p->n_heads; a.c = p->c; a.rope_dims = p->rope_dims;
+  a.n_win = p->n_win; a.k = k; a.n_cap = N_cap; a.l_raw = L_raw; a.rope_base = p->rope_base;
+  a.eps = p->rms_eps; a.scale = eff_scale(p); a.q = q; a.kv = kv; a.win = win;
+  a.q_rms_w = q_rms_w; a.idx = idx; a.q_pos = q_pos; a.win_pos0 = pos0; a.sink = sink;
+  a.out = out;
+  return a;
+}
+
+csa_status check_mqa_args(const csa_params* p, csa_dtype io, int32_t B, int32_t T,
+                          const void* q, const int64_t* q_pos, const void* kv, int64_t N_cap,
+                          const void* win, int64_t L_raw, const int64_t* pos0,
+                          const float* sink, const void* q_rms_w, const void* out) {
+  TRY(check_params(p));
+  TRY(check_attn(p));
+  TRY(check_sizes(B, T, N_cap));
+  REQUIRE(io == CSA_F32 || io == CSA_BF16, "attention io dtype must be CSA_F32 or CSA_BF16");
+  REQUIRE(L_raw >= 0, "L_raw must be >= 0");
+  if ((int64_t)B * T == 0) return CSA_OK;
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(q_pos);
+  REQUIRE_PTR(out);
+  if (N_cap > 0) REQUIRE_PTR(kv);
+  if (p->n_win > 0) {
+    REQUIRE(L_raw >= 1, "n_win > 0 needs window rows (L_raw >= 1)");
+    REQUIRE_PTR(win);
+    REQUIRE_PTR(pos0);
+  }
+  OPTIONAL_PTR(sink);
+  OPTIONAL_PTR(q_rms_w);
+  return CSA_OK;
+}
+
+csa_status check_index_args(const csa_params* p, csa_dtype kdt, int32_t B, int32_t T,
+                            int64_t N_cap, const void* qI, const void* qI_scale, const float* w,
+                            const void* KI, const void* KI_scale, const int64_t* q_pos) {
+  TRY(check_params(p));
+  TRY(check_index(p, kdt));
+  TRY(check_sizes(B, T, N_cap));
+  if ((int64_t)B * T == 0) return CSA_OK;
+  REQUIRE_PTR(qI);
+  REQUIRE_PTR(w);
+  REQUIRE_PTR(q_pos);
+  if (N_cap > 0) REQUIRE_PTR(KI);
+  if (kdt == CSA_FP8_E4M3_ROWSCALE && N_cap > 0) REQUIRE_PTR(KI_scale);
+  if (kdt == CSA_MXFP4) {
+    REQUIRE_PTR(qI_scale);
+    if (N_cap > 0) REQUIRE(KI_scale != nullptr, "KI_scale is required for MXFP4 keys");
+  }
+  return CSA_OK;
+}
+
+csa::IndexArgs make_index(const csa_params* p, csa_dtype kdt, int32_t B, int32_t T,
+                          int64_t N_cap, const void* qI, const void* qI_scale, const float* w,
+                          const void* KI, const void* KI_scale, const int64_t* q_pos,
+                          float* scores) {
+  csa::IndexArgs a{};
+  a.B = B; a.T = T; a.m = p->m; a.n_idx_heads = p->n_idx_heads; a.d_idx = p->d_idx;
+  a.kdt = (int)kdt; a.n_cap = N_cap; a.qI = qI; a.qI_scale = qI_scale; a.KI = KI;
+  a.KI_scale = KI_scale; a.w = w; a.q_pos = q_pos; a.scores = scores;
+  return a;
+}
+
+size_t scores_bytes(int32_t B, int32_t T, int64_t N_cap) {
+  return round_up((size_t)B * T * (size_t)N_cap * sizeof(float));
+}
+
+}  // namespace
+
+namespace csa {
+void timing_before(cudaStream_t st) {
+  if (!g_timing.before.empty())
+    cudaEventRecord(g_timing.before[g_timing.next % g_timing.before.size()], st);
+}
+void timing_after(cudaStream_t st) {
+  if (!g_timing.after.empty()) {
+    cudaEventRecord(g_timing.after[g_timing.next % g_timing.after.size()], st);
+    ++g_timing.next;
+  }
+}
+}  // namespace csa
+
+extern "C" {
+
+const char* csa_version(void) { return "libcsa 0.1 (sm_100a)"; }
+
+const char* csa_last_error(void) { return g_err; }
+
+const char* csa_status_string(csa_status s) {
+  switch (s) {
+    case CSA_OK: return "CSA_OK";
+    case CSA_ERR_INVALID_ARG: return "CSA_ERR_INVALID_ARG";
+    case CSA_ERR_UNSUPPORTED: return "CSA_ERR_UNSUPPORTED";
+    case CSA_ERR_WORKSPACE: return "CSA_ERR_WORKSPACE";
+    case CSA_ERR_CUDA: return "CSA_ERR_CUDA";
+  }
+  return "CSA_ERR_UNKNOWN";
+}
+
+void csa_set_index_timing_events(void* const* before, void* const* after, int32_t count) {
+  g_timing.before.clear();
+  g_timing.after.clear();
+  g_timing.next = 0;
+  if (count <= 0 || before == nullptr || after == nullptr) return;
+  for (int32_t i = 0; i < count; ++i) {
+    g_timing.before.push_back(static_cast<cudaEvent_t>(before[i]));
+    g_timing.after.push_back(static_cast<cudaEvent_t>(after[i]));
+  }
+}
+
+size_t csa_workspace_size(const csa_params* p, int32_t entry, csa_dtype kdt, int32_t B,
+                          int32_t T, int64_t N_cap) {
+  if (check_params(p) != CSA_OK || check_sizes(B, T, N_cap) != CSA_OK) return 0;
+  (void)kdt;
+  const size_t topk_ws = round_up(csa::topk_workspace_bytes(B, T, N_cap, p->topk));
+  csa::MqaArgs m = make_mqa(p, B, T, nullptr, nullptr, nullptr, N_cap, nullptr, p->topk,
+                            nullptr, 0, nullptr, nullptr, nullptr, nullptr);
+  switch (entry) {
+    case CSA_WS_INDEX_TOPK:
+      return scores_bytes(B, T, N_cap) + topk_ws;
+    case CSA_WS_TOPK:
+      return topk_ws;
+    case CSA_WS_SPARSE_MQA:
+      return round_up(csa::mqa_workspace_bytes(m));
+    case CSA_WS_HCA_MQA:
+      m.k = 0;
+      return round_up(csa::mqa_workspace_bytes(m));
+    case CSA_WS_FORWARD:
+      return scores_bytes(B, T, N_cap) + topk_ws + round_up(csa::mqa_workspace_bytes(m));
+    default:
+      fail(CSA_ERR_INVALID_ARG, "unknown workspace entry %d", entry);
+      return 0;
+  }
+}
+
+csa_status csa_compress(const csa_params* p, csa_dtype io, int32_t B, int64_t n_tok,
+                        int64_t first_entry, int64_t n_cap, const void* Ca, const void* Cb,
+                        const void* Za, const void* Zb, const void* bias, const void* prev_Cb,
+                        const void* prev_Zb, const void* kv_rms_w, int32_t finalize,
+                        void* out_cache, void* stream) {
+  TRY(check_params(p));
+  REQUIRE(io == CSA_F32 || io == CSA_BF16, "compression io dtype must be CSA_F32 or CSA_BF16");
+  REQUIRE(B >= 0 && B <= 65535, "B must be in [0, 65535]");
+  REQUIRE(n_tok >= 0 && n_tok % p->m == 0, "n_tok must be a non-negative multiple of m");
+  REQUIRE(first_entry >= 0 && n_cap >= 0 && first_entry + n_tok / p->m <= n_cap,
+          "first_entry + n_tok/m must not exceed n_cap");
+  REQUIRE(n_tok / p->m <= INT32_MAX, "too many entries");
+  REQUIRE(p->overlap == 0 || p->overlap == 1, "overlap must be 0 or 1");
+  REQUIRE(finalize == 0 || finalize == 1, "finalize must be 0 or 1");
+  REQUIRE((prev_Cb == nullptr) == (prev_Zb == nullptr), "prev_Cb and prev_Zb go together");
+  if (B == 0 || n_tok == 0) return ok();
+  REQUIRE_PTR(Ca);
+  REQUIRE_PTR(Za);
+  REQUIRE_PTR(bias);
+  REQUIRE_PTR(out_cache);
+  if (p->overlap) {
+    REQUIRE_PTR(Cb);
+    REQUIRE_PTR(Zb);
+    OPTIONAL_PTR(prev_Cb);
+    OPTIONAL_PTR(prev_Zb);
+  } else {
+    REQUIRE(Cb == nullptr && Zb == nullptr && prev_Cb == nullptr,
+            "HCA compression (overlap=0) takes no b-branch inputs");
+  }
+  OPTIONAL_PTR(kv_rms_w);
+  csa::CompressArgs a{};
+  a.B = B; a.m = p->m; a.c = p->c; a.overlap = p->overlap; a.rope_dims = p->rope_dims;
+  a.finalize = finalize; a.n_tok = n_tok; a.first_entry = first_entry; a.n_cap = n_cap;
+  a.rope_base = p->rope_base; a.eps = p->rms_eps; a.Ca = Ca; a.Cb = Cb; a.Za = Za; a.Zb = Zb;
+  a.bias = bias; a.prev_Cb = prev_Cb; a.prev_Zb = prev_Zb; a.rms_w = kv_rms_w; a.out = out_cache;
+  TRY(cuda_status(csa::launch_compress(a, io == CSA_BF16, (cudaStream_t)stream), "compress"));
+  return ok();
+}
+
+csa_status csa_index_scores(const csa_params* p, csa_dtype kdt, int32_t B, int32_t T,
+                            int64_t N_cap, const void* qI, const void* qI_scale, const float* w,
+                            const void* KI, const void* KI_scale, const int64_t* q_pos,
+                            float* out_scores, void* stream) {
+  TRY(check_index_args(p, kdt, B, T, N_cap, qI, qI_scale, w, KI, KI_scale, q_pos));
+  if ((int64_t)B * T == 0 || N_cap == 0) return ok();
+  REQUIRE_PTR(out_scores);
+  auto a = make_index(p, kdt, B, T, N_cap, qI, qI_scale, w, KI, KI_scale, q_pos, out_scores);
+  TRY(cuda_status(csa::launch_index_scores(a, (cudaStream_t)stream), "index scores"));
+  return ok();
+}
+
+csa_status csa_topk(const csa_params* p, int32_t B, int32_t T, int64_t N_cap,
+                    const float* scores, const int64_t* q_pos, int32_t* out_idx, void* ws,
+                    size_t ws_bytes, void* stream) {
+  TRY(check_params(p));
+  TRY(check_topk(p));
+  TRY(check_sizes(B, T, N_cap));
+  if ((int64_t)B * T == 0) return ok();
+  if (N_cap > 0) REQUIRE_PTR(scores);
+  REQUIRE_PTR(q_pos);
+  REQUIRE_PTR(out_idx);
+  const size_t need = csa::topk_workspace_bytes(B, T, N_cap, p->topk);
+  if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws)))
+    return fail(CSA_ERR_WORKSPACE, "top-k needs %zu workspace bytes", need);
+  csa::TopkArgs a{};
+  a.B = B; a.T = T; a.m = p->m; a.k = p->topk; a.n_cap = N_cap; a.scores = scores;
+  a.q_pos = q_pos; a.out_idx = out_idx;
+  TRY(cuda_status(csa::launch_topk(a, ws, ws_bytes, (cudaStream_t)stream), "top-k"));
+  return ok();
+}
+
+csa_status csa_index_topk(const csa_params* p, csa_dtype kdt, int32_t B, int32_t T,
+                          int64_t N_cap, const void* qI, const void* qI_scale, const float* w,
+                          const void* KI, const void* KI_scale, const int64_t* q_pos,
+                          int32_t* out_idx, float* out_scores, void* ws, size_t ws_bytes,
+                          void* stream) {
+  TRY(check_index_args(p, kdt, B, T, N_cap, qI, qI_scale, w, KI, KI_scale, q_pos));
+  TRY(check_topk(p));
+  if ((int64_t)B * T == 0) return ok();
+  REQUIRE_PTR(out_idx);
+  OPTIONAL_PTR(out_scores);
+  const size_t need = csa_workspace_size(p, CSA_WS_INDEX_TOPK, kdt, B, T, N_cap);
+  if (ws == nullptr || ws_bytes < need || !aligned16(ws))
+    return fail(CSA_ERR_WORKSPACE, "index+top-k needs %zu workspace bytes (got %zu)", need,
+                ws_bytes);
+  char* base = static_cast<char*>(ws);
+  float* scores = out_scores ? out_scores : reinterpret_cast<float*>(base);
+  char* topk_ws = base + scores_bytes(B, T, N_cap);
+  const size_t topk_bytes = need - scores_bytes(B, T, N_cap);
+  cudaStream_t st = (cudaStream_t)stream;
+  if (N_cap > 0) {
+    auto a = make_index(p, kdt, B, T, N_cap, qI, qI_scale, w, KI, KI_scale, q_pos, scores);
+    TRY(cuda_status(csa::launch_index_scores(a, st), "index scores"));
+  }
+  csa::TopkArgs t{};
+  t.B = B; t.T = T; t.m = p->m; t.k = p->topk; t.n_cap = N_cap; t.scores = scores;
+  t.q_pos = q_pos; t.out_idx = out_idx;
+  TRY(cuda_status(csa::launch_topk(t, topk_ws, topk_bytes, st), "top-k"));
+  return ok();
+}
+
+csa_status csa_sparse_mqa(const csa_params* p, csa_dtype io, int32_t B, int32_t T,
+                          const void* q, const int64_t* q_pos, const void* kv_cache,
+                          int64_t N_cap, const int32_t* idx, const void* win_kv, int64_t L_raw,
+                          const int64_t* win_pos0, const float* sink, const void* q_rms_w,
+                          void* out, void* ws, size_t ws_bytes, void* stream) {
+  TRY(check_mqa_args(p, io, B, T, q, q_pos, kv_cache, N_cap, win_kv, L_raw, win_pos0, sink,
+                     q_rms_w, out));
+  TRY(check_topk(p));
+  if ((int64_t)B * T == 0) return ok();
+  REQUIRE_PTR(idx);
+  auto a = make_mqa(p, B, T, q, q_pos, kv_cache, N_cap, idx, p->topk, win_kv, L_raw, win_pos0,
+                    sink, q_rms_w, out);
+  const size_t need = csa::mqa_workspace_bytes(a);
+  if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws)))
+    return fail(CSA_ERR_WORKSPACE, "sparse MQA needs %zu workspace bytes", need);
+  TRY(cuda_status(csa::launch_mqa(a, io == CSA_BF16, ws, ws_bytes, (cudaStream_t)stream),
+                  "sparse MQA"));
+  return ok();
+}
+
+csa_status hca_dense_mqa(const csa_params* p, csa_dtype io, int32_t B, int32_t T,
+                         const void* q, const int64_t* q_pos, const void* kv_cache,
+                         int64_t N_cap, const void* win_kv, int64_t L_raw,
+                         const int64_t* win_pos0, const float* sink, const void* q_rms_w,
+                         void* out, void* ws, size_t ws_bytes, void* stream) {
+  TRY(check_mqa_args(p, io, B, T, q, q_pos, kv_cache, N_cap, win_kv, L_raw, win_pos0, sink,
+                     q_rms_w, out));
+  if ((int64_t)B * T == 0) return ok();
+  auto a = make_mqa(p, B, T, q, q_pos, kv_cache, N_cap, nullptr, 0, win_kv, L_raw, win_pos0,
+                    sink, q_rms_w, out);
+  const size_t need = csa::mqa_workspace_bytes(a);
+  if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws)))
+    return fail(CSA_ERR_WORKSPACE, "dense MQA needs %zu workspace bytes", need);
+  TRY(cuda_status(csa::launch_mqa(a, io == CSA_BF16, ws, ws_bytes, (cudaStream_t)stream),
+                  "dense MQA"));
+  return ok();
+}
+
+csa_status csa_forward(const csa_params* p, csa_dtype io, int32_t B, int32_t T,
+                       const csa_forward_args* a, void* ws, size_t ws_bytes, void* stream) {
+  REQUIRE(a != nullptr, "args is NULL");
+  TRY(check_mqa_args(p, io, B, T, a->q, a->q_pos, a->kv_cache, a->N_cap, a->win_kv, a->L_raw,
+                     a->win_pos0, a->sink, a->q_rms_w, a->out));
+  TRY(check_index_args(p, a->idx_dtype, B, T, a->N_cap, a->qI, a->qI_scale, a->w, a->KI,
+                       a->KI_scale, a->q_pos));
+  TRY(check_topk(p));
+  REQUIRE(p->overlap == 1, "csa_forward is the CSA layer (overlap must be 1)");
+  if ((int64_t)B * T == 0) return ok();
+  REQUIRE_PTR(a->out_idx);
+  OPTIONAL_PTR(a->out_scores);
+  const size_t need = csa_workspace_size(p, CSA_WS_FORWARD, a->idx_dtype, B, T, a->N_cap);
+  if (ws == nullptr || ws_bytes < need || !aligned16(ws))
+    return fail(CSA_ERR_WORKSPACE, "csa_forward needs %zu workspace bytes (got %zu)", need,
+                ws_bytes);
+  cudaStream_t st = (cudaStream_t)stream;
+  if (a->Ca != nullptr) {
+    TRY(csa_compress(p, io, B, a->n_tok, a->first_entry, a->N_cap, a->Ca, a->Cb, a->Za, a->Zb,
+                     a->bias, a->prev_Cb, a->prev_Zb, a->kv_rms_w, 1, a->kv_cache, stream));
+  }
+  char* base = static_cast<char*>(ws);
+  const size_t sb = scores_bytes(B, T, a->N_cap);
+  const size_t tb = round_up(csa::topk_workspace_bytes(B, T, a->N_cap, p->topk));
+  float* scores = a->out_scores ? a->out_scores : reinterpret_cast<float*>(base);
+  if (a->N_cap > 0) {
+    auto ia = make_index(p, a->idx_dtype, B, T, a->N_cap, a->qI, a->qI_scale, a->w, a->KI,
+                         a->KI_scale, a->q_pos, scores);
+    TRY(cuda_status(csa::launch_index_scores(ia, st), "index scores"));
+  }
+  csa::TopkArgs t{};
+  t.B = B; t.T = T; t.m = p->m; t.k = p->topk; t.n_cap = a->N_cap; t.scores = scores;
+  t.q_pos = a->q_pos; t.out_idx = a->out_idx;
+  TRY(cuda_status(csa::launch_topk(t, base + sb, tb, st), "top-k"));
+  auto ma = make_mqa(p, B, T, a->q, a->q_pos, a->kv_cache, a->N_cap, a->out_idx, p->topk,
+                     a->win_kv, a->L_raw, a->win_pos0, a->sink, a->q_rms_w, a->out);
+  TRY(cuda_status(csa::launch_mqa(ma, io == CSA_BF16, base + sb + tb, ws_bytes - sb - tb, st),
+                  "sparse MQA"));
+  return ok();
+}
+
+}  // extern "C"

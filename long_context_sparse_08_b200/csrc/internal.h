@@ -1,0 +1,57 @@
+// Internal launch interface of libcsa: argument blocks passed by value to the kernels and
+// the launchers the C ABI layer (api.cu) calls after validating its arguments.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace csa {
+
+struct CompressArgs {
+  int B, m, c, overlap, rope_dims, finalize;
+  int64_t n_tok, first_entry, n_cap;
+  float rope_base, eps;
+  const void *Ca, *Cb, *Za, *Zb, *bias, *prev_Cb, *prev_Zb, *rms_w;
+  void* out;
+};
+cudaError_t launch_compress(const CompressArgs& a, bool bf16, cudaStream_t st);
+
+struct IndexArgs {
+  int B, T, m, n_idx_heads, d_idx, kdt;
+  int64_t n_cap;
+  const void *qI, *qI_scale, *KI, *KI_scale;
+  const float* w;
+  const int64_t* q_pos;
+  float* scores;  // [B, T, n_cap]
+};
+cudaError_t launch_index_scores(const IndexArgs& a, cudaStream_t st);
+
+struct TopkArgs {
+  int B, T, m, k;
+  int64_t n_cap;
+  const float* scores;
+  const int64_t* q_pos;
+  int32_t* out_idx;
+};
+size_t topk_workspace_bytes(int B, int T, int64_t n_cap, int k);
+cudaError_t launch_topk(const TopkArgs& a, void* ws, size_t ws_bytes, cudaStream_t st);
+
+struct MqaArgs {
+  int B, T, m, H, c, rope_dims, n_win, k;  // k = 0: dense (all visible entries)
+  int64_t n_cap, l_raw;
+  float rope_base, eps, scale;
+  const void *q, *kv, *win, *q_rms_w;
+  const int32_t* idx;
+  const int64_t *q_pos, *win_pos0;
+  const float* sink;
+  void* out;
+};
+size_t mqa_workspace_bytes(const MqaArgs& a);
+cudaError_t launch_mqa(const MqaArgs& a, bool bf16, void* ws, size_t ws_bytes, cudaStream_t st);
+
+// benchmarking hook (see csa_set_index_timing_events)
+void timing_before(cudaStream_t st);
+void timing_after(cudaStream_t st);
+
+}  // namespace csa

@@ -30,11 +30,18 @@ import numpy as np
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """fp32 -> bf16 bit patterns (uint16), round to nearest even. Finite inputs only."""
+    """fp32 -> bf16 bit patterns (uint16), round to nearest even. Finite inputs only.
+
+    Works in uint32 (finite patterns stay below 2^32 after the rounding add) and in
+    slices of 2^24 elements to bound temporary memory."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    return rounded.astype(np.uint16)
+    flat = x.reshape(-1).view(np.uint32)
+    out = np.empty(flat.shape, np.uint16)
+    step = 1 << 24
+    for i in range(0, flat.size, step):
+        u = flat[i:i + step]
+        out[i:i + step] = ((u + (np.uint32(0x7FFF) + ((u >> 16) & np.uint32(1)))) >> 16)
+    return out.reshape(x.shape)
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:

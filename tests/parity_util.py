@@ -1,0 +1,114 @@
+"""Comparison rules between the CUDA path and the float64 oracle.
+
+Tolerances (restated from the build's target):
+  - compressed entries and indexer scores agree to 1e-4 relative in fp32; for a score,
+    |dI| <= 1e-4 * max(|I_ref|, 1e-3 * max_s |I_ref|) (the floor covers near-zero sums of
+    signed head weights); a compressed row: ||d||/||ref|| <= 1e-4 and |d| <= 1e-4 rms(ref);
+    a bf16 row is within one bf16 ulp of the oracle value rounded to bf16;
+  - top-k sets are identical except at near-ties: with tau the oracle's k-th largest score
+    and tol = 1e-4 * max(|tau|, 1e-3 max|I|), every entry with I > tau + tol is selected and
+    every selected entry has I >= tau - tol;
+  - bf16 outputs: relative RMS error <= 5e-3 and max abs error <= 2e-2 (fp32 outputs: 2e-5
+    and 2e-4), against the oracle run on the same selection.
+"""
+from __future__ import annotations
+
+import functools
+
+import numpy as np
+
+from long_context_sparse_08_b200 import workloads as W
+
+
+@functools.lru_cache(maxsize=4)
+def inputs(name: str):
+    s = W.SHAPES[name]
+    return s, W.make_inputs(s)
+
+
+def dec_out(t, io: str) -> np.ndarray:
+    import torch
+
+    return t.float().cpu().numpy().astype(np.float64) if io == "bf16" else \
+        t.cpu().numpy().astype(np.float64)
+
+
+def check_scores(gpu: np.ndarray, ref: np.ndarray, what=""):
+    ref = np.asarray(ref, np.float64)
+    gpu = np.asarray(gpu, np.float64)
+    assert gpu.shape == ref.shape, what
+    if ref.size == 0:
+        return
+    floor = 1e-3 * np.abs(ref).max()
+    tol = 1e-4 * np.maximum(np.abs(ref), floor)
+    bad = np.abs(gpu - ref) > tol
+    assert not bad.any(), (f"{what}: {bad.sum()} scores off; worst rel "
+                           f"{(np.abs(gpu - ref) / np.maximum(np.abs(ref), floor)).max():.3e}")
+
+
+def check_topk(gpu_idx: np.ndarray, ref_scores: np.ndarray, k: int, gpu_scores=None, what=""):
+    """Near-tie rule of the module docstring, plus structure: distinct valid indices first,
+    -1 padding after, and (given the GPU's own scores) ordered by (score desc, index asc)."""
+    ref = np.asarray(ref_scores, np.float64)
+    n = ref.size
+    nv = min(k, n)
+    gi = np.asarray(gpu_idx, np.int64)
+    assert np.all(gi[nv:] == -1), f"{what}: padding"
+    sel = gi[:nv]
+    assert np.all((sel >= 0) & (sel < n)), f"{what}: index out of range"
+    assert np.unique(sel).size == nv, f"{what}: duplicate indices"
+    if nv == 0:
+        return 0
+    if nv == n:
+        return 0
+    tau = np.sort(ref)[::-1][k - 1]
+    tol = 1e-4 * max(abs(tau), 1e-3 * np.abs(ref).max())
+    must = np.nonzero(ref > tau + tol)[0]
+    missing = np.setdiff1d(must, sel)
+    assert missing.size == 0, f"{what}: {missing.size} clearly-top entries missing"
+    assert np.all(ref[sel] >= tau - tol), f"{what}: a selected entry is clearly below rank k"
+    if gpu_scores is not None:
+        gs = np.asarray(gpu_scores, np.float32)[sel]
+        for j in range(nv - 1):
+            a, b = gs[j], gs[j + 1]
+            assert a > b or (a == b and sel[j] < sel[j + 1]), f"{what}: order at {j}"
+    ref_set = set(np.argsort(-ref, kind="stable")[:k].tolist())
+    return len(ref_set - set(sel.tolist()))
+
+
+def recall(gpu_idx, ref_idx) -> float:
+    g = set(int(i) for i in gpu_idx if i >= 0)
+    r = set(int(i) for i in ref_idx if i >= 0)
+    return 1.0 if not r else len(g & r) / len(r)
+
+
+def check_out(gpu: np.ndarray, ref: np.ndarray, io: str, what=""):
+    ref = np.asarray(ref, np.float64)
+    d = np.asarray(gpu, np.float64) - ref
+    rel_rms = np.sqrt((d * d).sum() / max((ref * ref).sum(), 1e-300))
+    mx = np.abs(d).max() if d.size else 0.0
+    lim_rms, lim_max = (5e-3, 2e-2) if io == "bf16" else (2e-5, 2e-4)
+    assert rel_rms <= lim_rms and mx <= lim_max, \
+        f"{what}: rel RMS {rel_rms:.3e} (<= {lim_rms}), max abs {mx:.3e} (<= {lim_max})"
+    return rel_rms, mx
+
+
+def bf16_ulp(x: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 values at |x| (8 significant bits)."""
+    ax = np.maximum(np.abs(x), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(ax)) - 7)
+
+
+def check_rows(gpu: np.ndarray, ref: np.ndarray, io: str, what=""):
+    ref = np.asarray(ref, np.float64)
+    gpu = np.asarray(gpu, np.float64)
+    if io == "bf16":
+        rb = W.bf16_bits_to_f32(W.f32_to_bf16_bits(ref.astype(np.float32))).astype(np.float64)
+        ok = np.abs(gpu - rb) <= bf16_ulp(rb) * 1.0001
+        assert ok.all(), f"{what}: {(~ok).sum()} bf16 values off by more than one ulp"
+    else:
+        nrm = np.linalg.norm(ref, axis=-1)
+        rel = np.linalg.norm(gpu - ref, axis=-1) / np.maximum(nrm, 1e-300)
+        assert rel.max() <= 1e-4, f"{what}: row rel err {rel.max():.3e}"
+        rms = np.sqrt(np.mean(ref * ref, axis=-1, keepdims=True))
+        assert (np.abs(gpu - ref) <= 1e-4 * rms).all(), f"{what}: element err"

@@ -1,0 +1,182 @@
+"""The C ABI without a GPU: the library loads, exports every function include/csa.h declares,
+its structs match a C compiler's layout, and host-side validation rejects bad arguments
+with a status (no launch happens on any of these paths)."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+import long_context_sparse_08_b200 as csa
+from long_context_sparse_08_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "csa.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    B.build()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(csa_\w+|hca_\w+)\s*\(", src,
+                       flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_function_is_exported():
+    names = declared_functions()
+    assert len(names) >= 12
+    L = ctypes.CDLL(csa.LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(csa.EXPORTS)
+
+
+def test_status_strings_and_version():
+    assert csa.status_string(0) == "CSA_OK"
+    assert csa.status_string(3) == "CSA_ERR_WORKSPACE"
+    assert "sm_100a" in csa.version()
+
+
+def test_struct_layout_matches_the_c_compiler():
+    prog = r'''
+#include <stdio.h>
+#include <stddef.h>
+#include "csa.h"
+int main(void) {
+  printf("%zu %zu %zu %zu %zu %zu\n", sizeof(csa_params), sizeof(csa_forward_args),
+         offsetof(csa_forward_args, idx_dtype), offsetof(csa_forward_args, N_cap),
+         offsetof(csa_forward_args, out), offsetof(csa_params, n_win));
+  return 0;
+}
+'''
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "t.c")
+        exe = os.path.join(d, "t")
+        open(c, "w").write(prog)
+        subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), c, "-o", exe])
+        vals = [int(x) for x in subprocess.check_output([exe]).split()]
+    A = csa.CsaForwardArgs
+    assert vals == [ctypes.sizeof(csa.CsaParams), ctypes.sizeof(A), A.idx_dtype.offset,
+                    A.N_cap.offset, A.out.offset, csa.CsaParams.n_win.offset]
+
+
+def _p(**kw):
+    return csa.make_params(**kw)
+
+
+FAKE = 0x10000  # an aligned non-NULL address; never dereferenced on these paths
+
+
+def _call(name, *args):
+    fn = getattr(csa.lib(), name)
+    return fn(*args)
+
+
+def test_validation_rejects_bad_params():
+    L = csa.lib()
+    cases = [
+        dict(c=48), dict(c=0), dict(rope_dims=3), dict(rope_dims=1024), dict(m=0),
+        dict(rms_eps=-1.0),
+    ]
+    for kw in cases:
+        p = _p(**kw)
+        s = L.csa_compress(ctypes.byref(p), 1, 1, 16, 0, 8, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                           None, None, 1, FAKE, None)
+        assert s == csa.CSA_ERR_INVALID_ARG, kw
+        assert csa.last_error()
+    s = L.csa_compress(None, 1, 1, 16, 0, 8, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 1,
+                       FAKE, None)
+    assert s == csa.CSA_ERR_INVALID_ARG
+
+
+def test_compress_argument_checks():
+    L = csa.lib()
+    p = _p()
+    base = [ctypes.byref(p), 1, 1, 16, 0, 8, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 1,
+            FAKE, None]
+
+    def with_(**kw):
+        a = list(base)
+        pos = {"n_tok": 3, "first": 4, "n_cap": 5, "Ca": 6, "bias": 10, "prev_Cb": 11,
+               "out": 15, "io": 1, "finalize": 14}
+        for k, v in kw.items():
+            a[pos[k]] = v
+        return L.csa_compress(*a)
+
+    assert with_(n_tok=15) == csa.CSA_ERR_INVALID_ARG  # not a multiple of m
+    assert with_(first=6) == csa.CSA_ERR_INVALID_ARG  # 6 + 4 > 8
+    assert with_(Ca=None) == csa.CSA_ERR_INVALID_ARG
+    assert with_(Ca=FAKE + 4) == csa.CSA_ERR_INVALID_ARG  # misaligned
+    assert with_(prev_Cb=FAKE) == csa.CSA_ERR_INVALID_ARG  # prev_Cb without prev_Zb
+    assert with_(io=2) == csa.CSA_ERR_INVALID_ARG  # fp8 is not a compression io type
+    assert with_(finalize=2) == csa.CSA_ERR_INVALID_ARG
+    assert with_(n_tok=0) == csa.CSA_OK  # empty chunk: nothing to do, nothing launched
+    p2 = _p(overlap=0, m=16)
+    a = list(base)
+    a[0] = ctypes.byref(p2)
+    assert L.csa_compress(*a) == csa.CSA_ERR_INVALID_ARG  # HCA takes no b-branch
+
+
+def test_index_and_topk_checks():
+    L = csa.lib()
+    p = _p(topk=4096)
+    s = L.csa_topk(ctypes.byref(p), 1, 1, 100, FAKE, FAKE, FAKE, None, 0, None)
+    assert s == csa.CSA_ERR_INVALID_ARG
+    p = _p()
+    s = L.csa_index_scores(ctypes.byref(p), 7, 1, 1, 100, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                           FAKE, None)
+    assert s == csa.CSA_ERR_INVALID_ARG  # unknown key format
+    s = L.csa_index_scores(ctypes.byref(p), csa.CSA_MXFP4, 1, 1, 100, FAKE, None, FAKE, FAKE,
+                           FAKE, FAKE, FAKE, None)
+    assert s == csa.CSA_ERR_INVALID_ARG  # MXFP4 queries need their scales
+    s = L.csa_index_scores(ctypes.byref(p), csa.CSA_BF16, 0, 1, 100, None, None, None, None,
+                           None, None, None, None)
+    assert s == csa.CSA_OK  # B = 0: nothing to do
+    p = _p(d_idx=48)
+    s = L.csa_index_scores(ctypes.byref(p), csa.CSA_BF16, 1, 1, 100, FAKE, None, FAKE, FAKE,
+                           None, FAKE, FAKE, None)
+    assert s == csa.CSA_ERR_INVALID_ARG
+
+
+def test_workspace_checks():
+    L = csa.lib()
+    p = _p()
+    need = csa.workspace_size(p, csa.CSA_WS_INDEX_TOPK, csa.CSA_BF16, 2, 3, 1000)
+    assert need >= 2 * 3 * 1000 * 4
+    s = L.csa_index_topk(ctypes.byref(p), csa.CSA_BF16, 2, 3, 1000, FAKE, None, FAKE, FAKE,
+                         None, FAKE, FAKE, None, FAKE, need - 1, None)
+    assert s == csa.CSA_ERR_WORKSPACE
+    assert csa.workspace_size(p, 99, 0, 1, 1, 10) == 0
+
+
+def test_attention_checks():
+    L = csa.lib()
+    p = _p(n_heads=24)  # > 16 and not a multiple of 16
+    s = L.hca_dense_mqa(ctypes.byref(p), 1, 1, 1, FAKE, FAKE, FAKE, 10, FAKE, 128, FAKE, None,
+                        None, FAKE, None, 0, None)
+    assert s == csa.CSA_ERR_INVALID_ARG
+    p = _p()
+    s = L.hca_dense_mqa(ctypes.byref(p), 1, 1, 1, FAKE, FAKE, FAKE, 10, None, 0, None, None,
+                        None, FAKE, None, 0, None)
+    assert s == csa.CSA_ERR_INVALID_ARG  # n_win > 0 but no window rows
+    s = L.csa_sparse_mqa(ctypes.byref(p), 1, 1, 1, FAKE, FAKE, FAKE, 10, None, FAKE, 128, FAKE,
+                         None, None, FAKE, None, 0, None)
+    assert s == csa.CSA_ERR_INVALID_ARG  # no index list
+    p = _p(c=1024)
+    s = L.hca_dense_mqa(ctypes.byref(p), 1, 1, 1, FAKE, FAKE, FAKE, 10, FAKE, 128, FAKE, None,
+                        None, FAKE, None, 0, None)
+    assert s == csa.CSA_ERR_UNSUPPORTED
+
+
+def test_binding_refuses_host_tensors():
+    import torch
+
+    with pytest.raises(ValueError):
+        csa._ptr(torch.zeros(4))
