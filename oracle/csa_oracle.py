@@ -235,6 +235,16 @@ def index_scores(qI_t, w_t, KI, n_vis: int) -> np.ndarray:
     return np.maximum(dots, 0.0) @ np.asarray(w_t, np.float64)
 
 
+def index_score_scale(qI_t, w_t, KI, n_vis: int) -> np.ndarray:
+    """sum_h |w_{t,h}| * ReLU(q^I_{t,h} . K_s): the sum of the magnitudes of the terms that
+    make up I_{t,s}. Not part of the method: it is the scale against which a floating-point
+    evaluation of I is judged (a rounding error of a sum grows with this, not with |I|,
+    when signed head weights cancel). Equals |I| when every w >= 0."""
+    qI_t = np.asarray(qI_t, np.float64)
+    K = np.asarray(KI, np.float64)[:n_vis]
+    return np.maximum(K @ qI_t.T, 0.0) @ np.abs(np.asarray(w_t, np.float64))
+
+
 def topk_select(scores, k: int) -> np.ndarray:
     """Top-k of I_{t,:}: indices ordered by (score desc, index asc); slots past the
     number of candidates hold -1 (reading R7) [P1 1(2), C_t^SprsComp]."""

@@ -67,8 +67,9 @@ def run(s, inp, queries: Optional[Iterable[Tuple[int, int]]] = None, *,
         want_scores: bool = True) -> Dict[str, dict]:
     """Run the oracle for the listed (b, t-index) queries (default: all).
 
-    Returns {"scores": {(b,ti): [n_vis]}, "idx": {(b,ti): [k]}, "out": {(b,ti): [H,c]},
-    "chunk": the freshly compressed entries of a prefill chunk (or None)}. With
+    Returns {"scores": {(b,ti): [n_vis]}, "scale": {(b,ti): [n_vis]} (the magnitude sums of
+    index_score_scale), "idx": {(b,ti): [k]}, "out": {(b,ti): [H,c]}, "chunk": the freshly
+    compressed entries of a prefill chunk (or None)}. With
     ``idx_override`` the attention of those queries uses the given selection instead of
     the oracle's own (to compare the output of a CUDA selection that differs from the
     oracle's only at near-ties).
@@ -83,7 +84,7 @@ def run(s, inp, queries: Optional[Iterable[Tuple[int, int]]] = None, *,
     pos0 = np.asarray(inp["win_pos0"], np.int64)
     sink = np.asarray(inp["sink"], np.float64)
     scale = 1.0 / np.sqrt(s.c)
-    res = {"scores": {}, "idx": {}, "out": {}, "chunk": chunk}
+    res = {"scores": {}, "scale": {}, "idx": {}, "out": {}, "chunk": chunk}
     cur_b, qI_b, KI_b = None, None, None
     for (b, ti) in queries:
         t = int(pos[b, ti])
@@ -107,6 +108,8 @@ def run(s, inp, queries: Optional[Iterable[Tuple[int, int]]] = None, *,
                 sel = O.topk_select(sc, s.topk)
                 if want_scores:
                     res["scores"][(b, ti)] = sc
+                    res["scale"][(b, ti)] = O.index_score_scale(
+                        qI_b[ti], np.asarray(inp["w"][b, ti], np.float64), KI_b, n_vis)
                 res["idx"][(b, ti)] = sel
                 use = np.asarray(idx_override[(b, ti)], np.int64) if given else sel
             valid = use[(use >= 0) & (use < s.n_cap)]

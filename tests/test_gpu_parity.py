@@ -91,7 +91,8 @@ def test_index_scores_parity(name):
     res = P.run(s, inp)
     scores = st.scores.cpu().numpy()
     for (b, ti), ref in res["scores"].items():
-        U.check_scores(scores[b, ti, :ref.size], ref, f"{name} b={b} t={ti}")
+        U.check_scores(scores[b, ti, :ref.size], ref, res["scale"][(b, ti)],
+                       f"{name} b={b} t={ti}")
 
 
 # ---------------------------------------------------------------------------
@@ -178,7 +179,8 @@ def _forward_parity(name, queries=None):
     idx = st.out_idx.cpu().numpy()
     out = st.out.float().cpu().numpy()
     for (b, ti), ref in res["scores"].items():
-        U.check_scores(scores[b, ti, :ref.size], ref, f"{name} b={b} t={ti} scores")
+        U.check_scores(scores[b, ti, :ref.size], ref, res["scale"][(b, ti)],
+                       f"{name} b={b} t={ti} scores")
         U.check_topk(idx[b, ti], ref, s.topk, scores[b, ti], f"{name} b={b} t={ti} top-k")
     if res["chunk"] is not None:
         first = s.ctx // s.m

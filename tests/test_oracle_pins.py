@@ -449,3 +449,13 @@ def test_pipeline_tiny_first_queries_window_only():
     z = qh @ row / 8.0
     frac = np.exp(z) / (np.exp(z) + 1.0)
     np.testing.assert_allclose(res["out"][(0, 0)], frac[:, None] * row[None], atol=1e-13)
+
+
+def test_index_score_scale_bounds_the_score():
+    H, d, N = 6, 8, 40
+    q, K, w = _rand(H, d), _rand(N, d), _rand(H)
+    I = O.index_scores(q, w, K, N)
+    A = O.index_score_scale(q, w, K, N)
+    assert np.all(A >= np.abs(I) - 1e-12)
+    np.testing.assert_allclose(O.index_score_scale(q, np.abs(w), K, N),
+                               O.index_scores(q, np.abs(w), K, N), rtol=1e-14)
