@@ -6,7 +6,7 @@ Tolerances (restated from the build's target):
     terms summed (A = |I| when all w >= 0; with signed w it keeps the bound meaningful for
     scores that cancel to near zero); a compressed row: ||d||/||ref|| <= 1e-4 and
     |d| <= 1e-4 rms(ref);
-    a bf16 row is within one bf16 ulp of the oracle value rounded to bf16;
+    a bf16 row is that fp32 bound plus one rounding to bf16 (half a bf16 ulp);
   - top-k sets are identical except at near-ties: with tau the oracle's k-th largest score
     and tol = 1e-4 * max(|tau|, 1e-3 max|I|), every entry with I > tau + tol is selected and
     every selected entry has I >= tau - tol;
@@ -106,9 +106,11 @@ def check_rows(gpu: np.ndarray, ref: np.ndarray, io: str, what=""):
     ref = np.asarray(ref, np.float64)
     gpu = np.asarray(gpu, np.float64)
     if io == "bf16":
-        rb = W.bf16_bits_to_f32(W.f32_to_bf16_bits(ref.astype(np.float32))).astype(np.float64)
-        ok = np.abs(gpu - rb) <= bf16_ulp(rb) * 1.0001
-        assert ok.all(), f"{what}: {(~ok).sum()} bf16 values off by more than one ulp"
+        # the fp32 entry within 1e-4 * rms(row) of the oracle, then one rounding to bf16
+        rms = np.sqrt(np.mean(ref * ref, axis=-1, keepdims=True))
+        lim = 1e-4 * rms + 0.5 * bf16_ulp(ref) * 1.0001
+        ok = np.abs(gpu - ref) <= lim
+        assert ok.all(), f"{what}: {(~ok).sum()} bf16 values off"
     else:
         nrm = np.linalg.norm(ref, axis=-1)
         rel = np.linalg.norm(gpu - ref, axis=-1) / np.maximum(nrm, 1e-300)
