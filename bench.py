@@ -212,6 +212,9 @@ def run_ours(args, W, rank, world, local_rank):
     ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     has_index = s.kind != "hca_decode"
     if has_index:
+        for e in ev_b + ev_a:  # torch creates the CUDA event on first record
+            e.record(stream)
+        torch.cuda.synchronize()
         csa.set_index_timing_events(ev_b, ev_a)
     clocks = Clocks(local_rank)
     if world > 1:

@@ -222,6 +222,14 @@ const char* csa_last_error(void);
  */
 void csa_set_index_timing_events(void* const* before, void* const* after, int32_t count);
 
+/*
+ * Error word of the tensor-core kernels: every wait inside them is bounded (about a second);
+ * a wait that runs out stores a nonzero code (the first one wins) and the kernel returns
+ * early instead of hanging. Writes the code to *code (0 = none) and clears it. Synchronises
+ * the device. Returns CSA_ERR_CUDA if the copy fails.
+ */
+csa_status csa_device_error(int32_t* code);
+
 /* Library version string. */
 const char* csa_version(void);
 

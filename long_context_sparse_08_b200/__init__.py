@@ -22,7 +22,7 @@ CSA_WS_INDEX_TOPK, CSA_WS_TOPK, CSA_WS_SPARSE_MQA, CSA_WS_HCA_MQA, CSA_WS_FORWAR
 EXPORTS = (
     "csa_compress", "csa_index_scores", "csa_topk", "csa_index_topk", "csa_sparse_mqa",
     "hca_dense_mqa", "csa_forward", "csa_workspace_size", "csa_status_string",
-    "csa_last_error", "csa_set_index_timing_events", "csa_version",
+    "csa_last_error", "csa_set_index_timing_events", "csa_version", "csa_device_error",
 )
 
 
@@ -75,6 +75,7 @@ _SIGS = {
     "csa_last_error": [],
     "csa_set_index_timing_events": [ctypes.POINTER(_VP), ctypes.POINTER(_VP), _I32],
     "csa_version": [],
+    "csa_device_error": [ctypes.POINTER(ctypes.c_int32)],
 }
 _RES = {"csa_workspace_size": _SZ, "csa_status_string": ctypes.c_char_p,
         "csa_last_error": ctypes.c_char_p, "csa_version": ctypes.c_char_p,
@@ -113,6 +114,13 @@ def last_error() -> str:
 
 def version() -> str:
     return lib().csa_version().decode()
+
+
+def device_error() -> int:
+    """Read and clear the tensor-core kernels' error word (0 = no bounded wait ran out)."""
+    c = ctypes.c_int32(0)
+    _check("csa_device_error", lib().csa_device_error(ctypes.byref(c)))
+    return int(c.value)
 
 
 def _check(fn: str, status: int):

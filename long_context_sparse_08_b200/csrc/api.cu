@@ -197,6 +197,14 @@ const char* csa_version(void) { return "libcsa 0.1 (sm_100a)"; }
 
 const char* csa_last_error(void) { return g_err; }
 
+csa_status csa_device_error(int32_t* code) {
+  REQUIRE(code != nullptr, "code is NULL");
+  int c = 0;
+  TRY(cuda_status(csa::index_mxf4_device_error(&c), "device error word"));
+  *code = c;
+  return ok();
+}
+
 const char* csa_status_string(csa_status s) {
   switch (s) {
     case CSA_OK: return "CSA_OK";

@@ -26,6 +26,10 @@ struct IndexArgs {
   float* scores;  // [B, T, n_cap]
 };
 cudaError_t launch_index_scores(const IndexArgs& a, cudaStream_t st);
+// tensor-core kernel for MXFP4 keys (64 heads x 128 dims, N_cap % 32 == 0)
+bool index_mxf4_tc_supported(const IndexArgs& a);
+cudaError_t launch_index_mxf4_tc(const IndexArgs& a, cudaStream_t st);
+cudaError_t index_mxf4_device_error(int* code);
 
 struct TopkArgs {
   int B, T, m, k;

@@ -14,8 +14,8 @@ namespace tc {
 // ~1 s at 2 GHz
 constexpr long long kSpinCycles = 2000000000ll;
 
-// device-side error word (0 = none); read and cleared by csa_device_error()
-extern __device__ int g_device_error;
+// device-side error word of the including translation unit (0 = none)
+static __device__ int g_device_error = 0;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -186,26 +186,32 @@ HCA_DECODE = _reg(Shape("hca_decode_1m", "hca_decode", "bf16", "none", B=16, T=1
                         n_win=128, n_cap=8192, ctx=1048576, seed=4, overlap=0))
 
 # Mid-size parity cases: several tiles plus a ragged tail, ragged per-request contexts.
+# Cache capacities are whole pages of 32 entries (128 tokens, the lcm(m, m') block of the
+# paged cache); visibility inside them is ragged.
 _reg(Shape("mid_decode_fp8", "csa_decode", "bf16", "fp8", B=3, T=1, m=4, c=512, rope_dims=64,
-           n_heads=64, n_idx_heads=64, d_idx=128, topk=512, n_win=128, n_cap=5000, ctx=19993,
+           n_heads=64, n_idx_heads=64, d_idx=128, topk=512, n_win=128, n_cap=5024, ctx=19993,
            seed=11))
 _reg(Shape("mid_decode_mxfp4", "csa_decode", "bf16", "mxfp4", B=3, T=1, m=4, c=512,
            rope_dims=64, n_heads=128, n_idx_heads=64, d_idx=128, topk=1024, n_win=128,
-           n_cap=6000, ctx=23999, seed=12))
+           n_cap=6016, ctx=23999, seed=12))
 _reg(Shape("mid_decode_bf16", "csa_decode", "bf16", "bf16", B=2, T=1, m=4, c=512, rope_dims=64,
-           n_heads=64, n_idx_heads=64, d_idx=128, topk=512, n_win=128, n_cap=3001, ctx=12004,
+           n_heads=64, n_idx_heads=64, d_idx=128, topk=512, n_win=128, n_cap=3008, ctx=12004,
            seed=13))
 _reg(Shape("mid_prefill_bf16", "csa_prefill", "bf16", "bf16", B=1, T=384, m=4, c=512,
-           rope_dims=64, n_heads=64, n_idx_heads=64, d_idx=128, topk=512, n_win=128, n_cap=700,
+           rope_dims=64, n_heads=64, n_idx_heads=64, d_idx=128, topk=512, n_win=128, n_cap=704,
            ctx=2416, n_tok=384, seed=14))
 _reg(Shape("mid_hca_decode", "hca_decode", "bf16", "none", B=3, T=1, m=128, c=512, rope_dims=64,
            n_heads=64, n_idx_heads=0, d_idx=0, topk=0, n_win=128, n_cap=600, ctx=76900, seed=15,
            overlap=0))
 # Degenerate decode cases: no visible entry (t < m), fewer visible entries than k,
-# exactly k, and a cache shorter than floor(t/m).
+# exactly k, and a cache shorter than floor(t/m). Also an MXFP4 one for the tensor-core
+# indexer's edges (single partial tile, zero tiles, a request spanning many tiles).
 _reg(Shape("edge_decode_bf16", "csa_decode", "bf16", "bf16", B=4, T=1, m=4, c=512, rope_dims=64,
-           n_heads=64, n_idx_heads=64, d_idx=128, topk=512, n_win=128, n_cap=600, ctx=0,
+           n_heads=64, n_idx_heads=64, d_idx=128, topk=512, n_win=128, n_cap=608, ctx=0,
            seed=16, q_pos_override=(2, 37, 2051, 9999)))
+_reg(Shape("edge_decode_mxfp4", "csa_decode", "bf16", "mxfp4", B=5, T=1, m=4, c=512,
+           rope_dims=64, n_heads=128, n_idx_heads=64, d_idx=128, topk=1024, n_win=128,
+           n_cap=4096, ctx=0, seed=18, q_pos_override=(3, 7, 515, 4099, 16384 + 77)))
 _reg(Shape("edge_hca_decode", "hca_decode", "bf16", "none", B=3, T=1, m=128, c=512, rope_dims=64,
            n_heads=64, n_idx_heads=0, d_idx=0, topk=0, n_win=128, n_cap=40, ctx=0, seed=17,
            overlap=0, q_pos_override=(0, 127, 9000)))

@@ -82,7 +82,7 @@ def test_compress_parity(name):
 # ---------------------------------------------------------------------------
 
 INDEX_CASES = ["tiny_prefill_f32", "mid_decode_fp8", "mid_decode_mxfp4", "mid_decode_bf16",
-               "edge_decode_bf16", "mid_prefill_bf16"]
+               "edge_decode_bf16", "edge_decode_mxfp4", "mid_prefill_bf16"]
 
 
 @pytest.mark.parametrize("name", INDEX_CASES)
@@ -197,9 +197,11 @@ def _forward_parity(name, queries=None):
 
 
 @pytest.mark.parametrize("name", ["tiny_prefill_f32", "mid_decode_fp8", "mid_decode_mxfp4",
-                                  "mid_decode_bf16", "edge_decode_bf16", "mid_prefill_bf16"])
+                                  "mid_decode_bf16", "edge_decode_bf16", "edge_decode_mxfp4",
+                                  "mid_prefill_bf16"])
 def test_forward_parity(name):
     _forward_parity(name)
+    assert csa.device_error() == 0
 
 
 def test_forward_parity_flash_decode_131k():
@@ -229,6 +231,12 @@ def test_hca_dense_parity(name):
     out = st.out.float().cpu().numpy()
     for (b, ti), ref in res["out"].items():
         U.check_out(out[b, ti], ref, s.io, f"{name} b={b}")
+
+
+def test_no_bounded_wait_gave_up():
+    # every tensor-core kernel's waits are bounded; none may have run out in this session
+    torch.cuda.synchronize()
+    assert csa.device_error() == 0
 
 
 def test_forward_is_deterministic():
