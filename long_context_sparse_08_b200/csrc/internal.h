@@ -52,6 +52,11 @@ struct MqaArgs {
   void* out;
 };
 size_t mqa_workspace_bytes(const MqaArgs& a);
+// tensor-core attention (bf16, c = 512, heads in groups of 64)
+bool mqa_tc_supported(const MqaArgs& a, bool bf16);
+size_t mqa_tc_workspace_bytes(const MqaArgs& a);
+cudaError_t launch_mqa_tc(const MqaArgs& a, void* ws, size_t ws_bytes, cudaStream_t st);
+cudaError_t mqa_tc_device_error(int* code);
 cudaError_t launch_mqa(const MqaArgs& a, bool bf16, void* ws, size_t ws_bytes, cudaStream_t st);
 
 // benchmarking hook (see csa_set_index_timing_events)

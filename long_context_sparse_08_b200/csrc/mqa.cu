@@ -196,10 +196,14 @@ __global__ void __launch_bounds__(kThreads) k_mqa_cc(MqaArgs a) {
 
 }  // namespace
 
-size_t mqa_workspace_bytes(const MqaArgs&) { return 0; }
+size_t mqa_workspace_bytes(const MqaArgs& a) {
+  // sized for the tensor-core path whenever its shape constraints hold (bf16 or not)
+  return mqa_tc_supported(a, true) ? mqa_tc_workspace_bytes(a) : 0;
+}
 
-cudaError_t launch_mqa(const MqaArgs& a, bool bf16, void*, size_t, cudaStream_t st) {
+cudaError_t launch_mqa(const MqaArgs& a, bool bf16, void* ws, size_t ws_bytes, cudaStream_t st) {
   if (a.B == 0 || a.T == 0 || a.H == 0) return cudaSuccess;
+  if (mqa_tc_supported(a, bf16)) return launch_mqa_tc(a, ws, ws_bytes, st);
   const int hpb = a.H < kMaxHpb ? a.H : kMaxHpb;
   dim3 grid(a.H / hpb, a.B * a.T);
   const size_t smem = ((size_t)kMaxHpb * a.c + (size_t)kRows * a.c + kMaxHpb * kRows +

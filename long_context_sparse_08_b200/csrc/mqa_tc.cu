@@ -1,0 +1,617 @@
+// Stage 4 on tensor cores: shared-KV MQA (sparse CSA rows or dense HCA rows) plus the
+// sliding window, with query RMSNorm / RoPE, sink and output un-rotation.
+//
+// 【论文解读】DeepSeek-V4 一(三)1(3) / 2(2): every KV row is key and value for all heads;
+// 3(1) RMSNorm of each query head; 3(2) RoPE(t) on the last r dims of q, RoPE(-t) on the
+// output; 3(3) window rows attended with the compressed rows; 3(4) exp(z'_h) added to the
+// softmax denominator.
+//
+// Work: a stream is (query, group of 64 heads); its KV row list (selected or visible
+// entries, then the window) is cut into chunks of 128 rows, and the chunks of a stream are
+// split over `nsplit` CTAs. Per chunk, with bf16 operands in 128B-swizzled shared memory
+// and fp32 accumulators in TMEM:
+//   S^T[128 rows x 64 heads] = K_chunk . Q^T           (A = KV tile, K-major; B = q_hat)
+//   P^T = exp(S^T * scale - m_h) in bf16               (softmax warps, thread = row)
+//   O^T[4 x 128 dims x 64 heads] += V_chunk^T . P^T    (A = the same KV tile read MN-major)
+// so the gathered tile is read from shared memory by both products and never transposed.
+// The running max m_h is only raised when a chunk's max exceeds it by more than 8 (then
+// O^T and l are rescaled); exp(s - m) <= e^8 otherwise, exactly as correct.
+// One split: the CTA finalises (sink, RoPE(-t), bf16). Several: it writes (m, l, O)
+// partials and k_mqa_combine merges them in a fixed order (deterministic).
+#include "common.cuh"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace csa {
+
+namespace {
+
+using namespace tc;
+
+constexpr int kC = 512;          // head dim
+constexpr int kRows = 128;       // KV rows per chunk (MMA M of S^T)
+constexpr int kHg = 64;          // heads per CTA (MMA N)
+constexpr int kThreads = 160;    // warps 0-3: loads + softmax + epilogue; warp 4: MMA
+constexpr int kAtoms = kC / 64;  // 64-element (128 B) swizzle atoms along a row
+constexpr float kLazy = 8.f;     // rescale threshold (natural-log units)
+
+// shared memory (offsets from a 1024-aligned base)
+constexpr int kOffKV = 0;                                // [atom][row][128 B]  128 KB
+constexpr int kOffQ = kOffKV + kAtoms * kRows * 128;     // [atom][head][128 B]  64 KB
+constexpr int kOffP = kOffQ + kAtoms * kHg * 128;        // [row][128 B]         16 KB
+constexpr int kOffEnd = kOffP + kRows * 128;
+
+// TMEM columns
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;     // S^T: 64 columns
+constexpr uint32_t kColO = 256;   // O^T slice s: 256 + 64 s
+
+enum { kErrKvFull = 201, kErrSFull = 202, kErrPFull = 203, kErrKvFree = 204 };
+
+struct Smem {
+  uint64_t kv_full, s_full, p_full, kv_free, done;
+  uint32_t tmem_slot;
+  int any_rescale;
+  float red[4][kHg];
+  float m_used[kHg], l_sum[kHg], alpha[kHg], fin[kHg];
+  float cs[256], sn[256];  // RoPE table for pairs of the last r dims
+};
+
+struct MqaTcParams {
+  MqaArgs a;
+  int G;       // head groups (H / 64)
+  int nsplit;  // CTAs per stream
+  float* part; // partials [stream][split][64 * (kC + 2)] or nullptr
+};
+
+__device__ __forceinline__ void bar_softmax() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// AND of `ok` over the 128 softmax threads (keeps them in lockstep when a wait gives up).
+__device__ __forceinline__ bool all_ok_softmax(bool ok) {
+  uint32_t res;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 1, 128, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(res)
+      : "r"((uint32_t)ok)
+      : "memory");
+  return res != 0;
+}
+
+__device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
+  return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// Row list of a query: [selected (k) or visible (n_vis) entries][window tokens].
+struct RowList {
+  int64_t t, n_vis, n_sel, lo, n_w, L;
+};
+
+__device__ __forceinline__ RowList row_list(const MqaArgs& a, int bt) {
+  RowList r;
+  r.t = a.q_pos[bt];
+  r.n_vis = r.t < 0 ? 0 : (r.t / a.m < a.n_cap ? r.t / a.m : a.n_cap);
+  r.n_sel = a.k > 0 ? a.k : r.n_vis;
+  r.lo = (r.t - a.n_win + 1) > 0 ? (r.t - a.n_win + 1) : 0;
+  r.n_w = (a.n_win > 0 && r.t >= 0) ? r.t - r.lo + 1 : 0;
+  r.L = r.n_sel + r.n_w;
+  return r;
+}
+
+// Source row of list entry j (nullptr: masked).
+__device__ __forceinline__ const __nv_bfloat16* row_src(const MqaArgs& a, int bt, int b,
+                                                        const RowList& rl, int64_t j) {
+  if (j < rl.n_sel) {
+    int64_t e = j;
+    if (a.k > 0) e = a.idx[(size_t)bt * a.k + j];
+    else if (e >= rl.n_vis) return nullptr;
+    if (e < 0 || e >= a.n_cap) return nullptr;
+    return static_cast<const __nv_bfloat16*>(a.kv) + ((size_t)b * a.n_cap + e) * kC;
+  }
+  if (j < rl.L) {
+    const int64_t rr = rl.lo + (j - rl.n_sel) - a.win_pos0[b];
+    if (rr < 0 || rr >= a.l_raw) return nullptr;
+    return static_cast<const __nv_bfloat16*>(a.win) + ((size_t)b * a.l_raw + rr) * kC;
+  }
+  return nullptr;
+}
+
+// Reduce-scatter of 64 per-thread values across the warp: on return lane l holds the
+// reduction over the warp's 32 threads of heads 2l and 2l+1 in out[0], out[1].
+template <bool kMax>
+__device__ __forceinline__ void warp_reduce_scatter64(const float (&v)[64], float (&out)[2]) {
+  const int lane = threadIdx.x & 31;
+  float a32[32], a16[16], a8[8], a4[4];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const bool hi = lane & 16;
+    const float send = hi ? v[i] : v[32 + i];
+    const float keep = hi ? v[32 + i] : v[i];
+    const float got = __shfl_xor_sync(0xffffffffu, send, 16);
+    a32[i] = kMax ? fmaxf(keep, got) : keep + got;
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const bool hi = lane & 8;
+    const float send = hi ? a32[i] : a32[16 + i];
+    const float keep = hi ? a32[16 + i] : a32[i];
+    const float got = __shfl_xor_sync(0xffffffffu, send, 8);
+    a16[i] = kMax ? fmaxf(keep, got) : keep + got;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const bool hi = lane & 4;
+    const float send = hi ? a16[i] : a16[8 + i];
+    const float keep = hi ? a16[8 + i] : a16[i];
+    const float got = __shfl_xor_sync(0xffffffffu, send, 4);
+    a8[i] = kMax ? fmaxf(keep, got) : keep + got;
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const bool hi = lane & 2;
+    const float send = hi ? a8[i] : a8[4 + i];
+    const float keep = hi ? a8[4 + i] : a8[i];
+    const float got = __shfl_xor_sync(0xffffffffu, send, 2);
+    a4[i] = kMax ? fmaxf(keep, got) : keep + got;
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const bool hi = lane & 1;
+    const float send = hi ? a4[i] : a4[2 + i];
+    const float keep = hi ? a4[2 + i] : a4[i];
+    const float got = __shfl_xor_sync(0xffffffffu, send, 1);
+    out[i] = kMax ? fmaxf(keep, got) : keep + got;
+  }
+}
+
+__device__ __forceinline__ void tmem_st_32x32b_x64(uint32_t taddr, const uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0],"
+      " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16,"
+      " %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32,"
+      " %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48,"
+      " %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31]), "r"(r[32]), "r"(r[33]), "r"(r[34]), "r"(r[35]),
+      "r"(r[36]), "r"(r[37]), "r"(r[38]), "r"(r[39]), "r"(r[40]), "r"(r[41]), "r"(r[42]),
+      "r"(r[43]), "r"(r[44]), "r"(r[45]), "r"(r[46]), "r"(r[47]), "r"(r[48]), "r"(r[49]),
+      "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]), "r"(r[56]),
+      "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  Smem& S = *reinterpret_cast<Smem*>(base + kOffEnd);
+  const MqaArgs& a = P.a;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int stream = blockIdx.x / P.nsplit, split = blockIdx.x % P.nsplit;
+  const int bt = stream / P.G, g = stream % P.G;
+  const int b = bt / a.T;
+  const int h0 = g * kHg;
+  const RowList rl = row_list(a, bt);
+  const int nchunks = (int)((rl.L + kRows - 1) / kRows);
+  const int c0 = (int)(((int64_t)nchunks * split) / P.nsplit);
+  const int c1 = (int)(((int64_t)nchunks * (split + 1)) / P.nsplit);
+  const int r = a.rope_dims, r0 = kC - r;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      mbar_init(&S.kv_full, 128);
+      mbar_init(&S.s_full, 1);
+      mbar_init(&S.p_full, 128);
+      mbar_init(&S.kv_free, 1);
+      mbar_init(&S.done, 1);
+      fence_barrier_init();
+    }
+    tmem_alloc(&S.tmem_slot, kTmemCols);
+  } else {
+    // RoPE table, running stats, and q_hat = RoPE_t(RMSNorm(q)) into the B-operand layout
+    for (int p = tid; p < r / 2; p += 128)
+      rope_cos_sin((double)rl.t, p, r, (double)a.rope_base, &S.cs[p], &S.sn[p]);
+    if (tid < kHg) {
+      S.m_used[tid] = -INFINITY;
+      S.l_sum[tid] = 0.f;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_slot;
+
+  if (warp < 4) {
+    {
+      const int h = tid >> 1, half = tid & 1;
+      const __nv_bfloat16* qrow =
+          static_cast<const __nv_bfloat16*>(a.q) + ((size_t)bt * a.H + h0 + h) * kC + 256 * half;
+      const __nv_bfloat16* gw =
+          a.q_rms_w ? static_cast<const __nv_bfloat16*>(a.q_rms_w) + 256 * half : nullptr;
+      uint4 raw[32];
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        raw[i] = reinterpret_cast<const uint4*>(qrow)[i];
+        const uint32_t w4[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float x0 = __uint_as_float(w4[k] << 16), x1 = __uint_as_float(w4[k] & 0xffff0000u);
+          ss = fmaf(x0, x0, fmaf(x1, x1, ss));
+        }
+      }
+      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+      const float rstd = rsqrtf(ss / (float)kC + a.eps);
+      uint8_t* qs = base + kOffQ;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int d0 = 256 * half + 8 * i;
+        const uint32_t w4[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+        float x[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          x[2 * k] = __uint_as_float(w4[k] << 16) * rstd;
+          x[2 * k + 1] = __uint_as_float(w4[k] & 0xffff0000u) * rstd;
+        }
+        if (gw) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) x[k] *= __bfloat162float(gw[8 * i + k]);
+        }
+        if (d0 >= r0) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int p = (d0 + 2 * k - r0) >> 1;
+            const float c = S.cs[p], s = S.sn[p], u = x[2 * k], v = x[2 * k + 1];
+            x[2 * k] = u * c - v * s;
+            x[2 * k + 1] = u * s + v * c;
+          }
+        }
+        uint4 o;
+        o.x = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[0])) |
+              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[1])) << 16);
+        o.y = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[2])) |
+              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[3])) << 16);
+        o.z = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[4])) |
+              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[5])) << 16);
+        o.w = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[6])) |
+              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[7])) << 16);
+        const int atom = d0 >> 6, chunk = (d0 & 63) >> 3;
+        *reinterpret_cast<uint4*>(qs + atom * (kHg * 128) + sw128(h, chunk)) = o;
+      }
+    }
+
+    bool ok = true;
+    const uint32_t kv_base = smem_u32(base + kOffKV);
+    for (int j = c0; j < c1 && ok; ++j) {
+      const uint32_t it = (uint32_t)(j - c0);
+      if (j > c0) ok = all_ok_softmax(mbar_wait(&S.kv_free, (it - 1) & 1, kErrKvFree));
+      if (!ok) break;
+      // ---- gather the chunk's 128 rows: warp w loads rows w, w+4, ...; lane = 16B chunk ----
+      for (int rr = warp; rr < kRows; rr += 4) {
+        const __nv_bfloat16* src = row_src(a, bt, b, rl, (int64_t)j * kRows + rr);
+#pragma unroll
+        for (int hseg = 0; hseg < 2; ++hseg) {
+          const int gch = lane + 32 * hseg;  // 16-byte chunk of the 1 KB row
+          const int atom = gch >> 3, c = gch & 7;
+          const uint32_t dst = kv_base + atom * (kRows * 128) + sw128(rr, c);
+          cp_async16(dst, src ? src + 8 * gch : static_cast<const __nv_bfloat16*>(a.kv),
+                     src != nullptr);
+        }
+      }
+      cp_async_wait_all();
+      fence_proxy_async_smem();
+      mbar_arrive(&S.kv_full);
+
+      // ---- softmax of S^T (thread = row) ----
+      const int row = tid;
+      const int64_t jl = (int64_t)j * kRows + row;
+      const bool valid = row_src(a, bt, b, rl, jl) != nullptr;
+      ok = all_ok_softmax(mbar_wait(&S.s_full, it & 1, kErrSFull));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t v[64];
+      tmem_ld_32x32b_x64(tmem + ((uint32_t)(32 * warp) << 16) + kColS, v);
+      tmem_ld_wait();
+      float s[64];
+#pragma unroll
+      for (int h = 0; h < 64; ++h) s[h] = valid ? __uint_as_float(v[h]) * a.scale : -INFINITY;
+      float red2[2];
+      warp_reduce_scatter64<true>(s, red2);
+      S.red[warp][2 * lane] = red2[0];
+      S.red[warp][2 * lane + 1] = red2[1];
+      bar_softmax();
+      if (tid < kHg) {
+        const float cm = fmaxf(fmaxf(S.red[0][tid], S.red[1][tid]),
+                               fmaxf(S.red[2][tid], S.red[3][tid]));
+        const float mu = S.m_used[tid];
+        float al = 1.f;
+        if (cm > mu + kLazy || (mu == -INFINITY && cm != -INFINITY)) {
+          al = (mu == -INFINITY) ? 0.f : expf(mu - cm);
+          S.m_used[tid] = cm;
+        }
+        S.alpha[tid] = al;
+        S.l_sum[tid] *= al;
+      }
+      if (tid == 0) S.any_rescale = 0;
+      bar_softmax();
+      if (tid < kHg && S.alpha[tid] != 1.f && j > c0) S.any_rescale = 1;
+      bar_softmax();
+      if (S.any_rescale) {  // rare: scale O^T columns by alpha (previous O^T MMAs are done)
+#pragma unroll 1
+        for (int sl = 0; sl < 4; ++sl) {
+          uint32_t o[64];
+          const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16) + kColO + 64 * sl;
+          tmem_ld_32x32b_x64(ta, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int h = 0; h < 64; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * S.alpha[h]);
+          tmem_st_32x32b_x64(ta, o);
+        }
+        tmem_st_wait();
+      }
+      // P^T row (bf16) into the swizzled B-operand tile, and per-head row sums
+      float pr[64];
+      uint8_t* pt = base + kOffP;
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int h = 8 * c8 + 2 * k;
+          const float p0 = s[h] == -INFINITY ? 0.f : __expf(s[h] - S.m_used[h]);
+          const float p1 = s[h + 1] == -INFINITY ? 0.f : __expf(s[h + 1] - S.m_used[h + 1]);
+          const __nv_bfloat16 b0 = __float2bfloat16_rn(p0), b1 = __float2bfloat16_rn(p1);
+          pr[h] = __bfloat162float(b0);  // sum what the MMA multiplies
+          pr[h + 1] = __bfloat162float(b1);
+          pk[k] = (uint32_t)__bfloat16_as_ushort(b0) | ((uint32_t)__bfloat16_as_ushort(b1) << 16);
+        }
+        *reinterpret_cast<uint4*>(pt + sw128(row, c8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      warp_reduce_scatter64<false>(pr, red2);
+      bar_softmax();  // everyone has read S.red of the max pass
+      S.red[warp][2 * lane] = red2[0];
+      S.red[warp][2 * lane + 1] = red2[1];
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&S.p_full);
+      bar_softmax();
+      if (tid < kHg) S.l_sum[tid] += (S.red[0][tid] + S.red[1][tid]) + (S.red[2][tid] + S.red[3][tid]);
+    }
+    // ---- epilogue: wait for the last O^T, then finalise or write the partial ----
+    if (ok && c1 > c0)
+      ok = all_ok_softmax(mbar_wait(&S.kv_free, (uint32_t)(c1 - c0 - 1) & 1, kErrKvFree));
+    bar_softmax();
+    const bool single = P.nsplit == 1;
+    if (tid < kHg) {
+      const float m = S.m_used[tid], l = S.l_sum[tid];
+      if (single) {
+        const float zs = a.sink ? a.sink[h0 + tid] : -INFINITY;
+        float f = 0.f;
+        if (l > 0.f) {
+          const float M = fmaxf(m, zs);
+          f = expf(m - M) / (l * expf(m - M) + (zs == -INFINITY ? 0.f : expf(zs - M)));
+        }
+        S.fin[tid] = f;
+      } else {
+        float* pp = P.part + ((size_t)stream * P.nsplit + split) * (kHg * (kC + 2));
+        pp[tid] = m;
+        pp[kHg + tid] = l;
+      }
+    }
+    bar_softmax();
+    tc_fence_after();
+    const bool have = ok && c1 > c0;
+#pragma unroll 1
+    for (int sl = 0; sl < 4; ++sl) {
+      uint32_t o[64];
+      if (have) {
+        tmem_ld_32x32b_x64(tmem + ((uint32_t)(32 * warp) << 16) + kColO + 64 * sl, o);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int h = 0; h < 64; ++h) o[h] = 0u;
+      }
+      const int d = 128 * sl + tid;
+      if (single) {
+        float cs = 1.f, sn = 0.f;
+        const bool rot = d >= r0;
+        if (rot) {
+          cs = S.cs[(d - r0) >> 1];
+          sn = -S.sn[(d - r0) >> 1];  // rotation by -t
+        }
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) + ((size_t)bt * a.H + h0) * kC;
+#pragma unroll
+        for (int h = 0; h < 64; ++h) {
+          const float y = __uint_as_float(o[h]) * S.fin[h];
+          const float yp = __shfl_xor_sync(0xffffffffu, y, 1);
+          float z = y;
+          if (rot) z = (d & 1) == 0 ? y * cs - yp * sn : yp * sn + y * cs;
+          out[(size_t)h * kC + d] = __float2bfloat16_rn(z);
+        }
+      } else {
+        float* po = P.part + ((size_t)stream * P.nsplit + split) * (kHg * (kC + 2)) + 2 * kHg;
+#pragma unroll
+        for (int h = 0; h < 64; ++h) po[(size_t)h * kC + d] = __uint_as_float(o[h]);
+      }
+    }
+  } else {
+    // ------------------------------ MMA issuer (warp 4) ------------------------------
+    const uint32_t idS = idesc_f16(1, kRows, kHg);                       // K-major A and B
+    const uint32_t idO = idesc_f16(1, kRows, kHg) | (1u << 15) | (1u << 16);  // MN-major A, B
+    const uint32_t kv = smem_u32(base + kOffKV), qs = smem_u32(base + kOffQ),
+                   pt = smem_u32(base + kOffP);
+    bool ok = true;
+    for (int j = c0; j < c1 && ok; ++j) {
+      const uint32_t it = (uint32_t)(j - c0);
+      ok = __all_sync(0xffffffffu, mbar_wait(&S.kv_full, it & 1, kErrKvFull));
+      if (!ok) break;
+      tc_fence_after();
+      if (lane == 0) {
+#pragma unroll 1
+        for (int kk = 0; kk < 32; ++kk) {  // K = 512 in steps of 16
+          const uint32_t atom = kk >> 2, koff = (kk & 3) * 32;
+          const uint64_t ad = smem_desc(kv + atom * (kRows * 128) + koff, 16, 1024, kLayoutSw128);
+          const uint64_t bd = smem_desc(qs + atom * (kHg * 128) + koff, 16, 1024, kLayoutSw128);
+          mma_f16(tmem + kColS, ad, bd, idS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&S.s_full);
+      }
+      __syncwarp();
+      ok = __all_sync(0xffffffffu, mbar_wait(&S.p_full, it & 1, kErrPFull));
+      if (!ok) break;
+      tc_fence_after();
+      if (lane == 0) {
+#pragma unroll 1
+        for (int sl = 0; sl < 4; ++sl) {
+#pragma unroll 1
+          for (int kk = 0; kk < kRows / 16; ++kk) {  // K = 128 rows in steps of 16
+            const uint64_t ad = smem_desc(kv + sl * 2 * (kRows * 128) + kk * 2048, kRows * 128,
+                                          1024, kLayoutSw128);
+            const uint64_t bd = smem_desc(pt + kk * 2048, kRows * 128, 1024, kLayoutSw128);
+            mma_f16(tmem + kColO + 64 * sl, ad, bd, idO, (j > c0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit(&S.kv_free);
+      }
+      __syncwarp();
+    }
+    if (lane == 0) {  // nothing this thread issued is in flight once `done` fires
+      mma_commit(&S.done);
+      mbar_wait(&S.done, 0, kErrKvFree);
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Merge the partials of each stream (fixed split order), add the sink, rotate by -t.
+__global__ void __launch_bounds__(256) k_mqa_combine(MqaTcParams P) {
+  const MqaArgs& a = P.a;
+  const int stream = blockIdx.x, h = blockIdx.y;
+  const int bt = stream / P.G, g = stream % P.G;
+  const int64_t t = a.q_pos[bt];
+  const int tid = threadIdx.x;
+  const size_t stride = kHg * (kC + 2);
+  const float* base = P.part + (size_t)stream * P.nsplit * stride;
+  float M = -INFINITY;
+  for (int sp = 0; sp < P.nsplit; ++sp) M = fmaxf(M, base[sp * stride + h]);
+  const float zs = a.sink ? a.sink[g * kHg + h] : -INFINITY;
+  const float Mt = fmaxf(M, zs);
+  float l = 0.f, o0 = 0.f, o1 = 0.f;
+  const int d = 2 * tid;
+  for (int sp = 0; sp < P.nsplit; ++sp) {
+    const float* pp = base + sp * stride;
+    const float m = pp[h];
+    if (m == -INFINITY) continue;
+    const float f = expf(m - Mt);
+    l = fmaf(pp[kHg + h], f, l);
+    const float2 ov = *reinterpret_cast<const float2*>(pp + 2 * kHg + (size_t)h * kC + d);
+    o0 = fmaf(ov.x, f, o0);
+    o1 = fmaf(ov.y, f, o1);
+  }
+  float y0 = 0.f, y1 = 0.f;
+  const float den = l + (zs == -INFINITY ? 0.f : expf(zs - Mt));
+  if (l > 0.f) {
+    y0 = o0 / den;
+    y1 = o1 / den;
+  }
+  const int r = a.rope_dims, r0 = kC - r;
+  if (d >= r0) {
+    float cs, sn;
+    rope_cos_sin(-(double)t, (d - r0) >> 1, r, (double)a.rope_base, &cs, &sn);
+    const float u0 = y0 * cs - y1 * sn, u1 = y0 * sn + y1 * cs;
+    y0 = u0;
+    y1 = u1;
+  }
+  __nv_bfloat16* out =
+      static_cast<__nv_bfloat16*>(a.out) + ((size_t)bt * a.H + g * kHg + h) * kC + d;
+  *reinterpret_cast<__nv_bfloat162*>(out) = __floats2bfloat162_rn(y0, y1);
+}
+
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = 148;
+    }
+  }
+  return n;
+}
+
+int choose_nsplit(const MqaArgs& a) {
+  const int64_t streams = (int64_t)a.B * a.T * (a.H / kHg);
+  const int64_t rows_max = (a.k > 0 ? a.k : a.n_cap) + a.n_win;
+  const int64_t chunks_max = (rows_max + kRows - 1) / kRows;
+  int64_t ns = sm_count() / (streams > 0 ? streams : 1);
+  if (ns < 1) ns = 1;
+  if (ns > chunks_max) ns = chunks_max > 0 ? chunks_max : 1;
+  return (int)ns;
+}
+
+}  // namespace
+
+bool mqa_tc_supported(const MqaArgs& a, bool bf16) {
+  return bf16 && a.c == kC && a.H % kHg == 0 && a.rope_dims <= kC && a.rope_dims % 2 == 0 &&
+         a.rope_dims / 2 <= 256;
+}
+
+size_t mqa_tc_workspace_bytes(const MqaArgs& a) {
+  const int ns = choose_nsplit(a);
+  if (ns <= 1) return 0;
+  const size_t streams = (size_t)a.B * a.T * (a.H / kHg);
+  return streams * ns * kHg * (kC + 2) * sizeof(float);
+}
+
+cudaError_t launch_mqa_tc(const MqaArgs& a, void* ws, size_t ws_bytes, cudaStream_t st) {
+  MqaTcParams P;
+  P.a = a;
+  P.G = a.H / kHg;
+  P.nsplit = choose_nsplit(a);
+  P.part = P.nsplit > 1 ? static_cast<float*>(ws) : nullptr;
+  if (P.nsplit > 1 && ws_bytes < mqa_tc_workspace_bytes(a)) return cudaErrorInvalidValue;
+  const int64_t streams = (int64_t)a.B * a.T * P.G;
+  const size_t smem = 1024 + kOffEnd + sizeof(Smem);
+  cudaError_t e = cudaFuncSetAttribute(k_mqa_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  k_mqa_tc<<<(unsigned)(streams * P.nsplit), kThreads, smem, st>>>(P);
+  if (P.nsplit > 1) {
+    dim3 grid((unsigned)streams, kHg);
+    k_mqa_combine<<<grid, 256, 0, st>>>(P);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t mqa_tc_device_error(int* code) {
+  int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(code, tc::g_device_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyToSymbol(tc::g_device_error, &zero, sizeof(int));
+}
+
+}  // namespace csa
