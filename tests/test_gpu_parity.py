@@ -140,9 +140,11 @@ def test_sparse_mqa_parity_on_oracle_selection(name):
     p = R.params_for(s)
     io = csa.CSA_BF16 if s.io == "bf16" else csa.CSA_F32
     out = torch.empty((s.B, s.T, s.n_heads, s.c), dtype=dev["q"].dtype, device="cuda")
+    ws_bytes = csa.workspace_size(p, csa.CSA_WS_SPARSE_MQA, 0, s.B, s.T, s.n_cap)
+    ws = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device="cuda")
     csa.csa_sparse_mqa(p, io, s.B, s.T, dev["q"], dev["q_pos"], dev["kv_cache"], s.n_cap,
                        torch.from_numpy(idx).cuda(), dev["win_kv"], dev["win_kv"].shape[1],
-                       dev["win_pos0"], dev["sink"], None, out, None, 0)
+                       dev["win_pos0"], dev["sink"], None, out, ws, ws_bytes)
     torch.cuda.synchronize()
     got = out.float().cpu().numpy()
     for (b, ti), r in ref.items():
