@@ -176,6 +176,27 @@ size_t scores_bytes(int32_t B, int32_t T, int64_t N_cap) {
   return round_up((size_t)B * T * (size_t)N_cap * sizeof(float));
 }
 
+// index scores, then top-k; for few long rows the indexer also fills the top-k histogram
+csa_status index_then_topk(const csa_params* p, csa_dtype kdt, int32_t B, int32_t T,
+                           int64_t N_cap, const void* qI, const void* qI_scale, const float* w,
+                           const void* KI, const void* KI_scale, const int64_t* q_pos,
+                           float* scores, const csa::TopkArgs& t, void* topk_ws,
+                           size_t topk_bytes, cudaStream_t st) {
+  bool hist_done = false;
+  const bool decode = csa::topk_decode_path(B, T, N_cap, p->topk);
+  if (N_cap > 0) {
+    auto ia = make_index(p, kdt, B, T, N_cap, qI, qI_scale, w, KI, KI_scale, q_pos, scores);
+    if (decode) {
+      const csa::TopkDecodeArgs da = csa::topk_decode_args(t, topk_ws);
+      TRY(cuda_status(csa::topk_decode_clear(da, st), "top-k clear"));
+      ia.hist = da.hist;
+    }
+    TRY(cuda_status(csa::launch_index_scores(ia, st, &hist_done), "index scores"));
+  }
+  TRY(cuda_status(csa::launch_topk(t, topk_ws, topk_bytes, st, hist_done), "top-k"));
+  return CSA_OK;
+}
+
 }  // namespace
 
 namespace csa {
@@ -343,14 +364,11 @@ csa_status csa_index_topk(const csa_params* p, csa_dtype kdt, int32_t B, int32_t
   char* topk_ws = base + scores_bytes(B, T, N_cap);
   const size_t topk_bytes = need - scores_bytes(B, T, N_cap);
   cudaStream_t st = (cudaStream_t)stream;
-  if (N_cap > 0) {
-    auto a = make_index(p, kdt, B, T, N_cap, qI, qI_scale, w, KI, KI_scale, q_pos, scores);
-    TRY(cuda_status(csa::launch_index_scores(a, st), "index scores"));
-  }
   csa::TopkArgs t{};
   t.B = B; t.T = T; t.m = p->m; t.k = p->topk; t.n_cap = N_cap; t.scores = scores;
   t.q_pos = q_pos; t.out_idx = out_idx;
-  TRY(cuda_status(csa::launch_topk(t, topk_ws, topk_bytes, st), "top-k"));
+  TRY(index_then_topk(p, kdt, B, T, N_cap, qI, qI_scale, w, KI, KI_scale, q_pos, scores, t,
+                      topk_ws, topk_bytes, st));
   return ok();
 }
 
@@ -417,15 +435,11 @@ csa_status csa_forward(const csa_params* p, csa_dtype io, int32_t B, int32_t T,
   const size_t sb = scores_bytes(B, T, a->N_cap);
   const size_t tb = round_up(csa::topk_workspace_bytes(B, T, a->N_cap, p->topk));
   float* scores = a->out_scores ? a->out_scores : reinterpret_cast<float*>(base);
-  if (a->N_cap > 0) {
-    auto ia = make_index(p, a->idx_dtype, B, T, a->N_cap, a->qI, a->qI_scale, a->w, a->KI,
-                         a->KI_scale, a->q_pos, scores);
-    TRY(cuda_status(csa::launch_index_scores(ia, st), "index scores"));
-  }
   csa::TopkArgs t{};
   t.B = B; t.T = T; t.m = p->m; t.k = p->topk; t.n_cap = a->N_cap; t.scores = scores;
   t.q_pos = a->q_pos; t.out_idx = a->out_idx;
-  TRY(cuda_status(csa::launch_topk(t, base + sb, tb, st), "top-k"));
+  TRY(index_then_topk(p, a->idx_dtype, B, T, a->N_cap, a->qI, a->qI_scale, a->w, a->KI,
+                      a->KI_scale, a->q_pos, scores, t, base + sb, tb, st));
   auto ma = make_mqa(p, B, T, a->q, a->q_pos, a->kv_cache, a->N_cap, a->out_idx, p->topk,
                      a->win_kv, a->L_raw, a->win_pos0, a->sink, a->q_rms_w, a->out);
   TRY(cuda_status(csa::launch_mqa(ma, io == CSA_BF16, base + sb + tb, ws_bytes - sb - tb, st),

@@ -86,17 +86,21 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 }
 
 // ---------------------------------------------------------------------------
-// RoPE angles: computed in double so that positions up to ~1e6 keep full fp32 accuracy
-// after reduction (pos * theta_p in fp32 would lose ~0.06 rad at pos 1e6).
-// Pair p of the last r dims turns by pos * base^(-2p/r).
+// RoPE angles. Pair p of the last r dims turns by pos * base^(-2p/r). The angle reaches
+// ~1e6 rad at 1M positions, so it is formed in double and reduced modulo 2*pi with a
+// two-part 2*pi (Cody-Waite); the reduced angle (|a| <= pi) then goes through fp32
+// sincosf. Error ~1e-10 rad before the fp32 evaluation, which adds ~1 ulp.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void rope_cos_sin(double pos, int p, int r, double base, float* cs,
                                              float* sn) {
-  const double inv_freq = pow(base, -2.0 * (double)p / (double)r);
-  double s, c;
-  sincos(pos * inv_freq, &s, &c);
-  *cs = (float)c;
-  *sn = (float)s;
+  const double inv_freq = exp2(-2.0 * (double)p / (double)r * log2(base));
+  const double x = pos * inv_freq;
+  const double kTwoPiHi = 6.283185307179586232;     // nearest double to 2*pi
+  const double kTwoPiLo = 2.4492935982947064e-16;   // 2*pi - kTwoPiHi
+  const double k = rint(x * 0.15915494309189535);   // x / (2*pi)
+  double red = fma(-k, kTwoPiHi, x);
+  red = fma(-k, kTwoPiLo, red);
+  sincosf((float)red, sn, cs);
 }
 
 }  // namespace csa

@@ -133,9 +133,13 @@ __global__ void __launch_bounds__(kKeysPerCta) k_index_scores_cc(IndexArgs a) {
 
 }  // namespace
 
-cudaError_t launch_index_scores(const IndexArgs& a, cudaStream_t st) {
+cudaError_t launch_index_scores(const IndexArgs& a, cudaStream_t st, bool* hist_done) {
+  if (hist_done) *hist_done = false;
   if (a.B == 0 || a.T == 0 || a.n_cap == 0) return cudaSuccess;
-  if (index_mxf4_tc_supported(a)) return launch_index_mxf4_tc(a, st);
+  if (index_mxf4_tc_supported(a)) {
+    if (hist_done) *hist_done = a.hist != nullptr;
+    return launch_index_mxf4_tc(a, st);
+  }
   dim3 grid((unsigned)((a.n_cap + kKeysPerCta - 1) / kKeysPerCta), a.B * a.T);
   const size_t smem = ((size_t)a.n_idx_heads * a.d_idx + a.n_idx_heads) * sizeof(float);
   timing_before(st);

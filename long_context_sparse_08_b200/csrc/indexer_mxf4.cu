@@ -65,14 +65,33 @@ struct Mxf4Params {
   const int64_t* q_pos;
   const float* w;
   float* scores;
+  int* hist;  // optional [Q][4096] histogram of the scores' top 12 key bits
 };
+
+constexpr int kBins = 4096;
 
 struct Smem {
   uint64_t full[kStages], empty[kStages], tfull[2], tempty[2], done;
   uint32_t tmem_slot;
   int prefix[kMaxQueries + 1];
   int nvis[kMaxQueries];
+  int hist[kBins];
 };
+
+// named barrier of the 4 epilogue warps; returns the AND of `ok` over them
+__device__ __forceinline__ bool epi_all_ok(bool ok) {
+  uint32_t res;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 2, 128, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(res)
+      : "r"((uint32_t)ok)
+      : "memory");
+  return res != 0;
+}
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 
 __device__ __forceinline__ int find_query(const int* prefix, int Q, int u) {
   int lo = 0, hi = Q;  // largest q with prefix[q] <= u
@@ -220,6 +239,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------ epilogue ------------------------------
     const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+    const int etid = threadIdx.x - 64;
+    const bool hist = p.hist != nullptr;
+    if (hist) {
+      for (int i = etid; i < kBins; i += 128) S.hist[i] = 0;
+      epi_bar();
+    }
+    int hq = -1;
+    auto flush = [&](int qq) {  // smem histogram of query qq -> global, then clear
+      epi_bar();
+      for (int i = etid; i < kBins; i += 128) {
+        const int v = S.hist[i];
+        if (v) {
+          atomicAdd(&p.hist[(size_t)qq * kBins + i], v);
+          S.hist[i] = 0;
+        }
+      }
+      epi_bar();
+    };
     float wr[kHeads];
     int cur_q = -1;
     int q = u0 < u1 ? find_query(S.prefix, p.Q, u0) : 0;
@@ -232,9 +269,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int h = 0; h < kHeads; ++h) wr[h] = p.w[(size_t)q * kHeads + h];
         cur_q = q;
       }
+      if (hist && q != hq) {
+        if (hq >= 0) flush(hq);
+        hq = q;
+      }
       const int acc = k & 1;
       const uint32_t around = (uint32_t)(k >> 1);
-      if (!mbar_wait(&S.tfull[acc], around & 1, kErrTmemFull)) break;
+      if (!epi_all_ok(mbar_wait(&S.tfull[acc], around & 1, kErrTmemFull))) break;
       tc_fence_after();
       uint32_t v[kHeads];
       tmem_ld_32x32b_x64(tmem + ((uint32_t)(32 * quad) << 16) + acc_col(acc), v);
@@ -246,8 +287,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int h = 0; h < kHeads; ++h) sc = fmaf(wr[h], fmaxf(__uint_as_float(v[h]), 0.f), sc);
       const int s = tile * kTileKeys + 32 * quad + lane;
-      if (s < S.nvis[q]) p.scores[(size_t)q * p.n_cap + s] = sc;
+      if (s < S.nvis[q]) {
+        p.scores[(size_t)q * p.n_cap + s] = sc;
+        if (hist) atomicAdd(&S.hist[float_key(sc) >> 20], 1);
+      }
     }
+    if (hist && hq >= 0) flush(hq);
   }
   // ---- teardown: the MMA warp saw its last MMA complete; free TMEM ----
   __syncthreads();
@@ -322,7 +367,7 @@ cudaError_t launch_index_mxf4_tc(const IndexArgs& a, cudaStream_t st) {
       !make_map_2d(&mq, a.qI, (uint64_t)Q * kHeads, kHeads) ||
       !make_map_1d_words(&mqs, a.qI_scale, (uint64_t)Q * kHeads, kHeads))
     return cudaErrorInvalidValue;
-  Mxf4Params p{Q, a.T, a.m, a.n_cap, a.q_pos, a.w, a.scores};
+  Mxf4Params p{Q, a.T, a.m, a.n_cap, a.q_pos, a.w, a.scores, a.hist};
   const int64_t units_max = (int64_t)Q * ((a.n_cap + kTileKeys - 1) / kTileKeys);
   const int grid = (int)(units_max < num_sms() ? (units_max > 0 ? units_max : 1) : num_sms());
   const size_t smem = 1024 + (size_t)kStages * kStageBytes + sizeof(Smem);

@@ -24,8 +24,10 @@ struct IndexArgs {
   const float* w;
   const int64_t* q_pos;
   float* scores;  // [B, T, n_cap]
+  int* hist;      // optional [B*T][4096] histogram of the scores' top 12 key bits (zeroed)
 };
-cudaError_t launch_index_scores(const IndexArgs& a, cudaStream_t st);
+// *hist_done: whether the launched kernel also filled a.hist
+cudaError_t launch_index_scores(const IndexArgs& a, cudaStream_t st, bool* hist_done = nullptr);
 // tensor-core kernel for MXFP4 keys (64 heads x 128 dims, N_cap % 32 == 0)
 bool index_mxf4_tc_supported(const IndexArgs& a);
 cudaError_t launch_index_mxf4_tc(const IndexArgs& a, cudaStream_t st);
@@ -39,7 +41,26 @@ struct TopkArgs {
   int32_t* out_idx;
 };
 size_t topk_workspace_bytes(int B, int T, int64_t n_cap, int k);
-cudaError_t launch_topk(const TopkArgs& a, void* ws, size_t ws_bytes, cudaStream_t st);
+cudaError_t launch_topk(const TopkArgs& a, void* ws, size_t ws_bytes, cudaStream_t st,
+                        bool hist_ready = false);
+
+// few long rows (decode): histogram + filter + last-CTA selection
+struct TopkDecodeArgs {
+  int Q, m, k, nslice;
+  int64_t n_cap;
+  const float* scores;
+  const int64_t* q_pos;
+  int32_t* out_idx;
+  int* hist;          // [Q][4096]
+  int* cnt;           // [Q][4]: sure count, boundary count, ticket
+  uint64_t* sure;     // [Q][k]
+  uint64_t* bnd;      // [Q][n_cap]
+};
+bool topk_decode_path(int B, int T, int64_t n_cap, int k);
+size_t topk_decode_ws_bytes(int B, int T, int64_t n_cap, int k);
+TopkDecodeArgs topk_decode_args(const TopkArgs& t, void* ws);
+cudaError_t topk_decode_clear(const TopkDecodeArgs& a, cudaStream_t st);
+cudaError_t launch_topk_decode(TopkDecodeArgs a, bool hist_ready, cudaStream_t st);
 
 struct MqaArgs {
   int B, T, m, H, c, rope_dims, n_win, k;  // k = 0: dense (all visible entries)

@@ -153,10 +153,18 @@ __global__ void __launch_bounds__(kThreads) k_topk_rows(TopkArgs a) {
 
 }  // namespace
 
-size_t topk_workspace_bytes(int, int, int64_t, int) { return 0; }
+size_t topk_workspace_bytes(int B, int T, int64_t n_cap, int k) {
+  return topk_decode_path(B, T, n_cap, k) ? topk_decode_ws_bytes(B, T, n_cap, k) : 0;
+}
 
-cudaError_t launch_topk(const TopkArgs& a, void*, size_t, cudaStream_t st) {
+cudaError_t launch_topk(const TopkArgs& a, void* ws, size_t ws_bytes, cudaStream_t st,
+                        bool hist_ready) {
   if (a.B == 0 || a.T == 0) return cudaSuccess;
+  if (topk_decode_path(a.B, a.T, a.n_cap, a.k)) {
+    if (ws == nullptr || ws_bytes < topk_decode_ws_bytes(a.B, a.T, a.n_cap, a.k))
+      return cudaErrorInvalidValue;
+    return launch_topk_decode(topk_decode_args(a, ws), hist_ready, st);
+  }
   k_topk_rows<<<a.B * a.T, kThreads, 0, st>>>(a);
   return cudaGetLastError();
 }

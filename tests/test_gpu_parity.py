@@ -82,7 +82,8 @@ def test_compress_parity(name):
 # ---------------------------------------------------------------------------
 
 INDEX_CASES = ["tiny_prefill_f32", "mid_decode_fp8", "mid_decode_mxfp4", "mid_decode_bf16",
-               "edge_decode_bf16", "edge_decode_mxfp4", "mid_prefill_bf16"]
+               "edge_decode_bf16", "edge_decode_mxfp4", "edge_decode_mxfp4_long",
+               "mid_prefill_bf16"]
 
 
 @pytest.mark.parametrize("name", INDEX_CASES)
@@ -120,6 +121,34 @@ def test_topk_exact_on_given_scores(k):
             nv = O.visible_entries(int(pos[b, t]), 4, N)
             ref = O.topk_select(sc[b, t, :nv].astype(np.float64), k)
             np.testing.assert_array_equal(got[b, t], ref, err_msg=f"b={b} t={t} k={k}")
+
+
+@pytest.mark.parametrize("k", [512, 1024, 2000])
+def test_topk_exact_on_given_scores_long_rows(k):
+    # few long rows: the multi-CTA histogram / filter / last-CTA selection path
+    g = np.random.default_rng(200 + k)
+    B, T, N = 2, 3, 40000
+    sc = np.round(g.standard_normal((B, T, N)).astype(np.float32) * 4, 1)  # heavy ties
+    sc[0, 1, :500] = -0.0
+    sc[0, 1, 500:900] = 0.0
+    sc[1, 0] = -2.5  # every score equal
+    sc[1, 2, ::7] = 1e30
+    pos = np.array([[4 * N + 9, 4 * 30000, 4 * (k - 3)], [4 * N, 4 * 39999 + 3, 4 * (k + 1)]],
+                   np.int64)
+    p = csa.make_params(topk=k)
+    ws_bytes = csa.workspace_size(p, csa.CSA_WS_TOPK, 0, B, T, N)
+    assert ws_bytes > 0
+    ws = torch.empty((ws_bytes,), dtype=torch.uint8, device="cuda")
+    out = torch.empty((B, T, k), dtype=torch.int32, device="cuda")
+    for _ in range(2):  # the workspace is reused: counters must be reset per call
+        csa.csa_topk(p, B, T, N, torch.from_numpy(sc).cuda(), torch.from_numpy(pos).cuda(),
+                     out, ws, ws_bytes)
+        got = out.cpu().numpy()
+        for b in range(B):
+            for t in range(T):
+                nv = O.visible_entries(int(pos[b, t]), 4, N)
+                ref = O.topk_select(sc[b, t, :nv].astype(np.float64), k)
+                np.testing.assert_array_equal(got[b, t], ref, err_msg=f"b={b} t={t} k={k}")
 
 
 # ---------------------------------------------------------------------------
@@ -200,7 +229,7 @@ def _forward_parity(name, queries=None):
 
 @pytest.mark.parametrize("name", ["tiny_prefill_f32", "mid_decode_fp8", "mid_decode_mxfp4",
                                   "mid_decode_bf16", "edge_decode_bf16", "edge_decode_mxfp4",
-                                  "mid_prefill_bf16"])
+                                  "edge_decode_mxfp4_long", "mid_prefill_bf16"])
 def test_forward_parity(name):
     _forward_parity(name)
     assert csa.device_error() == 0
