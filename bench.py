@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="budget of the oracle CPU baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--replicas", type=int, default=0,
+                    help="input replicas rotated across steps (0: enough to defeat the L2)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end measurement")
     return ap.parse_args()
 
 
@@ -199,6 +202,8 @@ def run_ours(args, W, rank, world, local_rank):
     free = torch.cuda.mem_get_info()[0]
     while R_rep > 2 and R_rep * one_set > 0.6 * free:
         R_rep -= 1
+    if args.replicas > 0:
+        R_rep = args.replicas
     devs = [dev0] + [{k: v.clone() for k, v in dev0.items()} for _ in range(R_rep - 1)]
     steps = [R.Step(s, d) for d in devs]
     stream = torch.cuda.current_stream()
@@ -241,7 +246,7 @@ def run_ours(args, W, rank, world, local_rank):
 
     # end to end through the public API: per-step query-side inputs from pinned host
     # memory, the call, and the result back to pinned host memory
-    e2e = run_e2e(args, s, devs, steps, R_rep, world)
+    e2e = None if args.no_e2e else run_e2e(args, s, devs, steps, R_rep, world)
 
     n_vis = min(s.ctx // s.m, s.n_cap) if s.kind != "csa_prefill" else s.n_cap
     per_q = algorithmic_bytes_per_query(s, n_vis)

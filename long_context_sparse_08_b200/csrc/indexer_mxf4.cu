@@ -16,8 +16,8 @@
 //           copies into TMEM (row 32*j + i of the tile -> lane i, column j; the 4 bytes of
 //           a column are the row's 4 block scales), then issues the copy and the 2 MMAs;
 //   warps 2-5 epilogue: TMEM -> registers (32x32b.x64), w * ReLU head sum, fp32 store.
-// Accumulators are double-buffered in TMEM so the epilogue of tile j overlaps the MMA of
-// tile j+1 and the loads of the tiles after it. Work (query, tile) pairs are split
+// Four accumulator slots in TMEM let the MMAs of tiles j+1..j+3 run while the epilogue
+// reduces tile j. Work (query, tile) pairs are split
 // evenly over the CTAs; ragged per-query visibility is handled by masking the stores.
 #include <cudaTypedefs.h>
 
@@ -51,10 +51,11 @@ constexpr uint32_t kStageTx = kTileKeys * kRowBytes + kHeads * kRowBytes + kTile
                               kHeads * 4;
 
 // TMEM columns
-constexpr uint32_t kTmemCols = 256;
-__device__ __forceinline__ uint32_t acc_col(int acc) { return 64u * acc; }         // 0, 64
-__device__ __forceinline__ uint32_t sfa_col(int acc) { return 128u + 16u * acc; }  // 128, 144
-__device__ __forceinline__ uint32_t sfb_col(int acc) { return 160u + 16u * acc; }  // 160, 176
+constexpr int kAcc = 4;  // accumulator slots in TMEM
+constexpr uint32_t kTmemCols = 512;
+__device__ __forceinline__ uint32_t acc_col(int acc) { return 64u * acc; }         // 0..192
+__device__ __forceinline__ uint32_t sfa_col(int acc) { return 256u + 32u * acc; }  // 256..352
+__device__ __forceinline__ uint32_t sfb_col(int acc) { return 272u + 32u * acc; }  // 272..368
 
 // device error codes of this kernel
 enum { kErrFull = 101, kErrEmpty = 102, kErrTmemFull = 103, kErrTmemEmpty = 104 };
@@ -71,7 +72,7 @@ struct Mxf4Params {
 constexpr int kBins = 4096;
 
 struct Smem {
-  uint64_t full[kStages], empty[kStages], tfull[2], tempty[2], done;
+  uint64_t full[kStages], empty[kStages], tfull[kAcc], tempty[kAcc], done;
   uint32_t tmem_slot;
   int prefix[kMaxQueries + 1];
   int nvis[kMaxQueries];
@@ -141,7 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&S.full[i], 1);
         mbar_init(&S.empty[i], 1);
       }
-      for (int i = 0; i < 2; ++i) {
+      for (int i = 0; i < kAcc; ++i) {
         mbar_init(&S.tfull[i], 1);
         mbar_init(&S.tempty[i], 4);
       }
@@ -196,8 +197,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int u = u0; u < u1 && ok; ++u, ++k) {
       const int st = k % kStages;
       const uint32_t round = (uint32_t)(k / kStages);
-      const int acc = k & 1;
-      const uint32_t around = (uint32_t)(k >> 1);
+      const int acc = k % kAcc;
+      const uint32_t around = (uint32_t)(k / kAcc);
       ok = mbar_wait(&S.full[st], round & 1, kErrFull);
       if (!ok) break;
       uint8_t* sb = base + st * kStageBytes;
@@ -273,8 +274,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (hq >= 0) flush(hq);
         hq = q;
       }
-      const int acc = k & 1;
-      const uint32_t around = (uint32_t)(k >> 1);
+      const int acc = k % kAcc;
+      const uint32_t around = (uint32_t)(k / kAcc);
       if (!epi_all_ok(mbar_wait(&S.tfull[acc], around & 1, kErrTmemFull))) break;
       tc_fence_after();
       uint32_t v[kHeads];

@@ -55,6 +55,7 @@ struct Smem {
   float red[4][kHg];
   float m_used[kHg], l_sum[kHg], alpha[kHg], fin[kHg];
   float cs[256], sn[256];  // RoPE table for pairs of the last r dims
+  const __nv_bfloat16* src[kRows];  // source rows of the current chunk (nullptr: masked)
 };
 
 struct MqaTcParams {
@@ -304,9 +305,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
       const uint32_t it = (uint32_t)(j - c0);
       if (j > c0) ok = all_ok_softmax(mbar_wait(&S.kv_free, (it - 1) & 1, kErrKvFree));
       if (!ok) break;
-      // ---- gather the chunk's 128 rows: warp w loads rows w, w+4, ...; lane = 16B chunk ----
+      // ---- gather the chunk's 128 rows: thread r resolves row r, then warp w copies rows
+      //      w, w+4, ... with lane = 16-byte chunk (coalesced 512 B per instruction) ----
+      const __nv_bfloat16* my_src = row_src(a, bt, b, rl, (int64_t)j * kRows + tid);
+      S.src[tid] = my_src;
+      bar_softmax();
       for (int rr = warp; rr < kRows; rr += 4) {
-        const __nv_bfloat16* src = row_src(a, bt, b, rl, (int64_t)j * kRows + rr);
+        const __nv_bfloat16* src = S.src[rr];
 #pragma unroll
         for (int hseg = 0; hseg < 2; ++hseg) {
           const int gch = lane + 32 * hseg;  // 16-byte chunk of the 1 KB row
@@ -322,8 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
 
       // ---- softmax of S^T (thread = row) ----
       const int row = tid;
-      const int64_t jl = (int64_t)j * kRows + row;
-      const bool valid = row_src(a, bt, b, rl, jl) != nullptr;
+      const bool valid = my_src != nullptr;
       ok = all_ok_softmax(mbar_wait(&S.s_full, it & 1, kErrSFull));
       if (!ok) break;
       tc_fence_after();
@@ -515,21 +519,28 @@ __global__ void __launch_bounds__(256) k_mqa_combine(MqaTcParams P) {
   const int tid = threadIdx.x;
   const size_t stride = kHg * (kC + 2);
   const float* base = P.part + (size_t)stream * P.nsplit * stride;
+  constexpr int kMaxSplit = 32;  // choose_nsplit never exceeds this
+  float ms[kMaxSplit];
   float M = -INFINITY;
-  for (int sp = 0; sp < P.nsplit; ++sp) M = fmaxf(M, base[sp * stride + h]);
+#pragma unroll
+  for (int sp = 0; sp < kMaxSplit; ++sp) {
+    ms[sp] = sp < P.nsplit ? base[sp * stride + h] : -INFINITY;
+    M = fmaxf(M, ms[sp]);
+  }
   const float zs = a.sink ? a.sink[g * kHg + h] : -INFINITY;
   const float Mt = fmaxf(M, zs);
   float l = 0.f, o0 = 0.f, o1 = 0.f;
   const int d = 2 * tid;
-  for (int sp = 0; sp < P.nsplit; ++sp) {
-    const float* pp = base + sp * stride;
-    const float m = pp[h];
-    if (m == -INFINITY) continue;
-    const float f = expf(m - Mt);
-    l = fmaf(pp[kHg + h], f, l);
-    const float2 ov = *reinterpret_cast<const float2*>(pp + 2 * kHg + (size_t)h * kC + d);
-    o0 = fmaf(ov.x, f, o0);
-    o1 = fmaf(ov.y, f, o1);
+#pragma unroll
+  for (int sp = 0; sp < kMaxSplit; ++sp) {
+    if (sp < P.nsplit && ms[sp] != -INFINITY) {
+      const float* pp = base + sp * stride;
+      const float f = expf(ms[sp] - Mt);
+      l = fmaf(pp[kHg + h], f, l);
+      const float2 ov = *reinterpret_cast<const float2*>(pp + 2 * kHg + (size_t)h * kC + d);
+      o0 = fmaf(ov.x, f, o0);
+      o1 = fmaf(ov.y, f, o1);
+    }
   }
   float y0 = 0.f, y1 = 0.f;
   const float den = l + (zs == -INFINITY ? 0.f : expf(zs - Mt));
@@ -570,6 +581,7 @@ int choose_nsplit(const MqaArgs& a) {
   int64_t ns = sm_count() / (streams > 0 ? streams : 1);
   if (ns < 1) ns = 1;
   if (ns > chunks_max) ns = chunks_max > 0 ? chunks_max : 1;
+  if (ns > 32) ns = 32;
   return (int)ns;
 }
 

@@ -21,6 +21,7 @@ namespace {
 
 constexpr int kBins = 4096;
 constexpr int kFThreads = 512;
+constexpr int kBndCache = 2048;  // boundary entries kept in shared memory for the final pass
 
 __device__ __forceinline__ int64_t visible(const int64_t* q_pos, int q, int m, int64_t n_cap) {
   const int64_t t = q_pos[q];
@@ -81,13 +82,17 @@ __global__ void __launch_bounds__(kFThreads) k_topk_hist(TopkDecodeArgs a) {
 }
 
 __global__ void __launch_bounds__(kFThreads) k_topk_filter(TopkDecodeArgs a) {
-  __shared__ int h[kBins];
+  // the histogram is dead once the threshold bin is known; the final pass reuses it
+  __shared__ __align__(16) uint64_t hbuf[kBndCache];
+  static_assert(kBndCache * 8 == kBins * 4, "boundary cache aliases the histogram");
+  int* h = reinterpret_cast<int*>(hbuf);
+  uint64_t* bcache = hbuf;
   __shared__ int wsum[kFThreads / 32 + 1];
   __shared__ int s_bin, s_above, s_last;
   __shared__ uint64_t pairs[kMaxTopk];
   __shared__ int hist256[256];
   __shared__ uint32_t s_digit;
-  __shared__ int s_dabove, s_fill;
+  __shared__ int s_dabove, s_fill, s_fill_exact;
   const int q = blockIdx.y, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int64_t n = visible(a.q_pos, q, a.m, a.n_cap);
   const int k = a.k;
@@ -164,16 +169,26 @@ __global__ void __launch_bounds__(kFThreads) k_topk_filter(TopkDecodeArgs a) {
   if (tid == 0) s_fill = ns;
   __syncthreads();
   if (kk > 0) {
+    const bool cached = nb <= kBndCache;
+    if (cached)
+      for (int i = tid; i < nb; i += blockDim.x) bcache[i] = bnd[i];
+    __syncthreads();
+    const uint64_t* L = cached ? bcache : bnd;
     uint64_t thr = 0;  // take every boundary value >= thr
     if (kk < nb) {
-      uint64_t prefix = 0, mask = 0;
+      // every boundary value shares the top 12 key bits (bin T): start below them
+      uint64_t prefix = (uint64_t)T << 52, mask = (uint64_t)0xfff << 52;
       int need = kk;
-      for (int shift = 56; shift >= 0; shift -= 8) {
+      for (int hi_bit = 52; hi_bit > 0;) {
+        const int width = hi_bit >= 8 ? 8 : hi_bit;
+        const int shift = hi_bit - width;
+        const uint64_t dmask = ((uint64_t)1 << width) - 1;
         for (int i = tid; i < 256; i += blockDim.x) hist256[i] = 0;
+        if (tid == 0) s_fill_exact = 0;
         __syncthreads();
         for (int i = tid; i < nb; i += blockDim.x) {
-          const uint64_t v = bnd[i];
-          if ((v & mask) == prefix) atomicAdd(&hist256[(v >> shift) & 0xff], 1);
+          const uint64_t v = L[i];
+          if ((v & mask) == prefix) atomicAdd(&hist256[(v >> shift) & dmask], 1);
         }
         __syncthreads();
         if (tid < 32) {
@@ -195,20 +210,24 @@ __global__ void __launch_bounds__(kFThreads) k_topk_filter(TopkDecodeArgs a) {
             if (above < need && above + c[j] >= need) {
               s_digit = 255 - 8 * lane - j;
               s_dabove = above;
+              s_fill_exact = (above + c[j] == need);  // the digit's bucket is taken whole
             }
             above += c[j];
           }
         }
         __syncthreads();
         prefix |= (uint64_t)s_digit << shift;
-        mask |= (uint64_t)0xff << shift;
+        mask |= dmask << shift;
         need -= s_dabove;
+        const bool whole = s_fill_exact;
         __syncthreads();
+        hi_bit = shift;
+        if (whole) break;  // lower bits of prefix are zero: values >= prefix are exactly kk
       }
-      thr = prefix;  // values are unique: exactly kk values are >= thr
+      thr = prefix;
     }
     for (int i = tid; i < nb; i += blockDim.x) {
-      const uint64_t v = bnd[i];
+      const uint64_t v = L[i];
       if (v >= thr) {
         const int pos = atomicAdd(&s_fill, 1);
         if (pos < kMaxTopk) pairs[pos] = ~v;
