@@ -5,7 +5,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
-#include "../../include/csa.h"
+#include "csa.h"
 
 namespace csa {
 
