@@ -116,8 +116,11 @@ csa_status csa_compress(const csa_params* p, csa_dtype io, int32_t B, int64_t n_
  *   CSA_F32:  qI f32 [B,T,H_I,d_I],  KI f32 [B,N_cap,d_I]
  *   CSA_BF16: qI bf16,               KI bf16
  *   CSA_FP8_E4M3_ROWSCALE: qI bf16,  KI e4m3 codes [B,N_cap,d_I] + KI_scale f32 [B,N_cap]
- *   CSA_MXFP4 ([P1'] FP4 QK path): qI [B,T,H_I,d_I/2] bytes + qI_scale [B,T,H_I,d_I/32],
- *             KI [B,N_cap,d_I/2] bytes + KI_scale [B,N_cap,d_I/32] (e8m0)
+ *   CSA_MXFP4 ([P1'] FP4 QK path): qI [B,T,H_I,d_I/2] bytes + qI_scale [B,T,H_I,d_I/32]
+ *             (e8m0, in head order), KI [B,N_cap,d_I/2] bytes + KI_scale [B,N_cap,4] e8m0
+ *             stored per block of 128 keys as the tensor cores read it: byte 16*i + 4*j + b
+ *             of a block is block-scale b of key 32*j + i. Requires H_I = 64, d_I = 128,
+ *             N_cap a multiple of 128 and B*T <= 1024.
  * w: f32 [B,T,H_I]. q_pos: int64 [B,T]. Scores are fp32 sums of exact products.
  */
 csa_status csa_index_scores(const csa_params* p, csa_dtype kdt, int32_t B, int32_t T,

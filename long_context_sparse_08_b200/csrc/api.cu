@@ -156,7 +156,11 @@ csa_status check_index_args(const csa_params* p, csa_dtype kdt, int32_t B, int32
   if (kdt == CSA_FP8_E4M3_ROWSCALE && N_cap > 0) REQUIRE_PTR(KI_scale);
   if (kdt == CSA_MXFP4) {
     REQUIRE_PTR(qI_scale);
-    if (N_cap > 0) REQUIRE(KI_scale != nullptr, "KI_scale is required for MXFP4 keys");
+    if (N_cap > 0) REQUIRE_PTR(KI_scale);
+    if (p->n_idx_heads != 64 || p->d_idx != 128)
+      return fail(CSA_ERR_UNSUPPORTED, "MXFP4 keys need 64 indexer heads of dim 128");
+    REQUIRE(N_cap % 128 == 0, "MXFP4 key caches hold whole 128-key scale blocks (N_cap %% 128)");
+    REQUIRE((int64_t)B * T <= 1024, "MXFP4 indexer takes at most 1024 queries per call");
   }
   return CSA_OK;
 }

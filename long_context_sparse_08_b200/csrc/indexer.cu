@@ -2,9 +2,9 @@
 //
 // 【论文解读】DeepSeek-V4, 一(三)1(2) Lightning Indexer 稀疏选择:
 //   I[t,s] = sum_h w[t,h] * ReLU(q^I[t,h] . K^IComp[s]),  for s < floor(t/m).
-// The keys are read in the stored format (fp32, bf16, e4m3 with a row scale, or MXFP4 as
-// in 二(四) FP4 量化感知训练) and decoded exactly in registers; every product is exact in
-// fp32 and the sums are fp32. For e4m3 keys the row scale is applied after the dot
+// The keys are read in the stored format (fp32, bf16, or e4m3 with a row scale) and
+// decoded exactly in registers; every product is exact in fp32 and the sums are fp32.
+// (MXFP4 keys go through the tensor-core kernel of indexer_mxf4.cu.) For e4m3 keys the row scale is applied after the dot
 // product (ReLU(s*x) = s*ReLU(x) for s >= 0), so no product is rounded.
 //
 // One thread per key, 128 keys per CTA, one (request, query) per grid row; the query's
@@ -60,16 +60,6 @@ __device__ __forceinline__ void load_key_chunk(const IndexArgs& a, int b, int64_
         for (int by = 0; by < 4; ++by)
           v[16 * q + 4 * k + by] = e4m3_to_f32((w4[k] >> (8 * by)) & 0xff);
     }
-  } else {  // MXFP4: 16 bytes of e2m1 pairs and one e8m0 scale for these 32 elements
-    const uint4 x = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.KI) +
-                                                    row * (d / 2) + d0 / 2);
-    const float sc = e8m0_to_f32(static_cast<const uint8_t*>(a.KI_scale)[row * (d / 32) +
-                                                                           d0 / 32]);
-    const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-#pragma unroll
-      for (int nb = 0; nb < 8; ++nb) v[8 * k + nb] = e2m1_to_f32((w4[k] >> (4 * nb)) & 0xf) * sc;
   }
 }
 
@@ -90,10 +80,6 @@ __global__ void __launch_bounds__(kKeysPerCta) k_index_scores_cc(IndexArgs a) {
     const size_t off = (size_t)bt * H * d + e;
     if (KDT == CSA_F32) {
       v = static_cast<const float*>(a.qI)[off];
-    } else if (KDT == CSA_MXFP4) {
-      const uint8_t byte = static_cast<const uint8_t*>(a.qI)[off / 2];
-      v = e2m1_to_f32((e & 1) ? (byte >> 4) : (byte & 0xf)) *
-          e8m0_to_f32(static_cast<const uint8_t*>(a.qI_scale)[off / 32]);
     } else {
       v = to_f32(static_cast<const __nv_bfloat16*>(a.qI)[off]);
     }
@@ -150,11 +136,8 @@ cudaError_t launch_index_scores(const IndexArgs& a, cudaStream_t st, bool* hist_
     case CSA_BF16:
       k_index_scores_cc<CSA_BF16><<<grid, kKeysPerCta, smem, st>>>(a);
       break;
-    case CSA_FP8_E4M3_ROWSCALE:
-      k_index_scores_cc<CSA_FP8_E4M3_ROWSCALE><<<grid, kKeysPerCta, smem, st>>>(a);
-      break;
     default:
-      k_index_scores_cc<CSA_MXFP4><<<grid, kKeysPerCta, smem, st>>>(a);
+      k_index_scores_cc<CSA_FP8_E4M3_ROWSCALE><<<grid, kKeysPerCta, smem, st>>>(a);
       break;
   }
   timing_after(st);

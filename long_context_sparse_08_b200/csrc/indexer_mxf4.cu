@@ -3,22 +3,27 @@
 // 【论文解读】DeepSeek-V4, 一(三)1(2): I[t,s] = sum_h w[t,h] * ReLU(q^I[t,h] . K[s]);
 // 二(四) FP4 量化感知训练: the indexer's QK path is cached, loaded and multiplied in FP4.
 //
-// One tile = 128 keys of one query's request: D[128 keys x 64 heads] = K_tile . q^T over
-// d_I = 128, as two tcgen05 kind::mxf4 block-scaled MMAs (K = 64 each, one e8m0 scale per
-// 32 elements of A and of B, products exact, fp32 accumulation in TMEM). TMEM lane = key,
-// column = head, so each epilogue thread owns one key and reduces its 64 head dots with
-// w * ReLU(.) without any shuffle.
+// A unit is 256 keys of one query's request: two M-tiles of 128 keys, each
+// D[128 keys x 64 heads] = K_tile . q^T over d_I = 128 as two tcgen05 kind::mxf4
+// block-scaled MMAs (K = 64 each, one e8m0 scale per 32 elements of A and of B, exact
+// products, fp32 accumulation in TMEM). TMEM lane = key, column = head, so an epilogue
+// thread owns one key and reduces its 64 head dots with w * ReLU(.) without shuffles.
 //
-// Persistent kernel, one CTA per SM, 6 warps:
-//   warp 0  TMA producer: key tile (128 x 64 B, 64B-swizzled), its 128 scale words, the
-//           query's 64 x 64 B heads and their scale words, into an 8-stage ring;
-//   warp 1  MMA issuer: rearranges the scale words into the 32x128b layout tcgen05.cp
-//           copies into TMEM (row 32*j + i of the tile -> lane i, column j; the 4 bytes of
-//           a column are the row's 4 block scales), then issues the copy and the 2 MMAs;
-//   warps 2-5 epilogue: TMEM -> registers (32x32b.x64), w * ReLU head sum, fp32 store.
-// Four accumulator slots in TMEM let the MMAs of tiles j+1..j+3 run while the epilogue
-// reduces tile j. Work (query, tile) pairs are split
-// evenly over the CTAs; ragged per-query visibility is handled by masking the stores.
+// Key scales are stored in 128-key blocks laid out as tcgen05.cp's 32x128b source: byte
+// 16*i + 4*j + b of a block is block-scale b of key 32*j + i. One TMA copy of a unit's
+// 1 KB of scales therefore lands ready for tcgen05.cp (no rearrangement in the kernel).
+//
+// Persistent kernel, one CTA per SM, 10 warps:
+//   warp 0     TMA producer: per unit one 16 KB key box (64B-swizzled) and one 1 KB scale
+//              box; per query the 64 x 64 B heads and their scale words;
+//   warp 1     MMA issuer: per query the query scales into TMEM (rearranged once), per
+//              M-tile the key scales into TMEM (tcgen05.cp) and two MMAs;
+//   warps 2-9  two epilogue warpgroups; group g reduces M-tile g of every unit:
+//              TMEM -> registers, w * ReLU head sum, fp32 score store, and a 4096-bin
+//              histogram of the scores' top 12 key bits for the top-k selector.
+// Four accumulator slots in TMEM let the MMAs of the next unit run while both groups
+// reduce the current one. Units are split evenly over the CTAs; ragged per-query
+// visibility is handled by masking the stores.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -33,32 +38,35 @@ namespace {
 
 using namespace tc;
 
-constexpr int kStages = 8;
-constexpr int kTileKeys = 128;     // M
+constexpr int kStages = 6;
+constexpr int kTileKeys = 128;     // M of one MMA
+constexpr int kUnitKeys = 256;     // keys per pipeline stage (two M-tiles)
 constexpr int kHeads = 64;         // N (indexer heads)
 constexpr int kRowBytes = 64;      // 128 e2m1 per row
 constexpr int kMaxQueries = 1024;  // (request, query) pairs per launch
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kBins = 4096;
 
-constexpr int kOffA = 0;                                 // 8192 B, 1024-aligned
-constexpr int kOffQ = kOffA + kTileKeys * kRowBytes;     // 4096 B
-constexpr int kOffSA = kOffQ + kHeads * kRowBytes;       // 512 B  key scale words
-constexpr int kOffSQ = kOffSA + kTileKeys * 4;           // 256 B  query scale words
-constexpr int kOffSFA = kOffSQ + kHeads * 4;             // 512 B  rearranged for tcgen05.cp
-constexpr int kOffSFB = kOffSFA + 512;                   // 512 B
-constexpr int kStageBytes = ((kOffSFB + 512 + 1023) / 1024) * 1024;
-constexpr uint32_t kStageTx = kTileKeys * kRowBytes + kHeads * kRowBytes + kTileKeys * 4 +
-                              kHeads * 4;
+constexpr int kOffA = 0;                                // 16 KB, 1024-aligned
+constexpr int kOffSF = kOffA + kUnitKeys * kRowBytes;   // 1 KB key scales (cp layout)
+constexpr int kStageBytes = ((kOffSF + 1024 + 1023) / 1024) * 1024;
+constexpr uint32_t kStageTx = kUnitKeys * kRowBytes + kUnitKeys * 4;
+// per-query buffers (two slots)
+constexpr int kOffQ = 0;                                // 4 KB q heads (64B-swizzled)
+constexpr int kOffQS = kOffQ + kHeads * kRowBytes;      // 256 B query scale words
+constexpr int kOffQSF = kOffQS + kHeads * 4;            // 512 B rearranged for tcgen05.cp
+constexpr int kQBytes = ((kOffQSF + 512 + 1023) / 1024) * 1024;
+constexpr uint32_t kQTx = kHeads * kRowBytes + kHeads * 4;
 
 // TMEM columns
-constexpr int kAcc = 4;  // accumulator slots in TMEM
+constexpr int kAcc = 4;
 constexpr uint32_t kTmemCols = 512;
-__device__ __forceinline__ uint32_t acc_col(int acc) { return 64u * acc; }         // 0..192
-__device__ __forceinline__ uint32_t sfa_col(int acc) { return 256u + 32u * acc; }  // 256..352
-__device__ __forceinline__ uint32_t sfb_col(int acc) { return 272u + 32u * acc; }  // 272..368
+__device__ __forceinline__ uint32_t acc_col(int s) { return 64u * s; }          // 0..192
+__device__ __forceinline__ uint32_t sfa_col(int s) { return 256u + 8u * s; }    // 256..280
+__device__ __forceinline__ uint32_t sfb_col(int qs) { return 320u + 8u * qs; }  // 320, 328
 
-// device error codes of this kernel
-enum { kErrFull = 101, kErrEmpty = 102, kErrTmemFull = 103, kErrTmemEmpty = 104 };
+enum { kErrFull = 101, kErrEmpty = 102, kErrTmemFull = 103, kErrTmemEmpty = 104,
+       kErrQFull = 105, kErrQEmpty = 106 };
 
 struct Mxf4Params {
   int Q, T, m;
@@ -69,30 +77,13 @@ struct Mxf4Params {
   int* hist;  // optional [Q][4096] histogram of the scores' top 12 key bits
 };
 
-constexpr int kBins = 4096;
-
 struct Smem {
-  uint64_t full[kStages], empty[kStages], tfull[kAcc], tempty[kAcc], done;
+  uint64_t full[kStages], empty[kStages], tfull[kAcc], tempty[kAcc], qfull[2], qempty[2], done;
   uint32_t tmem_slot;
   int prefix[kMaxQueries + 1];
   int nvis[kMaxQueries];
   int hist[kBins];
 };
-
-// named barrier of the 4 epilogue warps; returns the AND of `ok` over them
-__device__ __forceinline__ bool epi_all_ok(bool ok) {
-  uint32_t res;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.and.pred p, 2, 128, q;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(res)
-      : "r"((uint32_t)ok)
-      : "memory");
-  return res != 0;
-}
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 
 __device__ __forceinline__ int find_query(const int* prefix, int Q, int u) {
   int lo = 0, hi = Q;  // largest q with prefix[q] <= u
@@ -103,6 +94,21 @@ __device__ __forceinline__ int find_query(const int* prefix, int Q, int u) {
   return lo;
 }
 
+// named barrier 2 over the 8 epilogue warps; returns the AND of `ok` over them
+__device__ __forceinline__ bool epi_all_ok(bool ok) {
+  uint32_t res;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 2, 256, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(res)
+      : "r"((uint32_t)ok)
+      : "memory");
+  return res != 0;
+}
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 2, 256;" ::: "memory"); }
+
 __global__ void __launch_bounds__(kThreads, 1)
     k_index_mxf4_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_ks,
                     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qs,
@@ -110,10 +116,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  Smem& S = *reinterpret_cast<Smem*>(base + kStages * kStageBytes);
+  uint8_t* qbase = base + kStages * kStageBytes;
+  Smem& S = *reinterpret_cast<Smem*>(qbase + 2 * kQBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- per-query visible counts and tile prefix (warp 0, warp-level scan) ----
+  // ---- per-query visible counts and unit prefix (warp 0, warp-level scan) ----
   if (warp == 0) {
     int run = 0;
     for (int q0 = 0; q0 < p.Q; q0 += 32) {
@@ -125,19 +132,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         nv = (int)v;
         S.nvis[q] = nv;
       }
-      const int tiles = (nv + kTileKeys - 1) / kTileKeys;
-      int incl = tiles;
+      const int units = (nv + kUnitKeys - 1) / kUnitKeys;
+      int incl = units;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int x = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += x;
       }
-      if (q < p.Q) S.prefix[q] = run + incl - tiles;
+      if (q < p.Q) S.prefix[q] = run + incl - units;
       run += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (lane == 0) {
       S.prefix[p.Q] = run;
-      mbar_init(&S.done, 1);
       for (int i = 0; i < kStages; ++i) {
         mbar_init(&S.full[i], 1);
         mbar_init(&S.empty[i], 1);
@@ -146,6 +152,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&S.tfull[i], 1);
         mbar_init(&S.tempty[i], 4);
       }
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&S.qfull[i], 1);
+        mbar_init(&S.qempty[i], 1);
+      }
+      mbar_init(&S.done, 1);
       fence_barrier_init();
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_ks);
@@ -154,6 +165,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     tmem_alloc(&S.tmem_slot, kTmemCols);
+  } else {
+    for (int i = threadIdx.x - 64; i < kBins; i += 256) S.hist[i] = 0;
   }
   tc_fence_before();
   __syncthreads();
@@ -167,67 +180,100 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------ TMA producer ------------------------------
     if (lane == 0 && u0 < u1) {
       int q = find_query(S.prefix, p.Q, u0);
-      int k = 0;
-      for (int u = u0; u < u1; ++u, ++k) {
+      int cur_q = -1, nq = -1;  // nq: index of the current query within this CTA
+      int k = 0, issued_q = 0;
+      bool ok = true;
+      for (int u = u0; u < u1 && ok; ++u, ++k) {
         while (u >= S.prefix[q + 1]) ++q;
-        const int tile = u - S.prefix[q];
+        if (q != cur_q) {  // this query's heads and their scale words into the next slot
+          ++nq;
+          cur_q = q;
+          const int qs = nq & 1;
+          ok = mbar_wait(&S.qempty[qs], ((nq >> 1) & 1) ^ 1, kErrQEmpty);
+          if (!ok) break;
+          uint8_t* qb = qbase + qs * kQBytes;
+          mbar_arrive_expect_tx(&S.qfull[qs], kQTx);
+          tma_load_2d(qb + kOffQ, &tm_q, 0, q * kHeads, &S.qfull[qs]);
+          tma_load_1d(qb + kOffQS, &tm_qs, q * kHeads, &S.qfull[qs]);
+          issued_q = nq + 1;
+        }
+        const int unit = u - S.prefix[q];
         const int st = k % kStages;
         const uint32_t round = (uint32_t)(k / kStages);
-        if (!mbar_wait(&S.empty[st], (round & 1) ^ 1, kErrEmpty)) break;
+        ok = mbar_wait(&S.empty[st], (round & 1) ^ 1, kErrEmpty);
+        if (!ok) break;
         uint8_t* sb = base + st * kStageBytes;
         const int b = q / p.T;
-        const int32_t row0 = (int32_t)(b * p.n_cap + (int64_t)tile * kTileKeys);
+        const int32_t row0 = (int32_t)(b * p.n_cap + (int64_t)unit * kUnitKeys);
         mbar_arrive_expect_tx(&S.full[st], kStageTx);
         tma_load_2d(sb + kOffA, &tm_k, 0, row0, &S.full[st]);
-        tma_load_1d(sb + kOffSA, &tm_ks, row0, &S.full[st]);
-        tma_load_2d(sb + kOffQ, &tm_q, 0, q * kHeads, &S.full[st]);
-        tma_load_1d(sb + kOffSQ, &tm_qs, q * kHeads, &S.full[st]);
+        tma_load_1d(sb + kOffSF, &tm_ks, row0, &S.full[st]);
       }
-      // drain: do not leave the CTA while copies into its shared memory are in flight
-      const int issued = k;
-      for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+      // drain: no copy into this CTA's shared memory may still be in flight at exit
+      for (int j = (k > kStages ? k - kStages : 0); j < k; ++j)
         mbar_wait(&S.full[j % kStages], (uint32_t)((j / kStages) & 1), kErrFull);
+      for (int j = (issued_q > 2 ? issued_q - 2 : 0); j < issued_q; ++j)
+        mbar_wait(&S.qfull[j & 1], (uint32_t)((j >> 1) & 1), kErrQFull);
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer ------------------------------
     const uint32_t id0 = idesc_mxf4(kTileKeys, kHeads, 0, 0);
     const uint32_t id1 = idesc_mxf4(kTileKeys, kHeads, 2, 2);
+    int q = u0 < u1 ? find_query(S.prefix, p.Q, u0) : 0;
+    int cur_q = -1, nq = -1;
     int k = 0;
     bool ok = true;
     for (int u = u0; u < u1 && ok; ++u, ++k) {
+      while (u >= S.prefix[q + 1]) ++q;
+      if (q != cur_q) {
+        if (cur_q >= 0 && lane == 0) mma_commit(&S.qempty[nq & 1]);  // old slot free when done
+        ++nq;
+        cur_q = q;
+        const int qs = nq & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(&S.qfull[qs], (nq >> 1) & 1, kErrQFull));
+        if (!ok) break;
+        // query scale words -> tcgen05.cp layout (16-byte row i: words of heads i, 32+i)
+        uint8_t* qb = qbase + qs * kQBytes;
+        const uint32_t* sq = reinterpret_cast<const uint32_t*>(qb + kOffQS);
+        *reinterpret_cast<uint4*>(qb + kOffQSF + 16 * lane) =
+            make_uint4(sq[lane], sq[32 + lane], 0u, 0u);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tc_fence_after();
+          tmem_cp_32x128b_warpx4(tmem + sfb_col(qs),
+                                 smem_desc(smem_u32(qb + kOffQSF), 0, 128, kLayoutNone));
+        }
+      }
+      const int qs = nq & 1;
       const int st = k % kStages;
       const uint32_t round = (uint32_t)(k / kStages);
-      const int acc = k % kAcc;
-      const uint32_t around = (uint32_t)(k / kAcc);
-      ok = mbar_wait(&S.full[st], round & 1, kErrFull);
+      ok = __all_sync(0xffffffffu, mbar_wait(&S.full[st], round & 1, kErrFull));
       if (!ok) break;
       uint8_t* sb = base + st * kStageBytes;
-      // scale words -> tcgen05.cp layout: 16-byte row i = words of tile rows i, 32+i, 64+i, 96+i
-      const uint32_t* sa = reinterpret_cast<const uint32_t*>(sb + kOffSA);
-      const uint32_t* sq = reinterpret_cast<const uint32_t*>(sb + kOffSQ);
-      *reinterpret_cast<uint4*>(sb + kOffSFA + 16 * lane) =
-          make_uint4(sa[lane], sa[32 + lane], sa[64 + lane], sa[96 + lane]);
-      *reinterpret_cast<uint4*>(sb + kOffSFB + 16 * lane) =
-          make_uint4(sq[lane], sq[32 + lane], 0u, 0u);
-      fence_proxy_async_smem();
-      __syncwarp();
       int good = 1;
       if (lane == 0) {
-        good = mbar_wait(&S.tempty[acc], (around & 1) ^ 1, kErrTmemEmpty);
-        if (good) {
+        const uint64_t b0 = smem_desc(smem_u32(qbase + qs * kQBytes + kOffQ), 16,
+                                      8 * kRowBytes, kLayoutSw64);
+        const uint32_t sfb = tmem + sfb_col(qs);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const int slot = 2 * (k & 1) + t;
+          good = mbar_wait(&S.tempty[slot], (((uint32_t)k >> 1) & 1) ^ 1, kErrTmemEmpty);
+          if (!good) break;
           tc_fence_after();
-          const uint32_t sfa = tmem + sfa_col(acc), sfb = tmem + sfb_col(acc);
-          tmem_cp_32x128b_warpx4(sfa, smem_desc(smem_u32(sb + kOffSFA), 0, 128, kLayoutNone));
-          tmem_cp_32x128b_warpx4(sfb, smem_desc(smem_u32(sb + kOffSFB), 0, 128, kLayoutNone));
-          const uint64_t a0 = smem_desc(smem_u32(sb + kOffA), 16, 8 * kRowBytes, kLayoutSw64);
-          const uint64_t b0 = smem_desc(smem_u32(sb + kOffQ), 16, 8 * kRowBytes, kLayoutSw64);
-          const uint32_t d = tmem + acc_col(acc);
+          const uint32_t sfa = tmem + sfa_col(slot);
+          tmem_cp_32x128b_warpx4(
+              sfa, smem_desc(smem_u32(sb + kOffSF + 512 * t), 0, 128, kLayoutNone));
+          const uint64_t a0 = smem_desc(smem_u32(sb + kOffA + t * kTileKeys * kRowBytes), 16,
+                                        8 * kRowBytes, kLayoutSw64);
+          const uint32_t d = tmem + acc_col(slot);
           mma_mxf4(d, a0, b0, id0, sfa, sfb, 0u);
           // second K half: +32 bytes inside the swizzled rows, scale bytes 2..3
           mma_mxf4(d, a0 + 2, b0 + 2, id1, sfa | (2u << 30), sfb | (2u << 30), 1u);
-          mma_commit(&S.empty[st]);
-          mma_commit(&S.tfull[acc]);
+          mma_commit(&S.tfull[slot]);
         }
+        if (good) mma_commit(&S.empty[st]);
       }
       ok = __shfl_sync(0xffffffffu, good, 0) != 0;
     }
@@ -239,17 +285,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------ epilogue ------------------------------
-    const int quad = warp & 3;  // TMEM lane quadrant this warp may access
-    const int etid = threadIdx.x - 64;
+    const int grp = (warp - 2) >> 2;  // M-tile this warpgroup reduces
+    const int quad = warp & 3;        // TMEM lane quadrant this warp may access
     const bool hist = p.hist != nullptr;
-    if (hist) {
-      for (int i = etid; i < kBins; i += 128) S.hist[i] = 0;
-      epi_bar();
-    }
     int hq = -1;
-    auto flush = [&](int qq) {  // smem histogram of query qq -> global, then clear
+    auto flush = [&](int qq) {  // shared histogram of query qq -> global, then clear
       epi_bar();
-      for (int i = etid; i < kBins; i += 128) {
+      for (int i = threadIdx.x - 64; i < kBins; i += 256) {
         const int v = S.hist[i];
         if (v) {
           atomicAdd(&p.hist[(size_t)qq * kBins + i], v);
@@ -264,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int k = 0;
     for (int u = u0; u < u1; ++u, ++k) {
       while (u >= S.prefix[q + 1]) ++q;
-      const int tile = u - S.prefix[q];
+      const int unit = u - S.prefix[q];
       if (q != cur_q) {
 #pragma unroll
         for (int h = 0; h < kHeads; ++h) wr[h] = p.w[(size_t)q * kHeads + h];
@@ -274,20 +316,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (hq >= 0) flush(hq);
         hq = q;
       }
-      const int acc = k % kAcc;
-      const uint32_t around = (uint32_t)(k / kAcc);
-      if (!epi_all_ok(mbar_wait(&S.tfull[acc], around & 1, kErrTmemFull))) break;
+      const int slot = 2 * (k & 1) + grp;
+      if (!epi_all_ok(mbar_wait(&S.tfull[slot], ((uint32_t)k >> 1) & 1, kErrTmemFull))) break;
       tc_fence_after();
       uint32_t v[kHeads];
-      tmem_ld_32x32b_x64(tmem + ((uint32_t)(32 * quad) << 16) + acc_col(acc), v);
+      tmem_ld_32x32b_x64(tmem + ((uint32_t)(32 * quad) << 16) + acc_col(slot), v);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&S.tempty[acc]);
-      float sc = 0.f;
+      if (lane == 0) mbar_arrive(&S.tempty[slot]);
+      float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int h = 0; h < kHeads; ++h) sc = fmaf(wr[h], fmaxf(__uint_as_float(v[h]), 0.f), sc);
-      const int s = tile * kTileKeys + 32 * quad + lane;
+      for (int h = 0; h < kHeads; ++h)
+        part[h & 3] = fmaf(wr[h], fmaxf(__uint_as_float(v[h]), 0.f), part[h & 3]);
+      const float sc = (part[0] + part[1]) + (part[2] + part[3]);
+      const int s = unit * kUnitKeys + grp * kTileKeys + 32 * quad + lane;
       if (s < S.nvis[q]) {
         p.scores[(size_t)q * p.n_cap + s] = sc;
         if (hist) atomicAdd(&S.hist[float_key(sc) >> 20], 1);
@@ -356,22 +399,22 @@ int num_sms() {
 }  // namespace
 
 bool index_mxf4_tc_supported(const IndexArgs& a) {
-  return a.kdt == CSA_MXFP4 && a.n_idx_heads == kHeads && a.d_idx == 128 && a.n_cap % 32 == 0 &&
+  return a.kdt == CSA_MXFP4 && a.n_idx_heads == kHeads && a.d_idx == 128 && a.n_cap % 128 == 0 &&
          (int64_t)a.B * a.T <= kMaxQueries && (int64_t)a.B * a.n_cap < (1ll << 31);
 }
 
 cudaError_t launch_index_mxf4_tc(const IndexArgs& a, cudaStream_t st) {
   const int Q = a.B * a.T;
   CUtensorMap mk, mks, mq, mqs;
-  if (!make_map_2d(&mk, a.KI, (uint64_t)a.B * a.n_cap, kTileKeys) ||
-      !make_map_1d_words(&mks, a.KI_scale, (uint64_t)a.B * a.n_cap, kTileKeys) ||
+  if (!make_map_2d(&mk, a.KI, (uint64_t)a.B * a.n_cap, kUnitKeys) ||
+      !make_map_1d_words(&mks, a.KI_scale, (uint64_t)a.B * a.n_cap, kUnitKeys) ||
       !make_map_2d(&mq, a.qI, (uint64_t)Q * kHeads, kHeads) ||
       !make_map_1d_words(&mqs, a.qI_scale, (uint64_t)Q * kHeads, kHeads))
     return cudaErrorInvalidValue;
   Mxf4Params p{Q, a.T, a.m, a.n_cap, a.q_pos, a.w, a.scores, a.hist};
-  const int64_t units_max = (int64_t)Q * ((a.n_cap + kTileKeys - 1) / kTileKeys);
+  const int64_t units_max = (int64_t)Q * ((a.n_cap + kUnitKeys - 1) / kUnitKeys);
   const int grid = (int)(units_max < num_sms() ? (units_max > 0 ? units_max : 1) : num_sms());
-  const size_t smem = 1024 + (size_t)kStages * kStageBytes + sizeof(Smem);
+  const size_t smem = 1024 + (size_t)kStages * kStageBytes + 2 * kQBytes + sizeof(Smem);
   cudaError_t e = cudaFuncSetAttribute(k_index_mxf4_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;

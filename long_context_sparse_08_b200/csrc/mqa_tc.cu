@@ -52,7 +52,7 @@ struct Smem {
   uint64_t kv_full, s_full, p_full, kv_free, done;
   uint32_t tmem_slot;
   int any_rescale;
-  float red[4][kHg];
+  float red[4][kHg], red2[4][kHg];
   float m_used[kHg], l_sum[kHg], alpha[kHg], fin[kHg];
   float cs[256], sn[256];  // RoPE table for pairs of the last r dims
   const __nv_bfloat16* src[kRows];  // source rows of the current chunk (nullptr: masked)
@@ -128,75 +128,67 @@ __device__ __forceinline__ const __nv_bfloat16* row_src(const MqaArgs& a, int bt
   return nullptr;
 }
 
-// Reduce-scatter of 64 per-thread values across the warp: on return lane l holds the
-// reduction over the warp's 32 threads of heads 2l and 2l+1 in out[0], out[1].
+// 32 lanes x 16 columns of 32-bit: thread i of the warp gets lane (quadrant*32 + i).
+__device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32"
+      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0],"
+      " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Reduce 16 per-thread values over the warp's 32 threads: on return lanes 2j and 2j+1 both
+// hold the reduction of value j (4 halving exchanges, then one pairwise exchange).
 template <bool kMax>
-__device__ __forceinline__ void warp_reduce_scatter64(const float (&v)[64], float (&out)[2]) {
+__device__ __forceinline__ float warp_reduce16(const float (&v)[16]) {
   const int lane = threadIdx.x & 31;
-  float a32[32], a16[16], a8[8], a4[4];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const bool hi = lane & 16;
-    const float send = hi ? v[i] : v[32 + i];
-    const float keep = hi ? v[32 + i] : v[i];
-    const float got = __shfl_xor_sync(0xffffffffu, send, 16);
-    a32[i] = kMax ? fmaxf(keep, got) : keep + got;
-  }
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const bool hi = lane & 8;
-    const float send = hi ? a32[i] : a32[16 + i];
-    const float keep = hi ? a32[16 + i] : a32[i];
-    const float got = __shfl_xor_sync(0xffffffffu, send, 8);
-    a16[i] = kMax ? fmaxf(keep, got) : keep + got;
-  }
+  float a8[8], a4[4], a2[2];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const bool hi = lane & 4;
-    const float send = hi ? a16[i] : a16[8 + i];
-    const float keep = hi ? a16[8 + i] : a16[i];
-    const float got = __shfl_xor_sync(0xffffffffu, send, 4);
+    const bool hi = lane & 16;
+    const float got = __shfl_xor_sync(0xffffffffu, hi ? v[i] : v[8 + i], 16);
+    const float keep = hi ? v[8 + i] : v[i];
     a8[i] = kMax ? fmaxf(keep, got) : keep + got;
   }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const bool hi = lane & 2;
-    const float send = hi ? a8[i] : a8[4 + i];
+    const bool hi = lane & 8;
+    const float got = __shfl_xor_sync(0xffffffffu, hi ? a8[i] : a8[4 + i], 8);
     const float keep = hi ? a8[4 + i] : a8[i];
-    const float got = __shfl_xor_sync(0xffffffffu, send, 2);
     a4[i] = kMax ? fmaxf(keep, got) : keep + got;
   }
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
-    const bool hi = lane & 1;
-    const float send = hi ? a4[i] : a4[2 + i];
+    const bool hi = lane & 4;
+    const float got = __shfl_xor_sync(0xffffffffu, hi ? a4[i] : a4[2 + i], 4);
     const float keep = hi ? a4[2 + i] : a4[i];
-    const float got = __shfl_xor_sync(0xffffffffu, send, 1);
-    out[i] = kMax ? fmaxf(keep, got) : keep + got;
+    a2[i] = kMax ? fmaxf(keep, got) : keep + got;
   }
+  const bool hi = lane & 2;
+  const float got = __shfl_xor_sync(0xffffffffu, hi ? a2[0] : a2[1], 2);
+  float r = hi ? a2[1] : a2[0];
+  r = kMax ? fmaxf(r, got) : r + got;
+  const float other = __shfl_xor_sync(0xffffffffu, r, 1);
+  return kMax ? fmaxf(r, other) : r + other;
 }
-
-__device__ __forceinline__ void tmem_st_32x32b_x64(uint32_t taddr, const uint32_t (&r)[64]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0],"
-      " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16,"
-      " %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32,"
-      " %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48,"
-      " %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64};" ::"r"(
-          taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
-      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
-      "r"(r[29]), "r"(r[30]), "r"(r[31]), "r"(r[32]), "r"(r[33]), "r"(r[34]), "r"(r[35]),
-      "r"(r[36]), "r"(r[37]), "r"(r[38]), "r"(r[39]), "r"(r[40]), "r"(r[41]), "r"(r[42]),
-      "r"(r[43]), "r"(r[44]), "r"(r[45]), "r"(r[46]), "r"(r[47]), "r"(r[48]), "r"(r[49]),
-      "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]), "r"(r[56]),
-      "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_st_wait() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+// value index held by lane after warp_reduce16: j = 8*b4 + 4*b3 + 2*b2 + b1 (lane bits)
+__device__ __forceinline__ int reduce16_index(int lane) {
+  return ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
@@ -241,59 +233,53 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
   const uint32_t tmem = S.tmem_slot;
 
   if (warp < 4) {
-    {
-      const int h = tid >> 1, half = tid & 1;
+    // ---- q_hat = RoPE_t(RMSNorm(q)) in bf16, one warp per head (lane = 16 dims) ----
+    uint8_t* qs = base + kOffQ;
+#pragma unroll 1
+    for (int h = warp; h < kHg; h += 4) {
       const __nv_bfloat16* qrow =
-          static_cast<const __nv_bfloat16*>(a.q) + ((size_t)bt * a.H + h0 + h) * kC + 256 * half;
-      const __nv_bfloat16* gw =
-          a.q_rms_w ? static_cast<const __nv_bfloat16*>(a.q_rms_w) + 256 * half : nullptr;
-      uint4 raw[32];
+          static_cast<const __nv_bfloat16*>(a.q) + ((size_t)bt * a.H + h0 + h) * kC;
+      float x[16];
       float ss = 0.f;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        raw[i] = reinterpret_cast<const uint4*>(qrow)[i];
-        const uint32_t w4[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+      for (int half = 0; half < 2; ++half) {
+        const uint4 raw = reinterpret_cast<const uint4*>(qrow)[lane + 32 * half];
+        const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const float x0 = __uint_as_float(w4[k] << 16), x1 = __uint_as_float(w4[k] & 0xffff0000u);
-          ss = fmaf(x0, x0, fmaf(x1, x1, ss));
+          x[8 * half + 2 * k] = __uint_as_float(w4[k] << 16);
+          x[8 * half + 2 * k + 1] = __uint_as_float(w4[k] & 0xffff0000u);
         }
       }
-      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) ss = fmaf(x[k], x[k], ss);
+      ss = warp_sum(ss);
       const float rstd = rsqrtf(ss / (float)kC + a.eps);
-      uint8_t* qs = base + kOffQ;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int d0 = 256 * half + 8 * i;
-        const uint32_t w4[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
-        float x[8];
+      for (int half = 0; half < 2; ++half) {
+        const int d0 = 8 * (lane + 32 * half);
+        float y[8];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          x[2 * k] = __uint_as_float(w4[k] << 16) * rstd;
-          x[2 * k + 1] = __uint_as_float(w4[k] & 0xffff0000u) * rstd;
-        }
-        if (gw) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) x[k] *= __bfloat162float(gw[8 * i + k]);
+        for (int k = 0; k < 8; ++k) {
+          y[k] = x[8 * half + k] * rstd;
+          if (a.q_rms_w)
+            y[k] *= __bfloat162float(static_cast<const __nv_bfloat16*>(a.q_rms_w)[d0 + k]);
         }
         if (d0 >= r0) {
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const int p = (d0 + 2 * k - r0) >> 1;
-            const float c = S.cs[p], s = S.sn[p], u = x[2 * k], v = x[2 * k + 1];
-            x[2 * k] = u * c - v * s;
-            x[2 * k + 1] = u * s + v * c;
+            const float c = S.cs[p], sn = S.sn[p], u = y[2 * k], v = y[2 * k + 1];
+            y[2 * k] = u * c - v * sn;
+            y[2 * k + 1] = u * sn + v * c;
           }
         }
         uint4 o;
-        o.x = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[0])) |
-              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[1])) << 16);
-        o.y = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[2])) |
-              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[3])) << 16);
-        o.z = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[4])) |
-              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[5])) << 16);
-        o.w = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[6])) |
-              ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x[7])) << 16);
+        uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          ow[k] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * k])) |
+                  ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * k + 1])) << 16);
         const int atom = d0 >> 6, chunk = (d0 & 63) >> 3;
         *reinterpret_cast<uint4*>(qs + atom * (kHg * 128) + sw128(h, chunk)) = o;
       }
@@ -301,6 +287,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
 
     bool ok = true;
     const uint32_t kv_base = smem_u32(base + kOffKV);
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+#pragma unroll 1
     for (int j = c0; j < c1 && ok; ++j) {
       const uint32_t it = (uint32_t)(j - c0);
       if (j > c0) ok = all_ok_softmax(mbar_wait(&S.kv_free, (it - 1) & 1, kErrKvFree));
@@ -310,6 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
       const __nv_bfloat16* my_src = row_src(a, bt, b, rl, (int64_t)j * kRows + tid);
       S.src[tid] = my_src;
       bar_softmax();
+#pragma unroll 1
       for (int rr = warp; rr < kRows; rr += 4) {
         const __nv_bfloat16* src = S.src[rr];
 #pragma unroll
@@ -325,22 +314,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
       fence_proxy_async_smem();
       mbar_arrive(&S.kv_full);
 
-      // ---- softmax of S^T (thread = row) ----
+      // ---- softmax of S^T (thread = row), heads in groups of 16 ----
       const int row = tid;
       const bool valid = my_src != nullptr;
       ok = all_ok_softmax(mbar_wait(&S.s_full, it & 1, kErrSFull));
       if (!ok) break;
       tc_fence_after();
-      uint32_t v[64];
-      tmem_ld_32x32b_x64(tmem + ((uint32_t)(32 * warp) << 16) + kColS, v);
-      tmem_ld_wait();
-      float s[64];
+#pragma unroll 1
+      for (int g16 = 0; g16 < 4; ++g16) {  // per-head chunk max
+        uint32_t v[16];
+        tmem_ld_x16(lane_base + kColS + 16 * g16, v);
+        tmem_ld_wait();
+        float sv[16];
 #pragma unroll
-      for (int h = 0; h < 64; ++h) s[h] = valid ? __uint_as_float(v[h]) * a.scale : -INFINITY;
-      float red2[2];
-      warp_reduce_scatter64<true>(s, red2);
-      S.red[warp][2 * lane] = red2[0];
-      S.red[warp][2 * lane + 1] = red2[1];
+        for (int h = 0; h < 16; ++h) sv[h] = valid ? __uint_as_float(v[h]) * a.scale : -INFINITY;
+        const float m = warp_reduce16<true>(sv);
+        if ((lane & 1) == 0) S.red[warp][16 * g16 + reduce16_index(lane)] = m;
+      }
       bar_softmax();
       if (tid < kHg) {
         const float cm = fmaxf(fmaxf(S.red[0][tid], S.red[1][tid]),
@@ -360,44 +350,52 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
       bar_softmax();
       if (S.any_rescale) {  // rare: scale O^T columns by alpha (previous O^T MMAs are done)
 #pragma unroll 1
-        for (int sl = 0; sl < 4; ++sl) {
-          uint32_t o[64];
-          const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16) + kColO + 64 * sl;
-          tmem_ld_32x32b_x64(ta, o);
+        for (int cgrp = 0; cgrp < 16; ++cgrp) {  // 4 slices x 4 groups of 16 heads
+          uint32_t o[16];
+          const uint32_t ta = lane_base + kColO + 16 * cgrp;
+          tmem_ld_x16(ta, o);
           tmem_ld_wait();
+          const int hb = 16 * (cgrp & 3);
 #pragma unroll
-          for (int h = 0; h < 64; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * S.alpha[h]);
-          tmem_st_32x32b_x64(ta, o);
+          for (int h = 0; h < 16; ++h)
+            o[h] = __float_as_uint(__uint_as_float(o[h]) * S.alpha[hb + h]);
+          tmem_st_x16(ta, o);
         }
         tmem_st_wait();
       }
-      // P^T row (bf16) into the swizzled B-operand tile, and per-head row sums
-      float pr[64];
+      // P^T row (bf16, swizzled B-operand tile) and per-head row sums
       uint8_t* pt = base + kOffP;
+#pragma unroll 1
+      for (int g16 = 0; g16 < 4; ++g16) {
+        uint32_t v[16];
+        tmem_ld_x16(lane_base + kColS + 16 * g16, v);
+        tmem_ld_wait();
+        float pr[16];
+        uint32_t pk[8];
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int h = 8 * c8 + 2 * k;
-          const float p0 = s[h] == -INFINITY ? 0.f : __expf(s[h] - S.m_used[h]);
-          const float p1 = s[h + 1] == -INFINITY ? 0.f : __expf(s[h + 1] - S.m_used[h + 1]);
+        for (int k = 0; k < 8; ++k) {
+          const int h = 16 * g16 + 2 * k;
+          const float s0 = __uint_as_float(v[2 * k]) * a.scale;
+          const float s1 = __uint_as_float(v[2 * k + 1]) * a.scale;
+          const float p0 = valid ? __expf(s0 - S.m_used[h]) : 0.f;
+          const float p1 = valid ? __expf(s1 - S.m_used[h + 1]) : 0.f;
           const __nv_bfloat16 b0 = __float2bfloat16_rn(p0), b1 = __float2bfloat16_rn(p1);
-          pr[h] = __bfloat162float(b0);  // sum what the MMA multiplies
-          pr[h + 1] = __bfloat162float(b1);
+          pr[2 * k] = __bfloat162float(b0);  // sum what the MMA multiplies
+          pr[2 * k + 1] = __bfloat162float(b1);
           pk[k] = (uint32_t)__bfloat16_as_ushort(b0) | ((uint32_t)__bfloat16_as_ushort(b1) << 16);
         }
-        *reinterpret_cast<uint4*>(pt + sw128(row, c8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(pt + sw128(row, 2 * g16)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(pt + sw128(row, 2 * g16 + 1)) =
+            make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        const float l = warp_reduce16<false>(pr);
+        if ((lane & 1) == 0) S.red2[warp][16 * g16 + reduce16_index(lane)] = l;
       }
-      warp_reduce_scatter64<false>(pr, red2);
-      bar_softmax();  // everyone has read S.red of the max pass
-      S.red[warp][2 * lane] = red2[0];
-      S.red[warp][2 * lane + 1] = red2[1];
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&S.p_full);
       bar_softmax();
-      if (tid < kHg) S.l_sum[tid] += (S.red[0][tid] + S.red[1][tid]) + (S.red[2][tid] + S.red[3][tid]);
+      if (tid < kHg)
+        S.l_sum[tid] += (S.red2[0][tid] + S.red2[1][tid]) + (S.red2[2][tid] + S.red2[3][tid]);
     }
     // ---- epilogue: wait for the last O^T, then finalise or write the partial ----
     if (ok && c1 > c0)
@@ -423,15 +421,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
     bar_softmax();
     tc_fence_after();
     const bool have = ok && c1 > c0;
+    float* po = single ? nullptr
+                       : P.part + ((size_t)stream * P.nsplit + split) * (kHg * (kC + 2)) + 2 * kHg;
+    __nv_bfloat16* out =
+        single ? static_cast<__nv_bfloat16*>(a.out) + ((size_t)bt * a.H + h0) * kC : nullptr;
 #pragma unroll 1
-    for (int sl = 0; sl < 4; ++sl) {
-      uint32_t o[64];
+    for (int cgrp = 0; cgrp < 16; ++cgrp) {  // slice = cgrp / 4, heads 16*(cgrp%4) ..
+      const int sl = cgrp >> 2, hb = 16 * (cgrp & 3);
+      uint32_t o[16];
       if (have) {
-        tmem_ld_32x32b_x64(tmem + ((uint32_t)(32 * warp) << 16) + kColO + 64 * sl, o);
+        tmem_ld_x16(lane_base + kColO + 64 * sl + hb, o);
         tmem_ld_wait();
       } else {
 #pragma unroll
-        for (int h = 0; h < 64; ++h) o[h] = 0u;
+        for (int h = 0; h < 16; ++h) o[h] = 0u;
       }
       const int d = 128 * sl + tid;
       if (single) {
@@ -441,19 +444,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
           cs = S.cs[(d - r0) >> 1];
           sn = -S.sn[(d - r0) >> 1];  // rotation by -t
         }
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) + ((size_t)bt * a.H + h0) * kC;
 #pragma unroll
-        for (int h = 0; h < 64; ++h) {
-          const float y = __uint_as_float(o[h]) * S.fin[h];
+        for (int h = 0; h < 16; ++h) {
+          const float y = __uint_as_float(o[h]) * S.fin[hb + h];
           const float yp = __shfl_xor_sync(0xffffffffu, y, 1);
           float z = y;
           if (rot) z = (d & 1) == 0 ? y * cs - yp * sn : yp * sn + y * cs;
-          out[(size_t)h * kC + d] = __float2bfloat16_rn(z);
+          out[(size_t)(hb + h) * kC + d] = __float2bfloat16_rn(z);
         }
       } else {
-        float* po = P.part + ((size_t)stream * P.nsplit + split) * (kHg * (kC + 2)) + 2 * kHg;
 #pragma unroll
-        for (int h = 0; h < 64; ++h) po[(size_t)h * kC + d] = __uint_as_float(o[h]);
+        for (int h = 0; h < 16; ++h) po[(size_t)(hb + h) * kC + d] = __uint_as_float(o[h]);
       }
     }
   } else {

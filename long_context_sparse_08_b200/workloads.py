@@ -119,6 +119,17 @@ def quant_mxfp4(x: np.ndarray):
     return packed, (e + 127).astype(np.uint8)
 
 
+def block_key_scales(scales: np.ndarray) -> np.ndarray:
+    """Key-cache scale layout: per block of 128 keys, byte 16*i + 4*j + b holds block-scale b
+    of key 32*j + i (the layout tcgen05.cp copies into TMEM). Input [..., N, 4] in key
+    order (N a multiple of 128); output has the same shape, reordered within blocks."""
+    sc = np.ascontiguousarray(scales, np.uint8)
+    *lead, n, nb = sc.shape
+    assert n % 128 == 0 and nb == 4
+    blk = sc.reshape(*lead, n // 128, 4, 32, 4)          # [.., blk, j, i, b]
+    return np.ascontiguousarray(np.swapaxes(blk, -3, -2)).reshape(*lead, n, 4)
+
+
 # ----------------------------------------------------------------------------
 # workloads
 # ----------------------------------------------------------------------------
@@ -270,7 +281,8 @@ def make_inputs(s: Shape, *, seed: Optional[int] = None) -> Dict[str, np.ndarray
       win_pos0 [B] int64, sink [H] f32,
       qI [B,T,H_I,d_I] (f32 / bf16; MXFP4: qI packed [..,d_I/2] u8 + qI_scale [..,d_I/32] u8),
       KI [B,N_cap,d_I] (f32 / bf16; FP8: u8 codes + KI_scale [B,N_cap] f32; MXFP4: packed
-      [..,d_I/2] + KI_scale [..,d_I/32] u8), w [B,T,H_I] f32,
+      [..,d_I/2] + KI_scale [..,d_I/32] u8 in the blocked order of block_key_scales),
+      w [B,T,H_I] f32,
       compression: Ca Cb Za Zb [n_tok,c], bias [2m,c] (rows 0..m-1 = B^a, m..2m-1 = B^b)
       (HCA: C, Z [n_tok,c], bias [m,c]); prev_Cb / prev_Zb [m,c] for a chunk that does not
       start the sequence. Also KI_f32 / qI_f32 (the fp32 draws before encoding) for the
@@ -345,7 +357,8 @@ def make_inputs(s: Shape, *, seed: Optional[int] = None) -> Dict[str, np.ndarray
             out["KI_f32"] = KI
         elif s.idx == "mxfp4":
             out["qI"], out["qI_scale"] = quant_mxfp4(qI)
-            out["KI"], out["KI_scale"] = quant_mxfp4(KI)
+            out["KI"], ks = quant_mxfp4(KI)
+            out["KI_scale"] = block_key_scales(ks)
             out["KI_f32"], out["qI_f32"] = KI, qI
         else:
             raise ValueError(s.idx)

@@ -105,6 +105,19 @@ def dec_mxfp4(packed, scales) -> np.ndarray:
     return vals * np.repeat(sc, 32, axis=-1)
 
 
+def unblock_key_scales(blocked) -> np.ndarray:
+    """MXFP4 key-cache scales are stored per block of 128 keys with byte 16*i + 4*j + b
+    holding block-scale b of key 32*j + i. Returns them in key order [..., N, 4]."""
+    sc = np.asarray(blocked, np.uint8)
+    *lead, n, nb = sc.shape
+    out = np.empty_like(sc)
+    for blk in range(n // 128):
+        for i in range(32):
+            for j in range(4):
+                out[..., 128 * blk + 32 * j + i, :] = sc[..., 128 * blk + 4 * i + j, :]
+    return out
+
+
 def dec_fp8_rows(codes, row_scale) -> np.ndarray:
     """FP8 e4m3 rows times their per-row fp32 scale."""
     return dec_e4m3(codes) * np.asarray(row_scale, np.float64)[..., None]

@@ -26,7 +26,7 @@ def decode_indexer_request(s, inp, b: int) -> Tuple[np.ndarray, np.ndarray]:
         return O.dec_bf16(inp["qI"][b]), O.dec_fp8_rows(inp["KI"][b], inp["KI_scale"][b])
     if s.idx == "mxfp4":
         return (O.dec_mxfp4(inp["qI"][b], inp["qI_scale"][b]),
-                O.dec_mxfp4(inp["KI"][b], inp["KI_scale"][b]))
+                O.dec_mxfp4(inp["KI"][b], O.unblock_key_scales(inp["KI_scale"][b])))
     raise ValueError(s.idx)
 
 

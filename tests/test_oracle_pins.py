@@ -75,6 +75,17 @@ def test_mxfp4_error_bound():
     assert np.all(err[inside] <= unit[inside] + 1e-12)
 
 
+def test_blocked_key_scale_layout():
+    nat = RNG.integers(0, 255, size=(2, 256, 4)).astype(np.uint8)
+    blk = W.block_key_scales(nat)
+    np.testing.assert_array_equal(O.unblock_key_scales(blk), nat)
+    # explicit position of one key's scales: key 32*j + i of block 1 at word 4*i + j
+    i, j = 5, 3
+    flat = blk[0].reshape(-1)
+    np.testing.assert_array_equal(flat[512 + 16 * i + 4 * j: 512 + 16 * i + 4 * j + 4],
+                                  nat[0, 128 + 32 * j + i])
+
+
 def test_fp8_rowwise_error_bound():
     x = RNG.standard_normal((32, 128)).astype(np.float32)
     codes, sc = W.quant_fp8_rowwise(x)
