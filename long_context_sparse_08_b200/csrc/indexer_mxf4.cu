@@ -3,7 +3,7 @@
 // 【论文解读】DeepSeek-V4, 一(三)1(2): I[t,s] = sum_h w[t,h] * ReLU(q^I[t,h] . K[s]);
 // 二(四) FP4 量化感知训练: the indexer's QK path is cached, loaded and multiplied in FP4.
 //
-// A unit is 256 keys of one query's request: two M-tiles of 128 keys, each
+// A unit is 512 keys of one query's request: four M-tiles of 128 keys, each
 // D[128 keys x 64 heads] = K_tile . q^T over d_I = 128 as two tcgen05 kind::mxf4
 // block-scaled MMAs (K = 64 each, one e8m0 scale per 32 elements of A and of B, exact
 // products, fp32 accumulation in TMEM). TMEM lane = key, column = head, so an epilogue
@@ -11,19 +11,19 @@
 //
 // Key scales are stored in 128-key blocks laid out as tcgen05.cp's 32x128b source: byte
 // 16*i + 4*j + b of a block is block-scale b of key 32*j + i. One TMA copy of a unit's
-// 1 KB of scales therefore lands ready for tcgen05.cp (no rearrangement in the kernel).
+// 2 KB of scales therefore lands ready for tcgen05.cp (no rearrangement in the kernel).
 //
 // Persistent kernel, one CTA per SM, 10 warps:
-//   warp 0     TMA producer: per unit one 16 KB key box (64B-swizzled) and one 1 KB scale
+//   warp 0     TMA producer: per unit one 32 KB key box (64B-swizzled) and one 2 KB scale
 //              box; per query the 64 x 64 B heads and their scale words;
-//   warp 1     MMA issuer: per query the query scales into TMEM (rearranged once), per
-//              M-tile the key scales into TMEM (tcgen05.cp) and two MMAs;
-//   warps 2-9  two epilogue warpgroups; group g reduces M-tile g of every unit:
+//   warp 1     MMA issuer (one lane): per query the query scales into TMEM (rearranged
+//              once), per M-tile the key scales into TMEM (tcgen05.cp) and two MMAs;
+//   warps 2-9  two epilogue warpgroups; group g reduces the M-tiles j with j % 2 == g:
 //              TMEM -> registers, w * ReLU head sum, fp32 score store, and a 4096-bin
 //              histogram of the scores' top 12 key bits for the top-k selector.
-// Four accumulator slots in TMEM let the MMAs of the next unit run while both groups
-// reduce the current one. Units are split evenly over the CTAs; ragged per-query
-// visibility is handled by masking the stores.
+// A ring of six accumulator slots in TMEM lets the MMAs run ahead of the reductions; the
+// fixed cost of each TMA / tcgen05 instruction is spread over 512 keys. Units are split
+// evenly over the CTAs; ragged per-query visibility is handled by masking the stores.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -38,18 +38,19 @@ namespace {
 
 using namespace tc;
 
-constexpr int kStages = 6;
+constexpr int kStages = 4;
 constexpr int kTileKeys = 128;     // M of one MMA
-constexpr int kUnitKeys = 256;     // keys per pipeline stage (two M-tiles)
+constexpr int kUnitTiles = 4;
+constexpr int kUnitKeys = kUnitTiles * kTileKeys;  // keys per pipeline stage
 constexpr int kHeads = 64;         // N (indexer heads)
 constexpr int kRowBytes = 64;      // 128 e2m1 per row
 constexpr int kMaxQueries = 1024;  // (request, query) pairs per launch
 constexpr int kThreads = 320;
 constexpr int kBins = 4096;
 
-constexpr int kOffA = 0;                                // 16 KB, 1024-aligned
-constexpr int kOffSF = kOffA + kUnitKeys * kRowBytes;   // 1 KB key scales (cp layout)
-constexpr int kStageBytes = ((kOffSF + 1024 + 1023) / 1024) * 1024;
+constexpr int kOffA = 0;                                // 32 KB, 1024-aligned
+constexpr int kOffSF = kOffA + kUnitKeys * kRowBytes;   // 2 KB key scales (cp layout)
+constexpr int kStageBytes = ((kOffSF + kUnitKeys * 4 + 1023) / 1024) * 1024;
 constexpr uint32_t kStageTx = kUnitKeys * kRowBytes + kUnitKeys * 4;
 // per-query buffers (two slots)
 constexpr int kOffQ = 0;                                // 4 KB q heads (64B-swizzled)
@@ -58,12 +59,12 @@ constexpr int kOffQSF = kOffQS + kHeads * 4;            // 512 B rearranged for 
 constexpr int kQBytes = ((kOffQSF + 512 + 1023) / 1024) * 1024;
 constexpr uint32_t kQTx = kHeads * kRowBytes + kHeads * 4;
 
-// TMEM columns
-constexpr int kAcc = 4;
+// TMEM columns: a ring of accumulator slots, their key-scale columns, two query-scale slots
+constexpr int kAcc = 6;
 constexpr uint32_t kTmemCols = 512;
-__device__ __forceinline__ uint32_t acc_col(int s) { return 64u * s; }          // 0..192
-__device__ __forceinline__ uint32_t sfa_col(int s) { return 256u + 8u * s; }    // 256..280
-__device__ __forceinline__ uint32_t sfb_col(int qs) { return 320u + 8u * qs; }  // 320, 328
+__device__ __forceinline__ uint32_t acc_col(int s) { return 64u * s; }          // 0..320
+__device__ __forceinline__ uint32_t sfa_col(int s) { return 384u + 8u * s; }    // 384..424
+__device__ __forceinline__ uint32_t sfb_col(int qs) { return 448u + 8u * qs; }  // 448, 456
 
 enum { kErrFull = 101, kErrEmpty = 102, kErrTmemFull = 103, kErrTmemEmpty = 104,
        kErrQFull = 105, kErrQEmpty = 106 };
@@ -204,10 +205,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         uint8_t* sb = base + st * kStageBytes;
         const int b = q / p.T;
-        const int32_t row0 = (int32_t)(b * p.n_cap + (int64_t)unit * kUnitKeys);
+        // keys and scales are viewed in 128-key blocks; a unit is 4 consecutive blocks
+        const int32_t blk0 = (int32_t)((b * p.n_cap + (int64_t)unit * kUnitKeys) / kTileKeys);
         mbar_arrive_expect_tx(&S.full[st], kStageTx);
-        tma_load_2d(sb + kOffA, &tm_k, 0, row0, &S.full[st]);
-        tma_load_1d(sb + kOffSF, &tm_ks, row0, &S.full[st]);
+        tma_load_3d(sb + kOffA, &tm_k, 0, 0, blk0, &S.full[st]);
+        tma_load_2d(sb + kOffSF, &tm_ks, 0, blk0, &S.full[st]);
       }
       // drain: no copy into this CTA's shared memory may still be in flight at exit
       for (int j = (k > kStages ? k - kStages : 0); j < k; ++j)
@@ -216,51 +218,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&S.qfull[j & 1], (uint32_t)((j >> 1) & 1), kErrQFull);
     }
   } else if (warp == 1) {
-    // ------------------------------ MMA issuer ------------------------------
-    const uint32_t id0 = idesc_mxf4(kTileKeys, kHeads, 0, 0);
-    const uint32_t id1 = idesc_mxf4(kTileKeys, kHeads, 2, 2);
-    int q = u0 < u1 ? find_query(S.prefix, p.Q, u0) : 0;
-    int cur_q = -1, nq = -1;
-    int k = 0;
-    bool ok = true;
-    for (int u = u0; u < u1 && ok; ++u, ++k) {
-      while (u >= S.prefix[q + 1]) ++q;
-      if (q != cur_q) {
-        if (cur_q >= 0 && lane == 0) mma_commit(&S.qempty[nq & 1]);  // old slot free when done
-        ++nq;
-        cur_q = q;
-        const int qs = nq & 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(&S.qfull[qs], (nq >> 1) & 1, kErrQFull));
-        if (!ok) break;
-        // query scale words -> tcgen05.cp layout (16-byte row i: words of heads i, 32+i)
-        uint8_t* qb = qbase + qs * kQBytes;
-        const uint32_t* sq = reinterpret_cast<const uint32_t*>(qb + kOffQS);
-        *reinterpret_cast<uint4*>(qb + kOffQSF + 16 * lane) =
-            make_uint4(sq[lane], sq[32 + lane], 0u, 0u);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
+    // ------------------------------ MMA issuer (one lane) ------------------------------
+    if (lane == 0) {
+      const uint32_t id0 = idesc_mxf4(kTileKeys, kHeads, 0, 0);
+      const uint32_t id1 = idesc_mxf4(kTileKeys, kHeads, 2, 2);
+      int q = u0 < u1 ? find_query(S.prefix, p.Q, u0) : 0;
+      int cur_q = -1, nq = -1;
+      int k = 0;
+      bool ok = true;
+      for (int u = u0; u < u1 && ok; ++u, ++k) {
+        while (u >= S.prefix[q + 1]) ++q;
+        if (q != cur_q) {
+          if (cur_q >= 0) mma_commit(&S.qempty[nq & 1]);  // old slot free once its MMAs end
+          ++nq;
+          cur_q = q;
+          const int qs = nq & 1;
+          ok = mbar_wait(&S.qfull[qs], (nq >> 1) & 1, kErrQFull);
+          if (!ok) break;
+          // query scale words -> tcgen05.cp layout (16-byte row i: words of heads i, 32+i)
+          uint8_t* qb = qbase + qs * kQBytes;
+          const uint32_t* sq = reinterpret_cast<const uint32_t*>(qb + kOffQS);
+          for (int i = 0; i < 32; ++i)
+            *reinterpret_cast<uint4*>(qb + kOffQSF + 16 * i) = make_uint4(sq[i], sq[32 + i], 0u, 0u);
+          fence_proxy_async_smem();
           tc_fence_after();
           tmem_cp_32x128b_warpx4(tmem + sfb_col(qs),
                                  smem_desc(smem_u32(qb + kOffQSF), 0, 128, kLayoutNone));
         }
-      }
-      const int qs = nq & 1;
-      const int st = k % kStages;
-      const uint32_t round = (uint32_t)(k / kStages);
-      ok = __all_sync(0xffffffffu, mbar_wait(&S.full[st], round & 1, kErrFull));
-      if (!ok) break;
-      uint8_t* sb = base + st * kStageBytes;
-      int good = 1;
-      if (lane == 0) {
+        const int qs = nq & 1;
+        const int st = k % kStages;
+        ok = mbar_wait(&S.full[st], (uint32_t)(k / kStages) & 1, kErrFull);
+        if (!ok) break;
+        uint8_t* sb = base + st * kStageBytes;
         const uint64_t b0 = smem_desc(smem_u32(qbase + qs * kQBytes + kOffQ), 16,
                                       8 * kRowBytes, kLayoutSw64);
         const uint32_t sfb = tmem + sfb_col(qs);
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          const int slot = 2 * (k & 1) + t;
-          good = mbar_wait(&S.tempty[slot], (((uint32_t)k >> 1) & 1) ^ 1, kErrTmemEmpty);
-          if (!good) break;
+#pragma unroll 1
+        for (int t = 0; t < kUnitTiles; ++t) {
+          const int g = kUnitTiles * k + t;  // tile index within this CTA
+          const int slot = g % kAcc;
+          ok = mbar_wait(&S.tempty[slot], ((uint32_t)(g / kAcc) & 1) ^ 1, kErrTmemEmpty);
+          if (!ok) break;
           tc_fence_after();
           const uint32_t sfa = tmem + sfa_col(slot);
           tmem_cp_32x128b_warpx4(
@@ -273,12 +271,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_mxf4(d, a0 + 2, b0 + 2, id1, sfa | (2u << 30), sfb | (2u << 30), 1u);
           mma_commit(&S.tfull[slot]);
         }
-        if (good) mma_commit(&S.empty[st]);
+        if (ok) mma_commit(&S.empty[st]);
       }
-      ok = __shfl_sync(0xffffffffu, good, 0) != 0;
-    }
-    // every MMA / copy this thread issued has completed once `done` fires
-    if (lane == 0) {
+      // every MMA / copy this thread issued has completed once `done` fires
       mma_commit(&S.done);
       mbar_wait(&S.done, 0, kErrTmemFull);
     }
@@ -304,7 +299,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int cur_q = -1;
     int q = u0 < u1 ? find_query(S.prefix, p.Q, u0) : 0;
     int k = 0;
-    for (int u = u0; u < u1; ++u, ++k) {
+    bool ok = true;
+    for (int u = u0; u < u1 && ok; ++u, ++k) {
       while (u >= S.prefix[q + 1]) ++q;
       const int unit = u - S.prefix[q];
       if (q != cur_q) {
@@ -316,24 +312,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (hq >= 0) flush(hq);
         hq = q;
       }
-      const int slot = 2 * (k & 1) + grp;
-      if (!epi_all_ok(mbar_wait(&S.tfull[slot], ((uint32_t)k >> 1) & 1, kErrTmemFull))) break;
-      tc_fence_after();
-      uint32_t v[kHeads];
-      tmem_ld_32x32b_x64(tmem + ((uint32_t)(32 * quad) << 16) + acc_col(slot), v);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.tempty[slot]);
-      float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+      for (int t = grp; t < kUnitTiles; t += 2) {
+        const int g = kUnitTiles * k + t;
+        const int slot = g % kAcc;
+        ok = epi_all_ok(mbar_wait(&S.tfull[slot], (uint32_t)(g / kAcc) & 1, kErrTmemFull));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t v[kHeads];
+        tmem_ld_32x32b_x64(tmem + ((uint32_t)(32 * quad) << 16) + acc_col(slot), v);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.tempty[slot]);
+        float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int h = 0; h < kHeads; ++h)
-        part[h & 3] = fmaf(wr[h], fmaxf(__uint_as_float(v[h]), 0.f), part[h & 3]);
-      const float sc = (part[0] + part[1]) + (part[2] + part[3]);
-      const int s = unit * kUnitKeys + grp * kTileKeys + 32 * quad + lane;
-      if (s < S.nvis[q]) {
-        p.scores[(size_t)q * p.n_cap + s] = sc;
-        if (hist) atomicAdd(&S.hist[float_key(sc) >> 20], 1);
+        for (int h = 0; h < kHeads; ++h)
+          part[h & 3] = fmaf(wr[h], fmaxf(__uint_as_float(v[h]), 0.f), part[h & 3]);
+        const float sc = (part[0] + part[1]) + (part[2] + part[3]);
+        const int s = unit * kUnitKeys + t * kTileKeys + 32 * quad + lane;
+        if (s < S.nvis[q]) {
+          p.scores[(size_t)q * p.n_cap + s] = sc;
+          if (hist) atomicAdd(&S.hist[float_key(sc) >> 20], 1);
+        }
       }
     }
     if (hist && hq >= 0) flush(hq);
@@ -359,6 +360,33 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
   });
   return fn;
+}
+
+// keys as [128-key blocks][128 rows][64 B], box = 4 blocks (one 512-key unit)
+bool make_map_keys(CUtensorMap* m, const void* ptr, uint64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kRowBytes, (cuuint64_t)kTileKeys,
+                        (cuuint64_t)(rows / kTileKeys)};
+  cuuint64_t strides[2] = {(cuuint64_t)kRowBytes, (cuuint64_t)kRowBytes * kTileKeys};
+  cuuint32_t box[3] = {(cuuint32_t)kRowBytes, (cuuint32_t)kTileKeys, (cuuint32_t)kUnitTiles};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// key scale words as [128-key blocks][128 words], box = 4 blocks
+bool make_map_key_scales(CUtensorMap* m, const void* ptr, uint64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kTileKeys, (cuuint64_t)(rows / kTileKeys)};
+  cuuint64_t strides[1] = {(cuuint64_t)kTileKeys * 4};
+  cuuint32_t box[2] = {(cuuint32_t)kTileKeys, (cuuint32_t)kUnitTiles};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool make_map_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows) {
@@ -406,8 +434,8 @@ bool index_mxf4_tc_supported(const IndexArgs& a) {
 cudaError_t launch_index_mxf4_tc(const IndexArgs& a, cudaStream_t st) {
   const int Q = a.B * a.T;
   CUtensorMap mk, mks, mq, mqs;
-  if (!make_map_2d(&mk, a.KI, (uint64_t)a.B * a.n_cap, kUnitKeys) ||
-      !make_map_1d_words(&mks, a.KI_scale, (uint64_t)a.B * a.n_cap, kUnitKeys) ||
+  if (!make_map_keys(&mk, a.KI, (uint64_t)a.B * a.n_cap) ||
+      !make_map_key_scales(&mks, a.KI_scale, (uint64_t)a.B * a.n_cap) ||
       !make_map_2d(&mq, a.qI, (uint64_t)Q * kHeads, kHeads) ||
       !make_map_1d_words(&mqs, a.qI_scale, (uint64_t)Q * kHeads, kHeads))
     return cudaErrorInvalidValue;
