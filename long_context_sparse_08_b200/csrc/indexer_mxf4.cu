@@ -18,12 +18,14 @@
 //              box; per query the 64 x 64 B heads and their scale words;
 //   warp 1     MMA issuer (one lane): per query the query scales into TMEM (rearranged
 //              once), per M-tile the key scales into TMEM (tcgen05.cp) and two MMAs;
-//   warps 2-9  two epilogue warpgroups; group g reduces the M-tiles j with j % 2 == g:
+//   warps 2-9  two epilogue warpgroups; group g reduces M-tiles g and 2 + g of each unit:
 //              TMEM -> registers, w * ReLU head sum, fp32 score store, and a 4096-bin
 //              histogram of the scores' top 12 key bits for the top-k selector.
-// A ring of six accumulator slots in TMEM lets the MMAs run ahead of the reductions; the
-// fixed cost of each TMA / tcgen05 instruction is spread over 512 keys. Units are split
-// evenly over the CTAs; ragged per-query visibility is handled by masking the stores.
+// TMEM holds two half-unit slots (2 M-tiles each): while both groups reduce one half-unit
+// the MMAs of the next run. Every wait and tcgen05 instruction costs tens of cycles on the
+// single issuing thread, so the loop precomputes descriptors and waits once per half-unit.
+// Units are split evenly over the CTAs; ragged per-query visibility is handled by masking
+// the stores.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -59,12 +61,12 @@ constexpr int kOffQSF = kOffQS + kHeads * 4;            // 512 B rearranged for 
 constexpr int kQBytes = ((kOffQSF + 512 + 1023) / 1024) * 1024;
 constexpr uint32_t kQTx = kHeads * kRowBytes + kHeads * 4;
 
-// TMEM columns: a ring of accumulator slots, their key-scale columns, two query-scale slots
-constexpr int kAcc = 6;
+// TMEM columns: two half-unit slots of two 64-column accumulators, their key-scale columns,
+// two query-scale slots
 constexpr uint32_t kTmemCols = 512;
-__device__ __forceinline__ uint32_t acc_col(int s) { return 64u * s; }          // 0..320
-__device__ __forceinline__ uint32_t sfa_col(int s) { return 384u + 8u * s; }    // 384..424
-__device__ __forceinline__ uint32_t sfb_col(int qs) { return 448u + 8u * qs; }  // 448, 456
+__device__ __forceinline__ uint32_t acc_col(int hs, int j) { return 128u * hs + 64u * j; }
+__device__ __forceinline__ uint32_t sfa_col(int hs, int j) { return 256u + 16u * hs + 8u * j; }
+__device__ __forceinline__ uint32_t sfb_col(int qs) { return 288u + 8u * qs; }
 
 enum { kErrFull = 101, kErrEmpty = 102, kErrTmemFull = 103, kErrTmemEmpty = 104,
        kErrQFull = 105, kErrQEmpty = 106 };
@@ -79,7 +81,7 @@ struct Mxf4Params {
 };
 
 struct Smem {
-  uint64_t full[kStages], empty[kStages], tfull[kAcc], tempty[kAcc], qfull[2], qempty[2], done;
+  uint64_t full[kStages], empty[kStages], tfull[2], tempty[2], qfull[2], qempty[2], done;
   uint32_t tmem_slot;
   int prefix[kMaxQueries + 1];
   int nvis[kMaxQueries];
@@ -149,9 +151,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&S.full[i], 1);
         mbar_init(&S.empty[i], 1);
       }
-      for (int i = 0; i < kAcc; ++i) {
+      for (int i = 0; i < 2; ++i) {
         mbar_init(&S.tfull[i], 1);
-        mbar_init(&S.tempty[i], 4);
+        mbar_init(&S.tempty[i], 8);  // every epilogue warp
       }
       for (int i = 0; i < 2; ++i) {
         mbar_init(&S.qfull[i], 1);
@@ -222,6 +224,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t id0 = idesc_mxf4(kTileKeys, kHeads, 0, 0);
       const uint32_t id1 = idesc_mxf4(kTileKeys, kHeads, 2, 2);
+      const uint64_t a_desc0 = smem_desc(smem_u32(base + kOffA), 16, 8 * kRowBytes, kLayoutSw64);
+      const uint64_t sf_desc0 = smem_desc(smem_u32(base + kOffSF), 0, 128, kLayoutNone);
+      const uint64_t q_desc0 = smem_desc(smem_u32(qbase + kOffQ), 16, 8 * kRowBytes, kLayoutSw64);
       int q = u0 < u1 ? find_query(S.prefix, p.Q, u0) : 0;
       int cur_q = -1, nq = -1;
       int k = 0;
@@ -249,29 +254,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int st = k % kStages;
         ok = mbar_wait(&S.full[st], (uint32_t)(k / kStages) & 1, kErrFull);
         if (!ok) break;
-        uint8_t* sb = base + st * kStageBytes;
-        const uint64_t b0 = smem_desc(smem_u32(qbase + qs * kQBytes + kOffQ), 16,
-                                      8 * kRowBytes, kLayoutSw64);
+        const uint64_t a_st = a_desc0 + (uint64_t)st * (kStageBytes >> 4);
+        const uint64_t sf_st = sf_desc0 + (uint64_t)st * (kStageBytes >> 4);
+        const uint64_t b0 = q_desc0 + (uint64_t)qs * (kQBytes >> 4);
         const uint32_t sfb = tmem + sfb_col(qs);
-#pragma unroll 1
-        for (int t = 0; t < kUnitTiles; ++t) {
-          const int g = kUnitTiles * k + t;  // tile index within this CTA
-          const int slot = g % kAcc;
-          ok = mbar_wait(&S.tempty[slot], ((uint32_t)(g / kAcc) & 1) ^ 1, kErrTmemEmpty);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // half-units: M-tiles 2h, 2h+1
+          const int n = 2 * k + h, hs = n & 1;
+          ok = mbar_wait(&S.tempty[hs], ((uint32_t)(n >> 1) & 1) ^ 1, kErrTmemEmpty);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t sfa = tmem + sfa_col(slot);
-          tmem_cp_32x128b_warpx4(
-              sfa, smem_desc(smem_u32(sb + kOffSF + 512 * t), 0, 128, kLayoutNone));
-          const uint64_t a0 = smem_desc(smem_u32(sb + kOffA + t * kTileKeys * kRowBytes), 16,
-                                        8 * kRowBytes, kLayoutSw64);
-          const uint32_t d = tmem + acc_col(slot);
-          mma_mxf4(d, a0, b0, id0, sfa, sfb, 0u);
-          // second K half: +32 bytes inside the swizzled rows, scale bytes 2..3
-          mma_mxf4(d, a0 + 2, b0 + 2, id1, sfa | (2u << 30), sfb | (2u << 30), 1u);
-          mma_commit(&S.tfull[slot]);
+#pragma unroll
+          for (int j = 0; j < 2; ++j)  // key scales of both tiles first (latencies overlap)
+            tmem_cp_32x128b_warpx4(tmem + sfa_col(hs, j), sf_st + (uint64_t)(2 * h + j) * 32);
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const uint64_t a0 = a_st + (uint64_t)(2 * h + j) * 512;  // 8 KB per M-tile
+            const uint32_t d = tmem + acc_col(hs, j), sfa = tmem + sfa_col(hs, j);
+            mma_mxf4(d, a0, b0, id0, sfa, sfb, 0u);
+            // second K half: +32 bytes inside the swizzled rows, scale bytes 2..3
+            mma_mxf4(d, a0 + 2, b0 + 2, id1, sfa | (2u << 30), sfb | (2u << 30), 1u);
+          }
+          mma_commit(&S.tfull[hs]);
         }
-        if (ok) mma_commit(&S.empty[st]);
+        if (!ok) break;
+        mma_commit(&S.empty[st]);
       }
       // every MMA / copy this thread issued has completed once `done` fires
       mma_commit(&S.done);
@@ -313,22 +320,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         hq = q;
       }
 #pragma unroll 1
-      for (int t = grp; t < kUnitTiles; t += 2) {
-        const int g = kUnitTiles * k + t;
-        const int slot = g % kAcc;
-        ok = epi_all_ok(mbar_wait(&S.tfull[slot], (uint32_t)(g / kAcc) & 1, kErrTmemFull));
+      for (int h = 0; h < 2; ++h) {  // this group reduces M-tile 2h + grp of the unit
+        const int n = 2 * k + h, hs = n & 1, t = 2 * h + grp;
+        ok = epi_all_ok(mbar_wait(&S.tfull[hs], (uint32_t)(n >> 1) & 1, kErrTmemFull));
         if (!ok) break;
         tc_fence_after();
         uint32_t v[kHeads];
-        tmem_ld_32x32b_x64(tmem + ((uint32_t)(32 * quad) << 16) + acc_col(slot), v);
+        tmem_ld_32x32b_x64(tmem + ((uint32_t)(32 * quad) << 16) + acc_col(hs, grp), v);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.tempty[slot]);
+        if (lane == 0) mbar_arrive(&S.tempty[hs]);
         float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int h = 0; h < kHeads; ++h)
-          part[h & 3] = fmaf(wr[h], fmaxf(__uint_as_float(v[h]), 0.f), part[h & 3]);
+        for (int hh = 0; hh < kHeads; ++hh)
+          part[hh & 3] = fmaf(wr[hh], fmaxf(__uint_as_float(v[hh]), 0.f), part[hh & 3]);
         const float sc = (part[0] + part[1]) + (part[2] + part[3]);
         const int s = unit * kUnitKeys + t * kTileKeys + 32 * quad + lane;
         if (s < S.nvis[q]) {
