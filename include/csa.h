@@ -138,6 +138,25 @@ csa_status csa_topk(const csa_params* p, int32_t B, int32_t T, int64_t N_cap,
                     const float* scores, const int64_t* q_pos, int32_t* out_idx, void* ws,
                     size_t ws_bytes, void* stream);
 
+/*
+ * Stage 3 as csa_topk, for callers that cannot hand the library device scratch (a host
+ * program without a device allocator of its own, or one whose device memory is already
+ * reserved for its caches). The paper has no counterpart: this is an interface variant.
+ * Allocates nothing: the scratch is one library-owned device array of
+ * CSA_TOPK_NOALLOC_SCRATCH_BYTES per device. The first call on a device looks up that
+ * array's address (with the device current) and should come before any stream capture.
+ * All calls on a device share the array; each call zeroes the counters it needs on its own
+ * stream, so calls whose execution overlaps (other streams, other host threads) race:
+ * serialise them. Returns CSA_ERR_WORKSPACE, launching nothing, when the call would need
+ * more scratch than the array holds (csa_workspace_size(p, CSA_WS_TOPK, ...) bytes; e.g.
+ * 4 rows of N_cap = 262144 with k = 1024 need about 8.5 MB; B*T > 64 or N_cap < 8192
+ * need none). Results are identical to csa_topk's. Other arguments and errors as csa_topk.
+ */
+#define CSA_TOPK_NOALLOC_SCRATCH_BYTES (16u << 20)
+csa_status csa_topk_noalloc(const csa_params* p, int32_t B, int32_t T, int64_t N_cap,
+                            const float* scores, const int64_t* q_pos, int32_t* out_idx,
+                            void* stream);
+
 /* Stages 2 + 3 in one call. out_scores may be NULL (the scores then live in the workspace). */
 csa_status csa_index_topk(const csa_params* p, csa_dtype kdt, int32_t B, int32_t T,
                           int64_t N_cap, const void* qI, const void* qI_scale, const float* w,

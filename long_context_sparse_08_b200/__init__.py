@@ -23,7 +23,10 @@ EXPORTS = (
     "csa_compress", "csa_index_scores", "csa_topk", "csa_index_topk", "csa_sparse_mqa",
     "hca_dense_mqa", "csa_forward", "csa_workspace_size", "csa_status_string",
     "csa_last_error", "csa_set_index_timing_events", "csa_version", "csa_device_error",
+    "csa_topk_noalloc",
 )
+# size of the library-owned scratch array behind csa_topk_noalloc (bytes, per device)
+TOPK_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class CsaParams(ctypes.Structure):
@@ -63,6 +66,7 @@ _SIGS = {
     "csa_compress": [_PP, ctypes.c_int, _I32, _I64, _I64, _I64] + [_VP] * 8 + [_I32, _VP, _VP],
     "csa_index_scores": [_PP, ctypes.c_int, _I32, _I32, _I64] + [_VP] * 7 + [_VP],
     "csa_topk": [_PP, _I32, _I32, _I64, _VP, _VP, _VP, _VP, _SZ, _VP],
+    "csa_topk_noalloc": [_PP, _I32, _I32, _I64, _VP, _VP, _VP, _VP],
     "csa_index_topk": [_PP, ctypes.c_int, _I32, _I32, _I64] + [_VP] * 9 + [_SZ, _VP],
     "csa_sparse_mqa": [_PP, ctypes.c_int, _I32, _I32, _VP, _VP, _VP, _I64, _VP, _VP, _I64,
                        _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
@@ -179,6 +183,15 @@ def csa_topk(p, B, T, N_cap, scores, q_pos, out_idx, ws, ws_bytes, stream=None):
     s = lib().csa_topk(ctypes.byref(p), B, T, N_cap, _ptr(scores), _ptr(q_pos), _ptr(out_idx),
                        _ptr(ws), ws_bytes, _stream(stream))
     _check("csa_topk", s)
+
+
+def csa_topk_noalloc(p, B, T, N_cap, scores, q_pos, out_idx, stream=None):
+    """csa_topk without caller scratch: the library's own device array serves as scratch
+    (nothing is allocated). Calls on one device share that array, so they must not overlap
+    in execution; the first call on a device should come before any stream capture."""
+    s = lib().csa_topk_noalloc(ctypes.byref(p), B, T, N_cap, _ptr(scores), _ptr(q_pos),
+                               _ptr(out_idx), _stream(stream))
+    _check("csa_topk_noalloc", s)
 
 
 def csa_index_topk(p, kdt, B, T, N_cap, qI, qI_scale, w, KI, KI_scale, q_pos, out_idx,

@@ -452,3 +452,15 @@ csa_status csa_forward(const csa_params* p, csa_dtype io, int32_t B, int32_t T,
 }
 
 }  // extern "C"
+
+namespace csa {
+
+csa_status report_error(csa_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+}  // namespace csa

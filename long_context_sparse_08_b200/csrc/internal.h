@@ -80,6 +80,9 @@ cudaError_t launch_mqa_tc(const MqaArgs& a, void* ws, size_t ws_bytes, cudaStrea
 cudaError_t mqa_tc_device_error(int* code);
 cudaError_t launch_mqa(const MqaArgs& a, bool bf16, void* ws, size_t ws_bytes, cudaStream_t st);
 
+// Records a formatted message as the calling thread's csa_last_error() and returns `s`.
+csa_status report_error(csa_status s, const char* fmt, ...);
+
 // benchmarking hook (see csa_set_index_timing_events)
 void timing_before(cudaStream_t st);
 void timing_after(cudaStream_t st);
