@@ -53,8 +53,7 @@ struct TopkDecodeArgs {
   int32_t* out_idx;
   int* hist;          // [Q][4096]
   int* cnt;           // [Q][4]: sure count, boundary count, ticket
-  uint64_t* sure;     // [Q][k]
-  uint64_t* bnd;      // [Q][n_cap]
+  uint64_t* list;     // [Q][k + n_cap]: sure list (k), then boundary list (n_cap)
 };
 bool topk_decode_path(int B, int T, int64_t n_cap, int k);
 size_t topk_decode_ws_bytes(int B, int T, int64_t n_cap, int k);

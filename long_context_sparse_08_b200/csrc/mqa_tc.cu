@@ -219,7 +219,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
     }
     tmem_alloc(&S.tmem_slot, kTmemCols);
   } else {
-    // RoPE table, running stats, and q_hat = RoPE_t(RMSNorm(q)) into the B-operand layout
+    // the group's 64 raw query rows (64 KB, contiguous) into the KV tile area, which the
+    // first gather only overwrites after q_hat is built; one pass, one latency
+    const uint32_t stage = smem_u32(base + kOffKV);
+    const uint4* qg = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) +
+                                                     ((size_t)bt * a.H + h0) * kC);
+#pragma unroll 4
+    for (int i = tid; i < kHg * kC / 8; i += 128) cp_async16(stage + 16 * i, qg + i, true);
+    // RoPE table and running stats while the copies are in flight
     for (int p = tid; p < r / 2; p += 128)
       rope_cos_sin((double)rl.t, p, r, (double)a.rope_base, &S.cs[p], &S.sn[p]);
     if (tid < kHg) {
@@ -235,15 +242,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
   if (warp < 4) {
     // ---- q_hat = RoPE_t(RMSNorm(q)) in bf16, one warp per head (lane = 16 dims) ----
     uint8_t* qs = base + kOffQ;
+    float wq[16];  // RMSNorm weights of this lane's dims (the same for every head)
+#pragma unroll
+    for (int half = 0; half < 2; ++half)
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        wq[8 * half + k] = a.q_rms_w ? __bfloat162float(static_cast<const __nv_bfloat16*>(
+                                           a.q_rms_w)[8 * (lane + 32 * half) + k])
+                                     : 1.f;
+    cp_async_wait_all();
+    bar_softmax();
 #pragma unroll 1
     for (int h = warp; h < kHg; h += 4) {
-      const __nv_bfloat16* qrow =
-          static_cast<const __nv_bfloat16*>(a.q) + ((size_t)bt * a.H + h0 + h) * kC;
+      const uint4* qrow = reinterpret_cast<const uint4*>(base + kOffKV + h * (kC * 2));
       float x[16];
       float ss = 0.f;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        const uint4 raw = reinterpret_cast<const uint4*>(qrow)[lane + 32 * half];
+        const uint4 raw = qrow[lane + 32 * half];
         const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -260,11 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
         const int d0 = 8 * (lane + 32 * half);
         float y[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          y[k] = x[8 * half + k] * rstd;
-          if (a.q_rms_w)
-            y[k] *= __bfloat162float(static_cast<const __nv_bfloat16*>(a.q_rms_w)[d0 + k]);
-        }
+        for (int k = 0; k < 8; ++k) y[k] = x[8 * half + k] * rstd * wq[8 * half + k];
         if (d0 >= r0) {
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
