@@ -255,6 +255,12 @@ csa_status csa_device_error(int32_t* code);
 /* Library version string. */
 const char* csa_version(void);
 
+/*
+ * Number of kernels this library has launched in the process so far (every entry point,
+ * every device). Diagnostic: the difference across a region counts its launches.
+ */
+uint64_t csa_kernel_launches(void);
+
 #ifdef __cplusplus
 }
 #endif

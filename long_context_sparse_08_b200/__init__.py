@@ -23,7 +23,7 @@ EXPORTS = (
     "csa_compress", "csa_index_scores", "csa_topk", "csa_index_topk", "csa_sparse_mqa",
     "hca_dense_mqa", "csa_forward", "csa_workspace_size", "csa_status_string",
     "csa_last_error", "csa_set_index_timing_events", "csa_version", "csa_device_error",
-    "csa_topk_noalloc",
+    "csa_topk_noalloc", "csa_kernel_launches",
 )
 # size of the library-owned scratch array behind csa_topk_noalloc (bytes, per device)
 TOPK_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -80,8 +80,9 @@ _SIGS = {
     "csa_set_index_timing_events": [ctypes.POINTER(_VP), ctypes.POINTER(_VP), _I32],
     "csa_version": [],
     "csa_device_error": [ctypes.POINTER(ctypes.c_int32)],
+    "csa_kernel_launches": [],
 }
-_RES = {"csa_workspace_size": _SZ, "csa_status_string": ctypes.c_char_p,
+_RES = {"csa_workspace_size": _SZ, "csa_kernel_launches": ctypes.c_uint64, "csa_status_string": ctypes.c_char_p,
         "csa_last_error": ctypes.c_char_p, "csa_version": ctypes.c_char_p,
         "csa_set_index_timing_events": None}
 
@@ -114,6 +115,11 @@ def status_string(s: int) -> str:
 
 def last_error() -> str:
     return lib().csa_last_error().decode()
+
+
+def kernel_launches() -> int:
+    """Kernels the library has launched in this process so far."""
+    return int(lib().csa_kernel_launches())
 
 
 def version() -> str:

@@ -4,10 +4,16 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <vector>
 
 #include "common.cuh"
 #include "internal.h"
+
+namespace csa {
+std::atomic<uint64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace csa
 
 namespace {
 
@@ -194,6 +200,7 @@ csa_status index_then_topk(const csa_params* p, csa_dtype kdt, int32_t B, int32_
       const csa::TopkDecodeArgs da = csa::topk_decode_args(t, topk_ws);
       TRY(cuda_status(csa::topk_decode_clear(da, st), "top-k clear"));
       ia.hist = da.hist;
+      ia.chained = true;
     }
     TRY(cuda_status(csa::launch_index_scores(ia, st, &hist_done), "index scores"));
   }
@@ -446,10 +453,13 @@ csa_status csa_forward(const csa_params* p, csa_dtype io, int32_t B, int32_t T,
                       a->KI_scale, a->q_pos, scores, t, base + sb, tb, st));
   auto ma = make_mqa(p, B, T, a->q, a->q_pos, a->kv_cache, a->N_cap, a->out_idx, p->topk,
                      a->win_kv, a->L_raw, a->win_pos0, a->sink, a->q_rms_w, a->out);
+  ma.chained = true;  // a top-k kernel of this library precedes it on the stream
   TRY(cuda_status(csa::launch_mqa(ma, io == CSA_BF16, base + sb + tb, ws_bytes - sb - tb, st),
                   "sparse MQA"));
   return ok();
 }
+
+uint64_t csa_kernel_launches(void) { return csa::g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"
 

@@ -57,6 +57,18 @@ __device__ __forceinline__ uint32_t float_key(float f) {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch. A kernel launched with the programmatic stream
+// serialisation attribute may start while its predecessor in the stream still runs;
+// pdl_wait() returns once every prerequisite grid has completed and its writes are
+// visible, pdl_trigger() lets the next such kernel start. Both do nothing in a kernel
+// launched the ordinary way.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // reductions
 // ---------------------------------------------------------------------------
 

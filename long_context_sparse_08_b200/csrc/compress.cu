@@ -101,9 +101,9 @@ cudaError_t launch_compress(const CompressArgs& a, bool bf16, cudaStream_t st) {
   const int threads = a.c >= 256 ? 256 : ((a.c + 31) / 32) * 32;
   const size_t smem = (size_t)a.c * sizeof(float);
   if (bf16)
-    k_compress<__nv_bfloat16><<<grid, threads, smem, st>>>(a);
+    launch(false, k_compress<__nv_bfloat16>, dim3(grid), dim3(threads), smem, st, a);
   else
-    k_compress<float><<<grid, threads, smem, st>>>(a);
+    launch(false, k_compress<float>, dim3(grid), dim3(threads), smem, st, a);
   return cudaGetLastError();
 }
 

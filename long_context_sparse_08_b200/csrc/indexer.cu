@@ -131,13 +131,14 @@ cudaError_t launch_index_scores(const IndexArgs& a, cudaStream_t st, bool* hist_
   timing_before(st);
   switch (a.kdt) {
     case CSA_F32:
-      k_index_scores_cc<CSA_F32><<<grid, kKeysPerCta, smem, st>>>(a);
+      launch(false, k_index_scores_cc<CSA_F32>, dim3(grid), dim3(kKeysPerCta), smem, st, a);
       break;
     case CSA_BF16:
-      k_index_scores_cc<CSA_BF16><<<grid, kKeysPerCta, smem, st>>>(a);
+      launch(false, k_index_scores_cc<CSA_BF16>, dim3(grid), dim3(kKeysPerCta), smem, st, a);
       break;
     default:
-      k_index_scores_cc<CSA_FP8_E4M3_ROWSCALE><<<grid, kKeysPerCta, smem, st>>>(a);
+      launch(false, k_index_scores_cc<CSA_FP8_E4M3_ROWSCALE>, dim3(grid), dim3(kKeysPerCta),
+             smem, st, a);
       break;
   }
   timing_after(st);

@@ -174,6 +174,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // scores and the histogram may still be read or cleared by the previous kernels
+  pdl_wait();
+  pdl_trigger();
   const uint32_t tmem = S.tmem_slot;
   const int U = S.prefix[p.Q];
   const int u0 = (int)(((int64_t)U * blockIdx.x) / gridDim.x);
@@ -453,9 +456,9 @@ cudaError_t launch_index_mxf4_tc(const IndexArgs& a, cudaStream_t st) {
                                        (int)smem);
   if (e != cudaSuccess) return e;
   timing_before(st);
-  k_index_mxf4_tc<<<grid, kThreads, smem, st>>>(mk, mks, mq, mqs, p);
+  e = launch(a.chained, k_index_mxf4_tc, dim3(grid), dim3(kThreads), smem, st, mk, mks, mq, mqs, p);
   timing_after(st);
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t index_mxf4_device_error(int* code) {

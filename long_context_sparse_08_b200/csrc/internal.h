@@ -8,6 +8,26 @@
 
 namespace csa {
 
+// Launch `kernel`; with `pdl` it may start before its predecessor in the stream ends (the
+// kernel calls pdl_wait() before it reads what a predecessor wrote).
+void count_launch();  // every kernel launch of the library goes through launch()
+template <typename... KArgs, typename... Args>
+cudaError_t launch(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                   cudaStream_t st, Args... args) {
+  count_launch();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 struct CompressArgs {
   int B, m, c, overlap, rope_dims, finalize;
   int64_t n_tok, first_entry, n_cap;
@@ -25,6 +45,8 @@ struct IndexArgs {
   const int64_t* q_pos;
   float* scores;  // [B, T, n_cap]
   int* hist;      // optional [B*T][4096] histogram of the scores' top 12 key bits (zeroed)
+  bool chained;   // the previous launch on the stream is a kernel of this library that has
+                  // waited for its own predecessors (the indexer may then start early)
 };
 // *hist_done: whether the launched kernel also filled a.hist
 cudaError_t launch_index_scores(const IndexArgs& a, cudaStream_t st, bool* hist_done = nullptr);
@@ -70,6 +92,7 @@ struct MqaArgs {
   const int64_t *q_pos, *win_pos0;
   const float* sink;
   void* out;
+  bool chained;  // as IndexArgs::chained (the attention may then prepare queries early)
 };
 size_t mqa_workspace_bytes(const MqaArgs& a);
 // tensor-core attention (bf16, c = 512, heads in groups of 64)

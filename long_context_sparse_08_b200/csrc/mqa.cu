@@ -213,12 +213,12 @@ cudaError_t launch_mqa(const MqaArgs& a, bool bf16, void* ws, size_t ws_bytes, c
     e = cudaFuncSetAttribute(k_mqa_cc<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
-    k_mqa_cc<__nv_bfloat16><<<grid, kThreads, smem, st>>>(a);
+    launch(false, k_mqa_cc<__nv_bfloat16>, dim3(grid), dim3(kThreads), smem, st, a);
   } else {
     e = cudaFuncSetAttribute(k_mqa_cc<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
-    k_mqa_cc<float><<<grid, kThreads, smem, st>>>(a);
+    launch(false, k_mqa_cc<float>, dim3(grid), dim3(kThreads), smem, st, a);
   }
   return cudaGetLastError();
 }

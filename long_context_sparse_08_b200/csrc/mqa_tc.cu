@@ -297,6 +297,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
       }
     }
 
+    // the selected rows, the partials and the output belong to the previous kernels
+    pdl_wait();
+    pdl_trigger();
     bool ok = true;
     const uint32_t kv_base = smem_u32(base + kOffKV);
     const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
@@ -525,6 +528,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
 
 // Merge the partials of each stream (fixed split order), add the sink, rotate by -t.
 __global__ void __launch_bounds__(256) k_mqa_combine(MqaTcParams P) {
+  pdl_wait();
+  pdl_trigger();
   const MqaArgs& a = P.a;
   const int stream = blockIdx.x, h = blockIdx.y;
   const int bt = stream / P.G, g = stream % P.G;
@@ -624,12 +629,10 @@ cudaError_t launch_mqa_tc(const MqaArgs& a, void* ws, size_t ws_bytes, cudaStrea
   cudaError_t e = cudaFuncSetAttribute(k_mqa_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  k_mqa_tc<<<(unsigned)(streams * P.nsplit), kThreads, smem, st>>>(P);
-  if (P.nsplit > 1) {
-    dim3 grid((unsigned)streams, kHg);
-    k_mqa_combine<<<grid, 256, 0, st>>>(P);
-  }
-  return cudaGetLastError();
+  e = launch(a.chained, k_mqa_tc, dim3((unsigned)(streams * P.nsplit)), dim3(kThreads), smem, st,
+             P);
+  if (e != cudaSuccess || P.nsplit == 1) return e;
+  return launch(true, k_mqa_combine, dim3((unsigned)streams, kHg), dim3(256), 0, st, P);
 }
 
 cudaError_t mqa_tc_device_error(int* code) {

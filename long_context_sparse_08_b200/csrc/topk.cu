@@ -165,7 +165,7 @@ cudaError_t launch_topk(const TopkArgs& a, void* ws, size_t ws_bytes, cudaStream
       return cudaErrorInvalidValue;
     return launch_topk_decode(topk_decode_args(a, ws), hist_ready, st);
   }
-  k_topk_rows<<<a.B * a.T, kThreads, 0, st>>>(a);
+  launch(false, k_topk_rows, dim3(a.B * a.T), dim3(kThreads), 0, st, a);
   return cudaGetLastError();
 }
 

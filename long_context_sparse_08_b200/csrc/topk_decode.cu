@@ -8,11 +8,14 @@
 //    into the tensor-core indexer's epilogue, or k_topk_hist here).
 // 2. k_topk_filter: every CTA loads its slice of the row, finds the bin T holding the k-th
 //    largest key, and appends the entries of bins > T to the "sure" list (fewer than k in
-//    all) and those of bin T to the "boundary" list, with one atomic per list per CTA. The
-//    last CTA of a query (atomic ticket) selects the remaining entries from the boundary
-//    list by an exact radix select on the 64-bit value (key << 32 | ~index), which is
-//    unique per entry, so ties resolve to the lower index, and sorts the winners. The
-//    result depends on the scores only.
+//    all) and those of bin T to the "boundary" list, with one atomic per list per CTA.
+// 3. k_topk_rank: every candidate (sure or boundary) is identified by the 64-bit value
+//    (key << 32 | ~index), unique per entry, larger = better (score desc, index asc). Its
+//    place in the result is the number of candidates with a larger value, counted by many
+//    CTAs per query, so no select or sort runs in one CTA; a candidate whose place is
+//    below min(k, n_vis) is written there. With more than 2048 boundary entries (heavy
+//    ties) one CTA per query instead radix-selects the boundary entries it needs and merge
+//    sorts the winners. Either way the result depends on the scores only.
 #include "common.cuh"
 #include "internal.h"
 
@@ -26,6 +29,9 @@ constexpr int kWarps = kFThreads / 32;
 constexpr int kBndCache = 2048;  // boundary entries kept in shared memory for the final pass
 constexpr int kDigitBits = 11;   // radix-select digit width
 constexpr int kDigits = 1 << kDigitBits;
+constexpr int kRankBnd = 2048;                 // boundary entries the rank path takes
+constexpr int kRankCand = kMaxTopk + kRankBnd;  // candidates per query, at most
+constexpr int kRankPerCta = 32;                // candidates ranked by one CTA
 
 __device__ __forceinline__ int64_t visible(const int64_t* q_pos, int q, int m, int64_t n_cap) {
   const int64_t t = q_pos[q];
@@ -37,79 +43,63 @@ __device__ __forceinline__ uint64_t sel_value(uint32_t key, uint32_t idx) {
   return ((uint64_t)key << 32) | (uint64_t)(0xffffffffu - idx);
 }
 
-// Ascending bitonic sort of arr[0..P) (P a power of two, 1024 or 2048), with kFThreads
-// threads. Thread t keeps elements E*t .. E*t+E-1 in registers; exchanges at distance < E
-// stay inside a thread, those below 32*E go through warp shuffles, and only the wider ones
-// through shared memory (one barrier each). Leaves the sorted values in arr.
+// Ascending merge sort of arr[0..P), P = E * kFThreads, with `tmp` (P entries) as the
+// second buffer; returns the buffer holding the result. Each thread first sorts E elements
+// in registers (odd-even transposition), then every level merges pairs of sorted runs:
+// thread t writes outputs E*t .. E*t+E-1 of its pair, locating its start by a binary
+// search along the merge path (ties go to the left run, so equal values are handled).
+// About log2(P/E) barriers in all: the latency of a long network of dependent
+// compare-exchange stages is what this replaces.
 template <int E>
-__device__ void bitonic_sort_regs(uint64_t* arr) {
+__device__ uint64_t* merge_sort(uint64_t* arr, uint64_t* tmp) {
   constexpr int P = E * kFThreads;
   const int tid = threadIdx.x;
-  uint64_t x[E];
+  {
+    uint64_t x[E];
 #pragma unroll
-  for (int e = 0; e < E; ++e) x[e] = arr[E * tid + e];
-  bool in_regs = true;
-#pragma unroll 1
-  for (int size = 2; size <= P; size <<= 1) {
-#pragma unroll 1
-    for (int s = size >> 1; s > 0; s >>= 1) {
-      if (s >= 32 * E) {  // partner in another warp
-        if (in_regs) {
+    for (int e = 0; e < E; ++e) x[e] = arr[E * tid + e];
 #pragma unroll
-          for (int e = 0; e < E; ++e) arr[E * tid + e] = x[e];
-          __syncthreads();
-          in_regs = false;
-        }
-        for (int i = tid; i < (P >> 1); i += kFThreads) {
-          const int lo = 2 * i - (i & (s - 1)), hi = lo + s;
-          const bool asc = (lo & size) == 0;
-          const uint64_t u = arr[lo], v = arr[hi];
-          if ((u > v) == asc) {
-            arr[lo] = v;
-            arr[hi] = u;
-          }
-        }
-        __syncthreads();
-        continue;
-      }
-      if (!in_regs) {
+    for (int round = 0; round < E; ++round) {
 #pragma unroll
-        for (int e = 0; e < E; ++e) x[e] = arr[E * tid + e];
-        in_regs = true;
-      }
-      if (s >= E) {  // partner element i ^ s sits in lane ^ (s / E), same slot
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          const int i = E * tid + e;
-          const uint64_t y = __shfl_xor_sync(0xffffffffu, x[e], s / E);
-          const bool asc = (i & size) == 0, lo = (i & s) == 0;
-          const bool take_min = asc == lo;
-          x[e] = take_min ? (x[e] < y ? x[e] : y) : (x[e] < y ? y : x[e]);
-        }
-      } else {  // partner inside this thread (s = E/2 .. 1; indices stay compile-time)
-#pragma unroll
-        for (int sc = E / 2; sc > 0; sc >>= 1) {
-          if (sc != s) continue;
-#pragma unroll
-          for (int e = 0; e < E; ++e) {
-            if ((e & sc) == 0) {
-              const bool asc = ((E * tid + e) & size) == 0;
-              const uint64_t u = x[e], v = x[e + sc];
-              if ((u > v) == asc) {
-                x[e] = v;
-                x[e + sc] = u;
-              }
-            }
-          }
-        }
+      for (int e = round & 1; e + 1 < E; e += 2) {
+        const uint64_t u = x[e], v = x[e + 1];
+        x[e] = u < v ? u : v;
+        x[e + 1] = u < v ? v : u;
       }
     }
-  }
-  if (in_regs) {  // each thread stores back the slots it loaded: no cross-thread hazard
 #pragma unroll
     for (int e = 0; e < E; ++e) arr[E * tid + e] = x[e];
   }
   __syncthreads();
+  uint64_t* src = arr;
+  uint64_t* dst = tmp;
+#pragma unroll 1
+  for (int L = E; L < P; L <<= 1) {
+    const int out0 = E * tid;
+    const int base = out0 & ~(2 * L - 1);
+    const int d = out0 - base;  // outputs of the merged pair before this thread's first
+    const uint64_t* A = src + base;
+    const uint64_t* B = A + L;
+    int lo = d > L ? d - L : 0, hi = d < L ? d : L;
+    while (lo < hi) {  // i = how many of the first d outputs come from A
+      const int mid = (lo + hi) >> 1;
+      if (A[mid] <= B[d - mid - 1]) lo = mid + 1; else hi = mid;
+    }
+    int i = lo, j = d - lo;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const uint64_t av = i < L ? A[i] : ~0ull, bv = j < L ? B[j] : ~0ull;
+      const bool take_a = j >= L || (i < L && av <= bv);
+      dst[out0 + e] = take_a ? av : bv;
+      i += take_a;
+      j += !take_a;
+    }
+    __syncthreads();
+    uint64_t* t = src;
+    src = dst;
+    dst = t;
+  }
+  return src;
 }
 
 __global__ void __launch_bounds__(kFThreads) k_topk_hist(TopkDecodeArgs a) {
@@ -164,20 +154,24 @@ __device__ __forceinline__ void block_scan2(int c0, int c1, int* ws, int* o0, in
   __syncthreads();
 }
 
+// zero n4 int4 words (the histogram and counters of a call), in stream order
+__global__ void __launch_bounds__(256) k_zero(int4* p, int n4) {
+  pdl_wait();
+  pdl_trigger();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += gridDim.x * blockDim.x)
+    p[i] = make_int4(0, 0, 0, 0);
+}
+
 __global__ void __launch_bounds__(kFThreads, 2) k_topk_filter(TopkDecodeArgs a) {
-  __shared__ __align__(16) uint64_t bcache[kBndCache];
-  __shared__ uint64_t pairs[kMaxTopk];
-  __shared__ int dh[kDigits];
   __shared__ int wsum[2 * kWarps];
-  __shared__ int s_bin, s_last, s_base_s, s_base_b;
-  __shared__ uint32_t s_digit;
-  __shared__ int s_dabove, s_fill, s_fill_exact;
+  __shared__ int s_bin, s_base_s, s_base_b;
+  pdl_wait();
+  pdl_trigger();
   const int q = blockIdx.y, tid = threadIdx.x;
   const int nslice = gridDim.x;
   const int64_t n = visible(a.q_pos, q, a.m, a.n_cap);
   const int k = a.k;
-  const int nsel = (int)(n < k ? n : k);
-  int* cnt = a.cnt + 4 * q;  // sure count, boundary count, ticket
+  int* cnt = a.cnt + 4 * q;  // sure count, boundary count
   uint64_t* sure = a.list + (size_t)q * (a.n_cap + k);
   uint64_t* bnd = sure + k;
 
@@ -264,48 +258,83 @@ __global__ void __launch_bounds__(kFThreads, 2) k_topk_filter(TopkDecodeArgs a) 
     __syncthreads();  // s_base_* are reused by the next batch
   }
 
-  // ---- the last CTA of this query finishes the selection ----
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    s_last = atomicAdd(&cnt[2], 1) == nslice - 1;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
+}
+
+__global__ void __launch_bounds__(kFThreads) k_topk_rank(TopkDecodeArgs a) {
+  __shared__ __align__(16) uint64_t cand[kRankCand];  // the fallback uses it as pairs + bcache
+  __shared__ int dh[kDigits];
+  __shared__ int wsum[2 * kWarps];
+  __shared__ int part[kWarps][kRankPerCta];
+  __shared__ uint32_t s_digit;
+  __shared__ int s_dabove, s_fill, s_fill_exact;
+  pdl_wait();
+  pdl_trigger();
+  uint64_t* pairs = cand;
+  uint64_t* bcache = cand + kMaxTopk;
+  const int q = blockIdx.y, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int64_t n = visible(a.q_pos, q, a.m, a.n_cap);
+  const int k = a.k;
+  const int nsel = (int)(n < k ? n : k);
+  const int* cnt = a.cnt + 4 * q;
+  const uint64_t* sure = a.list + (size_t)q * (a.n_cap + k);
+  const uint64_t* bnd = sure + k;
+  int32_t* out = a.out_idx + (size_t)q * k;
   const int ns = min(__ldcg(&cnt[0]), k);
   const int nb = (int)min((int64_t)__ldcg(&cnt[1]), a.n_cap);
+
+  if (nb <= kRankBnd) {
+    // ---- rank path: place = #candidates with a larger value ----
+    const int C = ns + nb;
+    const int c0 = blockIdx.x * kRankPerCta;
+    if (blockIdx.x == 0)
+      for (int i = nsel + tid; i < k; i += kFThreads) out[i] = -1;
+    if (c0 >= C) return;
+    constexpr int kLoads = kRankCand / kFThreads;
+    uint64_t v[kLoads];
+#pragma unroll
+    for (int j = 0; j < kLoads; ++j) {
+      const int c = tid + j * kFThreads;
+      v[j] = c < ns ? __ldcg(&sure[c]) : (c < C ? __ldcg(&bnd[c - ns]) : 0ull);
+    }
+#pragma unroll
+    for (int j = 0; j < kLoads; ++j) {
+      const int c = tid + j * kFThreads;
+      if (c < C) cand[c] = v[j];
+    }
+    __syncthreads();
+    // lane = candidate of this CTA, warp = a range of the others (broadcast reads)
+    const int ci = c0 + lane;
+    const uint64_t x = ci < C ? cand[ci] : ~0ull;
+    const int j0 = (int)((int64_t)C * wid / kWarps), j1 = (int)((int64_t)C * (wid + 1) / kWarps);
+    int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
+    int j = j0;
+    for (; j + 4 <= j1; j += 4) {
+      r0 += cand[j] > x;
+      r1 += cand[j + 1] > x;
+      r2 += cand[j + 2] > x;
+      r3 += cand[j + 3] > x;
+    }
+    for (; j < j1; ++j) r0 += cand[j] > x;
+    part[wid][lane] = (r0 + r1) + (r2 + r3);
+    __syncthreads();
+    if (wid == 0 && ci < C) {
+      int rank = 0;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) rank += part[w][lane];
+      if (rank < nsel) out[rank] = (int32_t)(0xffffffffu - (uint32_t)(x & 0xffffffffu));
+    }
+    return;
+  }
+
+  // ---- heavy ties (many boundary entries): one CTA selects and sorts ----
+  if (blockIdx.x != 0) return;
+  const int T = (int)(__ldcg(&bnd[0]) >> 52);  // every boundary value shares bin T
   int kk = nsel - ns;  // still to take from the boundary list
   if (kk < 0) kk = 0;
   if (kk > nb) kk = nb;
-  const bool cached = nb <= kBndCache;
-  {  // both lists into shared memory, all loads issued before the stores
-    constexpr int kS = kMaxTopk / kFThreads, kB = kBndCache / kFThreads;
-    uint64_t sv[kS], bv[kB];
-#pragma unroll
-    for (int j = 0; j < kS; ++j) {
-      const int e = tid + j * kFThreads;
-      sv[j] = e < ns ? __ldcg(&sure[e]) : 0ull;
-    }
-#pragma unroll
-    for (int j = 0; j < kB; ++j) {
-      const int e = tid + j * kFThreads;
-      bv[j] = (kk > 0 && cached && e < nb) ? __ldcg(&bnd[e]) : 0ull;
-    }
-#pragma unroll
-    for (int j = 0; j < kS; ++j) {
-      const int e = tid + j * kFThreads;
-      if (e < ns) pairs[e] = ~sv[j];
-    }
-#pragma unroll
-    for (int j = 0; j < kB; ++j) {
-      const int e = tid + j * kFThreads;
-      if (kk > 0 && cached && e < nb) bcache[e] = bv[j];
-    }
-  }
+  for (int i = tid; i < ns; i += kFThreads) pairs[i] = ~__ldcg(&sure[i]);
   if (tid == 0) s_fill = ns;
   __syncthreads();
-  const uint64_t* L = cached ? bcache : bnd;
   if (kk > 0) {
     uint64_t thr = 0;  // take every boundary value >= thr
     if (kk < nb) {
@@ -320,7 +349,7 @@ __global__ void __launch_bounds__(kFThreads, 2) k_topk_filter(TopkDecodeArgs a) 
         if (tid == 0) s_fill_exact = 0;
         __syncthreads();
         for (int i = tid; i < nb; i += kFThreads) {
-          const uint64_t v = cached ? L[i] : __ldcg(&L[i]);
+          const uint64_t v = __ldcg(&bnd[i]);
           if ((v & mask) == prefix) atomicAdd(&dh[(v >> shift) & dmask], 1);
         }
         __syncthreads();
@@ -356,7 +385,7 @@ __global__ void __launch_bounds__(kFThreads, 2) k_topk_filter(TopkDecodeArgs a) 
       thr = prefix;
     }
     for (int i = tid; i < nb; i += kFThreads) {
-      const uint64_t v = cached ? L[i] : __ldcg(&L[i]);
+      const uint64_t v = __ldcg(&bnd[i]);
       if (v >= thr) {
         const int pos = atomicAdd(&s_fill, 1);
         if (pos < kMaxTopk) pairs[pos] = ~v;
@@ -368,15 +397,12 @@ __global__ void __launch_bounds__(kFThreads, 2) k_topk_filter(TopkDecodeArgs a) 
   const int P = k <= kMaxTopk / 4 ? kMaxTopk / 4 : (k <= kMaxTopk / 2 ? kMaxTopk / 2 : kMaxTopk);
   for (int i = filled + tid; i < P; i += kFThreads) pairs[i] = ~0ull;
   __syncthreads();
-  if (P == kMaxTopk)
-    bitonic_sort_regs<kMaxTopk / kFThreads>(pairs);
-  else if (P == kMaxTopk / 2)
-    bitonic_sort_regs<kMaxTopk / 2 / kFThreads>(pairs);
-  else
-    bitonic_sort_regs<kMaxTopk / 4 / kFThreads>(pairs);
-  int32_t* out = a.out_idx + (size_t)q * k;
+  // bcache is free now: it is the merge sort's second buffer
+  const uint64_t* sorted = P == kMaxTopk       ? merge_sort<kMaxTopk / kFThreads>(pairs, bcache)
+                           : P == kMaxTopk / 2 ? merge_sort<kMaxTopk / 2 / kFThreads>(pairs, bcache)
+                                               : merge_sort<kMaxTopk / 4 / kFThreads>(pairs, bcache);
   for (int i = tid; i < k; i += kFThreads)
-    out[i] = i < filled ? (int32_t)(pairs[i] & 0xffffffffu) : -1;
+    out[i] = i < filled ? (int32_t)(sorted[i] & 0xffffffffu) : -1;
 }
 
 }  // namespace
@@ -409,7 +435,9 @@ TopkDecodeArgs topk_decode_args(const TopkArgs& t, void* ws) {
 cudaError_t topk_decode_clear(const TopkDecodeArgs& a, cudaStream_t st) {
   // hist and the counters are adjacent at the start of the workspace
   const size_t bytes = rup((size_t)a.Q * kBins * 4) + rup((size_t)a.Q * 16);
-  return cudaMemsetAsync(a.hist, 0, bytes, st);
+  const int n4 = (int)(bytes / 16);
+  return launch(true, k_zero, dim3((n4 + 255) / 256), dim3(256), 0, st,
+                reinterpret_cast<int4*>(a.hist), n4);
 }
 
 cudaError_t launch_topk_decode(TopkDecodeArgs a, bool hist_ready, cudaStream_t st) {
@@ -420,12 +448,15 @@ cudaError_t launch_topk_decode(TopkDecodeArgs a, bool hist_ready, cudaStream_t s
   if (slices < 1) slices = 1;
   a.nslice = slices;
   if (!hist_ready) {
-    cudaError_t e = topk_decode_clear(a, st);
+    const cudaError_t e = topk_decode_clear(a, st);
     if (e != cudaSuccess) return e;
-    k_topk_hist<<<dim3(slices, a.Q), kFThreads, 0, st>>>(a);
+    const cudaError_t eh = launch(false, k_topk_hist, dim3(slices, a.Q), dim3(kFThreads), 0, st, a);
+    if (eh != cudaSuccess) return eh;
   }
-  k_topk_filter<<<dim3(slices, a.Q), kFThreads, 0, st>>>(a);
-  return cudaGetLastError();
+  cudaError_t e = launch(true, k_topk_filter, dim3(slices, a.Q), dim3(kFThreads), 0, st, a);
+  if (e != cudaSuccess) return e;
+  const int rank_ctas = (a.k + kRankBnd + kRankPerCta - 1) / kRankPerCta;
+  return launch(true, k_topk_rank, dim3(rank_ctas, a.Q), dim3(kFThreads), 0, st, a);
 }
 
 }  // namespace csa
