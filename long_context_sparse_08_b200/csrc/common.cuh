@@ -103,9 +103,10 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
 // two-part 2*pi (Cody-Waite); the reduced angle (|a| <= pi) then goes through fp32
 // sincosf. Error ~1e-10 rad before the fp32 evaluation, which adds ~1 ulp.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void rope_cos_sin(double pos, int p, int r, double base, float* cs,
-                                             float* sn) {
-  const double inv_freq = exp2(-2.0 * (double)p / (double)r * log2(base));
+__host__ __device__ inline double rope_inv_freq(int p, int r, double base) {
+  return exp2(-2.0 * (double)p / (double)r * log2(base));
+}
+__device__ __forceinline__ void rope_angle_cs(double pos, double inv_freq, float* cs, float* sn) {
   const double x = pos * inv_freq;
   const double kTwoPiHi = 6.283185307179586232;     // nearest double to 2*pi
   const double kTwoPiLo = 2.4492935982947064e-16;   // 2*pi - kTwoPiHi
@@ -113,6 +114,10 @@ __device__ __forceinline__ void rope_cos_sin(double pos, int p, int r, double ba
   double red = fma(-k, kTwoPiHi, x);
   red = fma(-k, kTwoPiLo, red);
   sincosf((float)red, sn, cs);
+}
+__device__ __forceinline__ void rope_cos_sin(double pos, int p, int r, double base, float* cs,
+                                             float* sn) {
+  rope_angle_cs(pos, rope_inv_freq(p, r, base), cs, sn);
 }
 
 }  // namespace csa

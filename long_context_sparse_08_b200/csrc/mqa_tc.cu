@@ -34,6 +34,7 @@ constexpr int kHg = 64;          // heads per CTA (MMA N)
 constexpr int kThreads = 160;    // warps 0-3: loads + softmax + epilogue; warp 4: MMA
 constexpr int kAtoms = kC / 64;  // 64-element (128 B) swizzle atoms along a row
 constexpr float kLazy = 8.f;     // rescale threshold (natural-log units)
+constexpr int kMaxPairs = 256;   // RoPE pairs (r / 2)
 
 // shared memory (offsets from a 1024-aligned base)
 constexpr int kOffKV = 0;                                // [atom][row][128 B]  128 KB
@@ -54,7 +55,8 @@ struct Smem {
   int any_rescale;
   float red[4][kHg], red2[4][kHg];
   float m_used[kHg], l_sum[kHg], alpha[kHg], fin[kHg];
-  float cs[256], sn[256];  // RoPE table for pairs of the last r dims
+  float cs[kMaxPairs], sn[kMaxPairs];  // RoPE table for pairs of the last r dims
+  float wq[kC];                         // query RMSNorm weights
   const __nv_bfloat16* src[kRows];  // source rows of the current chunk (nullptr: masked)
 };
 
@@ -63,6 +65,7 @@ struct MqaTcParams {
   int G;       // head groups (H / 64)
   int nsplit;  // CTAs per stream
   float* part; // partials [stream][split][64 * (kC + 2)] or nullptr
+  double inv_freq[kMaxPairs];  // RoPE pair frequencies base^(-2p/r), formed once on the host
 };
 
 __device__ __forceinline__ void bar_softmax() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
@@ -226,9 +229,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
                                                      ((size_t)bt * a.H + h0) * kC);
 #pragma unroll 4
     for (int i = tid; i < kHg * kC / 8; i += 128) cp_async16(stage + 16 * i, qg + i, true);
-    // RoPE table and running stats while the copies are in flight
+    // RoPE table, norm weights and running stats while the copies are in flight
     for (int p = tid; p < r / 2; p += 128)
-      rope_cos_sin((double)rl.t, p, r, (double)a.rope_base, &S.cs[p], &S.sn[p]);
+      rope_angle_cs((double)rl.t, P.inv_freq[p], &S.cs[p], &S.sn[p]);
+    for (int d = tid; d < kC; d += 128)
+      S.wq[d] = a.q_rms_w ? __bfloat162float(static_cast<const __nv_bfloat16*>(a.q_rms_w)[d]) : 1.f;
     if (tid < kHg) {
       S.m_used[tid] = -INFINITY;
       S.l_sum[tid] = 0.f;
@@ -240,61 +245,58 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
   const uint32_t tmem = S.tmem_slot;
 
   if (warp < 4) {
-    // ---- q_hat = RoPE_t(RMSNorm(q)) in bf16, one warp per head (lane = 16 dims) ----
+    // ---- q_hat = RoPE_t(RMSNorm(q)) in bf16: two threads per head, 256 dims each. Thread
+    //      t reads its 32 chunks of 8 dims starting at chunk t % 32, so that a warp's reads
+    //      of one step spread over all banks. ----
     uint8_t* qs = base + kOffQ;
-    float wq[16];  // RMSNorm weights of this lane's dims (the same for every head)
-#pragma unroll
-    for (int half = 0; half < 2; ++half)
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        wq[8 * half + k] = a.q_rms_w ? __bfloat162float(static_cast<const __nv_bfloat16*>(
-                                           a.q_rms_w)[8 * (lane + 32 * half) + k])
-                                     : 1.f;
+    const int qh = tid >> 1, qhalf = tid & 1;
+    const uint4* qrow = reinterpret_cast<const uint4*>(base + kOffKV + qh * (kC * 2)) + 32 * qhalf;
     cp_async_wait_all();
     bar_softmax();
-#pragma unroll 1
-    for (int h = warp; h < kHg; h += 4) {
-      const uint4* qrow = reinterpret_cast<const uint4*>(base + kOffKV + h * (kC * 2));
-      float x[16];
-      float ss = 0.f;
+    float ss0 = 0.f, ss1 = 0.f;
+#pragma unroll 8
+    for (int i = 0; i < 32; ++i) {
+      const uint4 raw = qrow[(i + lane) & 31];
+      const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const uint4 raw = qrow[lane + 32 * half];
-        const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+      for (int k = 0; k < 4; ++k) {
+        const float lo = __uint_as_float(w4[k] << 16), hi = __uint_as_float(w4[k] & 0xffff0000u);
+        ss0 = fmaf(lo, lo, ss0);
+        ss1 = fmaf(hi, hi, ss1);
+      }
+    }
+    float ss = ss0 + ss1;
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    const float rstd = rsqrtf(ss / (float)kC + a.eps);
+#pragma unroll 4
+    for (int i = 0; i < 32; ++i) {
+      const int c = (i + lane) & 31;
+      const uint4 raw = qrow[c];
+      const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+      const int d0 = 256 * qhalf + 8 * c;
+      float y[8];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        y[2 * k] = __uint_as_float(w4[k] << 16) * rstd * S.wq[d0 + 2 * k];
+        y[2 * k + 1] = __uint_as_float(w4[k] & 0xffff0000u) * rstd * S.wq[d0 + 2 * k + 1];
+      }
+      if (d0 >= r0) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          x[8 * half + 2 * k] = __uint_as_float(w4[k] << 16);
-          x[8 * half + 2 * k + 1] = __uint_as_float(w4[k] & 0xffff0000u);
+          const int p = (d0 + 2 * k - r0) >> 1;
+          const float cs = S.cs[p], sn = S.sn[p], u = y[2 * k], v = y[2 * k + 1];
+          y[2 * k] = u * cs - v * sn;
+          y[2 * k + 1] = u * sn + v * cs;
         }
       }
+      uint4 o;
+      uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
-      for (int k = 0; k < 16; ++k) ss = fmaf(x[k], x[k], ss);
-      ss = warp_sum(ss);
-      const float rstd = rsqrtf(ss / (float)kC + a.eps);
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int d0 = 8 * (lane + 32 * half);
-        float y[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) y[k] = x[8 * half + k] * rstd * wq[8 * half + k];
-        if (d0 >= r0) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int p = (d0 + 2 * k - r0) >> 1;
-            const float c = S.cs[p], sn = S.sn[p], u = y[2 * k], v = y[2 * k + 1];
-            y[2 * k] = u * c - v * sn;
-            y[2 * k + 1] = u * sn + v * c;
-          }
-        }
-        uint4 o;
-        uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          ow[k] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * k])) |
-                  ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * k + 1])) << 16);
-        const int atom = d0 >> 6, chunk = (d0 & 63) >> 3;
-        *reinterpret_cast<uint4*>(qs + atom * (kHg * 128) + sw128(h, chunk)) = o;
-      }
+      for (int k = 0; k < 4; ++k)
+        ow[k] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * k])) |
+                ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * k + 1])) << 16);
+      const int atom = d0 >> 6, chunk = (d0 & 63) >> 3;
+      *reinterpret_cast<uint4*>(qs + atom * (kHg * 128) + sw128(qh, chunk)) = o;
     }
 
     // the selected rows, the partials and the output belong to the previous kernels
@@ -538,6 +540,7 @@ __global__ void __launch_bounds__(256) k_mqa_combine(MqaTcParams P) {
   const size_t stride = kHg * (kC + 2);
   const float* base = P.part + (size_t)stream * P.nsplit * stride;
   constexpr int kMaxSplit = 32;  // choose_nsplit never exceeds this
+  constexpr int kGroup = 8;      // splits whose partial rows are loaded together
   float ms[kMaxSplit];
   float M = -INFINITY;
 #pragma unroll
@@ -550,14 +553,28 @@ __global__ void __launch_bounds__(256) k_mqa_combine(MqaTcParams P) {
   float l = 0.f, o0 = 0.f, o1 = 0.f;
   const int d = 2 * tid;
 #pragma unroll
-  for (int sp = 0; sp < kMaxSplit; ++sp) {
-    if (sp < P.nsplit && ms[sp] != -INFINITY) {
+  for (int s0 = 0; s0 < kMaxSplit; s0 += kGroup) {
+    if (s0 >= P.nsplit) break;
+    float lv[kGroup];
+    float2 ov[kGroup];
+#pragma unroll
+    for (int j = 0; j < kGroup; ++j) {  // every load of the group in flight at once
+      const int sp = s0 + j;
+      const bool use = sp < P.nsplit && ms[sp] != -INFINITY;
       const float* pp = base + sp * stride;
-      const float f = expf(ms[sp] - Mt);
-      l = fmaf(pp[kHg + h], f, l);
-      const float2 ov = *reinterpret_cast<const float2*>(pp + 2 * kHg + (size_t)h * kC + d);
-      o0 = fmaf(ov.x, f, o0);
-      o1 = fmaf(ov.y, f, o1);
+      lv[j] = use ? pp[kHg + h] : 0.f;
+      ov[j] = use ? *reinterpret_cast<const float2*>(pp + 2 * kHg + (size_t)h * kC + d)
+                  : make_float2(0.f, 0.f);
+    }
+#pragma unroll
+    for (int j = 0; j < kGroup; ++j) {  // fixed split order: deterministic
+      const int sp = s0 + j;
+      if (sp < P.nsplit && ms[sp] != -INFINITY) {
+        const float f = expf(ms[sp] - Mt);
+        l = fmaf(lv[j], f, l);
+        o0 = fmaf(ov[j].x, f, o0);
+        o1 = fmaf(ov[j].y, f, o1);
+      }
     }
   }
   float y0 = 0.f, y1 = 0.f;
@@ -569,7 +586,7 @@ __global__ void __launch_bounds__(256) k_mqa_combine(MqaTcParams P) {
   const int r = a.rope_dims, r0 = kC - r;
   if (d >= r0) {
     float cs, sn;
-    rope_cos_sin(-(double)t, (d - r0) >> 1, r, (double)a.rope_base, &cs, &sn);
+    rope_angle_cs(-(double)t, P.inv_freq[(d - r0) >> 1], &cs, &sn);
     const float u0 = y0 * cs - y1 * sn, u1 = y0 * sn + y1 * cs;
     y0 = u0;
     y1 = u1;
@@ -623,6 +640,8 @@ cudaError_t launch_mqa_tc(const MqaArgs& a, void* ws, size_t ws_bytes, cudaStrea
   P.G = a.H / kHg;
   P.nsplit = choose_nsplit(a);
   P.part = P.nsplit > 1 ? static_cast<float*>(ws) : nullptr;
+  for (int p = 0; p < kMaxPairs; ++p)
+    P.inv_freq[p] = p < a.rope_dims / 2 ? rope_inv_freq(p, a.rope_dims, (double)a.rope_base) : 0.0;
   if (P.nsplit > 1 && ws_bytes < mqa_tc_workspace_bytes(a)) return cudaErrorInvalidValue;
   const int64_t streams = (int64_t)a.B * a.T * P.G;
   const size_t smem = 1024 + kOffEnd + sizeof(Smem);

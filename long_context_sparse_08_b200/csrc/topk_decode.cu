@@ -11,9 +11,10 @@
 //    all) and those of bin T to the "boundary" list, with one atomic per list per CTA.
 // 3. k_topk_rank: every candidate (sure or boundary) is identified by the 64-bit value
 //    (key << 32 | ~index), unique per entry, larger = better (score desc, index asc). Its
-//    place in the result is the number of candidates with a larger value, counted by many
-//    CTAs per query, so no select or sort runs in one CTA; a candidate whose place is
-//    below min(k, n_vis) is written there. With more than 2048 boundary entries (heavy
+//    place in the result is the number of candidates with a larger value (for a boundary
+//    entry: ns + those in the boundary list), counted by many CTAs per query, so no select
+//    or sort runs in one CTA; a candidate whose place is below min(k, n_vis) is written
+//    there. With more than 2048 boundary entries (heavy
 //    ties) one CTA per query instead radix-selects the boundary entries it needs and merge
 //    sorts the winners. Either way the result depends on the scores only.
 #include "common.cuh"
@@ -30,7 +31,6 @@ constexpr int kBndCache = 2048;  // boundary entries kept in shared memory for t
 constexpr int kDigitBits = 11;   // radix-select digit width
 constexpr int kDigits = 1 << kDigitBits;
 constexpr int kRankBnd = 2048;                 // boundary entries the rank path takes
-constexpr int kRankCand = kMaxTopk + kRankBnd;  // candidates per query, at most
 constexpr int kRankPerCta = 32;                // candidates ranked by one CTA
 
 __device__ __forceinline__ int64_t visible(const int64_t* q_pos, int q, int m, int64_t n_cap) {
@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(kFThreads, 2) k_topk_filter(TopkDecodeArgs a) 
 }
 
 __global__ void __launch_bounds__(kFThreads) k_topk_rank(TopkDecodeArgs a) {
-  __shared__ __align__(16) uint64_t cand[kRankCand];  // the fallback uses it as pairs + bcache
+  __shared__ __align__(16) uint64_t cand[kMaxTopk + kRankBnd];  // fallback: pairs + bcache
   __shared__ int dh[kDigits];
   __shared__ int wsum[2 * kWarps];
   __shared__ int part[kWarps][kRankPerCta];
@@ -283,18 +283,24 @@ __global__ void __launch_bounds__(kFThreads) k_topk_rank(TopkDecodeArgs a) {
   const int nb = (int)min((int64_t)__ldcg(&cnt[1]), a.n_cap);
 
   if (nb <= kRankBnd) {
-    // ---- rank path: place = #candidates with a larger value ----
-    const int C = ns + nb;
-    const int c0 = blockIdx.x * kRankPerCta;
+    // ---- rank path: every sure value is above every boundary value, so a sure entry's
+    //      place is its rank among the sure entries and a boundary entry's is ns + its
+    //      rank among the boundary entries; CTAs take 32 entries of one list each ----
+    const int cs = (ns + kRankPerCta - 1) / kRankPerCta;
     if (blockIdx.x == 0)
       for (int i = nsel + tid; i < k; i += kFThreads) out[i] = -1;
+    const bool in_sure = (int)blockIdx.x < cs;
+    const int C = in_sure ? ns : nb;
+    const int c0 = (in_sure ? blockIdx.x : blockIdx.x - cs) * kRankPerCta;
     if (c0 >= C) return;
-    constexpr int kLoads = kRankCand / kFThreads;
+    const uint64_t* list = in_sure ? sure : bnd;
+    const int place0 = in_sure ? 0 : ns;
+    constexpr int kLoads = kRankBnd / kFThreads;
     uint64_t v[kLoads];
 #pragma unroll
     for (int j = 0; j < kLoads; ++j) {
       const int c = tid + j * kFThreads;
-      v[j] = c < ns ? __ldcg(&sure[c]) : (c < C ? __ldcg(&bnd[c - ns]) : 0ull);
+      v[j] = c < C ? __ldcg(&list[c]) : 0ull;
     }
 #pragma unroll
     for (int j = 0; j < kLoads; ++j) {
@@ -302,7 +308,7 @@ __global__ void __launch_bounds__(kFThreads) k_topk_rank(TopkDecodeArgs a) {
       if (c < C) cand[c] = v[j];
     }
     __syncthreads();
-    // lane = candidate of this CTA, warp = a range of the others (broadcast reads)
+    // lane = entry of this CTA, warp = a range of the list (broadcast reads)
     const int ci = c0 + lane;
     const uint64_t x = ci < C ? cand[ci] : ~0ull;
     const int j0 = (int)((int64_t)C * wid / kWarps), j1 = (int)((int64_t)C * (wid + 1) / kWarps);
@@ -318,7 +324,7 @@ __global__ void __launch_bounds__(kFThreads) k_topk_rank(TopkDecodeArgs a) {
     part[wid][lane] = (r0 + r1) + (r2 + r3);
     __syncthreads();
     if (wid == 0 && ci < C) {
-      int rank = 0;
+      int rank = place0;
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) rank += part[w][lane];
       if (rank < nsel) out[rank] = (int32_t)(0xffffffffu - (uint32_t)(x & 0xffffffffu));
@@ -455,7 +461,8 @@ cudaError_t launch_topk_decode(TopkDecodeArgs a, bool hist_ready, cudaStream_t s
   }
   cudaError_t e = launch(true, k_topk_filter, dim3(slices, a.Q), dim3(kFThreads), 0, st, a);
   if (e != cudaSuccess) return e;
-  const int rank_ctas = (a.k + kRankBnd + kRankPerCta - 1) / kRankPerCta;
+  // enough CTAs for the sure list (< k) and the boundary list (<= kRankBnd) apart
+  const int rank_ctas = (a.k + kRankPerCta - 1) / kRankPerCta + kRankBnd / kRankPerCta;
   return launch(true, k_topk_rank, dim3(rank_ctas, a.Q), dim3(kFThreads), 0, st, a);
 }
 
