@@ -171,6 +171,19 @@ csa_status check_index_args(const csa_params* p, csa_dtype kdt, int32_t B, int32
   return CSA_OK;
 }
 
+// csa_forward with the decode selector and the tensor-core attention: the selector also
+// prepares the attention's q_hat (bf16 [B*T][H][c]) in the workspace
+bool forward_qhat(const csa_params* p, int32_t B, int32_t T, int64_t N_cap) {
+  csa::MqaArgs m = make_mqa(p, B, T, nullptr, nullptr, nullptr, N_cap, nullptr, p->topk, nullptr,
+                            0, nullptr, nullptr, nullptr, nullptr);
+  return csa::topk_decode_path(B, T, N_cap, p->topk) && csa::mqa_tc_supported(m, true);
+}
+size_t qhat_bytes(const csa_params* p, int32_t B, int32_t T, int64_t N_cap) {
+  return forward_qhat(p, B, T, N_cap)
+             ? round_up((size_t)B * T * (size_t)p->n_heads * (size_t)p->c * 2)
+             : 0;
+}
+
 csa::IndexArgs make_index(const csa_params* p, csa_dtype kdt, int32_t B, int32_t T,
                           int64_t N_cap, const void* qI, const void* qI_scale, const float* w,
                           const void* KI, const void* KI_scale, const int64_t* q_pos,
@@ -278,7 +291,8 @@ size_t csa_workspace_size(const csa_params* p, int32_t entry, csa_dtype kdt, int
       m.k = 0;
       return round_up(csa::mqa_workspace_bytes(m));
     case CSA_WS_FORWARD:
-      return scores_bytes(B, T, N_cap) + topk_ws + round_up(csa::mqa_workspace_bytes(m));
+      return scores_bytes(B, T, N_cap) + topk_ws + round_up(csa::mqa_workspace_bytes(m)) +
+             qhat_bytes(p, B, T, N_cap);
     default:
       fail(CSA_ERR_INVALID_ARG, "unknown workspace entry %d", entry);
       return 0;
@@ -446,16 +460,26 @@ csa_status csa_forward(const csa_params* p, csa_dtype io, int32_t B, int32_t T,
   const size_t sb = scores_bytes(B, T, a->N_cap);
   const size_t tb = round_up(csa::topk_workspace_bytes(B, T, a->N_cap, p->topk));
   float* scores = a->out_scores ? a->out_scores : reinterpret_cast<float*>(base);
-  csa::TopkArgs t{};
-  t.B = B; t.T = T; t.m = p->m; t.k = p->topk; t.n_cap = a->N_cap; t.scores = scores;
-  t.q_pos = a->q_pos; t.out_idx = a->out_idx;
-  TRY(index_then_topk(p, a->idx_dtype, B, T, a->N_cap, a->qI, a->qI_scale, a->w, a->KI,
-                      a->KI_scale, a->q_pos, scores, t, base + sb, tb, st));
   auto ma = make_mqa(p, B, T, a->q, a->q_pos, a->kv_cache, a->N_cap, a->out_idx, p->topk,
                      a->win_kv, a->L_raw, a->win_pos0, a->sink, a->q_rms_w, a->out);
   ma.chained = true;  // a top-k kernel of this library precedes it on the stream
-  TRY(cuda_status(csa::launch_mqa(ma, io == CSA_BF16, base + sb + tb, ws_bytes - sb - tb, st),
-                  "sparse MQA"));
+  const size_t mb = round_up(csa::mqa_workspace_bytes(ma));
+  csa::TopkArgs t{};
+  t.B = B; t.T = T; t.m = p->m; t.k = p->topk; t.n_cap = a->N_cap; t.scores = scores;
+  t.q_pos = a->q_pos; t.out_idx = a->out_idx;
+  if (io == CSA_BF16 && forward_qhat(p, B, T, a->N_cap)) {
+    t.qj.q = a->q;
+    t.qj.q_rms_w = a->q_rms_w;
+    t.qj.qhat = base + sb + tb + mb;
+    t.qj.H = p->n_heads;
+    t.qj.r = p->rope_dims;
+    t.qj.eps = p->rms_eps;
+    t.qj.rope_base = p->rope_base;
+    ma.qhat = t.qj.qhat;
+  }
+  TRY(index_then_topk(p, a->idx_dtype, B, T, a->N_cap, a->qI, a->qI_scale, a->w, a->KI,
+                      a->KI_scale, a->q_pos, scores, t, base + sb, tb, st));
+  TRY(cuda_status(csa::launch_mqa(ma, io == CSA_BF16, base + sb + tb, mb, st), "sparse MQA"));
   return ok();
 }
 

@@ -55,12 +55,23 @@ bool index_mxf4_tc_supported(const IndexArgs& a);
 cudaError_t launch_index_mxf4_tc(const IndexArgs& a, cudaStream_t st);
 cudaError_t index_mxf4_device_error(int* code);
 
+// q_hat = RoPE_t(RMSNorm(q) * q_rms_w) in bf16 for the attention that follows a top-k: an
+// optional side job of the decode selector (c = 512, bf16 io)
+struct QhatJob {
+  const void* q;        // bf16 [B*T][H][c]
+  const void* q_rms_w;  // bf16 [c] or nullptr
+  void* qhat;           // bf16 [B*T][H][c]; nullptr: no job
+  int H, r;
+  float eps, rope_base;
+};
+
 struct TopkArgs {
   int B, T, m, k;
   int64_t n_cap;
   const float* scores;
   const int64_t* q_pos;
   int32_t* out_idx;
+  QhatJob qj;
 };
 size_t topk_workspace_bytes(int B, int T, int64_t n_cap, int k);
 cudaError_t launch_topk(const TopkArgs& a, void* ws, size_t ws_bytes, cudaStream_t st,
@@ -76,6 +87,7 @@ struct TopkDecodeArgs {
   int* hist;          // [Q][4096]
   int* cnt;           // [Q][4]: sure count, boundary count, ticket
   uint64_t* list;     // [Q][k + n_cap]: sure list (k), then boundary list (n_cap)
+  QhatJob qj;
 };
 bool topk_decode_path(int B, int T, int64_t n_cap, int k);
 size_t topk_decode_ws_bytes(int B, int T, int64_t n_cap, int k);
@@ -93,6 +105,8 @@ struct MqaArgs {
   const float* sink;
   void* out;
   bool chained;  // as IndexArgs::chained (the attention may then prepare queries early)
+  const void* qhat;  // bf16 [B*T][H][c] prepared q_hat (written by an earlier kernel of the
+                     // chain) or nullptr: the attention prepares it
 };
 size_t mqa_workspace_bytes(const MqaArgs& a);
 // tensor-core attention (bf16, c = 512, heads in groups of 64)

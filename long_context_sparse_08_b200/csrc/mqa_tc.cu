@@ -222,13 +222,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
     }
     tmem_alloc(&S.tmem_slot, kTmemCols);
   } else {
-    // the group's 64 raw query rows (64 KB, contiguous) into the KV tile area, which the
-    // first gather only overwrites after q_hat is built; one pass, one latency
-    const uint32_t stage = smem_u32(base + kOffKV);
-    const uint4* qg = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) +
-                                                     ((size_t)bt * a.H + h0) * kC);
+    if (a.qhat != nullptr) {
+      // q_hat was prepared by an earlier kernel: copy it straight into the B-operand tile
+      const uint4* qg = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.qhat) +
+                                                       ((size_t)bt * a.H + h0) * kC);
+      const uint32_t qt = smem_u32(base + kOffQ);
 #pragma unroll 4
-    for (int i = tid; i < kHg * kC / 8; i += 128) cp_async16(stage + 16 * i, qg + i, true);
+      for (int i = tid; i < kHg * kC / 8; i += 128) {
+        const int h = i >> 6, d0 = 8 * (i & 63);
+        cp_async16(qt + (d0 >> 6) * (kHg * 128) + sw128(h, (d0 & 63) >> 3), qg + i, true);
+      }
+    } else {
+      // the group's 64 raw query rows (64 KB, contiguous) into the KV tile area, which the
+      // first gather only overwrites after q_hat is built; one pass, one latency
+      const uint32_t stage = smem_u32(base + kOffKV);
+      const uint4* qg = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) +
+                                                       ((size_t)bt * a.H + h0) * kC);
+#pragma unroll 4
+      for (int i = tid; i < kHg * kC / 8; i += 128) cp_async16(stage + 16 * i, qg + i, true);
+    }
     // RoPE table, norm weights and running stats while the copies are in flight
     for (int p = tid; p < r / 2; p += 128)
       rope_angle_cs((double)rl.t, P.inv_freq[p], &S.cs[p], &S.sn[p]);
@@ -245,58 +257,63 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
   const uint32_t tmem = S.tmem_slot;
 
   if (warp < 4) {
-    // ---- q_hat = RoPE_t(RMSNorm(q)) in bf16: two threads per head, 256 dims each. Thread
-    //      t reads its 32 chunks of 8 dims starting at chunk t % 32, so that a warp's reads
-    //      of one step spread over all banks. ----
-    uint8_t* qs = base + kOffQ;
-    const int qh = tid >> 1, qhalf = tid & 1;
-    const uint4* qrow = reinterpret_cast<const uint4*>(base + kOffKV + qh * (kC * 2)) + 32 * qhalf;
-    cp_async_wait_all();
-    bar_softmax();
-    float ss0 = 0.f, ss1 = 0.f;
-#pragma unroll 8
-    for (int i = 0; i < 32; ++i) {
-      const uint4 raw = qrow[(i + lane) & 31];
-      const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float lo = __uint_as_float(w4[k] << 16), hi = __uint_as_float(w4[k] & 0xffff0000u);
-        ss0 = fmaf(lo, lo, ss0);
-        ss1 = fmaf(hi, hi, ss1);
-      }
-    }
-    float ss = ss0 + ss1;
-    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-    const float rstd = rsqrtf(ss / (float)kC + a.eps);
-#pragma unroll 4
-    for (int i = 0; i < 32; ++i) {
-      const int c = (i + lane) & 31;
-      const uint4 raw = qrow[c];
-      const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-      const int d0 = 256 * qhalf + 8 * c;
-      float y[8];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        y[2 * k] = __uint_as_float(w4[k] << 16) * rstd * S.wq[d0 + 2 * k];
-        y[2 * k + 1] = __uint_as_float(w4[k] & 0xffff0000u) * rstd * S.wq[d0 + 2 * k + 1];
-      }
-      if (d0 >= r0) {
-#pragma unroll
+    if (a.qhat != nullptr) {
+      cp_async_wait_all();
+      fence_proxy_async_smem();  // the tile is read by the tensor cores
+    } else {
+      // ---- q_hat = RoPE_t(RMSNorm(q)) in bf16: two threads per head, 256 dims each. Thread
+      //      t reads its 32 chunks of 8 dims starting at chunk t % 32, so that a warp's reads
+      //      of one step spread over all banks. ----
+      uint8_t* qs = base + kOffQ;
+      const int qh = tid >> 1, qhalf = tid & 1;
+      const uint4* qrow = reinterpret_cast<const uint4*>(base + kOffKV + qh * (kC * 2)) + 32 * qhalf;
+      cp_async_wait_all();
+      bar_softmax();
+      float ss0 = 0.f, ss1 = 0.f;
+  #pragma unroll 8
+      for (int i = 0; i < 32; ++i) {
+        const uint4 raw = qrow[(i + lane) & 31];
+        const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+  #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int p = (d0 + 2 * k - r0) >> 1;
-          const float cs = S.cs[p], sn = S.sn[p], u = y[2 * k], v = y[2 * k + 1];
-          y[2 * k] = u * cs - v * sn;
-          y[2 * k + 1] = u * sn + v * cs;
+          const float lo = __uint_as_float(w4[k] << 16), hi = __uint_as_float(w4[k] & 0xffff0000u);
+          ss0 = fmaf(lo, lo, ss0);
+          ss1 = fmaf(hi, hi, ss1);
         }
       }
-      uint4 o;
-      uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        ow[k] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * k])) |
-                ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * k + 1])) << 16);
-      const int atom = d0 >> 6, chunk = (d0 & 63) >> 3;
-      *reinterpret_cast<uint4*>(qs + atom * (kHg * 128) + sw128(qh, chunk)) = o;
+      float ss = ss0 + ss1;
+      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+      const float rstd = rsqrtf(ss / (float)kC + a.eps);
+  #pragma unroll 4
+      for (int i = 0; i < 32; ++i) {
+        const int c = (i + lane) & 31;
+        const uint4 raw = qrow[c];
+        const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+        const int d0 = 256 * qhalf + 8 * c;
+        float y[8];
+  #pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          y[2 * k] = __uint_as_float(w4[k] << 16) * rstd * S.wq[d0 + 2 * k];
+          y[2 * k + 1] = __uint_as_float(w4[k] & 0xffff0000u) * rstd * S.wq[d0 + 2 * k + 1];
+        }
+        if (d0 >= r0) {
+  #pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int p = (d0 + 2 * k - r0) >> 1;
+            const float cs = S.cs[p], sn = S.sn[p], u = y[2 * k], v = y[2 * k + 1];
+            y[2 * k] = u * cs - v * sn;
+            y[2 * k + 1] = u * sn + v * cs;
+          }
+        }
+        uint4 o;
+        uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+  #pragma unroll
+        for (int k = 0; k < 4; ++k)
+          ow[k] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * k])) |
+                  ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * k + 1])) << 16);
+        const int atom = d0 >> 6, chunk = (d0 & 63) >> 3;
+        *reinterpret_cast<uint4*>(qs + atom * (kHg * 128) + sw128(qh, chunk)) = o;
+      }
     }
 
     // the selected rows, the partials and the output belong to the previous kernels

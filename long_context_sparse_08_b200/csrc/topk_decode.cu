@@ -162,9 +162,74 @@ __global__ void __launch_bounds__(256) k_zero(int4* p, int n4) {
     p[i] = make_int4(0, 0, 0, 0);
 }
 
+// The side job: q_hat rows of query q for heads [h0, h1), one warp per head, lane = 16 of
+// the 512 dims. Reads only caller inputs, so it runs before the dependency wait.
+__device__ void qhat_rows(const QhatJob& j, int q, double t, int h0, int h1, float* cs, float* sn) {
+  constexpr int kC = 512;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int r = j.r, r0 = kC - r;
+  for (int p = tid; p < r / 2; p += blockDim.x)
+    rope_cos_sin(t, p, r, (double)j.rope_base, &cs[p], &sn[p]);
+  __syncthreads();
+  for (int h = h0 + wid; h < h1; h += kWarps) {
+    const uint4* src = reinterpret_cast<const uint4*>(j.q) + ((size_t)q * j.H + h) * (kC / 8);
+    uint4* dst = reinterpret_cast<uint4*>(j.qhat) + ((size_t)q * j.H + h) * (kC / 8);
+    float x[16];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const uint4 raw = src[lane + 32 * half];
+      const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        x[8 * half + 2 * k] = __uint_as_float(w4[k] << 16);
+        x[8 * half + 2 * k + 1] = __uint_as_float(w4[k] & 0xffff0000u);
+      }
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) ss = fmaf(x[k], x[k], ss);
+    ss = warp_sum(ss);
+    const float rstd = rsqrtf(ss / (float)kC + j.eps);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int d0 = 8 * (lane + 32 * half);
+      float y[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float wgt = j.q_rms_w ? __bfloat162float(static_cast<const __nv_bfloat16*>(
+                                          j.q_rms_w)[d0 + k])
+                                    : 1.f;
+        y[k] = x[8 * half + k] * rstd * wgt;
+      }
+      if (d0 >= r0) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int p = (d0 + 2 * k - r0) >> 1;
+          const float c = cs[p], s = sn[p], u = y[2 * k], v = y[2 * k + 1];
+          y[2 * k] = u * c - v * s;
+          y[2 * k + 1] = u * s + v * c;
+        }
+      }
+      uint4 o;
+      uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        ow[k] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * k])) |
+                ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * k + 1])) << 16);
+      dst[lane + 32 * half] = o;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kFThreads, 2) k_topk_filter(TopkDecodeArgs a) {
   __shared__ int wsum[2 * kWarps];
   __shared__ int s_bin, s_base_s, s_base_b;
+  __shared__ float s_cs[256], s_sn[256];
+  if (a.qj.qhat != nullptr) {  // this CTA's share of the query's heads
+    const int hq = blockIdx.y;
+    qhat_rows(a.qj, hq, (double)a.q_pos[hq], a.qj.H * blockIdx.x / gridDim.x,
+              a.qj.H * (blockIdx.x + 1) / gridDim.x, s_cs, s_sn);
+  }
   pdl_wait();
   pdl_trigger();
   const int q = blockIdx.y, tid = threadIdx.x;
@@ -429,7 +494,7 @@ TopkDecodeArgs topk_decode_args(const TopkArgs& t, void* ws) {
   const size_t Q = (size_t)t.B * t.T;
   char* p = static_cast<char*>(ws);
   a.Q = (int)Q; a.m = t.m; a.k = t.k; a.n_cap = t.n_cap; a.scores = t.scores;
-  a.q_pos = t.q_pos; a.out_idx = t.out_idx;
+  a.q_pos = t.q_pos; a.out_idx = t.out_idx; a.qj = t.qj;
   a.hist = reinterpret_cast<int*>(p);
   p += rup(Q * kBins * 4);
   a.cnt = reinterpret_cast<int*>(p);
