@@ -213,7 +213,6 @@ csa_status index_then_topk(const csa_params* p, csa_dtype kdt, int32_t B, int32_
       const csa::TopkDecodeArgs da = csa::topk_decode_args(t, topk_ws);
       TRY(cuda_status(csa::topk_decode_clear(da, st), "top-k clear"));
       ia.hist = da.hist;
-      ia.chained = true;
     }
     TRY(cuda_status(csa::launch_index_scores(ia, st, &hist_done), "index scores"));
   }

@@ -123,30 +123,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   Smem& S = *reinterpret_cast<Smem*>(qbase + 2 * kQBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- per-query visible counts and unit prefix (warp 0, warp-level scan) ----
+  // ---- set-up that reads nothing a predecessor writes: barriers, TMEM, descriptors ----
   if (warp == 0) {
-    int run = 0;
-    for (int q0 = 0; q0 < p.Q; q0 += 32) {
-      const int q = q0 + lane;
-      int nv = 0;
-      if (q < p.Q) {
-        const int64_t t = p.q_pos[q];
-        const int64_t v = t < 0 ? 0 : (t / p.m < p.n_cap ? t / p.m : p.n_cap);
-        nv = (int)v;
-        S.nvis[q] = nv;
-      }
-      const int units = (nv + kUnitKeys - 1) / kUnitKeys;
-      int incl = units;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int x = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += x;
-      }
-      if (q < p.Q) S.prefix[q] = run + incl - units;
-      run += __shfl_sync(0xffffffffu, incl, 31);
-    }
     if (lane == 0) {
-      S.prefix[p.Q] = run;
       for (int i = 0; i < kStages; ++i) {
         mbar_init(&S.full[i], 1);
         mbar_init(&S.empty[i], 1);
@@ -174,9 +153,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // scores and the histogram may still be read or cleared by the previous kernels
+  // positions, scores and the histogram belong to the previous kernels from here on
   pdl_wait();
   pdl_trigger();
+  // ---- per-query visible counts and unit prefix (warp 0, warp-level scan) ----
+  if (warp == 0) {
+    int run = 0;
+    for (int q0 = 0; q0 < p.Q; q0 += 32) {
+      const int q = q0 + lane;
+      int nv = 0;
+      if (q < p.Q) {
+        const int64_t t = p.q_pos[q];
+        const int64_t v = t < 0 ? 0 : (t / p.m < p.n_cap ? t / p.m : p.n_cap);
+        nv = (int)v;
+        S.nvis[q] = nv;
+      }
+      const int units = (nv + kUnitKeys - 1) / kUnitKeys;
+      int incl = units;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += x;
+      }
+      if (q < p.Q) S.prefix[q] = run + incl - units;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) S.prefix[p.Q] = run;
+  }
+  __syncthreads();
   const uint32_t tmem = S.tmem_slot;
   const int U = S.prefix[p.Q];
   const int u0 = (int)(((int64_t)U * blockIdx.x) / gridDim.x);
@@ -456,7 +460,8 @@ cudaError_t launch_index_mxf4_tc(const IndexArgs& a, cudaStream_t st) {
                                        (int)smem);
   if (e != cudaSuccess) return e;
   timing_before(st);
-  e = launch(a.chained, k_index_mxf4_tc, dim3(grid), dim3(kThreads), smem, st, mk, mks, mq, mqs, p);
+  // programmatic launch always: the set-up before its wait reads no predecessor's data
+  e = launch(true, k_index_mxf4_tc, dim3(grid), dim3(kThreads), smem, st, mk, mks, mq, mqs, p);
   timing_after(st);
   return e;
 }

@@ -45,8 +45,6 @@ struct IndexArgs {
   const int64_t* q_pos;
   float* scores;  // [B, T, n_cap]
   int* hist;      // optional [B*T][4096] histogram of the scores' top 12 key bits (zeroed)
-  bool chained;   // the previous launch on the stream is a kernel of this library that has
-                  // waited for its own predecessors (the indexer may then start early)
 };
 // *hist_done: whether the launched kernel also filled a.hist
 cudaError_t launch_index_scores(const IndexArgs& a, cudaStream_t st, bool* hist_done = nullptr);
@@ -104,7 +102,9 @@ struct MqaArgs {
   const int64_t *q_pos, *win_pos0;
   const float* sink;
   void* out;
-  bool chained;  // as IndexArgs::chained (the attention may then prepare queries early)
+  bool chained;  // the previous launch on the stream is a kernel of this library that has
+                 // waited for its own predecessors (the attention may then prepare its
+                 // queries before its own wait)
   const void* qhat;  // bf16 [B*T][H][c] prepared q_hat (written by an earlier kernel of the
                      // chain) or nullptr: the attention prepares it
 };
@@ -112,6 +112,9 @@ size_t mqa_workspace_bytes(const MqaArgs& a);
 // tensor-core attention (bf16, c = 512, heads in groups of 64)
 bool mqa_tc_supported(const MqaArgs& a, bool bf16);
 size_t mqa_tc_workspace_bytes(const MqaArgs& a);
+// zero two 16-byte aligned ranges (sizes multiples of 16; the second may be empty) in
+// stream order; programmatic launch, waits for its predecessors
+cudaError_t launch_zero(void* p0, size_t b0, void* p1, size_t b1, cudaStream_t st);
 cudaError_t launch_mqa_tc(const MqaArgs& a, void* ws, size_t ws_bytes, cudaStream_t st);
 cudaError_t mqa_tc_device_error(int* code);
 cudaError_t launch_mqa(const MqaArgs& a, bool bf16, void* ws, size_t ws_bytes, cudaStream_t st);

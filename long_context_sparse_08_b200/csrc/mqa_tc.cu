@@ -10,10 +10,13 @@
 // entries, then the window) is cut into chunks of 128 rows, and the chunks of a stream are
 // split over `nsplit` CTAs. Per chunk, with bf16 operands in 128B-swizzled shared memory
 // and fp32 accumulators in TMEM:
-//   S^T[128 rows x 64 heads] = K_chunk . Q^T           (A = KV tile, K-major; B = q_hat)
-//   P^T = exp(S^T * scale - m_h) in bf16               (softmax warps, thread = row)
-//   O^T[4 x 128 dims x 64 heads] += V_chunk^T . P^T    (A = the same KV tile read MN-major)
-// so the gathered tile is read from shared memory by both products and never transposed.
+//   S[64 heads x 128 rows] = q_hat . K_chunk^T          (A = q_hat, M = 64; B = KV tile)
+//   P = exp(S * scale - m_h) in bf16                    (softmax: thread = head, its 128
+//                                                        row values in registers)
+//   O^T[4 x 128 dims x 64 heads] += V_chunk^T . P^T     (A = the same KV tile read MN-major,
+//                                                        B = P, K-major)
+// so the gathered tile is read from shared memory by both products and never transposed,
+// and every per-head reduction (max, sum) stays inside one thread.
 // The running max m_h is only raised when a chunk's max exceeds it by more than 8 (then
 // O^T and l are rescaled); exp(s - m) <= e^8 otherwise, exactly as correct.
 // One split: the CTA finalises (sink, RoPE(-t), bf16). Several: it writes (m, l, O)
@@ -44,7 +47,7 @@ constexpr int kOffEnd = kOffP + kRows * 128;
 
 // TMEM columns
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;     // S^T: 64 columns
+constexpr uint32_t kColS = 0;     // S: 128 columns (M = 64 layout)
 constexpr uint32_t kColO = 256;   // O^T slice s: 256 + 64 s
 
 enum { kErrKvFull = 201, kErrSFull = 202, kErrPFull = 203, kErrKvFree = 204 };
@@ -52,8 +55,7 @@ enum { kErrKvFull = 201, kErrSFull = 202, kErrPFull = 203, kErrKvFree = 204 };
 struct Smem {
   uint64_t kv_full, s_full, p_full, kv_free, done;
   uint32_t tmem_slot;
-  int any_rescale;
-  float red[4][kHg], red2[4][kHg];
+  uint32_t vmask[4];  // valid rows of the current chunk (bit j of word w: row 32w + j)
   float m_used[kHg], l_sum[kHg], alpha[kHg], fin[kHg];
   float cs[kMaxPairs], sn[kMaxPairs];  // RoPE table for pairs of the last r dims
   float wq[kC];                         // query RMSNorm weights
@@ -80,6 +82,20 @@ __device__ __forceinline__ bool all_ok_softmax(bool ok) {
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(res)
       : "r"((uint32_t)ok)
+      : "memory");
+  return res != 0;
+}
+
+// OR of `p` over the 128 softmax threads.
+__device__ __forceinline__ bool any_softmax(bool p) {
+  uint32_t res;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, 1, 128, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(res)
+      : "r"((uint32_t)p)
       : "memory");
   return res != 0;
 }
@@ -246,10 +262,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
       rope_angle_cs((double)rl.t, P.inv_freq[p], &S.cs[p], &S.sn[p]);
     for (int d = tid; d < kC; d += 128)
       S.wq[d] = a.q_rms_w ? __bfloat162float(static_cast<const __nv_bfloat16*>(a.q_rms_w)[d]) : 1.f;
-    if (tid < kHg) {
-      S.m_used[tid] = -INFINITY;
-      S.l_sum[tid] = 0.f;
-    }
   }
   tc_fence_before();
   __syncthreads();
@@ -322,6 +334,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
     bool ok = true;
     const uint32_t kv_base = smem_u32(base + kOffKV);
     const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+    const bool head_thr = lane < 16;  // lanes 0-15: the softmax of head hh
+    const int hh = 16 * warp + (lane & 15);
+    float mu_h = -INFINITY, l_h = 0.f;  // running max used and running sum of this head
 #pragma unroll 1
     for (int j = c0; j < c1 && ok; ++j) {
       const uint32_t it = (uint32_t)(j - c0);
@@ -331,8 +346,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
       //      w, w+4, ... with lane = 16-byte chunk (coalesced 512 B per instruction) ----
       const __nv_bfloat16* my_src = row_src(a, bt, b, rl, (int64_t)j * kRows + tid);
       S.src[tid] = my_src;
+      const uint32_t vb = __ballot_sync(0xffffffffu, my_src != nullptr);
+      if (lane == 0) S.vmask[warp] = vb;
       bar_softmax();
-#pragma unroll 1
+#pragma unroll 4
       for (int rr = warp; rr < kRows; rr += 4) {
         const __nv_bfloat16* src = S.src[rr];
 #pragma unroll
@@ -348,41 +365,42 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
       fence_proxy_async_smem();
       mbar_arrive(&S.kv_full);
 
-      // ---- softmax of S^T (thread = row), heads in groups of 16 ----
-      const int row = tid;
-      const bool valid = my_src != nullptr;
+      // ---- softmax: lanes 0-15 of warp w own heads 16w .. 16w+15 (the M = 64 accumulator
+      //      puts row 16w + i in TMEM lane 32w + i); a thread holds its head's 128 row values ----
       ok = all_ok_softmax(mbar_wait(&S.s_full, it & 1, kErrSFull));
       if (!ok) break;
       tc_fence_after();
-#pragma unroll 1
-      for (int g16 = 0; g16 < 4; ++g16) {  // per-head chunk max
-        uint32_t v[16];
-        tmem_ld_x16(lane_base + kColS + 16 * g16, v);
-        tmem_ld_wait();
-        float sv[16];
+      uint32_t sa[64], sb[64];
+      tmem_ld_32x32b_x64(lane_base + kColS, sa);
+      tmem_ld_32x32b_x64(lane_base + kColS + 64, sb);
+      tmem_ld_wait();
+      const uint32_t vm0 = S.vmask[0], vm1 = S.vmask[1], vm2 = S.vmask[2], vm3 = S.vmask[3];
+      // scaled logits in place (masked rows -> -inf); eight partial maxima keep the
+      // dependency chains short (max is exact in any order)
+      float cmx[8];
 #pragma unroll
-        for (int h = 0; h < 16; ++h) sv[h] = valid ? __uint_as_float(v[h]) * a.scale : -INFINITY;
-        const float m = warp_reduce16<true>(sv);
-        if ((lane & 1) == 0) S.red[warp][16 * g16 + reduce16_index(lane)] = m;
+      for (int i = 0; i < 8; ++i) cmx[i] = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < 64; ++r) {
+        const uint32_t w0 = r < 32 ? vm0 : vm1, w1 = r < 32 ? vm2 : vm3;
+        const float x0 = ((w0 >> (r & 31)) & 1u) ? __uint_as_float(sa[r]) * a.scale : -INFINITY;
+        const float x1 = ((w1 >> (r & 31)) & 1u) ? __uint_as_float(sb[r]) * a.scale : -INFINITY;
+        sa[r] = __float_as_uint(x0);
+        sb[r] = __float_as_uint(x1);
+        cmx[r & 3] = fmaxf(cmx[r & 3], x0);
+        cmx[4 + (r & 3)] = fmaxf(cmx[4 + (r & 3)], x1);
       }
-      bar_softmax();
-      if (tid < kHg) {
-        const float cm = fmaxf(fmaxf(S.red[0][tid], S.red[1][tid]),
-                               fmaxf(S.red[2][tid], S.red[3][tid]));
-        const float mu = S.m_used[tid];
-        float al = 1.f;
-        if (cm > mu + kLazy || (mu == -INFINITY && cm != -INFINITY)) {
-          al = (mu == -INFINITY) ? 0.f : expf(mu - cm);
-          S.m_used[tid] = cm;
-        }
-        S.alpha[tid] = al;
-        S.l_sum[tid] *= al;
+      const float cm = fmaxf(fmaxf(fmaxf(cmx[0], cmx[1]), fmaxf(cmx[2], cmx[3])),
+                             fmaxf(fmaxf(cmx[4], cmx[5]), fmaxf(cmx[6], cmx[7])));
+      float al = 1.f;
+      if (cm > mu_h + kLazy || (mu_h == -INFINITY && cm != -INFINITY)) {
+        al = (mu_h == -INFINITY) ? 0.f : expf(mu_h - cm);
+        mu_h = cm;
       }
-      if (tid == 0) S.any_rescale = 0;
-      bar_softmax();
-      if (tid < kHg && S.alpha[tid] != 1.f && j > c0) S.any_rescale = 1;
-      bar_softmax();
-      if (S.any_rescale) {  // rare: scale O^T columns by alpha (previous O^T MMAs are done)
+      l_h *= al;
+      if (head_thr) S.alpha[hh] = al;
+      if (any_softmax(head_thr && al != 1.f && j > c0)) {
+        // rare: scale O^T columns by alpha (the previous O^T MMAs are done)
 #pragma unroll 1
         for (int cgrp = 0; cgrp < 16; ++cgrp) {  // 4 slices x 4 groups of 16 heads
           uint32_t o[16];
@@ -397,39 +415,36 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
         }
         tmem_st_wait();
       }
-      // P^T row (bf16, swizzled B-operand tile) and per-head row sums
-      uint8_t* pt = base + kOffP;
-#pragma unroll 1
-      for (int g16 = 0; g16 < 4; ++g16) {
-        uint32_t v[16];
-        tmem_ld_x16(lane_base + kColS + 16 * g16, v);
-        tmem_ld_wait();
-        float pr[16];
-        uint32_t pk[8];
+      // P row of this head (bf16) into the K-major B tile: [row / 64][head][128 B]
+      if (head_thr) {
+        uint8_t* pt = base + kOffP;
+        float lc[4] = {0.f, 0.f, 0.f, 0.f};  // partial sums (sum what the MMA multiplies)
+        const float mref = mu_h == -INFINITY ? 0.f : mu_h;  // no valid row yet: every p is 0
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int h = 16 * g16 + 2 * k;
-          const float s0 = __uint_as_float(v[2 * k]) * a.scale;
-          const float s1 = __uint_as_float(v[2 * k + 1]) * a.scale;
-          const float p0 = valid ? __expf(s0 - S.m_used[h]) : 0.f;
-          const float p1 = valid ? __expf(s1 - S.m_used[h + 1]) : 0.f;
-          const __nv_bfloat16 b0 = __float2bfloat16_rn(p0), b1 = __float2bfloat16_rn(p1);
-          pr[2 * k] = __bfloat162float(b0);  // sum what the MMA multiplies
-          pr[2 * k + 1] = __bfloat162float(b1);
-          pk[k] = (uint32_t)__bfloat16_as_ushort(b0) | ((uint32_t)__bfloat16_as_ushort(b1) << 16);
+        for (int c8 = 0; c8 < 16; ++c8) {  // rows 8*c8 .. 8*c8+7
+          uint32_t pk[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int r = 8 * c8 + 2 * k;
+            const float s0 = __uint_as_float(r < 64 ? sa[r & 63] : sb[r & 63]);
+            const float s1 = __uint_as_float(r < 64 ? sa[(r + 1) & 63] : sb[(r + 1) & 63]);
+            const __nv_bfloat16 b0 = __float2bfloat16_rn(__expf(s0 - mref));  // -inf -> 0
+            const __nv_bfloat16 b1 = __float2bfloat16_rn(__expf(s1 - mref));
+            lc[k] += __bfloat162float(b0) + __bfloat162float(b1);
+            pk[k] = (uint32_t)__bfloat16_as_ushort(b0) | ((uint32_t)__bfloat16_as_ushort(b1) << 16);
+          }
+          *reinterpret_cast<uint4*>(pt + (c8 >> 3) * (kHg * 128) + sw128(hh, c8 & 7)) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
-        *reinterpret_cast<uint4*>(pt + sw128(row, 2 * g16)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        *reinterpret_cast<uint4*>(pt + sw128(row, 2 * g16 + 1)) =
-            make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        const float l = warp_reduce16<false>(pr);
-        if ((lane & 1) == 0) S.red2[warp][16 * g16 + reduce16_index(lane)] = l;
+        l_h += (lc[0] + lc[1]) + (lc[2] + lc[3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&S.p_full);
-      bar_softmax();
-      if (tid < kHg)
-        S.l_sum[tid] += (S.red2[0][tid] + S.red2[1][tid]) + (S.red2[2][tid] + S.red2[3][tid]);
+    }
+    if (head_thr) {
+      S.m_used[hh] = mu_h;
+      S.l_sum[hh] = l_h;
     }
     // ---- epilogue: wait for the last O^T, then finalise or write the partial ----
     if (ok && c1 > c0)
@@ -493,8 +508,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
     }
   } else {
     // ------------------------------ MMA issuer (warp 4) ------------------------------
-    const uint32_t idS = idesc_f16(1, kRows, kHg);                       // K-major A and B
-    const uint32_t idO = idesc_f16(1, kRows, kHg) | (1u << 15) | (1u << 16);  // MN-major A, B
+    const uint32_t idS = idesc_f16(1, kHg, kRows);                 // M = 64, N = 128, K-major
+    const uint32_t idO = idesc_f16(1, kRows, kHg) | (1u << 15);    // A MN-major, B K-major
     const uint32_t kv = smem_u32(base + kOffKV), qs = smem_u32(base + kOffQ),
                    pt = smem_u32(base + kOffP);
     bool ok = true;
@@ -507,8 +522,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
 #pragma unroll 1
         for (int kk = 0; kk < 32; ++kk) {  // K = 512 in steps of 16
           const uint32_t atom = kk >> 2, koff = (kk & 3) * 32;
-          const uint64_t ad = smem_desc(kv + atom * (kRows * 128) + koff, 16, 1024, kLayoutSw128);
-          const uint64_t bd = smem_desc(qs + atom * (kHg * 128) + koff, 16, 1024, kLayoutSw128);
+          const uint64_t ad = smem_desc(qs + atom * (kHg * 128) + koff, 16, 1024, kLayoutSw128);
+          const uint64_t bd = smem_desc(kv + atom * (kRows * 128) + koff, 16, 1024, kLayoutSw128);
           mma_f16(tmem + kColS, ad, bd, idS, kk > 0 ? 1u : 0u);
         }
         mma_commit(&S.s_full);
@@ -524,7 +539,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
           for (int kk = 0; kk < kRows / 16; ++kk) {  // K = 128 rows in steps of 16
             const uint64_t ad = smem_desc(kv + sl * 2 * (kRows * 128) + kk * 2048, kRows * 128,
                                           1024, kLayoutSw128);
-            const uint64_t bd = smem_desc(pt + kk * 2048, kRows * 128, 1024, kLayoutSw128);
+            const uint64_t bd = smem_desc(pt + (kk >> 2) * (kHg * 128) + (kk & 3) * 32, 16, 1024,
+                                          kLayoutSw128);
             mma_f16(tmem + kColO + 64 * sl, ad, bd, idO, (j > c0 || kk > 0) ? 1u : 0u);
           }
         }

@@ -154,12 +154,16 @@ __device__ __forceinline__ void block_scan2(int c0, int c1, int* ws, int* o0, in
   __syncthreads();
 }
 
-// zero n4 int4 words (the histogram and counters of a call), in stream order
-__global__ void __launch_bounds__(256) k_zero(int4* p, int n4) {
-  pdl_wait();
+// zero n0 + n1 int4 words of two ranges (histograms and counters of a call), in stream order
+// Triggers before it waits: the next kernel (the indexer) may then start its set-up while
+// this one waits, which is safe because that set-up reads nothing a predecessor writes.
+__global__ void __launch_bounds__(256) k_zero(int4* p0, int n0, int4* p1, int n1) {
   pdl_trigger();
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += gridDim.x * blockDim.x)
-    p[i] = make_int4(0, 0, 0, 0);
+  pdl_wait();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n0 + n1; i += gridDim.x * blockDim.x) {
+    if (i < n0) p0[i] = make_int4(0, 0, 0, 0);
+    else p1[i - n0] = make_int4(0, 0, 0, 0);
+  }
 }
 
 // The side job: q_hat rows of query q for heads [h0, h1), one warp per head, lane = 16 of
@@ -506,9 +510,14 @@ TopkDecodeArgs topk_decode_args(const TopkArgs& t, void* ws) {
 cudaError_t topk_decode_clear(const TopkDecodeArgs& a, cudaStream_t st) {
   // hist and the counters are adjacent at the start of the workspace
   const size_t bytes = rup((size_t)a.Q * kBins * 4) + rup((size_t)a.Q * 16);
-  const int n4 = (int)(bytes / 16);
-  return launch(true, k_zero, dim3((n4 + 255) / 256), dim3(256), 0, st,
-                reinterpret_cast<int4*>(a.hist), n4);
+  return launch_zero(a.hist, bytes, nullptr, 0, st);
+}
+
+cudaError_t launch_zero(void* p0, size_t b0, void* p1, size_t b1, cudaStream_t st) {
+  const int n0 = (int)(b0 / 16), n1 = p1 ? (int)(b1 / 16) : 0;
+  const int blocks = (n0 + n1 + 255) / 256;
+  return launch(true, k_zero, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, st,
+                reinterpret_cast<int4*>(p0), n0, reinterpret_cast<int4*>(p1), n1);
 }
 
 cudaError_t launch_topk_decode(TopkDecodeArgs a, bool hist_ready, cudaStream_t st) {
