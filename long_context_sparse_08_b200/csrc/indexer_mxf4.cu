@@ -13,17 +13,21 @@
 // 16*i + 4*j + b of a block is block-scale b of key 32*j + i. One TMA copy of a unit's
 // 2 KB of scales therefore lands ready for tcgen05.cp (no rearrangement in the kernel).
 //
-// Persistent kernel, one CTA per SM, 10 warps:
+// Persistent kernel, one CTA per SM, 11 warps:
 //   warp 0     TMA producer: per unit one 32 KB key box (64B-swizzled) and one 2 KB scale
 //              box; per query the 64 x 64 B heads and their scale words;
-//   warp 1     MMA issuer (one lane): per query the query scales into TMEM (rearranged
-//              once), per M-tile the key scales into TMEM (tcgen05.cp) and two MMAs;
+//   warps 1,10 MMA issuers (one lane each): warp 1 takes M-tiles 0-1 of every unit, warp 10
+//              M-tiles 2-3, each into its own TMEM slot; per query each copies the query
+//              scales into its own TMEM columns, per M-tile the key scales (tcgen05.cp),
+//              then two MMAs. An MMA of this shape costs the tensor unit ~50 cycles however
+//              many threads issue, but the copies, waits and commits cost the issuing
+//              thread; two issuers run those chains side by side;
 //   warps 2-9  two epilogue warpgroups; group g reduces M-tiles g and 2 + g of each unit:
 //              TMEM -> registers, w * ReLU head sum, fp32 score store, and a 4096-bin
 //              histogram of the scores' top 12 key bits for the top-k selector.
-// TMEM holds two half-unit slots (2 M-tiles each): while both groups reduce one half-unit
-// the MMAs of the next run. Every wait and tcgen05 instruction costs tens of cycles on the
-// single issuing thread, so the loop precomputes descriptors and waits once per half-unit.
+// TMEM holds two half-unit slots (2 M-tiles each), one per issuer: while both groups
+// reduce one half-unit the other issuer's MMAs run. Descriptors are precomputed and each
+// issuer waits once per unit for its slot.
 // Units are split evenly over the CTAs; ragged per-query visibility is handled by masking
 // the stores.
 #include <cudaTypedefs.h>
@@ -40,14 +44,15 @@ namespace {
 
 using namespace tc;
 
-constexpr int kStages = 4;
+constexpr int kStages = 5;
 constexpr int kTileKeys = 128;     // M of one MMA
 constexpr int kUnitTiles = 4;
 constexpr int kUnitKeys = kUnitTiles * kTileKeys;  // keys per pipeline stage
 constexpr int kHeads = 64;         // N (indexer heads)
 constexpr int kRowBytes = 64;      // 128 e2m1 per row
 constexpr int kMaxQueries = 1024;  // (request, query) pairs per launch
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
+constexpr int kWarpMma1 = kThreads / 32 - 1;  // second MMA issuer (last warp)
 constexpr int kBins = 4096;
 
 constexpr int kOffA = 0;                                // 32 KB, 1024-aligned
@@ -58,7 +63,7 @@ constexpr uint32_t kStageTx = kUnitKeys * kRowBytes + kUnitKeys * 4;
 constexpr int kOffQ = 0;                                // 4 KB q heads (64B-swizzled)
 constexpr int kOffQS = kOffQ + kHeads * kRowBytes;      // 256 B query scale words
 constexpr int kOffQSF = kOffQS + kHeads * 4;            // 512 B rearranged for tcgen05.cp
-constexpr int kQBytes = ((kOffQSF + 512 + 1023) / 1024) * 1024;
+constexpr int kQBytes = ((kOffQSF + 2 * 512 + 1023) / 1024) * 1024;  // one layout per issuer
 constexpr uint32_t kQTx = kHeads * kRowBytes + kHeads * 4;
 
 // TMEM columns: two half-unit slots of two 64-column accumulators, their key-scale columns,
@@ -66,7 +71,7 @@ constexpr uint32_t kQTx = kHeads * kRowBytes + kHeads * 4;
 constexpr uint32_t kTmemCols = 512;
 __device__ __forceinline__ uint32_t acc_col(int hs, int j) { return 128u * hs + 64u * j; }
 __device__ __forceinline__ uint32_t sfa_col(int hs, int j) { return 256u + 16u * hs + 8u * j; }
-__device__ __forceinline__ uint32_t sfb_col(int qs) { return 288u + 8u * qs; }
+__device__ __forceinline__ uint32_t sfb_col(int qs, int h) { return 288u + 16u * qs + 8u * h; }
 
 enum { kErrFull = 101, kErrEmpty = 102, kErrTmemFull = 103, kErrTmemEmpty = 104,
        kErrQFull = 105, kErrQEmpty = 106 };
@@ -128,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       for (int i = 0; i < kStages; ++i) {
         mbar_init(&S.full[i], 1);
-        mbar_init(&S.empty[i], 1);
+        mbar_init(&S.empty[i], 2);  // both issuers' MMAs read the stage
       }
       for (int i = 0; i < 2; ++i) {
         mbar_init(&S.tfull[i], 1);
@@ -136,9 +141,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int i = 0; i < 2; ++i) {
         mbar_init(&S.qfull[i], 1);
-        mbar_init(&S.qempty[i], 1);
+        mbar_init(&S.qempty[i], 2);
       }
-      mbar_init(&S.done, 1);
+      mbar_init(&S.done, 2);
       fence_barrier_init();
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_ks);
@@ -147,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     tmem_alloc(&S.tmem_slot, kTmemCols);
-  } else {
+  } else if (warp != kWarpMma1) {
     for (int i = threadIdx.x - 64; i < kBins; i += 256) S.hist[i] = 0;
   }
   tc_fence_before();
@@ -226,8 +231,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = (issued_q > 2 ? issued_q - 2 : 0); j < issued_q; ++j)
         mbar_wait(&S.qfull[j & 1], (uint32_t)((j >> 1) & 1), kErrQFull);
     }
-  } else if (warp == 1) {
-    // ------------------------------ MMA issuer (one lane) ------------------------------
+  } else if (warp == 1 || warp == kWarpMma1) {
+    // ------------------------- MMA issuers (one lane each) -------------------------
+    const int h = warp == 1 ? 0 : 1;  // this issuer's half of every unit and TMEM slot
     if (lane == 0) {
       const uint32_t id0 = idesc_mxf4(kTileKeys, kHeads, 0, 0);
       const uint32_t id1 = idesc_mxf4(kTileKeys, kHeads, 2, 2);
@@ -247,15 +253,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int qs = nq & 1;
           ok = mbar_wait(&S.qfull[qs], (nq >> 1) & 1, kErrQFull);
           if (!ok) break;
-          // query scale words -> tcgen05.cp layout (16-byte row i: words of heads i, 32+i)
+          // query scale words -> tcgen05.cp layout (16-byte row i: words of heads i, 32+i),
+          // one copy per issuer
           uint8_t* qb = qbase + qs * kQBytes;
           const uint32_t* sq = reinterpret_cast<const uint32_t*>(qb + kOffQS);
+          uint8_t* qsf = qb + kOffQSF + 512 * h;
           for (int i = 0; i < 32; ++i)
-            *reinterpret_cast<uint4*>(qb + kOffQSF + 16 * i) = make_uint4(sq[i], sq[32 + i], 0u, 0u);
+            *reinterpret_cast<uint4*>(qsf + 16 * i) = make_uint4(sq[i], sq[32 + i], 0u, 0u);
           fence_proxy_async_smem();
           tc_fence_after();
-          tmem_cp_32x128b_warpx4(tmem + sfb_col(qs),
-                                 smem_desc(smem_u32(qb + kOffQSF), 0, 128, kLayoutNone));
+          tmem_cp_32x128b_warpx4(tmem + sfb_col(qs, h),
+                                 smem_desc(smem_u32(qsf), 0, 128, kLayoutNone));
         }
         const int qs = nq & 1;
         const int st = k % kStages;
@@ -264,30 +272,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t a_st = a_desc0 + (uint64_t)st * (kStageBytes >> 4);
         const uint64_t sf_st = sf_desc0 + (uint64_t)st * (kStageBytes >> 4);
         const uint64_t b0 = q_desc0 + (uint64_t)qs * (kQBytes >> 4);
-        const uint32_t sfb = tmem + sfb_col(qs);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {  // half-units: M-tiles 2h, 2h+1
-          const int n = 2 * k + h, hs = n & 1;
-          ok = mbar_wait(&S.tempty[hs], ((uint32_t)(n >> 1) & 1) ^ 1, kErrTmemEmpty);
-          if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int j = 0; j < 2; ++j)  // key scales of both tiles first (latencies overlap)
-            tmem_cp_32x128b_warpx4(tmem + sfa_col(hs, j), sf_st + (uint64_t)(2 * h + j) * 32);
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const uint64_t a0 = a_st + (uint64_t)(2 * h + j) * 512;  // 8 KB per M-tile
-            const uint32_t d = tmem + acc_col(hs, j), sfa = tmem + sfa_col(hs, j);
-            mma_mxf4(d, a0, b0, id0, sfa, sfb, 0u);
-            // second K half: +32 bytes inside the swizzled rows, scale bytes 2..3
-            mma_mxf4(d, a0 + 2, b0 + 2, id1, sfa | (2u << 30), sfb | (2u << 30), 1u);
-          }
-          mma_commit(&S.tfull[hs]);
-        }
+        const uint32_t sfb = tmem + sfb_col(qs, h);
+        ok = mbar_wait(&S.tempty[h], ((uint32_t)k & 1) ^ 1, kErrTmemEmpty);
         if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int j = 0; j < 2; ++j)  // key scales of both tiles first (latencies overlap)
+          tmem_cp_32x128b_warpx4(tmem + sfa_col(h, j), sf_st + (uint64_t)(2 * h + j) * 32);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const uint64_t a0 = a_st + (uint64_t)(2 * h + j) * 512;  // 8 KB per M-tile
+          const uint32_t d = tmem + acc_col(h, j), sfa = tmem + sfa_col(h, j);
+          mma_mxf4(d, a0, b0, id0, sfa, sfb, 0u);
+          // second K half: +32 bytes inside the swizzled rows, scale bytes 2..3
+          mma_mxf4(d, a0 + 2, b0 + 2, id1, sfa | (2u << 30), sfb | (2u << 30), 1u);
+        }
+        mma_commit(&S.tfull[h]);
         mma_commit(&S.empty[st]);
       }
-      // every MMA / copy this thread issued has completed once `done` fires
+      // every MMA / copy this thread issued has completed once `done` fires (both issuers)
       mma_commit(&S.done);
       mbar_wait(&S.done, 0, kErrTmemFull);
     }
