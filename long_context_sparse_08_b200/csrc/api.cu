@@ -243,10 +243,11 @@ const char* csa_last_error(void) { return g_err; }
 
 csa_status csa_device_error(int32_t* code) {
   REQUIRE(code != nullptr, "code is NULL");
-  int c = 0, c2 = 0;
+  int c = 0, c2 = 0, c3 = 0;
   TRY(cuda_status(csa::index_mxf4_device_error(&c), "device error word"));
   TRY(cuda_status(csa::mqa_tc_device_error(&c2), "device error word"));
-  *code = c != 0 ? c : c2;
+  TRY(cuda_status(csa::index_bf16_device_error(&c3), "device error word"));
+  *code = c != 0 ? c : (c2 != 0 ? c2 : c3);
   return ok();
 }
 

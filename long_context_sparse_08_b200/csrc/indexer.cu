@@ -126,6 +126,10 @@ cudaError_t launch_index_scores(const IndexArgs& a, cudaStream_t st, bool* hist_
     if (hist_done) *hist_done = a.hist != nullptr;
     return launch_index_mxf4_tc(a, st);
   }
+  if (index_bf16_tc_supported(a)) {
+    if (hist_done) *hist_done = a.hist != nullptr;
+    return launch_index_bf16_tc(a, st);
+  }
   dim3 grid((unsigned)((a.n_cap + kKeysPerCta - 1) / kKeysPerCta), a.B * a.T);
   const size_t smem = ((size_t)a.n_idx_heads * a.d_idx + a.n_idx_heads) * sizeof(float);
   timing_before(st);

@@ -1,0 +1,490 @@
+// Stage 2 on tensor cores for FP8 (e4m3 + row scale) and bf16 indexer keys with bf16
+// queries (decode).
+//
+// 【论文解读】DeepSeek-V4, 一(三)1(2): I[t,s] = sum_h w[t,h] * ReLU(q^I[t,h] . K[s]).
+//
+// A tile is 128 keys of one query's request: D[128 keys x 64 heads] = K_tile . q^T over
+// d_I = 128 as eight tcgen05 kind::f16 MMAs (K = 16 each, bf16 operands, fp32 accumulation
+// in TMEM). TMEM lane = key, so an epilogue thread owns one key and reduces its 64 head
+// dots with w * ReLU(.) without shuffles.
+//
+// FP8 keys: an e4m3 code is exactly a bf16 value, so converter warps rewrite each staged
+// 16 KB tile of codes as the 32 KB bf16 operand (128B-swizzled, K-major); the row scale is
+// positive and commutes with ReLU, so the epilogue multiplies it into the finished sum (the
+// same order as the CUDA-core kernel). bf16 keys: TMA writes the operand tile directly.
+//
+// Persistent kernel, one CTA per SM, 10 warps:
+//   warp 0     TMA producer: per tile the key codes (fp8: into a staging ring; bf16: into
+//              the operand ring), per query the 64 heads of q^I (two 128B-swizzled boxes);
+//   warp 1     MMA issuer (one lane);
+//   warps 2-5  converters (fp8 only): staging -> bf16 operand tile;
+//   warps 6-9  epilogue: TMEM -> registers, w * ReLU head sum, times the row scale (fp8),
+//              fp32 score store, 4096-bin histogram of the scores' top 12 key bits.
+// Tiles are split evenly over the CTAs; ragged visibility is handled by masking the stores.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace csa {
+
+namespace {
+
+using namespace tc;
+
+constexpr int kTileKeys = 128;    // M of one MMA
+constexpr int kHeads = 64;        // N (indexer heads)
+constexpr int kDim = 128;         // d_I
+constexpr int kMaxQueries = 512;  // (request, query) pairs per launch
+constexpr int kThreads = 320;
+constexpr int kBins = 4096;
+constexpr int kStg = 4;           // fp8 staging tiles (16 KB of codes each)
+constexpr int kOps = 3;           // bf16 operand tiles (32 KB each); bf16 keys: 5
+constexpr int kOpsBf16 = 5;
+constexpr int kAcc = 4;           // TMEM accumulator slots (64 columns each)
+
+constexpr int kStgBytes = kTileKeys * kDim;         // 16 KB of e4m3 codes
+constexpr int kOpBytes = kTileKeys * kDim * 2;      // 32 KB: 2 atoms x 128 rows x 128 B
+constexpr int kAtomBytes = kTileKeys * 128;         // 16 KB
+constexpr int kQBytes = kHeads * kDim * 2;          // 16 KB: 2 atoms x 64 rows x 128 B
+constexpr int kQAtomBytes = kHeads * 128;           // 8 KB
+
+enum { kErrStgFull = 301, kErrStgEmpty = 302, kErrOpFull = 303, kErrOpEmpty = 304,
+       kErrTFull = 305, kErrTEmpty = 306, kErrQFull = 307, kErrQEmpty = 308 };
+
+struct Bf16IdxParams {
+  int Q, T, m;
+  int64_t n_cap;
+  const int64_t* q_pos;
+  const float* w;
+  const float* key_scale;  // fp8: [B * n_cap] row scales; bf16: nullptr
+  float* scores;
+  int* hist;  // optional [Q][4096]
+};
+
+struct Smem {
+  uint64_t stg_full[kStg], stg_empty[kStg], op_full[kOpsBf16], op_empty[kOpsBf16];
+  uint64_t tfull[kAcc], tempty[kAcc], qfull[2], qempty[2], done;
+  uint32_t tmem_slot;
+  int prefix[kMaxQueries + 1];
+  int nvis[kMaxQueries];
+  int hist[kBins];
+};
+
+__device__ __forceinline__ int find_query(const int* prefix, int Q, int u) {
+  int lo = 0, hi = Q;  // largest q with prefix[q] <= u
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (prefix[mid] <= u) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+// AND of `ok` over the 128 threads of named barrier `id`
+template <int kId>
+__device__ __forceinline__ bool group_all_ok(bool ok) {
+  uint32_t res;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, %2, 128, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(res)
+      : "r"((uint32_t)ok), "n"(kId)
+      : "memory");
+  return res != 0;
+}
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
+  return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+
+// two e4m3 codes (low byte = first) -> bf16x2, exact
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t v) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(v));
+  const __half2 hh = *reinterpret_cast<const __half2*>(&h2);
+  const float2 f = __half22float2(hh);
+  const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
+  return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+template <bool kFp8>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_index_bf16_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+                    Bf16IdxParams p) {
+  constexpr int kOpN = kFp8 ? kOps : kOpsBf16;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* opbase = base;                               // kOpN x 32 KB
+  uint8_t* qbase = opbase + kOpN * kOpBytes;            // 2 x 16 KB
+  uint8_t* stgbase = qbase + 2 * kQBytes;               // fp8: kStg x 16 KB
+  Smem& S = *reinterpret_cast<Smem*>(stgbase + (kFp8 ? kStg * kStgBytes : 0));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- set-up that reads nothing a predecessor writes ----
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int i = 0; i < kStg; ++i) {
+        mbar_init(&S.stg_full[i], 1);
+        mbar_init(&S.stg_empty[i], 128);
+      }
+      for (int i = 0; i < kOpN; ++i) {
+        mbar_init(&S.op_full[i], kFp8 ? 128 : 1);
+        mbar_init(&S.op_empty[i], 1);
+      }
+      for (int i = 0; i < kAcc; ++i) {
+        mbar_init(&S.tfull[i], 1);
+        mbar_init(&S.tempty[i], 4);  // the four epilogue warps
+      }
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&S.qfull[i], 1);
+        mbar_init(&S.qempty[i], 1);
+      }
+      mbar_init(&S.done, 1);
+      fence_barrier_init();
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_q);
+    }
+  } else if (warp == 1) {
+    tmem_alloc(&S.tmem_slot, 64 * kAcc);
+  } else if (warp >= 6) {
+    for (int i = threadIdx.x - 192; i < kBins; i += 128) S.hist[i] = 0;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  pdl_wait();
+  pdl_trigger();
+  // ---- per-query visible counts and tile prefix (warp 0) ----
+  if (warp == 0) {
+    int run = 0;
+    for (int q0 = 0; q0 < p.Q; q0 += 32) {
+      const int q = q0 + lane;
+      int nv = 0;
+      if (q < p.Q) {
+        const int64_t t = p.q_pos[q];
+        const int64_t v = t < 0 ? 0 : (t / p.m < p.n_cap ? t / p.m : p.n_cap);
+        nv = (int)v;
+        S.nvis[q] = nv;
+      }
+      const int tiles = (nv + kTileKeys - 1) / kTileKeys;
+      int incl = tiles;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += x;
+      }
+      if (q < p.Q) S.prefix[q] = run + incl - tiles;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) S.prefix[p.Q] = run;
+  }
+  __syncthreads();
+  const uint32_t tmem = S.tmem_slot;
+  const int U = S.prefix[p.Q];
+  const int u0 = (int)(((int64_t)U * blockIdx.x) / gridDim.x);
+  const int u1 = (int)(((int64_t)U * (blockIdx.x + 1)) / gridDim.x);
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    if (lane == 0 && u0 < u1) {
+      int q = find_query(S.prefix, p.Q, u0);
+      int cur_q = -1, nq = -1, k = 0, issued_q = 0;
+      bool ok = true;
+      for (int u = u0; u < u1 && ok; ++u, ++k) {
+        while (u >= S.prefix[q + 1]) ++q;
+        if (q != cur_q) {
+          ++nq;
+          cur_q = q;
+          const int qs = nq & 1;
+          ok = mbar_wait(&S.qempty[qs], ((nq >> 1) & 1) ^ 1, kErrQEmpty);
+          if (!ok) break;
+          uint8_t* qb = qbase + qs * kQBytes;
+          mbar_arrive_expect_tx(&S.qfull[qs], kQBytes);
+          tma_load_2d(qb, &tm_q, 0, q * kHeads, &S.qfull[qs]);
+          tma_load_2d(qb + kQAtomBytes, &tm_q, 64, q * kHeads, &S.qfull[qs]);
+          issued_q = nq + 1;
+        }
+        const int tile = u - S.prefix[q];
+        const int b = q / p.T;
+        const int32_t row = (int32_t)(b * p.n_cap + (int64_t)tile * kTileKeys);
+        if (kFp8) {
+          const int s = k % kStg;
+          ok = mbar_wait(&S.stg_empty[s], ((k / kStg) & 1) ^ 1, kErrStgEmpty);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&S.stg_full[s], kStgBytes);
+          tma_load_2d(stgbase + s * kStgBytes, &tm_k, 0, row, &S.stg_full[s]);
+        } else {
+          const int o = k % kOpN;
+          ok = mbar_wait(&S.op_empty[o], ((k / kOpN) & 1) ^ 1, kErrOpEmpty);
+          if (!ok) break;
+          uint8_t* ob = opbase + o * kOpBytes;
+          mbar_arrive_expect_tx(&S.op_full[o], kOpBytes);
+          tma_load_2d(ob, &tm_k, 0, row, &S.op_full[o]);
+          tma_load_2d(ob + kAtomBytes, &tm_k, 64, row, &S.op_full[o]);
+        }
+      }
+      // drain: no copy into this CTA's shared memory may still be in flight at exit
+      const int ring = kFp8 ? kStg : kOpN;
+      for (int j = (k > ring ? k - ring : 0); j < k; ++j) {
+        if (kFp8)
+          mbar_wait(&S.stg_full[j % kStg], (uint32_t)((j / kStg) & 1), kErrStgFull);
+        else
+          mbar_wait(&S.op_full[j % kOpN], (uint32_t)((j / kOpN) & 1), kErrOpFull);
+      }
+      for (int j = (issued_q > 2 ? issued_q - 2 : 0); j < issued_q; ++j)
+        mbar_wait(&S.qfull[j & 1], (uint32_t)((j >> 1) & 1), kErrQFull);
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer (one lane) ------------------------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16(1, kTileKeys, kHeads);  // bf16, M = 128, N = 64, K-major
+      const uint32_t op_s = smem_u32(opbase), q_s = smem_u32(qbase);
+      int q = u0 < u1 ? find_query(S.prefix, p.Q, u0) : 0;
+      int cur_q = -1, nq = -1, k = 0;
+      bool ok = true;
+      for (int u = u0; u < u1 && ok; ++u, ++k) {
+        while (u >= S.prefix[q + 1]) ++q;
+        if (q != cur_q) {
+          if (cur_q >= 0) mma_commit(&S.qempty[nq & 1]);  // old slot free once its MMAs end
+          ++nq;
+          cur_q = q;
+          ok = mbar_wait(&S.qfull[nq & 1], (nq >> 1) & 1, kErrQFull);
+          if (!ok) break;
+        }
+        const int o = k % kOpN, a = k % kAcc;
+        ok = mbar_wait(&S.op_full[o], (uint32_t)(k / kOpN) & 1, kErrOpFull);
+        if (!ok) break;
+        ok = mbar_wait(&S.tempty[a], ((uint32_t)(k / kAcc) & 1) ^ 1, kErrTEmpty);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t ob = op_s + o * kOpBytes, qb = q_s + (nq & 1) * kQBytes;
+#pragma unroll
+        for (int kk = 0; kk < kDim / 16; ++kk) {  // K = 128 in steps of 16
+          const uint32_t atom = kk >> 2, koff = (kk & 3) * 32;
+          const uint64_t ad = smem_desc(ob + atom * kAtomBytes + koff, 16, 1024, kLayoutSw128);
+          const uint64_t bd = smem_desc(qb + atom * kQAtomBytes + koff, 16, 1024, kLayoutSw128);
+          mma_f16(tmem + 64u * a, ad, bd, idesc, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&S.op_empty[o]);
+        mma_commit(&S.tfull[a]);
+      }
+      mma_commit(&S.done);  // every MMA this thread issued has completed once it fires
+      mbar_wait(&S.done, 0, kErrTFull);
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // ------------------------------ converters (fp8) ------------------------------
+    if (kFp8) {
+      const int ct = threadIdx.x - 64;  // 0..127
+      bool ok = true;
+      for (int u = u0, k = 0; u < u1 && ok; ++u, ++k) {
+        const int s = k % kStg, o = k % kOpN;
+        ok = group_all_ok<3>(mbar_wait(&S.stg_full[s], (uint32_t)(k / kStg) & 1, kErrStgFull) &&
+                             mbar_wait(&S.op_empty[o], ((uint32_t)(k / kOpN) & 1) ^ 1, kErrOpEmpty));
+        if (!ok) break;
+        const uint8_t* src = stgbase + s * kStgBytes;
+        uint8_t* dst = opbase + o * kOpBytes;
+        // a warp converts 4 rows per step: lane = (row % 4, 16-byte input chunk of 8)
+        const int rsub = (ct & 31) >> 3, ic = ct & 7;
+#pragma unroll 4
+        for (int r0 = 4 * (ct >> 5); r0 < kTileKeys; r0 += 16) {
+          const int r = r0 + rsub;
+          const uint4 raw = *reinterpret_cast<const uint4*>(src + r * kDim + 16 * ic);
+          const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+          uint32_t o8[8];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            o8[2 * j] = e4m3x2_to_bf16x2((uint16_t)(w4[j] & 0xffffu));
+            o8[2 * j + 1] = e4m3x2_to_bf16x2((uint16_t)(w4[j] >> 16));
+          }
+          // dims 16*ic .. 16*ic+15 -> atom ic / 4, output chunks 2*(ic % 4), +1
+          uint8_t* at = dst + (ic >> 2) * kAtomBytes;
+          const int c8 = 2 * (ic & 3);
+          *reinterpret_cast<uint4*>(at + sw128(r, c8)) = make_uint4(o8[0], o8[1], o8[2], o8[3]);
+          *reinterpret_cast<uint4*>(at + sw128(r, c8 + 1)) = make_uint4(o8[4], o8[5], o8[6], o8[7]);
+        }
+        fence_proxy_async_smem();  // the operand tile is read by the tensor cores
+        mbar_arrive(&S.op_full[o]);
+        mbar_arrive(&S.stg_empty[s]);
+      }
+    }
+  } else {
+    // ------------------------------ epilogue ------------------------------
+    const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+    const bool hist = p.hist != nullptr;
+    int hq = -1;
+    auto flush = [&](int qq) {  // shared histogram of query qq -> global, then clear
+      epi_bar();
+      for (int i = threadIdx.x - 192; i < kBins; i += 128) {
+        const int v = S.hist[i];
+        if (v) {
+          atomicAdd(&p.hist[(size_t)qq * kBins + i], v);
+          S.hist[i] = 0;
+        }
+      }
+      epi_bar();
+    };
+    float wr[kHeads];
+    int cur_q = -1;
+    int q = u0 < u1 ? find_query(S.prefix, p.Q, u0) : 0;
+    bool ok = true;
+    for (int u = u0, k = 0; u < u1 && ok; ++u, ++k) {
+      while (u >= S.prefix[q + 1]) ++q;
+      const int tile = u - S.prefix[q];
+      if (q != cur_q) {
+#pragma unroll
+        for (int h = 0; h < kHeads; ++h) wr[h] = p.w[(size_t)q * kHeads + h];
+        cur_q = q;
+      }
+      if (hist && q != hq) {
+        if (hq >= 0) flush(hq);
+        hq = q;
+      }
+      const int s = tile * kTileKeys + 32 * quad + lane;
+      const int b = q / p.T;
+      const bool vis = s < S.nvis[q];
+      // the row scale is loaded before the wait, so its latency hides behind the MMAs
+      const float scale = (kFp8 && vis) ? p.key_scale[(size_t)b * p.n_cap + s] : 1.f;
+      const int a = k % kAcc;
+      ok = group_all_ok<2>(mbar_wait(&S.tfull[a], (uint32_t)(k / kAcc) & 1, kErrTFull));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t v[kHeads];
+      tmem_ld_32x32b_x64(tmem + ((uint32_t)(32 * quad) << 16) + 64u * a, v);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.tempty[a]);
+      float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int hh = 0; hh < kHeads; ++hh)
+        part[hh & 3] = fmaf(wr[hh], fmaxf(__uint_as_float(v[hh]), 0.f), part[hh & 3]);
+      float sc = (part[0] + part[1]) + (part[2] + part[3]);
+      if (kFp8) sc *= scale;
+      if (vis) {
+        p.scores[(size_t)q * p.n_cap + s] = sc;
+        if (hist) atomicAdd(&S.hist[float_key(sc) >> 20], 1);
+      }
+    }
+    if (hist && hq >= 0) flush(hq);
+  }
+  // ---- teardown: the MMA warp saw its last MMA complete; free TMEM ----
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64 * kAcc);
+  }
+}
+
+// ---- host: tensor maps ----
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// bf16 rows of 128 values, box = 64 values (one 128-byte swizzle atom) x box_rows
+bool make_map_bf16_rows(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kDim, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kDim * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// e4m3 rows of 128 bytes, box = one 128-key tile, no swizzle (the converters read it)
+bool make_map_fp8_rows(CUtensorMap* m, const void* ptr, uint64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kDim, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kDim};
+  cuuint32_t box[2] = {(cuuint32_t)kDim, (cuuint32_t)kTileKeys};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <bool kFp8>
+size_t smem_bytes() {
+  return 1024 + (size_t)(kFp8 ? kOps : kOpsBf16) * kOpBytes + 2 * kQBytes +
+         (kFp8 ? (size_t)kStg * kStgBytes : 0) + sizeof(Smem);
+}
+
+}  // namespace
+
+bool index_bf16_tc_supported(const IndexArgs& a) {
+  return (a.kdt == CSA_FP8_E4M3_ROWSCALE || a.kdt == CSA_BF16) && a.n_idx_heads == kHeads &&
+         a.d_idx == kDim && a.n_cap % kTileKeys == 0 && (int64_t)a.B * a.T <= kMaxQueries &&
+         (int64_t)a.B * a.n_cap < (1ll << 31);
+}
+
+cudaError_t launch_index_bf16_tc(const IndexArgs& a, cudaStream_t st) {
+  const int Q = a.B * a.T;
+  const bool fp8 = a.kdt == CSA_FP8_E4M3_ROWSCALE;
+  CUtensorMap mk, mq;
+  const bool good = fp8 ? make_map_fp8_rows(&mk, a.KI, (uint64_t)a.B * a.n_cap)
+                        : make_map_bf16_rows(&mk, a.KI, (uint64_t)a.B * a.n_cap, kTileKeys);
+  if (!good || !make_map_bf16_rows(&mq, a.qI, (uint64_t)Q * kHeads, kHeads))
+    return cudaErrorInvalidValue;
+  Bf16IdxParams p{Q, a.T, a.m, a.n_cap, a.q_pos, a.w,
+                  fp8 ? static_cast<const float*>(a.KI_scale) : nullptr, a.scores, a.hist};
+  const int64_t tiles_max = (int64_t)Q * (a.n_cap / kTileKeys);
+  const int grid = (int)(tiles_max < num_sms() ? (tiles_max > 0 ? tiles_max : 1) : num_sms());
+  cudaError_t e;
+  timing_before(st);
+  if (fp8) {
+    const size_t smem = smem_bytes<true>();
+    e = cudaFuncSetAttribute(k_index_bf16_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e == cudaSuccess)
+      e = launch(true, k_index_bf16_tc<true>, dim3(grid), dim3(kThreads), smem, st, mk, mq, p);
+  } else {
+    const size_t smem = smem_bytes<false>();
+    e = cudaFuncSetAttribute(k_index_bf16_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e == cudaSuccess)
+      e = launch(true, k_index_bf16_tc<false>, dim3(grid), dim3(kThreads), smem, st, mk, mq, p);
+  }
+  timing_after(st);
+  return e;
+}
+
+cudaError_t index_bf16_device_error(int* code) {
+  int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(code, tc::g_device_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyToSymbol(tc::g_device_error, &zero, sizeof(int));
+}
+
+}  // namespace csa

@@ -52,6 +52,11 @@ cudaError_t launch_index_scores(const IndexArgs& a, cudaStream_t st, bool* hist_
 bool index_mxf4_tc_supported(const IndexArgs& a);
 cudaError_t launch_index_mxf4_tc(const IndexArgs& a, cudaStream_t st);
 cudaError_t index_mxf4_device_error(int* code);
+// tensor-core kernel for FP8 (e4m3 + row scale) and bf16 keys with bf16 queries (64 heads x
+// 128 dims, N_cap % 128 == 0, B*T <= 512)
+bool index_bf16_tc_supported(const IndexArgs& a);
+cudaError_t launch_index_bf16_tc(const IndexArgs& a, cudaStream_t st);
+cudaError_t index_bf16_device_error(int* code);
 
 // q_hat = RoPE_t(RMSNorm(q) * q_rms_w) in bf16 for the attention that follows a top-k: an
 // optional side job of the decode selector (c = 512, bf16 io)

@@ -226,6 +226,17 @@ _reg(Shape("edge_decode_mxfp4", "csa_decode", "bf16", "mxfp4", B=5, T=1, m=4, c=
 _reg(Shape("edge_decode_mxfp4_long", "csa_decode", "bf16", "mxfp4", B=4, T=1, m=4, c=512,
            rope_dims=64, n_heads=128, n_idx_heads=64, d_idx=128, topk=1024, n_win=128,
            n_cap=16384, ctx=0, seed=19, q_pos_override=(4 * 16384 + 301, 48001, 13, 4100)))
+# Tensor-core indexer cases for fp8 and bf16 keys (cache capacity a multiple of 128): zero
+# tiles, a single partial tile, several tiles, and more positions than the cache holds.
+_reg(Shape("edge_decode_fp8_tc", "csa_decode", "bf16", "fp8", B=5, T=1, m=4, c=512,
+           rope_dims=64, n_heads=64, n_idx_heads=64, d_idx=128, topk=512, n_win=128,
+           n_cap=4096, ctx=0, seed=20, q_pos_override=(3, 7, 515, 4099, 16384 + 77)))
+_reg(Shape("edge_decode_bf16_tc", "csa_decode", "bf16", "bf16", B=4, T=1, m=4, c=512,
+           rope_dims=64, n_heads=64, n_idx_heads=64, d_idx=128, topk=512, n_win=128,
+           n_cap=8192, ctx=0, seed=21, q_pos_override=(4 * 8192 + 301, 20001, 13, 4100)))
+_reg(Shape("mid_prefill_bf16_tc", "csa_prefill", "bf16", "bf16", B=1, T=384, m=4, c=512,
+           rope_dims=64, n_heads=64, n_idx_heads=64, d_idx=128, topk=512, n_win=128, n_cap=768,
+           ctx=2416, n_tok=384, seed=22))
 _reg(Shape("edge_hca_decode", "hca_decode", "bf16", "none", B=3, T=1, m=128, c=512, rope_dims=64,
            n_heads=64, n_idx_heads=0, d_idx=0, topk=0, n_win=128, n_cap=40, ctx=0, seed=17,
            overlap=0, q_pos_override=(0, 127, 9000)))

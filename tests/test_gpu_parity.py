@@ -83,7 +83,8 @@ def test_compress_parity(name):
 
 INDEX_CASES = ["tiny_prefill_f32", "mid_decode_fp8", "mid_decode_mxfp4", "mid_decode_bf16",
                "edge_decode_bf16", "edge_decode_mxfp4", "edge_decode_mxfp4_long",
-               "mid_prefill_bf16"]
+               "mid_prefill_bf16", "edge_decode_fp8_tc", "edge_decode_bf16_tc",
+               "mid_prefill_bf16_tc"]
 
 
 @pytest.mark.parametrize("name", INDEX_CASES)
@@ -229,7 +230,9 @@ def _forward_parity(name, queries=None):
 
 @pytest.mark.parametrize("name", ["tiny_prefill_f32", "mid_decode_fp8", "mid_decode_mxfp4",
                                   "mid_decode_bf16", "edge_decode_bf16", "edge_decode_mxfp4",
-                                  "edge_decode_mxfp4_long", "mid_prefill_bf16"])
+                                  "edge_decode_mxfp4_long", "mid_prefill_bf16",
+                                  "edge_decode_fp8_tc", "edge_decode_bf16_tc",
+                                  "mid_prefill_bf16_tc"])
 def test_forward_parity(name):
     _forward_parity(name)
     assert csa.device_error() == 0
