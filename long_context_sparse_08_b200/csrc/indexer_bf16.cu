@@ -57,6 +57,7 @@ enum { kErrStgFull = 301, kErrStgEmpty = 302, kErrOpFull = 303, kErrOpEmpty = 30
 
 struct Bf16IdxParams {
   int Q, T, m;
+  int q0;  // global index of this launch's first query (launches take <= kMaxQueries)
   int64_t n_cap;
   const int64_t* q_pos;
   const float* w;
@@ -212,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           issued_q = nq + 1;
         }
         const int tile = u - S.prefix[q];
-        const int b = q / p.T;
+        const int b = (p.q0 + q) / p.T;
         const int32_t row = (int32_t)(b * p.n_cap + (int64_t)tile * kTileKeys);
         if (kFp8) {
           const int s = k % kStg;
@@ -348,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         hq = q;
       }
       const int s = tile * kTileKeys + 32 * quad + lane;
-      const int b = q / p.T;
+      const int b = (p.q0 + q) / p.T;
       const bool vis = s < S.nvis[q];
       // the row scale is loaded before the wait, so its latency hides behind the MMAs
       const float scale = (kFp8 && vis) ? p.key_scale[(size_t)b * p.n_cap + s] : 1.f;
@@ -445,36 +446,40 @@ size_t smem_bytes() {
 
 bool index_bf16_tc_supported(const IndexArgs& a) {
   return (a.kdt == CSA_FP8_E4M3_ROWSCALE || a.kdt == CSA_BF16) && a.n_idx_heads == kHeads &&
-         a.d_idx == kDim && a.n_cap % kTileKeys == 0 && (int64_t)a.B * a.T <= kMaxQueries &&
-         (int64_t)a.B * a.n_cap < (1ll << 31);
+         a.d_idx == kDim && a.n_cap % kTileKeys == 0 && (int64_t)a.B * a.n_cap < (1ll << 31);
 }
 
 cudaError_t launch_index_bf16_tc(const IndexArgs& a, cudaStream_t st) {
-  const int Q = a.B * a.T;
+  const int Qall = a.B * a.T;
   const bool fp8 = a.kdt == CSA_FP8_E4M3_ROWSCALE;
-  CUtensorMap mk, mq;
+  CUtensorMap mk;
   const bool good = fp8 ? make_map_fp8_rows(&mk, a.KI, (uint64_t)a.B * a.n_cap)
                         : make_map_bf16_rows(&mk, a.KI, (uint64_t)a.B * a.n_cap, kTileKeys);
-  if (!good || !make_map_bf16_rows(&mq, a.qI, (uint64_t)Q * kHeads, kHeads))
-    return cudaErrorInvalidValue;
-  Bf16IdxParams p{Q, a.T, a.m, a.n_cap, a.q_pos, a.w,
-                  fp8 ? static_cast<const float*>(a.KI_scale) : nullptr, a.scores, a.hist};
-  const int64_t tiles_max = (int64_t)Q * (a.n_cap / kTileKeys);
-  const int grid = (int)(tiles_max < num_sms() ? (tiles_max > 0 ? tiles_max : 1) : num_sms());
-  cudaError_t e;
+  if (!good) return cudaErrorInvalidValue;
+  const size_t smem = fp8 ? smem_bytes<true>() : smem_bytes<false>();
+  cudaError_t e = fp8 ? cudaFuncSetAttribute(k_index_bf16_tc<true>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+                      : cudaFuncSetAttribute(k_index_bf16_tc<false>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   timing_before(st);
-  if (fp8) {
-    const size_t smem = smem_bytes<true>();
-    e = cudaFuncSetAttribute(k_index_bf16_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e == cudaSuccess)
-      e = launch(true, k_index_bf16_tc<true>, dim3(grid), dim3(kThreads), smem, st, mk, mq, p);
-  } else {
-    const size_t smem = smem_bytes<false>();
-    e = cudaFuncSetAttribute(k_index_bf16_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e == cudaSuccess)
-      e = launch(true, k_index_bf16_tc<false>, dim3(grid), dim3(kThreads), smem, st, mk, mq, p);
+  // queries in launches of at most kMaxQueries (each launch walks its queries' tiles)
+  for (int q0 = 0; q0 < Qall && e == cudaSuccess; q0 += kMaxQueries) {
+    const int Q = Qall - q0 < kMaxQueries ? Qall - q0 : kMaxQueries;
+    CUtensorMap mq;
+    const auto* qI = static_cast<const __nv_bfloat16*>(a.qI) + (size_t)q0 * kHeads * kDim;
+    if (!make_map_bf16_rows(&mq, qI, (uint64_t)Q * kHeads, kHeads)) {
+      e = cudaErrorInvalidValue;
+      break;
+    }
+    Bf16IdxParams p{Q, a.T, a.m, q0, a.n_cap, a.q_pos + q0, a.w + (size_t)q0 * kHeads,
+                    fp8 ? static_cast<const float*>(a.KI_scale) : nullptr,
+                    a.scores + (size_t)q0 * a.n_cap,
+                    a.hist ? a.hist + (size_t)q0 * kBins : nullptr};
+    const int64_t tiles_max = (int64_t)Q * (a.n_cap / kTileKeys);
+    const int grid = (int)(tiles_max < num_sms() ? (tiles_max > 0 ? tiles_max : 1) : num_sms());
+    e = fp8 ? launch(true, k_index_bf16_tc<true>, dim3(grid), dim3(kThreads), smem, st, mk, mq, p)
+            : launch(true, k_index_bf16_tc<false>, dim3(grid), dim3(kThreads), smem, st, mk, mq, p);
   }
   timing_after(st);
   return e;

@@ -53,7 +53,7 @@ bool index_mxf4_tc_supported(const IndexArgs& a);
 cudaError_t launch_index_mxf4_tc(const IndexArgs& a, cudaStream_t st);
 cudaError_t index_mxf4_device_error(int* code);
 // tensor-core kernel for FP8 (e4m3 + row scale) and bf16 keys with bf16 queries (64 heads x
-// 128 dims, N_cap % 128 == 0, B*T <= 512)
+// 128 dims, N_cap % 128 == 0; launched over batches of at most 512 queries)
 bool index_bf16_tc_supported(const IndexArgs& a);
 cudaError_t launch_index_bf16_tc(const IndexArgs& a, cudaStream_t st);
 cudaError_t index_bf16_device_error(int* code);
