@@ -80,6 +80,17 @@ def algorithmic_bytes_per_query(s, n_vis: int) -> dict:
     return {"index": idx, "total": idx + att}
 
 
+def prefill_flops(s) -> dict:
+    """Indexer: 2 * H_I * d_I per visible (t, s) pair; attention: 4 * c flops per head per
+    attended row (q.k and p.v), rows = min(k, visible) + window."""
+    vis = [min((s.ctx + i) // s.m, s.n_cap) for i in range(s.T)]
+    pairs = sum(vis)
+    rows = sum(min(s.topk, v) + min(s.n_win, s.ctx + i + 1) for i, v in enumerate(vis))
+    idx = 2 * s.n_idx_heads * s.d_idx * pairs * s.B
+    att = 4 * s.c * s.n_heads * rows * s.B
+    return {"index": idx, "attention": att, "total": idx + att}
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -265,8 +276,13 @@ def run_ours(args, W, rank, world, local_rank):
     if has_index and idx_ms:
         alg = queries * per_q["index"]
         achieved = alg / (idx_ms / 1e3) / 1e9
-        kname, kfile = (("k_index_mxf4_tc", "indexer_mxf4.cu") if s.idx == "mxfp4"
-                        else ("k_index_scores_cc", "indexer.cu"))
+        if s.idx == "mxfp4":
+            kname, kfile = "k_index_mxf4_tc", "indexer_mxf4.cu"
+        elif s.idx in ("fp8", "bf16") and s.n_cap % 128 == 0 and s.n_idx_heads == 64 \
+                and s.d_idx == 128:
+            kname, kfile = "k_index_bf16_tc", "indexer_bf16.cu"
+        else:
+            kname, kfile = "k_index_scores_cc", "indexer.cu"
         src = os.path.join(ROOT, "long_context_sparse_08_b200", "csrc", kfile)
         roof = {"kernel": kname, "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -296,6 +312,15 @@ def run_ours(args, W, rank, world, local_rank):
         "e2e": e2e,
         "gpu_launches": launches,
     }
+    if s.kind == "csa_prefill":
+        # a compute-bound step: algorithmic flops (indexer over the visible (t, s) pairs,
+        # attention over the selected and window rows) against the dense bf16 tensor peak
+        fl = prefill_flops(s)
+        tf = fl["total"] / (ms / K / 1e3) / 1e12
+        res["tflops"] = {"value": round(tf, 1), "flops_per_step": fl,
+                         "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
+                         "peak": peaks["bf16_tflops"],
+                         "peak_source": f"{peak_src} bf16_tflops (cuBLAS burst)"}
     return res, inp, s
 
 
