@@ -13,13 +13,19 @@
 // positive and commutes with ReLU, so the epilogue multiplies it into the finished sum (the
 // same order as the CUDA-core kernel). bf16 keys: TMA writes the operand tile directly.
 //
+// Prefill (bf16 keys, several queries per request): four consecutive queries of a request
+// share every key tile, so one MMA is N = 256 (4 x 64 heads). An f16 MMA of N = 64 costs the
+// tensor unit several times its arithmetic; at N = 256 the arithmetic dominates.
+//
 // Persistent kernel, one CTA per SM, 10 warps:
 //   warp 0     TMA producer: per tile the key codes (fp8: into a staging ring; bf16: into
-//              the operand ring), per query the 64 heads of q^I (two 128B-swizzled boxes);
+//              the operand ring), per query group the heads of q^I (two 128B-swizzled boxes);
 //   warp 1     MMA issuer (one lane);
-//   warps 2-5  converters (fp8 only): staging -> bf16 operand tile;
+//   warps 2-5  converters (fp8 only): staging -> bf16 operand tile; with query groups of
+//              four they are a second epilogue group instead;
 //   warps 6-9  epilogue: TMEM -> registers, w * ReLU head sum, times the row scale (fp8),
-//              fp32 score store, 4096-bin histogram of the scores' top 12 key bits.
+//              fp32 score store, 4096-bin histogram of the scores' top 12 key bits (one
+//              query per tile only).
 // Tiles are split evenly over the CTAs; ragged visibility is handled by masking the stores.
 #include <cudaTypedefs.h>
 
@@ -36,24 +42,36 @@ namespace {
 using namespace tc;
 
 constexpr int kTileKeys = 128;    // M of one MMA
-constexpr int kHeads = 64;        // N (indexer heads)
+constexpr int kHeads = 64;        // indexer heads (N of one query)
 constexpr int kDim = 128;         // d_I
 constexpr int kMaxQueries = 512;  // (request, query) pairs per launch
 constexpr int kThreads = 320;
 constexpr int kBins = 4096;
 constexpr int kStg = 4;           // fp8 staging tiles (16 KB of codes each)
-constexpr int kOps = 3;           // bf16 operand tiles (32 KB each); bf16 keys: 5
-constexpr int kOpsBf16 = 5;
-constexpr int kAcc = 4;           // TMEM accumulator slots (64 columns each)
 
 constexpr int kStgBytes = kTileKeys * kDim;         // 16 KB of e4m3 codes
 constexpr int kOpBytes = kTileKeys * kDim * 2;      // 32 KB: 2 atoms x 128 rows x 128 B
 constexpr int kAtomBytes = kTileKeys * 128;         // 16 KB
-constexpr int kQBytes = kHeads * kDim * 2;          // 16 KB: 2 atoms x 64 rows x 128 B
-constexpr int kQAtomBytes = kHeads * 128;           // 8 KB
+constexpr int kQBytes = kHeads * kDim * 2;          // 16 KB per query: 2 atoms x 64 x 128 B
 
 enum { kErrStgFull = 301, kErrStgEmpty = 302, kErrOpFull = 303, kErrOpEmpty = 304,
        kErrTFull = 305, kErrTEmpty = 306, kErrQFull = 307, kErrQEmpty = 308 };
+
+// G consecutive queries of one request share each key tile: N = 64 G per MMA.
+template <bool kFp8, int G>
+struct Cfg {
+  static constexpr int kQSlots = G == 1 ? 2 : 1;      // q tiles in flight
+  static constexpr int kOpN = kFp8 ? 3 : (G == 1 ? 5 : 4);
+  static constexpr int kAccN = G == 1 ? 4 : 2;        // TMEM accumulator slots
+  static constexpr int kAccCols = 64 * G;
+  static constexpr int kTmemCols = kAccN * kAccCols;  // 256 or 512
+  static constexpr int kQSlotBytes = G * kQBytes;
+  static constexpr int kQAtomBytes = G * kHeads * 128;
+  static constexpr int kEpiWarps = G == 1 ? 4 : 8;    // warps 6-9, or 2-9
+  static constexpr int kEpiThreads = 32 * kEpiWarps;
+  static constexpr int kEpiWarp0 = 10 - kEpiWarps;
+  static constexpr bool kHist = G == 1;
+};
 
 struct Bf16IdxParams {
   int Q, T, m;
@@ -66,17 +84,21 @@ struct Bf16IdxParams {
   int* hist;  // optional [Q][4096]
 };
 
+template <bool kHist>
 struct Smem {
-  uint64_t stg_full[kStg], stg_empty[kStg], op_full[kOpsBf16], op_empty[kOpsBf16];
-  uint64_t tfull[kAcc], tempty[kAcc], qfull[2], qempty[2], done;
+  uint64_t stg_full[kStg], stg_empty[kStg], op_full[5], op_empty[5];
+  uint64_t tfull[4], tempty[4], qfull[2], qempty[2], done;
   uint32_t tmem_slot;
-  int prefix[kMaxQueries + 1];
-  int nvis[kMaxQueries];
-  int hist[kBins];
+  int ngroups;
+  int prefix[kMaxQueries + 1];  // tile prefix over groups
+  int gfirst[kMaxQueries];      // first (local) query of each group
+  int nvis[kMaxQueries];        // visible entries of each query
+  float wst[4][kHeads];         // head weights of the current group (G > 1)
+  int hist[kHist ? kBins : 1];
 };
 
-__device__ __forceinline__ int find_query(const int* prefix, int Q, int u) {
-  int lo = 0, hi = Q;  // largest q with prefix[q] <= u
+__device__ __forceinline__ int find_group(const int* prefix, int ng, int u) {
+  int lo = 0, hi = ng;  // largest g with prefix[g] <= u
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (prefix[mid] <= u) lo = mid; else hi = mid;
@@ -84,21 +106,24 @@ __device__ __forceinline__ int find_query(const int* prefix, int Q, int u) {
   return lo;
 }
 
-// AND of `ok` over the 128 threads of named barrier `id`
-template <int kId>
+// AND of `ok` over the kN threads of named barrier kId
+template <int kId, int kN>
 __device__ __forceinline__ bool group_all_ok(bool ok) {
   uint32_t res;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.and.pred p, %2, 128, q;\n\t"
+      "bar.red.and.pred p, %2, %3, q;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(res)
-      : "r"((uint32_t)ok), "n"(kId)
+      : "r"((uint32_t)ok), "n"(kId), "n"(kN)
       : "memory");
   return res != 0;
 }
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+template <int kN>
+__device__ __forceinline__ void epi_bar() {
+  asm volatile("bar.sync 2, %0;" ::"n"(kN) : "memory");
+}
 
 __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
   return row * 128u + ((chunk ^ (row & 7u)) << 4);
@@ -114,18 +139,19 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t v) {
   return *reinterpret_cast<const uint32_t*>(&b);
 }
 
-template <bool kFp8>
+template <bool kFp8, int G>
 __global__ void __launch_bounds__(kThreads, 1)
     k_index_bf16_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                     Bf16IdxParams p) {
-  constexpr int kOpN = kFp8 ? kOps : kOpsBf16;
+  using C = Cfg<kFp8, G>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* opbase = base;                               // kOpN x 32 KB
-  uint8_t* qbase = opbase + kOpN * kOpBytes;            // 2 x 16 KB
-  uint8_t* stgbase = qbase + 2 * kQBytes;               // fp8: kStg x 16 KB
-  Smem& S = *reinterpret_cast<Smem*>(stgbase + (kFp8 ? kStg * kStgBytes : 0));
+  uint8_t* qbase = opbase + C::kOpN * kOpBytes;         // kQSlots x G x 16 KB
+  uint8_t* stgbase = qbase + C::kQSlots * C::kQSlotBytes;  // fp8: kStg x 16 KB
+  Smem<C::kHist>& S =
+      *reinterpret_cast<Smem<C::kHist>*>(stgbase + (kFp8 ? kStg * kStgBytes : 0));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // ---- set-up that reads nothing a predecessor writes ----
@@ -135,15 +161,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&S.stg_full[i], 1);
         mbar_init(&S.stg_empty[i], 128);
       }
-      for (int i = 0; i < kOpN; ++i) {
+      for (int i = 0; i < C::kOpN; ++i) {
         mbar_init(&S.op_full[i], kFp8 ? 128 : 1);
         mbar_init(&S.op_empty[i], 1);
       }
-      for (int i = 0; i < kAcc; ++i) {
+      for (int i = 0; i < C::kAccN; ++i) {
         mbar_init(&S.tfull[i], 1);
-        mbar_init(&S.tempty[i], 4);  // the four epilogue warps
+        mbar_init(&S.tempty[i], C::kEpiWarps);
       }
-      for (int i = 0; i < 2; ++i) {
+      for (int i = 0; i < C::kQSlots; ++i) {
         mbar_init(&S.qfull[i], 1);
         mbar_init(&S.qempty[i], 1);
       }
@@ -153,67 +179,86 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_q);
     }
   } else if (warp == 1) {
-    tmem_alloc(&S.tmem_slot, 64 * kAcc);
-  } else if (warp >= 6) {
-    for (int i = threadIdx.x - 192; i < kBins; i += 128) S.hist[i] = 0;
+    tmem_alloc(&S.tmem_slot, C::kTmemCols);
+  } else if (C::kHist && warp >= C::kEpiWarp0) {
+    for (int i = threadIdx.x - 32 * C::kEpiWarp0; i < kBins; i += C::kEpiThreads) S.hist[i] = 0;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   pdl_wait();
   pdl_trigger();
-  // ---- per-query visible counts and tile prefix (warp 0) ----
+  // ---- groups (G consecutive queries of one request) and their tile prefix (warp 0) ----
   if (warp == 0) {
-    int run = 0;
-    for (int q0 = 0; q0 < p.Q; q0 += 32) {
-      const int q = q0 + lane;
-      int nv = 0;
+    int ng = 0;
+    for (int qb0 = 0; qb0 < p.Q; qb0 += 32) {
+      const int q = qb0 + lane;
+      bool start = false;
       if (q < p.Q) {
         const int64_t t = p.q_pos[q];
         const int64_t v = t < 0 ? 0 : (t / p.m < p.n_cap ? t / p.m : p.n_cap);
-        nv = (int)v;
-        S.nvis[q] = nv;
+        S.nvis[q] = (int)v;
+        start = q == 0 || ((p.q0 + q) % p.T) % G == 0;
       }
-      const int tiles = (nv + kTileKeys - 1) / kTileKeys;
+      const uint32_t bal = __ballot_sync(0xffffffffu, start);
+      if (start) S.gfirst[ng + __popc(bal & ((1u << lane) - 1u))] = q;
+      ng += __popc(bal);
+    }
+    __syncwarp();
+    int run = 0;
+    for (int g0 = 0; g0 < ng; g0 += 32) {
+      const int g = g0 + lane;
+      int tiles = 0;
+      if (g < ng) {
+        const int f = S.gfirst[g], e = g + 1 < ng ? S.gfirst[g + 1] : p.Q;
+        int nv = 0;
+        for (int mq = f; mq < e; ++mq) nv = max(nv, S.nvis[mq]);
+        tiles = (nv + kTileKeys - 1) / kTileKeys;
+      }
       int incl = tiles;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int x = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += x;
       }
-      if (q < p.Q) S.prefix[q] = run + incl - tiles;
+      if (g < ng) S.prefix[g] = run + incl - tiles;
       run += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) S.prefix[p.Q] = run;
+    if (lane == 0) {
+      S.prefix[ng] = run;
+      S.ngroups = ng;
+    }
   }
   __syncthreads();
   const uint32_t tmem = S.tmem_slot;
-  const int U = S.prefix[p.Q];
+  const int NG = S.ngroups;
+  const int U = S.prefix[NG];
   const int u0 = (int)(((int64_t)U * blockIdx.x) / gridDim.x);
   const int u1 = (int)(((int64_t)U * (blockIdx.x + 1)) / gridDim.x);
+  auto gsize = [&](int g) { return (g + 1 < NG ? S.gfirst[g + 1] : p.Q) - S.gfirst[g]; };
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
     if (lane == 0 && u0 < u1) {
-      int q = find_query(S.prefix, p.Q, u0);
-      int cur_q = -1, nq = -1, k = 0, issued_q = 0;
+      int g = find_group(S.prefix, NG, u0);
+      int cur_g = -1, ng = -1, k = 0, issued_q = 0;
       bool ok = true;
       for (int u = u0; u < u1 && ok; ++u, ++k) {
-        while (u >= S.prefix[q + 1]) ++q;
-        if (q != cur_q) {
-          ++nq;
-          cur_q = q;
-          const int qs = nq & 1;
-          ok = mbar_wait(&S.qempty[qs], ((nq >> 1) & 1) ^ 1, kErrQEmpty);
+        while (u >= S.prefix[g + 1]) ++g;
+        if (g != cur_g) {  // this group's q^I heads into the next q slot
+          ++ng;
+          cur_g = g;
+          const int qs = ng % C::kQSlots;
+          ok = mbar_wait(&S.qempty[qs], ((ng / C::kQSlots) & 1) ^ 1, kErrQEmpty);
           if (!ok) break;
-          uint8_t* qb = qbase + qs * kQBytes;
-          mbar_arrive_expect_tx(&S.qfull[qs], kQBytes);
-          tma_load_2d(qb, &tm_q, 0, q * kHeads, &S.qfull[qs]);
-          tma_load_2d(qb + kQAtomBytes, &tm_q, 64, q * kHeads, &S.qfull[qs]);
-          issued_q = nq + 1;
+          uint8_t* qb = qbase + qs * C::kQSlotBytes;
+          mbar_arrive_expect_tx(&S.qfull[qs], C::kQSlotBytes);
+          tma_load_2d(qb, &tm_q, 0, S.gfirst[g] * kHeads, &S.qfull[qs]);
+          tma_load_2d(qb + C::kQAtomBytes, &tm_q, 64, S.gfirst[g] * kHeads, &S.qfull[qs]);
+          issued_q = ng + 1;
         }
-        const int tile = u - S.prefix[q];
-        const int b = (p.q0 + q) / p.T;
+        const int tile = u - S.prefix[g];
+        const int b = (p.q0 + S.gfirst[g]) / p.T;
         const int32_t row = (int32_t)(b * p.n_cap + (int64_t)tile * kTileKeys);
         if (kFp8) {
           const int s = k % kStg;
@@ -222,8 +267,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&S.stg_full[s], kStgBytes);
           tma_load_2d(stgbase + s * kStgBytes, &tm_k, 0, row, &S.stg_full[s]);
         } else {
-          const int o = k % kOpN;
-          ok = mbar_wait(&S.op_empty[o], ((k / kOpN) & 1) ^ 1, kErrOpEmpty);
+          const int o = k % C::kOpN;
+          ok = mbar_wait(&S.op_empty[o], ((k / C::kOpN) & 1) ^ 1, kErrOpEmpty);
           if (!ok) break;
           uint8_t* ob = opbase + o * kOpBytes;
           mbar_arrive_expect_tx(&S.op_full[o], kOpBytes);
@@ -232,46 +277,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // drain: no copy into this CTA's shared memory may still be in flight at exit
-      const int ring = kFp8 ? kStg : kOpN;
+      const int ring = kFp8 ? kStg : C::kOpN;
       for (int j = (k > ring ? k - ring : 0); j < k; ++j) {
         if (kFp8)
           mbar_wait(&S.stg_full[j % kStg], (uint32_t)((j / kStg) & 1), kErrStgFull);
         else
-          mbar_wait(&S.op_full[j % kOpN], (uint32_t)((j / kOpN) & 1), kErrOpFull);
+          mbar_wait(&S.op_full[j % C::kOpN], (uint32_t)((j / C::kOpN) & 1), kErrOpFull);
       }
-      for (int j = (issued_q > 2 ? issued_q - 2 : 0); j < issued_q; ++j)
-        mbar_wait(&S.qfull[j & 1], (uint32_t)((j >> 1) & 1), kErrQFull);
+      for (int j = (issued_q > C::kQSlots ? issued_q - C::kQSlots : 0); j < issued_q; ++j)
+        mbar_wait(&S.qfull[j % C::kQSlots], (uint32_t)((j / C::kQSlots) & 1), kErrQFull);
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer (one lane) ------------------------------
     if (lane == 0) {
-      const uint32_t idesc = idesc_f16(1, kTileKeys, kHeads);  // bf16, M = 128, N = 64, K-major
+      const uint32_t idesc = idesc_f16(1, kTileKeys, 64 * G);  // bf16, M = 128, N = 64 G
       const uint32_t op_s = smem_u32(opbase), q_s = smem_u32(qbase);
-      int q = u0 < u1 ? find_query(S.prefix, p.Q, u0) : 0;
-      int cur_q = -1, nq = -1, k = 0;
+      int g = u0 < u1 ? find_group(S.prefix, NG, u0) : 0;
+      int cur_g = -1, ng = -1, k = 0;
       bool ok = true;
       for (int u = u0; u < u1 && ok; ++u, ++k) {
-        while (u >= S.prefix[q + 1]) ++q;
-        if (q != cur_q) {
-          if (cur_q >= 0) mma_commit(&S.qempty[nq & 1]);  // old slot free once its MMAs end
-          ++nq;
-          cur_q = q;
-          ok = mbar_wait(&S.qfull[nq & 1], (nq >> 1) & 1, kErrQFull);
+        while (u >= S.prefix[g + 1]) ++g;
+        if (g != cur_g) {
+          if (cur_g >= 0) mma_commit(&S.qempty[ng % C::kQSlots]);  // free once its MMAs end
+          ++ng;
+          cur_g = g;
+          ok = mbar_wait(&S.qfull[ng % C::kQSlots], (ng / C::kQSlots) & 1, kErrQFull);
           if (!ok) break;
         }
-        const int o = k % kOpN, a = k % kAcc;
-        ok = mbar_wait(&S.op_full[o], (uint32_t)(k / kOpN) & 1, kErrOpFull);
+        const int o = k % C::kOpN, a = k % C::kAccN;
+        ok = mbar_wait(&S.op_full[o], (uint32_t)(k / C::kOpN) & 1, kErrOpFull);
         if (!ok) break;
-        ok = mbar_wait(&S.tempty[a], ((uint32_t)(k / kAcc) & 1) ^ 1, kErrTEmpty);
+        ok = mbar_wait(&S.tempty[a], ((uint32_t)(k / C::kAccN) & 1) ^ 1, kErrTEmpty);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t ob = op_s + o * kOpBytes, qb = q_s + (nq & 1) * kQBytes;
+        const uint32_t ob = op_s + o * kOpBytes, qb = q_s + (ng % C::kQSlots) * C::kQSlotBytes;
 #pragma unroll
         for (int kk = 0; kk < kDim / 16; ++kk) {  // K = 128 in steps of 16
           const uint32_t atom = kk >> 2, koff = (kk & 3) * 32;
           const uint64_t ad = smem_desc(ob + atom * kAtomBytes + koff, 16, 1024, kLayoutSw128);
-          const uint64_t bd = smem_desc(qb + atom * kQAtomBytes + koff, 16, 1024, kLayoutSw128);
-          mma_f16(tmem + 64u * a, ad, bd, idesc, kk > 0 ? 1u : 0u);
+          const uint64_t bd = smem_desc(qb + atom * C::kQAtomBytes + koff, 16, 1024, kLayoutSw128);
+          mma_f16(tmem + (uint32_t)C::kAccCols * a, ad, bd, idesc, kk > 0 ? 1u : 0u);
         }
         mma_commit(&S.op_empty[o]);
         mma_commit(&S.tfull[a]);
@@ -280,98 +325,123 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&S.done, 0, kErrTFull);
     }
     __syncwarp();
-  } else if (warp < 6) {
+  } else if (kFp8 && warp < 6) {
     // ------------------------------ converters (fp8) ------------------------------
-    if (kFp8) {
-      const int ct = threadIdx.x - 64;  // 0..127
-      bool ok = true;
-      for (int u = u0, k = 0; u < u1 && ok; ++u, ++k) {
-        const int s = k % kStg, o = k % kOpN;
-        ok = group_all_ok<3>(mbar_wait(&S.stg_full[s], (uint32_t)(k / kStg) & 1, kErrStgFull) &&
-                             mbar_wait(&S.op_empty[o], ((uint32_t)(k / kOpN) & 1) ^ 1, kErrOpEmpty));
-        if (!ok) break;
-        const uint8_t* src = stgbase + s * kStgBytes;
-        uint8_t* dst = opbase + o * kOpBytes;
-        // a warp converts 4 rows per step: lane = (row % 4, 16-byte input chunk of 8)
-        const int rsub = (ct & 31) >> 3, ic = ct & 7;
+    const int ct = threadIdx.x - 64;  // 0..127
+    bool ok = true;
+    for (int u = u0, k = 0; u < u1 && ok; ++u, ++k) {
+      const int s = k % kStg, o = k % C::kOpN;
+      ok = group_all_ok<3, 128>(
+          mbar_wait(&S.stg_full[s], (uint32_t)(k / kStg) & 1, kErrStgFull) &&
+          mbar_wait(&S.op_empty[o], ((uint32_t)(k / C::kOpN) & 1) ^ 1, kErrOpEmpty));
+      if (!ok) break;
+      const uint8_t* src = stgbase + s * kStgBytes;
+      uint8_t* dst = opbase + o * kOpBytes;
+      // a warp converts 4 rows per step: lane = (row % 4, 16-byte input chunk of 8)
+      const int rsub = (ct & 31) >> 3, ic = ct & 7;
 #pragma unroll 4
-        for (int r0 = 4 * (ct >> 5); r0 < kTileKeys; r0 += 16) {
-          const int r = r0 + rsub;
-          const uint4 raw = *reinterpret_cast<const uint4*>(src + r * kDim + 16 * ic);
-          const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-          uint32_t o8[8];
+      for (int r0 = 4 * (ct >> 5); r0 < kTileKeys; r0 += 16) {
+        const int r = r0 + rsub;
+        const uint4 raw = *reinterpret_cast<const uint4*>(src + r * kDim + 16 * ic);
+        const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+        uint32_t o8[8];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            o8[2 * j] = e4m3x2_to_bf16x2((uint16_t)(w4[j] & 0xffffu));
-            o8[2 * j + 1] = e4m3x2_to_bf16x2((uint16_t)(w4[j] >> 16));
-          }
-          // dims 16*ic .. 16*ic+15 -> atom ic / 4, output chunks 2*(ic % 4), +1
-          uint8_t* at = dst + (ic >> 2) * kAtomBytes;
-          const int c8 = 2 * (ic & 3);
-          *reinterpret_cast<uint4*>(at + sw128(r, c8)) = make_uint4(o8[0], o8[1], o8[2], o8[3]);
-          *reinterpret_cast<uint4*>(at + sw128(r, c8 + 1)) = make_uint4(o8[4], o8[5], o8[6], o8[7]);
+        for (int j = 0; j < 4; ++j) {
+          o8[2 * j] = e4m3x2_to_bf16x2((uint16_t)(w4[j] & 0xffffu));
+          o8[2 * j + 1] = e4m3x2_to_bf16x2((uint16_t)(w4[j] >> 16));
         }
-        fence_proxy_async_smem();  // the operand tile is read by the tensor cores
-        mbar_arrive(&S.op_full[o]);
-        mbar_arrive(&S.stg_empty[s]);
+        // dims 16*ic .. 16*ic+15 -> atom ic / 4, output chunks 2*(ic % 4), +1
+        uint8_t* at = dst + (ic >> 2) * kAtomBytes;
+        const int c8 = 2 * (ic & 3);
+        *reinterpret_cast<uint4*>(at + sw128(r, c8)) = make_uint4(o8[0], o8[1], o8[2], o8[3]);
+        *reinterpret_cast<uint4*>(at + sw128(r, c8 + 1)) = make_uint4(o8[4], o8[5], o8[6], o8[7]);
       }
+      fence_proxy_async_smem();  // the operand tile is read by the tensor cores
+      mbar_arrive(&S.op_full[o]);
+      mbar_arrive(&S.stg_empty[s]);
     }
-  } else {
+  } else if (warp >= C::kEpiWarp0) {
     // ------------------------------ epilogue ------------------------------
+    // G = 1: warps 6-9, one query; G = 4: warps 2-9, group e = members 2e, 2e+1
+    constexpr int kPer = G == 1 ? 1 : 2;  // members per epilogue thread
+    const int et = threadIdx.x - 32 * C::kEpiWarp0;
+    const int e = G == 1 ? 0 : (warp - 2) >> 2;
     const int quad = warp & 3;  // TMEM lane quadrant this warp may access
-    const bool hist = p.hist != nullptr;
+    const bool hist = C::kHist && p.hist != nullptr;
     int hq = -1;
     auto flush = [&](int qq) {  // shared histogram of query qq -> global, then clear
-      epi_bar();
-      for (int i = threadIdx.x - 192; i < kBins; i += 128) {
+      epi_bar<C::kEpiThreads>();
+      for (int i = et; i < kBins; i += C::kEpiThreads) {
         const int v = S.hist[i];
         if (v) {
           atomicAdd(&p.hist[(size_t)qq * kBins + i], v);
           S.hist[i] = 0;
         }
       }
-      epi_bar();
+      epi_bar<C::kEpiThreads>();
     };
-    float wr[kHeads];
-    int cur_q = -1;
-    int q = u0 < u1 ? find_query(S.prefix, p.Q, u0) : 0;
+    float wr[G == 1 ? kHeads : 1];  // G = 1: the query's head weights in registers
+    int cur_g = -1;
+    int g = u0 < u1 ? find_group(S.prefix, NG, u0) : 0;
     bool ok = true;
     for (int u = u0, k = 0; u < u1 && ok; ++u, ++k) {
-      while (u >= S.prefix[q + 1]) ++q;
-      const int tile = u - S.prefix[q];
-      if (q != cur_q) {
+      while (u >= S.prefix[g + 1]) ++g;
+      const int tile = u - S.prefix[g];
+      const int f = S.gfirst[g], gs = gsize(g);
+      if (g != cur_g) {
+        if (G == 1) {
 #pragma unroll
-        for (int h = 0; h < kHeads; ++h) wr[h] = p.w[(size_t)q * kHeads + h];
-        cur_q = q;
+          for (int h = 0; h < (G == 1 ? kHeads : 1); ++h) wr[h] = p.w[(size_t)f * kHeads + h];
+        } else {
+          epi_bar<C::kEpiThreads>();  // every thread is done with the previous weights
+          for (int i = et; i < G * kHeads; i += C::kEpiThreads) {
+            const int mq = i / kHeads;
+            S.wst[mq][i % kHeads] = mq < gs ? p.w[(size_t)(f + mq) * kHeads + i % kHeads] : 0.f;
+          }
+          epi_bar<C::kEpiThreads>();
+        }
+        cur_g = g;
       }
-      if (hist && q != hq) {
+      if (hist && f != hq) {
         if (hq >= 0) flush(hq);
-        hq = q;
+        hq = f;
       }
       const int s = tile * kTileKeys + 32 * quad + lane;
-      const int b = (p.q0 + q) / p.T;
-      const bool vis = s < S.nvis[q];
-      // the row scale is loaded before the wait, so its latency hides behind the MMAs
-      const float scale = (kFp8 && vis) ? p.key_scale[(size_t)b * p.n_cap + s] : 1.f;
-      const int a = k % kAcc;
-      ok = group_all_ok<2>(mbar_wait(&S.tfull[a], (uint32_t)(k / kAcc) & 1, kErrTFull));
+      const int b = (p.q0 + f) / p.T;
+      // the fp8 row scale is loaded before the wait, so its latency hides behind the MMAs
+      const float scale = (kFp8 && s < S.nvis[f]) ? p.key_scale[(size_t)b * p.n_cap + s] : 1.f;
+      const int a = k % C::kAccN;
+      ok = group_all_ok<2, C::kEpiThreads>(
+          mbar_wait(&S.tfull[a], (uint32_t)(k / C::kAccN) & 1, kErrTFull));
       if (!ok) break;
       tc_fence_after();
-      uint32_t v[kHeads];
-      tmem_ld_32x32b_x64(tmem + ((uint32_t)(32 * quad) << 16) + 64u * a, v);
+      uint32_t v[kPer][kHeads];
+#pragma unroll
+      for (int j = 0; j < kPer; ++j)
+        tmem_ld_32x32b_x64(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)C::kAccCols * a +
+                               64u * (kPer * e + j),
+                           v[j]);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.tempty[a]);
-      float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int hh = 0; hh < kHeads; ++hh)
-        part[hh & 3] = fmaf(wr[hh], fmaxf(__uint_as_float(v[hh]), 0.f), part[hh & 3]);
-      float sc = (part[0] + part[1]) + (part[2] + part[3]);
-      if (kFp8) sc *= scale;
-      if (vis) {
-        p.scores[(size_t)q * p.n_cap + s] = sc;
-        if (hist) atomicAdd(&S.hist[float_key(sc) >> 20], 1);
+      for (int j = 0; j < kPer; ++j) {
+        const int mq = kPer * e + j;  // member of the group
+        if (mq >= gs) continue;
+        const int q = f + mq;
+        float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int hh = 0; hh < kHeads; ++hh) {
+          const float wv = G == 1 ? wr[hh % (G == 1 ? kHeads : 1)] : S.wst[mq][hh];
+          part[hh & 3] = fmaf(wv, fmaxf(__uint_as_float(v[j][hh]), 0.f), part[hh & 3]);
+        }
+        float sc = (part[0] + part[1]) + (part[2] + part[3]);
+        if (kFp8) sc *= scale;
+        if (s < S.nvis[q]) {
+          p.scores[(size_t)q * p.n_cap + s] = sc;
+          if (hist) atomicAdd(&S.hist[float_key(sc) >> 20], 1);
+        }
       }
     }
     if (hist && hq >= 0) flush(hq);
@@ -380,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 64 * kAcc);
+    tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
@@ -436,10 +506,21 @@ int num_sms() {
   return n;
 }
 
-template <bool kFp8>
+template <bool kFp8, int G>
 size_t smem_bytes() {
-  return 1024 + (size_t)(kFp8 ? kOps : kOpsBf16) * kOpBytes + 2 * kQBytes +
-         (kFp8 ? (size_t)kStg * kStgBytes : 0) + sizeof(Smem);
+  using C = Cfg<kFp8, G>;
+  return 1024 + (size_t)C::kOpN * kOpBytes + (size_t)C::kQSlots * C::kQSlotBytes +
+         (kFp8 ? (size_t)kStg * kStgBytes : 0) + sizeof(Smem<C::kHist>);
+}
+
+template <bool kFp8, int G>
+cudaError_t launch_variant(const CUtensorMap& mk, const CUtensorMap& mq, const Bf16IdxParams& p,
+                           int grid, cudaStream_t st) {
+  const size_t smem = smem_bytes<kFp8, G>();
+  cudaError_t e = cudaFuncSetAttribute(k_index_bf16_tc<kFp8, G>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch(true, k_index_bf16_tc<kFp8, G>, dim3(grid), dim3(kThreads), smem, st, mk, mq, p);
 }
 
 }  // namespace
@@ -452,23 +533,21 @@ bool index_bf16_tc_supported(const IndexArgs& a) {
 cudaError_t launch_index_bf16_tc(const IndexArgs& a, cudaStream_t st) {
   const int Qall = a.B * a.T;
   const bool fp8 = a.kdt == CSA_FP8_E4M3_ROWSCALE;
+  // four queries of a request per MMA (N = 256) when several share the keys and no per-query
+  // histogram is wanted (bf16 keys, prefill); otherwise one
+  const bool grouped = !fp8 && a.hist == nullptr && a.T >= 4;
   CUtensorMap mk;
   const bool good = fp8 ? make_map_fp8_rows(&mk, a.KI, (uint64_t)a.B * a.n_cap)
                         : make_map_bf16_rows(&mk, a.KI, (uint64_t)a.B * a.n_cap, kTileKeys);
   if (!good) return cudaErrorInvalidValue;
-  const size_t smem = fp8 ? smem_bytes<true>() : smem_bytes<false>();
-  cudaError_t e = fp8 ? cudaFuncSetAttribute(k_index_bf16_tc<true>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
-                      : cudaFuncSetAttribute(k_index_bf16_tc<false>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
   timing_before(st);
-  // queries in launches of at most kMaxQueries (each launch walks its queries' tiles)
+  // queries in launches of at most kMaxQueries (each launch walks its groups' tiles)
   for (int q0 = 0; q0 < Qall && e == cudaSuccess; q0 += kMaxQueries) {
     const int Q = Qall - q0 < kMaxQueries ? Qall - q0 : kMaxQueries;
     CUtensorMap mq;
     const auto* qI = static_cast<const __nv_bfloat16*>(a.qI) + (size_t)q0 * kHeads * kDim;
-    if (!make_map_bf16_rows(&mq, qI, (uint64_t)Q * kHeads, kHeads)) {
+    if (!make_map_bf16_rows(&mq, qI, (uint64_t)Q * kHeads, grouped ? 4 * kHeads : kHeads)) {
       e = cudaErrorInvalidValue;
       break;
     }
@@ -478,8 +557,9 @@ cudaError_t launch_index_bf16_tc(const IndexArgs& a, cudaStream_t st) {
                     a.hist ? a.hist + (size_t)q0 * kBins : nullptr};
     const int64_t tiles_max = (int64_t)Q * (a.n_cap / kTileKeys);
     const int grid = (int)(tiles_max < num_sms() ? (tiles_max > 0 ? tiles_max : 1) : num_sms());
-    e = fp8 ? launch(true, k_index_bf16_tc<true>, dim3(grid), dim3(kThreads), smem, st, mk, mq, p)
-            : launch(true, k_index_bf16_tc<false>, dim3(grid), dim3(kThreads), smem, st, mk, mq, p);
+    e = fp8       ? launch_variant<true, 1>(mk, mq, p, grid, st)
+        : grouped ? launch_variant<false, 4>(mk, mq, p, grid, st)
+                  : launch_variant<false, 1>(mk, mq, p, grid, st);
   }
   timing_after(st);
   return e;
