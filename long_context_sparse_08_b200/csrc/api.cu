@@ -467,7 +467,7 @@ csa_status csa_forward(const csa_params* p, csa_dtype io, int32_t B, int32_t T,
   csa::TopkArgs t{};
   t.B = B; t.T = T; t.m = p->m; t.k = p->topk; t.n_cap = a->N_cap; t.scores = scores;
   t.q_pos = a->q_pos; t.out_idx = a->out_idx;
-  if (io == CSA_BF16 && forward_qhat(p, B, T, a->N_cap)) {
+  if (io == CSA_BF16 && p->rope_dims <= 128 && forward_qhat(p, B, T, a->N_cap)) {
     t.qj.q = a->q;
     t.qj.q_rms_w = a->q_rms_w;
     t.qj.qhat = base + sb + tb + mb;
@@ -475,6 +475,8 @@ csa_status csa_forward(const csa_params* p, csa_dtype io, int32_t B, int32_t T,
     t.qj.r = p->rope_dims;
     t.qj.eps = p->rms_eps;
     t.qj.rope_base = p->rope_base;
+    for (int i = 0; i < p->rope_dims / 2; ++i)
+      t.qj.inv_freq[i] = csa::rope_inv_freq(i, p->rope_dims, (double)p->rope_base);
     ma.qhat = t.qj.qhat;
   }
   TRY(index_then_topk(p, a->idx_dtype, B, T, a->N_cap, a->qI, a->qI_scale, a->w, a->KI,

@@ -66,6 +66,7 @@ struct QhatJob {
   void* qhat;           // bf16 [B*T][H][c]; nullptr: no job
   int H, r;
   float eps, rope_base;
+  double inv_freq[64];  // RoPE pair frequencies, formed on the host (r <= 128)
 };
 
 struct TopkArgs {

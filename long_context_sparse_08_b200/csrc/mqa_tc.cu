@@ -573,41 +573,44 @@ __global__ void __launch_bounds__(256) k_mqa_combine(MqaTcParams P) {
   const size_t stride = kHg * (kC + 2);
   const float* base = P.part + (size_t)stream * P.nsplit * stride;
   constexpr int kMaxSplit = 32;  // choose_nsplit never exceeds this
-  constexpr int kGroup = 8;      // splits whose partial rows are loaded together
-  float ms[kMaxSplit];
+  constexpr int kFirst = 16;     // splits whose (m, l, O) loads go out in the first round
+  const int ns = P.nsplit;
+  const int d = 2 * tid;
+  float ms[kMaxSplit], lv[kFirst];
+  float2 ov[kFirst];
+#pragma unroll
+  for (int sp = 0; sp < kMaxSplit; ++sp) ms[sp] = sp < ns ? base[sp * stride + h] : -INFINITY;
+#pragma unroll
+  for (int sp = 0; sp < kFirst; ++sp) {  // issued before the max is known: one round trip
+    const float* pp = base + sp * stride;
+    lv[sp] = sp < ns ? pp[kHg + h] : 0.f;
+    ov[sp] = sp < ns ? *reinterpret_cast<const float2*>(pp + 2 * kHg + (size_t)h * kC + d)
+                     : make_float2(0.f, 0.f);
+  }
   float M = -INFINITY;
 #pragma unroll
-  for (int sp = 0; sp < kMaxSplit; ++sp) {
-    ms[sp] = sp < P.nsplit ? base[sp * stride + h] : -INFINITY;
-    M = fmaxf(M, ms[sp]);
-  }
+  for (int sp = 0; sp < kMaxSplit; ++sp) M = fmaxf(M, ms[sp]);
   const float zs = a.sink ? a.sink[g * kHg + h] : -INFINITY;
   const float Mt = fmaxf(M, zs);
   float l = 0.f, o0 = 0.f, o1 = 0.f;
-  const int d = 2 * tid;
 #pragma unroll
-  for (int s0 = 0; s0 < kMaxSplit; s0 += kGroup) {
-    if (s0 >= P.nsplit) break;
-    float lv[kGroup];
-    float2 ov[kGroup];
-#pragma unroll
-    for (int j = 0; j < kGroup; ++j) {  // every load of the group in flight at once
-      const int sp = s0 + j;
-      const bool use = sp < P.nsplit && ms[sp] != -INFINITY;
-      const float* pp = base + sp * stride;
-      lv[j] = use ? pp[kHg + h] : 0.f;
-      ov[j] = use ? *reinterpret_cast<const float2*>(pp + 2 * kHg + (size_t)h * kC + d)
-                  : make_float2(0.f, 0.f);
+  for (int sp = 0; sp < kFirst; ++sp) {  // fixed split order: deterministic
+    if (sp < ns && ms[sp] != -INFINITY) {
+      const float f = expf(ms[sp] - Mt);
+      l = fmaf(lv[sp], f, l);
+      o0 = fmaf(ov[sp].x, f, o0);
+      o1 = fmaf(ov[sp].y, f, o1);
     }
-#pragma unroll
-    for (int j = 0; j < kGroup; ++j) {  // fixed split order: deterministic
-      const int sp = s0 + j;
-      if (sp < P.nsplit && ms[sp] != -INFINITY) {
-        const float f = expf(ms[sp] - Mt);
-        l = fmaf(lv[j], f, l);
-        o0 = fmaf(ov[j].x, f, o0);
-        o1 = fmaf(ov[j].y, f, o1);
-      }
+  }
+  for (int sp = kFirst; sp < ns; ++sp) {  // more splits than the first round covers
+    const float* pp = base + sp * stride;
+    const float m = pp[h];  // reloaded: indexing ms here would put it in local memory
+    if (m != -INFINITY) {
+      const float f = expf(m - Mt);
+      l = fmaf(pp[kHg + h], f, l);
+      const float2 o = *reinterpret_cast<const float2*>(pp + 2 * kHg + (size_t)h * kC + d);
+      o0 = fmaf(o.x, f, o0);
+      o1 = fmaf(o.y, f, o1);
     }
   }
   float y0 = 0.f, y1 = 0.f;

@@ -172,8 +172,7 @@ __device__ void qhat_rows(const QhatJob& j, int q, double t, int h0, int h1, flo
   constexpr int kC = 512;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int r = j.r, r0 = kC - r;
-  for (int p = tid; p < r / 2; p += blockDim.x)
-    rope_cos_sin(t, p, r, (double)j.rope_base, &cs[p], &sn[p]);
+  for (int p = tid; p < r / 2; p += blockDim.x) rope_angle_cs(t, j.inv_freq[p], &cs[p], &sn[p]);
   __syncthreads();
   for (int h = h0 + wid; h < h1; h += kWarps) {
     const uint4* src = reinterpret_cast<const uint4*>(j.q) + ((size_t)q * j.H + h) * (kC / 8);
