@@ -80,6 +80,14 @@ def algorithmic_bytes_per_query(s, n_vis: int) -> dict:
     return {"index": idx, "total": idx + att}
 
 
+def workload_config(s, l2: str, parallelism: str) -> dict:
+    """The `config` object of a bench line: the workload and its sizes (both arms)."""
+    n_vis = min(s.ctx // s.m, s.n_cap) if s.kind != "csa_prefill" else s.n_cap
+    return {"workload": s.name, "B_per_gpu": s.B, "T": s.T, "ctx": s.ctx, "entries": n_vis,
+            "heads": s.n_heads, "c": s.c, "topk": s.topk, "indexer_keys": s.idx,
+            "n_win": s.n_win, "l2": l2, "parallelism": parallelism}
+
+
 def prefill_flops(s) -> dict:
     """Indexer: 2 * H_I * d_I per visible (t, s) pair; attention: 4 * c flops per head per
     attended row (q.k and p.v), rows = min(k, visible) + window."""
@@ -298,12 +306,10 @@ def run_ours(args, W, rank, world, local_rank):
         "dtype": {"mxfp4": "mxfp4+bf16", "fp8": "e4m3+bf16", "bf16": "bf16",
                   "none": "bf16", "f32": "f32"}[s.idx],
         "data": "synthetic (seeded N(0,1); shapes of the Pro/Flash configs)",
-        "config": {"workload": s.name, "B_per_gpu": s.B, "T": s.T, "ctx": s.ctx,
-                   "entries": n_vis, "heads": s.n_heads, "c": s.c, "topk": s.topk,
-                   "indexer_keys": s.idx, "n_win": s.n_win,
-                   "l2": f"{R_rep} rotating input replicas ({R_rep * one_set / 1e9:.2f} GB); "
-                         f"bytes touched per cycle {R_rep * step_bytes / 1e6:.0f} MB > L2",
-                   "parallelism": f"replicas x{world} (independent requests)"},
+        "config": workload_config(
+            s, l2=f"{R_rep} rotating input replicas ({R_rep * one_set / 1e9:.2f} GB); "
+                  f"bytes touched per cycle {R_rep * step_bytes / 1e6:.0f} MB > L2",
+            parallelism=f"replicas x{world} (independent requests)"),
         "step_hbm_roofline": {"alg_bytes_per_step": step_bytes,
                               "frac_of_peak": round(step_bytes / (ms / K / 1e3) / 1e9 /
                                                     peaks["hbm_gbs"], 4)},
@@ -396,7 +402,9 @@ def main():
             "ms_per_step": round(1e3 * el / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded N(0,1); shapes of the Pro/Flash configs)",
-            "config": {"workload": s.name, "sample": "one query of the batch per step"},
+            "config": workload_config(s, l2="host memory (float64 oracle)",
+                                      parallelism="oracle on the host cores; "
+                                                  "one query of the batch per step"),
             "cpu_baseline": {"value": round(v, 4), "unit": "queries/s", "cores": cores,
                              "kind": "oracle", "sample": "one query per step"},
             "e2e": {"value": round(v, 4), "unit": "queries/s", "h2d_bytes_per_step": 0,
