@@ -21,6 +21,11 @@
 // O^T and l are rescaled); exp(s - m) <= e^8 otherwise, exactly as correct.
 // One split: the CTA finalises (sink, RoPE(-t), bf16). Several: it writes (m, l, O)
 // partials and k_mqa_combine merges them in a fixed order (deterministic).
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 #include "tc.cuh"
@@ -67,6 +72,7 @@ struct MqaTcParams {
   int G;       // head groups (H / 64)
   int nsplit;  // CTAs per stream
   float* part; // partials [stream][split][64 * (kC + 2)] or nullptr
+  int tma_kv, tma_win;  // tensor maps usable for chunks of contiguous cache / window rows
   double inv_freq[kMaxPairs];  // RoPE pair frequencies base^(-2p/r), formed once on the host
 };
 
@@ -210,7 +216,9 @@ __device__ __forceinline__ int reduce16_index(int lane) {
   return ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
 }
 
-__global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
+__global__ void __launch_bounds__(kThreads, 1)
+    k_mqa_tc(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_win,
+             MqaTcParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -229,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
 
   if (warp == 4) {
     if (lane == 0) {
-      mbar_init(&S.kv_full, 128);
+      mbar_init(&S.kv_full, 129);  // the 128 loading threads + the TMA issue or its stand-in
       mbar_init(&S.s_full, 1);
       mbar_init(&S.p_full, 128);
       mbar_init(&S.kv_free, 1);
@@ -348,21 +356,46 @@ __global__ void __launch_bounds__(kThreads, 1) k_mqa_tc(MqaTcParams P) {
       S.src[tid] = my_src;
       const uint32_t vb = __ballot_sync(0xffffffffu, my_src != nullptr);
       if (lane == 0) S.vmask[warp] = vb;
-      bar_softmax();
-#pragma unroll 4
-      for (int rr = warp; rr < kRows; rr += 4) {
-        const __nv_bfloat16* src = S.src[rr];
-#pragma unroll
-        for (int hseg = 0; hseg < 2; ++hseg) {
-          const int gch = lane + 32 * hseg;  // 16-byte chunk of the 1 KB row
-          const int atom = gch >> 3, c = gch & 7;
-          const uint32_t dst = kv_base + atom * (kRows * 128) + sw128(rr, c);
-          cp_async16(dst, src ? src + 8 * gch : static_cast<const __nv_bfloat16*>(a.kv),
-                     src != nullptr);
+      // a chunk of 128 contiguous rows (dense entries, or window rows) comes by TMA: eight
+      // 128B-swizzled boxes issued by one thread instead of 64 cp.async per thread
+      const int64_t r0 = (int64_t)j * kRows;
+      const CUtensorMap* tmap = nullptr;
+      int32_t trow = 0;
+      if (P.tma_kv && a.k == 0 && r0 + kRows <= rl.n_vis) {
+        tmap = &tm_kv;
+        trow = (int32_t)((int64_t)b * a.n_cap + r0);
+      } else if (P.tma_win && r0 >= rl.n_sel && r0 + kRows <= rl.L) {
+        const int64_t rr0 = rl.lo + (r0 - rl.n_sel) - a.win_pos0[b];
+        if (rr0 >= 0 && rr0 + kRows <= a.l_raw) {
+          tmap = &tm_win;
+          trow = (int32_t)((int64_t)b * a.l_raw + rr0);
         }
       }
-      cp_async_wait_all();
-      fence_proxy_async_smem();
+      bar_softmax();
+      if (tmap != nullptr) {
+        if (tid == 0) {
+          mbar_arrive_expect_tx(&S.kv_full, kRows * kC * 2);
+#pragma unroll
+          for (int atom = 0; atom < kAtoms; ++atom)
+            tma_load_2d(base + kOffKV + atom * (kRows * 128), tmap, 64 * atom, trow, &S.kv_full);
+        }
+      } else {
+#pragma unroll 4
+        for (int rr = warp; rr < kRows; rr += 4) {
+          const __nv_bfloat16* src = S.src[rr];
+#pragma unroll
+          for (int hseg = 0; hseg < 2; ++hseg) {
+            const int gch = lane + 32 * hseg;  // 16-byte chunk of the 1 KB row
+            const int atom = gch >> 3, c = gch & 7;
+            const uint32_t dst = kv_base + atom * (kRows * 128) + sw128(rr, c);
+            cp_async16(dst, src ? src + 8 * gch : static_cast<const __nv_bfloat16*>(a.kv),
+                       src != nullptr);
+          }
+        }
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+        if (tid == 0) mbar_arrive(&S.kv_full);  // stands in for the TMA issue
+      }
       mbar_arrive(&S.kv_full);
 
       // ---- softmax: lanes 0-15 of warp w own heads 16w .. 16w+15 (the M = 64 accumulator
@@ -632,6 +665,33 @@ __global__ void __launch_bounds__(256) k_mqa_combine(MqaTcParams P) {
   *reinterpret_cast<__nv_bfloat162*>(out) = __floats2bfloat162_rn(y0, y1);
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// bf16 rows of c = 512 values; box = one 128B swizzle atom (64 values) x 128 rows
+bool make_map_rows(CUtensorMap* m, const void* ptr, int64_t rows) {
+  auto fn = encode_fn();
+  if (!fn || ptr == nullptr || rows < kRows || rows >= (1ll << 31)) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kC, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kC * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kRows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int sm_count() {
   static int n = 0;
   if (n == 0) {
@@ -678,6 +738,11 @@ cudaError_t launch_mqa_tc(const MqaArgs& a, void* ws, size_t ws_bytes, cudaStrea
   P.part = P.nsplit > 1 ? static_cast<float*>(ws) : nullptr;
   for (int p = 0; p < kMaxPairs; ++p)
     P.inv_freq[p] = p < a.rope_dims / 2 ? rope_inv_freq(p, a.rope_dims, (double)a.rope_base) : 0.0;
+  CUtensorMap tm_kv, tm_win;
+  memset(&tm_kv, 0, sizeof(tm_kv));
+  memset(&tm_win, 0, sizeof(tm_win));
+  P.tma_kv = make_map_rows(&tm_kv, a.kv, (int64_t)a.B * a.n_cap) ? 1 : 0;
+  P.tma_win = make_map_rows(&tm_win, a.win, (int64_t)a.B * a.l_raw) ? 1 : 0;
   if (P.nsplit > 1 && ws_bytes < mqa_tc_workspace_bytes(a)) return cudaErrorInvalidValue;
   const int64_t streams = (int64_t)a.B * a.T * P.G;
   const size_t smem = 1024 + kOffEnd + sizeof(Smem);
@@ -685,7 +750,7 @@ cudaError_t launch_mqa_tc(const MqaArgs& a, void* ws, size_t ws_bytes, cudaStrea
                                        (int)smem);
   if (e != cudaSuccess) return e;
   e = launch(a.chained, k_mqa_tc, dim3((unsigned)(streams * P.nsplit)), dim3(kThreads), smem, st,
-             P);
+             tm_kv, tm_win, P);
   if (e != cudaSuccess || P.nsplit == 1) return e;
   return launch(true, k_mqa_combine, dim3((unsigned)streams, kHg), dim3(256), 0, st, P);
 }
