@@ -171,12 +171,12 @@ csa_status check_index_args(const csa_params* p, csa_dtype kdt, int32_t B, int32
   return CSA_OK;
 }
 
-// csa_forward with the decode selector and the tensor-core attention: the selector also
-// prepares the attention's q_hat (bf16 [B*T][H][c]) in the workspace
+// csa_forward with the tensor-core attention: the top-k kernel also prepares the
+// attention's q_hat (bf16 [B*T][H][c]) in the workspace
 bool forward_qhat(const csa_params* p, int32_t B, int32_t T, int64_t N_cap) {
   csa::MqaArgs m = make_mqa(p, B, T, nullptr, nullptr, nullptr, N_cap, nullptr, p->topk, nullptr,
                             0, nullptr, nullptr, nullptr, nullptr);
-  return csa::topk_decode_path(B, T, N_cap, p->topk) && csa::mqa_tc_supported(m, true);
+  return csa::mqa_tc_supported(m, true) && p->rope_dims <= 128;
 }
 size_t qhat_bytes(const csa_params* p, int32_t B, int32_t T, int64_t N_cap) {
   return forward_qhat(p, B, T, N_cap)
@@ -462,12 +462,15 @@ csa_status csa_forward(const csa_params* p, csa_dtype io, int32_t B, int32_t T,
   float* scores = a->out_scores ? a->out_scores : reinterpret_cast<float*>(base);
   auto ma = make_mqa(p, B, T, a->q, a->q_pos, a->kv_cache, a->N_cap, a->out_idx, p->topk,
                      a->win_kv, a->L_raw, a->win_pos0, a->sink, a->q_rms_w, a->out);
-  ma.chained = true;  // a top-k kernel of this library precedes it on the stream
+  // the decode selector's last kernel (rank) waited for the filter, which wrote q_hat, so the
+  // attention may copy q_hat before its own wait; after the one-kernel row selector, which
+  // writes q_hat itself, it is launched the ordinary way
+  ma.chained = csa::topk_decode_path(B, T, a->N_cap, p->topk);
   const size_t mb = round_up(csa::mqa_workspace_bytes(ma));
   csa::TopkArgs t{};
   t.B = B; t.T = T; t.m = p->m; t.k = p->topk; t.n_cap = a->N_cap; t.scores = scores;
   t.q_pos = a->q_pos; t.out_idx = a->out_idx;
-  if (io == CSA_BF16 && p->rope_dims <= 128 && forward_qhat(p, B, T, a->N_cap)) {
+  if (io == CSA_BF16 && forward_qhat(p, B, T, a->N_cap)) {
     t.qj.q = a->q;
     t.qj.q_rms_w = a->q_rms_w;
     t.qj.qhat = base + sb + tb + mb;

@@ -10,6 +10,7 @@
 // (lowest-index) keys == T, and a bitonic sort of the k (key, index) pairs orders them.
 #include "common.cuh"
 #include "internal.h"
+#include "qhat.cuh"
 
 namespace csa {
 
@@ -72,6 +73,11 @@ __global__ void __launch_bounds__(kThreads) k_topk_rows(TopkArgs a) {
   __shared__ int sel_above;
   const int bt = blockIdx.x;
   const int64_t t = a.q_pos[bt];
+  if (a.qj.qhat != nullptr) {  // side job: this row's query heads for the attention
+    __shared__ float s_cs[256], s_sn[256];
+    qhat_rows(a.qj, bt, (double)t, 0, a.qj.H, s_cs, s_sn);
+    __syncthreads();
+  }
   const int64_t n = t < 0 ? 0 : (t / a.m < a.n_cap ? t / a.m : a.n_cap);
   const float* sc = a.scores + (size_t)bt * a.n_cap;
   int32_t* out = a.out_idx + (size_t)bt * a.k;

@@ -19,6 +19,7 @@
 //    sorts the winners. Either way the result depends on the scores only.
 #include "common.cuh"
 #include "internal.h"
+#include "qhat.cuh"
 
 namespace csa {
 
@@ -163,64 +164,6 @@ __global__ void __launch_bounds__(256) k_zero(int4* p0, int n0, int4* p1, int n1
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n0 + n1; i += gridDim.x * blockDim.x) {
     if (i < n0) p0[i] = make_int4(0, 0, 0, 0);
     else p1[i - n0] = make_int4(0, 0, 0, 0);
-  }
-}
-
-// The side job: q_hat rows of query q for heads [h0, h1), one warp per head, lane = 16 of
-// the 512 dims. Reads only caller inputs, so it runs before the dependency wait.
-__device__ void qhat_rows(const QhatJob& j, int q, double t, int h0, int h1, float* cs, float* sn) {
-  constexpr int kC = 512;
-  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  const int r = j.r, r0 = kC - r;
-  for (int p = tid; p < r / 2; p += blockDim.x) rope_angle_cs(t, j.inv_freq[p], &cs[p], &sn[p]);
-  __syncthreads();
-  for (int h = h0 + wid; h < h1; h += kWarps) {
-    const uint4* src = reinterpret_cast<const uint4*>(j.q) + ((size_t)q * j.H + h) * (kC / 8);
-    uint4* dst = reinterpret_cast<uint4*>(j.qhat) + ((size_t)q * j.H + h) * (kC / 8);
-    float x[16];
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const uint4 raw = src[lane + 32 * half];
-      const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        x[8 * half + 2 * k] = __uint_as_float(w4[k] << 16);
-        x[8 * half + 2 * k + 1] = __uint_as_float(w4[k] & 0xffff0000u);
-      }
-    }
-    float ss = 0.f;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) ss = fmaf(x[k], x[k], ss);
-    ss = warp_sum(ss);
-    const float rstd = rsqrtf(ss / (float)kC + j.eps);
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int d0 = 8 * (lane + 32 * half);
-      float y[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float wgt = j.q_rms_w ? __bfloat162float(static_cast<const __nv_bfloat16*>(
-                                          j.q_rms_w)[d0 + k])
-                                    : 1.f;
-        y[k] = x[8 * half + k] * rstd * wgt;
-      }
-      if (d0 >= r0) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int p = (d0 + 2 * k - r0) >> 1;
-          const float c = cs[p], s = sn[p], u = y[2 * k], v = y[2 * k + 1];
-          y[2 * k] = u * c - v * s;
-          y[2 * k + 1] = u * s + v * c;
-        }
-      }
-      uint4 o;
-      uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        ow[k] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * k])) |
-                ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * k + 1])) << 16);
-      dst[lane + 32 * half] = o;
-    }
   }
 }
 
