@@ -6,8 +6,10 @@
 //
 // One CTA of 1024 threads per query row: an MSB-first radix select on order-preserving
 // 32-bit keys (4 passes of 8 bits, histograms in shared memory) finds the k-th largest
-// key T; a block-wide scan in index order then gathers every key > T and the first
-// (lowest-index) keys == T, and a bitonic sort of the k (key, index) pairs orders them.
+// key T. Every entry with key >= T is then appended (warp-aggregated, any order) and a
+// bitonic sort of the (key, index) pairs orders them; its first k are the result. Only
+// when ties at T overflow the 2048 shared slots does a block-wide scan in index order
+// gather the keys > T and the first (lowest-index) keys == T instead.
 #include "common.cuh"
 #include "internal.h"
 #include "qhat.cuh"
@@ -137,6 +139,38 @@ __global__ void __launch_bounds__(kThreads) k_topk_rows(TopkArgs a) {
     __syncthreads();
   }
   const uint32_t T = prefix;  // the k-th largest key; take kk of the keys equal to it
+  // Every entry with key >= T, in any order: the sort below orders them by (key desc, index
+  // asc), so its first k are the keys > T followed by the kk lowest-index keys == T.
+  {
+    __shared__ int s_cnt;
+    if (threadIdx.x == 0) s_cnt = 0;
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    for (int64_t base = 0; base < n; base += blockDim.x) {
+      const int64_t i = base + threadIdx.x;
+      const uint32_t u = i < n ? float_key(sc[i]) : 0u;
+      const bool take = i < n && u >= T;
+      const unsigned bal = __ballot_sync(0xffffffffu, take);
+      if (bal == 0) continue;
+      int pos = 0;
+      if (lane == __ffs(bal) - 1) pos = atomicAdd(&s_cnt, __popc(bal));
+      pos = __shfl_sync(0xffffffffu, pos, __ffs(bal) - 1) + __popc(bal & ((1u << lane) - 1u));
+      if (take && pos < kMaxTopk) pairs[pos] = pack_desc(u, (uint32_t)i);
+    }
+    __syncthreads();
+    const int cnt = s_cnt;
+    if (cnt <= kMaxTopk) {
+      int Pc = 1;
+      while (Pc < cnt) Pc <<= 1;
+      for (int i = cnt + threadIdx.x; i < Pc; i += blockDim.x) pairs[i] = ~0ull;
+      __syncthreads();
+      bitonic_sort(pairs, Pc);
+      for (int i = threadIdx.x; i < k; i += blockDim.x)
+        out[i] = (int32_t)(pairs[i] & 0xffffffffu);
+      return;
+    }
+    __syncthreads();  // too many ties for shared memory: the ordered gather below
+  }
   const int n_gt = k - kk;
   int run_gt = 0, run_eq = 0;
   for (int64_t base = 0; base < n; base += blockDim.x) {
