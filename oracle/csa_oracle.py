@@ -251,7 +251,7 @@ def index_scores(qI_t, w_t, KI, n_vis: int) -> np.ndarray:
 def index_score_scale(qI_t, w_t, KI, n_vis: int) -> np.ndarray:
     """sum_h |w_{t,h}| * ReLU(q^I_{t,h} . K_s): the sum of the magnitudes of the terms that
     make up I_{t,s}. Not part of the method: it is the scale against which a floating-point
-    evaluation of I is judged (a rounding error of a sum grows with this, not with |I|,
+    evaluation of I is compared (a rounding error of a sum grows with this, not with |I|,
     when signed head weights cancel). Equals |I| when every w >= 0."""
     qI_t = np.asarray(qI_t, np.float64)
     K = np.asarray(KI, np.float64)[:n_vis]
