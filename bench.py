@@ -268,10 +268,7 @@ def run_ours(args, W, rank, world, local_rank):
         torch.cuda.synchronize()
         idx_ms = sum(b.elapsed_time(a) for b, a in zip(ev_b, ev_a)) / K
         csa.set_index_timing_events([], [])
-    if world > 1:
-        tt = torch.tensor([ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, world, "cuda")
 
     # end to end through the public API: per-step query-side inputs from pinned host
     # memory, the call, and the result back to pinned host memory
@@ -280,7 +277,7 @@ def run_ours(args, W, rank, world, local_rank):
     n_vis = min(s.ctx // s.m, s.n_cap) if s.kind != "csa_prefill" else s.n_cap
     per_q = algorithmic_bytes_per_query(s, n_vis)
     queries = s.B * s.T
-    value = world * queries * K / (ms / 1e3)
+    value = whole_job_rate(world, queries, K, ms)
     peaks, peak_src = load_peaks()
     roof = None
     if has_index and idx_ms:
@@ -330,6 +327,24 @@ def run_ours(args, W, rank, world, local_rank):
                          "peak": peaks["bf16_tflops"],
                          "peak_source": f"{peak_src} bf16_tflops (cuBLAS burst)"}
     return res, inp, s
+
+
+def max_over_ranks(ms: float, world: int, device: str) -> float:
+    """The timed region's length as the slowest rank saw it (all ranks get the max)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+
+    tt = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def whole_job_rate(world: int, queries_per_rank: int, steps: int, ms: float) -> float:
+    """Queries per second of the whole job: every rank ran `steps` steps of its own batch
+    (weak scaling) and the job took `ms`, the max over ranks."""
+    return world * queries_per_rank * steps / (ms / 1e3)
 
 
 QUERY_INPUTS = ("q", "qI", "qI_scale", "w", "q_pos")
