@@ -122,6 +122,9 @@ csa_status csa_compress(const csa_params* p, csa_dtype io, int32_t B, int64_t n_
  *             of a block is block-scale b of key 32*j + i. Requires H_I = 64, d_I = 128,
  *             N_cap a multiple of 128 and B*T <= 1024.
  * w: f32 [B,T,H_I]. q_pos: int64 [B,T]. Scores are fp32 sums of exact products.
+ * With H_I = 64, d_I = 128 and N_cap a multiple of 128, bf16 and FP8 keys also run on the
+ * tensor cores (an e4m3 code widens exactly to bf16; the row scale is applied after the
+ * ReLU, which it commutes with as it is positive); other shapes and f32 run on CUDA cores.
  */
 csa_status csa_index_scores(const csa_params* p, csa_dtype kdt, int32_t B, int32_t T,
                             int64_t N_cap, const void* qI, const void* qI_scale, const float* w,

@@ -180,3 +180,18 @@ def test_binding_refuses_host_tensors():
 
     with pytest.raises(ValueError):
         csa._ptr(torch.zeros(4))
+
+
+def test_noalloc_topk_rejects_oversize_on_the_host():
+    # 64 rows of 65536 candidates need ~32 MB of lists: refused before any device work, so
+    # this runs without a GPU (the pointers are never dereferenced)
+    p = csa.make_params(topk=1024)
+    need = csa.workspace_size(p, csa.CSA_WS_TOPK, 0, 64, 1, 65536)
+    assert need > csa.TOPK_NOALLOC_SCRATCH_BYTES
+    s = csa.lib().csa_topk_noalloc(ctypes.byref(p), 64, 1, 65536, 0x1000, 0x2000, 0x3000, None)
+    assert s == csa.CSA_ERR_WORKSPACE
+    assert "scratch" in csa.last_error()
+
+
+def test_kernel_launch_counter_is_exported():
+    assert csa.kernel_launches() >= 0
