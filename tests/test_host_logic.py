@@ -1,0 +1,61 @@
+"""Host-side arithmetic behind the bench line and the FP8 tensor-core path, on CPU.
+
+- Algorithmic bytes per decode query and the prefill flop count, against the closed forms
+  built from the workload shapes (keys scanned x bytes per key, rows attended x row bytes,
+  visible (t, s) pairs x 2 H_I d_I flops, attended rows x 4 c H flops).
+- Every OCP e4m3 code is exactly a bf16 value: the FP8 indexer widens codes to bf16 for the
+  tensor cores, which is exact only because of this.
+"""
+import importlib.util
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from long_context_sparse_08_b200 import workloads as W
+from oracle import csa_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+@pytest.mark.parametrize("name,expected", [
+    # keys x (FP8 row 128 B + fp32 scale) + (k + window) x 1 KB rows + q + qI + w + out
+    ("flash_decode_131k", 32768 * 132 + 640 * 1024 + 65536 + 16384 + 256 + 65536),
+    # keys x (64 B e2m1 + 4 B e8m0) + 1152 rows + q (128 heads) + MXFP4 qI + w + out
+    ("pro_decode_1m", 262144 * 68 + 1152 * 1024 + 131072 + 4352 + 256 + 131072),
+    # every visible entry and the window, q and out (64 heads)
+    ("hca_decode_1m", 8320 * 1024 + 65536 + 65536),
+])
+def test_algorithmic_bytes_per_query(bench, name, expected):
+    s = W.SHAPES[name]
+    n_vis = min(s.ctx // s.m, s.n_cap)
+    assert bench.algorithmic_bytes_per_query(s, n_vis)["total"] == expected
+
+
+def test_prefill_flops(bench):
+    s = W.SHAPES["flash_prefill_8k"]
+    fl = bench.prefill_flops(s)
+    # visible (t, s) pairs of queries 57344 .. 65535 at m = 4, N_cap = 16384
+    pairs = sum(min((57344 + i) // 4, 16384) for i in range(8192))
+    assert pairs == 125_825_024
+    assert fl["index"] == 2 * 64 * 128 * pairs
+    # every query attends k = 512 selected rows and a full 128-token window
+    assert fl["attention"] == 8192 * 64 * 640 * 512 * 4
+    assert fl["total"] == fl["index"] + fl["attention"]
+
+
+def test_every_e4m3_code_is_a_bf16_value():
+    codes = np.arange(256, dtype=np.uint8)
+    vals = O.dec_e4m3(codes)  # float64, NaN for the two NaN codes
+    finite = np.isfinite(vals)
+    as_bf16 = torch.from_numpy(vals[finite]).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(as_bf16, vals[finite])
