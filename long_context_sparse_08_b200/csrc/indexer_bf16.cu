@@ -545,9 +545,11 @@ cudaError_t launch_index_bf16_tc(const IndexArgs& a, cudaStream_t st) {
   // queries in launches of at most kMaxQueries (each launch walks its groups' tiles)
   for (int q0 = 0; q0 < Qall && e == cudaSuccess; q0 += kMaxQueries) {
     const int Q = Qall - q0 < kMaxQueries ? Qall - q0 : kMaxQueries;
+    // a batch of fewer than four queries (a tail) has fewer q rows than a group's box
+    const bool grp = grouped && Q >= 4;
     CUtensorMap mq;
     const auto* qI = static_cast<const __nv_bfloat16*>(a.qI) + (size_t)q0 * kHeads * kDim;
-    if (!make_map_bf16_rows(&mq, qI, (uint64_t)Q * kHeads, grouped ? 4 * kHeads : kHeads)) {
+    if (!make_map_bf16_rows(&mq, qI, (uint64_t)Q * kHeads, grp ? 4 * kHeads : kHeads)) {
       e = cudaErrorInvalidValue;
       break;
     }
@@ -557,9 +559,9 @@ cudaError_t launch_index_bf16_tc(const IndexArgs& a, cudaStream_t st) {
                     a.hist ? a.hist + (size_t)q0 * kBins : nullptr};
     const int64_t tiles_max = (int64_t)Q * (a.n_cap / kTileKeys);
     const int grid = (int)(tiles_max < num_sms() ? (tiles_max > 0 ? tiles_max : 1) : num_sms());
-    e = fp8       ? launch_variant<true, 1>(mk, mq, p, grid, st)
-        : grouped ? launch_variant<false, 4>(mk, mq, p, grid, st)
-                  : launch_variant<false, 1>(mk, mq, p, grid, st);
+    e = fp8   ? launch_variant<true, 1>(mk, mq, p, grid, st)
+        : grp ? launch_variant<false, 4>(mk, mq, p, grid, st)
+              : launch_variant<false, 1>(mk, mq, p, grid, st);
   }
   timing_after(st);
   return e;

@@ -97,6 +97,36 @@ def test_index_scores_parity(name):
                        f"{name} b={b} t={ti}")
 
 
+def _bf16_tail_case(T=514, N=512, seed=77):
+    """One request of T queries with bf16 indexer keys; T = 514 makes launch batches of
+    512 queries and a short tail of 2 (which takes the one-query-per-tile form)."""
+    g = np.random.default_rng(seed)
+    H, D = 64, 128
+    qI = W.f32_to_bf16_bits(g.standard_normal((1, T, H, D)).astype(np.float32))
+    KI = W.f32_to_bf16_bits(g.standard_normal((1, N, D)).astype(np.float32))
+    w = g.standard_normal((1, T, H)).astype(np.float32)
+    pos = (1200 + np.arange(T, dtype=np.int64)).reshape(1, T)
+    return qI, KI, w, pos
+
+
+def test_bf16_indexer_launch_batches_with_a_short_tail():
+    T, N = 514, 512
+    qI, KI, w, pos = _bf16_tail_case(T, N)
+    p = csa.make_params(m=4, n_idx_heads=64, d_idx=128)
+    scores = torch.zeros((1, T, N), dtype=torch.float32, device="cuda")
+    as_bf16 = lambda x: torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+    csa.csa_index_scores(p, csa.CSA_BF16, 1, T, N, as_bf16(qI), None, torch.from_numpy(w).cuda(),
+                         as_bf16(KI), None, torch.from_numpy(pos).cuda(), scores)
+    got = scores.cpu().numpy()
+    qd, kd = O.dec_bf16(qI)[0], O.dec_bf16(KI)[0]
+    for t in (0, 3, 255, 511, 512, 513):
+        nv = O.visible_entries(int(pos[0, t]), 4, N)
+        ref = O.index_scores(qd[t], w[0, t], kd, nv)
+        scale = O.index_score_scale(qd[t], w[0, t], kd, nv)
+        U.check_scores(got[0, t, :nv], ref, scale, f"tail case t={t}")
+    assert csa.device_error() == 0
+
+
 # ---------------------------------------------------------------------------
 # stage 3: top-k, exact on given fp32 scores
 # ---------------------------------------------------------------------------
