@@ -71,6 +71,19 @@ def quant_fp8_rowwise(x: np.ndarray):
     return codes, scale
 
 
+def quant_mixed_kv(x: np.ndarray, r: int):
+    """Mixed-precision KV entry rows: the first d-r dims row-wise FP8 e4m3 (scale =
+    amax/448 over those dims), the last r dims bf16 (RNE).
+
+    Returns (codes uint8 [..., d-r], scale float32 [...], rope bf16 bits uint16 [..., r]).
+    """
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    d = x.shape[-1]
+    assert 0 < r < d
+    codes, scale = quant_fp8_rowwise(x[..., :d - r])
+    return codes, scale, f32_to_bf16_bits(np.ascontiguousarray(x[..., d - r:]))
+
+
 # e2m1 grid (magnitudes) and their 3-bit codes (exponent 2 bits bias 1, mantissa 1 bit)
 _E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float32)
 

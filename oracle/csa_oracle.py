@@ -19,8 +19,15 @@ Sources (cited by page title and section):
        3(2) 部分 RoPE -- RoPE on the last 64 dims of q and KV, output rotated at position -t;
        3(3) 滑动窗口注意力 -- n_win uncompressed entries of the most recent tokens;
        3(4) Attention Sink -- exp(z'_h) added to the softmax denominator (s_{h,i,j}).
+       1(4) 分组输出投影 -- n_h head outputs in g groups, each projected to d_g, then the
+            g*d_g concatenation projected to d; 2(2) applies the same to HCA;
+       4 效率分析 item 1 -- KV entries stored with the RoPE dims in BF16, the rest in FP8;
+     二、基础设施 (四) FP4 量化感知训练 -- index scores quantised from FP32 to BF16 before
+       the top-k selector (2x selector speed, 99.7% recall of the KV entries);
+     三、预训练 (二) 模型配置 -- g = 8 / 16, d_g = 1024, d = 4096 / 7168.
   [P4] DeepseekV4论文解析 (blog.chaseai.de), 2. Hybrid Attention：CSA + HCA -- entry counts
-       at 1M tokens (262,144 candidates; 1024+128 / 512+128 read; 8,192 + 128 for HCA).
+       at 1M tokens (262,144 candidates; 1024+128 / 512+128 read; 8,192 + 128 for HCA);
+       三、实验 -- the same precision split (RoPE dims BF16, rest FP8; BF16 index scores).
 
 Readings where the pages leave a step open (each is a constant of the convention,
 not a value the pages fix):
@@ -37,6 +44,14 @@ not a value the pages fix):
   R7  Top-k order is (score descending, index ascending); slots beyond the visible
       count hold -1.
   R8  Indexer keys and queries get no RMSNorm / RoPE; the index score has no scale.
+  R18 BF16 index scores: each score is rounded to the nearest bf16 value (ties to even)
+      and the selector orders the rounded values by (value descending, index ascending).
+  R19 Mixed-precision KV entry: the first c-r dims are FP8 e4m3 with one fp32 scale per
+      entry row (amax/448, as for the FP8 indexer keys), the last r (RoPE) dims are bf16.
+      Only compressed entries use it; sliding-window rows stay bf16.
+  R20 Grouped output projection: group i holds heads i*H/g .. (i+1)*H/g-1, concatenated
+      head after head; row vectors multiply weights from the left (x . W), as in the
+      pages' projections; the input is the un-rotated attention output.
 Parity of R1/R2 against the pages is unpinned (the pages fix neither); every other
 step is pinned by the CPU tests (closed forms, invariants, brute force).
 """
@@ -121,6 +136,13 @@ def unblock_key_scales(blocked) -> np.ndarray:
 def dec_fp8_rows(codes, row_scale) -> np.ndarray:
     """FP8 e4m3 rows times their per-row fp32 scale."""
     return dec_e4m3(codes) * np.asarray(row_scale, np.float64)[..., None]
+
+
+def dec_mixed_kv(nope_codes, nope_scale, rope_bits) -> np.ndarray:
+    """Mixed-precision KV entry rows (reading R19) [P1 一(三)4 item 1]: FP8 e4m3 codes of
+    the first c-r dims times the row's fp32 scale, followed by the last r (RoPE) dims as
+    bf16. Returns float64 [..., c]."""
+    return np.concatenate([dec_fp8_rows(nope_codes, nope_scale), dec_bf16(rope_bits)], axis=-1)
 
 
 # ----------------------------------------------------------------------------
@@ -268,6 +290,27 @@ def topk_select(scores, k: int) -> np.ndarray:
     return out
 
 
+def round_to_bf16(x) -> np.ndarray:
+    """Nearest bf16 value of each x (8 significant bits, ties to the even significand),
+    computed from the format's definition: with e = floor(log2|x|) (at least -126, bf16's
+    smallest normal exponent) the bf16 values near x are the multiples of 2^(e-7).
+    Finite inputs whose rounded value stays finite; zero stays zero."""
+    x = np.asarray(x, np.float64)
+    a = np.abs(x)
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, -126.0)
+    ulp = np.exp2(e - 7.0)
+    return np.rint(x / ulp) * ulp  # np.rint rounds halves to even
+
+
+def topk_select_bf16(scores, k: int) -> np.ndarray:
+    """Top-k on BF16 index scores (reading R18) [P1 二(四)]: the selector of
+    ``topk_select`` applied to the scores rounded to bf16, so that scores rounding to the
+    same bf16 value tie and the smaller index wins."""
+    return topk_select(round_to_bf16(scores), k)
+
+
 # ----------------------------------------------------------------------------
 # stage 4: shared-KV MQA with window and sink  [P1 1(3), 3(1)-(4)]
 # ----------------------------------------------------------------------------
@@ -339,3 +382,31 @@ def hca_query(q_t, t: int, kv_rows, n_vis: int, win_kv, pos0: int, sink, *, r: i
 def default_scale(c: int) -> float:
     """Logit scale 1/sqrt(c) (reading R4)."""
     return 1.0 / math.sqrt(c)
+
+
+# ----------------------------------------------------------------------------
+# grouped output projection  [P1 1(4), 2(2)]
+# ----------------------------------------------------------------------------
+
+
+def grouped_output_projection(o_t, w_grp, w_out) -> np.ndarray:
+    """Attention output of one query [P1 1(4) 分组输出投影] (reading R20).
+
+    o_t [H, c]: the un-rotated core-attention outputs o_{t,1..H}.
+    w_grp [g, c*H/g, d_g]: group i's projection of o^G_{t,i} (heads i*H/g .. (i+1)*H/g-1,
+    concatenated) to the intermediate output o^G'_{t,i}.
+    w_out [g*d_g, d]: projection of [o^G'_{t,1}; ...; o^G'_{t,g}] to the output.
+    Returns [d]."""
+    o_t = np.asarray(o_t, np.float64)
+    w_grp = np.asarray(w_grp, np.float64)
+    w_out = np.asarray(w_out, np.float64)
+    H, c = o_t.shape
+    g, width, d_g = w_grp.shape
+    assert H % g == 0 and width == c * (H // g) and w_out.shape[0] == g * d_g
+    hg = H // g
+    mid = np.empty((g, d_g))
+    for i in range(g):
+        o_group = o_t[i * hg:(i + 1) * hg].reshape(width)  # o^G_{t,i}
+        mid[i] = o_group @ w_grp[i]                          # o^G'_{t,i}
+    return mid.reshape(g * d_g) @ w_out
+

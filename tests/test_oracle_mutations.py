@@ -1,7 +1,8 @@
 """The oracle's pins catch plausible mistakes.
 
 Each case plants one slip in the float64 oracle (on the CPU, via monkeypatch) and
-checks that at least one pin of test_oracle_pins fails against the mutated oracle.
+checks that at least one pin of test_oracle_pins or test_oracle_next_pins fails against
+the mutated oracle.
 """
 import inspect
 import os
@@ -10,6 +11,8 @@ import numpy as np
 import pytest
 
 from oracle import csa_oracle as O
+from oracle import state_cache as SC
+import tests.test_oracle_next_pins as NEXT_PINS
 import tests.test_oracle_pins as PINS
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
@@ -17,25 +20,34 @@ GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
 def _pins():
     out = []
-    for name, fn in sorted(vars(PINS).items()):
-        if name.startswith("test_") and callable(fn):
-            out.append(fn)
+    for mod in (PINS, NEXT_PINS):
+        for name, fn in sorted(vars(mod).items()):
+            if name.startswith("test_") and callable(fn):
+                out.append(fn)
     return out
+
+
+def _calls(fn):
+    """Keyword sets to call a pin with: its parametrize marks expanded, the golden folder
+    supplied."""
+    calls = [dict()]
+    for mark in getattr(fn, "pytestmark", []):
+        if mark.name != "parametrize":
+            continue
+        names = [n.strip() for n in mark.args[0].split(",")] if isinstance(mark.args[0], str) \
+            else list(mark.args[0])
+        rows = [v if len(names) > 1 else (v,) for v in mark.args[1]]
+        calls = [dict(c, **dict(zip(names, row))) for c in calls for row in rows]
+    if "golden_dir" in inspect.signature(fn).parameters:
+        calls = [dict(c, golden_dir=GOLDEN) for c in calls]
+    return calls
 
 
 def _run_all_pins():
     """Run every pin; return the names of those that fail."""
     failed = []
     for fn in _pins():
-        params = inspect.signature(fn).parameters
-        calls = []
-        if "branch" in params:
-            calls = [dict(branch="a"), dict(branch="b")]
-        elif "golden_dir" in params:
-            calls = [dict(golden_dir=GOLDEN)]
-        else:
-            calls = [dict()]
-        for kw in calls:
+        for kw in _calls(fn):
             try:
                 fn(**kw)
             except (AssertionError, ValueError, IndexError):
@@ -140,6 +152,81 @@ MUTATIONS = {
 }
 
 
+def _bf16_ulp(x):
+    a = np.abs(np.asarray(x, np.float64))
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.exp2(np.maximum(e, -126.0) - 7.0)
+
+
+def _mut_bf16_truncate(x):
+    u = _bf16_ulp(x)
+    return np.trunc(np.asarray(x, np.float64) / u) * u
+
+
+def _mut_bf16_ties_away(x):
+    x = np.asarray(x, np.float64)
+    u = _bf16_ulp(x)
+    return np.sign(x) * np.floor(np.abs(x) / u + 0.5) * u
+
+
+def _mut_mixed_kv_rope_first(nope_codes, nope_scale, rope_bits):
+    return np.concatenate([O.dec_bf16(rope_bits), O.dec_fp8_rows(nope_codes, nope_scale)], -1)
+
+
+def _mut_mixed_kv_no_scale(nope_codes, nope_scale, rope_bits):
+    return np.concatenate([O.dec_e4m3(nope_codes), O.dec_bf16(rope_bits)], -1)
+
+
+def _mut_groups_interleaved(o_t, w_grp, w_out):
+    o_t = np.asarray(o_t, np.float64)
+    g = w_grp.shape[0]
+    mid = np.stack([o_t[i::g].reshape(-1) @ w_grp[i] for i in range(g)])  # heads i, i+g, ..
+    return mid.reshape(-1) @ w_out
+
+
+def _mut_groups_concat_transposed(o_t, w_grp, w_out):
+    o_t = np.asarray(o_t, np.float64)
+    g = w_grp.shape[0]
+    hg = o_t.shape[0] // g
+    mid = np.stack([o_t[i * hg:(i + 1) * hg].reshape(-1) @ w_grp[i] for i in range(g)])
+    return mid.T.reshape(-1) @ w_out  # [d_g, g] order instead of [g, d_g]
+
+
+def _mut_state_forgets_b_rows(self):
+    return np.full((self.m, self.c), -np.inf), np.zeros((self.m, self.c))
+
+
+def _mut_state_position_off_by_one(self, entry, i):
+    return O.finalize_entries(entry[None], i + 1, self.m, self.r, self.base, self.eps,
+                              self.gamma)[0]
+
+
+def _mut_ring_slot_shifted(self, row, pos):
+    if self.n_win > 0:
+        self.ring[(pos + 1) % self.n_win] = np.asarray(row, np.float64)
+
+
+def _mut_release_leaks(self):
+    self.page_table = []
+
+
+NEXT_MUTATIONS = {
+    "bf16_truncates": (O, "round_to_bf16", _mut_bf16_truncate),
+    "bf16_ties_away_from_zero": (O, "round_to_bf16", _mut_bf16_ties_away),
+    "bf16_scores_not_rounded": (O, "topk_select_bf16", lambda s, k: O.topk_select(s, k)),
+    "mixed_kv_rope_dims_first": (O, "dec_mixed_kv", _mut_mixed_kv_rope_first),
+    "mixed_kv_scale_dropped": (O, "dec_mixed_kv", _mut_mixed_kv_no_scale),
+    "output_groups_interleaved": (O, "grouped_output_projection", _mut_groups_interleaved),
+    "output_groups_concat_transposed": (O, "grouped_output_projection",
+                                        _mut_groups_concat_transposed),
+    "state_forgets_b_rows": (SC.CsaState, "_b_branch", _mut_state_forgets_b_rows),
+    "state_entry_position_off_by_one": (SC.CsaState, "_finalize", _mut_state_position_off_by_one),
+    "window_ring_slot_shifted": (SC._Request, "_push_window", _mut_ring_slot_shifted),
+    "release_leaks_pages": (SC._Request, "release", _mut_release_leaks),
+}
+
+
 def test_unmutated_oracle_passes_every_pin():
     assert _run_all_pins() == []
 
@@ -156,3 +243,11 @@ def test_e4m3_decoder_mutation_is_caught(monkeypatch):
     orig = O.dec_e4m3
     monkeypatch.setattr(O, "dec_e4m3", lambda c: orig(c) * 0.5)
     assert "test_e4m3_decoder_matches_torch_all_codes" in _run_all_pins()
+
+
+@pytest.mark.parametrize("name", sorted(NEXT_MUTATIONS))
+def test_next_step_mutation_is_caught(name, monkeypatch):
+    owner, attr, fn = NEXT_MUTATIONS[name]
+    monkeypatch.setattr(owner, attr, fn)
+    failed = _run_all_pins()
+    assert failed, f"no pin caught the planted mistake {name}"
