@@ -9,6 +9,7 @@
  *        3(1) query / KV RMSNorm, 3(2) partial RoPE and output rotation at -t,
  *        3(3) sliding window, 3(4) attention sink.
  *   [P1'] same page, 二、基础设施 (四) FP4 量化感知训练: the indexer's QK path in FP4.
+ *   [P1''] same page, 二、基础设施 (六) 推理框架: state cache and paged cache at inference.
  *
  * Conventions shared by every call
  *   - Every tensor pointer is device memory owned by the caller; the library never
@@ -107,6 +108,41 @@ csa_status csa_compress(const csa_params* p, csa_dtype io, int32_t B, int64_t n_
                         const void* Za, const void* Zb, const void* bias, const void* prev_Cb,
                         const void* prev_Zb, const void* kv_rms_w, int32_t finalize,
                         void* out_cache, void* stream);
+
+/*
+ * Decode-time compression with a state cache ([P1''] 二、基础设施 (六) 推理框架: a state
+ * cache holds the sliding window and the raw tail tokens of an unfinished compression
+ * block; finished entries live in a paged cache whose blocks cover a multiple of
+ * lcm(m, m') raw tokens -- 128 tokens = 32 CSA entries = 1 HCA entry).
+ *
+ * Appends one token to each of B requests. For request b, at position t = pos[b]:
+ *   - its raw rows go to slot t % S of `state` [B, S, R, c] (io dtype):
+ *       CSA (overlap = 1): S = 2m, R = 4 rows in the order Ca, Za, Cb, Zb;
+ *       HCA (overlap = 0): S = m,  R = 2 rows in the order C (= Ca), Z (= Za);
+ *     the token rows are Ca, Cb, Za, Zb [B, c] (Cb, Zb NULL for HCA);
+ *   - win_row [B, c] (final form: normed and rotated by the caller) goes to row t % n_win of
+ *     win_ring [B, n_win, c]; both NULL to keep no window;
+ *   - when t + 1 is a multiple of m, entry i = t / m is compressed from the state exactly as
+ *     csa_compress computes it ([P1] 1(1) / 2(1); the CSA b-branch is block i-1's rows for
+ *     i > 0 and absent for i = 0), and with finalize = 1 RMSNorm'd (kv_rms_w [c] or NULL)
+ *     and rotated at position m*i ([P1] 3(1), 3(2)). The row goes to row i % page_rows of
+ *     page page_table[b, i / page_rows] of `pages` [n_pages, page_rows, c].
+ * The slots of block i-1 and block i are read back, so a request's appends must arrive in
+ * position order (one per call), after its state was filled up to t-1: by earlier appends,
+ * or, for a request resumed after a prefill, by the caller writing those raw rows into their
+ * slots. Requests whose entry's logical page is >= max_pages, whose page id is outside
+ * [0, n_pages), or whose position is negative are skipped and leave a device error code
+ * (301 position, 302 page slot, 303 page id) for csa_device_error(). The pages use
+ * page_rows = 128 / m; with page_table[b, k] = b * max_pages + k they are the contiguous
+ * cache [B, N_cap = page_rows * max_pages, c] that the attention calls read.
+ * io: CSA_F32 or CSA_BF16 for every tensor (math is fp32); bias: [2m, c] or [m, c].
+ */
+csa_status csa_state_append(const csa_params* p, csa_dtype io, int32_t B, const int64_t* pos,
+                            const void* Ca, const void* Cb, const void* Za, const void* Zb,
+                            const void* win_row, const void* bias, const void* kv_rms_w,
+                            int32_t finalize, void* state, void* win_ring, void* pages,
+                            int32_t n_pages, int32_t page_rows, const int32_t* page_table,
+                            int32_t max_pages, void* stream);
 
 /*
  * Stage 2 -- lightning-indexer scores ([P1] 1(2)):
@@ -250,8 +286,9 @@ void csa_set_index_timing_events(void* const* before, void* const* after, int32_
 /*
  * Error word of the tensor-core kernels: every wait inside them is bounded (about a second);
  * a wait that runs out stores a nonzero code (the first one wins) and the kernel returns
- * early instead of hanging. Writes the code to *code (0 = none) and clears it. Synchronises
- * the device. Returns CSA_ERR_CUDA if the copy fails.
+ * early instead of hanging. csa_state_append also leaves a code for a request it skipped.
+ * Writes the code to *code (0 = none) and clears it. Synchronises the device. Returns
+ * CSA_ERR_CUDA if the copy fails.
  */
 csa_status csa_device_error(int32_t* code);
 

@@ -23,7 +23,7 @@ EXPORTS = (
     "csa_compress", "csa_index_scores", "csa_topk", "csa_index_topk", "csa_sparse_mqa",
     "hca_dense_mqa", "csa_forward", "csa_workspace_size", "csa_status_string",
     "csa_last_error", "csa_set_index_timing_events", "csa_version", "csa_device_error",
-    "csa_topk_noalloc", "csa_kernel_launches",
+    "csa_topk_noalloc", "csa_kernel_launches", "csa_state_append",
 )
 # size of the library-owned scratch array behind csa_topk_noalloc (bytes, per device)
 TOPK_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -81,6 +81,8 @@ _SIGS = {
     "csa_version": [],
     "csa_device_error": [ctypes.POINTER(ctypes.c_int32)],
     "csa_kernel_launches": [],
+    "csa_state_append": [_PP, ctypes.c_int, _I32] + [_VP] * 8 + [_I32, _VP, _VP, _VP, _I32, _I32,
+                                                             _VP, _I32, _VP],
 }
 _RES = {"csa_workspace_size": _SZ, "csa_kernel_launches": ctypes.c_uint64, "csa_status_string": ctypes.c_char_p,
         "csa_last_error": ctypes.c_char_p, "csa_version": ctypes.c_char_p,
@@ -127,7 +129,8 @@ def version() -> str:
 
 
 def device_error() -> int:
-    """Read and clear the tensor-core kernels' error word (0 = no bounded wait ran out)."""
+    """Read and clear the library's device error word (0 = no bounded wait ran out and no
+    state append was skipped)."""
     c = ctypes.c_int32(0)
     _check("csa_device_error", lib().csa_device_error(ctypes.byref(c)))
     return int(c.value)
@@ -175,6 +178,16 @@ def csa_compress(p, io, B, n_tok, first_entry, n_cap, Ca, Cb, Za, Zb, bias, prev
                            _ptr(prev_Zb), _ptr(kv_rms_w), int(finalize), _ptr(out_cache),
                            _stream(stream))
     _check("csa_compress", s)
+
+
+def csa_state_append(p, io, B, pos, Ca, Cb, Za, Zb, win_row, bias, kv_rms_w, finalize, state,
+                     win_ring, pages, n_pages, page_rows, page_table, max_pages, stream=None):
+    s = lib().csa_state_append(ctypes.byref(p), io, B, _ptr(pos), _ptr(Ca), _ptr(Cb), _ptr(Za),
+                               _ptr(Zb), _ptr(win_row), _ptr(bias), _ptr(kv_rms_w),
+                               int(finalize), _ptr(state), _ptr(win_ring), _ptr(pages),
+                               n_pages, page_rows, _ptr(page_table), max_pages,
+                               _stream(stream))
+    _check("csa_state_append", s)
 
 
 def csa_index_scores(p, kdt, B, T, N_cap, qI, qI_scale, w, KI, KI_scale, q_pos, out_scores,

@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "state_append.cuh"
 
 namespace csa {
 std::atomic<uint64_t> g_launches{0};
@@ -243,11 +244,14 @@ const char* csa_last_error(void) { return g_err; }
 
 csa_status csa_device_error(int32_t* code) {
   REQUIRE(code != nullptr, "code is NULL");
-  int c = 0, c2 = 0, c3 = 0;
-  TRY(cuda_status(csa::index_mxf4_device_error(&c), "device error word"));
-  TRY(cuda_status(csa::mqa_tc_device_error(&c2), "device error word"));
-  TRY(cuda_status(csa::index_bf16_device_error(&c3), "device error word"));
-  *code = c != 0 ? c : (c2 != 0 ? c2 : c3);
+  int words[4] = {0, 0, 0, 0};
+  TRY(cuda_status(csa::index_mxf4_device_error(&words[0]), "device error word"));
+  TRY(cuda_status(csa::mqa_tc_device_error(&words[1]), "device error word"));
+  TRY(cuda_status(csa::index_bf16_device_error(&words[2]), "device error word"));
+  TRY(cuda_status(csa::state_append_device_error(&words[3]), "device error word"));
+  *code = 0;
+  for (int w : words)
+    if (*code == 0) *code = w;
   return ok();
 }
 
@@ -335,6 +339,52 @@ csa_status csa_compress(const csa_params* p, csa_dtype io, int32_t B, int64_t n_
   a.rope_base = p->rope_base; a.eps = p->rms_eps; a.Ca = Ca; a.Cb = Cb; a.Za = Za; a.Zb = Zb;
   a.bias = bias; a.prev_Cb = prev_Cb; a.prev_Zb = prev_Zb; a.rms_w = kv_rms_w; a.out = out_cache;
   TRY(cuda_status(csa::launch_compress(a, io == CSA_BF16, (cudaStream_t)stream), "compress"));
+  return ok();
+}
+
+csa_status csa_state_append(const csa_params* p, csa_dtype io, int32_t B, const int64_t* pos,
+                            const void* Ca, const void* Cb, const void* Za, const void* Zb,
+                            const void* win_row, const void* bias, const void* kv_rms_w,
+                            int32_t finalize, void* state, void* win_ring, void* pages,
+                            int32_t n_pages, int32_t page_rows, const int32_t* page_table,
+                            int32_t max_pages, void* stream) {
+  TRY(check_params(p));
+  REQUIRE(io == CSA_F32 || io == CSA_BF16, "state io dtype must be CSA_F32 or CSA_BF16");
+  REQUIRE(B >= 0 && B <= 65535, "B must be in [0, 65535]");
+  REQUIRE(p->overlap == 0 || p->overlap == 1, "overlap must be 0 or 1");
+  REQUIRE(finalize == 0 || finalize == 1, "finalize must be 0 or 1");
+  REQUIRE(p->rope_dims / 2 <= 256, "rope_dims must be <= 512");
+  REQUIRE(n_pages >= 1 && page_rows >= 1 && max_pages >= 1,
+          "n_pages, page_rows and max_pages must be >= 1");
+  REQUIRE((win_row == nullptr) == (win_ring == nullptr), "win_row and win_ring go together");
+  REQUIRE(win_ring == nullptr || p->n_win >= 1, "a window ring needs n_win >= 1");
+  if (p->overlap) {
+    REQUIRE_PTR(Cb);
+    REQUIRE_PTR(Zb);
+  } else {
+    REQUIRE(Cb == nullptr && Zb == nullptr, "HCA (overlap=0) takes no b-branch rows");
+  }
+  if (B == 0) return ok();
+  REQUIRE_PTR(pos);
+  REQUIRE_PTR(Ca);
+  REQUIRE_PTR(Za);
+  REQUIRE_PTR(bias);
+  REQUIRE_PTR(state);
+  REQUIRE_PTR(pages);
+  REQUIRE_PTR(page_table);
+  OPTIONAL_PTR(win_row);
+  OPTIONAL_PTR(win_ring);
+  OPTIONAL_PTR(kv_rms_w);
+  csa::state::Args a{};
+  a.B = B; a.m = p->m; a.c = p->c; a.overlap = p->overlap; a.rope_dims = p->rope_dims;
+  a.finalize = finalize; a.n_win = p->n_win; a.n_pages = n_pages; a.page_rows = page_rows;
+  a.max_pages = max_pages; a.eps = p->rms_eps; a.pos = pos; a.Ca = Ca; a.Cb = Cb; a.Za = Za;
+  a.Zb = Zb; a.win_row = win_row; a.bias = bias; a.rms_w = kv_rms_w; a.state = state;
+  a.win_ring = win_ring; a.pages = pages; a.page_table = page_table;
+  for (int i = 0; i < p->rope_dims / 2; ++i)
+    a.inv_freq[i] = csa::rope_inv_freq(i, p->rope_dims, (double)p->rope_base);
+  TRY(cuda_status(csa::launch_state_append(a, io == CSA_BF16, (cudaStream_t)stream),
+                  "state append"));
   return ok();
 }
 

@@ -37,6 +37,11 @@ struct CompressArgs {
 };
 cudaError_t launch_compress(const CompressArgs& a, bool bf16, cudaStream_t st);
 
+namespace state { struct Args; }
+// decode-time append of one token per request into the state cache and its pages
+cudaError_t launch_state_append(const state::Args& a, bool bf16, cudaStream_t st);
+cudaError_t state_append_device_error(int* code);
+
 struct IndexArgs {
   int B, T, m, n_idx_heads, d_idx, kdt;
   int64_t n_cap;

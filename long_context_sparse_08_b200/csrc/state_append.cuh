@@ -1,0 +1,157 @@
+// Decode-time compression with a state cache: the index arithmetic and the per-channel
+// math of appending one token to one request, written once as __host__ __device__
+// functions. The kernel (state_append.cu) runs them with a CTA per request and threads
+// over channels; a host build of the same functions lets the CPU tests check slots, pages
+// and values without a GPU.
+//
+// 【论文解读】DeepSeek-V4, 二、基础设施 (六) 推理框架: a state cache holds the sliding
+// window and the raw tail tokens of a compression block not yet full; finished entries go
+// to a paged cache whose blocks cover a multiple of lcm(m, m') raw tokens.
+// 一(三)1(1) / 2(1): the compression of a block; 3(1), 3(2): RMSNorm and RoPE of an entry.
+//
+// State layout of request b ([B, S, R, c], io dtype): token p lives in slot p mod S, row r
+// of the slot is one of its raw tensors. CSA (overlap): S = 2m, rows Ca, Za, Cb, Zb -- the
+// 2m slots hold the open block (its a- and b-rows) and the previous block (whose b-rows
+// entry i reads). HCA: S = m', rows C, Z.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <math.h>
+#include <stdint.h>
+
+namespace csa {
+namespace state {
+
+#define CSA_HD __host__ __device__ __forceinline__
+
+enum { kRowCa = 0, kRowZa = 1, kRowCb = 2, kRowZb = 3 };  // HCA: C = row 0, Z = row 1
+
+// Status of one request's append (uniform over the CTA).
+enum {
+  kAppendOnly = 0,   // the token does not finish a block
+  kCompress = 1,     // the token finishes entry i: compress it into its page
+  kErrPosition = -1, // negative position
+  kErrPageSlot = -2, // entry's logical page beyond the page table
+  kErrPageId = -3    // page table entry outside [0, n_pages)
+};
+
+struct Args {
+  int B, m, c, overlap, rope_dims, finalize, n_win, n_pages, page_rows, max_pages;
+  float eps;
+  const int64_t* pos;  // [B] position of each request's new token
+  const void *Ca, *Cb, *Za, *Zb, *win_row, *bias, *rms_w;  // new rows [B, c]; bias; gamma
+  void *state, *win_ring, *pages;
+  const int32_t* page_table;  // [B, max_pages]
+  double inv_freq[256];       // RoPE pair frequencies base^(-2p/r), p < r/2
+};
+
+CSA_HD float ld(const float* p, size_t i) { return p[i]; }
+CSA_HD float ld(const __nv_bfloat16* p, size_t i) { return __bfloat162float(p[i]); }
+CSA_HD void st(float* p, size_t i, float v) { p[i] = v; }
+CSA_HD void st(__nv_bfloat16* p, size_t i, float v) { p[i] = __float2bfloat16_rn(v); }
+
+CSA_HD int slots(const Args& a) { return a.overlap ? 2 * a.m : a.m; }
+CSA_HD int rows(const Args& a) { return a.overlap ? 4 : 2; }
+
+// element (request b, token p, raw tensor r, channel j) of the state
+CSA_HD size_t state_index(const Args& a, int64_t b, int64_t p, int r, int j) {
+  return (((size_t)b * slots(a) + (size_t)(p % slots(a))) * rows(a) + r) * (size_t)a.c + j;
+}
+
+// What the token at position t of request b does; for kCompress also the entry index and
+// the element offset of its row in `pages`.
+CSA_HD int append_status(const Args& a, int64_t b, int64_t t, int64_t* entry, size_t* out_off) {
+  if (t < 0) return kErrPosition;
+  if ((t + 1) % a.m != 0) return kAppendOnly;
+  const int64_t i = t / a.m;
+  const int64_t pg = i / a.page_rows;
+  if (pg >= a.max_pages) return kErrPageSlot;
+  const int32_t page = a.page_table[(size_t)b * a.max_pages + pg];
+  if (page < 0 || page >= a.n_pages) return kErrPageId;
+  *entry = i;
+  *out_off = ((size_t)page * a.page_rows + (size_t)(i % a.page_rows)) * (size_t)a.c;
+  return kCompress;
+}
+
+// Channel j of the new token: raw rows into the state, window row into the ring.
+template <typename T>
+CSA_HD void store_channel(const Args& a, int64_t b, int64_t t, int j) {
+  T* s = static_cast<T*>(a.state);
+  const size_t src = (size_t)b * a.c + j;
+  st(s, state_index(a, b, t, kRowCa, j), ld(static_cast<const T*>(a.Ca), src));
+  st(s, state_index(a, b, t, kRowZa, j), ld(static_cast<const T*>(a.Za), src));
+  if (a.overlap) {
+    st(s, state_index(a, b, t, kRowCb, j), ld(static_cast<const T*>(a.Cb), src));
+    st(s, state_index(a, b, t, kRowZb, j), ld(static_cast<const T*>(a.Zb), src));
+  }
+  if (a.win_ring != nullptr) {
+    const size_t dst = ((size_t)b * a.n_win + (size_t)(t % a.n_win)) * a.c + j;
+    st(static_cast<T*>(a.win_ring), dst, ld(static_cast<const T*>(a.win_row), src));
+  }
+}
+
+// Channel j of entry i, pooled from the state: softmax over the block's logits plus biases
+// (CSA: the a-rows of block i, and for i > 0 the b-rows of block i-1), weighted sum of the
+// values. Same operation order as the whole-chunk compression kernel.
+template <typename T>
+CSA_HD float pool_channel(const Args& a, int64_t b, int64_t i, int j) {
+  const T* s = static_cast<const T*>(a.state);
+  const T* bias = static_cast<const T*>(a.bias);
+  const int m = a.m;
+  const bool has_b = a.overlap && i > 0;
+  float mx = -INFINITY;
+  for (int r = 0; r < m; ++r)
+    mx = fmaxf(mx, ld(s, state_index(a, b, m * i + r, kRowZa, j)) + ld(bias, (size_t)r * a.c + j));
+  if (has_b)
+    for (int r = 0; r < m; ++r)
+      mx = fmaxf(mx, ld(s, state_index(a, b, m * (i - 1) + r, kRowZb, j)) +
+                         ld(bias, (size_t)(m + r) * a.c + j));
+  float den = 0.f, num = 0.f;
+  for (int r = 0; r < m; ++r) {
+    const int64_t p = m * i + r;
+    const float e = expf(ld(s, state_index(a, b, p, kRowZa, j)) + ld(bias, (size_t)r * a.c + j) - mx);
+    den += e;
+    num = fmaf(e, ld(s, state_index(a, b, p, kRowCa, j)), num);
+  }
+  if (has_b)
+    for (int r = 0; r < m; ++r) {
+      const int64_t p = m * (i - 1) + r;
+      const float e = expf(ld(s, state_index(a, b, p, kRowZb, j)) +
+                           ld(bias, (size_t)(m + r) * a.c + j) - mx);
+      den += e;
+      num = fmaf(e, ld(s, state_index(a, b, p, kRowCb, j)), num);
+    }
+  return num / den;
+}
+
+// cos / sin of pos * inv_freq: the angle (up to ~1e6 rad) is reduced modulo 2*pi in double
+// with a two-part 2*pi, then evaluated in fp32.
+CSA_HD void rope_cs(double pos, double inv_freq, float* cs, float* sn) {
+  const double x = pos * inv_freq;
+  const double k = rint(x * 0.15915494309189535);  // x / (2*pi)
+  double red = fma(-k, 6.283185307179586232, x);
+  red = fma(-k, 2.4492935982947064e-16, red);
+  sincosf((float)red, sn, cs);
+}
+
+// Channel j of the finished row: RMSNorm (rstd = 1/sqrt(mean(x^2) + eps), weight gamma),
+// then RoPE at position m*i on the last r dims (pairs (2p, 2p+1) of that slice).
+template <typename T>
+CSA_HD float final_channel(const Args& a, const float* row, float rstd, int64_t i, int j) {
+  const T* g = static_cast<const T*>(a.rms_w);
+  float v = row[j] * rstd * (g ? ld(g, j) : 1.f);
+  const int r0 = a.c - a.rope_dims;
+  if (j >= r0) {
+    const int partner = j ^ 1;  // r0 is even
+    const float u = row[partner] * rstd * (g ? ld(g, partner) : 1.f);
+    float cs, sn;
+    rope_cs((double)a.m * (double)i, a.inv_freq[(j - r0) >> 1], &cs, &sn);
+    v = ((j - r0) & 1) == 0 ? v * cs - u * sn : u * sn + v * cs;
+  }
+  return v;
+}
+
+#undef CSA_HD
+
+}  // namespace state
+}  // namespace csa

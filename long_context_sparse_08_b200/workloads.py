@@ -396,3 +396,19 @@ def params_of(s: Shape) -> Dict[str, float]:
     return dict(m=s.m, overlap=s.overlap, c=s.c, rope_dims=s.rope_dims, rope_base=s.rope_base,
                 rms_eps=s.rms_eps, sm_scale=sm_scale(s), n_heads=s.n_heads,
                 n_idx_heads=s.n_idx_heads, d_idx=s.d_idx, topk=s.topk, n_win=s.n_win)
+
+
+def make_state_stream(*, B: int, n_tok: int, m: int, c: int, overlap: int, io: str,
+                      seed: int) -> Dict[str, np.ndarray]:
+    """Seeded raw token rows for decode-time appends to a state cache: for every request
+    b < B the rows of tokens 0 .. n_tok-1 (a request resumed at position t0 takes the
+    rows before t0 as its prefill), drawn ~N(0,1) in the order Ca, Cb, Za, Zb (CSA; C, Z
+    for HCA), then the window rows, then the pooling bias ([2m, c] CSA, [m, c] HCA; std
+    1), each [B, n_tok, c]; encoded as ``io`` ("f32" or "bf16" bit patterns). The shapes
+    follow the models' c = 512, m = 4 / m' = 128 [【论文解读】DeepSeek-V4 三、预训练 (二)]."""
+    g = np.random.default_rng(seed)
+    names = ("Ca", "Cb", "Za", "Zb") if overlap else ("Ca", "Za")
+    out = {k: _encode_io(_normal(g, (B, n_tok, c)), io) for k in names}
+    out["win"] = _encode_io(_normal(g, (B, n_tok, c)), io)
+    out["bias"] = _encode_io(_normal(g, ((2 if overlap else 1) * m, c)), io)
+    return out

@@ -217,6 +217,27 @@ class HcaState(_Request):
         return i
 
 
+def _hca_resume(self, C, Z, entries, win_rows) -> None:
+    """Take over a request after a prefill of n0 = len(C) tokens that wrote ``entries``
+    (its floor(n0/m') finished entries): entries to pages, the open block's rows to the
+    state, the last min(n0, n_win) window rows to the ring."""
+    assert self.n_tok == 0 and self.n_entries == 0
+    C, Z = np.asarray(C, np.float64), np.asarray(Z, np.float64)
+    n0 = C.shape[0]
+    nb = n0 // self.m
+    assert len(entries) == nb
+    for row in entries:
+        self._write_entry(np.asarray(row, np.float64))
+    self.cur_C, self.cur_Z = list(C[self.m * nb:n0]), list(Z[self.m * nb:n0])
+    win_rows = np.asarray(win_rows, np.float64)
+    for p in range(max(n0 - self.n_win, 0), n0):
+        self._push_window(win_rows[p], p)
+    self.n_tok = n0
+
+
+HcaState.resume = _hca_resume
+
+
 def block_tokens(m_csa: int, m_hca: int) -> int:
     """Raw tokens covered by one logical cache block: lcm(m, m') [P1 二(六)]."""
     return math.lcm(m_csa, m_hca)

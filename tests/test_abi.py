@@ -38,6 +38,24 @@ def test_every_declared_function_is_exported():
     assert set(names) == set(csa.EXPORTS)
 
 
+def declared_parameter_counts():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for m in re.finditer(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*((?:csa|hca)_\w+)\s*\(([^)]*)\)\s*;",
+                         src, flags=re.M):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_argument_counts_match_the_header():
+    counts = declared_parameter_counts()
+    assert set(counts) == set(csa.EXPORTS)
+    for name, n in counts.items():
+        assert len(csa._SIGS[name]) == n, f"{name}: binding {len(csa._SIGS[name])} vs header {n}"
+
+
 def test_status_strings_and_version():
     assert csa.status_string(0) == "CSA_OK"
     assert csa.status_string(3) == "CSA_ERR_WORKSPACE"
@@ -173,6 +191,44 @@ def test_attention_checks():
     s = L.hca_dense_mqa(ctypes.byref(p), 1, 1, 1, FAKE, FAKE, FAKE, 10, FAKE, 128, FAKE, None,
                         None, FAKE, None, 0, None)
     assert s == csa.CSA_ERR_UNSUPPORTED
+
+
+def test_state_append_checks():
+    L = csa.lib()
+    p = _p()
+    # p, io, B, pos, Ca, Cb, Za, Zb, win_row, bias, rms_w, finalize, state, win_ring, pages,
+    # n_pages, page_rows, page_table, max_pages, stream
+    base = [ctypes.byref(p), 1, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, FAKE, FAKE,
+            FAKE, 8, 32, FAKE, 4, None]
+
+    def with_(**kw):
+        a = list(base)
+        pos = {"io": 1, "B": 2, "pos": 3, "Cb": 5, "win_row": 8, "finalize": 11, "state": 12,
+               "win_ring": 13, "n_pages": 15, "page_rows": 16, "table": 17, "max_pages": 18}
+        for k, v in kw.items():
+            a[pos[k]] = v
+        return L.csa_state_append(*a)
+
+    assert with_(io=csa.CSA_MXFP4) == csa.CSA_ERR_INVALID_ARG
+    assert with_(B=-1) == csa.CSA_ERR_INVALID_ARG
+    assert with_(finalize=3) == csa.CSA_ERR_INVALID_ARG
+    assert with_(n_pages=0) == csa.CSA_ERR_INVALID_ARG
+    assert with_(page_rows=0) == csa.CSA_ERR_INVALID_ARG
+    assert with_(max_pages=0) == csa.CSA_ERR_INVALID_ARG
+    assert with_(win_ring=None) == csa.CSA_ERR_INVALID_ARG  # window row without a ring
+    assert with_(Cb=None) == csa.CSA_ERR_INVALID_ARG  # CSA needs its b-branch rows
+    assert with_(pos=None) == csa.CSA_ERR_INVALID_ARG
+    assert with_(state=FAKE + 8) == csa.CSA_ERR_INVALID_ARG  # misaligned
+    assert with_(table=None) == csa.CSA_ERR_INVALID_ARG
+    assert with_(B=0) == csa.CSA_OK  # nothing to append, nothing launched
+    hca = _p(overlap=0, m=128)
+    a = list(base)
+    a[0] = ctypes.byref(hca)
+    assert L.csa_state_append(*a) == csa.CSA_ERR_INVALID_ARG  # HCA takes no b-branch rows
+    nowin = _p(n_win=0)
+    a = list(base)
+    a[0] = ctypes.byref(nowin)
+    assert L.csa_state_append(*a) == csa.CSA_ERR_INVALID_ARG  # a ring needs n_win >= 1
 
 
 def test_binding_refuses_host_tensors():

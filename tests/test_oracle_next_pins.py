@@ -263,6 +263,23 @@ def test_prefill_then_decode_equals_whole_prefill(n0):
     assert np.allclose(st.entries(), _whole_csa(Ca, Cb, Za, Zb, bias, m, n), rtol=0, atol=1e-13)
 
 
+@pytest.mark.parametrize("n0", [0, 5, 32, 47])
+def test_hca_prefill_then_decode_equals_whole_prefill(n0):
+    m, c, n, n_win = 16, 16, 16 * 4 + 7, 4
+    C, _, Z, _, Wr = _seq(n, c)
+    bias = RNG.standard_normal((m, c))
+    whole = lambda k: O.finalize_entries(  # noqa: E731
+        O.compress_hca(C[:m * (k // m)], Z[:m * (k // m)], bias, m), 0, m, CFG["r"],
+        CFG["base"], CFG["eps"])
+    st = SC.HcaState(SC.PagePool(8, 1, c), m=m, c=c, bias=bias, n_win=n_win, block_tokens=16,
+                     **CFG)
+    st.resume(C[:n0], Z[:n0], whole(n0), Wr[:n0])
+    for t in range(n0, n):
+        st.append(C[t], Z[t], Wr[t])
+        assert np.array_equal(st.window_rows(t), Wr[max(t - n_win + 1, 0):t + 1])
+    assert np.allclose(st.entries(), whole(n), rtol=0, atol=1e-13)
+
+
 def test_window_ring_holds_the_most_recent_rows():
     m, c, n_win = 4, 8, 6
     Ca, Cb, Za, Zb, Wr = _seq(40, c)
