@@ -126,23 +126,34 @@ csa_status csa_compress(const csa_params* p, csa_dtype io, int32_t B, int64_t n_
  *     csa_compress computes it ([P1] 1(1) / 2(1); the CSA b-branch is block i-1's rows for
  *     i > 0 and absent for i = 0), and with finalize = 1 RMSNorm'd (kv_rms_w [c] or NULL)
  *     and rotated at position m*i ([P1] 3(1), 3(2)). The row goes to row i % page_rows of
- *     page page_table[b, i / page_rows] of `pages` [n_pages, page_rows, c].
+ *     page page_table[b, i / page_rows] of `pages`, stored as out_fmt:
+ *       out_fmt = io: pages [n_pages, page_rows, c] in the io dtype; page_scales unused;
+ *       CSA_FP8_E4M3_ROWSCALE: pages [n_pages, page_rows, c] e4m3 codes (round to nearest
+ *         even, saturating), page_scales [n_pages, page_rows] fp32 = amax(row) / 448;
+ *       CSA_MXFP4 (c = 128, page_rows a multiple of 128; the indexer keys of [P1'] as
+ *         csa_index_scores reads them): pages [n_pages, page_rows, 64] e2m1 pairs (element
+ *         2j in the low nibble), page_scales [n_pages, page_rows, 4] e8m0 exponents
+ *         floor(log2 amax) - 2 of each 32 values, per block of 128 rows with byte
+ *         16*i + 4*j + b holding exponent b of row 32*j + i.
+ *     Indexer keys are compressed like KV entries but take no RMSNorm / RoPE (finalize = 0).
  * The slots of block i-1 and block i are read back, so a request's appends must arrive in
  * position order (one per call), after its state was filled up to t-1: by earlier appends,
  * or, for a request resumed after a prefill, by the caller writing those raw rows into their
  * slots. Requests whose entry's logical page is >= max_pages, whose page id is outside
  * [0, n_pages), or whose position is negative are skipped and leave a device error code
  * (301 position, 302 page slot, 303 page id) for csa_device_error(). The pages use
- * page_rows = 128 / m; with page_table[b, k] = b * max_pages + k they are the contiguous
- * cache [B, N_cap = page_rows * max_pages, c] that the attention calls read.
- * io: CSA_F32 or CSA_BF16 for every tensor (math is fp32); bias: [2m, c] or [m, c].
+ * page_rows = 128 / m (a multiple of it for MXFP4 keys); with page_table[b, k] =
+ * b * max_pages + k they are the contiguous cache [B, N_cap = page_rows * max_pages, ...]
+ * that the attention and indexer calls read.
+ * io: CSA_F32 or CSA_BF16 for every input and state tensor (math is fp32); c <= 4096;
+ * bias: [2m, c] or [m, c].
  */
 csa_status csa_state_append(const csa_params* p, csa_dtype io, int32_t B, const int64_t* pos,
                             const void* Ca, const void* Cb, const void* Za, const void* Zb,
                             const void* win_row, const void* bias, const void* kv_rms_w,
-                            int32_t finalize, void* state, void* win_ring, void* pages,
-                            int32_t n_pages, int32_t page_rows, const int32_t* page_table,
-                            int32_t max_pages, void* stream);
+                            int32_t finalize, void* state, void* win_ring, csa_dtype out_fmt,
+                            void* pages, void* page_scales, int32_t n_pages, int32_t page_rows,
+                            const int32_t* page_table, int32_t max_pages, void* stream);
 
 /*
  * Stage 2 -- lightning-indexer scores ([P1] 1(2)):

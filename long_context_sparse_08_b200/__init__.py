@@ -81,8 +81,8 @@ _SIGS = {
     "csa_version": [],
     "csa_device_error": [ctypes.POINTER(ctypes.c_int32)],
     "csa_kernel_launches": [],
-    "csa_state_append": [_PP, ctypes.c_int, _I32] + [_VP] * 8 + [_I32, _VP, _VP, _VP, _I32, _I32,
-                                                             _VP, _I32, _VP],
+    "csa_state_append": [_PP, ctypes.c_int, _I32] + [_VP] * 8 + [_I32, _VP, _VP, ctypes.c_int,
+                                                             _VP, _VP, _I32, _I32, _VP, _I32, _VP],
 }
 _RES = {"csa_workspace_size": _SZ, "csa_kernel_launches": ctypes.c_uint64, "csa_status_string": ctypes.c_char_p,
         "csa_last_error": ctypes.c_char_p, "csa_version": ctypes.c_char_p,
@@ -181,12 +181,13 @@ def csa_compress(p, io, B, n_tok, first_entry, n_cap, Ca, Cb, Za, Zb, bias, prev
 
 
 def csa_state_append(p, io, B, pos, Ca, Cb, Za, Zb, win_row, bias, kv_rms_w, finalize, state,
-                     win_ring, pages, n_pages, page_rows, page_table, max_pages, stream=None):
+                     win_ring, out_fmt, pages, page_scales, n_pages, page_rows, page_table,
+                     max_pages, stream=None):
     s = lib().csa_state_append(ctypes.byref(p), io, B, _ptr(pos), _ptr(Ca), _ptr(Cb), _ptr(Za),
                                _ptr(Zb), _ptr(win_row), _ptr(bias), _ptr(kv_rms_w),
-                               int(finalize), _ptr(state), _ptr(win_ring), _ptr(pages),
-                               n_pages, page_rows, _ptr(page_table), max_pages,
-                               _stream(stream))
+                               int(finalize), _ptr(state), _ptr(win_ring), int(out_fmt),
+                               _ptr(pages), _ptr(page_scales), n_pages, page_rows,
+                               _ptr(page_table), max_pages, _stream(stream))
     _check("csa_state_append", s)
 
 

@@ -345,11 +345,18 @@ csa_status csa_compress(const csa_params* p, csa_dtype io, int32_t B, int64_t n_
 csa_status csa_state_append(const csa_params* p, csa_dtype io, int32_t B, const int64_t* pos,
                             const void* Ca, const void* Cb, const void* Za, const void* Zb,
                             const void* win_row, const void* bias, const void* kv_rms_w,
-                            int32_t finalize, void* state, void* win_ring, void* pages,
-                            int32_t n_pages, int32_t page_rows, const int32_t* page_table,
-                            int32_t max_pages, void* stream) {
+                            int32_t finalize, void* state, void* win_ring, csa_dtype out_fmt,
+                            void* pages, void* page_scales, int32_t n_pages, int32_t page_rows,
+                            const int32_t* page_table, int32_t max_pages, void* stream) {
   TRY(check_params(p));
   REQUIRE(io == CSA_F32 || io == CSA_BF16, "state io dtype must be CSA_F32 or CSA_BF16");
+  REQUIRE(p->c <= 4096, "state append supports c <= 4096 (got %d)", p->c);
+  REQUIRE(out_fmt == io || out_fmt == CSA_FP8_E4M3_ROWSCALE || out_fmt == CSA_MXFP4,
+          "out_fmt must be the io dtype, CSA_FP8_E4M3_ROWSCALE or CSA_MXFP4");
+  if (out_fmt == CSA_MXFP4) {
+    REQUIRE(p->c == 128, "MXFP4 rows are indexer keys of 128 values (c = %d)", p->c);
+    REQUIRE(page_rows % 128 == 0, "MXFP4 pages hold whole 128-row exponent blocks");
+  }
   REQUIRE(B >= 0 && B <= 65535, "B must be in [0, 65535]");
   REQUIRE(p->overlap == 0 || p->overlap == 1, "overlap must be 0 or 1");
   REQUIRE(finalize == 0 || finalize == 1, "finalize must be 0 or 1");
@@ -372,6 +379,7 @@ csa_status csa_state_append(const csa_params* p, csa_dtype io, int32_t B, const 
   REQUIRE_PTR(state);
   REQUIRE_PTR(pages);
   REQUIRE_PTR(page_table);
+  if (out_fmt != io) REQUIRE_PTR(page_scales);
   OPTIONAL_PTR(win_row);
   OPTIONAL_PTR(win_ring);
   OPTIONAL_PTR(kv_rms_w);
@@ -380,7 +388,10 @@ csa_status csa_state_append(const csa_params* p, csa_dtype io, int32_t B, const 
   a.finalize = finalize; a.n_win = p->n_win; a.n_pages = n_pages; a.page_rows = page_rows;
   a.max_pages = max_pages; a.eps = p->rms_eps; a.pos = pos; a.Ca = Ca; a.Cb = Cb; a.Za = Za;
   a.Zb = Zb; a.win_row = win_row; a.bias = bias; a.rms_w = kv_rms_w; a.state = state;
-  a.win_ring = win_ring; a.pages = pages; a.page_table = page_table;
+  a.win_ring = win_ring; a.pages = pages; a.page_scales = page_scales;
+  a.page_table = page_table;
+  a.out = out_fmt == io ? csa::state::kOutIo
+                        : (out_fmt == CSA_MXFP4 ? csa::state::kOutMxfp4 : csa::state::kOutFp8);
   for (int i = 0; i < p->rope_dims / 2; ++i)
     a.inv_freq[i] = csa::rope_inv_freq(i, p->rope_dims, (double)p->rope_base);
   TRY(cuda_status(csa::launch_state_append(a, io == CSA_BF16, (cudaStream_t)stream),

@@ -24,10 +24,25 @@ __device__ int g_state_error = 0;
 
 enum { kErrBase = 300 };  // stored code = kErrBase - status (301 position, 302 page slot, 303 page id)
 
+// Block-wide max of non-negative values; `red` is shared scratch of >= 32 floats.
+__device__ __forceinline__ float block_max_nonneg(float v, float* red) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  v = warp_max(v);
+  __syncthreads();
+  if (lane == 0) red[wid] = v;
+  __syncthreads();
+  float t = (threadIdx.x < nw) ? red[threadIdx.x] : 0.f;
+  if (wid == 0) t = warp_max(t);
+  if (threadIdx.x == 0) red[0] = t;
+  __syncthreads();
+  return red[0];
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) k_state_append(state::Args a) {
-  extern __shared__ float row[];  // [c]
+  extern __shared__ float row[];  // [2c]: pooled row, then the finished row
   __shared__ float red[32];
+  float* fin = row + a.c;
   const int b = blockIdx.x;
   const int64_t t = a.pos[b];
   int64_t i = 0;
@@ -45,15 +60,44 @@ __global__ void __launch_bounds__(256) k_state_append(state::Args a) {
     row[j] = v;
     ss = fmaf(v, v, ss);
   }
-  T* out = static_cast<T*>(a.pages) + off;
-  if (!a.finalize) {
-    for (int j = threadIdx.x; j < a.c; j += blockDim.x) state::st(out, j, row[j]);
+  float rstd = 1.f;
+  if (a.finalize) {
+    const float tot = block_sum(ss, red);  // also orders the row[] writes before the reads
+    rstd = rsqrtf(tot / (float)a.c + a.eps);
+  }
+  float amax = 0.f;
+  for (int j = threadIdx.x; j < a.c; j += blockDim.x) {
+    const float v = a.finalize ? state::final_channel<T>(a, row, rstd, i, j) : row[j];
+    fin[j] = v;  // read back by this thread only
+    amax = fmaxf(amax, fabsf(v));
+  }
+  if (a.out == state::kOutIo) {
+    T* out = static_cast<T*>(a.pages) + off;
+    for (int j = threadIdx.x; j < a.c; j += blockDim.x) state::st(out, j, fin[j]);
     return;
   }
-  const float tot = block_sum(ss, red);  // also orders the row[] writes before the reads
-  const float rstd = rsqrtf(tot / (float)a.c + a.eps);
-  for (int j = threadIdx.x; j < a.c; j += blockDim.x)
-    state::st(out, j, state::final_channel<T>(a, row, rstd, i, j));
+  const size_t prow = off / (size_t)a.c;  // global row index in the pages
+  if (a.out == state::kOutFp8) {
+    const float scale = state::fp8_row_scale(block_max_nonneg(amax, red));
+    uint8_t* codes = static_cast<uint8_t*>(a.pages) + off;
+    for (int j = threadIdx.x; j < a.c; j += blockDim.x)
+      codes[j] = (uint8_t)state::fp8_code(fin[j], scale);
+    if (threadIdx.x == 0) static_cast<float*>(a.page_scales)[prow] = scale;
+    return;
+  }
+  // MXFP4: a warp's 32 consecutive channels are one MX block (c and blockDim are multiples
+  // of 32, so a warp's lanes are all in or all out of the loop)
+  uint8_t* packed = static_cast<uint8_t*>(a.pages) + off / 2;
+  uint8_t* exps = static_cast<uint8_t*>(a.page_scales);
+  const int slot = (int)(prow % (size_t)a.page_rows);
+  for (int j = threadIdx.x; j < a.c; j += blockDim.x) {
+    const float v = fin[j];
+    const int E = state::mx_exponent(warp_max(fabsf(v)));
+    const uint32_t code = state::e2m1_code(v / state::pow2f(E));
+    const uint32_t hi = __shfl_xor_sync(0xffffffffu, code, 1);
+    if ((j & 1) == 0) packed[j >> 1] = (uint8_t)(code | (hi << 4));
+    if ((j & 31) == 0) exps[state::mx_scale_offset(prow - slot, slot, j >> 5)] = (uint8_t)(E + 127);
+  }
 }
 
 }  // namespace
@@ -61,7 +105,7 @@ __global__ void __launch_bounds__(256) k_state_append(state::Args a) {
 cudaError_t launch_state_append(const state::Args& a, bool bf16, cudaStream_t st) {
   if (a.B == 0) return cudaSuccess;
   const int threads = a.c >= 256 ? 256 : ((a.c + 31) / 32) * 32;
-  const size_t smem = (size_t)a.c * sizeof(float);
+  const size_t smem = 2 * (size_t)a.c * sizeof(float);
   cudaError_t e = bf16 ? launch(false, k_state_append<__nv_bfloat16>, dim3(a.B), dim3(threads),
                                 smem, st, a)
                        : launch(false, k_state_append<float>, dim3(a.B), dim3(threads), smem, st, a);

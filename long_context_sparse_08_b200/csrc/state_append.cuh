@@ -13,11 +13,20 @@
 // of the slot is one of its raw tensors. CSA (overlap): S = 2m, rows Ca, Za, Cb, Zb -- the
 // 2m slots hold the open block (its a- and b-rows) and the previous block (whose b-rows
 // entry i reads). HCA: S = m', rows C, Z.
+//
+// Finished rows are stored in the io dtype, or in the formats the indexers read (the
+// compressed indexer keys are one of the caches a decode step extends):
+//   FP8: e4m3 codes [page_rows, c] per page, one fp32 scale per row (amax / 448);
+//   MXFP4 (c = 128): e2m1 pairs [page_rows, 64] per page (element 2j in the low nibble),
+//     one e8m0 exponent per 32 elements (OCP MX v1.0: floor(log2 amax) - 2), stored per block
+//     of 128 rows with byte 16*i + 4*j + b holding exponent b of row 32*j + i.
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <math.h>
 #include <stdint.h>
+#include <string.h>
 
 namespace csa {
 namespace state {
@@ -35,12 +44,14 @@ enum {
   kErrPageId = -3    // page table entry outside [0, n_pages)
 };
 
+enum { kOutIo = 0, kOutFp8 = 1, kOutMxfp4 = 2 };  // storage of finished rows
+
 struct Args {
-  int B, m, c, overlap, rope_dims, finalize, n_win, n_pages, page_rows, max_pages;
+  int B, m, c, overlap, rope_dims, finalize, n_win, n_pages, page_rows, max_pages, out;
   float eps;
   const int64_t* pos;  // [B] position of each request's new token
   const void *Ca, *Cb, *Za, *Zb, *win_row, *bias, *rms_w;  // new rows [B, c]; bias; gamma
-  void *state, *win_ring, *pages;
+  void *state, *win_ring, *pages, *page_scales;
   const int32_t* page_table;  // [B, max_pages]
   double inv_freq[256];       // RoPE pair frequencies base^(-2p/r), p < r/2
 };
@@ -149,6 +160,57 @@ CSA_HD float final_channel(const Args& a, const float* row, float rstd, int64_t 
     v = ((j - r0) & 1) == 0 ? v * cs - u * sn : u * sn + v * cs;
   }
   return v;
+}
+
+// ---- storage formats of finished rows (the same encodings the input generators use) ----
+
+// e4m3 code of v: nearest value, ties to even, saturating at +-448 (CUDA's conversion).
+CSA_HD uint32_t e4m3_code(float v) {
+  return (uint32_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
+}
+
+// Row scale of the FP8 format: amax / 448 in fp32 (0 for an all-zero row, whose codes are 0).
+CSA_HD float fp8_row_scale(float amax) { return amax / 448.f; }
+CSA_HD uint32_t fp8_code(float v, float scale) {
+  return e4m3_code(v / (scale > 0.f ? scale : 1.f));
+}
+
+// Shared exponent of a 32-element MX block with largest magnitude amax: floor(log2 amax) - 2
+// (2 is e2m1's largest exponent), clamped to e8m0's [-127, 127]; -127 for a zero block.
+CSA_HD int mx_exponent(float amax) {
+  if (!(amax > 0.f)) return -127;
+  int e = 0;
+  frexpf(amax, &e);  // amax = f * 2^e with f in [0.5, 1): floor(log2 amax) = e - 1
+  const int E = e - 1 - 2;
+  return E < -127 ? -127 : (E > 127 ? 127 : E);
+}
+
+// 2^E as a float (E = -127 is a subnormal).
+CSA_HD float pow2f(int E) {
+  const uint32_t u = E >= -126 ? (uint32_t)(E + 127) << 23 : 0x00400000u;
+  float f;
+  memcpy(&f, &u, sizeof(f));
+  return f;
+}
+
+// e2m1 code of v (already divided by its block's 2^E): the nearest magnitude of
+// {0, .5, 1, 1.5, 2, 3, 4, 6} (at a midpoint the even code), saturating at 6; bit 3 is the
+// sign of a negative value with a nonzero magnitude.
+CSA_HD uint32_t e2m1_code(float v) {
+  const float a = fminf(fabsf(v), 6.f);
+  const float mids[7] = {0.25f, 0.75f, 1.25f, 1.75f, 2.5f, 3.5f, 5.f};
+  uint32_t code = 0;
+  for (int k = 0; k < 7; ++k) code += a > mids[k] ? 1u : 0u;
+  for (int k = 1; k < 7; k += 2)
+    if (a == mids[k]) code = (uint32_t)k + 1;  // midpoint above an odd code: round up
+  return (v < 0.f && code > 0) ? (code | 8u) : code;
+}
+
+// Byte offset, in a page's MXFP4 exponents, of exponent b of page row `row`: rows are
+// stored in blocks of 128 with byte 16*i + 4*j + b holding exponent b of row 32*j + i.
+CSA_HD size_t mx_scale_offset(size_t page_row0, int row, int b) {
+  const int blk = row / 128, kk = row % 128;
+  return (page_row0 + (size_t)blk * 128) * 4 + (size_t)(16 * (kk % 32) + 4 * (kk / 32) + b);
 }
 
 #undef CSA_HD

@@ -30,6 +30,8 @@ Readings where the pages leave the mechanics open:
   S4  Finished entries live in pages of one logical block (128 raw tokens): 32 CSA entries
       or 1 HCA entry. A request takes a page from a shared pool when its first entry of
       a new block is written, and a page table maps its logical pages to physical ones.
+  S5  The compressed indexer keys are extended the same way, without RMSNorm / RoPE (the
+      pages attach those to the attention's queries and KV entries only): finalize=False.
 """
 from __future__ import annotations
 
@@ -111,11 +113,13 @@ class CsaState(_Request):
     """One request's CSA state cache (S1) and its pages of finished entries."""
 
     def __init__(self, pool: PagePool, *, m: int, c: int, bias, n_win: int, r: int,
-                 base: float, eps: float, gamma=None, block_tokens: int = 128):
+                 base: float, eps: float, gamma=None, block_tokens: int = 128,
+                 finalize: bool = True):
         super().__init__(pool, m, c, n_win, block_tokens)
         bias = np.asarray(bias, np.float64)
         self.Ba, self.Bb = bias[:m], bias[m:2 * m]
         self.r, self.base, self.eps, self.gamma = r, base, eps, gamma
+        self.finalize = finalize
         self.cur = {k: [] for k in ("Ca", "Za", "Cb", "Zb")}  # rows of the open block
         self.prev_Cb: Optional[np.ndarray] = None  # b-rows of the last finished block
         self.prev_Zb: Optional[np.ndarray] = None
@@ -158,6 +162,8 @@ class CsaState(_Request):
         return self._finalize(entry, i)
 
     def _finalize(self, entry, i: int) -> np.ndarray:
+        if not self.finalize:  # indexer keys (S5)
+            return entry
         return O.finalize_entries(entry[None], i, self.m, self.r, self.base, self.eps,
                                   self.gamma)[0]
 
@@ -189,10 +195,12 @@ class HcaState(_Request):
     """One request's HCA state cache (S2) and its pages of finished entries."""
 
     def __init__(self, pool: PagePool, *, m: int, c: int, bias, n_win: int, r: int,
-                 base: float, eps: float, gamma=None, block_tokens: int = 128):
+                 base: float, eps: float, gamma=None, block_tokens: int = 128,
+                 finalize: bool = True):
         super().__init__(pool, m, c, n_win, block_tokens)
         self.B = np.asarray(bias, np.float64)
         self.r, self.base, self.eps, self.gamma = r, base, eps, gamma
+        self.finalize = finalize
         self.cur_C: List[np.ndarray] = []
         self.cur_Z: List[np.ndarray] = []
 
@@ -211,8 +219,10 @@ class HcaState(_Request):
         i = t // self.m
         S = O._softmax_rows(np.stack(self.cur_Z) + self.B)
         entry = (S * np.stack(self.cur_C)).sum(axis=0)
-        self._write_entry(O.finalize_entries(entry[None], i, self.m, self.r, self.base,
-                                             self.eps, self.gamma)[0])
+        if self.finalize:
+            entry = O.finalize_entries(entry[None], i, self.m, self.r, self.base, self.eps,
+                                       self.gamma)[0]
+        self._write_entry(entry)
         self.cur_C, self.cur_Z = [], []
         return i
 

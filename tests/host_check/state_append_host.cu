@@ -11,11 +11,48 @@
 
 namespace {
 
+using namespace csa::state;
+
+// One finished row `fin` [c] stored at page row `prow` in the chosen format; returns a
+// negative code if an offset would fall outside its buffer.
+int store_row(const Args& a, const std::vector<float>& fin, size_t prow, size_t page_bytes,
+              size_t scale_bytes) {
+  const int c = a.c;
+  if (a.out == kOutFp8) {
+    if ((prow + 1) * c > page_bytes || (prow + 1) * sizeof(float) > scale_bytes) return -13;
+    float amax = 0.f;
+    for (int j = 0; j < c; ++j) amax = fmaxf(amax, fabsf(fin[j]));
+    const float scale = fp8_row_scale(amax);
+    uint8_t* codes = static_cast<uint8_t*>(a.pages) + prow * c;
+    for (int j = 0; j < c; ++j) codes[j] = (uint8_t)fp8_code(fin[j], scale);
+    static_cast<float*>(a.page_scales)[prow] = scale;
+    return 0;
+  }
+  // MXFP4
+  if ((prow + 1) * (c / 2) > page_bytes) return -14;
+  uint8_t* packed = static_cast<uint8_t*>(a.pages) + prow * (c / 2);
+  uint8_t* exps = static_cast<uint8_t*>(a.page_scales);
+  const int slot = (int)(prow % (size_t)a.page_rows);
+  for (int blk = 0; blk < c / 32; ++blk) {
+    float amax = 0.f;
+    for (int k = 0; k < 32; ++k) amax = fmaxf(amax, fabsf(fin[32 * blk + k]));
+    const int E = mx_exponent(amax);
+    for (int k = 0; k < 32; k += 2) {
+      const int j = 32 * blk + k;
+      const uint32_t lo = e2m1_code(fin[j] / pow2f(E)), hi = e2m1_code(fin[j + 1] / pow2f(E));
+      packed[j >> 1] = (uint8_t)(lo | (hi << 4));
+    }
+    const size_t so = mx_scale_offset(prow - slot, slot, blk);
+    if (so >= scale_bytes) return -15;
+    exps[so] = (uint8_t)(E + 127);
+  }
+  return 0;
+}
+
 template <typename T>
-int run(csa::state::Args a, int32_t* status, size_t state_elems, size_t ring_elems,
-        size_t page_elems) {
-  using namespace csa::state;
-  std::vector<float> row(a.c);
+int run(Args a, int32_t* status, size_t state_elems, size_t ring_elems, size_t page_bytes,
+        size_t scale_bytes) {
+  std::vector<float> row(a.c), fin(a.c);
   for (int b = 0; b < a.B; ++b) {
     const int64_t t = a.pos[b];
     int64_t i = 0;
@@ -31,43 +68,67 @@ int run(csa::state::Args a, int32_t* status, size_t state_elems, size_t ring_ele
       store_channel<T>(a, b, t, j);
     }
     if (s == kAppendOnly) continue;
-    if (off + (size_t)a.c > page_elems) return -12;
-    float ssf = 0.f;
+    float ss = 0.f;
     for (int j = 0; j < a.c; ++j) {
       row[j] = pool_channel<T>(a, b, i, j);
-      ssf = fmaf(row[j], row[j], ssf);
+      ss = fmaf(row[j], row[j], ss);
     }
-    T* out = static_cast<T*>(a.pages) + off;
-    if (!a.finalize) {
-      for (int j = 0; j < a.c; ++j) st(out, j, row[j]);
+    const float rstd = a.finalize ? 1.f / sqrtf(ss / (float)a.c + a.eps) : 1.f;
+    for (int j = 0; j < a.c; ++j)
+      fin[j] = a.finalize ? final_channel<T>(a, row.data(), rstd, i, j) : row[j];
+    if (a.out == kOutIo) {
+      if ((off + a.c) * sizeof(T) > page_bytes) return -12;
+      T* out = static_cast<T*>(a.pages) + off;
+      for (int j = 0; j < a.c; ++j) st(out, j, fin[j]);
       continue;
     }
-    const float rstd = 1.f / sqrtf(ssf / (float)a.c + a.eps);
-    for (int j = 0; j < a.c; ++j) st(out, j, final_channel<T>(a, row.data(), rstd, i, j));
+    const int rc = store_row(a, fin, off / (size_t)a.c, page_bytes, scale_bytes);
+    if (rc != 0) return rc;
   }
   return 0;
 }
 
 }  // namespace
 
+// out: 0 = io dtype, 1 = FP8 rows, 2 = MXFP4 rows; page_bytes / scale_bytes: buffer sizes.
 extern "C" int state_append_host(int bf16, int B, int m, int c, int overlap, int rope_dims,
                                  double rope_base, int finalize, int n_win, int n_pages,
-                                 int page_rows, int max_pages, float eps, const int64_t* pos,
-                                 const void* Ca, const void* Cb, const void* Za, const void* Zb,
-                                 const void* win_row, const void* bias, const void* rms_w,
-                                 void* state, void* win_ring, void* pages,
+                                 int page_rows, int max_pages, float eps, int out,
+                                 const int64_t* pos, const void* Ca, const void* Cb,
+                                 const void* Za, const void* Zb, const void* win_row,
+                                 const void* bias, const void* rms_w, void* state,
+                                 void* win_ring, void* pages, size_t page_bytes,
+                                 void* page_scales, size_t scale_bytes,
                                  const int32_t* page_table, int32_t* status) {
-  csa::state::Args a{};
+  Args a{};
   a.B = B; a.m = m; a.c = c; a.overlap = overlap; a.rope_dims = rope_dims;
   a.finalize = finalize; a.n_win = n_win; a.n_pages = n_pages; a.page_rows = page_rows;
-  a.max_pages = max_pages; a.eps = eps; a.pos = pos; a.Ca = Ca; a.Cb = Cb; a.Za = Za;
-  a.Zb = Zb; a.win_row = win_row; a.bias = bias; a.rms_w = rms_w; a.state = state;
-  a.win_ring = win_ring; a.pages = pages; a.page_table = page_table;
+  a.max_pages = max_pages; a.eps = eps; a.out = out; a.pos = pos; a.Ca = Ca; a.Cb = Cb;
+  a.Za = Za; a.Zb = Zb; a.win_row = win_row; a.bias = bias; a.rms_w = rms_w; a.state = state;
+  a.win_ring = win_ring; a.pages = pages; a.page_scales = page_scales;
+  a.page_table = page_table;
   for (int p = 0; p < rope_dims / 2; ++p)
     a.inv_freq[p] = std::exp2(-2.0 * p / rope_dims * std::log2(rope_base));
   const size_t state_elems = (size_t)B * (overlap ? 2 * m : m) * (overlap ? 4 : 2) * c;
   const size_t ring_elems = (size_t)B * (n_win > 0 ? n_win : 0) * c;
-  const size_t page_elems = (size_t)n_pages * page_rows * c;
-  return bf16 ? run<__nv_bfloat16>(a, status, state_elems, ring_elems, page_elems)
-              : run<float>(a, status, state_elems, ring_elems, page_elems);
+  return bf16 ? run<__nv_bfloat16>(a, status, state_elems, ring_elems, page_bytes, scale_bytes)
+              : run<float>(a, status, state_elems, ring_elems, page_bytes, scale_bytes);
+}
+
+// The row encoders alone: rows [n, c] fp32 -> FP8 (out = 1: codes [n, c], scales [n] fp32)
+// or MXFP4 (out = 2: packed [n, c/2], exponents [n, 4] in the 128-row blocked layout;
+// n a multiple of 128, c = 128).
+extern "C" int encode_rows_host(int out, int n, int c, const float* rows, void* codes,
+                                void* scales) {
+  Args a{};
+  a.c = c; a.out = out; a.page_rows = n; a.pages = codes; a.page_scales = scales;
+  std::vector<float> fin(c);
+  const size_t page_bytes = out == kOutFp8 ? (size_t)n * c : (size_t)n * c / 2;
+  const size_t scale_bytes = out == kOutFp8 ? (size_t)n * sizeof(float) : (size_t)n * 4;
+  for (int r = 0; r < n; ++r) {
+    for (int j = 0; j < c; ++j) fin[j] = rows[(size_t)r * c + j];
+    const int rc = store_row(a, fin, (size_t)r, page_bytes, scale_bytes);
+    if (rc != 0) return rc;
+  }
+  return 0;
 }

@@ -196,15 +196,16 @@ def test_attention_checks():
 def test_state_append_checks():
     L = csa.lib()
     p = _p()
-    # p, io, B, pos, Ca, Cb, Za, Zb, win_row, bias, rms_w, finalize, state, win_ring, pages,
-    # n_pages, page_rows, page_table, max_pages, stream
+    # p, io, B, pos, Ca, Cb, Za, Zb, win_row, bias, rms_w, finalize, state, win_ring, out_fmt,
+    # pages, page_scales, n_pages, page_rows, page_table, max_pages, stream
     base = [ctypes.byref(p), 1, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, FAKE, FAKE,
-            FAKE, 8, 32, FAKE, 4, None]
+            1, FAKE, None, 8, 32, FAKE, 4, None]
 
     def with_(**kw):
         a = list(base)
         pos = {"io": 1, "B": 2, "pos": 3, "Cb": 5, "win_row": 8, "finalize": 11, "state": 12,
-               "win_ring": 13, "n_pages": 15, "page_rows": 16, "table": 17, "max_pages": 18}
+               "win_ring": 13, "out": 14, "scales": 16, "n_pages": 17, "page_rows": 18,
+               "table": 19, "max_pages": 20}
         for k, v in kw.items():
             a[pos[k]] = v
         return L.csa_state_append(*a)
@@ -221,6 +222,16 @@ def test_state_append_checks():
     assert with_(state=FAKE + 8) == csa.CSA_ERR_INVALID_ARG  # misaligned
     assert with_(table=None) == csa.CSA_ERR_INVALID_ARG
     assert with_(B=0) == csa.CSA_OK  # nothing to append, nothing launched
+    assert with_(out=csa.CSA_F32) == csa.CSA_ERR_INVALID_ARG  # neither io nor an indexer format
+    assert with_(out=csa.CSA_FP8_E4M3_ROWSCALE) == csa.CSA_ERR_INVALID_ARG  # no scales
+    assert with_(out=csa.CSA_MXFP4, scales=FAKE) == csa.CSA_ERR_INVALID_ARG  # c = 512
+    keys = _p(c=128)
+    a = list(base)
+    a[0], a[14], a[16] = ctypes.byref(keys), csa.CSA_MXFP4, FAKE
+    assert L.csa_state_append(*a) == csa.CSA_ERR_INVALID_ARG  # 32-row pages split a block
+    a[18] = 128
+    a[2] = 0
+    assert L.csa_state_append(*a) == csa.CSA_OK
     hca = _p(overlap=0, m=128)
     a = list(base)
     a[0] = ctypes.byref(hca)

@@ -280,6 +280,19 @@ def test_hca_prefill_then_decode_equals_whole_prefill(n0):
     assert np.allclose(st.entries(), whole(n), rtol=0, atol=1e-13)
 
 
+def test_indexer_key_state_gives_the_raw_compressed_keys():
+    # keys take no RMSNorm / RoPE: token-by-token entries equal the plain compression
+    m, c, n = 4, 16, 70
+    Ca, Cb, Za, Zb, Wr = _seq(n, c)
+    bias = RNG.standard_normal((2 * m, c))
+    st = SC.CsaState(SC.PagePool(2, 32, c), m=m, c=c, bias=bias, n_win=4, finalize=False, **CFG)
+    for t in range(n):
+        st.append(Ca[t], Cb[t], Za[t], Zb[t], Wr[t])
+    nb = n // m
+    want = O.compress_csa(Ca[:m * nb], Cb[:m * nb], Za[:m * nb], Zb[:m * nb], bias, m)
+    assert np.allclose(st.entries(), want, rtol=0, atol=1e-13)
+
+
 def test_window_ring_holds_the_most_recent_rows():
     m, c, n_win = 4, 8, 6
     Ca, Cb, Za, Zb, Wr = _seq(40, c)
