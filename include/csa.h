@@ -56,8 +56,11 @@ typedef enum {
   CSA_F32 = 0,               /* IEEE binary32 */
   CSA_BF16 = 1,              /* bfloat16 */
   CSA_FP8_E4M3_ROWSCALE = 2, /* OCP e4m3 codes, one fp32 scale per row (value = code * scale) */
-  CSA_MXFP4 = 3              /* OCP MXFP4: e2m1 pairs per byte (element 2j in the low nibble)
+  CSA_MXFP4 = 3,             /* OCP MXFP4: e2m1 pairs per byte (element 2j in the low nibble)
                                 and one e8m0 scale byte per 32 elements */
+  CSA_MIXED_FP8_BF16 = 4     /* KV entry row ([P1] 一(三)4 item 1): the first c-r values as e4m3
+                                codes with one fp32 scale per row (amax of those values / 448),
+                                then the last r (RoPE) values as bf16: c + r bytes per row */
 } csa_dtype;
 
 /* Method constants, passed by pointer, read on the host during the call only. */
@@ -134,7 +137,10 @@ csa_status csa_compress(const csa_params* p, csa_dtype io, int32_t B, int64_t n_
  *         csa_index_scores reads them): pages [n_pages, page_rows, 64] e2m1 pairs (element
  *         2j in the low nibble), page_scales [n_pages, page_rows, 4] e8m0 exponents
  *         floor(log2 amax) - 2 of each 32 values, per block of 128 rows with byte
- *         16*i + 4*j + b holding exponent b of row 32*j + i.
+ *         16*i + 4*j + b holding exponent b of row 32*j + i;
+ *       CSA_MIXED_FP8_BF16 (0 < r < c): pages [n_pages, page_rows, c + r] bytes, each row the
+ *         e4m3 codes of its first c-r values then its last r values as bf16; page_scales
+ *         [n_pages, page_rows] fp32 = amax(first c-r values) / 448.
  *     Indexer keys are compressed like KV entries but take no RMSNorm / RoPE (finalize = 0).
  * The slots of block i-1 and block i are read back, so a request's appends must arrive in
  * position order (one per call), after its state was filled up to t-1: by earlier appends,

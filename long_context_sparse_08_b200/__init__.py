@@ -15,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libcsa.so")
 
 CSA_OK, CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_WORKSPACE, CSA_ERR_CUDA = range(5)
-CSA_F32, CSA_BF16, CSA_FP8_E4M3_ROWSCALE, CSA_MXFP4 = range(4)
+CSA_F32, CSA_BF16, CSA_FP8_E4M3_ROWSCALE, CSA_MXFP4, CSA_MIXED_FP8_BF16 = range(5)
 DTYPES = {"f32": CSA_F32, "bf16": CSA_BF16, "fp8": CSA_FP8_E4M3_ROWSCALE, "mxfp4": CSA_MXFP4}
 CSA_WS_INDEX_TOPK, CSA_WS_TOPK, CSA_WS_SPARSE_MQA, CSA_WS_HCA_MQA, CSA_WS_FORWARD = range(1, 6)
 

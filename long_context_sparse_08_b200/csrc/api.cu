@@ -351,8 +351,11 @@ csa_status csa_state_append(const csa_params* p, csa_dtype io, int32_t B, const 
   TRY(check_params(p));
   REQUIRE(io == CSA_F32 || io == CSA_BF16, "state io dtype must be CSA_F32 or CSA_BF16");
   REQUIRE(p->c <= 4096, "state append supports c <= 4096 (got %d)", p->c);
-  REQUIRE(out_fmt == io || out_fmt == CSA_FP8_E4M3_ROWSCALE || out_fmt == CSA_MXFP4,
-          "out_fmt must be the io dtype, CSA_FP8_E4M3_ROWSCALE or CSA_MXFP4");
+  REQUIRE(out_fmt == io || out_fmt == CSA_FP8_E4M3_ROWSCALE || out_fmt == CSA_MXFP4 ||
+              out_fmt == CSA_MIXED_FP8_BF16,
+          "out_fmt must be the io dtype, CSA_FP8_E4M3_ROWSCALE, CSA_MXFP4 or CSA_MIXED_FP8_BF16");
+  if (out_fmt == CSA_MIXED_FP8_BF16)
+    REQUIRE(p->rope_dims > 0 && p->rope_dims < p->c, "mixed rows need 0 < rope_dims < c");
   if (out_fmt == CSA_MXFP4) {
     REQUIRE(p->c == 128, "MXFP4 rows are indexer keys of 128 values (c = %d)", p->c);
     REQUIRE(page_rows % 128 == 0, "MXFP4 pages hold whole 128-row exponent blocks");
@@ -390,8 +393,10 @@ csa_status csa_state_append(const csa_params* p, csa_dtype io, int32_t B, const 
   a.Zb = Zb; a.win_row = win_row; a.bias = bias; a.rms_w = kv_rms_w; a.state = state;
   a.win_ring = win_ring; a.pages = pages; a.page_scales = page_scales;
   a.page_table = page_table;
-  a.out = out_fmt == io ? csa::state::kOutIo
-                        : (out_fmt == CSA_MXFP4 ? csa::state::kOutMxfp4 : csa::state::kOutFp8);
+  a.out = out_fmt == io                   ? csa::state::kOutIo
+          : out_fmt == CSA_MXFP4          ? csa::state::kOutMxfp4
+          : out_fmt == CSA_MIXED_FP8_BF16 ? csa::state::kOutMixed
+                                          : csa::state::kOutFp8;
   for (int i = 0; i < p->rope_dims / 2; ++i)
     a.inv_freq[i] = csa::rope_inv_freq(i, p->rope_dims, (double)p->rope_base);
   TRY(cuda_status(csa::launch_state_append(a, io == CSA_BF16, (cudaStream_t)stream),

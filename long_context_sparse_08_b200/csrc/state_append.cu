@@ -77,6 +77,21 @@ __global__ void __launch_bounds__(256) k_state_append(state::Args a) {
     return;
   }
   const size_t prow = off / (size_t)a.c;  // global row index in the pages
+  if (a.out == state::kOutMixed) {
+    // e4m3 for the first c - r values (their own amax), bf16 for the RoPE values
+    const int r0 = a.c - a.rope_dims;
+    float am = 0.f;
+    for (int j = threadIdx.x; j < r0; j += blockDim.x) am = fmaxf(am, fabsf(fin[j]));
+    const float scale = state::fp8_row_scale(block_max_nonneg(am, red));
+    uint8_t* rowp = static_cast<uint8_t*>(a.pages) + prow * (size_t)(a.c + a.rope_dims);
+    __nv_bfloat16* rope = reinterpret_cast<__nv_bfloat16*>(rowp + r0);
+    for (int j = threadIdx.x; j < a.c; j += blockDim.x) {
+      if (j < r0) rowp[j] = (uint8_t)state::fp8_code(fin[j], scale);
+      else rope[j - r0] = __float2bfloat16_rn(fin[j]);
+    }
+    if (threadIdx.x == 0) static_cast<float*>(a.page_scales)[prow] = scale;
+    return;
+  }
   if (a.out == state::kOutFp8) {
     const float scale = state::fp8_row_scale(block_max_nonneg(amax, red));
     uint8_t* codes = static_cast<uint8_t*>(a.pages) + off;

@@ -20,6 +20,9 @@
 //   MXFP4 (c = 128): e2m1 pairs [page_rows, 64] per page (element 2j in the low nibble),
 //     one e8m0 exponent per 32 elements (OCP MX v1.0: floor(log2 amax) - 2), stored per block
 //     of 128 rows with byte 16*i + 4*j + b holding exponent b of row 32*j + i.
+// and the KV entries in the mixed precision of 一(三)4 item 1:
+//   mixed: c + r bytes per row, the e4m3 codes of the first c-r values (one fp32 row scale,
+//     amax of those values / 448) then the last r (RoPE) values as bf16.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -44,7 +47,7 @@ enum {
   kErrPageId = -3    // page table entry outside [0, n_pages)
 };
 
-enum { kOutIo = 0, kOutFp8 = 1, kOutMxfp4 = 2 };  // storage of finished rows
+enum { kOutIo = 0, kOutFp8 = 1, kOutMxfp4 = 2, kOutMixed = 3 };  // storage of finished rows
 
 struct Args {
   int B, m, c, overlap, rope_dims, finalize, n_win, n_pages, page_rows, max_pages, out;

@@ -18,6 +18,22 @@ using namespace csa::state;
 int store_row(const Args& a, const std::vector<float>& fin, size_t prow, size_t page_bytes,
               size_t scale_bytes) {
   const int c = a.c;
+  if (a.out == kOutMixed) {
+    const int r0 = c - a.rope_dims;
+    const size_t rb = (size_t)(c + a.rope_dims);
+    if ((prow + 1) * rb > page_bytes || (prow + 1) * sizeof(float) > scale_bytes) return -16;
+    float amax = 0.f;
+    for (int j = 0; j < r0; ++j) amax = fmaxf(amax, fabsf(fin[j]));
+    const float scale = fp8_row_scale(amax);
+    uint8_t* rowp = static_cast<uint8_t*>(a.pages) + prow * rb;
+    __nv_bfloat16* rope = reinterpret_cast<__nv_bfloat16*>(rowp + r0);
+    for (int j = 0; j < c; ++j) {
+      if (j < r0) rowp[j] = (uint8_t)fp8_code(fin[j], scale);
+      else rope[j - r0] = __float2bfloat16_rn(fin[j]);
+    }
+    static_cast<float*>(a.page_scales)[prow] = scale;
+    return 0;
+  }
   if (a.out == kOutFp8) {
     if ((prow + 1) * c > page_bytes || (prow + 1) * sizeof(float) > scale_bytes) return -13;
     float amax = 0.f;
@@ -90,7 +106,8 @@ int run(Args a, int32_t* status, size_t state_elems, size_t ring_elems, size_t p
 
 }  // namespace
 
-// out: 0 = io dtype, 1 = FP8 rows, 2 = MXFP4 rows; page_bytes / scale_bytes: buffer sizes.
+// out: 0 = io dtype, 1 = FP8 rows, 2 = MXFP4 rows, 3 = mixed FP8 / bf16 rows;
+// page_bytes / scale_bytes: buffer sizes.
 extern "C" int state_append_host(int bf16, int B, int m, int c, int overlap, int rope_dims,
                                  double rope_base, int finalize, int n_win, int n_pages,
                                  int page_rows, int max_pages, float eps, int out,

@@ -232,6 +232,12 @@ def test_state_append_checks():
     a[18] = 128
     a[2] = 0
     assert L.csa_state_append(*a) == csa.CSA_OK
+    norope = _p(rope_dims=0)
+    a = list(base)
+    a[0], a[14], a[16] = ctypes.byref(norope), csa.CSA_MIXED_FP8_BF16, FAKE
+    assert L.csa_state_append(*a) == csa.CSA_ERR_INVALID_ARG  # mixed rows need RoPE dims
+    assert with_(out=csa.CSA_MIXED_FP8_BF16) == csa.CSA_ERR_INVALID_ARG  # no scales
+    assert with_(out=csa.CSA_MIXED_FP8_BF16, scales=FAKE, B=0) == csa.CSA_OK
     hca = _p(overlap=0, m=128)
     a = list(base)
     a[0] = ctypes.byref(hca)

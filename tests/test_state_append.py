@@ -36,7 +36,7 @@ CASES = [
     ("hca", 128, 0, 1, (0, 300), 300),
 ]
 C, R, N_WIN, BASE, EPS = 512, 64, 128, 10000.0, 1e-6
-OUT_IO, OUT_FP8, OUT_MXFP4 = 0, 1, 2
+OUT_IO, OUT_FP8, OUT_MXFP4, OUT_MIXED = 0, 1, 2, 3
 
 
 @functools.lru_cache(maxsize=1)
@@ -102,6 +102,9 @@ class Scenario:
             self.scales = None
         elif self.out == OUT_FP8:
             self.pages = np.zeros((n, pr, c), np.uint8)
+            self.scales = np.zeros((n, pr), np.float32)
+        elif self.out == OUT_MIXED:
+            self.pages = np.zeros((n, pr, c + R), np.uint8)
             self.scales = np.zeros((n, pr), np.float32)
         else:
             self.pages = np.zeros((n, pr, c // 2), np.uint8)
@@ -183,7 +186,8 @@ class Scenario:
         return [(b, i) for b in range(self.B) for i in range(*self.entry_range(b))]
 
     def keys(self, pages):
-        """fp32 keys of the appended entries [n, c], from pages stored as f32."""
+        """fp32 rows (keys or KV entries) the appends finished, [n, c], from pages stored as
+        f32."""
         return np.stack([pages[self.page_row(b, i)] for b, i in self.appended()])
 
     def check_encoded(self, keys_f32, pages, scales, what):
@@ -194,6 +198,21 @@ class Scenario:
         ref = np.stack([ora[b].entries()[i] for b, i in at])
         U.check_rows(keys_f32, ref, "f32", f"{what}: fp32 keys")
         got = np.stack([pages[self.page_row(b, i)] for b, i in at])
+        if self.out == OUT_MIXED:
+            codes, sc, rope = W.quant_mixed_kv(keys_f32, R)
+            got_sc = np.array([scales[self.page_row(b, i)] for b, i in at])
+            r0 = self.c - R
+            got_rope = np.ascontiguousarray(got[:, r0:]).view(np.uint16)
+            assert np.array_equal(got[:, :r0], codes), f"{what}: e4m3 codes"
+            assert np.array_equal(got_sc, sc), f"{what}: row scales"
+            assert np.array_equal(got_rope, rope), f"{what}: bf16 RoPE values"
+            dq = O.dec_mixed_kv(got[:, :r0], got_sc, got_rope)
+            rms = np.sqrt(np.mean(ref * ref, axis=1, keepdims=True))
+            bound = np.concatenate([
+                np.maximum(np.abs(ref[:, :r0]) * 2.0 ** -4, got_sc[:, None] * 2.0 ** -10) * 1.01,
+                np.abs(ref[:, r0:]) * 2.0 ** -8 * 1.01], axis=1) + 2e-4 * rms
+            assert np.all(np.abs(dq - ref) <= bound), f"{what}: mixed rows vs oracle"
+            return
         if self.out == OUT_FP8:
             codes, sc = W.quant_fp8_rowwise(keys_f32)
             got_sc = np.array([scales[self.page_row(b, i)] for b, i in at])
@@ -260,6 +279,20 @@ def test_host_build_stores_indexer_keys_in_the_indexer_formats(out):
     pages_f32 = _run_host(plain)[0]
     pages = _run_host(enc)[0]
     enc.check_encoded(plain.keys(pages_f32), pages, enc.scales, f"host keys {out}")
+
+
+def _mixed_scenarios():
+    # KV entries (c = 512, RMSNorm + RoPE) stored with their RoPE dims in bf16 and the rest
+    # in FP8; pages of 32 entries
+    return [Scenario("kv", 4, 1, 32, (0, 150, 256), 120, io="f32", out=o, seed=41)
+            for o in (OUT_IO, OUT_MIXED)]
+
+
+def test_host_build_stores_mixed_precision_kv_rows():
+    plain, enc = _mixed_scenarios()
+    pages_f32 = _run_host(plain)[0]
+    pages = _run_host(enc)[0]
+    enc.check_encoded(plain.keys(pages_f32), pages, enc.scales, "host mixed KV")
 
 
 def test_host_encoders_equal_the_input_encoders():
@@ -339,7 +372,8 @@ def _run_gpu(sc: Scenario, check_error=True):
     p = csa.make_params(m=sc.m, overlap=sc.overlap, c=sc.c, rope_dims=R, rope_base=BASE,
                         rms_eps=EPS, n_win=sc.n_win)
     io = csa.CSA_BF16 if sc.io == "bf16" else csa.CSA_F32
-    out_fmt = {OUT_IO: io, OUT_FP8: csa.CSA_FP8_E4M3_ROWSCALE, OUT_MXFP4: csa.CSA_MXFP4}[sc.out]
+    out_fmt = {OUT_IO: io, OUT_FP8: csa.CSA_FP8_E4M3_ROWSCALE, OUT_MXFP4: csa.CSA_MXFP4,
+               OUT_MIXED: csa.CSA_MIXED_FP8_BF16}[sc.out]
     state, ring, pages = up(sc.state), up(sc.ring), up(sc.pages)
     scales = None if sc.scales is None else up(sc.scales)
     table = up(sc.page_table)
@@ -376,6 +410,14 @@ def test_gpu_stores_indexer_keys_in_the_indexer_formats(out):
     pages_f32 = _run_gpu(plain)[0]
     pages, _, _, scales = _run_gpu(enc)
     enc.check_encoded(plain.keys(pages_f32), pages, scales, f"gpu keys {out}")
+
+
+@pytest.mark.gpu
+def test_gpu_stores_mixed_precision_kv_rows():
+    plain, enc = _mixed_scenarios()
+    pages_f32 = _run_gpu(plain)[0]
+    pages, _, _, scales = _run_gpu(enc)
+    enc.check_encoded(plain.keys(pages_f32), pages, scales, "gpu mixed KV")
 
 
 @pytest.mark.gpu
