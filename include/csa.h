@@ -245,6 +245,29 @@ csa_status hca_dense_mqa(const csa_params* p, csa_dtype io, int32_t B, int32_t T
                          const int64_t* win_pos0, const float* sink, const void* q_rms_w,
                          void* out, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * Stage 4 over a mixed-precision KV cache ([P1] 一(三)4 item 1: the RoPE dims in BF16, the
+ * rest in FP8): as csa_sparse_mqa / hca_dense_mqa with io = CSA_BF16, except that
+ * kv_rows [B, N_cap, c + r] bytes holds each cache row as CSA_MIXED_FP8_BF16 (the e4m3
+ * codes of its first c - r values, then its last r values as bf16) and kv_scale
+ * [B, N_cap] fp32 the rows' FP8 scales (value = code * scale), as csa_state_append writes
+ * them. Window rows stay bf16. The attention widens code * scale to bf16 (one rounding) and
+ * then runs as in the bf16 path. Needs c = 512, n_heads a multiple of 64 and rope_dims a
+ * multiple of 16 in (0, 512), else CSA_ERR_UNSUPPORTED. Workspace: as the bf16 calls.
+ */
+csa_status csa_sparse_mqa_mixed_kv(const csa_params* p, int32_t B, int32_t T, const void* q,
+                                   const int64_t* q_pos, const void* kv_rows,
+                                   const float* kv_scale, int64_t N_cap, const int32_t* idx,
+                                   const void* win_kv, int64_t L_raw, const int64_t* win_pos0,
+                                   const float* sink, const void* q_rms_w, void* out, void* ws,
+                                   size_t ws_bytes, void* stream);
+csa_status hca_dense_mqa_mixed_kv(const csa_params* p, int32_t B, int32_t T, const void* q,
+                                  const int64_t* q_pos, const void* kv_rows,
+                                  const float* kv_scale, int64_t N_cap, const void* win_kv,
+                                  int64_t L_raw, const int64_t* win_pos0, const float* sink,
+                                  const void* q_rms_w, void* out, void* ws, size_t ws_bytes,
+                                  void* stream);
+
 /* Inputs of the fused CSA layer call. Pointers as in the stage calls above. */
 typedef struct {
   /* optional compression of a new chunk into kv_cache (skipped when Ca == NULL) */

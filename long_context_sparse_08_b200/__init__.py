@@ -23,7 +23,8 @@ EXPORTS = (
     "csa_compress", "csa_index_scores", "csa_topk", "csa_index_topk", "csa_sparse_mqa",
     "hca_dense_mqa", "csa_forward", "csa_workspace_size", "csa_status_string",
     "csa_last_error", "csa_set_index_timing_events", "csa_version", "csa_device_error",
-    "csa_topk_noalloc", "csa_kernel_launches", "csa_state_append",
+    "csa_topk_noalloc", "csa_kernel_launches", "csa_state_append", "csa_sparse_mqa_mixed_kv",
+    "hca_dense_mqa_mixed_kv",
 )
 # size of the library-owned scratch array behind csa_topk_noalloc (bytes, per device)
 TOPK_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -81,6 +82,10 @@ _SIGS = {
     "csa_version": [],
     "csa_device_error": [ctypes.POINTER(ctypes.c_int32)],
     "csa_kernel_launches": [],
+    "csa_sparse_mqa_mixed_kv": [_PP, _I32, _I32, _VP, _VP, _VP, _VP, _I64, _VP, _VP, _I64, _VP,
+                                _VP, _VP, _VP, _VP, _SZ, _VP],
+    "hca_dense_mqa_mixed_kv": [_PP, _I32, _I32, _VP, _VP, _VP, _VP, _I64, _VP, _I64, _VP, _VP,
+                               _VP, _VP, _VP, _SZ, _VP],
     "csa_state_append": [_PP, ctypes.c_int, _I32] + [_VP] * 8 + [_I32, _VP, _VP, ctypes.c_int,
                                                              _VP, _VP, _I32, _I32, _VP, _I32, _VP],
 }
@@ -236,6 +241,25 @@ def hca_dense_mqa(p, io, B, T, q, q_pos, kv_cache, N_cap, win_kv, L_raw, win_pos
                             N_cap, _ptr(win_kv), L_raw, _ptr(win_pos0), _ptr(sink),
                             _ptr(q_rms_w), _ptr(out), _ptr(ws), ws_bytes, _stream(stream))
     _check("hca_dense_mqa", s)
+
+
+def csa_sparse_mqa_mixed_kv(p, B, T, q, q_pos, kv_rows, kv_scale, N_cap, idx, win_kv, L_raw,
+                            win_pos0, sink, q_rms_w, out, ws, ws_bytes, stream=None):
+    s = lib().csa_sparse_mqa_mixed_kv(ctypes.byref(p), B, T, _ptr(q), _ptr(q_pos),
+                                      _ptr(kv_rows), _ptr(kv_scale), N_cap, _ptr(idx),
+                                      _ptr(win_kv), L_raw, _ptr(win_pos0), _ptr(sink),
+                                      _ptr(q_rms_w), _ptr(out), _ptr(ws), ws_bytes,
+                                      _stream(stream))
+    _check("csa_sparse_mqa_mixed_kv", s)
+
+
+def hca_dense_mqa_mixed_kv(p, B, T, q, q_pos, kv_rows, kv_scale, N_cap, win_kv, L_raw,
+                           win_pos0, sink, q_rms_w, out, ws, ws_bytes, stream=None):
+    s = lib().hca_dense_mqa_mixed_kv(ctypes.byref(p), B, T, _ptr(q), _ptr(q_pos), _ptr(kv_rows),
+                                     _ptr(kv_scale), N_cap, _ptr(win_kv), L_raw, _ptr(win_pos0),
+                                     _ptr(sink), _ptr(q_rms_w), _ptr(out), _ptr(ws), ws_bytes,
+                                     _stream(stream))
+    _check("hca_dense_mqa_mixed_kv", s)
 
 
 def forward_args(**kw) -> CsaForwardArgs:

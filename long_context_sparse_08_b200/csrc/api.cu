@@ -501,6 +501,58 @@ csa_status hca_dense_mqa(const csa_params* p, csa_dtype io, int32_t B, int32_t T
   return ok();
 }
 
+namespace {
+csa_status mixed_kv_mqa(const char* what, const csa_params* p, int32_t B, int32_t T,
+                        const void* q, const int64_t* q_pos, const void* kv_rows,
+                        const float* kv_scale, int64_t N_cap, const int32_t* idx, int k,
+                        const void* win_kv, int64_t L_raw, const int64_t* win_pos0,
+                        const float* sink, const void* q_rms_w, void* out, void* ws,
+                        size_t ws_bytes, void* stream) {
+  TRY(check_mqa_args(p, CSA_BF16, B, T, q, q_pos, kv_rows, N_cap, win_kv, L_raw, win_pos0, sink,
+                     q_rms_w, out));
+  if ((int64_t)B * T == 0) return ok();
+  if (k > 0) REQUIRE_PTR(idx);
+  if (N_cap > 0) REQUIRE_PTR(kv_scale);
+  auto a = make_mqa(p, B, T, q, q_pos, kv_rows, N_cap, idx, k, win_kv, L_raw, win_pos0, sink,
+                    q_rms_w, out);
+  const bool rope_ok = p->rope_dims > 0 && p->rope_dims < p->c && p->rope_dims % 16 == 0;
+  if (!rope_ok || !csa::mqa_tc_supported(a, true))
+    return fail(CSA_ERR_UNSUPPORTED,
+                "%s: mixed-precision KV needs the tensor-core attention (c = 512, n_heads a "
+                "multiple of 64, rope_dims a multiple of 16 in (0, 512))", what);
+  a.kv_scale = N_cap > 0 ? kv_scale : nullptr;  // no cache rows: nothing to widen
+  const size_t need = csa::mqa_workspace_bytes(a);
+  if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws)))
+    return fail(CSA_ERR_WORKSPACE, "%s needs %zu workspace bytes", what, need);
+  TRY(cuda_status(csa::launch_mqa(a, true, ws, ws_bytes, (cudaStream_t)stream), what));
+  return ok();
+}
+}  // namespace
+
+csa_status csa_sparse_mqa_mixed_kv(const csa_params* p, int32_t B, int32_t T, const void* q,
+                                   const int64_t* q_pos, const void* kv_rows,
+                                   const float* kv_scale, int64_t N_cap, const int32_t* idx,
+                                   const void* win_kv, int64_t L_raw, const int64_t* win_pos0,
+                                   const float* sink, const void* q_rms_w, void* out, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  TRY(check_params(p));
+  TRY(check_topk(p));
+  return mixed_kv_mqa("sparse MQA (mixed KV)", p, B, T, q, q_pos, kv_rows, kv_scale, N_cap, idx,
+                      p->topk, win_kv, L_raw, win_pos0, sink, q_rms_w, out, ws, ws_bytes, stream);
+}
+
+csa_status hca_dense_mqa_mixed_kv(const csa_params* p, int32_t B, int32_t T, const void* q,
+                                  const int64_t* q_pos, const void* kv_rows,
+                                  const float* kv_scale, int64_t N_cap, const void* win_kv,
+                                  int64_t L_raw, const int64_t* win_pos0, const float* sink,
+                                  const void* q_rms_w, void* out, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  TRY(check_params(p));
+  return mixed_kv_mqa("dense MQA (mixed KV)", p, B, T, q, q_pos, kv_rows, kv_scale, N_cap,
+                      nullptr, 0, win_kv, L_raw, win_pos0, sink, q_rms_w, out, ws, ws_bytes,
+                      stream);
+}
+
 csa_status csa_forward(const csa_params* p, csa_dtype io, int32_t B, int32_t T,
                        const csa_forward_args* a, void* ws, size_t ws_bytes, void* stream) {
   REQUIRE(a != nullptr, "args is NULL");

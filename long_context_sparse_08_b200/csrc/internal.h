@@ -118,6 +118,8 @@ struct MqaArgs {
                  // queries before its own wait)
   const void* qhat;  // bf16 [B*T][H][c] prepared q_hat (written by an earlier kernel of the
                      // chain) or nullptr: the attention prepares it
+  const float* kv_scale;  // non-null: `kv` holds mixed-precision rows (c - r e4m3 codes, then
+                          // r bf16 values; c + r bytes) and this their per-row scales [B, n_cap]
 };
 size_t mqa_workspace_bytes(const MqaArgs& a);
 // tensor-core attention (bf16, c = 512, heads in groups of 64)

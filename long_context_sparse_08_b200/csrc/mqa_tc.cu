@@ -21,6 +21,13 @@
 // O^T and l are rescaled); exp(s - m) <= e^8 otherwise, exactly as correct.
 // One split: the CTA finalises (sink, RoPE(-t), bf16). Several: it writes (m, l, O)
 // partials and k_mqa_combine merges them in a fixed order (deterministic).
+//
+// Mixed-precision KV rows (一(三)4 item 1: RoPE dims in BF16, the rest in FP8; kMixed):
+// a cache row is c + r bytes, the e4m3 codes of its first c - r values (one fp32 scale per
+// row) then its last r values as bf16. The gather widens code * scale to bf16 into the
+// same swizzled tile (one rounding) and copies the bf16 values as they are, so the tensor
+// core work is unchanged and each selected row moves 580 bytes instead of 1024. Window rows
+// stay bf16.
 #include <cudaTypedefs.h>
 
 #include <cstring>
@@ -57,7 +64,8 @@ constexpr uint32_t kColO = 256;   // O^T slice s: 256 + 64 s
 
 enum { kErrKvFull = 201, kErrSFull = 202, kErrPFull = 203, kErrKvFree = 204 };
 
-struct Smem {
+template <bool kMixed>
+struct SmemT {
   uint64_t kv_full, s_full, p_full, kv_free, done;
   uint32_t tmem_slot;
   uint32_t vmask[4];  // valid rows of the current chunk (bit j of word w: row 32w + j)
@@ -65,6 +73,7 @@ struct Smem {
   float cs[kMaxPairs], sn[kMaxPairs];  // RoPE table for pairs of the last r dims
   float wq[kC];                         // query RMSNorm weights
   const __nv_bfloat16* src[kRows];  // source rows of the current chunk (nullptr: masked)
+  float rscale[kMixed ? kRows : 1];  // mixed rows: the row's FP8 scale; bf16 rows: -1
 };
 
 struct MqaTcParams {
@@ -153,6 +162,37 @@ __device__ __forceinline__ const __nv_bfloat16* row_src(const MqaArgs& a, int bt
   return nullptr;
 }
 
+// Source of list entry j with mixed-precision cache rows: a cache row (c + r bytes) with its
+// scale in *scale, or a bf16 window row with *scale = -1; nullptr when masked.
+__device__ __forceinline__ const void* row_src_mixed(const MqaArgs& a, int bt, int b,
+                                                     const RowList& rl, int64_t j, float* scale) {
+  *scale = -1.f;
+  if (j < rl.n_sel) {
+    int64_t e = j;
+    if (a.k > 0) e = a.idx[(size_t)bt * a.k + j];
+    else if (e >= rl.n_vis) return nullptr;
+    if (e < 0 || e >= a.n_cap) return nullptr;
+    const size_t row = (size_t)b * a.n_cap + e;
+    *scale = a.kv_scale[row];
+    return static_cast<const uint8_t*>(a.kv) + row * (size_t)(kC + a.rope_dims);
+  }
+  if (j < rl.L) {
+    const int64_t rr = rl.lo + (j - rl.n_sel) - a.win_pos0[b];
+    if (rr < 0 || rr >= a.l_raw) return nullptr;
+    return static_cast<const __nv_bfloat16*>(a.win) + ((size_t)b * a.l_raw + rr) * kC;
+  }
+  return nullptr;
+}
+
+// two e4m3 codes (low byte first) times `scale`, rounded to bf16x2
+__device__ __forceinline__ uint32_t e4m3x2_scaled_bf16x2(uint32_t v, float scale) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)v));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+  const __nv_bfloat162 r = __floats2bfloat162_rn(f.x * scale, f.y * scale);
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
 // 32 lanes x 16 columns of 32-bit: thread i of the warp gets lane (quadrant*32 + i).
 __device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
@@ -216,9 +256,11 @@ __device__ __forceinline__ int reduce16_index(int lane) {
   return ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
 }
 
+template <bool kMixed>
 __global__ void __launch_bounds__(kThreads, 1)
     k_mqa_tc(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_win,
              MqaTcParams P) {
+  using Smem = SmemT<kMixed>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -290,11 +332,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       cp_async_wait_all();
       bar_softmax();
       float ss0 = 0.f, ss1 = 0.f;
-  #pragma unroll 8
+#pragma unroll 8
       for (int i = 0; i < 32; ++i) {
         const uint4 raw = qrow[(i + lane) & 31];
         const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-  #pragma unroll
+#pragma unroll
         for (int k = 0; k < 4; ++k) {
           const float lo = __uint_as_float(w4[k] << 16), hi = __uint_as_float(w4[k] & 0xffff0000u);
           ss0 = fmaf(lo, lo, ss0);
@@ -304,20 +346,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       float ss = ss0 + ss1;
       ss += __shfl_xor_sync(0xffffffffu, ss, 1);
       const float rstd = rsqrtf(ss / (float)kC + a.eps);
-  #pragma unroll 4
+#pragma unroll 4
       for (int i = 0; i < 32; ++i) {
         const int c = (i + lane) & 31;
         const uint4 raw = qrow[c];
         const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
         const int d0 = 256 * qhalf + 8 * c;
         float y[8];
-  #pragma unroll
+#pragma unroll
         for (int k = 0; k < 4; ++k) {
           y[2 * k] = __uint_as_float(w4[k] << 16) * rstd * S.wq[d0 + 2 * k];
           y[2 * k + 1] = __uint_as_float(w4[k] & 0xffff0000u) * rstd * S.wq[d0 + 2 * k + 1];
         }
         if (d0 >= r0) {
-  #pragma unroll
+#pragma unroll
           for (int k = 0; k < 4; ++k) {
             const int p = (d0 + 2 * k - r0) >> 1;
             const float cs = S.cs[p], sn = S.sn[p], u = y[2 * k], v = y[2 * k + 1];
@@ -327,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         uint4 o;
         uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-  #pragma unroll
+#pragma unroll
         for (int k = 0; k < 4; ++k)
           ow[k] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * k])) |
                   ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * k + 1])) << 16);
@@ -352,7 +394,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       // ---- gather the chunk's 128 rows: thread r resolves row r, then warp w copies rows
       //      w, w+4, ... with lane = 16-byte chunk (coalesced 512 B per instruction) ----
-      const __nv_bfloat16* my_src = row_src(a, bt, b, rl, (int64_t)j * kRows + tid);
+      const __nv_bfloat16* my_src;
+      if constexpr (kMixed) {
+        float sc;
+        my_src = static_cast<const __nv_bfloat16*>(
+            row_src_mixed(a, bt, b, rl, (int64_t)j * kRows + tid, &sc));
+        S.rscale[tid] = sc;
+      } else {
+        my_src = row_src(a, bt, b, rl, (int64_t)j * kRows + tid);
+      }
       S.src[tid] = my_src;
       const uint32_t vb = __ballot_sync(0xffffffffu, my_src != nullptr);
       if (lane == 0) S.vmask[warp] = vb;
@@ -380,16 +430,67 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(base + kOffKV + atom * (kRows * 128), tmap, 64 * atom, trow, &S.kv_full);
         }
       } else {
-#pragma unroll 4
-        for (int rr = warp; rr < kRows; rr += 4) {
-          const __nv_bfloat16* src = S.src[rr];
+        if constexpr (kMixed) {
+          // a warp takes rows w, w+4, ...: a mixed row's lanes 0..27 widen 16 codes each
+          // (dims 16*lane ..: atom lane / 4, chunks 2*(lane % 4) and +1), lanes 28..31 copy
+          // two 16-byte chunks of its bf16 RoPE values (dims 448 + 8*q: atom 7, chunk q);
+          // a bf16 window row (scale -1) or a masked row is copied as in the bf16 path
+          const int r = a.rope_dims, nope = kC - r;  // nope = 448 (c = 512, r = 64)
+#pragma unroll 1
+          for (int rr = warp; rr < kRows; rr += 4) {
+            const __nv_bfloat16* src = S.src[rr];
+            const float sc = S.rscale[rr];
+            if (src == nullptr || sc < 0.f) {
 #pragma unroll
-          for (int hseg = 0; hseg < 2; ++hseg) {
-            const int gch = lane + 32 * hseg;  // 16-byte chunk of the 1 KB row
-            const int atom = gch >> 3, c = gch & 7;
-            const uint32_t dst = kv_base + atom * (kRows * 128) + sw128(rr, c);
-            cp_async16(dst, src ? src + 8 * gch : static_cast<const __nv_bfloat16*>(a.kv),
-                       src != nullptr);
+              for (int hseg = 0; hseg < 2; ++hseg) {
+                const int gch = lane + 32 * hseg;
+                const int atom = gch >> 3, c = gch & 7;
+                const uint32_t dst = kv_base + atom * (kRows * 128) + sw128(rr, c);
+                cp_async16(dst, src ? src + 8 * gch : static_cast<const __nv_bfloat16*>(a.kv),
+                           src != nullptr);
+              }
+            } else {
+              const uint8_t* row = reinterpret_cast<const uint8_t*>(src);
+              if (lane < nope / 16) {
+                const uint4 raw = __ldg(reinterpret_cast<const uint4*>(row) + lane);
+                const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+                uint32_t o8[8];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  o8[2 * q] = e4m3x2_scaled_bf16x2(w4[q] & 0xffffu, sc);
+                  o8[2 * q + 1] = e4m3x2_scaled_bf16x2(w4[q] >> 16, sc);
+                }
+                uint8_t* at = base + kOffKV + (lane >> 2) * (kRows * 128);
+                const int c8 = 2 * (lane & 3);
+                *reinterpret_cast<uint4*>(at + sw128(rr, c8)) = make_uint4(o8[0], o8[1], o8[2], o8[3]);
+                *reinterpret_cast<uint4*>(at + sw128(rr, c8 + 1)) =
+                    make_uint4(o8[4], o8[5], o8[6], o8[7]);
+              } else {
+                const int q0 = 2 * (lane - nope / 16);  // RoPE chunks q0, q0 + 1 of r / 8
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  const int q = q0 + h;
+                  if (q < r / 8) {
+                    const int d = nope + 8 * q;
+                    const uint32_t dst = kv_base + (d >> 6) * (kRows * 128) + sw128(rr, (d & 63) >> 3);
+                    cp_async16(dst, row + nope + 16 * q, true);
+                  }
+                }
+              }
+            }
+          }
+        } else {
+#pragma unroll 4
+          for (int rr = warp; rr < kRows; rr += 4) {
+            const __nv_bfloat16* src = S.src[rr];
+#pragma unroll
+            for (int hseg = 0; hseg < 2; ++hseg) {
+              const int gch = lane + 32 * hseg;  // 16-byte chunk of the 1 KB row
+              const int atom = gch >> 3, c = gch & 7;
+              const uint32_t dst = kv_base + atom * (kRows * 128) + sw128(rr, c);
+              cp_async16(dst, src ? src + 8 * gch : static_cast<const __nv_bfloat16*>(a.kv),
+                         src != nullptr);
+            }
           }
         }
         cp_async_wait_all();
@@ -719,8 +820,10 @@ int choose_nsplit(const MqaArgs& a) {
 }  // namespace
 
 bool mqa_tc_supported(const MqaArgs& a, bool bf16) {
+  const bool kv_ok = a.kv_scale == nullptr ||
+                     (a.rope_dims > 0 && a.rope_dims < kC && a.rope_dims % 16 == 0);
   return bf16 && a.c == kC && a.H % kHg == 0 && a.rope_dims <= kC && a.rope_dims % 2 == 0 &&
-         a.rope_dims / 2 <= 256;
+         a.rope_dims / 2 <= 256 && kv_ok;
 }
 
 size_t mqa_tc_workspace_bytes(const MqaArgs& a) {
@@ -741,15 +844,17 @@ cudaError_t launch_mqa_tc(const MqaArgs& a, void* ws, size_t ws_bytes, cudaStrea
   CUtensorMap tm_kv, tm_win;
   memset(&tm_kv, 0, sizeof(tm_kv));
   memset(&tm_win, 0, sizeof(tm_win));
-  P.tma_kv = make_map_rows(&tm_kv, a.kv, (int64_t)a.B * a.n_cap) ? 1 : 0;
+  const bool mixed = a.kv_scale != nullptr;  // mixed-precision cache rows: gathered, no TMA
+  P.tma_kv = !mixed && make_map_rows(&tm_kv, a.kv, (int64_t)a.B * a.n_cap) ? 1 : 0;
   P.tma_win = make_map_rows(&tm_win, a.win, (int64_t)a.B * a.l_raw) ? 1 : 0;
   if (P.nsplit > 1 && ws_bytes < mqa_tc_workspace_bytes(a)) return cudaErrorInvalidValue;
   const int64_t streams = (int64_t)a.B * a.T * P.G;
-  const size_t smem = 1024 + kOffEnd + sizeof(Smem);
-  cudaError_t e = cudaFuncSetAttribute(k_mqa_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kern = mixed ? k_mqa_tc<true> : k_mqa_tc<false>;
+  const size_t smem = 1024 + kOffEnd + (mixed ? sizeof(SmemT<true>) : sizeof(SmemT<false>));
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  e = launch(a.chained, k_mqa_tc, dim3((unsigned)(streams * P.nsplit)), dim3(kThreads), smem, st,
+  e = launch(a.chained, kern, dim3((unsigned)(streams * P.nsplit)), dim3(kThreads), smem, st,
              tm_kv, tm_win, P);
   if (e != cudaSuccess || P.nsplit == 1) return e;
   return launch(true, k_mqa_combine, dim3((unsigned)streams, kHg), dim3(256), 0, st, P);

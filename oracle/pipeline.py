@@ -45,16 +45,27 @@ def compressed_chunk(s, inp) -> np.ndarray:
 
 
 class _Cache:
-    """Row access to request b's compressed cache, decoding only the rows asked for."""
+    """Row access to request b's compressed cache, decoding only the rows asked for. A cache
+    given as mixed-precision rows (inputs kv_codes, kv_scale, kv_rope instead of kv_cache)
+    is decoded with dec_mixed_kv."""
 
     def __init__(self, s, inp, chunk: Optional[np.ndarray]):
-        self.s, self.raw, self.chunk = s, inp["kv_cache"], chunk
+        self.s, self.chunk = s, chunk
+        self.mixed = "kv_scale" in inp
+        if self.mixed:
+            self.codes, self.kscale, self.rope = inp["kv_codes"], inp["kv_scale"], inp["kv_rope"]
+        else:
+            self.raw = inp["kv_cache"]
         self.first = s.ctx // s.m if chunk is not None else None
 
     def rows(self, b: int, sel: np.ndarray) -> np.ndarray:
         sel = np.asarray(sel, np.int64)
-        out = O.dec_io(self.raw[b][sel], self.s.io) if sel.size else \
-            np.zeros((0, self.s.c))
+        if not sel.size:
+            out = np.zeros((0, self.s.c))
+        elif self.mixed:
+            out = O.dec_mixed_kv(self.codes[b][sel], self.kscale[b][sel], self.rope[b][sel])
+        else:
+            out = O.dec_io(self.raw[b][sel], self.s.io)
         if self.chunk is not None and sel.size:
             n_new = self.chunk.shape[1]
             inside = (sel >= self.first) & (sel < self.first + n_new)

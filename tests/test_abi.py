@@ -248,6 +248,34 @@ def test_state_append_checks():
     assert L.csa_state_append(*a) == csa.CSA_ERR_INVALID_ARG  # a ring needs n_win >= 1
 
 
+def test_mixed_kv_attention_checks():
+    L = csa.lib()
+    p = _p()
+    # p, B, T, q, q_pos, kv_rows, kv_scale, N_cap, idx, win_kv, L_raw, win_pos0, sink, q_rms_w,
+    # out, ws, ws_bytes, stream
+    base = [ctypes.byref(p), 1, 1, FAKE, FAKE, FAKE, FAKE, 1024, FAKE, FAKE, 128, FAKE, None,
+            None, FAKE, None, 0, None]
+
+    def call(i=None, v=None, params=None):
+        a = list(base)
+        if i is not None:
+            a[i] = v
+        if params is not None:
+            a[0] = ctypes.byref(params)
+        return L.csa_sparse_mqa_mixed_kv(*a)
+
+    assert call(6, None) == csa.CSA_ERR_INVALID_ARG   # cache rows without their scales
+    assert call(8, None) == csa.CSA_ERR_INVALID_ARG   # no index list
+    assert call(1, 0) == csa.CSA_OK                   # nothing to do
+    assert call(params=_p(rope_dims=8)) == csa.CSA_ERR_UNSUPPORTED   # r not a multiple of 16
+    assert call(params=_p(rope_dims=0)) == csa.CSA_ERR_UNSUPPORTED   # no bf16 part
+    assert call(params=_p(n_heads=16)) == csa.CSA_ERR_UNSUPPORTED    # heads in groups of 64
+    assert call(params=_p(c=256)) == csa.CSA_ERR_UNSUPPORTED
+    h = [ctypes.byref(_p(m=128, overlap=0)), 1, 1, FAKE, FAKE, FAKE, None, 64, FAKE, 128, FAKE,
+         None, None, FAKE, None, 0, None]
+    assert L.hca_dense_mqa_mixed_kv(*h) == csa.CSA_ERR_INVALID_ARG  # no scales
+
+
 def test_binding_refuses_host_tensors():
     import torch
 
