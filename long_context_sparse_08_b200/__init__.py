@@ -24,7 +24,7 @@ EXPORTS = (
     "hca_dense_mqa", "csa_forward", "csa_workspace_size", "csa_status_string",
     "csa_last_error", "csa_set_index_timing_events", "csa_version", "csa_device_error",
     "csa_topk_noalloc", "csa_kernel_launches", "csa_state_append", "csa_sparse_mqa_mixed_kv",
-    "hca_dense_mqa_mixed_kv",
+    "hca_dense_mqa_mixed_kv", "csa_grouped_out_proj", "csa_grouped_out_proj_workspace_size",
 )
 # size of the library-owned scratch array behind csa_topk_noalloc (bytes, per device)
 TOPK_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -82,6 +82,8 @@ _SIGS = {
     "csa_version": [],
     "csa_device_error": [ctypes.POINTER(ctypes.c_int32)],
     "csa_kernel_launches": [],
+    "csa_grouped_out_proj": [_PP, _I32, _I32, _I32, _I32, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
+    "csa_grouped_out_proj_workspace_size": [_PP, _I32, _I32, _I32, _I32],
     "csa_sparse_mqa_mixed_kv": [_PP, _I32, _I32, _VP, _VP, _VP, _VP, _I64, _VP, _VP, _I64, _VP,
                                 _VP, _VP, _VP, _VP, _SZ, _VP],
     "hca_dense_mqa_mixed_kv": [_PP, _I32, _I32, _VP, _VP, _VP, _VP, _I64, _VP, _I64, _VP, _VP,
@@ -89,7 +91,7 @@ _SIGS = {
     "csa_state_append": [_PP, ctypes.c_int, _I32] + [_VP] * 8 + [_I32, _VP, _VP, ctypes.c_int,
                                                              _VP, _VP, _I32, _I32, _VP, _I32, _VP],
 }
-_RES = {"csa_workspace_size": _SZ, "csa_kernel_launches": ctypes.c_uint64, "csa_status_string": ctypes.c_char_p,
+_RES = {"csa_workspace_size": _SZ, "csa_grouped_out_proj_workspace_size": _SZ, "csa_kernel_launches": ctypes.c_uint64, "csa_status_string": ctypes.c_char_p,
         "csa_last_error": ctypes.c_char_p, "csa_version": ctypes.c_char_p,
         "csa_set_index_timing_events": None}
 
@@ -260,6 +262,16 @@ def hca_dense_mqa_mixed_kv(p, B, T, q, q_pos, kv_rows, kv_scale, N_cap, win_kv, 
                                      _ptr(sink), _ptr(q_rms_w), _ptr(out), _ptr(ws), ws_bytes,
                                      _stream(stream))
     _check("hca_dense_mqa_mixed_kv", s)
+
+
+def grouped_out_proj_workspace_size(p, Q, g, d_g, d) -> int:
+    return int(lib().csa_grouped_out_proj_workspace_size(ctypes.byref(p), Q, g, d_g, d))
+
+
+def csa_grouped_out_proj(p, Q, g, d_g, d, o, w_grp, w_out, out, ws, ws_bytes, stream=None):
+    s = lib().csa_grouped_out_proj(ctypes.byref(p), Q, g, d_g, d, _ptr(o), _ptr(w_grp),
+                                   _ptr(w_out), _ptr(out), _ptr(ws), ws_bytes, _stream(stream))
+    _check("csa_grouped_out_proj", s)
 
 
 def forward_args(**kw) -> CsaForwardArgs:

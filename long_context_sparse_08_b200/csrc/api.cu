@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "out_proj.cuh"
 #include "state_append.cuh"
 
 namespace csa {
@@ -401,6 +402,51 @@ csa_status csa_state_append(const csa_params* p, csa_dtype io, int32_t B, const 
     a.inv_freq[i] = csa::rope_inv_freq(i, p->rope_dims, (double)p->rope_base);
   TRY(cuda_status(csa::launch_state_append(a, io == CSA_BF16, (cudaStream_t)stream),
                   "state append"));
+  return ok();
+}
+
+namespace {
+csa_status check_out_proj(const csa_params* p, int32_t Q, int32_t g, int32_t d_g, int32_t d) {
+  TRY(check_params(p));
+  REQUIRE(Q >= 0, "Q must be >= 0");
+  REQUIRE(p->n_heads >= 1 && g >= 1 && p->n_heads % g == 0,
+          "n_heads (%d) must be a positive multiple of g (%d)", p->n_heads, g);
+  REQUIRE(d_g >= 8 && d_g % 8 == 0 && d >= 8 && d % 8 == 0,
+          "d_g and d must be positive multiples of 8 (got %d, %d)", d_g, d);
+  REQUIRE((int64_t)p->c * p->n_heads <= (1 << 24) && (int64_t)g * d_g <= (1 << 24) &&
+              d <= (1 << 24), "sizes too large");
+  if (Q > 16)
+    return fail(CSA_ERR_UNSUPPORTED,
+                "grouped output projection: decode batches of at most 16 queries (got %d)", Q);
+  return CSA_OK;
+}
+}  // namespace
+
+size_t csa_grouped_out_proj_workspace_size(const csa_params* p, int32_t Q, int32_t g,
+                                           int32_t d_g, int32_t d) {
+  if (check_out_proj(p, Q, g, d_g, d) != CSA_OK || Q == 0) return 0;
+  return csa::out_proj_workspace_bytes(csa::out_proj_geom(Q, p->n_heads, p->c, g, d_g, d));
+}
+
+csa_status csa_grouped_out_proj(const csa_params* p, int32_t Q, int32_t g, int32_t d_g,
+                                int32_t d, const void* o, const void* w_grp, const void* w_out,
+                                void* out, void* ws, size_t ws_bytes, void* stream) {
+  TRY(check_out_proj(p, Q, g, d_g, d));
+  if (Q == 0) return ok();
+  REQUIRE_PTR(o);
+  REQUIRE_PTR(w_grp);
+  REQUIRE_PTR(w_out);
+  REQUIRE_PTR(out);
+  csa::OutProjArgs a{};
+  a.G = csa::out_proj_geom(Q, p->n_heads, p->c, g, d_g, d);
+  const size_t need = csa::out_proj_workspace_bytes(a.G);
+  if (ws == nullptr || ws_bytes < need || !aligned16(ws))
+    return fail(CSA_ERR_WORKSPACE, "grouped output projection needs %zu workspace bytes", need);
+  a.o = static_cast<const __nv_bfloat16*>(o);
+  a.w_grp = static_cast<const __nv_bfloat16*>(w_grp);
+  a.w_out = static_cast<const __nv_bfloat16*>(w_out);
+  a.out = static_cast<__nv_bfloat16*>(out);
+  TRY(cuda_status(csa::launch_out_proj(a, ws, (cudaStream_t)stream), "grouped output projection"));
   return ok();
 }
 

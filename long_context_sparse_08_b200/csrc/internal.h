@@ -37,6 +37,13 @@ struct CompressArgs {
 };
 cudaError_t launch_compress(const CompressArgs& a, bool bf16, cudaStream_t st);
 
+namespace proj { struct Geom; }
+struct OutProjArgs;
+// grouped output projection (decode: Q <= 16 queries)
+proj::Geom out_proj_geom(int Q, int H, int c, int g, int d_g, int d);
+size_t out_proj_workspace_bytes(const proj::Geom& G);
+cudaError_t launch_out_proj(OutProjArgs a, void* ws, cudaStream_t st);
+
 namespace state { struct Args; }
 // decode-time append of one token per request into the state cache and its pages
 cudaError_t launch_state_append(const state::Args& a, bool bf16, cudaStream_t st);

@@ -412,3 +412,20 @@ def make_state_stream(*, B: int, n_tok: int, m: int, c: int, overlap: int, io: s
     out["win"] = _encode_io(_normal(g, (B, n_tok, c)), io)
     out["bias"] = _encode_io(_normal(g, ((2 if overlap else 1) * m, c)), io)
     return out
+
+
+def make_out_proj_inputs(*, Q: int, H: int, c: int, g: int, d_g: int, d: int,
+                         seed: int) -> Dict[str, np.ndarray]:
+    """Seeded inputs of the grouped output projection, as bf16 bit patterns: the attention
+    outputs o [Q, H*c] ~ N(0,1), then the group matrices w_grp [g, c*H/g, d_g] and the
+    output matrix w_out [g*d_g, d], each ~N(0, 1/rows) (random initialisation that keeps
+    the sums O(1)). Shapes of 【论文解读】DeepSeek-V4 三、预训练 (二): g = 8 / 16,
+    d_g = 1024, d = 4096 / 7168."""
+    g_ = np.random.default_rng(seed)
+    k1 = c * (H // g)
+    o = _normal(g_, (Q, H * c))
+    w_grp = _normal(g_, (g, k1, d_g), std=1.0 / math.sqrt(k1))
+    w_out = _normal(g_, (g * d_g, d), std=1.0 / math.sqrt(g * d_g))
+    return {"o": f32_to_bf16_bits(o), "w_grp": f32_to_bf16_bits(w_grp),
+            "w_out": f32_to_bf16_bits(w_out)}
+
