@@ -268,6 +268,41 @@ csa_status hca_dense_mqa_mixed_kv(const csa_params* p, int32_t B, int32_t T, con
                                   const void* q_rms_w, void* out, void* ws, size_t ws_bytes,
                                   void* stream);
 
+/*
+ * A paged classical KV cache ([P1''] 二、基础设施 (六): finished entries in blocks of a
+ * multiple of lcm(m, m') raw tokens), as csa_state_append writes it: a pool of n_pages pages
+ * of page_rows rows each; entry e of request b is row e % page_rows of page
+ * page_table[b * max_pages + e / page_rows]. The logical capacity is
+ * N_cap = page_rows * max_pages. Passed by pointer, read on the host during the call.
+ */
+typedef struct {
+  csa_dtype fmt;              /* CSA_BF16 (pages [n_pages, page_rows, c]) or CSA_MIXED_FP8_BF16
+                                 (pages [n_pages, page_rows, c + r] bytes)                  */
+  const void* pages;          /* device                                                     */
+  const float* scales;        /* CSA_MIXED_FP8_BF16: [n_pages, page_rows] fp32; else NULL   */
+  const int32_t* page_table;  /* device int32 [B, max_pages]                               */
+  int32_t n_pages, page_rows, max_pages;
+} csa_paged_kv;
+
+/*
+ * Stage 4 over a paged cache: as csa_sparse_mqa / hca_dense_mqa with io = CSA_BF16 (the
+ * mixed format as in csa_sparse_mqa_mixed_kv), reading each cache row through the page
+ * table. An entry whose page id lies outside [0, n_pages) is skipped and leaves device
+ * error code 205 for csa_device_error(). Tensor-core attention only (c = 512, n_heads a
+ * multiple of 64; mixed rows: rope_dims a multiple of 16 in (0, 512)), else
+ * CSA_ERR_UNSUPPORTED. Workspace: csa_workspace_size() with N_cap = page_rows * max_pages.
+ */
+csa_status csa_sparse_mqa_paged(const csa_params* p, int32_t B, int32_t T, const void* q,
+                                const int64_t* q_pos, const csa_paged_kv* kv, const int32_t* idx,
+                                const void* win_kv, int64_t L_raw, const int64_t* win_pos0,
+                                const float* sink, const void* q_rms_w, void* out, void* ws,
+                                size_t ws_bytes, void* stream);
+csa_status hca_dense_mqa_paged(const csa_params* p, int32_t B, int32_t T, const void* q,
+                               const int64_t* q_pos, const csa_paged_kv* kv, const void* win_kv,
+                               int64_t L_raw, const int64_t* win_pos0, const float* sink,
+                               const void* q_rms_w, void* out, void* ws, size_t ws_bytes,
+                               void* stream);
+
 /* Inputs of the fused CSA layer call. Pointers as in the stage calls above. */
 typedef struct {
   /* optional compression of a new chunk into kv_cache (skipped when Ca == NULL) */

@@ -25,6 +25,7 @@ EXPORTS = (
     "csa_last_error", "csa_set_index_timing_events", "csa_version", "csa_device_error",
     "csa_topk_noalloc", "csa_kernel_launches", "csa_state_append", "csa_sparse_mqa_mixed_kv",
     "hca_dense_mqa_mixed_kv", "csa_grouped_out_proj", "csa_grouped_out_proj_workspace_size",
+    "csa_sparse_mqa_paged", "hca_dense_mqa_paged",
 )
 # size of the library-owned scratch array behind csa_topk_noalloc (bytes, per device)
 TOPK_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -60,6 +61,16 @@ class CsaForwardArgs(ctypes.Structure):
     ]
 
 
+class CsaPagedKv(ctypes.Structure):
+    """Mirror of ``csa_paged_kv``."""
+
+    _fields_ = [
+        ("fmt", ctypes.c_int), ("pages", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+        ("page_table", ctypes.c_void_p), ("n_pages", ctypes.c_int32),
+        ("page_rows", ctypes.c_int32), ("max_pages", ctypes.c_int32),
+    ]
+
+
 _LIB = None
 _VP, _I32, _I64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
 _PP = ctypes.POINTER(CsaParams)
@@ -82,6 +93,10 @@ _SIGS = {
     "csa_version": [],
     "csa_device_error": [ctypes.POINTER(ctypes.c_int32)],
     "csa_kernel_launches": [],
+    "csa_sparse_mqa_paged": [_PP, _I32, _I32, _VP, _VP, ctypes.POINTER(CsaPagedKv), _VP, _VP,
+                             _I64, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
+    "hca_dense_mqa_paged": [_PP, _I32, _I32, _VP, _VP, ctypes.POINTER(CsaPagedKv), _VP, _I64,
+                            _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "csa_grouped_out_proj": [_PP, _I32, _I32, _I32, _I32, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "csa_grouped_out_proj_workspace_size": [_PP, _I32, _I32, _I32, _I32],
     "csa_sparse_mqa_mixed_kv": [_PP, _I32, _I32, _VP, _VP, _VP, _VP, _I64, _VP, _VP, _I64, _VP,
@@ -262,6 +277,29 @@ def hca_dense_mqa_mixed_kv(p, B, T, q, q_pos, kv_rows, kv_scale, N_cap, win_kv, 
                                      _ptr(sink), _ptr(q_rms_w), _ptr(out), _ptr(ws), ws_bytes,
                                      _stream(stream))
     _check("hca_dense_mqa_mixed_kv", s)
+
+
+def paged_kv(fmt, pages, scales, page_table, n_pages, page_rows, max_pages) -> CsaPagedKv:
+    """A csa_paged_kv over device tensors."""
+    return CsaPagedKv(int(fmt), _ptr(pages), _ptr(scales), _ptr(page_table), n_pages,
+                      page_rows, max_pages)
+
+
+def csa_sparse_mqa_paged(p, B, T, q, q_pos, kv: CsaPagedKv, idx, win_kv, L_raw, win_pos0, sink,
+                         q_rms_w, out, ws, ws_bytes, stream=None):
+    s = lib().csa_sparse_mqa_paged(ctypes.byref(p), B, T, _ptr(q), _ptr(q_pos), ctypes.byref(kv),
+                                   _ptr(idx), _ptr(win_kv), L_raw, _ptr(win_pos0), _ptr(sink),
+                                   _ptr(q_rms_w), _ptr(out), _ptr(ws), ws_bytes,
+                                   _stream(stream))
+    _check("csa_sparse_mqa_paged", s)
+
+
+def hca_dense_mqa_paged(p, B, T, q, q_pos, kv: CsaPagedKv, win_kv, L_raw, win_pos0, sink,
+                        q_rms_w, out, ws, ws_bytes, stream=None):
+    s = lib().hca_dense_mqa_paged(ctypes.byref(p), B, T, _ptr(q), _ptr(q_pos), ctypes.byref(kv),
+                                  _ptr(win_kv), L_raw, _ptr(win_pos0), _ptr(sink),
+                                  _ptr(q_rms_w), _ptr(out), _ptr(ws), ws_bytes, _stream(stream))
+    _check("hca_dense_mqa_paged", s)
 
 
 def grouped_out_proj_workspace_size(p, Q, g, d_g, d) -> int:

@@ -548,30 +548,62 @@ csa_status hca_dense_mqa(const csa_params* p, csa_dtype io, int32_t B, int32_t T
 }
 
 namespace {
-csa_status mixed_kv_mqa(const char* what, const csa_params* p, int32_t B, int32_t T,
-                        const void* q, const int64_t* q_pos, const void* kv_rows,
-                        const float* kv_scale, int64_t N_cap, const int32_t* idx, int k,
-                        const void* win_kv, int64_t L_raw, const int64_t* win_pos0,
-                        const float* sink, const void* q_rms_w, void* out, void* ws,
-                        size_t ws_bytes, void* stream) {
-  TRY(check_mqa_args(p, CSA_BF16, B, T, q, q_pos, kv_rows, N_cap, win_kv, L_raw, win_pos0, sink,
+// Tensor-core attention over mixed-precision and / or paged cache rows.
+struct KvLayout {
+  bool mixed;
+  const void* rows;            // contiguous cache [B, N_cap, ...] or page pool
+  const float* scales;         // mixed: per-row scales (same indexing as rows)
+  const int32_t* page_table;   // paged: [B, max_pages]; NULL: contiguous
+  int32_t n_pages, page_rows, max_pages;
+};
+
+csa_status tc_mqa_ext(const char* what, const csa_params* p, int32_t B, int32_t T,
+                      const void* q, const int64_t* q_pos, const KvLayout& kv, int64_t N_cap,
+                      const int32_t* idx, int k, const void* win_kv, int64_t L_raw,
+                      const int64_t* win_pos0, const float* sink, const void* q_rms_w,
+                      void* out, void* ws, size_t ws_bytes, void* stream) {
+  TRY(check_mqa_args(p, CSA_BF16, B, T, q, q_pos, kv.rows, N_cap, win_kv, L_raw, win_pos0, sink,
                      q_rms_w, out));
   if ((int64_t)B * T == 0) return ok();
   if (k > 0) REQUIRE_PTR(idx);
-  if (N_cap > 0) REQUIRE_PTR(kv_scale);
-  auto a = make_mqa(p, B, T, q, q_pos, kv_rows, N_cap, idx, k, win_kv, L_raw, win_pos0, sink,
+  if (kv.mixed && N_cap > 0) REQUIRE_PTR(kv.scales);
+  if (kv.page_table != nullptr) REQUIRE_PTR(kv.page_table);
+  auto a = make_mqa(p, B, T, q, q_pos, kv.rows, N_cap, idx, k, win_kv, L_raw, win_pos0, sink,
                     q_rms_w, out);
-  const bool rope_ok = p->rope_dims > 0 && p->rope_dims < p->c && p->rope_dims % 16 == 0;
+  const bool rope_ok = !kv.mixed ||
+                       (p->rope_dims > 0 && p->rope_dims < p->c && p->rope_dims % 16 == 0);
   if (!rope_ok || !csa::mqa_tc_supported(a, true))
     return fail(CSA_ERR_UNSUPPORTED,
-                "%s: mixed-precision KV needs the tensor-core attention (c = 512, n_heads a "
-                "multiple of 64, rope_dims a multiple of 16 in (0, 512))", what);
-  a.kv_scale = N_cap > 0 ? kv_scale : nullptr;  // no cache rows: nothing to widen
+                "%s: needs the tensor-core attention (c = 512, n_heads a multiple of 64; "
+                "mixed rows: rope_dims a multiple of 16 in (0, 512))", what);
+  if (N_cap > 0) {  // no cache rows: nothing to widen or look up
+    a.kv_scale = kv.mixed ? kv.scales : nullptr;
+    a.page_table = kv.page_table;
+    a.n_pages = kv.n_pages;
+    a.page_rows = kv.page_rows;
+    a.max_pages = kv.max_pages;
+  }
   const size_t need = csa::mqa_workspace_bytes(a);
   if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws)))
     return fail(CSA_ERR_WORKSPACE, "%s needs %zu workspace bytes", what, need);
   TRY(cuda_status(csa::launch_mqa(a, true, ws, ws_bytes, (cudaStream_t)stream), what));
   return ok();
+}
+
+csa_status paged_layout(const csa_paged_kv* kv, KvLayout* out, int64_t* N_cap) {
+  REQUIRE(kv != nullptr, "paged KV descriptor is NULL");
+  REQUIRE(kv->fmt == CSA_BF16 || kv->fmt == CSA_MIXED_FP8_BF16,
+          "paged KV format must be CSA_BF16 or CSA_MIXED_FP8_BF16");
+  REQUIRE(kv->n_pages >= 1 && kv->page_rows >= 1 && kv->max_pages >= 1,
+          "n_pages, page_rows and max_pages must be >= 1");
+  REQUIRE((int64_t)kv->page_rows * kv->max_pages <= INT32_MAX, "page_rows * max_pages too large");
+  REQUIRE_PTR(kv->pages);
+  REQUIRE_PTR(kv->page_table);
+  if (kv->fmt == CSA_MIXED_FP8_BF16) REQUIRE_PTR(kv->scales);
+  *out = KvLayout{kv->fmt == CSA_MIXED_FP8_BF16, kv->pages, kv->scales, kv->page_table,
+                  kv->n_pages, kv->page_rows, kv->max_pages};
+  *N_cap = (int64_t)kv->page_rows * kv->max_pages;
+  return CSA_OK;
 }
 }  // namespace
 
@@ -583,8 +615,9 @@ csa_status csa_sparse_mqa_mixed_kv(const csa_params* p, int32_t B, int32_t T, co
                                    size_t ws_bytes, void* stream) {
   TRY(check_params(p));
   TRY(check_topk(p));
-  return mixed_kv_mqa("sparse MQA (mixed KV)", p, B, T, q, q_pos, kv_rows, kv_scale, N_cap, idx,
-                      p->topk, win_kv, L_raw, win_pos0, sink, q_rms_w, out, ws, ws_bytes, stream);
+  const KvLayout kv{true, kv_rows, kv_scale, nullptr, 0, 0, 0};
+  return tc_mqa_ext("sparse MQA (mixed KV)", p, B, T, q, q_pos, kv, N_cap, idx, p->topk, win_kv,
+                    L_raw, win_pos0, sink, q_rms_w, out, ws, ws_bytes, stream);
 }
 
 csa_status hca_dense_mqa_mixed_kv(const csa_params* p, int32_t B, int32_t T, const void* q,
@@ -594,9 +627,36 @@ csa_status hca_dense_mqa_mixed_kv(const csa_params* p, int32_t B, int32_t T, con
                                   const void* q_rms_w, void* out, void* ws, size_t ws_bytes,
                                   void* stream) {
   TRY(check_params(p));
-  return mixed_kv_mqa("dense MQA (mixed KV)", p, B, T, q, q_pos, kv_rows, kv_scale, N_cap,
-                      nullptr, 0, win_kv, L_raw, win_pos0, sink, q_rms_w, out, ws, ws_bytes,
-                      stream);
+  const KvLayout kv{true, kv_rows, kv_scale, nullptr, 0, 0, 0};
+  return tc_mqa_ext("dense MQA (mixed KV)", p, B, T, q, q_pos, kv, N_cap, nullptr, 0, win_kv,
+                    L_raw, win_pos0, sink, q_rms_w, out, ws, ws_bytes, stream);
+}
+
+csa_status csa_sparse_mqa_paged(const csa_params* p, int32_t B, int32_t T, const void* q,
+                                const int64_t* q_pos, const csa_paged_kv* kv, const int32_t* idx,
+                                const void* win_kv, int64_t L_raw, const int64_t* win_pos0,
+                                const float* sink, const void* q_rms_w, void* out, void* ws,
+                                size_t ws_bytes, void* stream) {
+  TRY(check_params(p));
+  TRY(check_topk(p));
+  KvLayout lay;
+  int64_t N_cap = 0;
+  TRY(paged_layout(kv, &lay, &N_cap));
+  return tc_mqa_ext("sparse MQA (paged KV)", p, B, T, q, q_pos, lay, N_cap, idx, p->topk, win_kv,
+                    L_raw, win_pos0, sink, q_rms_w, out, ws, ws_bytes, stream);
+}
+
+csa_status hca_dense_mqa_paged(const csa_params* p, int32_t B, int32_t T, const void* q,
+                               const int64_t* q_pos, const csa_paged_kv* kv, const void* win_kv,
+                               int64_t L_raw, const int64_t* win_pos0, const float* sink,
+                               const void* q_rms_w, void* out, void* ws, size_t ws_bytes,
+                               void* stream) {
+  TRY(check_params(p));
+  KvLayout lay;
+  int64_t N_cap = 0;
+  TRY(paged_layout(kv, &lay, &N_cap));
+  return tc_mqa_ext("dense MQA (paged KV)", p, B, T, q, q_pos, lay, N_cap, nullptr, 0, win_kv,
+                    L_raw, win_pos0, sink, q_rms_w, out, ws, ws_bytes, stream);
 }
 
 csa_status csa_forward(const csa_params* p, csa_dtype io, int32_t B, int32_t T,

@@ -126,7 +126,12 @@ struct MqaArgs {
   const void* qhat;  // bf16 [B*T][H][c] prepared q_hat (written by an earlier kernel of the
                      // chain) or nullptr: the attention prepares it
   const float* kv_scale;  // non-null: `kv` holds mixed-precision rows (c - r e4m3 codes, then
-                          // r bf16 values; c + r bytes) and this their per-row scales [B, n_cap]
+                          // r bf16 values; c + r bytes) and this their per-row scales
+  const int32_t* page_table;  // non-null: `kv` (and kv_scale) are a pool of n_pages pages of
+                              // page_rows rows; entry e of request b is row e % page_rows of
+                              // page page_table[b * max_pages + e / page_rows];
+                              // n_cap = page_rows * max_pages
+  int page_rows, max_pages, n_pages;
 };
 size_t mqa_workspace_bytes(const MqaArgs& a);
 // tensor-core attention (bf16, c = 512, heads in groups of 64)

@@ -28,6 +28,10 @@
 // same swizzled tile (one rounding) and copies the bf16 values as they are, so the tensor
 // core work is unchanged and each selected row moves 580 bytes instead of 1024. Window rows
 // stay bf16.
+//
+// Paged cache (kPaged; 二、基础设施 (六) 推理框架): the classical cache is a pool of pages and
+// a request's entry e is row e % page_rows of page page_table[b, e / page_rows]; only the
+// gather's address changes. A page id outside the pool masks the row and records an error.
 #include <cudaTypedefs.h>
 
 #include <cstring>
@@ -62,7 +66,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;     // S: 128 columns (M = 64 layout)
 constexpr uint32_t kColO = 256;   // O^T slice s: 256 + 64 s
 
-enum { kErrKvFull = 201, kErrSFull = 202, kErrPFull = 203, kErrKvFree = 204 };
+enum { kErrKvFull = 201, kErrSFull = 202, kErrPFull = 203, kErrKvFree = 204, kErrPageId = 205 };
 
 template <bool kMixed>
 struct SmemT {
@@ -162,19 +166,33 @@ __device__ __forceinline__ const __nv_bfloat16* row_src(const MqaArgs& a, int bt
   return nullptr;
 }
 
-// Source of list entry j with mixed-precision cache rows: a cache row (c + r bytes) with its
-// scale in *scale, or a bf16 window row with *scale = -1; nullptr when masked.
-__device__ __forceinline__ const void* row_src_mixed(const MqaArgs& a, int bt, int b,
-                                                     const RowList& rl, int64_t j, float* scale) {
+// Source of list entry j for the mixed-precision and / or paged variants: a cache row (bf16,
+// or c + r mixed bytes with its scale in *scale) found through the page table when kPaged,
+// or a bf16 window row (*scale = -1); nullptr when masked.
+template <bool kMixed, bool kPaged>
+__device__ __forceinline__ const void* row_src_ext(const MqaArgs& a, int bt, int b,
+                                                   const RowList& rl, int64_t j, float* scale) {
   *scale = -1.f;
   if (j < rl.n_sel) {
     int64_t e = j;
     if (a.k > 0) e = a.idx[(size_t)bt * a.k + j];
     else if (e >= rl.n_vis) return nullptr;
     if (e < 0 || e >= a.n_cap) return nullptr;
-    const size_t row = (size_t)b * a.n_cap + e;
-    *scale = a.kv_scale[row];
-    return static_cast<const uint8_t*>(a.kv) + row * (size_t)(kC + a.rope_dims);
+    size_t row = (size_t)b * a.n_cap + e;
+    if constexpr (kPaged) {
+      const int32_t pg = a.page_table[(size_t)b * a.max_pages + e / a.page_rows];
+      if (pg < 0 || pg >= a.n_pages) {
+        set_error(kErrPageId);
+        return nullptr;
+      }
+      row = (size_t)pg * a.page_rows + (size_t)(e % a.page_rows);
+    }
+    if constexpr (kMixed) {
+      *scale = a.kv_scale[row];
+      return static_cast<const uint8_t*>(a.kv) + row * (size_t)(kC + a.rope_dims);
+    } else {
+      return static_cast<const __nv_bfloat16*>(a.kv) + row * kC;
+    }
   }
   if (j < rl.L) {
     const int64_t rr = rl.lo + (j - rl.n_sel) - a.win_pos0[b];
@@ -256,7 +274,7 @@ __device__ __forceinline__ int reduce16_index(int lane) {
   return ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
 }
 
-template <bool kMixed>
+template <bool kMixed, bool kPaged>
 __global__ void __launch_bounds__(kThreads, 1)
     k_mqa_tc(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_win,
              MqaTcParams P) {
@@ -395,11 +413,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- gather the chunk's 128 rows: thread r resolves row r, then warp w copies rows
       //      w, w+4, ... with lane = 16-byte chunk (coalesced 512 B per instruction) ----
       const __nv_bfloat16* my_src;
-      if constexpr (kMixed) {
+      if constexpr (kMixed || kPaged) {
         float sc;
         my_src = static_cast<const __nv_bfloat16*>(
-            row_src_mixed(a, bt, b, rl, (int64_t)j * kRows + tid, &sc));
-        S.rscale[tid] = sc;
+            row_src_ext<kMixed, kPaged>(a, bt, b, rl, (int64_t)j * kRows + tid, &sc));
+        if constexpr (kMixed) S.rscale[tid] = sc;
       } else {
         my_src = row_src(a, bt, b, rl, (int64_t)j * kRows + tid);
       }
@@ -844,12 +862,15 @@ cudaError_t launch_mqa_tc(const MqaArgs& a, void* ws, size_t ws_bytes, cudaStrea
   CUtensorMap tm_kv, tm_win;
   memset(&tm_kv, 0, sizeof(tm_kv));
   memset(&tm_win, 0, sizeof(tm_win));
-  const bool mixed = a.kv_scale != nullptr;  // mixed-precision cache rows: gathered, no TMA
-  P.tma_kv = !mixed && make_map_rows(&tm_kv, a.kv, (int64_t)a.B * a.n_cap) ? 1 : 0;
+  const bool mixed = a.kv_scale != nullptr;    // mixed-precision cache rows
+  const bool paged = a.page_table != nullptr;  // cache rows through the page table
+  // cache rows come by TMA only when they are contiguous bf16 rows
+  P.tma_kv = !mixed && !paged && make_map_rows(&tm_kv, a.kv, (int64_t)a.B * a.n_cap) ? 1 : 0;
   P.tma_win = make_map_rows(&tm_win, a.win, (int64_t)a.B * a.l_raw) ? 1 : 0;
   if (P.nsplit > 1 && ws_bytes < mqa_tc_workspace_bytes(a)) return cudaErrorInvalidValue;
   const int64_t streams = (int64_t)a.B * a.T * P.G;
-  auto kern = mixed ? k_mqa_tc<true> : k_mqa_tc<false>;
+  auto kern = mixed ? (paged ? k_mqa_tc<true, true> : k_mqa_tc<true, false>)
+                    : (paged ? k_mqa_tc<false, true> : k_mqa_tc<false, false>);
   const size_t smem = 1024 + kOffEnd + (mixed ? sizeof(SmemT<true>) : sizeof(SmemT<false>));
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);

@@ -68,9 +68,10 @@ def test_struct_layout_matches_the_c_compiler():
 #include <stddef.h>
 #include "csa.h"
 int main(void) {
-  printf("%zu %zu %zu %zu %zu %zu\n", sizeof(csa_params), sizeof(csa_forward_args),
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(csa_params), sizeof(csa_forward_args),
          offsetof(csa_forward_args, idx_dtype), offsetof(csa_forward_args, N_cap),
-         offsetof(csa_forward_args, out), offsetof(csa_params, n_win));
+         offsetof(csa_forward_args, out), offsetof(csa_params, n_win), sizeof(csa_paged_kv),
+         offsetof(csa_paged_kv, page_table), offsetof(csa_paged_kv, max_pages));
   return 0;
 }
 '''
@@ -81,8 +82,10 @@ int main(void) {
         subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), c, "-o", exe])
         vals = [int(x) for x in subprocess.check_output([exe]).split()]
     A = csa.CsaForwardArgs
+    K = csa.CsaPagedKv
     assert vals == [ctypes.sizeof(csa.CsaParams), ctypes.sizeof(A), A.idx_dtype.offset,
-                    A.N_cap.offset, A.out.offset, csa.CsaParams.n_win.offset]
+                    A.N_cap.offset, A.out.offset, csa.CsaParams.n_win.offset, ctypes.sizeof(K),
+                    K.page_table.offset, K.max_pages.offset]
 
 
 def _p(**kw):
@@ -274,6 +277,32 @@ def test_mixed_kv_attention_checks():
     h = [ctypes.byref(_p(m=128, overlap=0)), 1, 1, FAKE, FAKE, FAKE, None, 64, FAKE, 128, FAKE,
          None, None, FAKE, None, 0, None]
     assert L.hca_dense_mqa_mixed_kv(*h) == csa.CSA_ERR_INVALID_ARG  # no scales
+
+
+def test_paged_attention_checks():
+    L = csa.lib()
+    p = _p()
+    kv = csa.CsaPagedKv(csa.CSA_BF16, FAKE, None, FAKE, 64, 32, 16)
+
+    def call(kvd, idx=FAKE, params=p):
+        return L.csa_sparse_mqa_paged(ctypes.byref(params), 1, 1, FAKE, FAKE, ctypes.byref(kvd),
+                                      idx, FAKE, 128, FAKE, None, None, FAKE, None, 0, None)
+
+    assert L.csa_sparse_mqa_paged(ctypes.byref(p), 1, 1, FAKE, FAKE, None, FAKE, FAKE, 128, FAKE,
+                                  None, None, FAKE, None, 0, None) == csa.CSA_ERR_INVALID_ARG
+    assert call(csa.CsaPagedKv(csa.CSA_FP8_E4M3_ROWSCALE, FAKE, FAKE, FAKE, 64, 32, 16)) == \
+        csa.CSA_ERR_INVALID_ARG  # not a cache format
+    assert call(csa.CsaPagedKv(csa.CSA_BF16, FAKE, None, None, 64, 32, 16)) == \
+        csa.CSA_ERR_INVALID_ARG  # no page table
+    assert call(csa.CsaPagedKv(csa.CSA_BF16, FAKE, None, FAKE, 0, 32, 16)) == \
+        csa.CSA_ERR_INVALID_ARG  # empty pool
+    assert call(csa.CsaPagedKv(csa.CSA_MIXED_FP8_BF16, FAKE, None, FAKE, 64, 32, 16)) == \
+        csa.CSA_ERR_INVALID_ARG  # mixed rows without scales
+    assert call(kv, idx=None) == csa.CSA_ERR_INVALID_ARG
+    assert call(kv, params=_p(n_heads=32)) == csa.CSA_ERR_UNSUPPORTED
+    assert L.hca_dense_mqa_paged(ctypes.byref(_p(m=128, overlap=0)), 0, 1, None, None,
+                                 ctypes.byref(kv), None, 0, None, None, None, None, None, 0,
+                                 None) == csa.CSA_OK  # nothing to do
 
 
 def test_binding_refuses_host_tensors():

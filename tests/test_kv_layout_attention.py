@@ -1,0 +1,186 @@
+"""Attention over other KV cache layouts against the float64 oracle on the same bytes:
+mixed-precision rows (csa_sparse_mqa_mixed_kv, hca_dense_mqa_mixed_kv) and paged caches
+(csa_sparse_mqa_paged, hca_dense_mqa_paged).
+
+For mixed rows the workloads' bf16 caches are re-encoded by the input encoder (the first
+c - r values as e4m3 with a row scale, the RoPE values as bf16); the oracle decodes those
+bytes exactly, and the kernel widens code * scale to bf16 before its tensor-core products.
+For paged caches the rows are scattered into a pool of pages through a shuffled page
+table, and the oracle reads the contiguous cache. The outputs must meet the bf16 output
+tolerance.
+
+These kernels have not yet run on a B200: the module runs only with
+CSA_RUN_FIRST_GPU_CHECKS=1, so a first run is a deliberate, separate step.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import long_context_sparse_08_b200 as csa
+from long_context_sparse_08_b200 import runner as R
+from long_context_sparse_08_b200 import workloads as W
+from oracle import pipeline as P
+import tests.parity_util as U
+
+pytestmark = [
+    pytest.mark.gpu,
+    pytest.mark.skipif(os.environ.get("CSA_RUN_FIRST_GPU_CHECKS") != "1",
+                       reason="awaiting its first run on a B200 (CSA_RUN_FIRST_GPU_CHECKS=1)"),
+]
+
+
+def _mixed(name):
+    s, inp = U.inputs(name)
+    kv = W.bf16_bits_to_f32(inp["kv_cache"])
+    codes, scale, rope = W.quant_mixed_kv(kv, s.rope_dims)
+    rows = np.concatenate([codes, rope.view(np.uint8)], axis=-1)  # c + r bytes per row
+    inp2 = {k: v for k, v in inp.items() if k != "kv_cache"}
+    inp2.update(kv_codes=codes, kv_scale=scale, kv_rope=rope)
+    return s, inp, inp2, torch.from_numpy(np.ascontiguousarray(rows)).cuda(), \
+        torch.from_numpy(scale).cuda()
+
+
+@pytest.mark.parametrize("name", ["mid_decode_fp8", "mid_decode_mxfp4", "edge_decode_bf16"])
+def test_sparse_mqa_over_mixed_rows(name):
+    s, inp, inp2, rows, scale = _mixed(name)
+    res = P.run(s, inp2, want_scores=False)
+    dev = R.upload(inp, s)
+    idx = np.full((s.B, s.T, s.topk), -1, np.int32)
+    for (b, ti), sel in res["idx"].items():
+        idx[b, ti] = sel
+    p = R.params_for(s)
+    out = torch.empty((s.B, s.T, s.n_heads, s.c), dtype=dev["q"].dtype, device="cuda")
+    ws_bytes = csa.workspace_size(p, csa.CSA_WS_SPARSE_MQA, 0, s.B, s.T, s.n_cap)
+    ws = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device="cuda")
+    csa.csa_sparse_mqa_mixed_kv(p, s.B, s.T, dev["q"], dev["q_pos"], rows, scale, s.n_cap,
+                                torch.from_numpy(idx).cuda(), dev["win_kv"],
+                                dev["win_kv"].shape[1], dev["win_pos0"], dev["sink"], None, out,
+                                ws, ws_bytes)
+    torch.cuda.synchronize()
+    assert csa.device_error() == 0
+    got = out.float().cpu().numpy()
+    for (b, ti), ref in res["out"].items():
+        U.check_out(got[b, ti], ref, "bf16", f"{name} mixed KV b={b} t={ti}")
+
+
+@pytest.mark.parametrize("name", ["mid_hca_decode", "edge_hca_decode"])
+def test_dense_mqa_over_mixed_rows(name):
+    s, inp, inp2, rows, scale = _mixed(name)
+    res = P.run(s, inp2)
+    dev = R.upload(inp, s)
+    p = R.params_for(s)
+    out = torch.empty((s.B, s.T, s.n_heads, s.c), dtype=dev["q"].dtype, device="cuda")
+    ws_bytes = csa.workspace_size(p, csa.CSA_WS_HCA_MQA, 0, s.B, s.T, s.n_cap)
+    ws = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device="cuda")
+    csa.hca_dense_mqa_mixed_kv(p, s.B, s.T, dev["q"], dev["q_pos"], rows, scale, s.n_cap,
+                               dev["win_kv"], dev["win_kv"].shape[1], dev["win_pos0"],
+                               dev["sink"], None, out, ws, ws_bytes)
+    torch.cuda.synchronize()
+    assert csa.device_error() == 0
+    got = out.float().cpu().numpy()
+    for (b, ti), ref in res["out"].items():
+        U.check_out(got[b, ti], ref, "bf16", f"{name} mixed KV b={b}")
+
+
+def _paged(cache, page_rows, seed, extra_pages=5):
+    """Scatter a contiguous cache [B, n_cap, ...] into a page pool through a shuffled page
+    table; returns (pool, table [B, max_pages] int32)."""
+    B, n_cap = cache.shape[:2]
+    assert n_cap % page_rows == 0
+    max_pages = n_cap // page_rows
+    n_pages = B * max_pages + extra_pages
+    perm = np.random.default_rng(seed).permutation(n_pages).astype(np.int32)
+    table = perm[:B * max_pages].reshape(B, max_pages)
+    pool = np.zeros((n_pages, page_rows) + cache.shape[2:], cache.dtype)
+    for b in range(B):
+        for lp in range(max_pages):
+            pool[table[b, lp]] = cache[b, lp * page_rows:(lp + 1) * page_rows]
+    return pool, np.ascontiguousarray(table)
+
+
+def _dev(a):
+    a = np.ascontiguousarray(a)
+    return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).cuda()
+
+
+@pytest.mark.parametrize("name,mixed,page_rows", [("mid_decode_fp8", False, 32),
+                                                  ("mid_decode_mxfp4", True, 32),
+                                                  ("edge_decode_bf16", False, 32)])
+def test_sparse_mqa_over_paged_cache(name, mixed, page_rows):
+    s, inp = U.inputs(name)
+    if mixed:
+        s, inp, inp2, _, _ = _mixed(name)
+        codes, rope = inp2["kv_codes"], inp2["kv_rope"]
+        rows = np.concatenate([codes, rope.view(np.uint8)], axis=-1)
+        pool, table = _paged(rows, page_rows, 3)
+        spool, _ = _paged(inp2["kv_scale"][..., None], page_rows, 3)
+        scales = _dev(spool[..., 0])
+    else:
+        inp2 = inp
+        pool, table = _paged(inp["kv_cache"], page_rows, 3)
+        scales = None
+    res = P.run(s, inp2, want_scores=False)
+    dev = R.upload(inp, s)
+    idx = np.full((s.B, s.T, s.topk), -1, np.int32)
+    for (b, ti), sel in res["idx"].items():
+        idx[b, ti] = sel
+    p = R.params_for(s)
+    fmt = csa.CSA_MIXED_FP8_BF16 if mixed else csa.CSA_BF16
+    pool_d, table_d = _dev(pool), _dev(table)
+    kv = csa.paged_kv(fmt, pool_d, scales, table_d, pool.shape[0], page_rows, table.shape[1])
+    out = torch.empty((s.B, s.T, s.n_heads, s.c), dtype=dev["q"].dtype, device="cuda")
+    ws_bytes = csa.workspace_size(p, csa.CSA_WS_SPARSE_MQA, 0, s.B, s.T, s.n_cap)
+    ws = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device="cuda")
+    csa.csa_sparse_mqa_paged(p, s.B, s.T, dev["q"], dev["q_pos"], kv,
+                             torch.from_numpy(idx).cuda(), dev["win_kv"], dev["win_kv"].shape[1],
+                             dev["win_pos0"], dev["sink"], None, out, ws, ws_bytes)
+    torch.cuda.synchronize()
+    assert csa.device_error() == 0
+    got = out.float().cpu().numpy()
+    for (b, ti), ref in res["out"].items():
+        U.check_out(got[b, ti], ref, "bf16", f"{name} paged b={b} t={ti}")
+
+
+@pytest.mark.parametrize("page_rows", [1, 8])
+def test_dense_mqa_over_paged_cache(page_rows):
+    s, inp = U.inputs("mid_hca_decode")
+    res = P.run(s, inp)
+    dev = R.upload(inp, s)
+    pool, table = _paged(inp["kv_cache"], page_rows, 4)
+    p = R.params_for(s)
+    kv = csa.paged_kv(csa.CSA_BF16, _dev(pool), None, _dev(table), pool.shape[0], page_rows,
+                      table.shape[1])
+    out = torch.empty((s.B, s.T, s.n_heads, s.c), dtype=dev["q"].dtype, device="cuda")
+    ws_bytes = csa.workspace_size(p, csa.CSA_WS_HCA_MQA, 0, s.B, s.T, s.n_cap)
+    ws = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device="cuda")
+    csa.hca_dense_mqa_paged(p, s.B, s.T, dev["q"], dev["q_pos"], kv, dev["win_kv"],
+                            dev["win_kv"].shape[1], dev["win_pos0"], dev["sink"], None, out, ws,
+                            ws_bytes)
+    torch.cuda.synchronize()
+    assert csa.device_error() == 0
+    got = out.float().cpu().numpy()
+    for (b, ti), ref in res["out"].items():
+        U.check_out(got[b, ti], ref, "bf16", f"mid_hca_decode paged({page_rows}) b={b}")
+
+
+def test_paged_cache_with_a_bad_page_id_reports_it():
+    s, inp = U.inputs("mid_hca_decode")
+    dev = R.upload(inp, s)
+    pool, table = _paged(inp["kv_cache"], 8, 5)
+    table[0, 0] = pool.shape[0]  # outside the pool
+    p = R.params_for(s)
+    kv = csa.paged_kv(csa.CSA_BF16, _dev(pool), None, _dev(table), pool.shape[0], 8,
+                      table.shape[1])
+    out = torch.empty((s.B, s.T, s.n_heads, s.c), dtype=dev["q"].dtype, device="cuda")
+    ws_bytes = csa.workspace_size(p, csa.CSA_WS_HCA_MQA, 0, s.B, s.T, s.n_cap)
+    ws = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+    csa.device_error()
+    csa.hca_dense_mqa_paged(p, s.B, s.T, dev["q"], dev["q_pos"], kv, dev["win_kv"],
+                            dev["win_kv"].shape[1], dev["win_pos0"], dev["sink"], None, out, ws,
+                            ws_bytes)
+    torch.cuda.synchronize()
+    assert csa.device_error() == 205
+
