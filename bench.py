@@ -49,6 +49,9 @@ def parse():
     ap.add_argument("--replicas", type=int, default=0,
                     help="input replicas rotated across steps (0: enough to defeat the L2)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end measurement")
+    ap.add_argument("--part", default=None, choices=sorted(PARTS),
+                    help="time one extension kernel family on the workload's shape instead of "
+                         "the hot path (its own JSON line; see run_part)")
     return ap.parse_args()
 
 
@@ -428,8 +431,217 @@ def run_e2e(args, s, devs, steps, R_rep, world):
             "state_resident": "compressed KV, indexer keys and window rows stay in HBM"}
 
 
+# ---------------------------------------------------------------------------
+# --part: the extension kernels timed alone on the workload's shapes
+# ---------------------------------------------------------------------------
+
+# grouped output projection (Q, H, c, g, d_g, d) per decode workload: the model table's
+# g / d_g / d with the workload's batch as the queries
+OUT_PROJ_SHAPES = {"pro_decode_1m": (4, 128, 512, 16, 1024, 7168),
+                   "flash_decode_131k": (8, 64, 512, 8, 1024, 4096),
+                   "hca_decode_1m": (16, 64, 512, 8, 1024, 4096)}
+
+
+def out_proj_bytes(Q, H, c, g, d_g, d) -> int:
+    """Algorithmic bytes of one grouped output projection: both weight matrices (bf16), the
+    attention outputs read and the projection written (fp32 partials are scratch)."""
+    k1 = c * H // g
+    return 2 * (g * k1 * d_g + g * d_g * d) + 2 * Q * H * c + 2 * Q * d
+
+
+def state_append_bytes(c, m, overlap, key_c=128, key_fmt_bytes=68) -> dict:
+    """Algorithmic bytes of appending one token to one request, averaged over a block: the
+    raw rows read and stored in the state, the window row read and stored (KV only), and,
+    every m-th token, the block's rows read back and the finished row written. KV entries
+    are bf16 rows of c values; indexer keys are c = 128 values stored as MXFP4 (68 B)."""
+    rows = 4 if overlap else 2
+    kv = 2 * c * (rows * 2 + 2) + (2 * m * rows * c + 2 * c) // m
+    keys = 2 * key_c * rows * 2 + (2 * m * rows * key_c + key_fmt_bytes) // m
+    return {"kv": kv, "keys": keys, "total": kv + keys}
+
+
+def _time_calls(fn, n_rep, warmup, steps):
+    """Mean ms per call of fn(i) over `steps` calls (rotating i over n_rep replicas),
+    timed with CUDA events on the current stream after `warmup` calls."""
+    import torch
+
+    for i in range(warmup):
+        fn(i % n_rep)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(steps):
+        fn(i % n_rep)
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
+
+
+def run_part(args, W):
+    """One JSON line for an extension kernel family on the workload's shape:
+    out_proj      grouped output projection of the batch's queries (HBM roofline);
+    state_append  one decode token per request into the KV and indexer-key state caches;
+    kv_layouts    the attention alone over bf16, mixed-precision and paged caches."""
+    import torch
+    import long_context_sparse_08_b200 as csa
+    from long_context_sparse_08_b200 import runner as R
+
+    torch.cuda.set_device(0)
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
+    s = W.SHAPES[args.workload]
+    before = csa.kernel_launches()
+    clocks = Clocks(0)
+    line = {"part": args.part, "workload": args.workload, "steps": args.steps,
+            "warmup": args.warmup, "data": "synthetic (seeded)"}
+    if args.part == "out_proj":
+        Q, H, c, g, d_g, d = OUT_PROJ_SHAPES[args.workload]
+        inp = W.make_out_proj_inputs(Q=Q, H=H, c=c, g=g, d_g=d_g, d=d, seed=11)
+        nbytes = out_proj_bytes(Q, H, c, g, d_g, d)
+        n_rep = max(1, min(4, int(np.ceil(3 * L2_BYTES / nbytes))))
+        p = csa.make_params(c=c, n_heads=H)
+        reps = []
+        for _ in range(n_rep):
+            dv = {k: torch.from_numpy(v.view(np.int16)).cuda() for k, v in inp.items()}
+            need = csa.grouped_out_proj_workspace_size(p, Q, g, d_g, d)
+            dv["ws"] = torch.empty((need,), dtype=torch.uint8, device="cuda")
+            dv["out"] = torch.empty((Q, d), dtype=torch.int16, device="cuda")
+            reps.append((dv, need))
+
+        def call(i):
+            dv, need = reps[i]
+            csa.csa_grouped_out_proj(p, Q, g, d_g, d, dv["o"], dv["w_grp"], dv["w_out"],
+                                     dv["out"], dv["ws"], need)
+
+        ms = _time_calls(call, n_rep, args.warmup, args.steps)
+        ach = nbytes / (ms / 1e3) / 1e9
+        line.update(metric="grouped output projection calls/s", value=round(1e3 / ms, 2),
+                    unit="calls/s", ms_per_call=round(ms, 5),
+                    config={"Q": Q, "H": H, "c": c, "g": g, "d_g": d_g, "d": d,
+                            "replicas": n_rep},
+                    roofline={"bound": "hbm", "achieved": round(ach, 1), "peak": hbm,
+                              "peak_source": peak_src, "unit": "GB/s",
+                              "frac": round(ach / hbm, 4), "bytes_per_call": nbytes})
+    elif args.part == "state_append":
+        B, c = s.B, s.c
+        p_kv = csa.make_params(m=4, overlap=1, c=c, rope_dims=s.rope_dims, n_win=s.n_win)
+        p_k = csa.make_params(m=4, overlap=1, c=128, rope_dims=64, n_win=s.n_win)
+        g = torch.Generator(device="cuda").manual_seed(5)
+        rnd = lambda *sh: torch.randn(*sh, generator=g, device="cuda").to(torch.bfloat16)  # noqa
+        n_steps = args.warmup + args.steps
+        t0 = 4 * 128  # every request past its first page
+        kv_rows = {k: rnd(n_steps, B, c) for k in ("Ca", "Cb", "Za", "Zb", "win")}
+        key_rows = {k: rnd(n_steps, B, 128) for k in ("Ca", "Cb", "Za", "Zb")}
+        bias_kv, bias_k = rnd(8, c), rnd(8, 128)
+        max_pages = (t0 + n_steps) // 128 + 2
+        table32 = torch.arange(B * max_pages, dtype=torch.int32, device="cuda").view(B, -1)
+        table128 = table32.clone()
+        st_kv = torch.zeros((B, 8, 4, c), dtype=torch.bfloat16, device="cuda")
+        st_k = torch.zeros((B, 8, 4, 128), dtype=torch.bfloat16, device="cuda")
+        ring = torch.zeros((B, s.n_win, c), dtype=torch.bfloat16, device="cuda")
+        pages_kv = torch.zeros((B * max_pages, 32, c), dtype=torch.bfloat16, device="cuda")
+        pages_k = torch.zeros((B * max_pages, 128, 64), dtype=torch.uint8, device="cuda")
+        exps_k = torch.zeros((B * max_pages, 128, 4), dtype=torch.uint8, device="cuda")
+        pos_all = t0 + torch.arange(n_steps, device="cuda", dtype=torch.int64)[:, None].repeat(1, B)
+
+        def call(i):
+            pos = pos_all[i]
+            csa.csa_state_append(p_kv, csa.CSA_BF16, B, pos, kv_rows["Ca"][i], kv_rows["Cb"][i],
+                                 kv_rows["Za"][i], kv_rows["Zb"][i], kv_rows["win"][i], bias_kv,
+                                 None, 1, st_kv, ring, csa.CSA_BF16, pages_kv, None,
+                                 B * max_pages, 32, table32, max_pages)
+            csa.csa_state_append(p_k, csa.CSA_BF16, B, pos, key_rows["Ca"][i], key_rows["Cb"][i],
+                                 key_rows["Za"][i], key_rows["Zb"][i], None, bias_k, None, 0,
+                                 st_k, None, csa.CSA_MXFP4, pages_k, exps_k, B * max_pages, 128,
+                                 table128, max_pages)
+
+        for i in range(args.warmup):
+            call(i)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for i in range(args.warmup, n_steps):
+            call(i)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / args.steps
+        per = state_append_bytes(c, 4, 1)
+        ach = B * per["total"] / (ms / 1e3) / 1e9
+        line.update(metric="decode appends/s (KV + indexer keys, one token per request)",
+                    value=round(B / (ms / 1e3), 1), unit="appends/s", ms_per_step=round(ms, 5),
+                    config={"requests": B, "c": c, "kv": "bf16 pages of 32 entries",
+                            "keys": "MXFP4 pages of 128 keys"},
+                    roofline={"bound": "latency (a few KB per request)", "achieved": round(ach, 2),
+                              "peak": hbm, "peak_source": peak_src, "unit": "GB/s",
+                              "frac": round(ach / hbm, 6), "bytes_per_append": per})
+    elif args.part == "kv_layouts":
+        inp = W.make_inputs(s)
+        dev = R.upload(inp, s)
+        p = R.params_for(s)
+        B, T, k = s.B, s.T, s.topk
+        g = torch.Generator(device="cpu").manual_seed(9)
+        n_vis = min(s.ctx // s.m, s.n_cap)
+        idx = torch.stack([torch.randperm(n_vis, generator=g)[:k] for _ in range(B * T)])
+        idx = idx.view(B, T, k).to(torch.int32).cuda()
+        kv = W.bf16_bits_to_f32(inp["kv_cache"])
+        codes, scale, rope = W.quant_mixed_kv(kv, s.rope_dims)
+        del kv
+        mixed = torch.from_numpy(np.concatenate([codes, rope.view(np.uint8)], axis=-1)).cuda()
+        mscale = torch.from_numpy(scale).cuda()
+        del codes, rope
+        pr = 32
+        max_pages = s.n_cap // pr
+        perm = torch.randperm(B * max_pages, generator=g).to(torch.int32)
+        table = perm.view(B, max_pages).cuda()
+        pool = torch.empty((B * max_pages, pr, s.c), dtype=dev["kv_cache"].dtype, device="cuda")
+        pool[table.view(-1).long()] = dev["kv_cache"].view(B * max_pages, pr, s.c)
+        out = torch.empty((B, T, s.n_heads, s.c), dtype=dev["q"].dtype, device="cuda")
+        ws_bytes = csa.workspace_size(p, csa.CSA_WS_SPARSE_MQA, 0, B, T, s.n_cap)
+        ws = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device="cuda")
+        pkv = csa.paged_kv(csa.CSA_BF16, pool, None, table, B * max_pages, pr, max_pages)
+        L = dev["win_kv"].shape[1]
+        calls = {
+            "bf16": lambda i: csa.csa_sparse_mqa(p, csa.CSA_BF16, B, T, dev["q"], dev["q_pos"],
+                                                 dev["kv_cache"], s.n_cap, idx, dev["win_kv"], L,
+                                                 dev["win_pos0"], dev["sink"], None, out, ws,
+                                                 ws_bytes),
+            "mixed": lambda i: csa.csa_sparse_mqa_mixed_kv(p, B, T, dev["q"], dev["q_pos"], mixed,
+                                                           mscale, s.n_cap, idx, dev["win_kv"], L,
+                                                           dev["win_pos0"], dev["sink"], None,
+                                                           out, ws, ws_bytes),
+            "paged_bf16": lambda i: csa.csa_sparse_mqa_paged(p, B, T, dev["q"], dev["q_pos"], pkv,
+                                                             idx, dev["win_kv"], L,
+                                                             dev["win_pos0"], dev["sink"], None,
+                                                             out, ws, ws_bytes)}
+        res = {}
+        for name, fn in calls.items():
+            ms = _time_calls(fn, 1, args.warmup, args.steps)
+            row = 1024 if name != "mixed" else s.c + s.rope_dims + 4
+            nbytes = B * T * ((k * row) + s.n_win * 2 * s.c + 2 * 2 * s.n_heads * s.c)
+            res[name] = {"ms_per_call": round(ms, 5), "bytes_per_call": nbytes,
+                         "achieved_gbs": round(nbytes / (ms / 1e3) / 1e9, 1)}
+        line.update(metric="sparse MQA calls/s by cache layout",
+                    value=round(1e3 / res["mixed"]["ms_per_call"], 2), unit="calls/s (mixed)",
+                    layouts=res, config={"B": B, "T": T, "k": k, "n_cap": s.n_cap,
+                                         "page_rows": pr},
+                    roofline={"bound": "latency (see the attention in DESIGN)", "peak": hbm,
+                              "peak_source": peak_src, "unit": "GB/s"})
+    line["gpu_launches"] = int(csa.kernel_launches() - before)
+    line["clocks"] = clocks.stop()
+    line["device_error"] = csa.device_error()
+    print(json.dumps(line))
+    return 0
+
+
+PARTS = {"out_proj", "state_append", "kv_layouts"}
+
+
 def main():
     args = parse()
+    if args.part is not None:
+        from long_context_sparse_08_b200 import workloads as W
+
+        return run_part(args, W)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -85,3 +85,15 @@ def test_reference_arm_prints_the_contract_line():
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_extension_bytes(bench):
+    # grouped projection, Pro decode: 16 groups of 4096 x 1024 and 16384 x 7168 bf16 weights,
+    # 4 queries of 128 x 512 bf16 in, 7168 bf16 out
+    assert bench.out_proj_bytes(4, 128, 512, 16, 1024, 7168) == \
+        2 * (16 * 4096 * 1024 + 16384 * 7168) + 2 * 4 * 128 * 512 + 2 * 4 * 7168
+    # one CSA append, c = 512: 4 raw rows read and stored, the window row read and stored;
+    # every 4th token reads back 4 x 4 rows and writes one entry
+    kv = 2 * 512 * (4 + 4 + 1 + 1) + (16 * 512 * 2 + 512 * 2) // 4
+    keys = 2 * 128 * (4 + 4) + (16 * 128 * 2 + 68) // 4
+    assert bench.state_append_bytes(512, 4, 1) == {"kv": kv, "keys": keys, "total": kv + keys}
