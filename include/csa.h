@@ -345,16 +345,19 @@ size_t csa_workspace_size(const csa_params* p, int32_t entry, csa_dtype kdt, int
                           int32_t T, int64_t N_cap);
 
 /*
- * Grouped output projection ([P1] 一(三)1(4) 分组输出投影; 2(2) for HCA) of Q <= 16 decode
- * queries: the H = p->n_heads head outputs of query q, o[q] bf16 [H * c] (head after head,
+ * Grouped output projection ([P1] 一(三)1(4) 分组输出投影; 2(2) for HCA) of Q queries: the
+ * H = p->n_heads head outputs of query q, o[q] bf16 [H * c] (head after head,
  * the attention's out), are split into g groups of H/g heads; group i's c*H/g values times
  * w_grp[i] (bf16 [c*H/g, d_g]) give the intermediate o'[q, i*d_g .. (i+1)*d_g-1], and the
  * g*d_g intermediate values times w_out (bf16 [g*d_g, d]) give out[q] (bf16 [d]). Row
  * vectors multiply matrices from the left (x . W). Sums are fp32 over splits of the rows,
  * added in a fixed order (the intermediate stays fp32); the result is rounded to bf16 once.
- * With few queries each weight byte carries ~Q flops: the call streams the weights from
- * HBM on CUDA cores. Needs d_g and d multiples of 8 and n_heads a multiple of g; Q > 16
- * returns CSA_ERR_UNSUPPORTED. Workspace: csa_grouped_out_proj_workspace_size().
+ * Decode (Q < 128): each weight byte carries ~Q flops, so the call streams the weights from
+ * HBM on CUDA cores, 16 queries per pass; sums stay fp32 until the final rounding.
+ * Prefill (Q >= 128): two tcgen05 bf16 GEMMs with fp32 accumulation; the intermediate is
+ * stored once in bf16 (needs c*H/g and g*d_g multiples of 64, d_g and d >= 64, else
+ * CSA_ERR_UNSUPPORTED). Needs d_g and d multiples of 8 and n_heads a multiple of g.
+ * Workspace: csa_grouped_out_proj_workspace_size().
  */
 csa_status csa_grouped_out_proj(const csa_params* p, int32_t Q, int32_t g, int32_t d_g,
                                 int32_t d, const void* o, const void* w_grp, const void* w_out,

@@ -245,11 +245,12 @@ const char* csa_last_error(void) { return g_err; }
 
 csa_status csa_device_error(int32_t* code) {
   REQUIRE(code != nullptr, "code is NULL");
-  int words[4] = {0, 0, 0, 0};
+  int words[5] = {0, 0, 0, 0, 0};
   TRY(cuda_status(csa::index_mxf4_device_error(&words[0]), "device error word"));
   TRY(cuda_status(csa::mqa_tc_device_error(&words[1]), "device error word"));
   TRY(cuda_status(csa::index_bf16_device_error(&words[2]), "device error word"));
   TRY(cuda_status(csa::state_append_device_error(&words[3]), "device error word"));
+  TRY(cuda_status(csa::out_proj_tc_device_error(&words[4]), "device error word"));
   *code = 0;
   for (int w : words)
     if (*code == 0) *code = w;
@@ -415,17 +416,28 @@ csa_status check_out_proj(const csa_params* p, int32_t Q, int32_t g, int32_t d_g
           "d_g and d must be positive multiples of 8 (got %d, %d)", d_g, d);
   REQUIRE((int64_t)p->c * p->n_heads <= (1 << 24) && (int64_t)g * d_g <= (1 << 24) &&
               d <= (1 << 24), "sizes too large");
-  if (Q > 16)
-    return fail(CSA_ERR_UNSUPPORTED,
-                "grouped output projection: decode batches of at most 16 queries (got %d)", Q);
+  if (Q >= 128) {
+    const csa::proj::Geom G = csa::out_proj_geom(Q, p->n_heads, p->c, g, d_g, d);
+    if (!csa::out_proj_tc_shape_ok(G))
+      return fail(CSA_ERR_UNSUPPORTED,
+                  "grouped output projection of %d queries: the tensor-core form needs c*H/g "
+                  "and g*d_g multiples of 64 and d_g, d >= 64", Q);
+  }
   return CSA_OK;
 }
+
+// Queries per pass of the weight-streaming (decode) kernels, and the form a call takes.
+constexpr int32_t kStreamQueries = 16;
+bool out_proj_uses_tc(int32_t Q) { return Q >= 128; }
 }  // namespace
 
 size_t csa_grouped_out_proj_workspace_size(const csa_params* p, int32_t Q, int32_t g,
                                            int32_t d_g, int32_t d) {
   if (check_out_proj(p, Q, g, d_g, d) != CSA_OK || Q == 0) return 0;
-  return csa::out_proj_workspace_bytes(csa::out_proj_geom(Q, p->n_heads, p->c, g, d_g, d));
+  if (out_proj_uses_tc(Q))
+    return csa::out_proj_tc_workspace_bytes(csa::out_proj_geom(Q, p->n_heads, p->c, g, d_g, d));
+  const int32_t q = Q < kStreamQueries ? Q : kStreamQueries;
+  return csa::out_proj_workspace_bytes(csa::out_proj_geom(q, p->n_heads, p->c, g, d_g, d));
 }
 
 csa_status csa_grouped_out_proj(const csa_params* p, int32_t Q, int32_t g, int32_t d_g,
@@ -437,16 +449,28 @@ csa_status csa_grouped_out_proj(const csa_params* p, int32_t Q, int32_t g, int32
   REQUIRE_PTR(w_grp);
   REQUIRE_PTR(w_out);
   REQUIRE_PTR(out);
-  csa::OutProjArgs a{};
-  a.G = csa::out_proj_geom(Q, p->n_heads, p->c, g, d_g, d);
-  const size_t need = csa::out_proj_workspace_bytes(a.G);
+  const size_t need = csa_grouped_out_proj_workspace_size(p, Q, g, d_g, d);
   if (ws == nullptr || ws_bytes < need || !aligned16(ws))
     return fail(CSA_ERR_WORKSPACE, "grouped output projection needs %zu workspace bytes", need);
-  a.o = static_cast<const __nv_bfloat16*>(o);
+  csa::OutProjArgs a{};
   a.w_grp = static_cast<const __nv_bfloat16*>(w_grp);
   a.w_out = static_cast<const __nv_bfloat16*>(w_out);
-  a.out = static_cast<__nv_bfloat16*>(out);
-  TRY(cuda_status(csa::launch_out_proj(a, ws, (cudaStream_t)stream), "grouped output projection"));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (out_proj_uses_tc(Q)) {  // prefill: two tensor-core GEMMs
+    a.G = csa::out_proj_geom(Q, p->n_heads, p->c, g, d_g, d);
+    a.o = static_cast<const __nv_bfloat16*>(o);
+    a.out = static_cast<__nv_bfloat16*>(out);
+    TRY(cuda_status(csa::launch_out_proj_tc(a, ws, st), "grouped output projection"));
+    return ok();
+  }
+  // decode: weight streaming, at most kStreamQueries queries per pass
+  for (int32_t q0 = 0; q0 < Q; q0 += kStreamQueries) {
+    const int32_t q = Q - q0 < kStreamQueries ? Q - q0 : kStreamQueries;
+    a.G = csa::out_proj_geom(q, p->n_heads, p->c, g, d_g, d);
+    a.o = static_cast<const __nv_bfloat16*>(o) + (size_t)q0 * p->n_heads * p->c;
+    a.out = static_cast<__nv_bfloat16*>(out) + (size_t)q0 * d;
+    TRY(cuda_status(csa::launch_out_proj(a, ws, st), "grouped output projection"));
+  }
   return ok();
 }
 

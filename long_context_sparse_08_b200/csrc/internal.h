@@ -43,6 +43,11 @@ struct OutProjArgs;
 proj::Geom out_proj_geom(int Q, int H, int c, int g, int d_g, int d);
 size_t out_proj_workspace_bytes(const proj::Geom& G);
 cudaError_t launch_out_proj(OutProjArgs a, void* ws, cudaStream_t st);
+// prefill form on tensor cores (Q >= 128 queries)
+bool out_proj_tc_shape_ok(const proj::Geom& G);
+size_t out_proj_tc_workspace_bytes(const proj::Geom& G);
+cudaError_t launch_out_proj_tc(const OutProjArgs& a, void* ws, cudaStream_t st);
+cudaError_t out_proj_tc_device_error(int* code);
 
 namespace state { struct Args; }
 // decode-time append of one token per request into the state cache and its pages

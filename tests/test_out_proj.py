@@ -93,7 +93,9 @@ def test_checks_on_the_host():
     F = 0x10000
     p = _p(128, 512)
     args = lambda Q, g, dg, d: (ctypes.byref(p), Q, g, dg, d, F, F, F, F, F, 1 << 30, None)  # noqa
-    assert L.csa_grouped_out_proj(*args(17, 16, 1024, 7168)) == csa.CSA_ERR_UNSUPPORTED
+    # the tensor-core form (Q >= 128) needs g * d_g a multiple of 64 and d_g >= 64
+    assert L.csa_grouped_out_proj(*args(128, 1, 8, 7168)) == csa.CSA_ERR_UNSUPPORTED
+    assert L.csa_grouped_out_proj(*args(128, 16, 8, 7168)) == csa.CSA_ERR_UNSUPPORTED
     assert L.csa_grouped_out_proj(*args(4, 16, 1024, 7100 + 1)) == csa.CSA_ERR_INVALID_ARG
     assert L.csa_grouped_out_proj(*args(4, 48, 1024, 7168)) == csa.CSA_ERR_INVALID_ARG
     assert L.csa_grouped_out_proj(*args(0, 16, 1024, 7168)) == csa.CSA_OK
@@ -102,6 +104,12 @@ def test_checks_on_the_host():
     assert L.csa_grouped_out_proj(*a) == csa.CSA_ERR_INVALID_ARG
     need = csa.grouped_out_proj_workspace_size(p, 4, 16, 1024, 7168)
     assert need >= (4 * 16 * 1024 + 4 * 7168) * 4
+    # larger decode batches run 16 queries per pass in the same workspace; prefill keeps the
+    # bf16 intermediate
+    assert csa.grouped_out_proj_workspace_size(p, 100, 16, 1024, 7168) == \
+        csa.grouped_out_proj_workspace_size(p, 16, 16, 1024, 7168)
+    assert csa.grouped_out_proj_workspace_size(p, 4096, 16, 1024, 7168) == \
+        4096 * 16 * 1024 * 2 + 256
     a = list(args(4, 16, 1024, 7168))
     a[10] = need - 1
     assert L.csa_grouped_out_proj(*a) == csa.CSA_ERR_WORKSPACE
@@ -143,3 +151,37 @@ def test_gpu_decode_shapes_sampled(shape):
     got = _run_gpu(inp, *shape)
     cols = np.unique(np.concatenate([np.arange(0, d, 97), [d - 1]]))
     _check(got[:, cols], _oracle(inp, *shape, cols=cols), f"gpu {shape} sampled")
+
+
+@pytest.mark.gpu
+def test_gpu_decode_batch_of_forty_queries():
+    # 40 queries: three passes of the weight-streaming kernels (16 + 16 + 8)
+    shape = (40, 8, 64, 2, 96, 136)
+    Q, H, c, g, d_g, d = shape
+    inp = W.make_out_proj_inputs(Q=Q, H=H, c=c, g=g, d_g=d_g, d=d, seed=40)
+    _check(_run_gpu(inp, *shape), _oracle(inp, *shape), f"gpu {shape}")
+
+
+# prefill (tensor-core GEMMs): not yet run on a B200, so only with CSA_RUN_FIRST_GPU_CHECKS=1
+PREFILL = [(128, 8, 64, 2, 64, 128), (1000, 64, 512, 8, 1024, 4096)]
+
+
+@pytest.mark.gpu
+@pytest.mark.skipif(os.environ.get("CSA_RUN_FIRST_GPU_CHECKS") != "1",
+                    reason="awaiting its first run on a B200 (CSA_RUN_FIRST_GPU_CHECKS=1)")
+@pytest.mark.parametrize("shape", PREFILL, ids=["small", "flash_1000_queries"])
+def test_gpu_prefill_gemm_sampled(shape):
+    Q, H, c, g, d_g, d = shape
+    inp = W.make_out_proj_inputs(Q=Q, H=H, c=c, g=g, d_g=d_g, d=d, seed=8)
+    got = _run_gpu(inp, *shape)
+    import long_context_sparse_08_b200 as csa
+
+    assert csa.device_error() == 0
+    qs = np.unique(np.concatenate([np.arange(0, Q, 61), [Q - 1]]))
+    cols = np.unique(np.concatenate([np.arange(0, d, 37), [d - 1]]))
+    sub = dict(inp, o=inp["o"][qs])
+    ref = _oracle(sub, len(qs), H, c, g, d_g, d, cols=cols)
+    # the bf16 intermediate adds a rounding: the bf16 output tolerance applies
+    for i, q in enumerate(qs):
+        U.check_out(O.dec_bf16(got[q, cols]), ref[i], "bf16", f"prefill {shape} q={q}")
+
