@@ -85,7 +85,8 @@ typedef enum {
   CSA_WS_TOPK = 2,
   CSA_WS_SPARSE_MQA = 3,
   CSA_WS_HCA_MQA = 4,
-  CSA_WS_FORWARD = 5
+  CSA_WS_FORWARD = 5,
+  CSA_WS_INDEX_TOPK_BF16 = 6
 } csa_ws_entry;
 
 /*
@@ -219,6 +220,22 @@ csa_status csa_index_topk(const csa_params* p, csa_dtype kdt, int32_t B, int32_t
                           const void* KI, const void* KI_scale, const int64_t* q_pos,
                           int32_t* out_idx, float* out_scores, void* ws, size_t ws_bytes,
                           void* stream);
+
+/*
+ * Stages 2 + 3 with BF16 index scores ([P1'] 二(四): the scores are quantised from FP32 to
+ * BF16 before the top-k selector). Each score is computed in fp32 as in csa_index_scores,
+ * rounded to the nearest bf16 (ties to even) and stored as bf16 [B, T, N_cap] (out_scores16,
+ * or the workspace when NULL); the selector then orders the bf16 values by (value desc,
+ * index asc), so scores that round alike tie and the smaller index wins. Half the score
+ * bytes of csa_index_topk. Keys: CSA_FP8_E4M3_ROWSCALE or CSA_BF16 on the tensor-core
+ * indexer (64 heads of 128, N_cap a multiple of 128), else CSA_ERR_UNSUPPORTED. Workspace:
+ * csa_workspace_size(..., CSA_WS_INDEX_TOPK_BF16, ...).
+ */
+csa_status csa_index_topk_bf16(const csa_params* p, csa_dtype kdt, int32_t B, int32_t T,
+                               int64_t N_cap, const void* qI, const void* qI_scale,
+                               const float* w, const void* KI, const void* KI_scale,
+                               const int64_t* q_pos, int32_t* out_idx, void* out_scores16,
+                               void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Stage 4 -- shared-KV MQA over the selected entries plus the window ([P1] 1(3), 3(1)-(4)).

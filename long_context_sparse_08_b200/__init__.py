@@ -17,7 +17,8 @@ LIB_PATH = os.path.join(HERE, "libcsa.so")
 CSA_OK, CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_WORKSPACE, CSA_ERR_CUDA = range(5)
 CSA_F32, CSA_BF16, CSA_FP8_E4M3_ROWSCALE, CSA_MXFP4, CSA_MIXED_FP8_BF16 = range(5)
 DTYPES = {"f32": CSA_F32, "bf16": CSA_BF16, "fp8": CSA_FP8_E4M3_ROWSCALE, "mxfp4": CSA_MXFP4}
-CSA_WS_INDEX_TOPK, CSA_WS_TOPK, CSA_WS_SPARSE_MQA, CSA_WS_HCA_MQA, CSA_WS_FORWARD = range(1, 6)
+(CSA_WS_INDEX_TOPK, CSA_WS_TOPK, CSA_WS_SPARSE_MQA, CSA_WS_HCA_MQA, CSA_WS_FORWARD,
+ CSA_WS_INDEX_TOPK_BF16) = range(1, 7)
 
 EXPORTS = (
     "csa_compress", "csa_index_scores", "csa_topk", "csa_index_topk", "csa_sparse_mqa",
@@ -25,7 +26,7 @@ EXPORTS = (
     "csa_last_error", "csa_set_index_timing_events", "csa_version", "csa_device_error",
     "csa_topk_noalloc", "csa_kernel_launches", "csa_state_append", "csa_sparse_mqa_mixed_kv",
     "hca_dense_mqa_mixed_kv", "csa_grouped_out_proj", "csa_grouped_out_proj_workspace_size",
-    "csa_sparse_mqa_paged", "hca_dense_mqa_paged",
+    "csa_sparse_mqa_paged", "hca_dense_mqa_paged", "csa_index_topk_bf16",
 )
 # size of the library-owned scratch array behind csa_topk_noalloc (bytes, per device)
 TOPK_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -97,6 +98,7 @@ _SIGS = {
                              _I64, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "hca_dense_mqa_paged": [_PP, _I32, _I32, _VP, _VP, ctypes.POINTER(CsaPagedKv), _VP, _I64,
                             _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
+    "csa_index_topk_bf16": [_PP, ctypes.c_int, _I32, _I32, _I64] + [_VP] * 9 + [_SZ, _VP],
     "csa_grouped_out_proj": [_PP, _I32, _I32, _I32, _I32, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "csa_grouped_out_proj_workspace_size": [_PP, _I32, _I32, _I32, _I32],
     "csa_sparse_mqa_mixed_kv": [_PP, _I32, _I32, _VP, _VP, _VP, _VP, _I64, _VP, _VP, _I64, _VP,
@@ -242,6 +244,14 @@ def csa_index_topk(p, kdt, B, T, N_cap, qI, qI_scale, w, KI, KI_scale, q_pos, ou
                              _ptr(w), _ptr(KI), _ptr(KI_scale), _ptr(q_pos), _ptr(out_idx),
                              _ptr(out_scores), _ptr(ws), ws_bytes, _stream(stream))
     _check("csa_index_topk", s)
+
+
+def csa_index_topk_bf16(p, kdt, B, T, N_cap, qI, qI_scale, w, KI, KI_scale, q_pos, out_idx,
+                        out_scores16, ws, ws_bytes, stream=None):
+    s = lib().csa_index_topk_bf16(ctypes.byref(p), kdt, B, T, N_cap, _ptr(qI), _ptr(qI_scale),
+                                  _ptr(w), _ptr(KI), _ptr(KI_scale), _ptr(q_pos), _ptr(out_idx),
+                                  _ptr(out_scores16), _ptr(ws), ws_bytes, _stream(stream))
+    _check("csa_index_topk_bf16", s)
 
 
 def csa_sparse_mqa(p, io, B, T, q, q_pos, kv_cache, N_cap, idx, win_kv, L_raw, win_pos0, sink,

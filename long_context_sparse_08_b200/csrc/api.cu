@@ -206,11 +206,12 @@ csa_status index_then_topk(const csa_params* p, csa_dtype kdt, int32_t B, int32_
                            int64_t N_cap, const void* qI, const void* qI_scale, const float* w,
                            const void* KI, const void* KI_scale, const int64_t* q_pos,
                            float* scores, const csa::TopkArgs& t, void* topk_ws,
-                           size_t topk_bytes, cudaStream_t st) {
+                           size_t topk_bytes, cudaStream_t st, void* scores16 = nullptr) {
   bool hist_done = false;
   const bool decode = csa::topk_decode_path(B, T, N_cap, p->topk);
   if (N_cap > 0) {
     auto ia = make_index(p, kdt, B, T, N_cap, qI, qI_scale, w, KI, KI_scale, q_pos, scores);
+    ia.scores16 = scores16;
     if (decode) {
       const csa::TopkDecodeArgs da = csa::topk_decode_args(t, topk_ws);
       TRY(cuda_status(csa::topk_decode_clear(da, st), "top-k clear"));
@@ -289,6 +290,8 @@ size_t csa_workspace_size(const csa_params* p, int32_t entry, csa_dtype kdt, int
   switch (entry) {
     case CSA_WS_INDEX_TOPK:
       return scores_bytes(B, T, N_cap) + topk_ws;
+    case CSA_WS_INDEX_TOPK_BF16:
+      return round_up((size_t)B * T * (size_t)N_cap * 2) + topk_ws;
     case CSA_WS_TOPK:
       return topk_ws;
     case CSA_WS_SPARSE_MQA:
@@ -530,6 +533,37 @@ csa_status csa_index_topk(const csa_params* p, csa_dtype kdt, int32_t B, int32_t
   t.q_pos = q_pos; t.out_idx = out_idx;
   TRY(index_then_topk(p, kdt, B, T, N_cap, qI, qI_scale, w, KI, KI_scale, q_pos, scores, t,
                       topk_ws, topk_bytes, st));
+  return ok();
+}
+
+csa_status csa_index_topk_bf16(const csa_params* p, csa_dtype kdt, int32_t B, int32_t T,
+                               int64_t N_cap, const void* qI, const void* qI_scale,
+                               const float* w, const void* KI, const void* KI_scale,
+                               const int64_t* q_pos, int32_t* out_idx, void* out_scores16,
+                               void* ws, size_t ws_bytes, void* stream) {
+  TRY(check_index_args(p, kdt, B, T, N_cap, qI, qI_scale, w, KI, KI_scale, q_pos));
+  TRY(check_topk(p));
+  if ((int64_t)B * T == 0) return ok();
+  REQUIRE_PTR(out_idx);
+  OPTIONAL_PTR(out_scores16);
+  {
+    auto ia = make_index(p, kdt, B, T, N_cap, qI, qI_scale, w, KI, KI_scale, q_pos, nullptr);
+    if (N_cap > 0 && !csa::index_bf16_tc_supported(ia))
+      return fail(CSA_ERR_UNSUPPORTED,
+                  "BF16 index scores come from the tensor-core FP8 / bf16 indexer (64 heads of "
+                  "128, N_cap a multiple of 128)");
+  }
+  const size_t need = csa_workspace_size(p, CSA_WS_INDEX_TOPK_BF16, kdt, B, T, N_cap);
+  if (ws == nullptr || ws_bytes < need || !aligned16(ws))
+    return fail(CSA_ERR_WORKSPACE, "index+top-k (bf16 scores) needs %zu workspace bytes", need);
+  char* base = static_cast<char*>(ws);
+  const size_t sb = round_up((size_t)B * T * (size_t)N_cap * 2);
+  void* s16 = out_scores16 ? out_scores16 : base;
+  csa::TopkArgs t{};
+  t.B = B; t.T = T; t.m = p->m; t.k = p->topk; t.n_cap = N_cap; t.scores = nullptr;
+  t.scores16 = s16; t.q_pos = q_pos; t.out_idx = out_idx;
+  TRY(index_then_topk(p, kdt, B, T, N_cap, qI, qI_scale, w, KI, KI_scale, q_pos, nullptr, t,
+                      base + sb, need - sb, (cudaStream_t)stream, s16));
   return ok();
 }
 

@@ -50,6 +50,12 @@ __device__ __forceinline__ float e8m0_to_f32(uint32_t b) {
   return __uint_as_float(b << 23);
 }
 
+// An index score of either storage type, widened to fp32 (bf16 -> fp32 is exact).
+__device__ __forceinline__ float ld_score(const float* p, int64_t i) { return p[i]; }
+__device__ __forceinline__ float ld_score(const __nv_bfloat16* p, int64_t i) {
+  return __bfloat162float(p[i]);
+}
+
 // Order-preserving map of a float to uint32 (larger float -> larger key). -0 maps like +0.
 __device__ __forceinline__ uint32_t float_key(float f) {
   uint32_t u = __float_as_uint(f + 0.0f);

@@ -82,6 +82,7 @@ struct Bf16IdxParams {
   const float* key_scale;  // fp8: [B * n_cap] row scales; bf16: nullptr
   float* scores;
   int* hist;  // optional [Q][4096]
+  __nv_bfloat16* scores16;  // kB16: scores rounded to bf16 (the selector reads these)
 };
 
 template <bool kHist>
@@ -139,7 +140,7 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t v) {
   return *reinterpret_cast<const uint32_t*>(&b);
 }
 
-template <bool kFp8, int G>
+template <bool kFp8, int G, bool kB16>
 __global__ void __launch_bounds__(kThreads, 1)
     k_index_bf16_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                     Bf16IdxParams p) {
@@ -439,8 +440,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         float sc = (part[0] + part[1]) + (part[2] + part[3]);
         if (kFp8) sc *= scale;
         if (s < S.nvis[q]) {
-          p.scores[(size_t)q * p.n_cap + s] = sc;
-          if (hist) atomicAdd(&S.hist[float_key(sc) >> 20], 1);
+          if constexpr (kB16) {  // BF16 index scores: round once, select on the rounded value
+            const __nv_bfloat16 r = __float2bfloat16_rn(sc);
+            p.scores16[(size_t)q * p.n_cap + s] = r;
+            if (hist) atomicAdd(&S.hist[float_key(__bfloat162float(r)) >> 20], 1);
+          } else {
+            p.scores[(size_t)q * p.n_cap + s] = sc;
+            if (hist) atomicAdd(&S.hist[float_key(sc) >> 20], 1);
+          }
         }
       }
     }
@@ -513,14 +520,23 @@ size_t smem_bytes() {
          (kFp8 ? (size_t)kStg * kStgBytes : 0) + sizeof(Smem<C::kHist>);
 }
 
-template <bool kFp8, int G>
+template <bool kFp8, int G, bool kB16>
 cudaError_t launch_variant(const CUtensorMap& mk, const CUtensorMap& mq, const Bf16IdxParams& p,
                            int grid, cudaStream_t st) {
   const size_t smem = smem_bytes<kFp8, G>();
-  cudaError_t e = cudaFuncSetAttribute(k_index_bf16_tc<kFp8, G>,
+  cudaError_t e = cudaFuncSetAttribute(k_index_bf16_tc<kFp8, G, kB16>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch(true, k_index_bf16_tc<kFp8, G>, dim3(grid), dim3(kThreads), smem, st, mk, mq, p);
+  return launch(true, k_index_bf16_tc<kFp8, G, kB16>, dim3(grid), dim3(kThreads), smem, st, mk,
+                mq, p);
+}
+
+template <bool kB16>
+cudaError_t launch_one(bool fp8, bool grp, const CUtensorMap& mk, const CUtensorMap& mq,
+                       const Bf16IdxParams& p, int grid, cudaStream_t st) {
+  return fp8   ? launch_variant<true, 1, kB16>(mk, mq, p, grid, st)
+         : grp ? launch_variant<false, 4, kB16>(mk, mq, p, grid, st)
+               : launch_variant<false, 1, kB16>(mk, mq, p, grid, st);
 }
 
 }  // namespace
@@ -553,15 +569,16 @@ cudaError_t launch_index_bf16_tc(const IndexArgs& a, cudaStream_t st) {
       e = cudaErrorInvalidValue;
       break;
     }
+    const bool b16 = a.scores16 != nullptr;
     Bf16IdxParams p{Q, a.T, a.m, q0, a.n_cap, a.q_pos + q0, a.w + (size_t)q0 * kHeads,
                     fp8 ? static_cast<const float*>(a.KI_scale) : nullptr,
-                    a.scores + (size_t)q0 * a.n_cap,
-                    a.hist ? a.hist + (size_t)q0 * kBins : nullptr};
+                    b16 ? nullptr : a.scores + (size_t)q0 * a.n_cap,
+                    a.hist ? a.hist + (size_t)q0 * kBins : nullptr,
+                    b16 ? static_cast<__nv_bfloat16*>(a.scores16) + (size_t)q0 * a.n_cap : nullptr};
     const int64_t tiles_max = (int64_t)Q * (a.n_cap / kTileKeys);
     const int grid = (int)(tiles_max < num_sms() ? (tiles_max > 0 ? tiles_max : 1) : num_sms());
-    e = fp8   ? launch_variant<true, 1>(mk, mq, p, grid, st)
-        : grp ? launch_variant<false, 4>(mk, mq, p, grid, st)
-              : launch_variant<false, 1>(mk, mq, p, grid, st);
+    e = b16 ? launch_one<true>(fp8, grp, mk, mq, p, grid, st)
+            : launch_one<false>(fp8, grp, mk, mq, p, grid, st);
   }
   timing_after(st);
   return e;

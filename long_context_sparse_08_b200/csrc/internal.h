@@ -62,6 +62,7 @@ struct IndexArgs {
   const int64_t* q_pos;
   float* scores;  // [B, T, n_cap]
   int* hist;      // optional [B*T][4096] histogram of the scores' top 12 key bits (zeroed)
+  void* scores16;  // non-null: the scores are rounded to bf16 and stored here instead
 };
 // *hist_done: whether the launched kernel also filled a.hist
 cudaError_t launch_index_scores(const IndexArgs& a, cudaStream_t st, bool* hist_done = nullptr);
@@ -90,6 +91,7 @@ struct TopkArgs {
   int B, T, m, k;
   int64_t n_cap;
   const float* scores;
+  const void* scores16;  // non-null: bf16 scores [B, T, n_cap] in place of `scores`
   const int64_t* q_pos;
   int32_t* out_idx;
   QhatJob qj;
@@ -103,6 +105,7 @@ struct TopkDecodeArgs {
   int Q, m, k, nslice;
   int64_t n_cap;
   const float* scores;
+  const void* scores16;  // non-null: bf16 scores in place of `scores`
   const int64_t* q_pos;
   int32_t* out_idx;
   int* hist;          // [Q][4096]

@@ -67,6 +67,7 @@ __device__ void bitonic_sort(uint64_t* arr, int P) {
   }
 }
 
+template <typename TS>
 __global__ void __launch_bounds__(kThreads) k_topk_rows(TopkArgs a) {
   __shared__ uint64_t pairs[kMaxTopk];
   __shared__ int hist[256];
@@ -81,7 +82,8 @@ __global__ void __launch_bounds__(kThreads) k_topk_rows(TopkArgs a) {
     __syncthreads();
   }
   const int64_t n = t < 0 ? 0 : (t / a.m < a.n_cap ? t / a.m : a.n_cap);
-  const float* sc = a.scores + (size_t)bt * a.n_cap;
+  const TS* sc = (sizeof(TS) == 4 ? static_cast<const TS*>(static_cast<const void*>(a.scores))
+                                  : static_cast<const TS*>(a.scores16)) + (size_t)bt * a.n_cap;
   int32_t* out = a.out_idx + (size_t)bt * a.k;
   const int k = a.k;
   int P = 1;
@@ -89,7 +91,7 @@ __global__ void __launch_bounds__(kThreads) k_topk_rows(TopkArgs a) {
 
   if (n <= k) {  // everything visible is selected; just order it
     for (int i = threadIdx.x; i < P; i += blockDim.x)
-      pairs[i] = i < n ? pack_desc(float_key(sc[i]), (uint32_t)i) : ~0ull;
+      pairs[i] = i < n ? pack_desc(float_key(ld_score(sc, i)), (uint32_t)i) : ~0ull;
     __syncthreads();
     bitonic_sort(pairs, P);
     for (int i = threadIdx.x; i < k; i += blockDim.x)
@@ -104,7 +106,7 @@ __global__ void __launch_bounds__(kThreads) k_topk_rows(TopkArgs a) {
     for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
     __syncthreads();
     for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
-      const uint32_t u = float_key(sc[i]);
+      const uint32_t u = float_key(ld_score(sc, i));
       if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 0xff], 1);
     }
     __syncthreads();
@@ -148,7 +150,7 @@ __global__ void __launch_bounds__(kThreads) k_topk_rows(TopkArgs a) {
     const int lane = threadIdx.x & 31;
     for (int64_t base = 0; base < n; base += blockDim.x) {
       const int64_t i = base + threadIdx.x;
-      const uint32_t u = i < n ? float_key(sc[i]) : 0u;
+      const uint32_t u = i < n ? float_key(ld_score(sc, i)) : 0u;
       const bool take = i < n && u >= T;
       const unsigned bal = __ballot_sync(0xffffffffu, take);
       if (bal == 0) continue;
@@ -175,7 +177,7 @@ __global__ void __launch_bounds__(kThreads) k_topk_rows(TopkArgs a) {
   int run_gt = 0, run_eq = 0;
   for (int64_t base = 0; base < n; base += blockDim.x) {
     const int64_t i = base + threadIdx.x;
-    const uint32_t u = i < n ? float_key(sc[i]) : 0u;
+    const uint32_t u = i < n ? float_key(ld_score(sc, i)) : 0u;
     const bool gt = i < n && u > T, eq = i < n && u == T;
     int tot_gt, tot_eq;
     const int o_gt = block_excl_scan(gt, wsum, &tot_gt);
@@ -205,7 +207,10 @@ cudaError_t launch_topk(const TopkArgs& a, void* ws, size_t ws_bytes, cudaStream
       return cudaErrorInvalidValue;
     return launch_topk_decode(topk_decode_args(a, ws), hist_ready, st);
   }
-  launch(false, k_topk_rows, dim3(a.B * a.T), dim3(kThreads), 0, st, a);
+  if (a.scores16 != nullptr)
+    launch(false, k_topk_rows<__nv_bfloat16>, dim3(a.B * a.T), dim3(kThreads), 0, st, a);
+  else
+    launch(false, k_topk_rows<float>, dim3(a.B * a.T), dim3(kThreads), 0, st, a);
   return cudaGetLastError();
 }
 

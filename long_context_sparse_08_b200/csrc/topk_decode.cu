@@ -103,6 +103,15 @@ __device__ uint64_t* merge_sort(uint64_t* arr, uint64_t* tmp) {
   return src;
 }
 
+// Row q of the scores, in their storage type (fp32, or bf16 for the selector on BF16 index
+// scores).
+template <typename TS>
+__device__ __forceinline__ const TS* score_row(const TopkDecodeArgs& a, int q) {
+  if constexpr (sizeof(TS) == 4) return a.scores + (size_t)q * a.n_cap;
+  else return static_cast<const TS*>(a.scores16) + (size_t)q * a.n_cap;
+}
+
+template <typename TS>
 __global__ void __launch_bounds__(kFThreads) k_topk_hist(TopkDecodeArgs a) {
   __shared__ int h[kBins];
   const int q = blockIdx.y;
@@ -110,9 +119,9 @@ __global__ void __launch_bounds__(kFThreads) k_topk_hist(TopkDecodeArgs a) {
   for (int i = threadIdx.x; i < kBins; i += blockDim.x) h[i] = 0;
   __syncthreads();
   const int64_t lo = n * blockIdx.x / gridDim.x, hi = n * (blockIdx.x + 1) / gridDim.x;
-  const float* sc = a.scores + (size_t)q * a.n_cap;
+  const TS* sc = score_row<TS>(a, q);
   for (int64_t i = lo + threadIdx.x; i < hi; i += blockDim.x)
-    atomicAdd(&h[float_key(sc[i]) >> 20], 1);
+    atomicAdd(&h[float_key(ld_score(sc, i)) >> 20], 1);
   __syncthreads();
   for (int i = threadIdx.x; i < kBins; i += blockDim.x)
     if (h[i]) atomicAdd(&a.hist[(size_t)q * kBins + i], h[i]);
@@ -167,6 +176,7 @@ __global__ void __launch_bounds__(256) k_zero(int4* p0, int n0, int4* p1, int n1
   }
 }
 
+template <typename TS>
 __global__ void __launch_bounds__(kFThreads, 2) k_topk_filter(TopkDecodeArgs a) {
   __shared__ int wsum[2 * kWarps];
   __shared__ int s_bin, s_base_s, s_base_b;
@@ -188,13 +198,13 @@ __global__ void __launch_bounds__(kFThreads, 2) k_topk_filter(TopkDecodeArgs a) 
 
   // ---- this CTA's slice: first batch of loads in flight before the threshold is known ----
   const int64_t lo = n * blockIdx.x / nslice, hi = n * (blockIdx.x + 1) / nslice;
-  const float* sc = a.scores + (size_t)q * a.n_cap;
+  const TS* sc = score_row<TS>(a, q);
   constexpr int kBatch = 16;  // loads in flight per thread
   float f[kBatch];
 #pragma unroll
   for (int j = 0; j < kBatch; ++j) {
     const int64_t i = lo + j * kFThreads + tid;
-    f[j] = i < hi ? sc[i] : 0.f;
+    f[j] = i < hi ? ld_score(sc, i) : 0.f;
   }
 
   // ---- threshold bin: the bin holding the k-th largest key ----
@@ -233,7 +243,7 @@ __global__ void __launch_bounds__(kFThreads, 2) k_topk_filter(TopkDecodeArgs a) 
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) {
         const int64_t i = base + j * kFThreads + tid;
-        f[j] = i < hi ? sc[i] : 0.f;
+        f[j] = i < hi ? ld_score(sc, i) : 0.f;
       }
     }
     uint32_t fs = 0, fb = 0;
@@ -440,6 +450,7 @@ TopkDecodeArgs topk_decode_args(const TopkArgs& t, void* ws) {
   const size_t Q = (size_t)t.B * t.T;
   char* p = static_cast<char*>(ws);
   a.Q = (int)Q; a.m = t.m; a.k = t.k; a.n_cap = t.n_cap; a.scores = t.scores;
+  a.scores16 = t.scores16;
   a.q_pos = t.q_pos; a.out_idx = t.out_idx; a.qj = t.qj;
   a.hist = reinterpret_cast<int*>(p);
   p += rup(Q * kBins * 4);
@@ -472,10 +483,16 @@ cudaError_t launch_topk_decode(TopkDecodeArgs a, bool hist_ready, cudaStream_t s
   if (!hist_ready) {
     const cudaError_t e = topk_decode_clear(a, st);
     if (e != cudaSuccess) return e;
-    const cudaError_t eh = launch(false, k_topk_hist, dim3(slices, a.Q), dim3(kFThreads), 0, st, a);
+    const cudaError_t eh =
+        a.scores16 ? launch(false, k_topk_hist<__nv_bfloat16>, dim3(slices, a.Q), dim3(kFThreads),
+                            0, st, a)
+                   : launch(false, k_topk_hist<float>, dim3(slices, a.Q), dim3(kFThreads), 0, st, a);
     if (eh != cudaSuccess) return eh;
   }
-  cudaError_t e = launch(true, k_topk_filter, dim3(slices, a.Q), dim3(kFThreads), 0, st, a);
+  cudaError_t e =
+      a.scores16
+          ? launch(true, k_topk_filter<__nv_bfloat16>, dim3(slices, a.Q), dim3(kFThreads), 0, st, a)
+          : launch(true, k_topk_filter<float>, dim3(slices, a.Q), dim3(kFThreads), 0, st, a);
   if (e != cudaSuccess) return e;
   // enough CTAs for the sure list (< k) and the boundary list (<= kRankBnd) apart
   const int rank_ctas = (a.k + kRankPerCta - 1) / kRankPerCta + kRankBnd / kRankPerCta;
