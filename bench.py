@@ -479,9 +479,11 @@ def _time_calls(fn, n_rep, warmup, steps):
 
 def run_part(args, W):
     """One JSON line for an extension kernel family on the workload's shape:
-    out_proj      grouped output projection of the batch's queries (HBM roofline);
-    state_append  one decode token per request into the KV and indexer-key state caches;
-    kv_layouts    the attention alone over bf16, mixed-precision and paged caches."""
+    out_proj          grouped output projection of the batch's queries (HBM roofline);
+    out_proj_prefill  its tensor-core form on a prefill chunk's queries (tensor roofline);
+    state_append      one decode token per request into the KV and indexer-key state caches;
+    kv_layouts        the attention alone over bf16, mixed-precision and paged caches;
+    bf16_scores       index + top-k with fp32 and with BF16 scores (FP8 / bf16 keys)."""
     import torch
     import long_context_sparse_08_b200 as csa
     from long_context_sparse_08_b200 import runner as R
@@ -626,6 +628,57 @@ def run_part(args, W):
                                          "page_rows": pr},
                     roofline={"bound": "latency (see the attention in DESIGN)", "peak": hbm,
                               "peak_source": peak_src, "unit": "GB/s"})
+    elif args.part == "bf16_scores":
+        # index + top-k with fp32 scores (csa_index_topk) and with BF16 scores
+        # (csa_index_topk_bf16) on the workload's keys (FP8 / bf16 tensor-core indexer)
+        inp = W.make_inputs(s)
+        dev = R.upload(inp, s)
+        p = R.params_for(s)
+        kdt = csa.DTYPES[s.idx]
+        B, T, N = s.B, s.T, s.n_cap
+        out_idx = torch.empty((B, T, s.topk), dtype=torch.int32, device="cuda")
+        res = {}
+        for name, entry in (("fp32", csa.CSA_WS_INDEX_TOPK), ("bf16", csa.CSA_WS_INDEX_TOPK_BF16)):
+            need = csa.workspace_size(p, entry, kdt, B, T, N)
+            ws = torch.empty((need,), dtype=torch.uint8, device="cuda")
+            if name == "fp32":
+                fn = lambda i, ws=ws, need=need: csa.csa_index_topk(  # noqa: E731
+                    p, kdt, B, T, N, dev["qI"], dev.get("qI_scale"), dev["w"], dev["KI"],
+                    dev.get("KI_scale"), dev["q_pos"], out_idx, None, ws, need)
+            else:
+                fn = lambda i, ws=ws, need=need: csa.csa_index_topk_bf16(  # noqa: E731
+                    p, kdt, B, T, N, dev["qI"], dev.get("qI_scale"), dev["w"], dev["KI"],
+                    dev.get("KI_scale"), dev["q_pos"], out_idx, None, ws, need)
+            ms = _time_calls(fn, 1, args.warmup, args.steps)
+            res[name] = {"ms_per_call": round(ms, 5),
+                         "score_bytes_per_call": B * T * N * (4 if name == "fp32" else 2)}
+        line.update(metric="index + top-k calls/s by score precision",
+                    value=round(1e3 / res["bf16"]["ms_per_call"], 2), unit="calls/s (bf16)",
+                    precisions=res, config={"B": B, "T": T, "n_cap": N, "k": s.topk,
+                                            "keys": s.idx},
+                    roofline={"bound": "hbm (key stream)", "peak": hbm, "peak_source": peak_src,
+                              "unit": "GB/s"})
+    elif args.part == "out_proj_prefill":
+        # the tensor-core form on a prefill chunk: Flash shapes, the workload's queries
+        Q, (H, c, g, d_g, d) = max(s.B * s.T, 128), (64, 512, 8, 1024, 4096)
+        inp = W.make_out_proj_inputs(Q=Q, H=H, c=c, g=g, d_g=d_g, d=d, seed=12)
+        p = csa.make_params(c=c, n_heads=H)
+        dv = {k: torch.from_numpy(v.view(np.int16)).cuda() for k, v in inp.items()}
+        need = csa.grouped_out_proj_workspace_size(p, Q, g, d_g, d)
+        ws = torch.empty((need,), dtype=torch.uint8, device="cuda")
+        out = torch.empty((Q, d), dtype=torch.int16, device="cuda")
+        fn = lambda i: csa.csa_grouped_out_proj(p, Q, g, d_g, d, dv["o"], dv["w_grp"],  # noqa
+                                                dv["w_out"], out, ws, need)
+        ms = _time_calls(fn, 1, args.warmup, args.steps)
+        flops = 2.0 * Q * (c * H * d_g + g * d_g * d)
+        tf = flops / (ms / 1e3) / 1e12
+        peak_tf = float(peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"]))
+        line.update(metric="grouped output projection TFLOP/s (prefill)", value=round(tf, 1),
+                    unit="TFLOP/s", ms_per_call=round(ms, 5),
+                    config={"Q": Q, "H": H, "c": c, "g": g, "d_g": d_g, "d": d},
+                    roofline={"bound": "tensor", "achieved": round(tf, 1), "peak": peak_tf,
+                              "peak_source": peak_src, "unit": "TFLOP/s",
+                              "frac": round(tf / peak_tf, 4), "flops_per_call": flops})
     line["gpu_launches"] = int(csa.kernel_launches() - before)
     line["clocks"] = clocks.stop()
     line["device_error"] = csa.device_error()
@@ -633,7 +686,7 @@ def run_part(args, W):
     return 0
 
 
-PARTS = {"out_proj", "state_append", "kv_layouts"}
+PARTS = {"out_proj", "state_append", "kv_layouts", "bf16_scores", "out_proj_prefill"}
 
 
 def main():
