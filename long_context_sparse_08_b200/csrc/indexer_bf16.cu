@@ -29,9 +29,9 @@
 // Tiles are split evenly over the CTAs; ragged visibility is handled by masking the stores.
 #include <cudaTypedefs.h>
 
-#include <mutex>
 
 #include "common.cuh"
+#include "host_util.cuh"
 #include "internal.h"
 #include "tc.cuh"
 
@@ -462,23 +462,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---- host: tensor maps ----
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
-}
-
 // bf16 rows of 128 values, box = 64 values (one 128-byte swizzle atom) x box_rows
 bool make_map_bf16_rows(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows) {
-  auto fn = encode_fn();
+  auto fn = tensor_map_encoder();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)kDim, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)kDim * 2};
@@ -491,7 +477,7 @@ bool make_map_bf16_rows(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t
 
 // e4m3 rows of 128 bytes, box = one 128-key tile, no swizzle (the converters read it)
 bool make_map_fp8_rows(CUtensorMap* m, const void* ptr, uint64_t rows) {
-  auto fn = encode_fn();
+  auto fn = tensor_map_encoder();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)kDim, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)kDim};
@@ -500,17 +486,6 @@ bool make_map_fp8_rows(CUtensorMap* m, const void* ptr, uint64_t rows) {
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
 }
 
 template <bool kFp8, int G>
@@ -576,7 +551,7 @@ cudaError_t launch_index_bf16_tc(const IndexArgs& a, cudaStream_t st) {
                     a.hist ? a.hist + (size_t)q0 * kBins : nullptr,
                     b16 ? static_cast<__nv_bfloat16*>(a.scores16) + (size_t)q0 * a.n_cap : nullptr};
     const int64_t tiles_max = (int64_t)Q * (a.n_cap / kTileKeys);
-    const int grid = (int)(tiles_max < num_sms() ? (tiles_max > 0 ? tiles_max : 1) : num_sms());
+    const int grid = (int)(tiles_max < device_sm_count() ? (tiles_max > 0 ? tiles_max : 1) : device_sm_count());
     e = b16 ? launch_one<true>(fp8, grp, mk, mq, p, grid, st)
             : launch_one<false>(fp8, grp, mk, mq, p, grid, st);
   }

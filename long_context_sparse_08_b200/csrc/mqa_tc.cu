@@ -35,9 +35,9 @@
 #include <cudaTypedefs.h>
 
 #include <cstring>
-#include <mutex>
 
 #include "common.cuh"
+#include "host_util.cuh"
 #include "internal.h"
 #include "tc.cuh"
 
@@ -784,23 +784,9 @@ __global__ void __launch_bounds__(256) k_mqa_combine(MqaTcParams P) {
   *reinterpret_cast<__nv_bfloat162*>(out) = __floats2bfloat162_rn(y0, y1);
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
-}
-
 // bf16 rows of c = 512 values; box = one 128B swizzle atom (64 values) x 128 rows
 bool make_map_rows(CUtensorMap* m, const void* ptr, int64_t rows) {
-  auto fn = encode_fn();
+  auto fn = tensor_map_encoder();
   if (!fn || ptr == nullptr || rows < kRows || rows >= (1ll << 31)) return false;
   cuuint64_t dims[2] = {(cuuint64_t)kC, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)kC * 2};
@@ -811,24 +797,11 @@ bool make_map_rows(CUtensorMap* m, const void* ptr, int64_t rows) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
-      cudaGetLastError();
-      n = 148;
-    }
-  }
-  return n;
-}
-
 int choose_nsplit(const MqaArgs& a) {
   const int64_t streams = (int64_t)a.B * a.T * (a.H / kHg);
   const int64_t rows_max = (a.k > 0 ? a.k : a.n_cap) + a.n_win;
   const int64_t chunks_max = (rows_max + kRows - 1) / kRows;
-  int64_t ns = sm_count() / (streams > 0 ? streams : 1);
+  int64_t ns = device_sm_count() / (streams > 0 ? streams : 1);
   if (ns < 1) ns = 1;
   if (ns > chunks_max) ns = chunks_max > 0 ? chunks_max : 1;
   if (ns > 32) ns = 32;

@@ -9,6 +9,7 @@
 // separate CTAs, about two waves of the SMs; the partial sums are added in a fixed order, so
 // results do not depend on the schedule.
 #include "common.cuh"
+#include "host_util.cuh"
 #include "internal.h"
 #include "out_proj.cuh"
 
@@ -111,19 +112,6 @@ __global__ void __launch_bounds__(256) k_out_proj_reduce(OutProjArgs a) {
   }
 }
 
-int sm_count_proj() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
-      cudaGetLastError();
-      n = 148;
-    }
-  }
-  return n;
-}
-
 template <int QM>
 cudaError_t launch_splits(const OutProjArgs& a, cudaStream_t st) {
   const Geom& G = a.G;
@@ -131,7 +119,7 @@ cudaError_t launch_splits(const OutProjArgs& a, cudaStream_t st) {
   const size_t smem2 = (size_t)QM * G.ks2 * sizeof(float);
   const dim3 grid1(G.g * proj::ceil_div(G.d_g, proj::kColsPerCta), G.S1);
   const dim3 grid2(proj::ceil_div(G.d, proj::kColsPerCta), G.S2);
-  const int red_blocks = 2 * sm_count_proj();
+  const int red_blocks = 2 * device_sm_count();
   cudaError_t e = launch(false, k_out_proj_split<QM, false>, grid1, dim3(128), smem1, st, a);
   if (e == cudaSuccess)
     e = launch(false, k_out_proj_reduce<false>, dim3(red_blocks), dim3(256), 0, st, a);
@@ -145,7 +133,7 @@ cudaError_t launch_splits(const OutProjArgs& a, cudaStream_t st) {
 }  // namespace
 
 proj::Geom out_proj_geom(int Q, int H, int c, int g, int d_g, int d) {
-  return proj::make_geom(Q, H, c, g, d_g, d, sm_count_proj());
+  return proj::make_geom(Q, H, c, g, d_g, d, device_sm_count());
 }
 
 size_t out_proj_workspace_bytes(const proj::Geom& G) {

@@ -23,9 +23,9 @@
 #include <cudaTypedefs.h>
 
 #include <cstring>
-#include <mutex>
 
 #include "common.cuh"
+#include "host_util.cuh"
 #include "internal.h"
 #include "out_proj.cuh"
 #include "tc.cuh"
@@ -200,23 +200,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
-}
-
 // bf16 matrix [rows, cols] (row-major), box = 64 columns (128 B, swizzled) x box_rows
 bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-  auto fn = encode_fn();
+  auto fn = tensor_map_encoder();
   if (!fn || ptr == nullptr || (cols * 2) % 16 != 0 || rows < box_rows || cols < 64) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
@@ -227,23 +213,10 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uin
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int sm_count_tc() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
-      cudaGetLastError();
-      n = 148;
-    }
-  }
-  return n;
-}
-
 cudaError_t gemm(const CUtensorMap& ma, const CUtensorMap& mb, const GemmParams& p,
                  cudaStream_t st) {
   const int tiles = p.batches * ((p.N + kBN - 1) / kBN) * ((p.M + kBM - 1) / kBM);
-  const int grid = tiles < sm_count_tc() ? tiles : sm_count_tc();
+  const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
   const size_t smem = 1024 + (size_t)kStages * kStageBytes + sizeof(SmemG);
   cudaError_t e = cudaFuncSetAttribute(k_out_proj_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
