@@ -148,7 +148,7 @@ csa_status csa_compress(const csa_params* p, csa_dtype io, int32_t B, int64_t n_
  * or, for a request resumed after a prefill, by the caller writing those raw rows into their
  * slots. Requests whose entry's logical page is >= max_pages, whose page id is outside
  * [0, n_pages), or whose position is negative are skipped and leave a device error code
- * (301 position, 302 page slot, 303 page id) for csa_device_error(). The pages use
+ * (321 position, 322 page slot, 323 page id) for csa_device_error(). The pages use
  * page_rows = 128 / m (a multiple of it for MXFP4 keys); with page_table[b, k] =
  * b * max_pages + k they are the contiguous cache [B, N_cap = page_rows * max_pages, ...]
  * that the attention and indexer calls read.
@@ -320,6 +320,21 @@ csa_status hca_dense_mqa_paged(const csa_params* p, int32_t B, int32_t T, const 
                                const void* q_rms_w, void* out, void* ws, size_t ws_bytes,
                                void* stream);
 
+/*
+ * Stages 2 + 3 over indexer keys kept in a page pool (the compressed indexer keys of the
+ * state cache, [P1''] 二(六)): as csa_index_topk with bf16 queries qI [B, T, 64, 128], the keys
+ * of request b read through the page table. keys->fmt is CSA_BF16 (pages [n_pages,
+ * page_rows, 128]) or CSA_FP8_E4M3_ROWSCALE (e4m3 pages and scales [n_pages, page_rows]);
+ * page_rows is a multiple of 128; N_cap = page_rows * max_pages. bf16_scores = 1 selects on
+ * BF16 index scores as csa_index_topk_bf16 does. out_scores (fp32, or bf16 with bf16_scores)
+ * may be NULL. A key whose page id lies outside the pool reads row 0 and leaves device error
+ * code 309. Workspace: csa_workspace_size() with CSA_WS_INDEX_TOPK or CSA_WS_INDEX_TOPK_BF16.
+ */
+csa_status csa_index_topk_paged(const csa_params* p, int32_t B, int32_t T,
+                                const csa_paged_kv* keys, const void* qI, const float* w,
+                                const int64_t* q_pos, int32_t bf16_scores, int32_t* out_idx,
+                                void* out_scores, void* ws, size_t ws_bytes, void* stream);
+
 /* Inputs of the fused CSA layer call. Pointers as in the stage calls above. */
 typedef struct {
   /* optional compression of a new chunk into kv_cache (skipped when Ca == NULL) */
@@ -400,8 +415,10 @@ void csa_set_index_timing_events(void* const* before, void* const* after, int32_
  * Error word of the tensor-core kernels: every wait inside them is bounded (about a second);
  * a wait that runs out stores a nonzero code (the first one wins) and the kernel returns
  * early instead of hanging. csa_state_append also leaves a code for a request it skipped.
- * Writes the code to *code (0 = none) and clears it. Synchronises the device. Returns
- * CSA_ERR_CUDA if the copy fails.
+ * Codes by kernel family: 101-106 MXFP4 indexer, 201-205 attention (205: a page id outside
+ * the pool), 301-309 FP8 / bf16 indexer (309: a page id outside the pool), 321-323 state
+ * append, 401-405 prefill output projection. Writes the code to *code (0 = none) and clears
+ * it. Synchronises the device. Returns CSA_ERR_CUDA if the copy fails.
  */
 csa_status csa_device_error(int32_t* code);
 

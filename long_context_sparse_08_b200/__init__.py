@@ -27,6 +27,7 @@ EXPORTS = (
     "csa_topk_noalloc", "csa_kernel_launches", "csa_state_append", "csa_sparse_mqa_mixed_kv",
     "hca_dense_mqa_mixed_kv", "csa_grouped_out_proj", "csa_grouped_out_proj_workspace_size",
     "csa_sparse_mqa_paged", "hca_dense_mqa_paged", "csa_index_topk_bf16",
+    "csa_index_topk_paged",
 )
 # size of the library-owned scratch array behind csa_topk_noalloc (bytes, per device)
 TOPK_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -99,6 +100,8 @@ _SIGS = {
     "hca_dense_mqa_paged": [_PP, _I32, _I32, _VP, _VP, ctypes.POINTER(CsaPagedKv), _VP, _I64,
                             _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "csa_index_topk_bf16": [_PP, ctypes.c_int, _I32, _I32, _I64] + [_VP] * 9 + [_SZ, _VP],
+    "csa_index_topk_paged": [_PP, _I32, _I32, ctypes.POINTER(CsaPagedKv), _VP, _VP, _VP, _I32,
+                             _VP, _VP, _VP, _SZ, _VP],
     "csa_grouped_out_proj": [_PP, _I32, _I32, _I32, _I32, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "csa_grouped_out_proj_workspace_size": [_PP, _I32, _I32, _I32, _I32],
     "csa_sparse_mqa_mixed_kv": [_PP, _I32, _I32, _VP, _VP, _VP, _VP, _I64, _VP, _VP, _I64, _VP,
@@ -310,6 +313,14 @@ def hca_dense_mqa_paged(p, B, T, q, q_pos, kv: CsaPagedKv, win_kv, L_raw, win_po
                                   _ptr(win_kv), L_raw, _ptr(win_pos0), _ptr(sink),
                                   _ptr(q_rms_w), _ptr(out), _ptr(ws), ws_bytes, _stream(stream))
     _check("hca_dense_mqa_paged", s)
+
+
+def csa_index_topk_paged(p, B, T, keys: CsaPagedKv, qI, w, q_pos, bf16_scores, out_idx,
+                         out_scores, ws, ws_bytes, stream=None):
+    s = lib().csa_index_topk_paged(ctypes.byref(p), B, T, ctypes.byref(keys), _ptr(qI), _ptr(w),
+                                   _ptr(q_pos), int(bf16_scores), _ptr(out_idx), _ptr(out_scores),
+                                   _ptr(ws), ws_bytes, _stream(stream))
+    _check("csa_index_topk_paged", s)
 
 
 def grouped_out_proj_workspace_size(p, Q, g, d_g, d) -> int:

@@ -206,12 +206,19 @@ csa_status index_then_topk(const csa_params* p, csa_dtype kdt, int32_t B, int32_
                            int64_t N_cap, const void* qI, const void* qI_scale, const float* w,
                            const void* KI, const void* KI_scale, const int64_t* q_pos,
                            float* scores, const csa::TopkArgs& t, void* topk_ws,
-                           size_t topk_bytes, cudaStream_t st, void* scores16 = nullptr) {
+                           size_t topk_bytes, cudaStream_t st, void* scores16 = nullptr,
+                           const csa_paged_kv* key_pages = nullptr) {
   bool hist_done = false;
   const bool decode = csa::topk_decode_path(B, T, N_cap, p->topk);
   if (N_cap > 0) {
     auto ia = make_index(p, kdt, B, T, N_cap, qI, qI_scale, w, KI, KI_scale, q_pos, scores);
     ia.scores16 = scores16;
+    if (key_pages != nullptr) {
+      ia.page_table = key_pages->page_table;
+      ia.page_rows = key_pages->page_rows;
+      ia.max_pages = key_pages->max_pages;
+      ia.n_pages = key_pages->n_pages;
+    }
     if (decode) {
       const csa::TopkDecodeArgs da = csa::topk_decode_args(t, topk_ws);
       TRY(cuda_status(csa::topk_decode_clear(da, st), "top-k clear"));
@@ -564,6 +571,57 @@ csa_status csa_index_topk_bf16(const csa_params* p, csa_dtype kdt, int32_t B, in
   t.scores16 = s16; t.q_pos = q_pos; t.out_idx = out_idx;
   TRY(index_then_topk(p, kdt, B, T, N_cap, qI, qI_scale, w, KI, KI_scale, q_pos, nullptr, t,
                       base + sb, need - sb, (cudaStream_t)stream, s16));
+  return ok();
+}
+
+csa_status csa_index_topk_paged(const csa_params* p, int32_t B, int32_t T,
+                                const csa_paged_kv* keys, const void* qI, const float* w,
+                                const int64_t* q_pos, int32_t bf16_scores, int32_t* out_idx,
+                                void* out_scores, void* ws, size_t ws_bytes, void* stream) {
+  TRY(check_params(p));
+  TRY(check_topk(p));
+  REQUIRE(keys != nullptr, "paged key descriptor is NULL");
+  REQUIRE(keys->fmt == CSA_BF16 || keys->fmt == CSA_FP8_E4M3_ROWSCALE,
+          "paged indexer keys must be CSA_BF16 or CSA_FP8_E4M3_ROWSCALE");
+  REQUIRE(keys->n_pages >= 1 && keys->max_pages >= 1 && keys->page_rows >= 1,
+          "n_pages, page_rows and max_pages must be >= 1");
+  REQUIRE((int64_t)keys->page_rows * keys->max_pages <= INT32_MAX, "page_rows * max_pages too large");
+  REQUIRE(bf16_scores == 0 || bf16_scores == 1, "bf16_scores must be 0 or 1");
+  REQUIRE_PTR(keys->page_table);
+  const int64_t N_cap = (int64_t)keys->page_rows * keys->max_pages;
+  const csa_dtype kdt = keys->fmt;
+  TRY(check_index_args(p, kdt, B, T, N_cap, qI, nullptr, w, keys->pages, keys->scales, q_pos));
+  if ((int64_t)B * T == 0) return ok();
+  REQUIRE_PTR(out_idx);
+  OPTIONAL_PTR(out_scores);
+  {
+    auto ia = make_index(p, kdt, B, T, N_cap, qI, nullptr, w, keys->pages, keys->scales, q_pos,
+                         nullptr);
+    ia.page_table = keys->page_table;
+    ia.page_rows = keys->page_rows;
+    ia.max_pages = keys->max_pages;
+    ia.n_pages = keys->n_pages;
+    if (!csa::index_bf16_tc_supported(ia))
+      return fail(CSA_ERR_UNSUPPORTED,
+                  "paged keys are read by the tensor-core FP8 / bf16 indexer (64 heads of 128, "
+                  "page_rows a multiple of 128)");
+  }
+  const int entry = bf16_scores ? CSA_WS_INDEX_TOPK_BF16 : CSA_WS_INDEX_TOPK;
+  const size_t need = csa_workspace_size(p, entry, kdt, B, T, N_cap);
+  if (ws == nullptr || ws_bytes < need || !aligned16(ws))
+    return fail(CSA_ERR_WORKSPACE, "index+top-k (paged keys) needs %zu workspace bytes", need);
+  char* base = static_cast<char*>(ws);
+  const size_t sb = bf16_scores ? round_up((size_t)B * T * (size_t)N_cap * 2)
+                                : scores_bytes(B, T, N_cap);
+  void* sc = out_scores ? out_scores : base;
+  csa::TopkArgs t{};
+  t.B = B; t.T = T; t.m = p->m; t.k = p->topk; t.n_cap = N_cap; t.q_pos = q_pos;
+  t.out_idx = out_idx;
+  if (bf16_scores) t.scores16 = sc;
+  else t.scores = static_cast<float*>(sc);
+  TRY(index_then_topk(p, kdt, B, T, N_cap, qI, nullptr, w, keys->pages, keys->scales, q_pos,
+                      bf16_scores ? nullptr : static_cast<float*>(sc), t, base + sb, need - sb,
+                      (cudaStream_t)stream, bf16_scores ? sc : nullptr, keys));
   return ok();
 }
 

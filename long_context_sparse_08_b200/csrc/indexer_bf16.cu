@@ -55,7 +55,7 @@ constexpr int kAtomBytes = kTileKeys * 128;         // 16 KB
 constexpr int kQBytes = kHeads * kDim * 2;          // 16 KB per query: 2 atoms x 64 x 128 B
 
 enum { kErrStgFull = 301, kErrStgEmpty = 302, kErrOpFull = 303, kErrOpEmpty = 304,
-       kErrTFull = 305, kErrTEmpty = 306, kErrQFull = 307, kErrQEmpty = 308 };
+       kErrTFull = 305, kErrTEmpty = 306, kErrQFull = 307, kErrQEmpty = 308, kErrPageId = 309 };
 
 // G consecutive queries of one request share each key tile: N = 64 G per MMA.
 template <bool kFp8, int G>
@@ -83,7 +83,26 @@ struct Bf16IdxParams {
   float* scores;
   int* hist;  // optional [Q][4096]
   __nv_bfloat16* scores16;  // kB16: scores rounded to bf16 (the selector reads these)
+  const int32_t* page_table;  // kPaged: keys (and FP8 row scales) in a page pool
+  int page_rows, max_pages, n_pages;
 };
+
+// Row of key e of request b in the key rows the tensor map covers: contiguous [B, n_cap], or
+// (kPaged) the page pool through the page table. A page id outside the pool records an
+// error and reads row 0 (that tile's scores are then meaningless).
+template <bool kPaged>
+__device__ __forceinline__ int64_t key_row(const Bf16IdxParams& p, int b, int64_t e) {
+  if constexpr (kPaged) {
+    const int32_t pg = p.page_table[(size_t)b * p.max_pages + e / p.page_rows];
+    if (pg < 0 || pg >= p.n_pages) {
+      tc::set_error(kErrPageId);
+      return 0;
+    }
+    return (int64_t)pg * p.page_rows + e % p.page_rows;
+  } else {
+    return (int64_t)b * p.n_cap + e;
+  }
+}
 
 template <bool kHist>
 struct Smem {
@@ -140,7 +159,7 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t v) {
   return *reinterpret_cast<const uint32_t*>(&b);
 }
 
-template <bool kFp8, int G, bool kB16>
+template <bool kFp8, int G, bool kB16, bool kPaged>
 __global__ void __launch_bounds__(kThreads, 1)
     k_index_bf16_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                     Bf16IdxParams p) {
@@ -260,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int tile = u - S.prefix[g];
         const int b = (p.q0 + S.gfirst[g]) / p.T;
-        const int32_t row = (int32_t)(b * p.n_cap + (int64_t)tile * kTileKeys);
+        const int32_t row = (int32_t)key_row<kPaged>(p, b, (int64_t)tile * kTileKeys);
         if (kFp8) {
           const int s = k % kStg;
           ok = mbar_wait(&S.stg_empty[s], ((k / kStg) & 1) ^ 1, kErrStgEmpty);
@@ -410,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int s = tile * kTileKeys + 32 * quad + lane;
       const int b = (p.q0 + f) / p.T;
       // the fp8 row scale is loaded before the wait, so its latency hides behind the MMAs
-      const float scale = (kFp8 && s < S.nvis[f]) ? p.key_scale[(size_t)b * p.n_cap + s] : 1.f;
+      const float scale = (kFp8 && s < S.nvis[f]) ? p.key_scale[key_row<kPaged>(p, b, s)] : 1.f;
       const int a = k % C::kAccN;
       ok = group_all_ok<2, C::kEpiThreads>(
           mbar_wait(&S.tfull[a], (uint32_t)(k / C::kAccN) & 1, kErrTFull));
@@ -495,30 +514,34 @@ size_t smem_bytes() {
          (kFp8 ? (size_t)kStg * kStgBytes : 0) + sizeof(Smem<C::kHist>);
 }
 
-template <bool kFp8, int G, bool kB16>
+template <bool kFp8, int G, bool kB16, bool kPaged>
 cudaError_t launch_variant(const CUtensorMap& mk, const CUtensorMap& mq, const Bf16IdxParams& p,
                            int grid, cudaStream_t st) {
   const size_t smem = smem_bytes<kFp8, G>();
-  cudaError_t e = cudaFuncSetAttribute(k_index_bf16_tc<kFp8, G, kB16>,
+  cudaError_t e = cudaFuncSetAttribute(k_index_bf16_tc<kFp8, G, kB16, kPaged>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch(true, k_index_bf16_tc<kFp8, G, kB16>, dim3(grid), dim3(kThreads), smem, st, mk,
-                mq, p);
+  return launch(true, k_index_bf16_tc<kFp8, G, kB16, kPaged>, dim3(grid), dim3(kThreads), smem,
+                st, mk, mq, p);
 }
 
-template <bool kB16>
+template <bool kB16, bool kPaged>
 cudaError_t launch_one(bool fp8, bool grp, const CUtensorMap& mk, const CUtensorMap& mq,
                        const Bf16IdxParams& p, int grid, cudaStream_t st) {
-  return fp8   ? launch_variant<true, 1, kB16>(mk, mq, p, grid, st)
-         : grp ? launch_variant<false, 4, kB16>(mk, mq, p, grid, st)
-               : launch_variant<false, 1, kB16>(mk, mq, p, grid, st);
+  return fp8   ? launch_variant<true, 1, kB16, kPaged>(mk, mq, p, grid, st)
+         : grp ? launch_variant<false, 4, kB16, kPaged>(mk, mq, p, grid, st)
+               : launch_variant<false, 1, kB16, kPaged>(mk, mq, p, grid, st);
 }
 
 }  // namespace
 
 bool index_bf16_tc_supported(const IndexArgs& a) {
+  const bool rows_ok = a.page_table == nullptr
+                           ? (int64_t)a.B * a.n_cap < (1ll << 31)
+                           : a.page_rows % kTileKeys == 0 &&
+                                 (int64_t)a.n_pages * a.page_rows < (1ll << 31);
   return (a.kdt == CSA_FP8_E4M3_ROWSCALE || a.kdt == CSA_BF16) && a.n_idx_heads == kHeads &&
-         a.d_idx == kDim && a.n_cap % kTileKeys == 0 && (int64_t)a.B * a.n_cap < (1ll << 31);
+         a.d_idx == kDim && a.n_cap % kTileKeys == 0 && rows_ok;
 }
 
 cudaError_t launch_index_bf16_tc(const IndexArgs& a, cudaStream_t st) {
@@ -527,9 +550,11 @@ cudaError_t launch_index_bf16_tc(const IndexArgs& a, cudaStream_t st) {
   // four queries of a request per MMA (N = 256) when several share the keys and no per-query
   // histogram is wanted (bf16 keys, prefill); otherwise one
   const bool grouped = !fp8 && a.hist == nullptr && a.T >= 4;
+  const bool paged = a.page_table != nullptr;
+  const uint64_t key_rows = paged ? (uint64_t)a.n_pages * a.page_rows : (uint64_t)a.B * a.n_cap;
   CUtensorMap mk;
-  const bool good = fp8 ? make_map_fp8_rows(&mk, a.KI, (uint64_t)a.B * a.n_cap)
-                        : make_map_bf16_rows(&mk, a.KI, (uint64_t)a.B * a.n_cap, kTileKeys);
+  const bool good = fp8 ? make_map_fp8_rows(&mk, a.KI, key_rows)
+                        : make_map_bf16_rows(&mk, a.KI, key_rows, kTileKeys);
   if (!good) return cudaErrorInvalidValue;
   cudaError_t e = cudaSuccess;
   timing_before(st);
@@ -549,11 +574,14 @@ cudaError_t launch_index_bf16_tc(const IndexArgs& a, cudaStream_t st) {
                     fp8 ? static_cast<const float*>(a.KI_scale) : nullptr,
                     b16 ? nullptr : a.scores + (size_t)q0 * a.n_cap,
                     a.hist ? a.hist + (size_t)q0 * kBins : nullptr,
-                    b16 ? static_cast<__nv_bfloat16*>(a.scores16) + (size_t)q0 * a.n_cap : nullptr};
+                    b16 ? static_cast<__nv_bfloat16*>(a.scores16) + (size_t)q0 * a.n_cap : nullptr,
+                    a.page_table, a.page_rows, a.max_pages, a.n_pages};
     const int64_t tiles_max = (int64_t)Q * (a.n_cap / kTileKeys);
     const int grid = (int)(tiles_max < device_sm_count() ? (tiles_max > 0 ? tiles_max : 1) : device_sm_count());
-    e = b16 ? launch_one<true>(fp8, grp, mk, mq, p, grid, st)
-            : launch_one<false>(fp8, grp, mk, mq, p, grid, st);
+    e = paged ? (b16 ? launch_one<true, true>(fp8, grp, mk, mq, p, grid, st)
+                     : launch_one<false, true>(fp8, grp, mk, mq, p, grid, st))
+              : (b16 ? launch_one<true, false>(fp8, grp, mk, mq, p, grid, st)
+                     : launch_one<false, false>(fp8, grp, mk, mq, p, grid, st));
   }
   timing_after(st);
   return e;

@@ -63,6 +63,10 @@ struct IndexArgs {
   float* scores;  // [B, T, n_cap]
   int* hist;      // optional [B*T][4096] histogram of the scores' top 12 key bits (zeroed)
   void* scores16;  // non-null: the scores are rounded to bf16 and stored here instead
+  const int32_t* page_table;  // non-null: KI / KI_scale are a pool of n_pages pages of
+                              // page_rows keys; key e of request b is row e % page_rows of
+                              // page page_table[b * max_pages + e / page_rows]
+  int page_rows, max_pages, n_pages;
 };
 // *hist_done: whether the launched kernel also filled a.hist
 cudaError_t launch_index_scores(const IndexArgs& a, cudaStream_t st, bool* hist_done = nullptr);

@@ -22,7 +22,7 @@ namespace {
 // device-side error word of this translation unit (0 = none; the first code wins)
 __device__ int g_state_error = 0;
 
-enum { kErrBase = 300 };  // stored code = kErrBase - status (301 position, 302 page slot, 303 page id)
+enum { kErrBase = 320 };  // stored code = kErrBase - status (321 position, 322 page slot, 323 page id)
 
 // Block-wide max of non-negative values; `red` is shared scratch of >= 32 floats.
 __device__ __forceinline__ float block_max_nonneg(float v, float* red) {

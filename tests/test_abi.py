@@ -305,6 +305,26 @@ def test_paged_attention_checks():
                                  None) == csa.CSA_OK  # nothing to do
 
 
+def test_paged_index_checks():
+    L = csa.lib()
+    p = _p(topk=512)
+
+    def call(kv, bf16=0):
+        return L.csa_index_topk_paged(ctypes.byref(p), 2, 1, ctypes.byref(kv), FAKE, FAKE, FAKE,
+                                      bf16, FAKE, None, FAKE, 1 << 30, None)
+
+    assert call(csa.CsaPagedKv(csa.CSA_FP8_E4M3_ROWSCALE, FAKE, FAKE, FAKE, 64, 32, 16)) == \
+        csa.CSA_ERR_UNSUPPORTED  # 32-row pages split a 128-key tile
+    assert call(csa.CsaPagedKv(csa.CSA_MIXED_FP8_BF16, FAKE, FAKE, FAKE, 64, 128, 4)) == \
+        csa.CSA_ERR_INVALID_ARG  # not an indexer key format
+    assert call(csa.CsaPagedKv(csa.CSA_BF16, FAKE, None, None, 64, 128, 4)) == \
+        csa.CSA_ERR_INVALID_ARG  # no page table
+    assert call(csa.CsaPagedKv(csa.CSA_FP8_E4M3_ROWSCALE, FAKE, None, FAKE, 64, 128, 4)) == \
+        csa.CSA_ERR_INVALID_ARG  # FP8 keys without their scales
+    assert call(csa.CsaPagedKv(csa.CSA_BF16, FAKE, None, FAKE, 64, 128, 4), bf16=2) == \
+        csa.CSA_ERR_INVALID_ARG
+
+
 def test_binding_refuses_host_tensors():
     import torch
 

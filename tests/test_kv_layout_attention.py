@@ -1,6 +1,8 @@
 """Attention over other KV cache layouts against the float64 oracle on the same bytes:
 mixed-precision rows (csa_sparse_mqa_mixed_kv, hca_dense_mqa_mixed_kv) and paged caches
-(csa_sparse_mqa_paged, hca_dense_mqa_paged).
+(csa_sparse_mqa_paged, hca_dense_mqa_paged); and the indexer over paged keys
+(csa_index_topk_paged), which must give exactly the scores and selection of the contiguous
+keys.
 
 For mixed rows the workloads' bf16 caches are re-encoded by the input encoder (the first
 c - r values as e4m3 with a row scale, the RoPE values as bf16); the oracle decodes those
@@ -183,4 +185,47 @@ def test_paged_cache_with_a_bad_page_id_reports_it():
                             ws_bytes)
     torch.cuda.synchronize()
     assert csa.device_error() == 205
+
+
+@pytest.mark.parametrize("name", ["edge_decode_fp8_tc", "edge_decode_bf16_tc",
+                                  "mid_prefill_bf16_tc"])
+@pytest.mark.parametrize("bf16_scores", [0, 1])
+def test_index_topk_over_paged_keys_equals_contiguous(name, bf16_scores):
+    s, inp = U.inputs(name)
+    dev = R.upload(inp, s)
+    p = R.params_for(s)
+    kdt = csa.DTYPES[s.idx]
+    B, T, N = s.B, s.T, s.n_cap
+    entry = csa.CSA_WS_INDEX_TOPK_BF16 if bf16_scores else csa.CSA_WS_INDEX_TOPK
+    need = csa.workspace_size(p, entry, kdt, B, T, N)
+    ws = torch.empty((need,), dtype=torch.uint8, device="cuda")
+    sdt = torch.int16 if bf16_scores else torch.float32
+    idx_c = torch.empty((B, T, s.topk), dtype=torch.int32, device="cuda")
+    sc_c = torch.zeros((B, T, N), dtype=sdt, device="cuda")
+    if bf16_scores:
+        csa.csa_index_topk_bf16(p, kdt, B, T, N, dev["qI"], None, dev["w"], dev["KI"],
+                                dev.get("KI_scale"), dev["q_pos"], idx_c, sc_c, ws, need)
+    else:
+        csa.csa_index_topk(p, kdt, B, T, N, dev["qI"], None, dev["w"], dev["KI"],
+                           dev.get("KI_scale"), dev["q_pos"], idx_c, sc_c, ws, need)
+    pool, table = _paged(inp["KI"], 128, 6)
+    scales = None
+    if "KI_scale" in inp:
+        spool, _ = _paged(inp["KI_scale"][..., None], 128, 6)
+        scales = _dev(np.ascontiguousarray(spool[..., 0]))
+    keys = csa.paged_kv(kdt, _dev(pool), scales, _dev(table), pool.shape[0], 128, table.shape[1])
+    idx_p = torch.empty_like(idx_c)
+    sc_p = torch.zeros_like(sc_c)
+    torch.cuda.synchronize()
+    csa.device_error()
+    csa.csa_index_topk_paged(p, B, T, keys, dev["qI"], dev["w"], dev["q_pos"], bf16_scores, idx_p,
+                             sc_p, ws, need)
+    torch.cuda.synchronize()
+    assert csa.device_error() == 0
+    assert torch.equal(idx_p, idx_c)
+    pos = inp["q_pos"]
+    for b in range(B):
+        for t in range(T):
+            n = int(max(0, min(pos[b, t] // s.m, N)))
+            assert torch.equal(sc_p[b, t, :n], sc_c[b, t, :n]), f"{name} b={b} t={t}"
 

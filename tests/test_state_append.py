@@ -455,7 +455,7 @@ def test_gpu_state_append_skips_requests_with_bad_pages():
     sc.page_table[1, 0] = sc.n_pages
     before = sc.state.copy()
     pages, _, state, _ = _run_gpu(sc, check_error=False)
-    assert csa.device_error() == 303
+    assert csa.device_error() == 323
     assert np.array_equal(state[:2], before[:2])  # skipped requests stored nothing
     own = sc.page_table[2, 0]
     assert np.abs(pages[own, 0]).sum() > 0
