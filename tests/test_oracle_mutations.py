@@ -211,7 +211,48 @@ def _mut_release_leaks(self):
     self.page_table = []
 
 
+def _mut_resume_wrong_block(self, Ca, Cb, Za, Zb, entries, win_rows):
+    # takes the open block's b-rows as the last finished block's
+    assert self.n_tok == 0 and self.n_entries == 0
+    Ca, Cb, Za, Zb = (np.asarray(x, np.float64) for x in (Ca, Cb, Za, Zb))
+    n0 = Ca.shape[0]
+    nb = n0 // self.m
+    for row in entries:
+        self._write_entry(np.asarray(row, np.float64))
+    if nb > 0:
+        lo = min(self.m * nb, n0 - self.m)
+        self.prev_Cb, self.prev_Zb = Cb[lo:lo + self.m].copy(), Zb[lo:lo + self.m].copy()
+    tail = slice(self.m * nb, n0)
+    self.cur = {"Ca": list(Ca[tail]), "Za": list(Za[tail]), "Cb": list(Cb[tail]),
+                "Zb": list(Zb[tail])}
+    win_rows = np.asarray(win_rows, np.float64)
+    for p in range(max(n0 - self.n_win, 0), n0):
+        self._push_window(win_rows[p], p)
+    self.n_tok = n0
+
+
+def _mut_hca_bias_on_values(self, cv, zv, win_row):
+    t = self.n_tok
+    self.cur_C.append(np.asarray(cv, np.float64))
+    self.cur_Z.append(np.asarray(zv, np.float64))
+    self._push_window(win_row, t)
+    self.n_tok += 1
+    if self.n_tok % self.m:
+        return None
+    i = t // self.m
+    S = O._softmax_rows(np.stack(self.cur_Z))
+    entry = (S * (np.stack(self.cur_C) + self.B)).sum(axis=0)  # bias on the values
+    if self.finalize:
+        entry = O.finalize_entries(entry[None], i, self.m, self.r, self.base, self.eps,
+                                   self.gamma)[0]
+    self._write_entry(entry)
+    self.cur_C, self.cur_Z = [], []
+    return i
+
+
 NEXT_MUTATIONS = {
+    "resume_takes_open_block_b_rows": (SC.CsaState, "resume", _mut_resume_wrong_block),
+    "hca_bias_on_values": (SC.HcaState, "append", _mut_hca_bias_on_values),
     "bf16_truncates": (O, "round_to_bf16", _mut_bf16_truncate),
     "bf16_ties_away_from_zero": (O, "round_to_bf16", _mut_bf16_ties_away),
     "bf16_scores_not_rounded": (O, "topk_select_bf16", lambda s, k: O.topk_select(s, k)),
