@@ -335,6 +335,23 @@ csa_status csa_index_topk_paged(const csa_params* p, int32_t B, int32_t T,
                                 const int64_t* q_pos, int32_t bf16_scores, int32_t* out_idx,
                                 void* out_scores, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * The CSA layer over the state cache's paged caches: csa_index_topk_paged on `keys`
+ * (optionally with BF16 index scores), then the sparse MQA over `kv` (bf16 or mixed rows,
+ * as csa_sparse_mqa_paged), in one call with the decode chain of csa_forward. io = bf16 for
+ * q [B, T, H, c], the window and out; qI bf16 [B, T, 64, 128]; w f32 [B, T, 64]. Both pools
+ * cover N_cap = page_rows * max_pages entries. out_idx [B, T, k]; out_scores (fp32, or bf16
+ * with bf16_scores) may be NULL. Workspace: csa_workspace_size(..., CSA_WS_FORWARD, ...)
+ * with that N_cap.
+ */
+csa_status csa_forward_paged(const csa_params* p, int32_t B, int32_t T, const csa_paged_kv* kv,
+                             const csa_paged_kv* keys, int32_t bf16_scores, const void* qI,
+                             const float* w, const void* q, const void* q_rms_w,
+                             const int64_t* q_pos, const void* win_kv, int64_t L_raw,
+                             const int64_t* win_pos0, const float* sink, int32_t* out_idx,
+                             void* out_scores, void* out, void* ws, size_t ws_bytes,
+                             void* stream);
+
 /* Inputs of the fused CSA layer call. Pointers as in the stage calls above. */
 typedef struct {
   /* optional compression of a new chunk into kv_cache (skipped when Ca == NULL) */

@@ -27,7 +27,7 @@ EXPORTS = (
     "csa_topk_noalloc", "csa_kernel_launches", "csa_state_append", "csa_sparse_mqa_mixed_kv",
     "hca_dense_mqa_mixed_kv", "csa_grouped_out_proj", "csa_grouped_out_proj_workspace_size",
     "csa_sparse_mqa_paged", "hca_dense_mqa_paged", "csa_index_topk_bf16",
-    "csa_index_topk_paged",
+    "csa_index_topk_paged", "csa_forward_paged",
 )
 # size of the library-owned scratch array behind csa_topk_noalloc (bytes, per device)
 TOPK_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -102,6 +102,8 @@ _SIGS = {
     "csa_index_topk_bf16": [_PP, ctypes.c_int, _I32, _I32, _I64] + [_VP] * 9 + [_SZ, _VP],
     "csa_index_topk_paged": [_PP, _I32, _I32, ctypes.POINTER(CsaPagedKv), _VP, _VP, _VP, _I32,
                              _VP, _VP, _VP, _SZ, _VP],
+    "csa_forward_paged": [_PP, _I32, _I32, ctypes.POINTER(CsaPagedKv), ctypes.POINTER(CsaPagedKv),
+                          _I32] + [_VP] * 5 + [_VP, _I64] + [_VP] * 6 + [_SZ, _VP],
     "csa_grouped_out_proj": [_PP, _I32, _I32, _I32, _I32, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "csa_grouped_out_proj_workspace_size": [_PP, _I32, _I32, _I32, _I32],
     "csa_sparse_mqa_mixed_kv": [_PP, _I32, _I32, _VP, _VP, _VP, _VP, _I64, _VP, _VP, _I64, _VP,
@@ -321,6 +323,17 @@ def csa_index_topk_paged(p, B, T, keys: CsaPagedKv, qI, w, q_pos, bf16_scores, o
                                    _ptr(q_pos), int(bf16_scores), _ptr(out_idx), _ptr(out_scores),
                                    _ptr(ws), ws_bytes, _stream(stream))
     _check("csa_index_topk_paged", s)
+
+
+def csa_forward_paged(p, B, T, kv: CsaPagedKv, keys: CsaPagedKv, bf16_scores, qI, w, q, q_rms_w,
+                      q_pos, win_kv, L_raw, win_pos0, sink, out_idx, out_scores, out, ws, ws_bytes,
+                      stream=None):
+    s = lib().csa_forward_paged(ctypes.byref(p), B, T, ctypes.byref(kv), ctypes.byref(keys),
+                                int(bf16_scores), _ptr(qI), _ptr(w), _ptr(q), _ptr(q_rms_w),
+                                _ptr(q_pos), _ptr(win_kv), L_raw, _ptr(win_pos0), _ptr(sink),
+                                _ptr(out_idx), _ptr(out_scores), _ptr(out), _ptr(ws), ws_bytes,
+                                _stream(stream))
+    _check("csa_forward_paged", s)
 
 
 def grouped_out_proj_workspace_size(p, Q, g, d_g, d) -> int:

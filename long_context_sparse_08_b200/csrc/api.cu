@@ -828,6 +828,95 @@ csa_status csa_forward(const csa_params* p, csa_dtype io, int32_t B, int32_t T,
   return ok();
 }
 
+csa_status csa_forward_paged(const csa_params* p, int32_t B, int32_t T, const csa_paged_kv* kv,
+                             const csa_paged_kv* keys, int32_t bf16_scores, const void* qI,
+                             const float* w, const void* q, const void* q_rms_w,
+                             const int64_t* q_pos, const void* win_kv, int64_t L_raw,
+                             const int64_t* win_pos0, const float* sink, int32_t* out_idx,
+                             void* out_scores, void* out, void* ws, size_t ws_bytes,
+                             void* stream) {
+  TRY(check_params(p));
+  TRY(check_topk(p));
+  REQUIRE(p->overlap == 1, "csa_forward_paged is the CSA layer (overlap must be 1)");
+  REQUIRE(bf16_scores == 0 || bf16_scores == 1, "bf16_scores must be 0 or 1");
+  KvLayout lay;
+  int64_t N_cap = 0;
+  TRY(paged_layout(kv, &lay, &N_cap));
+  REQUIRE(keys != nullptr, "paged key descriptor is NULL");
+  REQUIRE(keys->fmt == CSA_BF16 || keys->fmt == CSA_FP8_E4M3_ROWSCALE,
+          "paged indexer keys must be CSA_BF16 or CSA_FP8_E4M3_ROWSCALE");
+  REQUIRE(keys->n_pages >= 1 && keys->page_rows >= 1 && keys->max_pages >= 1,
+          "n_pages, page_rows and max_pages must be >= 1");
+  REQUIRE((int64_t)keys->page_rows * keys->max_pages == N_cap,
+          "the KV and key pools must cover the same entries (page_rows * max_pages)");
+  REQUIRE_PTR(keys->page_table);
+  TRY(check_mqa_args(p, CSA_BF16, B, T, q, q_pos, kv->pages, N_cap, win_kv, L_raw, win_pos0, sink,
+                     q_rms_w, out));
+  TRY(check_index_args(p, keys->fmt, B, T, N_cap, qI, nullptr, w, keys->pages, keys->scales,
+                       q_pos));
+  if ((int64_t)B * T == 0) return ok();
+  REQUIRE_PTR(out_idx);
+  OPTIONAL_PTR(out_scores);
+  {
+    auto ia = make_index(p, keys->fmt, B, T, N_cap, qI, nullptr, w, keys->pages, keys->scales,
+                         q_pos, nullptr);
+    ia.page_table = keys->page_table;
+    ia.page_rows = keys->page_rows;
+    ia.max_pages = keys->max_pages;
+    ia.n_pages = keys->n_pages;
+    if (!csa::index_bf16_tc_supported(ia))
+      return fail(CSA_ERR_UNSUPPORTED,
+                  "paged keys are read by the tensor-core FP8 / bf16 indexer (64 heads of 128, "
+                  "page_rows a multiple of 128)");
+  }
+  auto ma = make_mqa(p, B, T, q, q_pos, kv->pages, N_cap, out_idx, p->topk, win_kv, L_raw,
+                     win_pos0, sink, q_rms_w, out);
+  const bool rope_ok = !lay.mixed ||
+                       (p->rope_dims > 0 && p->rope_dims < p->c && p->rope_dims % 16 == 0);
+  if (!rope_ok || !csa::mqa_tc_supported(ma, true))
+    return fail(CSA_ERR_UNSUPPORTED,
+                "csa_forward_paged: needs the tensor-core attention (c = 512, n_heads a multiple "
+                "of 64; mixed rows: rope_dims a multiple of 16 in (0, 512))");
+  const size_t need = csa_workspace_size(p, CSA_WS_FORWARD, keys->fmt, B, T, N_cap);
+  if (ws == nullptr || ws_bytes < need || !aligned16(ws))
+    return fail(CSA_ERR_WORKSPACE, "csa_forward_paged needs %zu workspace bytes (got %zu)", need,
+                ws_bytes);
+  cudaStream_t st = (cudaStream_t)stream;
+  char* base = static_cast<char*>(ws);
+  const size_t sb = scores_bytes(B, T, N_cap);  // room for fp32 (or bf16) scores
+  const size_t tb = round_up(csa::topk_workspace_bytes(B, T, N_cap, p->topk));
+  void* sc = out_scores ? out_scores : base;
+  ma.kv_scale = lay.mixed ? lay.scales : nullptr;
+  ma.page_table = lay.page_table;
+  ma.n_pages = lay.n_pages;
+  ma.page_rows = lay.page_rows;
+  ma.max_pages = lay.max_pages;
+  ma.chained = csa::topk_decode_path(B, T, N_cap, p->topk);  // as in csa_forward
+  const size_t mb = round_up(csa::mqa_workspace_bytes(ma));
+  csa::TopkArgs t{};
+  t.B = B; t.T = T; t.m = p->m; t.k = p->topk; t.n_cap = N_cap; t.q_pos = q_pos;
+  t.out_idx = out_idx;
+  if (bf16_scores) t.scores16 = sc;
+  else t.scores = static_cast<float*>(sc);
+  if (forward_qhat(p, B, T, N_cap)) {
+    t.qj.q = q;
+    t.qj.q_rms_w = q_rms_w;
+    t.qj.qhat = base + sb + tb + mb;
+    t.qj.H = p->n_heads;
+    t.qj.r = p->rope_dims;
+    t.qj.eps = p->rms_eps;
+    t.qj.rope_base = p->rope_base;
+    for (int i = 0; i < p->rope_dims / 2; ++i)
+      t.qj.inv_freq[i] = csa::rope_inv_freq(i, p->rope_dims, (double)p->rope_base);
+    ma.qhat = t.qj.qhat;
+  }
+  TRY(index_then_topk(p, keys->fmt, B, T, N_cap, qI, nullptr, w, keys->pages, keys->scales,
+                      q_pos, bf16_scores ? nullptr : static_cast<float*>(sc), t, base + sb, tb,
+                      st, bf16_scores ? sc : nullptr, keys));
+  TRY(cuda_status(csa::launch_mqa(ma, true, base + sb + tb, mb, st), "sparse MQA (paged)"));
+  return ok();
+}
+
 uint64_t csa_kernel_launches(void) { return csa::g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"

@@ -229,3 +229,72 @@ def test_index_topk_over_paged_keys_equals_contiguous(name, bf16_scores):
             n = int(max(0, min(pos[b, t] // s.m, N)))
             assert torch.equal(sc_p[b, t, :n], sc_c[b, t, :n]), f"{name} b={b} t={t}"
 
+
+def _paged_forward(s, inp, dev, kv_fmt, kv_rows, kv_scale, bf16_scores):
+    """csa_forward_paged over KV pages of 32 rows and key pages of 128 rows (shuffled)."""
+    p = R.params_for(s)
+    B, T, N = s.B, s.T, s.n_cap
+    kv_pool, kv_table = _paged(kv_rows, 32, 7)
+    kvs = None
+    if kv_scale is not None:
+        sp, _ = _paged(kv_scale[..., None], 32, 7)
+        kvs = _dev(np.ascontiguousarray(sp[..., 0]))
+    k_pool, k_table = _paged(inp["KI"], 128, 8)
+    ks = None
+    if "KI_scale" in inp:
+        sp, _ = _paged(inp["KI_scale"][..., None], 128, 8)
+        ks = _dev(np.ascontiguousarray(sp[..., 0]))
+    kv = csa.paged_kv(kv_fmt, _dev(kv_pool), kvs, _dev(kv_table), kv_pool.shape[0], 32,
+                      kv_table.shape[1])
+    keys = csa.paged_kv(csa.DTYPES[s.idx], _dev(k_pool), ks, _dev(k_table), k_pool.shape[0], 128,
+                        k_table.shape[1])
+    need = csa.workspace_size(p, csa.CSA_WS_FORWARD, csa.DTYPES[s.idx], B, T, N)
+    ws = torch.empty((need,), dtype=torch.uint8, device="cuda")
+    out = torch.empty((B, T, s.n_heads, s.c), dtype=dev["q"].dtype, device="cuda")
+    idx = torch.empty((B, T, s.topk), dtype=torch.int32, device="cuda")
+    sc = torch.zeros((B, T, N), dtype=torch.int16 if bf16_scores else torch.float32,
+                     device="cuda")
+    torch.cuda.synchronize()
+    csa.device_error()
+    csa.csa_forward_paged(p, B, T, kv, keys, bf16_scores, dev["qI"], dev["w"], dev["q"], None,
+                          dev["q_pos"], dev["win_kv"], dev["win_kv"].shape[1], dev["win_pos0"],
+                          dev["sink"], idx, sc, out, ws, need)
+    torch.cuda.synchronize()
+    assert csa.device_error() == 0
+    return out, idx, sc
+
+
+@pytest.mark.parametrize("name", ["edge_decode_fp8_tc", "edge_decode_bf16_tc"])
+def test_forward_paged_equals_contiguous(name):
+    s, inp = U.inputs(name)
+    dev = R.upload(inp, s)
+    st = R.Step(s, dev, want_scores=True)
+    st()
+    torch.cuda.synchronize()
+    out, idx, sc = _paged_forward(s, inp, dev, csa.CSA_BF16, inp["kv_cache"], None, 0)
+    assert torch.equal(idx, st.out_idx)
+    assert torch.equal(out, st.out)
+
+
+@pytest.mark.parametrize("name", ["edge_decode_fp8_tc", "edge_decode_bf16_tc"])
+def test_forward_paged_bf16_scores_over_mixed_kv(name):
+    s, inp, inp2, _, _ = _mixed(name)
+    dev = R.upload(inp, s)
+    codes, rope = inp2["kv_codes"], inp2["kv_rope"]
+    rows = np.concatenate([codes, rope.view(np.uint8)], axis=-1)
+    out, idx, sc = _paged_forward(s, inp, dev, csa.CSA_MIXED_FP8_BF16, rows, inp2["kv_scale"], 1)
+    idx = idx.cpu().numpy()
+    got16 = sc.cpu().numpy().view(np.uint16)
+    res = P.run(s, inp2, want_scores=True)
+    from oracle import csa_oracle as O
+    import tests.test_bf16_scores as BS
+
+    for (b, ti), ref in res["scores"].items():
+        g = O.dec_bf16(got16[b, ti, :ref.size])
+        BS._valid_selection(idx[b, ti], g, s.topk)
+    sel = {(b, ti): idx[b, ti] for (b, ti) in res["out"]}
+    ref_out = P.run(s, inp2, list(sel), idx_override=sel, want_scores=False)["out"]
+    got = out.float().cpu().numpy()
+    for (b, ti), r in ref_out.items():
+        U.check_out(got[b, ti], r, "bf16", f"{name} paged mixed b={b} t={ti}")
+
