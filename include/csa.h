@@ -352,6 +352,28 @@ csa_status csa_forward_paged(const csa_params* p, int32_t B, int32_t T, const cs
                              void* out_scores, void* out, void* ws, size_t ws_bytes,
                              void* stream);
 
+/*
+ * The hand-over from a prefill chunk to decode over the state cache ([P1''] 二(六)):
+ *   csa_compress_paged: as csa_compress, writing entry first_entry + i of request b into row
+ *     (first_entry + i) % page_rows of page page_table[b, (first_entry + i) / page_rows] of
+ *     out_pages (fmt = io; N_cap = page_rows * max_pages). An entry whose page id lies
+ *     outside the pool is skipped and leaves device error code 331.
+ *   csa_state_resume: copies the chunk's last raw rows (Ca, Za, Cb, Zb [B, n_tok, c]; the
+ *     chunk is tokens first_tok .. first_tok + n_tok - 1) into their slots of `state` and its
+ *     last n_win window rows (win_rows [B, n_tok, c], final form; NULL with win_ring NULL)
+ *     into `win_ring`, in the layouts of csa_state_append, so that appends continue at
+ *     position first_tok + n_tok.
+ */
+csa_status csa_compress_paged(const csa_params* p, csa_dtype io, int32_t B, int64_t n_tok,
+                              int64_t first_entry, const void* Ca, const void* Cb,
+                              const void* Za, const void* Zb, const void* bias,
+                              const void* prev_Cb, const void* prev_Zb, const void* kv_rms_w,
+                              int32_t finalize, const csa_paged_kv* out_pages, void* stream);
+csa_status csa_state_resume(const csa_params* p, csa_dtype io, int32_t B, int64_t first_tok,
+                            int64_t n_tok, const void* Ca, const void* Cb, const void* Za,
+                            const void* Zb, const void* win_rows, void* state, void* win_ring,
+                            void* stream);
+
 /* Inputs of the fused CSA layer call. Pointers as in the stage calls above. */
 typedef struct {
   /* optional compression of a new chunk into kv_cache (skipped when Ca == NULL) */
@@ -434,7 +456,7 @@ void csa_set_index_timing_events(void* const* before, void* const* after, int32_
  * early instead of hanging. csa_state_append also leaves a code for a request it skipped.
  * Codes by kernel family: 101-106 MXFP4 indexer, 201-205 attention (205: a page id outside
  * the pool), 301-309 FP8 / bf16 indexer (309: a page id outside the pool), 321-323 state
- * append, 401-405 prefill output projection. Writes the code to *code (0 = none) and clears
+ * append, 331 paged compression, 401-405 prefill output projection. Writes the code to *code (0 = none) and clears
  * it. Synchronises the device. Returns CSA_ERR_CUDA if the copy fails.
  */
 csa_status csa_device_error(int32_t* code);

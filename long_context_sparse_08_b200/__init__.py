@@ -27,7 +27,7 @@ EXPORTS = (
     "csa_topk_noalloc", "csa_kernel_launches", "csa_state_append", "csa_sparse_mqa_mixed_kv",
     "hca_dense_mqa_mixed_kv", "csa_grouped_out_proj", "csa_grouped_out_proj_workspace_size",
     "csa_sparse_mqa_paged", "hca_dense_mqa_paged", "csa_index_topk_bf16",
-    "csa_index_topk_paged", "csa_forward_paged",
+    "csa_index_topk_paged", "csa_forward_paged", "csa_compress_paged", "csa_state_resume",
 )
 # size of the library-owned scratch array behind csa_topk_noalloc (bytes, per device)
 TOPK_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -104,6 +104,9 @@ _SIGS = {
                              _VP, _VP, _VP, _SZ, _VP],
     "csa_forward_paged": [_PP, _I32, _I32, ctypes.POINTER(CsaPagedKv), ctypes.POINTER(CsaPagedKv),
                           _I32] + [_VP] * 5 + [_VP, _I64] + [_VP] * 6 + [_SZ, _VP],
+    "csa_compress_paged": [_PP, ctypes.c_int, _I32, _I64, _I64] + [_VP] * 8 +
+                          [_I32, ctypes.POINTER(CsaPagedKv), _VP],
+    "csa_state_resume": [_PP, ctypes.c_int, _I32, _I64, _I64] + [_VP] * 8,
     "csa_grouped_out_proj": [_PP, _I32, _I32, _I32, _I32, _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "csa_grouped_out_proj_workspace_size": [_PP, _I32, _I32, _I32, _I32],
     "csa_sparse_mqa_mixed_kv": [_PP, _I32, _I32, _VP, _VP, _VP, _VP, _I64, _VP, _VP, _I64, _VP,
@@ -334,6 +337,23 @@ def csa_forward_paged(p, B, T, kv: CsaPagedKv, keys: CsaPagedKv, bf16_scores, qI
                                 _ptr(out_idx), _ptr(out_scores), _ptr(out), _ptr(ws), ws_bytes,
                                 _stream(stream))
     _check("csa_forward_paged", s)
+
+
+def csa_compress_paged(p, io, B, n_tok, first_entry, Ca, Cb, Za, Zb, bias, prev_Cb, prev_Zb,
+                       kv_rms_w, finalize, out_pages: CsaPagedKv, stream=None):
+    s = lib().csa_compress_paged(ctypes.byref(p), io, B, n_tok, first_entry, _ptr(Ca), _ptr(Cb),
+                                 _ptr(Za), _ptr(Zb), _ptr(bias), _ptr(prev_Cb), _ptr(prev_Zb),
+                                 _ptr(kv_rms_w), int(finalize), ctypes.byref(out_pages),
+                                 _stream(stream))
+    _check("csa_compress_paged", s)
+
+
+def csa_state_resume(p, io, B, first_tok, n_tok, Ca, Cb, Za, Zb, win_rows, state, win_ring,
+                     stream=None):
+    s = lib().csa_state_resume(ctypes.byref(p), io, B, first_tok, n_tok, _ptr(Ca), _ptr(Cb),
+                               _ptr(Za), _ptr(Zb), _ptr(win_rows), _ptr(state), _ptr(win_ring),
+                               _stream(stream))
+    _check("csa_state_resume", s)
 
 
 def grouped_out_proj_workspace_size(p, Q, g, d_g, d) -> int:

@@ -253,12 +253,13 @@ const char* csa_last_error(void) { return g_err; }
 
 csa_status csa_device_error(int32_t* code) {
   REQUIRE(code != nullptr, "code is NULL");
-  int words[5] = {0, 0, 0, 0, 0};
+  int words[6] = {0, 0, 0, 0, 0, 0};
   TRY(cuda_status(csa::index_mxf4_device_error(&words[0]), "device error word"));
   TRY(cuda_status(csa::mqa_tc_device_error(&words[1]), "device error word"));
   TRY(cuda_status(csa::index_bf16_device_error(&words[2]), "device error word"));
   TRY(cuda_status(csa::state_append_device_error(&words[3]), "device error word"));
   TRY(cuda_status(csa::out_proj_tc_device_error(&words[4]), "device error word"));
+  TRY(cuda_status(csa::compress_device_error(&words[5]), "device error word"));
   *code = 0;
   for (int w : words)
     if (*code == 0) *code = w;
@@ -315,11 +316,12 @@ size_t csa_workspace_size(const csa_params* p, int32_t entry, csa_dtype kdt, int
   }
 }
 
-csa_status csa_compress(const csa_params* p, csa_dtype io, int32_t B, int64_t n_tok,
-                        int64_t first_entry, int64_t n_cap, const void* Ca, const void* Cb,
-                        const void* Za, const void* Zb, const void* bias, const void* prev_Cb,
-                        const void* prev_Zb, const void* kv_rms_w, int32_t finalize,
-                        void* out_cache, void* stream) {
+namespace {
+csa_status compress_impl(const csa_params* p, csa_dtype io, int32_t B, int64_t n_tok,
+                         int64_t first_entry, int64_t n_cap, const void* Ca, const void* Cb,
+                         const void* Za, const void* Zb, const void* bias, const void* prev_Cb,
+                         const void* prev_Zb, const void* kv_rms_w, int32_t finalize,
+                         void* out_cache, const csa_paged_kv* pages, void* stream) {
   TRY(check_params(p));
   REQUIRE(io == CSA_F32 || io == CSA_BF16, "compression io dtype must be CSA_F32 or CSA_BF16");
   REQUIRE(B >= 0 && B <= 65535, "B must be in [0, 65535]");
@@ -350,7 +352,70 @@ csa_status csa_compress(const csa_params* p, csa_dtype io, int32_t B, int64_t n_
   a.finalize = finalize; a.n_tok = n_tok; a.first_entry = first_entry; a.n_cap = n_cap;
   a.rope_base = p->rope_base; a.eps = p->rms_eps; a.Ca = Ca; a.Cb = Cb; a.Za = Za; a.Zb = Zb;
   a.bias = bias; a.prev_Cb = prev_Cb; a.prev_Zb = prev_Zb; a.rms_w = kv_rms_w; a.out = out_cache;
-  TRY(cuda_status(csa::launch_compress(a, io == CSA_BF16, (cudaStream_t)stream), "compress"));
+  csa::CompressPages pg{};
+  if (pages != nullptr)
+    pg = csa::CompressPages{pages->page_table, pages->page_rows, pages->max_pages, pages->n_pages};
+  TRY(cuda_status(csa::launch_compress(a, io == CSA_BF16, (cudaStream_t)stream,
+                                       pages != nullptr ? &pg : nullptr),
+                  "compress"));
+  return ok();
+}
+}  // namespace
+
+csa_status csa_compress(const csa_params* p, csa_dtype io, int32_t B, int64_t n_tok,
+                        int64_t first_entry, int64_t n_cap, const void* Ca, const void* Cb,
+                        const void* Za, const void* Zb, const void* bias, const void* prev_Cb,
+                        const void* prev_Zb, const void* kv_rms_w, int32_t finalize,
+                        void* out_cache, void* stream) {
+  return compress_impl(p, io, B, n_tok, first_entry, n_cap, Ca, Cb, Za, Zb, bias, prev_Cb,
+                       prev_Zb, kv_rms_w, finalize, out_cache, nullptr, stream);
+}
+
+csa_status csa_compress_paged(const csa_params* p, csa_dtype io, int32_t B, int64_t n_tok,
+                              int64_t first_entry, const void* Ca, const void* Cb,
+                              const void* Za, const void* Zb, const void* bias,
+                              const void* prev_Cb, const void* prev_Zb, const void* kv_rms_w,
+                              int32_t finalize, const csa_paged_kv* out_pages, void* stream) {
+  REQUIRE(out_pages != nullptr, "page descriptor is NULL");
+  REQUIRE(out_pages->fmt == io, "the pages hold rows in the io dtype");
+  REQUIRE(out_pages->n_pages >= 1 && out_pages->page_rows >= 1 && out_pages->max_pages >= 1,
+          "n_pages, page_rows and max_pages must be >= 1");
+  REQUIRE_PTR(out_pages->page_table);
+  const int64_t n_cap = (int64_t)out_pages->page_rows * out_pages->max_pages;
+  return compress_impl(p, io, B, n_tok, first_entry, n_cap, Ca, Cb, Za, Zb, bias, prev_Cb,
+                       prev_Zb, kv_rms_w, finalize, const_cast<void*>(out_pages->pages),
+                       out_pages, stream);
+}
+
+csa_status csa_state_resume(const csa_params* p, csa_dtype io, int32_t B, int64_t first_tok,
+                            int64_t n_tok, const void* Ca, const void* Cb, const void* Za,
+                            const void* Zb, const void* win_rows, void* state, void* win_ring,
+                            void* stream) {
+  TRY(check_params(p));
+  REQUIRE(io == CSA_F32 || io == CSA_BF16, "state io dtype must be CSA_F32 or CSA_BF16");
+  REQUIRE(B >= 0 && B <= 65535, "B must be in [0, 65535]");
+  REQUIRE(first_tok >= 0 && n_tok >= 0, "first_tok and n_tok must be >= 0");
+  REQUIRE(p->overlap == 0 || p->overlap == 1, "overlap must be 0 or 1");
+  REQUIRE((win_rows == nullptr) == (win_ring == nullptr), "win_rows and win_ring go together");
+  REQUIRE(win_ring == nullptr || p->n_win >= 1, "a window ring needs n_win >= 1");
+  if (p->overlap) {
+    REQUIRE_PTR(Cb);
+    REQUIRE_PTR(Zb);
+  } else {
+    REQUIRE(Cb == nullptr && Zb == nullptr, "HCA (overlap=0) takes no b-branch rows");
+  }
+  if (B == 0 || n_tok == 0) return ok();
+  REQUIRE_PTR(Ca);
+  REQUIRE_PTR(Za);
+  REQUIRE_PTR(state);
+  OPTIONAL_PTR(win_rows);
+  OPTIONAL_PTR(win_ring);
+  csa::state::Args a{};
+  a.B = B; a.m = p->m; a.c = p->c; a.overlap = p->overlap; a.n_win = p->n_win;
+  a.Ca = Ca; a.Cb = Cb; a.Za = Za; a.Zb = Zb; a.win_row = win_rows; a.state = state;
+  a.win_ring = win_ring;
+  TRY(cuda_status(csa::launch_state_resume(a, io == CSA_BF16, first_tok, n_tok,
+                                           (cudaStream_t)stream), "state resume"));
   return ok();
 }
 

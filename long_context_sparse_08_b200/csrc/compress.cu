@@ -15,8 +15,10 @@
 
 namespace csa {
 
-template <typename T>
-__global__ void __launch_bounds__(256) k_compress(CompressArgs a) {
+__device__ int g_compress_error = 0;  // 331: a page id outside the pool (the entry is skipped)
+
+template <typename T, bool kPaged>
+__device__ __forceinline__ void compress_body(const CompressArgs& a, const CompressPages& pg) {
   extern __shared__ float row[];  // [c]
   __shared__ float red[32];
   const int i = blockIdx.x;       // entry within the chunk
@@ -69,7 +71,18 @@ __global__ void __launch_bounds__(256) k_compress(CompressArgs a) {
     row[j] = v;
     ss = fmaf(v, v, ss);
   }
-  T* out = static_cast<T*>(a.out) + ((size_t)b * a.n_cap + a.first_entry + i) * c;
+  T* out;
+  if constexpr (kPaged) {  // the state cache's page pool
+    const int64_t e = a.first_entry + i;
+    const int32_t page = pg.page_table[(size_t)b * pg.max_pages + e / pg.page_rows];
+    if (page < 0 || page >= pg.n_pages) {  // uniform over the CTA
+      if (threadIdx.x == 0) atomicCAS(&g_compress_error, 0, 331);
+      return;
+    }
+    out = static_cast<T*>(a.out) + ((size_t)page * pg.page_rows + (size_t)(e % pg.page_rows)) * c;
+  } else {
+    out = static_cast<T*>(a.out) + ((size_t)b * a.n_cap + a.first_entry + i) * c;
+  }
   if (!a.finalize) {
     __syncthreads();
     for (int j = threadIdx.x; j < c; j += blockDim.x) out[j] = from_f32<T>(row[j]);
@@ -94,17 +107,42 @@ __global__ void __launch_bounds__(256) k_compress(CompressArgs a) {
   }
 }
 
-cudaError_t launch_compress(const CompressArgs& a, bool bf16, cudaStream_t st) {
+template <typename T>
+__global__ void __launch_bounds__(256) k_compress(CompressArgs a) {
+  compress_body<T, false>(a, CompressPages{});
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) k_compress_paged(CompressArgs a, CompressPages pg) {
+  compress_body<T, true>(a, pg);
+}
+
+cudaError_t launch_compress(const CompressArgs& a, bool bf16, cudaStream_t st,
+                            const CompressPages* pages) {
   const int n_ent = (int)(a.n_tok / a.m);
   if (n_ent == 0 || a.B == 0) return cudaSuccess;
   dim3 grid(n_ent, a.B);
   const int threads = a.c >= 256 ? 256 : ((a.c + 31) / 32) * 32;
   const size_t smem = (size_t)a.c * sizeof(float);
-  if (bf16)
+  if (pages != nullptr) {
+    if (bf16)
+      launch(false, k_compress_paged<__nv_bfloat16>, dim3(grid), dim3(threads), smem, st, a,
+             *pages);
+    else
+      launch(false, k_compress_paged<float>, dim3(grid), dim3(threads), smem, st, a, *pages);
+  } else if (bf16) {
     launch(false, k_compress<__nv_bfloat16>, dim3(grid), dim3(threads), smem, st, a);
-  else
+  } else {
     launch(false, k_compress<float>, dim3(grid), dim3(threads), smem, st, a);
+  }
   return cudaGetLastError();
+}
+
+cudaError_t compress_device_error(int* code) {
+  int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(code, g_compress_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyToSymbol(g_compress_error, &zero, sizeof(int));
 }
 
 }  // namespace csa

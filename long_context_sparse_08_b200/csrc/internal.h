@@ -35,7 +35,15 @@ struct CompressArgs {
   const void *Ca, *Cb, *Za, *Zb, *bias, *prev_Cb, *prev_Zb, *rms_w;
   void* out;
 };
-cudaError_t launch_compress(const CompressArgs& a, bool bf16, cudaStream_t st);
+// Page pool of a paged compression: entry e of request b goes to row e % page_rows of page
+// page_table[b * max_pages + e / page_rows] of `out`.
+struct CompressPages {
+  const int32_t* page_table;
+  int page_rows, max_pages, n_pages;
+};
+// pages == nullptr: the contiguous cache [B, n_cap, c]
+cudaError_t launch_compress(const CompressArgs& a, bool bf16, cudaStream_t st,
+                            const CompressPages* pages = nullptr);
 
 namespace proj { struct Geom; }
 struct OutProjArgs;
@@ -53,6 +61,10 @@ namespace state { struct Args; }
 // decode-time append of one token per request into the state cache and its pages
 cudaError_t launch_state_append(const state::Args& a, bool bf16, cudaStream_t st);
 cudaError_t state_append_device_error(int* code);
+// after a prefill chunk: its last raw rows and window rows into the state cache
+cudaError_t launch_state_resume(const state::Args& a, bool bf16, int64_t first_tok,
+                                int64_t n_tok, cudaStream_t st);
+cudaError_t compress_device_error(int* code);
 
 struct IndexArgs {
   int B, T, m, n_idx_heads, d_idx, kdt;

@@ -115,7 +115,25 @@ __global__ void __launch_bounds__(256) k_state_append(state::Args a) {
   }
 }
 
+template <typename T>
+__global__ void __launch_bounds__(256) k_state_resume(state::Args a, int64_t first_tok,
+                                                      int64_t n_tok) {
+  for (int j = threadIdx.x; j < a.c; j += blockDim.x)
+    state::resume_channel<T>(a, blockIdx.x, first_tok, n_tok, j);
+}
+
 }  // namespace
+
+cudaError_t launch_state_resume(const state::Args& a, bool bf16, int64_t first_tok,
+                                int64_t n_tok, cudaStream_t st) {
+  if (a.B == 0 || n_tok == 0) return cudaSuccess;
+  const int threads = a.c >= 256 ? 256 : ((a.c + 31) / 32) * 32;
+  cudaError_t e = bf16 ? launch(false, k_state_resume<__nv_bfloat16>, dim3(a.B), dim3(threads), 0,
+                                st, a, first_tok, n_tok)
+                       : launch(false, k_state_resume<float>, dim3(a.B), dim3(threads), 0, st, a,
+                                first_tok, n_tok);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
 
 cudaError_t launch_state_append(const state::Args& a, bool bf16, cudaStream_t st) {
   if (a.B == 0) return cudaSuccess;

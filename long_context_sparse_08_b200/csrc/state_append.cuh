@@ -104,6 +104,31 @@ CSA_HD void store_channel(const Args& a, int64_t b, int64_t t, int j) {
   }
 }
 
+// Channel j of a request resumed after a prefill chunk of tokens first_tok .. first_tok +
+// n_tok - 1 (rows [B, n_tok, c] in a.Ca / a.Za / a.Cb / a.Zb and a.win_row): the chunk's last
+// raw rows into their state slots, its last window rows into the ring, by absolute position.
+template <typename T>
+CSA_HD void resume_channel(const Args& a, int64_t b, int64_t first_tok, int64_t n_tok, int j) {
+  T* s = static_cast<T*>(a.state);
+  const int S = slots(a);
+  for (int64_t t = n_tok > S ? n_tok - S : 0; t < n_tok; ++t) {
+    const size_t src = ((size_t)b * n_tok + t) * a.c + j;
+    const int64_t pabs = first_tok + t;
+    st(s, state_index(a, b, pabs, kRowCa, j), ld(static_cast<const T*>(a.Ca), src));
+    st(s, state_index(a, b, pabs, kRowZa, j), ld(static_cast<const T*>(a.Za), src));
+    if (a.overlap) {
+      st(s, state_index(a, b, pabs, kRowCb, j), ld(static_cast<const T*>(a.Cb), src));
+      st(s, state_index(a, b, pabs, kRowZb, j), ld(static_cast<const T*>(a.Zb), src));
+    }
+  }
+  if (a.win_ring != nullptr)
+    for (int64_t t = n_tok > a.n_win ? n_tok - a.n_win : 0; t < n_tok; ++t) {
+      const size_t src = ((size_t)b * n_tok + t) * a.c + j;
+      const size_t dst = ((size_t)b * a.n_win + (size_t)((first_tok + t) % a.n_win)) * a.c + j;
+      st(static_cast<T*>(a.win_ring), dst, ld(static_cast<const T*>(a.win_row), src));
+    }
+}
+
 // Channel j of entry i, pooled from the state: softmax over the block's logits plus biases
 // (CSA: the a-rows of block i, and for i > 0 the b-rows of block i-1), weighted sum of the
 // values. Same operation order as the whole-chunk compression kernel.

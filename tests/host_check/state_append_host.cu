@@ -149,3 +149,18 @@ extern "C" int encode_rows_host(int out, int n, int c, const float* rows, void* 
   }
   return 0;
 }
+
+// csa_state_resume's arithmetic: the chunk's last raw rows and window rows into the state.
+extern "C" int state_resume_host(int bf16, int B, int m, int c, int overlap, int n_win,
+                                 int64_t first_tok, int64_t n_tok, const void* Ca, const void* Cb,
+                                 const void* Za, const void* Zb, const void* win_rows,
+                                 void* state, void* win_ring) {
+  Args a{};
+  a.B = B; a.m = m; a.c = c; a.overlap = overlap; a.n_win = n_win; a.Ca = Ca; a.Cb = Cb;
+  a.Za = Za; a.Zb = Zb; a.win_row = win_rows; a.state = state; a.win_ring = win_ring;
+  for (int b = 0; b < B; ++b)
+    for (int j = 0; j < c; ++j)
+      bf16 ? resume_channel<__nv_bfloat16>(a, b, first_tok, n_tok, j)
+           : resume_channel<float>(a, b, first_tok, n_tok, j);
+  return 0;
+}

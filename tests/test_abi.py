@@ -325,6 +325,33 @@ def test_paged_index_checks():
         csa.CSA_ERR_INVALID_ARG
 
 
+def test_prefill_handover_checks():
+    L = csa.lib()
+    p = _p()
+    pages = csa.CsaPagedKv(csa.CSA_BF16, FAKE, None, FAKE, 8, 32, 4)
+    args = [ctypes.byref(p), csa.CSA_BF16, 1, 16, 0, FAKE, FAKE, FAKE, FAKE, FAKE, None, None,
+            None, 1, ctypes.byref(pages), None]
+    bad_fmt = csa.CsaPagedKv(csa.CSA_F32, FAKE, None, FAKE, 8, 32, 4)
+    a = list(args)
+    a[14] = ctypes.byref(bad_fmt)
+    assert L.csa_compress_paged(*a) == csa.CSA_ERR_INVALID_ARG  # pages not in the io dtype
+    small = csa.CsaPagedKv(csa.CSA_BF16, FAKE, None, FAKE, 8, 1, 1)
+    a = list(args)
+    a[14] = ctypes.byref(small)
+    assert L.csa_compress_paged(*a) == csa.CSA_ERR_INVALID_ARG  # 4 entries past 1 page of 1 row
+    a = list(args)
+    a[14] = None
+    assert L.csa_compress_paged(*a) == csa.CSA_ERR_INVALID_ARG
+    r = [ctypes.byref(p), csa.CSA_BF16, 1, 0, 16, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None]
+    assert L.csa_state_resume(*r) == csa.CSA_ERR_INVALID_ARG  # window rows without a ring
+    r[1] = csa.CSA_FP8_E4M3_ROWSCALE
+    assert L.csa_state_resume(*r) == csa.CSA_ERR_INVALID_ARG
+    r = [ctypes.byref(p), csa.CSA_BF16, 1, -1, 16, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, None]
+    assert L.csa_state_resume(*r) == csa.CSA_ERR_INVALID_ARG  # negative first token
+    r[3], r[4] = 0, 0
+    assert L.csa_state_resume(*r) == csa.CSA_OK  # an empty chunk: nothing to copy
+
+
 def test_binding_refuses_host_tensors():
     import torch
 

@@ -55,6 +55,7 @@ def host_lib():
     L = ctypes.CDLL(so)
     L.state_append_host.restype = ctypes.c_int
     L.encode_rows_host.restype = ctypes.c_int
+    L.state_resume_host.restype = ctypes.c_int
     return L
 
 
@@ -295,6 +296,28 @@ def test_host_build_stores_mixed_precision_kv_rows():
     enc.check_encoded(plain.keys(pages_f32), pages, enc.scales, "host mixed KV")
 
 
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_host_build_of_the_resume_fills_the_state_of_a_prefill(case):
+    """csa_state_resume's arithmetic fills the state slots and the window ring of requests
+    resumed after a prefill exactly as the scenario's own (independently written) fill."""
+    name, m, overlap, page_rows, starts, appends = case
+    L = host_lib()
+    for t0 in starts:
+        if t0 == 0:
+            continue
+        sc = Scenario(name, m, overlap, page_rows, (t0,), appends, io="bf16")
+        st = np.zeros_like(sc.state)
+        ring = np.zeros_like(sc.ring)
+        rows = {k: np.ascontiguousarray(sc.inp[k][:, :t0]) for k in sc.inp if k != "bias"}
+        rc = L.state_resume_host(1, 1, m, C, overlap, N_WIN, ctypes.c_int64(0),
+                                 ctypes.c_int64(t0), _np_ptr(rows["Ca"]),
+                                 _np_ptr(rows.get("Cb")), _np_ptr(rows["Za"]),
+                                 _np_ptr(rows.get("Zb")), _np_ptr(rows["win"]), _np_ptr(st),
+                                 _np_ptr(ring))
+        assert rc == 0
+        assert np.array_equal(st, sc.state) and np.array_equal(ring, sc.ring)
+
+
 def test_host_encoders_equal_the_input_encoders():
     """The row encoders alone, on rows with zero, tiny, huge and midpoint values."""
     L = host_lib()
@@ -462,3 +485,62 @@ def test_gpu_state_append_skips_requests_with_bad_pages():
     rest = pages.copy()
     rest[own, 0] = 0
     assert not rest.any()
+
+
+# ---------------------------------------------------------------------------
+# prefill -> decode hand-over on paged caches (not yet run on a B200: gated)
+# ---------------------------------------------------------------------------
+
+_FIRST = pytest.mark.skipif(os.environ.get("CSA_RUN_FIRST_GPU_CHECKS") != "1",
+                            reason="awaiting its first run on a B200 (CSA_RUN_FIRST_GPU_CHECKS=1)")
+
+
+@pytest.mark.gpu
+@_FIRST
+def test_gpu_paged_compression_equals_contiguous():
+    import torch
+    import long_context_sparse_08_b200 as csa
+
+    sc = Scenario("csa", 4, 1, 32, (0, 0), 512, io="bf16", seed=78)
+    p = csa.make_params(m=4, overlap=1, c=C, rope_dims=R, rope_base=BASE, rms_eps=EPS,
+                        n_win=N_WIN)
+    dev = lambda k: torch.from_numpy(sc.inp[k].view(np.int16)).cuda()  # noqa: E731
+    cache = torch.zeros((2, 128, C), dtype=torch.int16, device="cuda")
+    csa.csa_compress(p, csa.CSA_BF16, 2, 512, 0, 128, dev("Ca"), dev("Cb"), dev("Za"),
+                     dev("Zb"), dev("bias"), None, None, None, 1, cache)
+    perm = np.random.default_rng(3).permutation(8).astype(np.int32)
+    table = torch.from_numpy(perm.reshape(2, 4)).cuda()
+    pool = torch.zeros((8, 32, C), dtype=torch.int16, device="cuda")
+    pages = csa.paged_kv(csa.CSA_BF16, pool, None, table, 8, 32, 4)
+    torch.cuda.synchronize()
+    csa.device_error()
+    csa.csa_compress_paged(p, csa.CSA_BF16, 2, 512, 0, dev("Ca"), dev("Cb"), dev("Za"),
+                           dev("Zb"), dev("bias"), None, None, None, 1, pages)
+    torch.cuda.synchronize()
+    assert csa.device_error() == 0
+    got = pool[table.view(-1).long()].view(2, 128, C)
+    assert torch.equal(got, cache)
+
+
+@pytest.mark.gpu
+@_FIRST
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_gpu_resume_fills_the_state_of_a_prefill(case):
+    import torch
+    import long_context_sparse_08_b200 as csa
+
+    name, m, overlap, page_rows, starts, appends = case
+    t0 = max(starts)
+    sc = Scenario(name, m, overlap, page_rows, (t0,), appends, io="bf16")
+    p = csa.make_params(m=m, overlap=overlap, c=C, rope_dims=R, rope_base=BASE, rms_eps=EPS,
+                        n_win=N_WIN)
+    up = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()  # noqa
+    rows = {k: up(sc.inp[k][:, :t0]) for k in sc.inp if k != "bias"}
+    st = torch.zeros(sc.state.shape, dtype=torch.int16, device="cuda")
+    ring = torch.zeros(sc.ring.shape, dtype=torch.int16, device="cuda")
+    csa.csa_state_resume(p, csa.CSA_BF16, 1, 0, t0, rows["Ca"], rows.get("Cb"), rows["Za"],
+                         rows.get("Zb"), rows["win"], st, ring)
+    torch.cuda.synchronize()
+    assert np.array_equal(st.cpu().numpy().view(np.uint16), sc.state)
+    assert np.array_equal(ring.cpu().numpy().view(np.uint16), sc.ring)
+
