@@ -177,7 +177,7 @@ class Scenario:
                     f"{what} request {b}: ring slot of position {p}"
             # raw state: the rows of the last S tokens, each in slot p % S
             S = state.shape[1]
-            names = ("Ca", "Za", "Cb", "Zb") if self.overlap else ("Ca", "Za")
+            names = ("Ca", "Za", "Cb", "Zb") if self.overlap else ("Ca", "Za")  # slot rows
             for p in range(max(t1 - S, 0), t1):
                 for r, k in enumerate(names):
                     assert np.array_equal(state[b, p % S, r], self.dec(self.inp[k][b, p]))
@@ -264,6 +264,26 @@ def _run_host(sc: Scenario):
 def test_host_build_of_the_kernel_arithmetic_matches_the_oracle(case, io):
     sc = Scenario(*case, io=io)
     sc.check(*_run_host(sc), what=f"host {case[0]} {io}")
+
+
+# odd geometries for the host build: pages of 7 and 3 entries, a window shorter than a
+# block, c = 128 and c = 64, finalize off, HCA with a small m'
+ODD = [
+    dict(name="csa", m=4, overlap=1, page_rows=7, starts=(0, 57, 130), appends=90, c=128, n_win=3),
+    dict(name="csa", m=4, overlap=1, page_rows=3, starts=(5, 64), appends=70, c=64, n_win=9,
+         finalize=0),
+    dict(name="hca", m=16, overlap=0, page_rows=1, starts=(0, 37), appends=80, c=64, n_win=5),
+]
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("cfg", ODD, ids=["csa_pages7", "csa_pages3_raw", "hca_m16"])
+def test_host_build_on_odd_geometries(cfg, io):
+    cfg = dict(cfg)
+    sc = Scenario(cfg.pop("name"), cfg.pop("m"), cfg.pop("overlap"), cfg.pop("page_rows"),
+                  cfg.pop("starts"), cfg.pop("appends"), io=io, seed=55, **cfg)
+    pages, ring, state = _run_host(sc)
+    sc.check(pages, ring, state, what=f"host odd {io}")
 
 
 def _key_scenarios(out):
@@ -424,6 +444,15 @@ def _run_gpu(sc: Scenario, check_error=True):
 def test_gpu_state_append_matches_the_oracle(case, io):
     sc = Scenario(*case, io=io)
     sc.check(*_run_gpu(sc)[:3], what=f"gpu {case[0]} {io}")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("cfg", ODD, ids=["csa_pages7", "csa_pages3_raw", "hca_m16"])
+def test_gpu_state_append_on_odd_geometries(cfg):
+    cfg = dict(cfg)
+    sc = Scenario(cfg.pop("name"), cfg.pop("m"), cfg.pop("overlap"), cfg.pop("page_rows"),
+                  cfg.pop("starts"), cfg.pop("appends"), io="bf16", seed=55, **cfg)
+    sc.check(*_run_gpu(sc)[:3], what="gpu odd")
 
 
 @pytest.mark.gpu
