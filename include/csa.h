@@ -305,7 +305,9 @@ typedef struct {
  * Stage 4 over a paged cache: as csa_sparse_mqa / hca_dense_mqa with io = CSA_BF16 (the
  * mixed format as in csa_sparse_mqa_mixed_kv), reading each cache row through the page
  * table. An entry whose page id lies outside [0, n_pages) is skipped and leaves device
- * error code 205 for csa_device_error(). Tensor-core attention only (c = 512, n_heads a
+ * error code 205 for csa_device_error(). The window may be the state cache's ring
+ * (csa_state_append's win_ring): pass win_pos0 = NULL and L_raw = n_win, one query per
+ * request (T = 1); window position p is then read from row p mod n_win. Tensor-core attention only (c = 512, n_heads a
  * multiple of 64; mixed rows: rope_dims a multiple of 16 in (0, 512)), else
  * CSA_ERR_UNSUPPORTED. Workspace: csa_workspace_size() with N_cap = page_rows * max_pages.
  */
@@ -340,9 +342,10 @@ csa_status csa_index_topk_paged(const csa_params* p, int32_t B, int32_t T,
  * (optionally with BF16 index scores), then the sparse MQA over `kv` (bf16 or mixed rows,
  * as csa_sparse_mqa_paged), in one call with the decode chain of csa_forward. io = bf16 for
  * q [B, T, H, c], the window and out; qI bf16 [B, T, 64, 128]; w f32 [B, T, 64]. Both pools
- * cover N_cap = page_rows * max_pages entries. out_idx [B, T, k]; out_scores (fp32, or bf16
- * with bf16_scores) may be NULL. Workspace: csa_workspace_size(..., CSA_WS_FORWARD, ...)
- * with that N_cap.
+ * cover N_cap = page_rows * max_pages entries. The window is a linear buffer with win_pos0,
+ * or the state cache's ring (win_pos0 = NULL, L_raw = n_win, T = 1) as in
+ * csa_sparse_mqa_paged. out_idx [B, T, k]; out_scores (fp32, or bf16 with bf16_scores) may
+ * be NULL. Workspace: csa_workspace_size(..., CSA_WS_FORWARD, ...) with that N_cap.
  */
 csa_status csa_forward_paged(const csa_params* p, int32_t B, int32_t T, const csa_paged_kv* kv,
                              const csa_paged_kv* keys, int32_t bf16_scores, const void* qI,

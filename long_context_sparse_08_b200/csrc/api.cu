@@ -129,7 +129,8 @@ csa::MqaArgs make_mqa(const csa_params* p, int32_t B, int32_t T, const void* q,
 csa_status check_mqa_args(const csa_params* p, csa_dtype io, int32_t B, int32_t T,
                           const void* q, const int64_t* q_pos, const void* kv, int64_t N_cap,
                           const void* win, int64_t L_raw, const int64_t* pos0,
-                          const float* sink, const void* q_rms_w, const void* out) {
+                          const float* sink, const void* q_rms_w, const void* out,
+                          bool ring_ok = false) {
   TRY(check_params(p));
   TRY(check_attn(p));
   TRY(check_sizes(B, T, N_cap));
@@ -143,7 +144,12 @@ csa_status check_mqa_args(const csa_params* p, csa_dtype io, int32_t B, int32_t 
   if (p->n_win > 0) {
     REQUIRE(L_raw >= 1, "n_win > 0 needs window rows (L_raw >= 1)");
     REQUIRE_PTR(win);
-    REQUIRE_PTR(pos0);
+    if (ring_ok && pos0 == nullptr) {  // the state cache's window ring
+      REQUIRE(L_raw == p->n_win, "a window ring holds n_win rows (L_raw = n_win)");
+      REQUIRE(T == 1, "a window ring serves one query per request (T = 1)");
+    } else {
+      REQUIRE_PTR(pos0);
+    }
   }
   OPTIONAL_PTR(sink);
   OPTIONAL_PTR(q_rms_w);
@@ -744,7 +750,7 @@ csa_status tc_mqa_ext(const char* what, const csa_params* p, int32_t B, int32_t 
                       const int64_t* win_pos0, const float* sink, const void* q_rms_w,
                       void* out, void* ws, size_t ws_bytes, void* stream) {
   TRY(check_mqa_args(p, CSA_BF16, B, T, q, q_pos, kv.rows, N_cap, win_kv, L_raw, win_pos0, sink,
-                     q_rms_w, out));
+                     q_rms_w, out, kv.page_table != nullptr));
   if ((int64_t)B * T == 0) return ok();
   if (k > 0) REQUIRE_PTR(idx);
   if (kv.mixed && N_cap > 0) REQUIRE_PTR(kv.scales);
@@ -916,7 +922,7 @@ csa_status csa_forward_paged(const csa_params* p, int32_t B, int32_t T, const cs
           "the KV and key pools must cover the same entries (page_rows * max_pages)");
   REQUIRE_PTR(keys->page_table);
   TRY(check_mqa_args(p, CSA_BF16, B, T, q, q_pos, kv->pages, N_cap, win_kv, L_raw, win_pos0, sink,
-                     q_rms_w, out));
+                     q_rms_w, out, true));
   TRY(check_index_args(p, keys->fmt, B, T, N_cap, qI, nullptr, w, keys->pages, keys->scales,
                        q_pos));
   if ((int64_t)B * T == 0) return ok();

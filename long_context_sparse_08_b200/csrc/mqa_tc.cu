@@ -195,7 +195,9 @@ __device__ __forceinline__ const void* row_src_ext(const MqaArgs& a, int bt, int
     }
   }
   if (j < rl.L) {
-    const int64_t rr = rl.lo + (j - rl.n_sel) - a.win_pos0[b];
+    const int64_t p = rl.lo + (j - rl.n_sel);  // the window token's position
+    // win_pos0 == nullptr: the state cache's window ring (position p in row p mod l_raw)
+    const int64_t rr = a.win_pos0 != nullptr ? p - a.win_pos0[b] : p % a.l_raw;
     if (rr < 0 || rr >= a.l_raw) return nullptr;
     return static_cast<const __nv_bfloat16*>(a.win) + ((size_t)b * a.l_raw + rr) * kC;
   }
@@ -839,7 +841,8 @@ cudaError_t launch_mqa_tc(const MqaArgs& a, void* ws, size_t ws_bytes, cudaStrea
   const bool paged = a.page_table != nullptr;  // cache rows through the page table
   // cache rows come by TMA only when they are contiguous bf16 rows
   P.tma_kv = !mixed && !paged && make_map_rows(&tm_kv, a.kv, (int64_t)a.B * a.n_cap) ? 1 : 0;
-  P.tma_win = make_map_rows(&tm_win, a.win, (int64_t)a.B * a.l_raw) ? 1 : 0;
+  // window rows by TMA only from a linear window buffer (a ring wraps)
+  P.tma_win = a.win_pos0 != nullptr && make_map_rows(&tm_win, a.win, (int64_t)a.B * a.l_raw) ? 1 : 0;
   if (P.nsplit > 1 && ws_bytes < mqa_tc_workspace_bytes(a)) return cudaErrorInvalidValue;
   const int64_t streams = (int64_t)a.B * a.T * P.G;
   auto kern = mixed ? (paged ? k_mqa_tc<true, true> : k_mqa_tc<true, false>)

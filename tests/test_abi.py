@@ -300,6 +300,16 @@ def test_paged_attention_checks():
         csa.CSA_ERR_INVALID_ARG  # mixed rows without scales
     assert call(kv, idx=None) == csa.CSA_ERR_INVALID_ARG
     assert call(kv, params=_p(n_heads=32)) == csa.CSA_ERR_UNSUPPORTED
+    # the window ring: win_pos0 = NULL needs L_raw = n_win and one query per request
+    ring = lambda B, T, L: L.csa_sparse_mqa_paged(  # noqa: E731
+        ctypes.byref(p), B, T, FAKE, FAKE, ctypes.byref(kv), FAKE, FAKE, 64, None, None, None,
+        FAKE, None, 0, None)
+    assert ring(1, 1, L) == csa.CSA_ERR_INVALID_ARG  # L_raw 64 != n_win 128
+    assert L.csa_sparse_mqa_paged(ctypes.byref(p), 1, 2, FAKE, FAKE, ctypes.byref(kv), FAKE,
+                                  FAKE, 128, None, None, None, FAKE, None, 0,
+                                  None) == csa.CSA_ERR_INVALID_ARG  # T = 2
+    assert L.csa_sparse_mqa(ctypes.byref(p), 1, 1, 1, FAKE, FAKE, FAKE, 10, FAKE, FAKE, 128, None,
+                            None, None, FAKE, None, 0, None) == csa.CSA_ERR_INVALID_ARG
     assert L.hca_dense_mqa_paged(ctypes.byref(_p(m=128, overlap=0)), 0, 1, None, None,
                                  ctypes.byref(kv), None, 0, None, None, None, None, None, 0,
                                  None) == csa.CSA_OK  # nothing to do

@@ -230,8 +230,9 @@ def test_index_topk_over_paged_keys_equals_contiguous(name, bf16_scores):
             assert torch.equal(sc_p[b, t, :n], sc_c[b, t, :n]), f"{name} b={b} t={t}"
 
 
-def _paged_forward(s, inp, dev, kv_fmt, kv_rows, kv_scale, bf16_scores):
-    """csa_forward_paged over KV pages of 32 rows and key pages of 128 rows (shuffled)."""
+def _paged_forward(s, inp, dev, kv_fmt, kv_rows, kv_scale, bf16_scores, ring=None):
+    """csa_forward_paged over KV pages of 32 rows and key pages of 128 rows (shuffled); with
+    `ring` ([B, n_win, c] device rows) the window is read as the state cache's ring."""
     p = R.params_for(s)
     B, T, N = s.B, s.T, s.n_cap
     kv_pool, kv_table = _paged(kv_rows, 32, 7)
@@ -256,9 +257,10 @@ def _paged_forward(s, inp, dev, kv_fmt, kv_rows, kv_scale, bf16_scores):
                      device="cuda")
     torch.cuda.synchronize()
     csa.device_error()
+    win, L, pos0 = (dev["win_kv"], dev["win_kv"].shape[1], dev["win_pos0"]) if ring is None \
+        else (ring, ring.shape[1], None)
     csa.csa_forward_paged(p, B, T, kv, keys, bf16_scores, dev["qI"], dev["w"], dev["q"], None,
-                          dev["q_pos"], dev["win_kv"], dev["win_kv"].shape[1], dev["win_pos0"],
-                          dev["sink"], idx, sc, out, ws, need)
+                          dev["q_pos"], win, L, pos0, dev["sink"], idx, sc, out, ws, need)
     torch.cuda.synchronize()
     assert csa.device_error() == 0
     return out, idx, sc
@@ -297,4 +299,23 @@ def test_forward_paged_bf16_scores_over_mixed_kv(name):
     got = out.float().cpu().numpy()
     for (b, ti), r in ref_out.items():
         U.check_out(got[b, ti], r, "bf16", f"{name} paged mixed b={b} t={ti}")
+
+
+@pytest.mark.parametrize("name", ["edge_decode_fp8_tc", "edge_decode_bf16_tc"])
+def test_forward_paged_reads_the_window_ring(name):
+    """The state cache's window ring (position p in row p mod n_win) gives the same output as
+    the linear window buffer."""
+    s, inp = U.inputs(name)
+    dev = R.upload(inp, s)
+    win = inp["win_kv"]
+    ring = np.zeros((s.B, s.n_win, s.c), win.dtype)
+    for b in range(s.B):
+        t, p0 = int(inp["q_pos"][b, 0]), int(inp["win_pos0"][b])
+        for pos in range(max(t - s.n_win + 1, 0), t + 1):
+            ring[b, pos % s.n_win] = win[b, pos - p0]
+    out_l, idx_l, _ = _paged_forward(s, inp, dev, csa.CSA_BF16, inp["kv_cache"], None, 0)
+    out_r, idx_r, _ = _paged_forward(s, inp, dev, csa.CSA_BF16, inp["kv_cache"], None, 0,
+                                     ring=_dev(ring))
+    assert torch.equal(idx_r, idx_l)
+    assert torch.equal(out_r, out_l)
 
