@@ -47,7 +47,7 @@ extern "C" {
 typedef enum {
   CSA_OK = 0,
   CSA_ERR_INVALID_ARG = 1, /* a pointer, size or alignment the call cannot accept */
-  CSA_ERR_UNSUPPORTED = 2, /* a valid shape / dtype combination this build does not implement */
+  CSA_ERR_UNSUPPORTED = 2, /* a valid shape / dtype combination this library does not implement */
   CSA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than csa_workspace_size() */
   CSA_ERR_CUDA = 4         /* the CUDA runtime reported an error while queueing */
 } csa_status;
