@@ -477,13 +477,31 @@ def _time_calls(fn, n_rep, warmup, steps):
     return a.elapsed_time(b) / steps
 
 
+def check_part_workload(part, s):
+    """Exit with a message when a part cannot run on the workload's caches (before any GPU
+    work): the paged indexer and the BF16-score path take FP8 or bf16 keys, the paged layer a
+    CSA decode step."""
+    want = None
+    if part in ("bf16_scores", "forward_paged") and s.idx not in ("fp8", "bf16"):
+        want = "FP8 or bf16 indexer keys"
+    elif part == "forward_paged" and s.kind != "csa_decode":
+        want = "a CSA decode step"
+    if want:
+        raise SystemExit(f"--part {part} wants a workload with {want} "
+                         f"(e.g. --workload flash_decode_131k); {s.name} has "
+                         f"{s.kind} / {s.idx} keys")
+
+
 def run_part(args, W):
     """One JSON line for an extension kernel family on the workload's shape:
     out_proj          grouped output projection of the batch's queries (HBM roofline);
     out_proj_prefill  its tensor-core form on a prefill chunk's queries (tensor roofline);
     state_append      one decode token per request into the KV and indexer-key state caches;
     kv_layouts        the attention alone over bf16, mixed-precision and paged caches;
-    bf16_scores       index + top-k with fp32 and with BF16 scores (FP8 / bf16 keys)."""
+    bf16_scores       index + top-k with fp32 and with BF16 scores (FP8 / bf16 keys);
+    forward_paged     the CSA layer over page pools and a window ring vs the contiguous one."""
+    s = W.SHAPES[args.workload]
+    check_part_workload(args.part, s)
     import torch
     import long_context_sparse_08_b200 as csa
     from long_context_sparse_08_b200 import runner as R
@@ -491,7 +509,6 @@ def run_part(args, W):
     torch.cuda.set_device(0)
     peaks, peak_src = load_peaks()
     hbm = float(peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]))
-    s = W.SHAPES[args.workload]
     before = csa.kernel_launches()
     clocks = Clocks(0)
     line = {"part": args.part, "workload": args.workload, "steps": args.steps,
@@ -679,6 +696,59 @@ def run_part(args, W):
                     roofline={"bound": "tensor", "achieved": round(tf, 1), "peak": peak_tf,
                               "peak_source": peak_src, "unit": "TFLOP/s",
                               "frac": round(tf / peak_tf, 4), "flops_per_call": flops})
+    elif args.part == "forward_paged":
+        # the CSA layer over page pools (KV pages of 32 entries, key pages of 128 keys, both
+        # shuffled; the window as a ring) against csa_forward on the contiguous caches
+        inp = W.make_inputs(s)
+        dev = R.upload(inp, s)
+        p = R.params_for(s)
+        B, T, N = s.B, s.T, s.n_cap
+        contiguous = R.Step(s, dev)
+        g = torch.Generator(device="cpu").manual_seed(10)
+
+        def pool_of(t, rows, perm=None):
+            # t [B, n, ...] -> a pool of B * n / rows pages in shuffled order and its table
+            pages = t.shape[1] // rows
+            if perm is None:
+                perm = torch.randperm(t.shape[0] * pages, generator=g).to(torch.int32).cuda()
+            pool = torch.empty((t.shape[0] * pages, rows) + tuple(t.shape[2:]), dtype=t.dtype,
+                               device="cuda")
+            pool[perm.long()] = t.reshape((t.shape[0] * pages, rows) + tuple(t.shape[2:]))
+            return pool, perm.view(t.shape[0], pages)
+
+        kv_pool, kv_table = pool_of(dev["kv_cache"], 32)
+        k_pool, k_table = pool_of(dev["KI"], 128)
+        k_scales = None
+        if "KI_scale" in dev:  # the key scales in the keys' page order
+            k_scales, _ = pool_of(dev["KI_scale"], 128, k_table.view(-1))
+        kv = csa.paged_kv(csa.CSA_BF16, kv_pool, None, kv_table, kv_pool.shape[0], 32,
+                          kv_table.shape[1])
+        keys = csa.paged_kv(csa.DTYPES[s.idx], k_pool, k_scales, k_table, k_pool.shape[0], 128,
+                            k_table.shape[1])
+        # the window ring: position p in row p mod n_win
+        ring = torch.empty((B, s.n_win, s.c), dtype=dev["win_kv"].dtype, device="cuda")
+        for b in range(B):
+            t, p0 = int(inp["q_pos"][b, 0]), int(inp["win_pos0"][b])
+            for q0 in range(max(t - s.n_win + 1, 0), t + 1):
+                ring[b, q0 % s.n_win] = dev["win_kv"][b, q0 - p0]
+        need = csa.workspace_size(p, csa.CSA_WS_FORWARD, csa.DTYPES[s.idx], B, T, N)
+        ws = torch.empty((need,), dtype=torch.uint8, device="cuda")
+        out = torch.empty((B, T, s.n_heads, s.c), dtype=dev["q"].dtype, device="cuda")
+        idx = torch.empty((B, T, s.topk), dtype=torch.int32, device="cuda")
+        res = {"contiguous": round(_time_calls(lambda i: contiguous(), 1, args.warmup,
+                                               args.steps), 5)}
+        for name, b16 in (("paged", 0), ("paged_bf16_scores", 1)):
+            fn = lambda i, b16=b16: csa.csa_forward_paged(  # noqa: E731
+                p, B, T, kv, keys, b16, dev["qI"], dev["w"], dev["q"], None, dev["q_pos"], ring,
+                s.n_win, None, dev["sink"], idx, None, out, ws, need)
+            res[name] = round(_time_calls(fn, 1, args.warmup, args.steps), 5)
+        line.update(metric="CSA layer calls/s over the state cache's page pools",
+                    value=round(1e3 / res["paged"], 2), unit="calls/s (paged, fp32 scores)",
+                    ms_per_call=res, config={"B": B, "T": T, "n_cap": N, "keys": s.idx,
+                                             "kv_page_rows": 32, "key_page_rows": 128,
+                                             "window": "ring"},
+                    roofline={"bound": "hbm (key stream)", "peak": hbm, "peak_source": peak_src,
+                              "unit": "GB/s"})
     line["gpu_launches"] = int(csa.kernel_launches() - before)
     line["clocks"] = clocks.stop()
     line["device_error"] = csa.device_error()
@@ -686,7 +756,8 @@ def run_part(args, W):
     return 0
 
 
-PARTS = {"out_proj", "state_append", "kv_layouts", "bf16_scores", "out_proj_prefill"}
+PARTS = {"out_proj", "state_append", "kv_layouts", "bf16_scores", "out_proj_prefill",
+         "forward_paged"}
 
 
 def main():

@@ -97,3 +97,15 @@ def test_extension_bytes(bench):
     kv = 2 * 512 * (4 + 4 + 1 + 1) + (16 * 512 * 2 + 512 * 2) // 4
     keys = 2 * 128 * (4 + 4) + (16 * 128 * 2 + 68) // 4
     assert bench.state_append_bytes(512, 4, 1) == {"kv": kv, "keys": keys, "total": kv + keys}
+
+
+def test_parts_refuse_workloads_they_cannot_run(bench):
+    # the checks run before any GPU work, so they can be exercised here
+    for part in ("bf16_scores", "forward_paged"):
+        with pytest.raises(SystemExit, match="FP8 or bf16 indexer keys"):
+            bench.check_part_workload(part, W.SHAPES["pro_decode_1m"])
+        bench.check_part_workload(part, W.SHAPES["flash_decode_131k"])
+    with pytest.raises(SystemExit, match="a CSA decode step"):
+        bench.check_part_workload("forward_paged", W.SHAPES["flash_prefill_8k"])
+    bench.check_part_workload("bf16_scores", W.SHAPES["flash_prefill_8k"])
+    bench.check_part_workload("out_proj", W.SHAPES["pro_decode_1m"])
