@@ -430,7 +430,9 @@ size_t csa_workspace_size(const csa_params* p, int32_t entry, csa_dtype kdt, int
  * HBM on CUDA cores, 16 queries per pass; sums stay fp32 until the final rounding.
  * Prefill (Q >= 128): two tcgen05 bf16 GEMMs with fp32 accumulation; the intermediate is
  * stored once in bf16 (needs c*H/g and g*d_g multiples of 64, d_g and d >= 64, else
- * CSA_ERR_UNSUPPORTED). Needs d_g and d multiples of 8 and n_heads a multiple of g.
+ * CSA_ERR_UNSUPPORTED). Needs d_g and d multiples of 8, n_heads a multiple of g, and o,
+ * w_grp, w_out, out and ws 16-byte aligned (16-byte weight loads, tensor-map copies and
+ * stores), else CSA_ERR_INVALID_ARG (CSA_ERR_WORKSPACE for ws).
  * Workspace: csa_grouped_out_proj_workspace_size().
  */
 csa_status csa_grouped_out_proj(const csa_params* p, int32_t Q, int32_t g, int32_t d_g,

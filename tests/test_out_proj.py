@@ -113,6 +113,12 @@ def test_checks_on_the_host():
     a = list(args(4, 16, 1024, 7168))
     a[10] = need - 1
     assert L.csa_grouped_out_proj(*a) == csa.CSA_ERR_WORKSPACE
+    # every operand 16-byte aligned (weights are read 16 bytes at a time)
+    for i in (5, 6, 7, 8):
+        for q in (4, 128):
+            a = list(args(q, 16, 1024, 7168))
+            a[i] = F + 8
+            assert L.csa_grouped_out_proj(*a) == csa.CSA_ERR_INVALID_ARG, (i, q)
 
 
 # ---------------------------------------------------------------------------
