@@ -479,16 +479,16 @@ def _time_calls(fn, n_rep, warmup, steps):
 
 def check_part_workload(part, s):
     """Exit with a message when a part cannot run on the workload's caches (before any GPU
-    work): the paged indexer and the BF16-score path take FP8 or bf16 keys, the paged layer a
-    CSA decode step."""
+    work): the paged indexer and the BF16-score path take the tensor-core indexers' keys
+    (MXFP4, FP8 or bf16), the paged layer a CSA decode step."""
     want = None
-    if part in ("bf16_scores", "forward_paged") and s.idx not in ("fp8", "bf16"):
-        want = "FP8 or bf16 indexer keys"
+    if part in ("bf16_scores", "forward_paged") and s.idx not in ("mxfp4", "fp8", "bf16"):
+        want = "MXFP4, FP8 or bf16 indexer keys"
     elif part == "forward_paged" and s.kind != "csa_decode":
         want = "a CSA decode step"
     if want:
         raise SystemExit(f"--part {part} wants a workload with {want} "
-                         f"(e.g. --workload flash_decode_131k); {s.name} has "
+                         f"(e.g. --workload pro_decode_1m); {s.name} has "
                          f"{s.kind} / {s.idx} keys")
 
 
@@ -498,7 +498,7 @@ def run_part(args, W):
     out_proj_prefill  its tensor-core form on a prefill chunk's queries (tensor roofline);
     state_append      one decode token per request into the KV and indexer-key state caches;
     kv_layouts        the attention alone over bf16, mixed-precision and paged caches;
-    bf16_scores       index + top-k with fp32 and with BF16 scores (FP8 / bf16 keys);
+    bf16_scores       index + top-k with fp32 and with BF16 scores;
     forward_paged     the CSA layer over page pools and a window ring vs the contiguous one."""
     s = W.SHAPES[args.workload]
     check_part_workload(args.part, s)
@@ -647,7 +647,7 @@ def run_part(args, W):
                               "peak_source": peak_src, "unit": "GB/s"})
     elif args.part == "bf16_scores":
         # index + top-k with fp32 scores (csa_index_topk) and with BF16 scores
-        # (csa_index_topk_bf16) on the workload's keys (FP8 / bf16 tensor-core indexer)
+        # (csa_index_topk_bf16) on the workload's keys (MXFP4 / FP8 / bf16 tensor-core indexers)
         inp = W.make_inputs(s)
         dev = R.upload(inp, s)
         p = R.params_for(s)
@@ -739,8 +739,8 @@ def run_part(args, W):
                                                args.steps), 5)}
         for name, b16 in (("paged", 0), ("paged_bf16_scores", 1)):
             fn = lambda i, b16=b16: csa.csa_forward_paged(  # noqa: E731
-                p, B, T, kv, keys, b16, dev["qI"], dev["w"], dev["q"], None, dev["q_pos"], ring,
-                s.n_win, None, dev["sink"], idx, None, out, ws, need)
+                p, B, T, kv, keys, b16, dev["qI"], dev.get("qI_scale"), dev["w"], dev["q"], None,
+                dev["q_pos"], ring, s.n_win, None, dev["sink"], idx, None, out, ws, need)
             res[name] = round(_time_calls(fn, 1, args.warmup, args.steps), 5)
         line.update(metric="CSA layer calls/s over the state cache's page pools",
                     value=round(1e3 / res["paged"], 2), unit="calls/s (paged, fp32 scores)",

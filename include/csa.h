@@ -227,9 +227,9 @@ csa_status csa_index_topk(const csa_params* p, csa_dtype kdt, int32_t B, int32_t
  * rounded to the nearest bf16 (ties to even) and stored as bf16 [B, T, N_cap] (out_scores16,
  * or the workspace when NULL); the selector then orders the bf16 values by (value desc,
  * index asc), so scores that round alike tie and the smaller index wins. Half the score
- * bytes of csa_index_topk. Keys: CSA_FP8_E4M3_ROWSCALE or CSA_BF16 on the tensor-core
- * indexer (64 heads of 128, N_cap a multiple of 128), else CSA_ERR_UNSUPPORTED. Workspace:
- * csa_workspace_size(..., CSA_WS_INDEX_TOPK_BF16, ...).
+ * bytes of csa_index_topk. Keys: CSA_FP8_E4M3_ROWSCALE, CSA_BF16 or CSA_MXFP4 on the
+ * tensor-core indexers (64 heads of 128, N_cap a multiple of 128), else
+ * CSA_ERR_UNSUPPORTED. Workspace: csa_workspace_size(..., CSA_WS_INDEX_TOPK_BF16, ...).
  */
 csa_status csa_index_topk_bf16(const csa_params* p, csa_dtype kdt, int32_t B, int32_t T,
                                int64_t N_cap, const void* qI, const void* qI_scale,
@@ -296,7 +296,9 @@ typedef struct {
   csa_dtype fmt;              /* CSA_BF16 (pages [n_pages, page_rows, c]) or CSA_MIXED_FP8_BF16
                                  (pages [n_pages, page_rows, c + r] bytes)                  */
   const void* pages;          /* device                                                     */
-  const float* scales;        /* CSA_MIXED_FP8_BF16: [n_pages, page_rows] fp32; else NULL   */
+  const void* scales;         /* CSA_MIXED_FP8_BF16 and CSA_FP8_E4M3_ROWSCALE: fp32
+                                 [n_pages, page_rows]; CSA_MXFP4 keys: the e8m0 exponent
+                                 blocks as csa_state_append writes them; else NULL          */
   const int32_t* page_table;  /* device int32 [B, max_pages]                               */
   int32_t n_pages, page_rows, max_pages;
 } csa_paged_kv;
@@ -324,24 +326,31 @@ csa_status hca_dense_mqa_paged(const csa_params* p, int32_t B, int32_t T, const 
 
 /*
  * Stages 2 + 3 over indexer keys kept in a page pool (the compressed indexer keys of the
- * state cache, [P1''] 二(六)): as csa_index_topk with bf16 queries qI [B, T, 64, 128], the keys
- * of request b read through the page table. keys->fmt is CSA_BF16 (pages [n_pages,
- * page_rows, 128]) or CSA_FP8_E4M3_ROWSCALE (e4m3 pages and scales [n_pages, page_rows]);
- * page_rows is a multiple of 128; N_cap = page_rows * max_pages. bf16_scores = 1 selects on
- * BF16 index scores as csa_index_topk_bf16 does. out_scores (fp32, or bf16 with bf16_scores)
- * may be NULL. A key whose page id lies outside the pool reads row 0 and leaves device error
- * code 309. Workspace: csa_workspace_size() with CSA_WS_INDEX_TOPK or CSA_WS_INDEX_TOPK_BF16.
+ * state cache, [P1''] 二(六)): as csa_index_topk, the keys of request b read through the page
+ * table; page_rows is a multiple of 128 and N_cap = page_rows * max_pages. keys->fmt:
+ *   CSA_BF16: pages [n_pages, page_rows, 128] bf16; qI bf16 [B, T, 64, 128], qI_scale NULL;
+ *   CSA_FP8_E4M3_ROWSCALE: e4m3 pages, scales fp32 [n_pages, page_rows]; qI as for bf16;
+ *   CSA_MXFP4 ([P1'] 二(四)): pages [n_pages, page_rows, 64] e2m1 pairs and their e8m0
+ *     exponent blocks, the layout csa_state_append writes with out_fmt = CSA_MXFP4 (a page is
+ *     page_rows / 128 blocks, each laid out as for csa_index_scores); qI and qI_scale in
+ *     MXFP4 as for csa_index_topk; at most 1024 queries per call.
+ * bf16_scores = 1 selects on BF16 index scores as csa_index_topk_bf16 does. out_scores (fp32,
+ * or bf16 with bf16_scores) may be NULL. A visible key whose page id lies outside the pool
+ * reads pool row 0 and leaves device error code 309 (FP8 / bf16 keys) or 107 (MXFP4 keys).
+ * Workspace: csa_workspace_size() with CSA_WS_INDEX_TOPK or CSA_WS_INDEX_TOPK_BF16.
  */
 csa_status csa_index_topk_paged(const csa_params* p, int32_t B, int32_t T,
-                                const csa_paged_kv* keys, const void* qI, const float* w,
-                                const int64_t* q_pos, int32_t bf16_scores, int32_t* out_idx,
-                                void* out_scores, void* ws, size_t ws_bytes, void* stream);
+                                const csa_paged_kv* keys, const void* qI, const void* qI_scale,
+                                const float* w, const int64_t* q_pos, int32_t bf16_scores,
+                                int32_t* out_idx, void* out_scores, void* ws, size_t ws_bytes,
+                                void* stream);
 
 /*
  * The CSA layer over the state cache's paged caches: csa_index_topk_paged on `keys`
  * (optionally with BF16 index scores), then the sparse MQA over `kv` (bf16 or mixed rows,
  * as csa_sparse_mqa_paged), in one call with the decode chain of csa_forward. io = bf16 for
- * q [B, T, H, c], the window and out; qI bf16 [B, T, 64, 128]; w f32 [B, T, 64]. Both pools
+ * q [B, T, H, c], the window and out; qI (and qI_scale for MXFP4 keys) as for
+ * csa_index_topk_paged with keys->fmt; w f32 [B, T, 64]. Both pools
  * cover N_cap = page_rows * max_pages entries. The window is a linear buffer with win_pos0,
  * or the state cache's ring (win_pos0 = NULL, L_raw = n_win, T = 1) as in
  * csa_sparse_mqa_paged. out_idx [B, T, k]; out_scores (fp32, or bf16 with bf16_scores) may
@@ -349,7 +358,8 @@ csa_status csa_index_topk_paged(const csa_params* p, int32_t B, int32_t T,
  */
 csa_status csa_forward_paged(const csa_params* p, int32_t B, int32_t T, const csa_paged_kv* kv,
                              const csa_paged_kv* keys, int32_t bf16_scores, const void* qI,
-                             const float* w, const void* q, const void* q_rms_w,
+                             const void* qI_scale, const float* w, const void* q,
+                             const void* q_rms_w,
                              const int64_t* q_pos, const void* win_kv, int64_t L_raw,
                              const int64_t* win_pos0, const float* sink, int32_t* out_idx,
                              void* out_scores, void* out, void* ws, size_t ws_bytes,
@@ -459,10 +469,11 @@ void csa_set_index_timing_events(void* const* before, void* const* after, int32_
  * Error word of the tensor-core kernels: every wait inside them is bounded (about a second);
  * a wait that runs out stores a nonzero code (the first one wins) and the kernel returns
  * early instead of hanging. csa_state_append also leaves a code for a request it skipped.
- * Codes by kernel family: 101-106 MXFP4 indexer, 201-205 attention (205: a page id outside
- * the pool), 301-309 FP8 / bf16 indexer (309: a page id outside the pool), 321-323 state
- * append, 331 paged compression, 401-405 prefill output projection. Writes the code to *code (0 = none) and clears
- * it. Synchronises the device. Returns CSA_ERR_CUDA if the copy fails.
+ * Codes by kernel family: 101-107 MXFP4 indexer (107: a page id outside the pool), 201-205
+ * attention (205: a page id outside the pool), 301-309 FP8 / bf16 indexer (309: a page id
+ * outside the pool), 321-323 state append, 331 paged compression, 401-405 prefill output
+ * projection. Writes the code to *code (0 = none) and clears it. Synchronises the device.
+ * Returns CSA_ERR_CUDA if the copy fails.
  */
 csa_status csa_device_error(int32_t* code);
 

@@ -100,10 +100,10 @@ _SIGS = {
     "hca_dense_mqa_paged": [_PP, _I32, _I32, _VP, _VP, ctypes.POINTER(CsaPagedKv), _VP, _I64,
                             _VP, _VP, _VP, _VP, _VP, _SZ, _VP],
     "csa_index_topk_bf16": [_PP, ctypes.c_int, _I32, _I32, _I64] + [_VP] * 9 + [_SZ, _VP],
-    "csa_index_topk_paged": [_PP, _I32, _I32, ctypes.POINTER(CsaPagedKv), _VP, _VP, _VP, _I32,
-                             _VP, _VP, _VP, _SZ, _VP],
+    "csa_index_topk_paged": [_PP, _I32, _I32, ctypes.POINTER(CsaPagedKv), _VP, _VP, _VP, _VP,
+                             _I32, _VP, _VP, _VP, _SZ, _VP],
     "csa_forward_paged": [_PP, _I32, _I32, ctypes.POINTER(CsaPagedKv), ctypes.POINTER(CsaPagedKv),
-                          _I32] + [_VP] * 5 + [_VP, _I64] + [_VP] * 6 + [_SZ, _VP],
+                          _I32] + [_VP] * 6 + [_VP, _I64] + [_VP] * 6 + [_SZ, _VP],
     "csa_compress_paged": [_PP, ctypes.c_int, _I32, _I64, _I64] + [_VP] * 8 +
                           [_I32, ctypes.POINTER(CsaPagedKv), _VP],
     "csa_state_resume": [_PP, ctypes.c_int, _I32, _I64, _I64] + [_VP] * 8,
@@ -320,22 +320,23 @@ def hca_dense_mqa_paged(p, B, T, q, q_pos, kv: CsaPagedKv, win_kv, L_raw, win_po
     _check("hca_dense_mqa_paged", s)
 
 
-def csa_index_topk_paged(p, B, T, keys: CsaPagedKv, qI, w, q_pos, bf16_scores, out_idx,
+def csa_index_topk_paged(p, B, T, keys: CsaPagedKv, qI, qI_scale, w, q_pos, bf16_scores, out_idx,
                          out_scores, ws, ws_bytes, stream=None):
-    s = lib().csa_index_topk_paged(ctypes.byref(p), B, T, ctypes.byref(keys), _ptr(qI), _ptr(w),
-                                   _ptr(q_pos), int(bf16_scores), _ptr(out_idx), _ptr(out_scores),
-                                   _ptr(ws), ws_bytes, _stream(stream))
+    s = lib().csa_index_topk_paged(ctypes.byref(p), B, T, ctypes.byref(keys), _ptr(qI),
+                                   _ptr(qI_scale), _ptr(w), _ptr(q_pos), int(bf16_scores),
+                                   _ptr(out_idx), _ptr(out_scores), _ptr(ws), ws_bytes,
+                                   _stream(stream))
     _check("csa_index_topk_paged", s)
 
 
-def csa_forward_paged(p, B, T, kv: CsaPagedKv, keys: CsaPagedKv, bf16_scores, qI, w, q, q_rms_w,
-                      q_pos, win_kv, L_raw, win_pos0, sink, out_idx, out_scores, out, ws, ws_bytes,
-                      stream=None):
+def csa_forward_paged(p, B, T, kv: CsaPagedKv, keys: CsaPagedKv, bf16_scores, qI, qI_scale, w, q,
+                      q_rms_w, q_pos, win_kv, L_raw, win_pos0, sink, out_idx, out_scores, out, ws,
+                      ws_bytes, stream=None):
     s = lib().csa_forward_paged(ctypes.byref(p), B, T, ctypes.byref(kv), ctypes.byref(keys),
-                                int(bf16_scores), _ptr(qI), _ptr(w), _ptr(q), _ptr(q_rms_w),
-                                _ptr(q_pos), _ptr(win_kv), L_raw, _ptr(win_pos0), _ptr(sink),
-                                _ptr(out_idx), _ptr(out_scores), _ptr(out), _ptr(ws), ws_bytes,
-                                _stream(stream))
+                                int(bf16_scores), _ptr(qI), _ptr(qI_scale), _ptr(w), _ptr(q),
+                                _ptr(q_rms_w), _ptr(q_pos), _ptr(win_kv), L_raw, _ptr(win_pos0),
+                                _ptr(sink), _ptr(out_idx), _ptr(out_scores), _ptr(out), _ptr(ws),
+                                ws_bytes, _stream(stream))
     _check("csa_forward_paged", s)
 
 

@@ -626,10 +626,10 @@ csa_status csa_index_topk_bf16(const csa_params* p, csa_dtype kdt, int32_t B, in
   OPTIONAL_PTR(out_scores16);
   {
     auto ia = make_index(p, kdt, B, T, N_cap, qI, qI_scale, w, KI, KI_scale, q_pos, nullptr);
-    if (N_cap > 0 && !csa::index_bf16_tc_supported(ia))
+    if (N_cap > 0 && !csa::index_bf16_tc_supported(ia) && !csa::index_mxf4_tc_supported(ia))
       return fail(CSA_ERR_UNSUPPORTED,
-                  "BF16 index scores come from the tensor-core FP8 / bf16 indexer (64 heads of "
-                  "128, N_cap a multiple of 128)");
+                  "BF16 index scores come from the tensor-core indexers (MXFP4, FP8 or bf16 "
+                  "keys; 64 heads of 128, N_cap a multiple of 128)");
   }
   const size_t need = csa_workspace_size(p, CSA_WS_INDEX_TOPK_BF16, kdt, B, T, N_cap);
   if (ws == nullptr || ws_bytes < need || !aligned16(ws))
@@ -645,38 +645,58 @@ csa_status csa_index_topk_bf16(const csa_params* p, csa_dtype kdt, int32_t B, in
   return ok();
 }
 
-csa_status csa_index_topk_paged(const csa_params* p, int32_t B, int32_t T,
-                                const csa_paged_kv* keys, const void* qI, const float* w,
-                                const int64_t* q_pos, int32_t bf16_scores, int32_t* out_idx,
-                                void* out_scores, void* ws, size_t ws_bytes, void* stream) {
-  TRY(check_params(p));
-  TRY(check_topk(p));
+namespace {
+
+// the paged indexer-key descriptor: its format and pool sizes
+csa_status check_paged_keys(const csa_paged_kv* keys) {
   REQUIRE(keys != nullptr, "paged key descriptor is NULL");
-  REQUIRE(keys->fmt == CSA_BF16 || keys->fmt == CSA_FP8_E4M3_ROWSCALE,
-          "paged indexer keys must be CSA_BF16 or CSA_FP8_E4M3_ROWSCALE");
+  REQUIRE(keys->fmt == CSA_BF16 || keys->fmt == CSA_FP8_E4M3_ROWSCALE || keys->fmt == CSA_MXFP4,
+          "paged indexer keys must be CSA_BF16, CSA_FP8_E4M3_ROWSCALE or CSA_MXFP4");
   REQUIRE(keys->n_pages >= 1 && keys->max_pages >= 1 && keys->page_rows >= 1,
           "n_pages, page_rows and max_pages must be >= 1");
-  REQUIRE((int64_t)keys->page_rows * keys->max_pages <= INT32_MAX, "page_rows * max_pages too large");
-  REQUIRE(bf16_scores == 0 || bf16_scores == 1, "bf16_scores must be 0 or 1");
+  REQUIRE((int64_t)keys->page_rows * keys->max_pages <= INT32_MAX,
+          "page_rows * max_pages too large");
   REQUIRE_PTR(keys->page_table);
+  return CSA_OK;
+}
+
+// the tensor-core indexer that reads paged keys of this format, or CSA_ERR_UNSUPPORTED
+csa_status check_paged_index(const csa_params* p, const csa_paged_kv* keys, int32_t B,
+                             int32_t T, const void* qI, const void* qI_scale, const float* w,
+                             const int64_t* q_pos) {
+  const int64_t N_cap = (int64_t)keys->page_rows * keys->max_pages;
+  auto ia = make_index(p, keys->fmt, B, T, N_cap, qI, qI_scale, w, keys->pages, keys->scales,
+                       q_pos, nullptr);
+  ia.page_table = keys->page_table;
+  ia.page_rows = keys->page_rows;
+  ia.max_pages = keys->max_pages;
+  ia.n_pages = keys->n_pages;
+  if (!csa::index_bf16_tc_supported(ia) && !csa::index_mxf4_tc_supported(ia))
+    return fail(CSA_ERR_UNSUPPORTED,
+                "paged keys are read by the tensor-core indexers (64 heads of 128, page_rows a "
+                "multiple of 128)");
+  return CSA_OK;
+}
+
+}  // namespace
+
+csa_status csa_index_topk_paged(const csa_params* p, int32_t B, int32_t T,
+                                const csa_paged_kv* keys, const void* qI, const void* qI_scale,
+                                const float* w, const int64_t* q_pos, int32_t bf16_scores,
+                                int32_t* out_idx, void* out_scores, void* ws, size_t ws_bytes,
+                                void* stream) {
+  TRY(check_params(p));
+  TRY(check_topk(p));
+  TRY(check_paged_keys(keys));
+  REQUIRE(bf16_scores == 0 || bf16_scores == 1, "bf16_scores must be 0 or 1");
   const int64_t N_cap = (int64_t)keys->page_rows * keys->max_pages;
   const csa_dtype kdt = keys->fmt;
-  TRY(check_index_args(p, kdt, B, T, N_cap, qI, nullptr, w, keys->pages, keys->scales, q_pos));
+  if (kdt != CSA_MXFP4) REQUIRE(qI_scale == nullptr, "qI_scale is for MXFP4 queries only");
+  TRY(check_index_args(p, kdt, B, T, N_cap, qI, qI_scale, w, keys->pages, keys->scales, q_pos));
   if ((int64_t)B * T == 0) return ok();
   REQUIRE_PTR(out_idx);
   OPTIONAL_PTR(out_scores);
-  {
-    auto ia = make_index(p, kdt, B, T, N_cap, qI, nullptr, w, keys->pages, keys->scales, q_pos,
-                         nullptr);
-    ia.page_table = keys->page_table;
-    ia.page_rows = keys->page_rows;
-    ia.max_pages = keys->max_pages;
-    ia.n_pages = keys->n_pages;
-    if (!csa::index_bf16_tc_supported(ia))
-      return fail(CSA_ERR_UNSUPPORTED,
-                  "paged keys are read by the tensor-core FP8 / bf16 indexer (64 heads of 128, "
-                  "page_rows a multiple of 128)");
-  }
+  TRY(check_paged_index(p, keys, B, T, qI, qI_scale, w, q_pos));
   const int entry = bf16_scores ? CSA_WS_INDEX_TOPK_BF16 : CSA_WS_INDEX_TOPK;
   const size_t need = csa_workspace_size(p, entry, kdt, B, T, N_cap);
   if (ws == nullptr || ws_bytes < need || !aligned16(ws))
@@ -690,7 +710,7 @@ csa_status csa_index_topk_paged(const csa_params* p, int32_t B, int32_t T,
   t.out_idx = out_idx;
   if (bf16_scores) t.scores16 = sc;
   else t.scores = static_cast<float*>(sc);
-  TRY(index_then_topk(p, kdt, B, T, N_cap, qI, nullptr, w, keys->pages, keys->scales, q_pos,
+  TRY(index_then_topk(p, kdt, B, T, N_cap, qI, qI_scale, w, keys->pages, keys->scales, q_pos,
                       bf16_scores ? nullptr : static_cast<float*>(sc), t, base + sb, need - sb,
                       (cudaStream_t)stream, bf16_scores ? sc : nullptr, keys));
   return ok();
@@ -787,8 +807,9 @@ csa_status paged_layout(const csa_paged_kv* kv, KvLayout* out, int64_t* N_cap) {
   REQUIRE_PTR(kv->pages);
   REQUIRE_PTR(kv->page_table);
   if (kv->fmt == CSA_MIXED_FP8_BF16) REQUIRE_PTR(kv->scales);
-  *out = KvLayout{kv->fmt == CSA_MIXED_FP8_BF16, kv->pages, kv->scales, kv->page_table,
-                  kv->n_pages, kv->page_rows, kv->max_pages};
+  *out = KvLayout{kv->fmt == CSA_MIXED_FP8_BF16, kv->pages,
+                  static_cast<const float*>(kv->scales), kv->page_table, kv->n_pages,
+                  kv->page_rows, kv->max_pages};
   *N_cap = (int64_t)kv->page_rows * kv->max_pages;
   return CSA_OK;
 }
@@ -901,7 +922,8 @@ csa_status csa_forward(const csa_params* p, csa_dtype io, int32_t B, int32_t T,
 
 csa_status csa_forward_paged(const csa_params* p, int32_t B, int32_t T, const csa_paged_kv* kv,
                              const csa_paged_kv* keys, int32_t bf16_scores, const void* qI,
-                             const float* w, const void* q, const void* q_rms_w,
+                             const void* qI_scale, const float* w, const void* q,
+                             const void* q_rms_w,
                              const int64_t* q_pos, const void* win_kv, int64_t L_raw,
                              const int64_t* win_pos0, const float* sink, int32_t* out_idx,
                              void* out_scores, void* out, void* ws, size_t ws_bytes,
@@ -913,33 +935,18 @@ csa_status csa_forward_paged(const csa_params* p, int32_t B, int32_t T, const cs
   KvLayout lay;
   int64_t N_cap = 0;
   TRY(paged_layout(kv, &lay, &N_cap));
-  REQUIRE(keys != nullptr, "paged key descriptor is NULL");
-  REQUIRE(keys->fmt == CSA_BF16 || keys->fmt == CSA_FP8_E4M3_ROWSCALE,
-          "paged indexer keys must be CSA_BF16 or CSA_FP8_E4M3_ROWSCALE");
-  REQUIRE(keys->n_pages >= 1 && keys->page_rows >= 1 && keys->max_pages >= 1,
-          "n_pages, page_rows and max_pages must be >= 1");
+  TRY(check_paged_keys(keys));
   REQUIRE((int64_t)keys->page_rows * keys->max_pages == N_cap,
           "the KV and key pools must cover the same entries (page_rows * max_pages)");
-  REQUIRE_PTR(keys->page_table);
+  if (keys->fmt != CSA_MXFP4) REQUIRE(qI_scale == nullptr, "qI_scale is for MXFP4 queries only");
   TRY(check_mqa_args(p, CSA_BF16, B, T, q, q_pos, kv->pages, N_cap, win_kv, L_raw, win_pos0, sink,
                      q_rms_w, out, true));
-  TRY(check_index_args(p, keys->fmt, B, T, N_cap, qI, nullptr, w, keys->pages, keys->scales,
+  TRY(check_index_args(p, keys->fmt, B, T, N_cap, qI, qI_scale, w, keys->pages, keys->scales,
                        q_pos));
   if ((int64_t)B * T == 0) return ok();
   REQUIRE_PTR(out_idx);
   OPTIONAL_PTR(out_scores);
-  {
-    auto ia = make_index(p, keys->fmt, B, T, N_cap, qI, nullptr, w, keys->pages, keys->scales,
-                         q_pos, nullptr);
-    ia.page_table = keys->page_table;
-    ia.page_rows = keys->page_rows;
-    ia.max_pages = keys->max_pages;
-    ia.n_pages = keys->n_pages;
-    if (!csa::index_bf16_tc_supported(ia))
-      return fail(CSA_ERR_UNSUPPORTED,
-                  "paged keys are read by the tensor-core FP8 / bf16 indexer (64 heads of 128, "
-                  "page_rows a multiple of 128)");
-  }
+  TRY(check_paged_index(p, keys, B, T, qI, qI_scale, w, q_pos));
   auto ma = make_mqa(p, B, T, q, q_pos, kv->pages, N_cap, out_idx, p->topk, win_kv, L_raw,
                      win_pos0, sink, q_rms_w, out);
   const bool rope_ok = !lay.mixed ||
@@ -981,7 +988,7 @@ csa_status csa_forward_paged(const csa_params* p, int32_t B, int32_t T, const cs
       t.qj.inv_freq[i] = csa::rope_inv_freq(i, p->rope_dims, (double)p->rope_base);
     ma.qhat = t.qj.qhat;
   }
-  TRY(index_then_topk(p, keys->fmt, B, T, N_cap, qI, nullptr, w, keys->pages, keys->scales,
+  TRY(index_then_topk(p, keys->fmt, B, T, N_cap, qI, qI_scale, w, keys->pages, keys->scales,
                       q_pos, bf16_scores ? nullptr : static_cast<float*>(sc), t, base + sb, tb,
                       st, bf16_scores ? sc : nullptr, keys));
   TRY(cuda_status(csa::launch_mqa(ma, true, base + sb + tb, mb, st), "sparse MQA (paged)"));

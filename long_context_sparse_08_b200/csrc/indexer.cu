@@ -122,15 +122,15 @@ __global__ void __launch_bounds__(kKeysPerCta) k_index_scores_cc(IndexArgs a) {
 cudaError_t launch_index_scores(const IndexArgs& a, cudaStream_t st, bool* hist_done) {
   if (hist_done) *hist_done = false;
   if (a.B == 0 || a.T == 0 || a.n_cap == 0) return cudaSuccess;
+  if (index_mxf4_tc_supported(a)) {  // MXFP4 keys (contiguous or paged; fp32 or bf16 scores)
+    if (hist_done) *hist_done = a.hist != nullptr;
+    return launch_index_mxf4_tc(a, st);
+  }
   if (a.scores16 != nullptr || a.page_table != nullptr) {
-    // BF16 index scores or paged keys: the FP8 / bf16 tensor-core kernel only
+    // BF16 index scores or paged keys otherwise: the FP8 / bf16 tensor-core kernel only
     if (!index_bf16_tc_supported(a)) return cudaErrorNotSupported;
     if (hist_done) *hist_done = a.hist != nullptr;
     return launch_index_bf16_tc(a, st);
-  }
-  if (index_mxf4_tc_supported(a)) {
-    if (hist_done) *hist_done = a.hist != nullptr;
-    return launch_index_mxf4_tc(a, st);
   }
   if (index_bf16_tc_supported(a)) {
     if (hist_done) *hist_done = a.hist != nullptr;

@@ -74,7 +74,7 @@ __device__ __forceinline__ uint32_t sfa_col(int hs, int j) { return 256u + 16u *
 __device__ __forceinline__ uint32_t sfb_col(int qs, int h) { return 288u + 16u * qs + 8u * h; }
 
 enum { kErrFull = 101, kErrEmpty = 102, kErrTmemFull = 103, kErrTmemEmpty = 104,
-       kErrQFull = 105, kErrQEmpty = 106 };
+       kErrQFull = 105, kErrQEmpty = 106, kErrPageId = 107 };
 
 struct Mxf4Params {
   int Q, T, m;
@@ -83,6 +83,15 @@ struct Mxf4Params {
   const float* w;
   float* scores;
   int* hist;  // optional [Q][4096] histogram of the scores' top 12 key bits
+};
+
+// The variants' extra inputs (a separate kernel parameter, so the plain kernel's stays as is)
+struct Mxf4Ext {
+  __nv_bfloat16* scores16;    // kB16: the scores rounded once to bf16, stored instead
+  const int32_t* page_table;  // kPaged: keys and their scale blocks in a page pool; key e of
+                              // request b is row e % page_rows of page
+                              // page_table[b * max_pages + e / page_rows]
+  int page_rows, max_pages, n_pages;  // page_rows a multiple of 128
 };
 
 struct Smem {
@@ -117,10 +126,14 @@ __device__ __forceinline__ bool epi_all_ok(bool ok) {
 }
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 2, 256;" ::: "memory"); }
 
-__global__ void __launch_bounds__(kThreads, 1)
-    k_index_mxf4_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_ks,
-                    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qs,
-                    Mxf4Params p) {
+// The kernel body. kPaged: each 128-key block of a unit is its own TMA box, read through the
+// page table (tm_k / tm_ks then cover the pool with one-block boxes); a block past the
+// query's visible keys reads pool block 0 and is masked like any invisible key, and a page id
+// outside the pool records kErrPageId and reads block 0. kB16: bf16 score stores.
+template <bool kPaged, bool kB16>
+__device__ __forceinline__ void index_mxf4_body(const CUtensorMap& tm_k, const CUtensorMap& tm_ks,
+                                                const CUtensorMap& tm_q, const CUtensorMap& tm_qs,
+                                                const Mxf4Params& p, const Mxf4Ext& x) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -219,11 +232,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         uint8_t* sb = base + st * kStageBytes;
         const int b = q / p.T;
-        // keys and scales are viewed in 128-key blocks; a unit is 4 consecutive blocks
-        const int32_t blk0 = (int32_t)((b * p.n_cap + (int64_t)unit * kUnitKeys) / kTileKeys);
-        mbar_arrive_expect_tx(&S.full[st], kStageTx);
-        tma_load_3d(sb + kOffA, &tm_k, 0, 0, blk0, &S.full[st]);
-        tma_load_2d(sb + kOffSF, &tm_ks, 0, blk0, &S.full[st]);
+        if constexpr (kPaged) {
+          mbar_arrive_expect_tx(&S.full[st], kStageTx);
+#pragma unroll 1
+          for (int j = 0; j < kUnitTiles; ++j) {
+            const int64_t e = (int64_t)unit * kUnitKeys + j * kTileKeys;  // block's first key
+            int32_t blk = 0;
+            if (e < S.nvis[q]) {
+              const int32_t pg = x.page_table[(size_t)b * x.max_pages + e / x.page_rows];
+              if (pg >= 0 && pg < x.n_pages)
+                blk = (int32_t)(((int64_t)pg * x.page_rows + e % x.page_rows) / kTileKeys);
+              else
+                set_error(kErrPageId);
+            }
+            tma_load_3d(sb + kOffA + j * (kTileKeys * kRowBytes), &tm_k, 0, 0, blk, &S.full[st]);
+            tma_load_2d(sb + kOffSF + j * (kTileKeys * 4), &tm_ks, 0, blk, &S.full[st]);
+          }
+        } else {
+          // keys and scales are viewed in 128-key blocks; a unit is 4 consecutive blocks
+          const int32_t blk0 =
+              (int32_t)((b * p.n_cap + (int64_t)unit * kUnitKeys) / kTileKeys);
+          mbar_arrive_expect_tx(&S.full[st], kStageTx);
+          tma_load_3d(sb + kOffA, &tm_k, 0, 0, blk0, &S.full[st]);
+          tma_load_2d(sb + kOffSF, &tm_ks, 0, blk0, &S.full[st]);
+        }
       }
       // drain: no copy into this CTA's shared memory may still be in flight at exit
       for (int j = (k > kStages ? k - kStages : 0); j < k; ++j)
@@ -348,8 +380,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float sc = (part[0] + part[1]) + (part[2] + part[3]);
         const int s = unit * kUnitKeys + t * kTileKeys + 32 * quad + lane;
         if (s < S.nvis[q]) {
-          p.scores[(size_t)q * p.n_cap + s] = sc;
-          if (hist) atomicAdd(&S.hist[float_key(sc) >> 20], 1);
+          if constexpr (kB16) {  // BF16 index scores: round once, select on the rounded value
+            const __nv_bfloat16 r = __float2bfloat16_rn(sc);
+            x.scores16[(size_t)q * p.n_cap + s] = r;
+            if (hist) atomicAdd(&S.hist[float_key(__bfloat162float(r)) >> 20], 1);
+          } else {
+            p.scores[(size_t)q * p.n_cap + s] = sc;
+            if (hist) atomicAdd(&S.hist[float_key(sc) >> 20], 1);
+          }
         }
       }
     }
@@ -361,6 +399,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_index_mxf4_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_ks,
+                    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qs,
+                    Mxf4Params p) {
+  index_mxf4_body<false, false>(tm_k, tm_ks, tm_q, tm_qs, p, Mxf4Ext{});
+}
+
+// paged keys and / or BF16 index scores
+template <bool kPaged, bool kB16>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_index_mxf4_ext(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_ks,
+                     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qs,
+                     Mxf4Params p, Mxf4Ext x) {
+  index_mxf4_body<kPaged, kB16>(tm_k, tm_ks, tm_q, tm_qs, p, x);
 }
 
 // ---- host: tensor maps ----
@@ -378,27 +432,28 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// keys as [128-key blocks][128 rows][64 B], box = 4 blocks (one 512-key unit)
-bool make_map_keys(CUtensorMap* m, const void* ptr, uint64_t rows) {
+// keys as [128-key blocks][128 rows][64 B], box = `blocks` blocks (4: one 512-key unit;
+// 1: one block, for page pools)
+bool make_map_keys(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t blocks) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)kRowBytes, (cuuint64_t)kTileKeys,
                         (cuuint64_t)(rows / kTileKeys)};
   cuuint64_t strides[2] = {(cuuint64_t)kRowBytes, (cuuint64_t)kRowBytes * kTileKeys};
-  cuuint32_t box[3] = {(cuuint32_t)kRowBytes, (cuuint32_t)kTileKeys, (cuuint32_t)kUnitTiles};
+  cuuint32_t box[3] = {(cuuint32_t)kRowBytes, (cuuint32_t)kTileKeys, blocks};
   cuuint32_t es[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// key scale words as [128-key blocks][128 words], box = 4 blocks
-bool make_map_key_scales(CUtensorMap* m, const void* ptr, uint64_t rows) {
+// key scale words as [128-key blocks][128 words], box = `blocks` blocks
+bool make_map_key_scales(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t blocks) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)kTileKeys, (cuuint64_t)(rows / kTileKeys)};
   cuuint64_t strides[1] = {(cuuint64_t)kTileKeys * 4};
-  cuuint32_t box[2] = {(cuuint32_t)kTileKeys, (cuuint32_t)kUnitTiles};
+  cuuint32_t box[2] = {(cuuint32_t)kTileKeys, blocks};
   cuuint32_t es[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(ptr), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -443,15 +498,36 @@ int num_sms() {
 }  // namespace
 
 bool index_mxf4_tc_supported(const IndexArgs& a) {
+  const bool rows_ok = a.page_table == nullptr
+                           ? (int64_t)a.B * a.n_cap < (1ll << 31)
+                           : a.page_rows > 0 && a.page_rows % kTileKeys == 0 && a.n_pages > 0 &&
+                                 (int64_t)a.n_pages * a.page_rows < (1ll << 31);
   return a.kdt == CSA_MXFP4 && a.n_idx_heads == kHeads && a.d_idx == 128 && a.n_cap % 128 == 0 &&
-         (int64_t)a.B * a.T <= kMaxQueries && (int64_t)a.B * a.n_cap < (1ll << 31);
+         (int64_t)a.B * a.T <= kMaxQueries && rows_ok;
 }
+
+namespace {
+template <bool kPaged, bool kB16>
+cudaError_t launch_ext(const CUtensorMap& mk, const CUtensorMap& mks, const CUtensorMap& mq,
+                       const CUtensorMap& mqs, const Mxf4Params& p, const Mxf4Ext& x, int grid,
+                       size_t smem, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(k_index_mxf4_ext<kPaged, kB16>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch(true, k_index_mxf4_ext<kPaged, kB16>, dim3(grid), dim3(kThreads), smem, st, mk,
+                mks, mq, mqs, p, x);
+}
+}  // namespace
 
 cudaError_t launch_index_mxf4_tc(const IndexArgs& a, cudaStream_t st) {
   const int Q = a.B * a.T;
+  const bool paged = a.page_table != nullptr, b16 = a.scores16 != nullptr;
+  // keys: the contiguous cache [B, n_cap] in 4-block boxes, or the pool in 1-block boxes
+  const uint64_t key_rows = paged ? (uint64_t)a.n_pages * a.page_rows : (uint64_t)a.B * a.n_cap;
+  const uint32_t blocks = paged ? 1u : (uint32_t)kUnitTiles;
   CUtensorMap mk, mks, mq, mqs;
-  if (!make_map_keys(&mk, a.KI, (uint64_t)a.B * a.n_cap) ||
-      !make_map_key_scales(&mks, a.KI_scale, (uint64_t)a.B * a.n_cap) ||
+  if (!make_map_keys(&mk, a.KI, key_rows, blocks) ||
+      !make_map_key_scales(&mks, a.KI_scale, key_rows, blocks) ||
       !make_map_2d(&mq, a.qI, (uint64_t)Q * kHeads, kHeads) ||
       !make_map_1d_words(&mqs, a.qI_scale, (uint64_t)Q * kHeads, kHeads))
     return cudaErrorInvalidValue;
@@ -459,6 +535,17 @@ cudaError_t launch_index_mxf4_tc(const IndexArgs& a, cudaStream_t st) {
   const int64_t units_max = (int64_t)Q * ((a.n_cap + kUnitKeys - 1) / kUnitKeys);
   const int grid = (int)(units_max < num_sms() ? (units_max > 0 ? units_max : 1) : num_sms());
   const size_t smem = 1024 + (size_t)kStages * kStageBytes + 2 * kQBytes + sizeof(Smem);
+  if (paged || b16) {
+    const Mxf4Ext x{static_cast<__nv_bfloat16*>(a.scores16), a.page_table, a.page_rows,
+                    a.max_pages, a.n_pages};
+    timing_before(st);
+    const cudaError_t e =
+        paged ? (b16 ? launch_ext<true, true>(mk, mks, mq, mqs, p, x, grid, smem, st)
+                     : launch_ext<true, false>(mk, mks, mq, mqs, p, x, grid, smem, st))
+              : launch_ext<false, true>(mk, mks, mq, mqs, p, x, grid, smem, st);
+    timing_after(st);
+    return e;
+  }
   cudaError_t e = cudaFuncSetAttribute(k_index_mxf4_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;

@@ -319,9 +319,9 @@ def test_paged_index_checks():
     L = csa.lib()
     p = _p(topk=512)
 
-    def call(kv, bf16=0):
-        return L.csa_index_topk_paged(ctypes.byref(p), 2, 1, ctypes.byref(kv), FAKE, FAKE, FAKE,
-                                      bf16, FAKE, None, FAKE, 1 << 30, None)
+    def call(kv, bf16=0, qs=None):
+        return L.csa_index_topk_paged(ctypes.byref(p), 2, 1, ctypes.byref(kv), FAKE, qs, FAKE,
+                                      FAKE, bf16, FAKE, None, FAKE, 1 << 30, None)
 
     assert call(csa.CsaPagedKv(csa.CSA_FP8_E4M3_ROWSCALE, FAKE, FAKE, FAKE, 64, 32, 16)) == \
         csa.CSA_ERR_UNSUPPORTED  # 32-row pages split a 128-key tile
@@ -333,6 +333,15 @@ def test_paged_index_checks():
         csa.CSA_ERR_INVALID_ARG  # FP8 keys without their scales
     assert call(csa.CsaPagedKv(csa.CSA_BF16, FAKE, None, FAKE, 64, 128, 4), bf16=2) == \
         csa.CSA_ERR_INVALID_ARG
+    # MXFP4 keys: the queries' scales are required, other formats take none
+    assert call(csa.CsaPagedKv(csa.CSA_MXFP4, FAKE, FAKE, FAKE, 64, 128, 4)) == \
+        csa.CSA_ERR_INVALID_ARG  # MXFP4 queries without their scales
+    assert call(csa.CsaPagedKv(csa.CSA_MXFP4, FAKE, None, FAKE, 64, 128, 4), qs=FAKE) == \
+        csa.CSA_ERR_INVALID_ARG  # MXFP4 keys without their exponent blocks
+    assert call(csa.CsaPagedKv(csa.CSA_MXFP4, FAKE, FAKE, FAKE, 64, 64, 8), qs=FAKE) == \
+        csa.CSA_ERR_UNSUPPORTED  # 64-row pages split a 128-key scale block
+    assert call(csa.CsaPagedKv(csa.CSA_BF16, FAKE, None, FAKE, 64, 128, 4), qs=FAKE) == \
+        csa.CSA_ERR_INVALID_ARG  # bf16 queries carry no scales
 
 
 def test_prefill_handover_checks():

@@ -1,4 +1,5 @@
-"""BF16 index scores into the top-k selector (csa_index_topk_bf16) against the oracle.
+"""BF16 index scores into the top-k selector (csa_index_topk_bf16; FP8, bf16 and MXFP4 keys)
+against the oracle.
 
 The scores are computed in fp32 and rounded once to bf16; the selector orders the bf16
 values by (value desc, index asc). Checks:
@@ -26,7 +27,8 @@ from oracle import csa_oracle as O
 from oracle import pipeline as P
 import tests.parity_util as U
 
-CASES = ["edge_decode_fp8_tc", "edge_decode_bf16_tc", "mid_decode_fp8", "mid_prefill_bf16_tc"]
+CASES = ["edge_decode_fp8_tc", "edge_decode_bf16_tc", "mid_decode_fp8", "mid_prefill_bf16_tc",
+         "edge_decode_mxfp4", "mid_decode_mxfp4"]
 
 
 def test_checks_on_the_host():

@@ -1,8 +1,8 @@
 """Attention over other KV cache layouts against the float64 oracle on the same bytes:
 mixed-precision rows (csa_sparse_mqa_mixed_kv, hca_dense_mqa_mixed_kv) and paged caches
 (csa_sparse_mqa_paged, hca_dense_mqa_paged); and the indexer over paged keys
-(csa_index_topk_paged), which must give exactly the scores and selection of the contiguous
-keys.
+(csa_index_topk_paged: FP8, bf16 and MXFP4 keys), which must give exactly the scores and
+selection of the contiguous keys.
 
 For mixed rows the workloads' bf16 caches are re-encoded by the input encoder (the first
 c - r values as e4m3 with a row scale, the RoPE values as bf16); the oracle decodes those
@@ -188,9 +188,13 @@ def test_paged_cache_with_a_bad_page_id_reports_it():
 
 
 @pytest.mark.parametrize("name", ["edge_decode_fp8_tc", "edge_decode_bf16_tc",
-                                  "mid_prefill_bf16_tc"])
+                                  "mid_prefill_bf16_tc", "edge_decode_mxfp4",
+                                  "edge_decode_mxfp4_long"])
 @pytest.mark.parametrize("bf16_scores", [0, 1])
-def test_index_topk_over_paged_keys_equals_contiguous(name, bf16_scores):
+@pytest.mark.parametrize("holes", [False, True], ids=["all_pages", "unallocated_tail"])
+def test_index_topk_over_paged_keys_equals_contiguous(name, bf16_scores, holes):
+    """With `holes`, the table entries of pages past a request's visible keys are -1 (pages
+    not yet allocated): the indexer must not read them, nor report a bad page id."""
     s, inp = U.inputs(name)
     dev = R.upload(inp, s)
     p = R.params_for(s)
@@ -203,12 +207,17 @@ def test_index_topk_over_paged_keys_equals_contiguous(name, bf16_scores):
     idx_c = torch.empty((B, T, s.topk), dtype=torch.int32, device="cuda")
     sc_c = torch.zeros((B, T, N), dtype=sdt, device="cuda")
     if bf16_scores:
-        csa.csa_index_topk_bf16(p, kdt, B, T, N, dev["qI"], None, dev["w"], dev["KI"],
-                                dev.get("KI_scale"), dev["q_pos"], idx_c, sc_c, ws, need)
+        csa.csa_index_topk_bf16(p, kdt, B, T, N, dev["qI"], dev.get("qI_scale"), dev["w"],
+                                dev["KI"], dev.get("KI_scale"), dev["q_pos"], idx_c, sc_c, ws,
+                                need)
     else:
-        csa.csa_index_topk(p, kdt, B, T, N, dev["qI"], None, dev["w"], dev["KI"],
+        csa.csa_index_topk(p, kdt, B, T, N, dev["qI"], dev.get("qI_scale"), dev["w"], dev["KI"],
                            dev.get("KI_scale"), dev["q_pos"], idx_c, sc_c, ws, need)
     pool, table = _paged(inp["KI"], 128, 6)
+    if holes:
+        for b in range(B):
+            nv = int(max(0, min(int(inp["q_pos"][b].max()) // s.m, N)))
+            table[b, -(-nv // 128):] = -1
     scales = None
     if "KI_scale" in inp:
         spool, _ = _paged(inp["KI_scale"][..., None], 128, 6)
@@ -218,8 +227,8 @@ def test_index_topk_over_paged_keys_equals_contiguous(name, bf16_scores):
     sc_p = torch.zeros_like(sc_c)
     torch.cuda.synchronize()
     csa.device_error()
-    csa.csa_index_topk_paged(p, B, T, keys, dev["qI"], dev["w"], dev["q_pos"], bf16_scores, idx_p,
-                             sc_p, ws, need)
+    csa.csa_index_topk_paged(p, B, T, keys, dev["qI"], dev.get("qI_scale"), dev["w"],
+                             dev["q_pos"], bf16_scores, idx_p, sc_p, ws, need)
     torch.cuda.synchronize()
     assert csa.device_error() == 0
     assert torch.equal(idx_p, idx_c)
@@ -259,14 +268,16 @@ def _paged_forward(s, inp, dev, kv_fmt, kv_rows, kv_scale, bf16_scores, ring=Non
     csa.device_error()
     win, L, pos0 = (dev["win_kv"], dev["win_kv"].shape[1], dev["win_pos0"]) if ring is None \
         else (ring, ring.shape[1], None)
-    csa.csa_forward_paged(p, B, T, kv, keys, bf16_scores, dev["qI"], dev["w"], dev["q"], None,
-                          dev["q_pos"], win, L, pos0, dev["sink"], idx, sc, out, ws, need)
+    csa.csa_forward_paged(p, B, T, kv, keys, bf16_scores, dev["qI"], dev.get("qI_scale"),
+                          dev["w"], dev["q"], None, dev["q_pos"], win, L, pos0, dev["sink"], idx,
+                          sc, out, ws, need)
     torch.cuda.synchronize()
     assert csa.device_error() == 0
     return out, idx, sc
 
 
-@pytest.mark.parametrize("name", ["edge_decode_fp8_tc", "edge_decode_bf16_tc"])
+@pytest.mark.parametrize("name", ["edge_decode_fp8_tc", "edge_decode_bf16_tc",
+                                  "edge_decode_mxfp4"])
 def test_forward_paged_equals_contiguous(name):
     s, inp = U.inputs(name)
     dev = R.upload(inp, s)
