@@ -1,0 +1,252 @@
+"""A decode step over the state cache, end to end, against the float64 oracle.
+
+Three requests feed their tokens one at a time to csa_state_append: the KV entries go into
+pages of 32 entries (bf16), the compressed indexer keys into pages of 128 keys (MXFP4, the
+FP4 indexer cache of 【论文解读】DeepSeek-V4 二(四) and 二(六)) and the window rows into the
+ring. One csa_forward_paged call at every request's last position then runs index -> top-k
+-> sparse MQA over the pools. Page tables are shuffled, and the entries of pages nothing has
+been written to yet are -1.
+
+The oracle feeds the same raw rows through its own state cache (oracle/state_cache.py),
+stores the finished entries with the input encoders (bf16; MXFP4), and runs its indexer and
+attention on those. Checks:
+  - KV pages: every entry within one bf16 rounding of the oracle's;
+  - key pages: the MXFP4 bytes equal the encoder's bytes of the oracle's keys, except where
+    the fp32 key lies within fp32 error of an e2m1 / exponent rounding boundary (at most 1%
+    of the keys; such keys are left out of the score checks);
+  - index scores within 1e-4 of the sum of the magnitudes of their terms (BF16 scores: plus
+    one bf16 rounding);
+  - the selection: valid for the scores the GPU stored, and equal to the oracle's except at
+    near-ties of the k-th score;
+  - the output: the oracle's attention over the GPU's selection, within the bf16 output
+    tolerance.
+The N_cap = 8192 case takes the decode top-k (histogram filled by the indexer), 1024 the
+row top-k. Not yet run on a B200: the module runs only with CSA_RUN_FIRST_GPU_CHECKS=1.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import csa_oracle as O
+from oracle import state_cache as SC
+from long_context_sparse_08_b200 import workloads as W
+import tests.parity_util as U
+
+pytestmark = [
+    pytest.mark.gpu,
+    pytest.mark.skipif(os.environ.get("CSA_RUN_FIRST_GPU_CHECKS") != "1",
+                       reason="awaiting its first run on a B200 (CSA_RUN_FIRST_GPU_CHECKS=1)"),
+]
+
+M, C, R, D_I, H, H_I, K, N_WIN = 4, 512, 64, 128, 64, 64, 64, 128
+BASE, EPS = 10000.0, 1e-6
+KV_ROWS, KEY_ROWS = 32, 128  # entries per page
+N_TOK = (1100, 517, 2051)    # tokens each request appends (129 visible keys: a page and one)
+
+
+class Stream:
+    """Seeded raw rows, queries and page tables of the three requests (host arrays)."""
+
+    def __init__(self, n_cap, seed=2026):
+        self.B, self.n_cap = len(N_TOK), n_cap
+        n = max(N_TOK)
+        self.kv = W.make_state_stream(B=self.B, n_tok=n, m=M, c=C, overlap=1, io="bf16",
+                                      seed=seed)
+        self.key = W.make_state_stream(B=self.B, n_tok=n, m=M, c=D_I, overlap=1, io="bf16",
+                                       seed=seed + 1)
+        g = np.random.default_rng(seed + 2)
+        self.q = W.f32_to_bf16_bits(g.standard_normal((self.B, 1, H, C), np.float32))
+        qI = g.standard_normal((self.B, 1, H_I, D_I), np.float32)
+        self.qI, self.qI_scale = W.quant_mxfp4(qI)
+        self.w = g.standard_normal((self.B, 1, H_I), np.float32)
+        self.sink = g.standard_normal((H,), np.float32)
+        self.pos = np.array([[t - 1] for t in N_TOK], np.int64)
+        self.kv_table, self.n_kv_pages = self._table(KV_ROWS, g)
+        self.key_table, self.n_key_pages = self._table(KEY_ROWS, g)
+
+    def _table(self, rows, g):
+        """Shuffled page table [B, n_cap / rows]: the pages a request's entries fill, in a
+        pool with 3 spare pages; -1 past them."""
+        max_pages = self.n_cap // rows
+        used = [-(-(t // M) // rows) for t in N_TOK]
+        n_pages = sum(used) + 3
+        perm = g.permutation(n_pages).astype(np.int32)
+        table = np.full((self.B, max_pages), -1, np.int32)
+        k = 0
+        for b, u in enumerate(used):
+            table[b, :u] = perm[k:k + u]
+            k += u
+        return table, n_pages
+
+    def n_vis(self, b):
+        return O.visible_entries(int(self.pos[b, 0]), M, self.n_cap)
+
+
+def oracle_caches(st: Stream):
+    """Per request: the oracle's KV entries (bf16-stored, decoded), its fp32-cast keys, the
+    MXFP4 bytes the encoder makes of them, and those keys decoded."""
+    out = []
+    for b, n in enumerate(N_TOK):
+        caches = []
+        for src, c, fin, rows in ((st.kv, C, True, KV_ROWS), (st.key, D_I, False, KEY_ROWS)):
+            pool = SC.PagePool(-(-(n // M) // rows) + 1, rows, c)
+            cs = SC.CsaState(pool, m=M, c=c, bias=O.dec_bf16(src["bias"]), n_win=N_WIN, r=R,
+                             base=BASE, eps=EPS, block_tokens=M * rows, finalize=fin)
+            r = {k: O.dec_bf16(src[k][b, :n]) for k in ("Ca", "Cb", "Za", "Zb", "win")}
+            for t in range(n):
+                cs.append(r["Ca"][t], r["Cb"][t], r["Za"][t], r["Zb"][t], r["win"][t])
+            caches.append(cs.entries())
+        kv, keys = caches
+        kv_bf16 = O.dec_bf16(W.f32_to_bf16_bits(kv.astype(np.float32)))
+        packed, ex = W.quant_mxfp4(keys.astype(np.float32))
+        out.append(dict(kv_f64=kv, kv=kv_bf16, keys_packed=packed, keys_ex=ex,
+                        keys=O.dec_mxfp4(packed, ex), win=O.dec_bf16(st.kv["win"][b, :n])))
+    return out
+
+
+def run_gpu(st: Stream, bf16_scores: int):
+    """The appends and the forward call; returns host copies of the pools and the results."""
+    import torch
+    import long_context_sparse_08_b200 as csa
+
+    def up(x):
+        a = np.ascontiguousarray(x)
+        return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).cuda()
+
+    torch.cuda.synchronize()
+    csa.device_error()
+    B = st.B
+    p_kv = csa.make_params(m=M, overlap=1, c=C, rope_dims=R, rope_base=BASE, rms_eps=EPS,
+                           n_heads=H, n_idx_heads=H_I, d_idx=D_I, topk=K, n_win=N_WIN)
+    p_key = csa.make_params(m=M, overlap=1, c=D_I, rope_dims=R, rope_base=BASE, rms_eps=EPS,
+                            n_win=N_WIN)
+    kv_pages = torch.zeros((st.n_kv_pages, KV_ROWS, C), dtype=torch.int16, device="cuda")
+    key_pages = torch.zeros((st.n_key_pages, KEY_ROWS, D_I // 2), dtype=torch.uint8,
+                            device="cuda")
+    key_ex = torch.zeros((st.n_key_pages, KEY_ROWS, 4), dtype=torch.uint8, device="cuda")
+    kv_state = torch.zeros((B, 2 * M, 4, C), dtype=torch.int16, device="cuda")
+    key_state = torch.zeros((B, 2 * M, 4, D_I), dtype=torch.int16, device="cuda")
+    ring = torch.zeros((B, N_WIN, C), dtype=torch.int16, device="cuda")
+    kv_table, key_table = up(st.kv_table), up(st.key_table)
+    kv_src = {k: up(st.kv[k]) for k in st.kv}
+    key_src = {k: up(st.key[k]) for k in st.key}
+    for b, n in enumerate(N_TOK):  # one request per call, its own state / ring / table rows
+        # every pointer 16-byte aligned: the position in a 16-byte row, the table row a copy
+        pos_all = torch.zeros((n, 2), dtype=torch.int64, device="cuda")
+        pos_all[:, 0] = torch.arange(n, device="cuda")
+        kv_tb, key_tb = up(st.kv_table[b:b + 1]), up(st.key_table[b:b + 1])
+        for t in range(n):
+            pos = pos_all[t, :1]
+            r = {k: v[b, t:t + 1] for k, v in kv_src.items() if k != "bias"}
+            csa.csa_state_append(p_kv, csa.CSA_BF16, 1, pos, r["Ca"], r["Cb"], r["Za"], r["Zb"],
+                                 r["win"], kv_src["bias"], None, 1, kv_state[b:b + 1],
+                                 ring[b:b + 1], csa.CSA_BF16, kv_pages, None, st.n_kv_pages,
+                                 KV_ROWS, kv_tb, kv_table.shape[1])
+            r = {k: v[b, t:t + 1] for k, v in key_src.items() if k != "bias"}
+            csa.csa_state_append(p_key, csa.CSA_BF16, 1, pos, r["Ca"], r["Cb"], r["Za"],
+                                 r["Zb"], None, key_src["bias"], None, 0, key_state[b:b + 1],
+                                 None, csa.CSA_MXFP4, key_pages, key_ex, st.n_key_pages,
+                                 KEY_ROWS, key_tb, key_table.shape[1])
+    torch.cuda.synchronize()
+    assert csa.device_error() == 0, "appends"
+    kv = csa.paged_kv(csa.CSA_BF16, kv_pages, None, kv_table, st.n_kv_pages, KV_ROWS,
+                      kv_table.shape[1])
+    keys = csa.paged_kv(csa.CSA_MXFP4, key_pages, key_ex, key_table, st.n_key_pages, KEY_ROWS,
+                        key_table.shape[1])
+    need = csa.workspace_size(p_kv, csa.CSA_WS_FORWARD, csa.CSA_MXFP4, B, 1, st.n_cap)
+    ws = torch.empty((need,), dtype=torch.uint8, device="cuda")
+    out = torch.empty((B, 1, H, C), dtype=torch.int16, device="cuda")
+    idx = torch.empty((B, 1, K), dtype=torch.int32, device="cuda")
+    sc = torch.zeros((B, 1, st.n_cap), dtype=torch.int16 if bf16_scores else torch.float32,
+                     device="cuda")
+    csa.csa_forward_paged(p_kv, B, 1, kv, keys, bf16_scores, up(st.qI), up(st.qI_scale),
+                          up(st.w), up(st.q), None, up(st.pos), ring, N_WIN, None, up(st.sink),
+                          idx, sc, out, ws, need)
+    torch.cuda.synchronize()
+    assert csa.device_error() == 0, "forward"
+    scores = sc.cpu().numpy()
+    scores = O.dec_bf16(scores.view(np.uint16)) if bf16_scores else scores.astype(np.float64)
+    return dict(kv_pages=kv_pages.cpu().numpy().view(np.uint16),
+                key_pages=key_pages.cpu().numpy(), key_ex=key_ex.cpu().numpy(),
+                idx=idx.cpu().numpy(), scores=scores,
+                out=O.dec_bf16(out.cpu().numpy().view(np.uint16)))
+
+
+def page_rows_of(table, rows, b, n):
+    """(page, slot) of entries 0 .. n-1 of request b."""
+    i = np.arange(n)
+    return table[b, i // rows], i % rows
+
+
+def check_pages(st, ora, got):
+    """KV entries within a bf16 rounding; key bytes equal except near rounding boundaries.
+    Returns, per request, the keys whose stored bytes differ from the oracle's."""
+    off = []
+    for b, n in enumerate(N_TOK):
+        o = ora[b]
+        ne = n // M
+        pg, sl = page_rows_of(st.kv_table, KV_ROWS, b, ne)
+        U.check_rows(O.dec_bf16(got["kv_pages"][pg, sl]), o["kv_f64"], "bf16",
+                     f"request {b}: KV entries")
+        pg, sl = page_rows_of(st.key_table, KEY_ROWS, b, ne)
+        packed = got["key_pages"][pg, sl]
+        ex = np.stack([O.unblock_key_scales(got["key_ex"][p])[s] for p, s in zip(pg, sl)])
+        bad = np.flatnonzero(np.any(packed != o["keys_packed"], axis=1) |
+                             np.any(ex != o["keys_ex"], axis=1))
+        assert bad.size <= max(1, ne // 100), f"request {b}: {bad.size} keys stored differently"
+        # a differing key is still the same key to within one e2m1 step of its block
+        if bad.size:
+            dq = O.dec_mxfp4(packed[bad], ex[bad])
+            step = np.repeat(np.exp2(o["keys_ex"][bad].astype(np.float64) - 126.0), 32, axis=1)
+            assert np.all(np.abs(dq - o["keys"][bad]) <= 2 * step), f"request {b}: key codes"
+        off.append(set(bad.tolist()))
+    return off
+
+
+def check_selection_and_output(st, ora, got, off, bf16_scores):
+    qI = O.dec_mxfp4(st.qI, st.qI_scale)
+    for b in range(st.B):
+        o, t, nv = ora[b], int(st.pos[b, 0]), st.n_vis(b)
+        ref = O.index_scores(qI[b, 0], st.w[b, 0], o["keys"], nv)
+        scale = O.index_score_scale(qI[b, 0], st.w[b, 0], o["keys"], nv)
+        g = got["scores"][b, 0, :nv]
+        ok = np.array([s not in off[b] for s in range(nv)], bool)
+        lim = 1e-4 * scale + (U.bf16_ulp(ref) if bf16_scores else 0.0)
+        assert np.all(np.abs(g - ref)[ok] <= lim[ok]), f"request {b}: index scores"
+        sel = got["idx"][b, 0]
+        kk = min(K, nv)
+        assert np.all(sel[kk:] == -1) and len(set(sel[:kk].tolist())) == kk
+        # valid for the GPU's own scores: larger first, ties by index, nothing larger left out
+        gs = g.astype(np.float64)
+        for j in range(kk - 1):
+            a, c = gs[sel[j]], gs[sel[j + 1]]
+            assert a > c or (a == c and sel[j] < sel[j + 1]), f"request {b}: order at {j}"
+        if kk < nv:
+            last = gs[sel[kk - 1]]
+            assert last >= np.delete(gs, sel[:kk]).max(), f"request {b}: k-th"
+            tied = np.flatnonzero(gs == last)  # among equal values the smaller indices win
+            n_tied = int(np.sum(gs[sel[:kk]] == last))
+            assert sorted(sel[:kk][gs[sel[:kk]] == last].tolist()) == tied[:n_tied].tolist()
+        # against the oracle: different only at near-ties of the k-th score (or at a key
+        # stored differently)
+        theirs = (O.topk_select_bf16 if bf16_scores else O.topk_select)(ref, K)[:kk]
+        tau = (O.round_to_bf16(ref) if bf16_scores else ref)[theirs[-1]]
+        tol = 1e-4 * scale.max() + (U.bf16_ulp(np.array([tau]))[0] if bf16_scores else 0.0)
+        for i in set(sel[:kk].tolist()).symmetric_difference(theirs.tolist()):
+            assert i in off[b] or abs(ref[i] - tau) <= tol, f"request {b}: {i} not a near-tie"
+        # the oracle's attention over the GPU's selection
+        want = O.csa_query(O.dec_bf16(st.q[b, 0]), t, o["kv"], sel, o["win"], 0, st.sink, r=R,
+                           base=BASE, eps=EPS, scale=1.0 / math.sqrt(C), n_win=N_WIN)
+        U.check_out(got["out"][b, 0], want, "bf16", f"request {b}: output")
+
+
+@pytest.mark.parametrize("n_cap", [1024, 8192], ids=["row_topk", "decode_topk"])
+@pytest.mark.parametrize("bf16_scores", [0, 1], ids=["fp32_scores", "bf16_scores"])
+def test_decode_step_over_the_state_cache(n_cap, bf16_scores):
+    st = Stream(n_cap)
+    ora = oracle_caches(st)
+    got = run_gpu(st, bf16_scores)
+    off = check_pages(st, ora, got)
+    check_selection_and_output(st, ora, got, off, bf16_scores)
