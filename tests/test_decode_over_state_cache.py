@@ -21,7 +21,11 @@ attention on those. Checks:
   - the output: the oracle's attention over the GPU's selection, within the bf16 output
     tolerance.
 The N_cap = 8192 case takes the decode top-k (histogram filled by the indexer), 1024 the
-row top-k. Not yet run on a B200: the module runs only with CSA_RUN_FIRST_GPU_CHECKS=1.
+row top-k. One case stores the KV entries as mixed-precision rows (e4m3 with a row scale,
+bf16 RoPE dims; 一(三)4): they must decode to within one step of each format of the
+oracle's entries, and the oracle attends its own mixed rows. The HCA case (m' = 128, pages
+of one entry, hca_dense_mqa_paged over the ring) attends every visible entry.
+Not yet run on a B200: the module runs only with CSA_RUN_FIRST_GPU_CHECKS=1.
 """
 import math
 import os
@@ -84,8 +88,16 @@ class Stream:
         return O.visible_entries(int(self.pos[b, 0]), M, self.n_cap)
 
 
-def oracle_caches(st: Stream):
-    """Per request: the oracle's KV entries (bf16-stored, decoded), its fp32-cast keys, the
+def stored_kv(kv_f64, kv_fmt):
+    """The oracle's entries as the cache stores them (input encoders), decoded."""
+    x = kv_f64.astype(np.float32)
+    if kv_fmt == "mixed":
+        return O.dec_mixed_kv(*W.quant_mixed_kv(x, R))
+    return O.dec_bf16(W.f32_to_bf16_bits(x))
+
+
+def oracle_caches(st: Stream, kv_fmt="bf16"):
+    """Per request: the oracle's KV entries (as stored, decoded), its fp32-cast keys, the
     MXFP4 bytes the encoder makes of them, and those keys decoded."""
     out = []
     for b, n in enumerate(N_TOK):
@@ -99,30 +111,38 @@ def oracle_caches(st: Stream):
                 cs.append(r["Ca"][t], r["Cb"][t], r["Za"][t], r["Zb"][t], r["win"][t])
             caches.append(cs.entries())
         kv, keys = caches
-        kv_bf16 = O.dec_bf16(W.f32_to_bf16_bits(kv.astype(np.float32)))
         packed, ex = W.quant_mxfp4(keys.astype(np.float32))
-        out.append(dict(kv_f64=kv, kv=kv_bf16, keys_packed=packed, keys_ex=ex,
+        out.append(dict(kv_f64=kv, kv=stored_kv(kv, kv_fmt), keys_packed=packed, keys_ex=ex,
                         keys=O.dec_mxfp4(packed, ex), win=O.dec_bf16(st.kv["win"][b, :n])))
     return out
 
 
-def run_gpu(st: Stream, bf16_scores: int):
+def _up(x):
+    import torch
+
+    a = np.ascontiguousarray(x)
+    return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).cuda()
+
+
+def run_gpu(st: Stream, bf16_scores: int, kv_fmt="bf16"):
     """The appends and the forward call; returns host copies of the pools and the results."""
     import torch
     import long_context_sparse_08_b200 as csa
 
-    def up(x):
-        a = np.ascontiguousarray(x)
-        return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).cuda()
-
+    up = _up
     torch.cuda.synchronize()
     csa.device_error()
     B = st.B
+    mixed = kv_fmt == "mixed"
     p_kv = csa.make_params(m=M, overlap=1, c=C, rope_dims=R, rope_base=BASE, rms_eps=EPS,
                            n_heads=H, n_idx_heads=H_I, d_idx=D_I, topk=K, n_win=N_WIN)
     p_key = csa.make_params(m=M, overlap=1, c=D_I, rope_dims=R, rope_base=BASE, rms_eps=EPS,
                             n_win=N_WIN)
-    kv_pages = torch.zeros((st.n_kv_pages, KV_ROWS, C), dtype=torch.int16, device="cuda")
+    kv_pages = torch.zeros((st.n_kv_pages, KV_ROWS, C + R), dtype=torch.uint8, device="cuda") \
+        if mixed else torch.zeros((st.n_kv_pages, KV_ROWS, C), dtype=torch.int16, device="cuda")
+    kv_scales = torch.zeros((st.n_kv_pages, KV_ROWS), dtype=torch.float32, device="cuda") \
+        if mixed else None
+    kv_out = csa.CSA_MIXED_FP8_BF16 if mixed else csa.CSA_BF16
     key_pages = torch.zeros((st.n_key_pages, KEY_ROWS, D_I // 2), dtype=torch.uint8,
                             device="cuda")
     key_ex = torch.zeros((st.n_key_pages, KEY_ROWS, 4), dtype=torch.uint8, device="cuda")
@@ -142,7 +162,7 @@ def run_gpu(st: Stream, bf16_scores: int):
             r = {k: v[b, t:t + 1] for k, v in kv_src.items() if k != "bias"}
             csa.csa_state_append(p_kv, csa.CSA_BF16, 1, pos, r["Ca"], r["Cb"], r["Za"], r["Zb"],
                                  r["win"], kv_src["bias"], None, 1, kv_state[b:b + 1],
-                                 ring[b:b + 1], csa.CSA_BF16, kv_pages, None, st.n_kv_pages,
+                                 ring[b:b + 1], kv_out, kv_pages, kv_scales, st.n_kv_pages,
                                  KV_ROWS, kv_tb, kv_table.shape[1])
             r = {k: v[b, t:t + 1] for k, v in key_src.items() if k != "bias"}
             csa.csa_state_append(p_key, csa.CSA_BF16, 1, pos, r["Ca"], r["Cb"], r["Za"],
@@ -151,7 +171,7 @@ def run_gpu(st: Stream, bf16_scores: int):
                                  KEY_ROWS, key_tb, key_table.shape[1])
     torch.cuda.synchronize()
     assert csa.device_error() == 0, "appends"
-    kv = csa.paged_kv(csa.CSA_BF16, kv_pages, None, kv_table, st.n_kv_pages, KV_ROWS,
+    kv = csa.paged_kv(kv_out, kv_pages, kv_scales, kv_table, st.n_kv_pages, KV_ROWS,
                       kv_table.shape[1])
     keys = csa.paged_kv(csa.CSA_MXFP4, key_pages, key_ex, key_table, st.n_key_pages, KEY_ROWS,
                         key_table.shape[1])
@@ -168,7 +188,9 @@ def run_gpu(st: Stream, bf16_scores: int):
     assert csa.device_error() == 0, "forward"
     scores = sc.cpu().numpy()
     scores = O.dec_bf16(scores.view(np.uint16)) if bf16_scores else scores.astype(np.float64)
-    return dict(kv_pages=kv_pages.cpu().numpy().view(np.uint16),
+    kvp = kv_pages.cpu().numpy()
+    return dict(kv_pages=kvp if mixed else kvp.view(np.uint16),
+                kv_scales=None if kv_scales is None else kv_scales.cpu().numpy(),
                 key_pages=key_pages.cpu().numpy(), key_ex=key_ex.cpu().numpy(),
                 idx=idx.cpu().numpy(), scores=scores,
                 out=O.dec_bf16(out.cpu().numpy().view(np.uint16)))
@@ -180,16 +202,34 @@ def page_rows_of(table, rows, b, n):
     return table[b, i // rows], i % rows
 
 
-def check_pages(st, ora, got):
-    """KV entries within a bf16 rounding; key bytes equal except near rounding boundaries.
-    Returns, per request, the keys whose stored bytes differ from the oracle's."""
+def check_kv_rows(got_rows, got_scales, ref, kv_fmt, what):
+    """Stored KV entries against the oracle's fp64 entries: within the fp32 error and one
+    rounding of the storage format."""
+    if kv_fmt != "mixed":
+        U.check_rows(O.dec_bf16(got_rows), ref, "bf16", what)
+        return
+    r0 = C - R
+    dq = O.dec_mixed_kv(got_rows[:, :r0], got_scales,
+                        np.ascontiguousarray(got_rows[:, r0:]).view(np.uint16))
+    rms = np.sqrt(np.mean(ref * ref, axis=1, keepdims=True))
+    # half an e4m3 step (2^-4 of |x|, 2^-10 x scale below the normal range); half a bf16 ulp
+    bound = np.concatenate([
+        np.maximum(np.abs(ref[:, :r0]) * 2.0 ** -4, got_scales[:, None] * 2.0 ** -10) * 1.01,
+        np.abs(ref[:, r0:]) * 2.0 ** -8 * 1.01], axis=1) + 2e-4 * rms
+    assert np.all(np.abs(dq - ref) <= bound), f"{what}: mixed rows"
+
+
+def check_pages(st, ora, got, kv_fmt="bf16"):
+    """KV entries within one rounding of their format; key bytes equal except near rounding
+    boundaries. Returns, per request, the keys whose stored bytes differ from the oracle's."""
     off = []
     for b, n in enumerate(N_TOK):
         o = ora[b]
         ne = n // M
         pg, sl = page_rows_of(st.kv_table, KV_ROWS, b, ne)
-        U.check_rows(O.dec_bf16(got["kv_pages"][pg, sl]), o["kv_f64"], "bf16",
-                     f"request {b}: KV entries")
+        check_kv_rows(got["kv_pages"][pg, sl],
+                      None if got["kv_scales"] is None else got["kv_scales"][pg, sl],
+                      o["kv_f64"], kv_fmt, f"request {b}: KV entries")
         pg, sl = page_rows_of(st.key_table, KEY_ROWS, b, ne)
         packed = got["key_pages"][pg, sl]
         ex = np.stack([O.unblock_key_scales(got["key_ex"][p])[s] for p, s in zip(pg, sl)])
@@ -242,11 +282,95 @@ def check_selection_and_output(st, ora, got, off, bf16_scores):
         U.check_out(got["out"][b, 0], want, "bf16", f"request {b}: output")
 
 
-@pytest.mark.parametrize("n_cap", [1024, 8192], ids=["row_topk", "decode_topk"])
-@pytest.mark.parametrize("bf16_scores", [0, 1], ids=["fp32_scores", "bf16_scores"])
-def test_decode_step_over_the_state_cache(n_cap, bf16_scores):
+CASES = [(1024, 0, "bf16"), (1024, 1, "bf16"), (8192, 0, "bf16"), (8192, 1, "bf16"),
+         (8192, 0, "mixed")]
+
+
+@pytest.mark.parametrize("n_cap,bf16_scores,kv_fmt", CASES,
+                         ids=[f"ncap{n}_{'bf16' if s else 'fp32'}_scores_{f}_kv"
+                              for n, s, f in CASES])
+def test_decode_step_over_the_state_cache(n_cap, bf16_scores, kv_fmt):
     st = Stream(n_cap)
-    ora = oracle_caches(st)
-    got = run_gpu(st, bf16_scores)
-    off = check_pages(st, ora, got)
+    ora = oracle_caches(st, kv_fmt)
+    got = run_gpu(st, bf16_scores, kv_fmt)
+    off = check_pages(st, ora, got, kv_fmt)
     check_selection_and_output(st, ora, got, off, bf16_scores)
+
+
+# ---------------------------------------------------------------------------
+# HCA: m' = 128, one entry per page, dense attention over every visible entry
+# ---------------------------------------------------------------------------
+
+HCA_M, HCA_N_TOK, HCA_N_CAP = 128, (2000, 900, 4100), 64
+
+
+class HcaStream:
+    def __init__(self, seed=2027):
+        self.B = len(HCA_N_TOK)
+        self.kv = W.make_state_stream(B=self.B, n_tok=max(HCA_N_TOK), m=HCA_M, c=C, overlap=0,
+                                      io="bf16", seed=seed)
+        g = np.random.default_rng(seed + 1)
+        self.q = W.f32_to_bf16_bits(g.standard_normal((self.B, 1, H, C), np.float32))
+        self.sink = g.standard_normal((H,), np.float32)
+        self.pos = np.array([[t - 1] for t in HCA_N_TOK], np.int64)
+        used = [t // HCA_M for t in HCA_N_TOK]
+        self.n_pages = sum(used) + 3
+        perm = g.permutation(self.n_pages).astype(np.int32)
+        self.table = np.full((self.B, HCA_N_CAP), -1, np.int32)
+        k = 0
+        for b, u in enumerate(used):
+            self.table[b, :u] = perm[k:k + u]
+            k += u
+
+
+def test_hca_decode_step_over_the_state_cache():
+    import torch
+    import long_context_sparse_08_b200 as csa
+
+    st = HcaStream()
+    B = st.B
+    p = csa.make_params(m=HCA_M, overlap=0, c=C, rope_dims=R, rope_base=BASE, rms_eps=EPS,
+                        n_heads=H, n_win=N_WIN)
+    torch.cuda.synchronize()
+    csa.device_error()
+    pages = torch.zeros((st.n_pages, 1, C), dtype=torch.int16, device="cuda")
+    state = torch.zeros((B, HCA_M, 2, C), dtype=torch.int16, device="cuda")
+    ring = torch.zeros((B, N_WIN, C), dtype=torch.int16, device="cuda")
+    src = {k: _up(st.kv[k]) for k in st.kv}
+    for b, n in enumerate(HCA_N_TOK):
+        pos_all = torch.zeros((n, 2), dtype=torch.int64, device="cuda")
+        pos_all[:, 0] = torch.arange(n, device="cuda")
+        tb = _up(st.table[b:b + 1])
+        for t in range(n):
+            csa.csa_state_append(p, csa.CSA_BF16, 1, pos_all[t, :1], src["Ca"][b, t:t + 1], None,
+                                 src["Za"][b, t:t + 1], None, src["win"][b, t:t + 1],
+                                 src["bias"], None, 1, state[b:b + 1], ring[b:b + 1],
+                                 csa.CSA_BF16, pages, None, st.n_pages, 1, tb, HCA_N_CAP)
+    torch.cuda.synchronize()
+    assert csa.device_error() == 0, "appends"
+    table = _up(st.table)
+    kv = csa.paged_kv(csa.CSA_BF16, pages, None, table, st.n_pages, 1, HCA_N_CAP)
+    need = csa.workspace_size(p, csa.CSA_WS_HCA_MQA, 0, B, 1, HCA_N_CAP)
+    ws = torch.empty((max(need, 1),), dtype=torch.uint8, device="cuda")
+    out = torch.empty((B, 1, H, C), dtype=torch.int16, device="cuda")
+    csa.hca_dense_mqa_paged(p, B, 1, _up(st.q), _up(st.pos), kv, ring, N_WIN, None,
+                            _up(st.sink), None, out, ws, need)
+    torch.cuda.synchronize()
+    assert csa.device_error() == 0, "attention"
+    got_pages = pages.cpu().numpy().view(np.uint16)
+    got = O.dec_bf16(out.cpu().numpy().view(np.uint16))
+    for b, n in enumerate(HCA_N_TOK):
+        pool = SC.PagePool(n // HCA_M + 1, 1, C)
+        cs = SC.HcaState(pool, m=HCA_M, c=C, bias=O.dec_bf16(st.kv["bias"]), n_win=N_WIN, r=R,
+                         base=BASE, eps=EPS, block_tokens=HCA_M)
+        r = {k: O.dec_bf16(st.kv[k][b, :n]) for k in ("Ca", "Za", "win")}
+        for t in range(n):
+            cs.append(r["Ca"][t], r["Za"][t], r["win"][t])
+        ent = cs.entries()
+        U.check_rows(O.dec_bf16(got_pages[st.table[b, :len(ent)], 0]), ent, "bf16",
+                     f"HCA request {b}: entries")
+        t = int(st.pos[b, 0])
+        want = O.hca_query(O.dec_bf16(st.q[b, 0]), t, stored_kv(ent, "bf16"),
+                           O.visible_entries(t, HCA_M, HCA_N_CAP), r["win"], 0, st.sink, r=R,
+                           base=BASE, eps=EPS, scale=1.0 / math.sqrt(C), n_win=N_WIN)
+        U.check_out(got[b, 0], want, "bf16", f"HCA request {b}: output")
