@@ -33,6 +33,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "CSA decode queries/s at 1M ctx (Flash/Pro shape); % of B200 HBM roofline"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+NOMINAL_HBM_GBS = 8000.0  # a B200's nominal HBM3e bandwidth, reported beside the measured one
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -297,6 +298,8 @@ def run_ours(args, W, rank, world, local_rank):
         roof = {"kernel": kname, "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
+                "nominal_peak": NOMINAL_HBM_GBS,
                 "traffic": traffic_from_profile(src, kname, s.name),
                 "alg_bytes_per_launch": alg, "avg_launch_ms": round(idx_ms, 5),
                 "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)"}
@@ -314,7 +317,9 @@ def run_ours(args, W, rank, world, local_rank):
             parallelism=f"replicas x{world} (independent requests)"),
         "step_hbm_roofline": {"alg_bytes_per_step": step_bytes,
                               "frac_of_peak": round(step_bytes / (ms / K / 1e3) / 1e9 /
-                                                    peaks["hbm_gbs"], 4)},
+                                                    peaks["hbm_gbs"], 4),
+                              "frac_of_nominal": round(step_bytes / (ms / K / 1e3) / 1e9 /
+                                                       NOMINAL_HBM_GBS, 4)},
         "roofline": roof,
         "clocks": clk,
         "e2e": e2e,
