@@ -332,6 +332,8 @@ def run_ours(args, W, rank, world, local_rank):
         tf = fl["total"] / (ms / K / 1e3) / 1e12
         res["tflops"] = {"value": round(tf, 1), "flops_per_step": fl,
                          "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
+                         "frac_of_bf16_sustained": round(
+                             tf / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]), 4),
                          "peak": peaks["bf16_tflops"],
                          "peak_source": f"{peak_src} bf16_tflops (cuBLAS burst)"}
     return res, inp, s
