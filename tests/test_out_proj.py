@@ -86,6 +86,22 @@ def test_host_build_matches_the_oracle(shape, sms):
     _check(out, _oracle(inp, Q, H, c, g, d_g, d), f"host {shape} sms={sms}")
 
 
+@pytest.mark.parametrize("shape", FULL, ids=["flash_decode", "pro_decode"])
+def test_host_build_on_the_decode_shapes_sampled(shape):
+    # the model's decode shapes with the B200's 148 SMs: every column computed by the host
+    # build, sampled columns against the oracle
+    Q, H, c, g, d_g, d = shape
+    inp = W.make_out_proj_inputs(Q=Q, H=H, c=c, g=g, d_g=d_g, d=d, seed=7)
+    out = np.zeros((Q, d), np.uint16)
+    geom = np.zeros(4, np.int32)
+    ptr = lambda a: a.ctypes.data_as(ctypes.c_void_p)  # noqa: E731
+    rc = host_lib().out_proj_host(Q, H, c, g, d_g, d, 148, ptr(inp["o"]), ptr(inp["w_grp"]),
+                                  ptr(inp["w_out"]), ptr(out), ptr(geom))
+    assert rc == 0, f"index outside a buffer ({rc})"
+    cols = np.unique(np.concatenate([np.arange(0, d, 97), [d - 1]]))
+    _check(out[:, cols], _oracle(inp, Q, H, c, g, d_g, d, cols=cols), f"host {shape} sampled")
+
+
 def test_checks_on_the_host():
     import long_context_sparse_08_b200 as csa
 
