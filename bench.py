@@ -487,12 +487,15 @@ def _time_calls(fn, n_rep, warmup, steps):
 def check_part_workload(part, s):
     """Exit with a message when a part cannot run on the workload's caches (before any GPU
     work): the paged indexer and the BF16-score path take the tensor-core indexers' keys
-    (MXFP4, FP8 or bf16), the paged layer a CSA decode step."""
+    (MXFP4, FP8 or bf16), the paged layer a CSA decode step, the layout comparison a decode
+    step."""
     want = None
     if part in ("bf16_scores", "forward_paged") and s.idx not in ("mxfp4", "fp8", "bf16"):
         want = "MXFP4, FP8 or bf16 indexer keys"
     elif part == "forward_paged" and s.kind != "csa_decode":
         want = "a CSA decode step"
+    elif part == "kv_layouts" and s.kind not in ("csa_decode", "hca_decode"):
+        want = "a CSA or HCA decode step"
     if want:
         raise SystemExit(f"--part {part} wants a workload with {want} "
                          f"(e.g. --workload pro_decode_1m); {s.name} has "
@@ -504,7 +507,8 @@ def run_part(args, W):
     out_proj          grouped output projection of the batch's queries (HBM roofline);
     out_proj_prefill  its tensor-core form on a prefill chunk's queries (tensor roofline);
     state_append      one decode token per request into the KV and indexer-key state caches;
-    kv_layouts        the attention alone over bf16, mixed-precision and paged caches;
+    kv_layouts        the attention alone over bf16, mixed-precision and paged caches (CSA
+                      or, on an HCA workload, the dense form);
     bf16_scores       index + top-k with fp32 and with BF16 scores;
     forward_paged     the CSA layer over page pools and a window ring vs the contiguous one."""
     s = W.SHAPES[args.workload]
@@ -601,56 +605,73 @@ def run_part(args, W):
                               "peak": hbm, "peak_source": peak_src, "unit": "GB/s",
                               "frac": round(ach / hbm, 6), "bytes_per_append": per})
     elif args.part == "kv_layouts":
+        # the attention alone over the bf16 cache, mixed-precision rows and a shuffled page
+        # pool: CSA (the selected rows; pages of 32 entries) or HCA (every visible entry;
+        # pages of one entry)
         inp = W.make_inputs(s)
         dev = R.upload(inp, s)
         p = R.params_for(s)
         B, T, k = s.B, s.T, s.topk
+        hca = s.kind == "hca_decode"
         g = torch.Generator(device="cpu").manual_seed(9)
         n_vis = min(s.ctx // s.m, s.n_cap)
-        idx = torch.stack([torch.randperm(n_vis, generator=g)[:k] for _ in range(B * T)])
-        idx = idx.view(B, T, k).to(torch.int32).cuda()
+        if not hca:
+            idx = torch.stack([torch.randperm(n_vis, generator=g)[:k] for _ in range(B * T)])
+            idx = idx.view(B, T, k).to(torch.int32).cuda()
         kv = W.bf16_bits_to_f32(inp["kv_cache"])
         codes, scale, rope = W.quant_mixed_kv(kv, s.rope_dims)
         del kv
         mixed = torch.from_numpy(np.concatenate([codes, rope.view(np.uint8)], axis=-1)).cuda()
         mscale = torch.from_numpy(scale).cuda()
         del codes, rope
-        pr = 32
+        pr = 1 if hca else 32
         max_pages = s.n_cap // pr
         perm = torch.randperm(B * max_pages, generator=g).to(torch.int32)
         table = perm.view(B, max_pages).cuda()
         pool = torch.empty((B * max_pages, pr, s.c), dtype=dev["kv_cache"].dtype, device="cuda")
         pool[table.view(-1).long()] = dev["kv_cache"].view(B * max_pages, pr, s.c)
         out = torch.empty((B, T, s.n_heads, s.c), dtype=dev["q"].dtype, device="cuda")
-        ws_bytes = csa.workspace_size(p, csa.CSA_WS_SPARSE_MQA, 0, B, T, s.n_cap)
+        entry = csa.CSA_WS_HCA_MQA if hca else csa.CSA_WS_SPARSE_MQA
+        ws_bytes = csa.workspace_size(p, entry, 0, B, T, s.n_cap)
         ws = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device="cuda")
         pkv = csa.paged_kv(csa.CSA_BF16, pool, None, table, B * max_pages, pr, max_pages)
         L = dev["win_kv"].shape[1]
-        calls = {
-            "bf16": lambda i: csa.csa_sparse_mqa(p, csa.CSA_BF16, B, T, dev["q"], dev["q_pos"],
-                                                 dev["kv_cache"], s.n_cap, idx, dev["win_kv"], L,
-                                                 dev["win_pos0"], dev["sink"], None, out, ws,
-                                                 ws_bytes),
-            "mixed": lambda i: csa.csa_sparse_mqa_mixed_kv(p, B, T, dev["q"], dev["q_pos"], mixed,
-                                                           mscale, s.n_cap, idx, dev["win_kv"], L,
-                                                           dev["win_pos0"], dev["sink"], None,
-                                                           out, ws, ws_bytes),
-            "paged_bf16": lambda i: csa.csa_sparse_mqa_paged(p, B, T, dev["q"], dev["q_pos"], pkv,
-                                                             idx, dev["win_kv"], L,
-                                                             dev["win_pos0"], dev["sink"], None,
-                                                             out, ws, ws_bytes)}
+        q, qp, win, w0, sink = dev["q"], dev["q_pos"], dev["win_kv"], dev["win_pos0"], dev["sink"]
+        if hca:
+            calls = {
+                "bf16": lambda i: csa.hca_dense_mqa(p, csa.CSA_BF16, B, T, q, qp, dev["kv_cache"],
+                                                    s.n_cap, win, L, w0, sink, None, out, ws,
+                                                    ws_bytes),
+                "mixed": lambda i: csa.hca_dense_mqa_mixed_kv(p, B, T, q, qp, mixed, mscale,
+                                                              s.n_cap, win, L, w0, sink, None,
+                                                              out, ws, ws_bytes),
+                "paged_bf16": lambda i: csa.hca_dense_mqa_paged(p, B, T, q, qp, pkv, win, L, w0,
+                                                                sink, None, out, ws, ws_bytes)}
+        else:
+            calls = {
+                "bf16": lambda i: csa.csa_sparse_mqa(p, csa.CSA_BF16, B, T, q, qp,
+                                                     dev["kv_cache"], s.n_cap, idx, win, L, w0,
+                                                     sink, None, out, ws, ws_bytes),
+                "mixed": lambda i: csa.csa_sparse_mqa_mixed_kv(p, B, T, q, qp, mixed, mscale,
+                                                               s.n_cap, idx, win, L, w0, sink,
+                                                               None, out, ws, ws_bytes),
+                "paged_bf16": lambda i: csa.csa_sparse_mqa_paged(p, B, T, q, qp, pkv, idx, win,
+                                                                 L, w0, sink, None, out, ws,
+                                                                 ws_bytes)}
+        rows = n_vis if hca else k  # cache rows each query reads
         res = {}
         for name, fn in calls.items():
             ms = _time_calls(fn, 1, args.warmup, args.steps)
             row = 1024 if name != "mixed" else s.c + s.rope_dims + 4
-            nbytes = B * T * ((k * row) + s.n_win * 2 * s.c + 2 * 2 * s.n_heads * s.c)
+            nbytes = B * T * ((rows * row) + s.n_win * 2 * s.c + 2 * 2 * s.n_heads * s.c)
             res[name] = {"ms_per_call": round(ms, 5), "bytes_per_call": nbytes,
                          "achieved_gbs": round(nbytes / (ms / 1e3) / 1e9, 1)}
-        line.update(metric="sparse MQA calls/s by cache layout",
+        line.update(metric=f"{'dense' if hca else 'sparse'} MQA calls/s by cache layout",
                     value=round(1e3 / res["mixed"]["ms_per_call"], 2), unit="calls/s (mixed)",
-                    layouts=res, config={"B": B, "T": T, "k": k, "n_cap": s.n_cap,
-                                         "page_rows": pr},
-                    roofline={"bound": "latency (see the attention in DESIGN)", "peak": hbm,
+                    layouts=res, config={"B": B, "T": T, "rows_per_query": rows,
+                                         "n_cap": s.n_cap, "page_rows": pr},
+                    roofline={"bound": "hbm (dense rows)" if hca else
+                              "latency (one CTA per query and head group)", "peak": hbm,
                               "peak_source": peak_src, "unit": "GB/s"})
     elif args.part == "bf16_scores":
         # index + top-k with fp32 scores (csa_index_topk) and with BF16 scores

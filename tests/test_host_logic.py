@@ -109,4 +109,7 @@ def test_parts_refuse_workloads_they_cannot_run(bench):
     with pytest.raises(SystemExit, match="a CSA decode step"):
         bench.check_part_workload("forward_paged", W.SHAPES["flash_prefill_8k"])
     bench.check_part_workload("bf16_scores", W.SHAPES["flash_prefill_8k"])
+    with pytest.raises(SystemExit, match="a CSA or HCA decode step"):
+        bench.check_part_workload("kv_layouts", W.SHAPES["flash_prefill_8k"])
+    bench.check_part_workload("kv_layouts", W.SHAPES["hca_decode_1m"])
     bench.check_part_workload("out_proj", W.SHAPES["pro_decode_1m"])
