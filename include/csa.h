@@ -49,7 +49,8 @@ typedef enum {
   CSA_ERR_INVALID_ARG = 1, /* a pointer, size or alignment the call cannot accept */
   CSA_ERR_UNSUPPORTED = 2, /* a valid shape / dtype combination this library does not implement */
   CSA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than csa_workspace_size() */
-  CSA_ERR_CUDA = 4         /* the CUDA runtime reported an error while queueing */
+  CSA_ERR_CUDA = 4,        /* the CUDA runtime reported an error while queueing */
+  CSA_ERR_NO_PAGES = 5     /* a page pool has too few free pages for the request */
 } csa_status;
 
 typedef enum {
@@ -386,6 +387,40 @@ csa_status csa_state_resume(const csa_params* p, csa_dtype io, int32_t B, int64_
                             int64_t n_tok, const void* Ca, const void* Cb, const void* Za,
                             const void* Zb, const void* win_rows, void* state, void* win_ring,
                             void* stream);
+
+/*
+ * Page allocation for the state cache's pools ([P1''] 二(六): finished entries in a
+ * classical cache of blocks, each a multiple of lcm(m, m') raw tokens; [P4] §2: one logical
+ * block of 128 raw tokens is 32 CSA entries or 1 HCA entry). One allocator serves one pool
+ * of n_pages physical pages shared by B requests. It owns a host page table int32
+ * [B, max_pages]: entry [b, k] is the physical page of request b's logical page k, or -1.
+ * The caller copies the table (or the rows it changed) to the device before the launches
+ * that read it. Free pages are handed out in order (first 0 .. n_pages-1, then pages given
+ * back, in the order they were given back). Host memory only; not thread-safe.
+ *
+ *   csa_page_alloc_create: a pool with every page free and every table entry -1.
+ *     *out = NULL on failure.
+ *   csa_page_alloc_reserve: maps logical pages [0, n_logical) of request b, taking free
+ *     pages for those not yet mapped (mapped ones stay). CSA_ERR_NO_PAGES, with nothing
+ *     taken, when too few are free.
+ *   csa_page_alloc_release: gives all of request b's pages back; its row becomes -1.
+ *   csa_page_alloc_table: the host table [B, max_pages] (valid until destroy).
+ *   csa_page_alloc_free_pages / csa_page_alloc_mapped: free pages in the pool / logical pages
+ *     mapped for request b (-1 for an invalid handle or b).
+ *   csa_state_pages_needed: logical pages that hold the entries of a request's first n_tok
+ *     tokens, ceil(floor(n_tok / m) / page_rows); reserving that many before appending the
+ *     token at position n_tok - 1 maps the page its entry goes to (-1 for invalid sizes).
+ */
+typedef struct csa_page_alloc csa_page_alloc;
+csa_status csa_page_alloc_create(int32_t n_pages, int32_t B, int32_t max_pages,
+                                 csa_page_alloc** out);
+void csa_page_alloc_destroy(csa_page_alloc* a);
+csa_status csa_page_alloc_reserve(csa_page_alloc* a, int32_t b, int32_t n_logical);
+csa_status csa_page_alloc_release(csa_page_alloc* a, int32_t b);
+const int32_t* csa_page_alloc_table(const csa_page_alloc* a);
+int32_t csa_page_alloc_free_pages(const csa_page_alloc* a);
+int32_t csa_page_alloc_mapped(const csa_page_alloc* a, int32_t b);
+int32_t csa_state_pages_needed(int32_t m, int32_t page_rows, int64_t n_tok);
 
 /* Inputs of the fused CSA layer call. Pointers as in the stage calls above. */
 typedef struct {

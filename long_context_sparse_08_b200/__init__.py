@@ -14,7 +14,8 @@ from typing import Optional
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libcsa.so")
 
-CSA_OK, CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_WORKSPACE, CSA_ERR_CUDA = range(5)
+(CSA_OK, CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_WORKSPACE, CSA_ERR_CUDA,
+ CSA_ERR_NO_PAGES) = range(6)
 CSA_F32, CSA_BF16, CSA_FP8_E4M3_ROWSCALE, CSA_MXFP4, CSA_MIXED_FP8_BF16 = range(5)
 DTYPES = {"f32": CSA_F32, "bf16": CSA_BF16, "fp8": CSA_FP8_E4M3_ROWSCALE, "mxfp4": CSA_MXFP4}
 (CSA_WS_INDEX_TOPK, CSA_WS_TOPK, CSA_WS_SPARSE_MQA, CSA_WS_HCA_MQA, CSA_WS_FORWARD,
@@ -28,6 +29,9 @@ EXPORTS = (
     "hca_dense_mqa_mixed_kv", "csa_grouped_out_proj", "csa_grouped_out_proj_workspace_size",
     "csa_sparse_mqa_paged", "hca_dense_mqa_paged", "csa_index_topk_bf16",
     "csa_index_topk_paged", "csa_forward_paged", "csa_compress_paged", "csa_state_resume",
+    "csa_page_alloc_create", "csa_page_alloc_destroy", "csa_page_alloc_reserve",
+    "csa_page_alloc_release", "csa_page_alloc_table", "csa_page_alloc_free_pages",
+    "csa_page_alloc_mapped", "csa_state_pages_needed",
 )
 # size of the library-owned scratch array behind csa_topk_noalloc (bytes, per device)
 TOPK_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -115,10 +119,21 @@ _SIGS = {
                                _VP, _VP, _VP, _SZ, _VP],
     "csa_state_append": [_PP, ctypes.c_int, _I32] + [_VP] * 8 + [_I32, _VP, _VP, ctypes.c_int,
                                                              _VP, _VP, _I32, _I32, _VP, _I32, _VP],
+    "csa_page_alloc_create": [_I32, _I32, _I32, ctypes.POINTER(_VP)],
+    "csa_page_alloc_destroy": [_VP],
+    "csa_page_alloc_reserve": [_VP, _I32, _I32],
+    "csa_page_alloc_release": [_VP, _I32],
+    "csa_page_alloc_table": [_VP],
+    "csa_page_alloc_free_pages": [_VP],
+    "csa_page_alloc_mapped": [_VP, _I32],
+    "csa_state_pages_needed": [_I32, _I32, _I64],
 }
 _RES = {"csa_workspace_size": _SZ, "csa_grouped_out_proj_workspace_size": _SZ, "csa_kernel_launches": ctypes.c_uint64, "csa_status_string": ctypes.c_char_p,
         "csa_last_error": ctypes.c_char_p, "csa_version": ctypes.c_char_p,
-        "csa_set_index_timing_events": None}
+        "csa_set_index_timing_events": None, "csa_page_alloc_destroy": None,
+        "csa_page_alloc_table": ctypes.POINTER(ctypes.c_int32),
+        "csa_page_alloc_free_pages": ctypes.c_int32, "csa_page_alloc_mapped": ctypes.c_int32,
+        "csa_state_pages_needed": ctypes.c_int32}
 
 
 class CsaError(RuntimeError):
@@ -171,6 +186,54 @@ def device_error() -> int:
 def _check(fn: str, status: int):
     if status != CSA_OK:
         raise CsaError(fn, status, last_error())
+
+
+def state_pages_needed(m: int, page_rows: int, n_tok: int) -> int:
+    """Logical pages that hold the entries of a request's first n_tok tokens."""
+    return int(lib().csa_state_pages_needed(m, page_rows, n_tok))
+
+
+class PageAlloc:
+    """A csa_page_alloc: physical pages of one pool handed to B requests' page tables (host
+    memory; copy ``table`` to the device before the launches that read it)."""
+
+    def __init__(self, n_pages: int, B: int, max_pages: int):
+        h = _VP()
+        _check("csa_page_alloc_create",
+               lib().csa_page_alloc_create(n_pages, B, max_pages, ctypes.byref(h)))
+        self._h, self.B, self.max_pages = h, B, max_pages
+
+    def close(self):
+        if self._h:
+            lib().csa_page_alloc_destroy(self._h)
+            self._h = _VP()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # interpreter shutdown
+            pass
+
+    def reserve(self, b: int, n_logical: int) -> None:
+        _check("csa_page_alloc_reserve", lib().csa_page_alloc_reserve(self._h, b, n_logical))
+
+    def release(self, b: int) -> None:
+        _check("csa_page_alloc_release", lib().csa_page_alloc_release(self._h, b))
+
+    @property
+    def table(self):
+        """The host page table as a numpy int32 [B, max_pages] view (no copy)."""
+        import numpy as np
+
+        ptr = lib().csa_page_alloc_table(self._h)
+        return np.ctypeslib.as_array(ptr, shape=(self.B, self.max_pages))
+
+    @property
+    def free_pages(self) -> int:
+        return int(lib().csa_page_alloc_free_pages(self._h))
+
+    def mapped(self, b: int) -> int:
+        return int(lib().csa_page_alloc_mapped(self._h, b))
 
 
 def _ptr(t) -> Optional[int]:

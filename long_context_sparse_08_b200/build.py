@@ -2,8 +2,9 @@
 
     python -m long_context_sparse_08_b200.build [-v]
 
-Compiles every csrc/*.cu into one shared library next to this file. Objects go to
-csrc/_build/ and are rebuilt only when a source or header is newer than the object.
+Compiles every csrc/*.cu (and the host-only csrc/*.cpp) into one shared library next to
+this file. Objects go to csrc/_build/ and are rebuilt only when a source or header is newer
+than the object.
 """
 from __future__ import annotations
 
@@ -48,13 +49,13 @@ def build(verbose: bool = False, extra: list | None = None) -> str:
     """Compile and link libcsa.so; return its path. Raises on compiler errors."""
     os.makedirs(OBJ, exist_ok=True)
     cc = nvcc()
-    srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
     hdr_mtime = max([os.path.getmtime(h) for h in _headers()] + [0.0])
     extra = list(extra or [])
     incs = ["-I", os.path.join(ROOT, "include"), "-I", CSRC]
 
     def compile_one(src):
-        obj = os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(OBJ, os.path.splitext(os.path.basename(src))[0] + ".o")
         if not _stale(obj, src, hdr_mtime):
             return obj, ""
         cmd = [cc, *ARCH, *FLAGS, *incs, *extra, "-c", src, "-o", obj]

@@ -279,6 +279,7 @@ const char* csa_status_string(csa_status s) {
     case CSA_ERR_UNSUPPORTED: return "CSA_ERR_UNSUPPORTED";
     case CSA_ERR_WORKSPACE: return "CSA_ERR_WORKSPACE";
     case CSA_ERR_CUDA: return "CSA_ERR_CUDA";
+    case CSA_ERR_NO_PAGES: return "CSA_ERR_NO_PAGES";
   }
   return "CSA_ERR_UNKNOWN";
 }
