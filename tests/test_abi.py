@@ -391,3 +391,37 @@ def test_noalloc_topk_rejects_oversize_on_the_host():
 
 def test_kernel_launch_counter_is_exported():
     assert csa.kernel_launches() >= 0
+
+
+def test_a_c_program_drives_the_page_allocator():
+    # the host-only calls of the C ABI, from C, linked against libcsa.so
+    prog = r'''
+#include <stdio.h>
+#include "csa.h"
+int main(void) {
+  csa_page_alloc* a = NULL;
+  if (csa_page_alloc_create(5, 2, 3, &a) != CSA_OK) return 1;
+  if (csa_page_alloc_reserve(a, 0, csa_state_pages_needed(4, 32, 132)) != CSA_OK) return 2;
+  if (csa_page_alloc_reserve(a, 1, 3) != CSA_OK) return 3;
+  if (csa_page_alloc_reserve(a, 0, 3) != CSA_ERR_NO_PAGES) return 4;
+  csa_page_alloc_release(a, 1);
+  if (csa_page_alloc_reserve(a, 0, 3) != CSA_OK) return 5;
+  const int32_t* t = csa_page_alloc_table(a);
+  for (int i = 0; i < 6; ++i) printf("%d ", t[i]);
+  printf("%d %s\n", csa_page_alloc_free_pages(a), csa_status_string(CSA_ERR_NO_PAGES));
+  csa_page_alloc_destroy(a);
+  return 0;
+}
+'''
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "t.c")
+        exe = os.path.join(d, "t")
+        open(c, "w").write(prog)
+        libdir = os.path.dirname(csa.LIB_PATH)
+        subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), c, "-o", exe,
+                               "-L", libdir, "-lcsa", f"-Wl,-rpath,{libdir}"])
+        out = subprocess.check_output([exe]).decode().split()
+    # request 0: 132 tokens make 33 entries, 2 pages of 32 (0, 1); request 1: 3 pages (2, 3,
+    # 4); request 0's third page fails with none free, then takes page 2 once request 1 gave
+    # 2, 3, 4 back
+    assert out == ["0", "1", "2", "-1", "-1", "-1", "2", "CSA_ERR_NO_PAGES"]
