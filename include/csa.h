@@ -10,11 +10,15 @@
  *        3(3) sliding window, 3(4) attention sink.
  *   [P1'] same page, 二、基础设施 (四) FP4 量化感知训练: the indexer's QK path in FP4.
  *   [P1''] same page, 二、基础设施 (六) 推理框架: state cache and paged cache at inference.
+ *   [P4] DeepseekV4论文解析, 2. Hybrid Attention：CSA + HCA (从注意力公式到可部署系统): the
+ *        per-request state and the paged cache in logical blocks of lcm(4, 128) = 128 raw
+ *        tokens (32 CSA entries or 1 HCA entry).
  *
  * Conventions shared by every call
  *   - Every tensor pointer is device memory owned by the caller; the library never
- *     allocates or frees device memory. Scratch comes from a caller-provided workspace
- *     whose size csa_workspace_size() returns.
+ *     allocates or frees device memory (the state cache's page allocator owns host memory
+ *     only). Scratch comes from a caller-provided workspace whose size
+ *     csa_workspace_size() returns.
  *   - Layouts are dense row-major with the shapes given per argument. Pointers must be
  *     16-byte aligned; c is a multiple of 64 (or exactly 64 for fp32 inputs), 0 <= r <= c,
  *     r even.
