@@ -426,6 +426,22 @@ int32_t csa_page_alloc_free_pages(const csa_page_alloc* a);
 int32_t csa_page_alloc_mapped(const csa_page_alloc* a, int32_t b);
 int32_t csa_state_pages_needed(int32_t m, int32_t page_rows, int64_t n_tok);
 
+/*
+ * Entries given as rows into a page pool in a storage format: the rows [B, n, c] (io =
+ * CSA_F32 or CSA_BF16; e.g. a prefill chunk's entries from csa_compress) are entries
+ * first_entry .. first_entry + n - 1 of every request, stored in out_pages->fmt exactly as
+ * csa_state_append stores a finished row: the io dtype, CSA_FP8_E4M3_ROWSCALE (scales fp32
+ * [n_pages, page_rows]), CSA_MXFP4 (c = 128, page_rows a multiple of 128; exponent blocks
+ * as for csa_state_append) or CSA_MIXED_FP8_BF16 (0 < p->rope_dims < c). This is the
+ * prefill -> decode hand-over for pools kept in a quantised format ([P1''] 二(六); [P1']
+ * 二(四) for the FP4 indexer keys). An entry whose page id lies outside the pool is skipped
+ * and leaves device error code 325 (324: its logical page is past the table, which the host
+ * check rules out).
+ */
+csa_status csa_encode_paged(const csa_params* p, csa_dtype io, int32_t B, int64_t n,
+                            int64_t first_entry, const void* rows,
+                            const csa_paged_kv* out_pages, void* stream);
+
 /* Inputs of the fused CSA layer call. Pointers as in the stage calls above. */
 typedef struct {
   /* optional compression of a new chunk into kv_cache (skipped when Ca == NULL) */
@@ -510,8 +526,8 @@ void csa_set_index_timing_events(void* const* before, void* const* after, int32_
  * early instead of hanging. csa_state_append also leaves a code for a request it skipped.
  * Codes by kernel family: 101-107 MXFP4 indexer (107: a page id outside the pool), 201-205
  * attention (205: a page id outside the pool), 301-309 FP8 / bf16 indexer (309: a page id
- * outside the pool), 321-323 state append, 331 paged compression, 401-405 prefill output
- * projection. Writes the code to *code (0 = none) and clears it. Synchronises the device.
+ * outside the pool), 321-323 state append, 324-325 encoding into pages, 331 paged
+ * compression, 401-405 prefill output projection. Writes the code to *code (0 = none) and clears it. Synchronises the device.
  * Returns CSA_ERR_CUDA if the copy fails.
  */
 csa_status csa_device_error(int32_t* code);

@@ -31,7 +31,7 @@ EXPORTS = (
     "csa_index_topk_paged", "csa_forward_paged", "csa_compress_paged", "csa_state_resume",
     "csa_page_alloc_create", "csa_page_alloc_destroy", "csa_page_alloc_reserve",
     "csa_page_alloc_release", "csa_page_alloc_table", "csa_page_alloc_free_pages",
-    "csa_page_alloc_mapped", "csa_state_pages_needed",
+    "csa_page_alloc_mapped", "csa_state_pages_needed", "csa_encode_paged",
 )
 # size of the library-owned scratch array behind csa_topk_noalloc (bytes, per device)
 TOPK_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -127,6 +127,8 @@ _SIGS = {
     "csa_page_alloc_free_pages": [_VP],
     "csa_page_alloc_mapped": [_VP, _I32],
     "csa_state_pages_needed": [_I32, _I32, _I64],
+    "csa_encode_paged": [_PP, ctypes.c_int, _I32, _I64, _I64, _VP, ctypes.POINTER(CsaPagedKv),
+                         _VP],
 }
 _RES = {"csa_workspace_size": _SZ, "csa_grouped_out_proj_workspace_size": _SZ, "csa_kernel_launches": ctypes.c_uint64, "csa_status_string": ctypes.c_char_p,
         "csa_last_error": ctypes.c_char_p, "csa_version": ctypes.c_char_p,
@@ -410,6 +412,12 @@ def csa_compress_paged(p, io, B, n_tok, first_entry, Ca, Cb, Za, Zb, bias, prev_
                                  _ptr(kv_rms_w), int(finalize), ctypes.byref(out_pages),
                                  _stream(stream))
     _check("csa_compress_paged", s)
+
+
+def csa_encode_paged(p, io, B, n, first_entry, rows, out_pages: CsaPagedKv, stream=None):
+    s = lib().csa_encode_paged(ctypes.byref(p), io, B, n, first_entry, _ptr(rows),
+                               ctypes.byref(out_pages), _stream(stream))
+    _check("csa_encode_paged", s)
 
 
 def csa_state_resume(p, io, B, first_tok, n_tok, Ca, Cb, Za, Zb, win_rows, state, win_ring,

@@ -488,6 +488,53 @@ csa_status csa_state_append(const csa_params* p, csa_dtype io, int32_t B, const 
   return ok();
 }
 
+csa_status csa_encode_paged(const csa_params* p, csa_dtype io, int32_t B, int64_t n,
+                            int64_t first_entry, const void* rows,
+                            const csa_paged_kv* out_pages, void* stream) {
+  TRY(check_params(p));
+  REQUIRE(io == CSA_F32 || io == CSA_BF16, "rows must be CSA_F32 or CSA_BF16");
+  REQUIRE(p->c <= 4096, "encoding supports c <= 4096 (got %d)", p->c);
+  REQUIRE(out_pages != nullptr, "page descriptor is NULL");
+  const csa_dtype fmt = out_pages->fmt;
+  REQUIRE(fmt == io || fmt == CSA_FP8_E4M3_ROWSCALE || fmt == CSA_MXFP4 ||
+              fmt == CSA_MIXED_FP8_BF16,
+          "page format must be the io dtype, CSA_FP8_E4M3_ROWSCALE, CSA_MXFP4 or "
+          "CSA_MIXED_FP8_BF16");
+  if (fmt == CSA_MIXED_FP8_BF16)
+    REQUIRE(p->rope_dims > 0 && p->rope_dims < p->c, "mixed rows need 0 < rope_dims < c");
+  if (fmt == CSA_MXFP4) {
+    REQUIRE(p->c == 128, "MXFP4 rows are indexer keys of 128 values (c = %d)", p->c);
+    REQUIRE(out_pages->page_rows % 128 == 0, "MXFP4 pages hold whole 128-row exponent blocks");
+  }
+  REQUIRE(B >= 0 && B <= 65535, "B must be in [0, 65535]");
+  REQUIRE(n >= 0 && n <= INT32_MAX && first_entry >= 0, "n and first_entry must be >= 0");
+  REQUIRE(out_pages->n_pages >= 1 && out_pages->page_rows >= 1 && out_pages->max_pages >= 1,
+          "n_pages, page_rows and max_pages must be >= 1");
+  REQUIRE(first_entry + n <= (int64_t)out_pages->page_rows * out_pages->max_pages,
+          "entries %lld .. %lld lie past the page table (%d pages of %d rows)",
+          (long long)first_entry, (long long)(first_entry + n - 1), out_pages->max_pages,
+          out_pages->page_rows);
+  if ((int64_t)B * n == 0) return ok();
+  REQUIRE_PTR(rows);
+  REQUIRE_PTR(out_pages->pages);
+  REQUIRE_PTR(out_pages->page_table);
+  if (fmt != io) REQUIRE_PTR(out_pages->scales);
+  csa::state::Args a{};
+  a.B = B; a.m = p->m; a.c = p->c; a.overlap = p->overlap; a.rope_dims = p->rope_dims;
+  a.n_pages = out_pages->n_pages; a.page_rows = out_pages->page_rows;
+  a.max_pages = out_pages->max_pages; a.eps = p->rms_eps;
+  a.pages = const_cast<void*>(out_pages->pages);
+  a.page_scales = const_cast<void*>(out_pages->scales);
+  a.page_table = out_pages->page_table;
+  a.out = fmt == io                   ? csa::state::kOutIo
+          : fmt == CSA_MXFP4          ? csa::state::kOutMxfp4
+          : fmt == CSA_MIXED_FP8_BF16 ? csa::state::kOutMixed
+                                      : csa::state::kOutFp8;
+  TRY(cuda_status(csa::launch_encode_paged(a, io == CSA_BF16, rows, n, first_entry,
+                                           (cudaStream_t)stream), "encode into pages"));
+  return ok();
+}
+
 namespace {
 csa_status check_out_proj(const csa_params* p, int32_t Q, int32_t g, int32_t d_g, int32_t d) {
   TRY(check_params(p));

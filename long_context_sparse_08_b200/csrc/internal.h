@@ -60,6 +60,10 @@ cudaError_t out_proj_tc_device_error(int* code);
 namespace state { struct Args; }
 // decode-time append of one token per request into the state cache and its pages
 cudaError_t launch_state_append(const state::Args& a, bool bf16, cudaStream_t st);
+// rows [B, n, c] (io dtype) = entries first_entry .. first_entry + n - 1 into their pages in
+// the format a.out (csa_encode_paged)
+cudaError_t launch_encode_paged(const state::Args& a, bool bf16, const void* rows, int64_t n,
+                                int64_t first_entry, cudaStream_t st);
 cudaError_t state_append_device_error(int* code);
 // after a prefill chunk: its last raw rows and window rows into the state cache
 cudaError_t launch_state_resume(const state::Args& a, bool bf16, int64_t first_tok,

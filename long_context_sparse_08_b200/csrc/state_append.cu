@@ -23,6 +23,7 @@ namespace {
 __device__ int g_state_error = 0;
 
 enum { kErrBase = 320 };  // stored code = kErrBase - status (321 position, 322 page slot, 323 page id)
+enum { kErrEncodeBase = 322 };  // csa_encode_paged: 324 page slot, 325 page id
 
 // Block-wide max of non-negative values; `red` is shared scratch of >= 32 floats.
 __device__ __forceinline__ float block_max_nonneg(float v, float* red) {
@@ -38,39 +39,12 @@ __device__ __forceinline__ float block_max_nonneg(float v, float* red) {
   return red[0];
 }
 
+// The finished row fin[c] (this thread's channels j = threadIdx.x + k*blockDim.x written by
+// this thread; amax = this thread's max |fin[j]|) stored at element offset `off` of `pages`
+// in the format a.out. Every thread of the CTA calls it (block reductions inside).
 template <typename T>
-__global__ void __launch_bounds__(256) k_state_append(state::Args a) {
-  extern __shared__ float row[];  // [2c]: pooled row, then the finished row
-  __shared__ float red[32];
-  float* fin = row + a.c;
-  const int b = blockIdx.x;
-  const int64_t t = a.pos[b];
-  int64_t i = 0;
-  size_t off = 0;
-  const int s = state::append_status(a, b, t, &i, &off);  // the same in every thread
-  if (s < 0) {
-    if (threadIdx.x == 0) atomicCAS(&g_state_error, 0, kErrBase - s);
-    return;
-  }
-  for (int j = threadIdx.x; j < a.c; j += blockDim.x) state::store_channel<T>(a, b, t, j);
-  if (s == state::kAppendOnly) return;
-  float ss = 0.f;
-  for (int j = threadIdx.x; j < a.c; j += blockDim.x) {
-    const float v = state::pool_channel<T>(a, b, i, j);
-    row[j] = v;
-    ss = fmaf(v, v, ss);
-  }
-  float rstd = 1.f;
-  if (a.finalize) {
-    const float tot = block_sum(ss, red);  // also orders the row[] writes before the reads
-    rstd = rsqrtf(tot / (float)a.c + a.eps);
-  }
-  float amax = 0.f;
-  for (int j = threadIdx.x; j < a.c; j += blockDim.x) {
-    const float v = a.finalize ? state::final_channel<T>(a, row, rstd, i, j) : row[j];
-    fin[j] = v;  // read back by this thread only
-    amax = fmaxf(amax, fabsf(v));
-  }
+__device__ __forceinline__ void store_finished(const state::Args& a, const float* fin,
+                                               float amax, size_t off, float* red) {
   if (a.out == state::kOutIo) {
     T* out = static_cast<T*>(a.pages) + off;
     for (int j = threadIdx.x; j < a.c; j += blockDim.x) state::st(out, j, fin[j]);
@@ -116,10 +90,71 @@ __global__ void __launch_bounds__(256) k_state_append(state::Args a) {
 }
 
 template <typename T>
+__global__ void __launch_bounds__(256) k_state_append(state::Args a) {
+  extern __shared__ float row[];  // [2c]: pooled row, then the finished row
+  __shared__ float red[32];
+  float* fin = row + a.c;
+  const int b = blockIdx.x;
+  const int64_t t = a.pos[b];
+  int64_t i = 0;
+  size_t off = 0;
+  const int s = state::append_status(a, b, t, &i, &off);  // the same in every thread
+  if (s < 0) {
+    if (threadIdx.x == 0) atomicCAS(&g_state_error, 0, kErrBase - s);
+    return;
+  }
+  for (int j = threadIdx.x; j < a.c; j += blockDim.x) state::store_channel<T>(a, b, t, j);
+  if (s == state::kAppendOnly) return;
+  float ss = 0.f;
+  for (int j = threadIdx.x; j < a.c; j += blockDim.x) {
+    const float v = state::pool_channel<T>(a, b, i, j);
+    row[j] = v;
+    ss = fmaf(v, v, ss);
+  }
+  float rstd = 1.f;
+  if (a.finalize) {
+    const float tot = block_sum(ss, red);  // also orders the row[] writes before the reads
+    rstd = rsqrtf(tot / (float)a.c + a.eps);
+  }
+  float amax = 0.f;
+  for (int j = threadIdx.x; j < a.c; j += blockDim.x) {
+    const float v = a.finalize ? state::final_channel<T>(a, row, rstd, i, j) : row[j];
+    fin[j] = v;  // read back by this thread only
+    amax = fmaxf(amax, fabsf(v));
+  }
+  store_finished<T>(a, fin, amax, off, red);
+}
+
+template <typename T>
 __global__ void __launch_bounds__(256) k_state_resume(state::Args a, int64_t first_tok,
                                                       int64_t n_tok) {
   for (int j = threadIdx.x; j < a.c; j += blockDim.x)
     state::resume_channel<T>(a, blockIdx.x, first_tok, n_tok, j);
+}
+
+// csa_encode_paged: entry first_entry + blockIdx.x of request blockIdx.y, given in the io
+// dtype (rows [B, n, c]), stored into its page in the format a.out exactly as
+// k_state_append stores a finished row.
+template <typename T>
+__global__ void __launch_bounds__(256) k_encode_paged(state::Args a, const void* rows,
+                                                      int64_t n, int64_t first_entry) {
+  extern __shared__ float fin[];  // [c]
+  __shared__ float red[32];
+  const int b = blockIdx.y;
+  size_t off = 0;
+  const int s = state::entry_offset(a, b, first_entry + blockIdx.x, &off);  // CTA-uniform
+  if (s != state::kCompress) {
+    if (threadIdx.x == 0) atomicCAS(&g_state_error, 0, kErrEncodeBase - s);
+    return;
+  }
+  const T* src = static_cast<const T*>(rows) + ((size_t)b * n + blockIdx.x) * (size_t)a.c;
+  float amax = 0.f;
+  for (int j = threadIdx.x; j < a.c; j += blockDim.x) {
+    const float v = state::ld(src, (size_t)j);
+    fin[j] = v;  // read back by this thread only
+    amax = fmaxf(amax, fabsf(v));
+  }
+  store_finished<T>(a, fin, amax, off, red);
 }
 
 }  // namespace
@@ -142,6 +177,19 @@ cudaError_t launch_state_append(const state::Args& a, bool bf16, cudaStream_t st
   cudaError_t e = bf16 ? launch(false, k_state_append<__nv_bfloat16>, dim3(a.B), dim3(threads),
                                 smem, st, a)
                        : launch(false, k_state_append<float>, dim3(a.B), dim3(threads), smem, st, a);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+cudaError_t launch_encode_paged(const state::Args& a, bool bf16, const void* rows, int64_t n,
+                                int64_t first_entry, cudaStream_t st) {
+  if (a.B == 0 || n == 0) return cudaSuccess;
+  const int threads = a.c >= 256 ? 256 : ((a.c + 31) / 32) * 32;
+  const size_t smem = (size_t)a.c * sizeof(float);
+  const dim3 grid((unsigned)n, (unsigned)a.B);
+  cudaError_t e = bf16 ? launch(false, k_encode_paged<__nv_bfloat16>, grid, dim3(threads), smem,
+                                st, a, rows, n, first_entry)
+                       : launch(false, k_encode_paged<float>, grid, dim3(threads), smem, st, a,
+                                rows, n, first_entry);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -72,19 +72,26 @@ CSA_HD size_t state_index(const Args& a, int64_t b, int64_t p, int r, int j) {
   return (((size_t)b * slots(a) + (size_t)(p % slots(a))) * rows(a) + r) * (size_t)a.c + j;
 }
 
+// Element offset in `pages` of the row of entry i of request b, through the page table:
+// kCompress, or kErrPageSlot / kErrPageId when the entry has no valid page.
+CSA_HD int entry_offset(const Args& a, int64_t b, int64_t i, size_t* out_off) {
+  const int64_t pg = i / a.page_rows;
+  if (pg >= a.max_pages) return kErrPageSlot;
+  const int32_t page = a.page_table[(size_t)b * a.max_pages + pg];
+  if (page < 0 || page >= a.n_pages) return kErrPageId;
+  *out_off = ((size_t)page * a.page_rows + (size_t)(i % a.page_rows)) * (size_t)a.c;
+  return kCompress;
+}
+
 // What the token at position t of request b does; for kCompress also the entry index and
 // the element offset of its row in `pages`.
 CSA_HD int append_status(const Args& a, int64_t b, int64_t t, int64_t* entry, size_t* out_off) {
   if (t < 0) return kErrPosition;
   if ((t + 1) % a.m != 0) return kAppendOnly;
   const int64_t i = t / a.m;
-  const int64_t pg = i / a.page_rows;
-  if (pg >= a.max_pages) return kErrPageSlot;
-  const int32_t page = a.page_table[(size_t)b * a.max_pages + pg];
-  if (page < 0 || page >= a.n_pages) return kErrPageId;
-  *entry = i;
-  *out_off = ((size_t)page * a.page_rows + (size_t)(i % a.page_rows)) * (size_t)a.c;
-  return kCompress;
+  const int s = entry_offset(a, b, i, out_off);
+  if (s == kCompress) *entry = i;
+  return s;
 }
 
 // Channel j of the new token: raw rows into the state, window row into the ring.

@@ -164,3 +164,41 @@ extern "C" int state_resume_host(int bf16, int B, int m, int c, int overlap, int
            : resume_channel<float>(a, b, first_tok, n_tok, j);
   return 0;
 }
+
+// csa_encode_paged's arithmetic: rows [B, n, c] (io dtype) = entries first_entry .. of every
+// request, stored through the page table in the format `out` (0 io, 1 FP8, 2 MXFP4, 3 mixed);
+// status[b * n + i] = the entry's status (1 stored, < 0 skipped).
+extern "C" int encode_paged_host(int bf16, int B, int64_t n, int64_t first_entry, int c,
+                                 int rope_dims, int out, int n_pages, int page_rows,
+                                 int max_pages, const void* rows, void* pages,
+                                 size_t page_bytes, void* page_scales, size_t scale_bytes,
+                                 const int32_t* page_table, int32_t* status) {
+  Args a{};
+  a.B = B; a.c = c; a.rope_dims = rope_dims; a.out = out; a.n_pages = n_pages;
+  a.page_rows = page_rows; a.max_pages = max_pages; a.pages = pages;
+  a.page_scales = page_scales; a.page_table = page_table;
+  std::vector<float> fin(c);
+  for (int b = 0; b < B; ++b)
+    for (int64_t i = 0; i < n; ++i) {
+      size_t off = 0;
+      const int s = entry_offset(a, b, first_entry + i, &off);
+      status[(size_t)b * n + i] = s;
+      if (s != kCompress) continue;
+      for (int j = 0; j < c; ++j) {
+        const size_t k = ((size_t)b * n + i) * c + j;
+        fin[j] = bf16 ? ld(static_cast<const __nv_bfloat16*>(rows), k)
+                      : ld(static_cast<const float*>(rows), k);
+      }
+      if (out == kOutIo) {
+        if ((off + c) * (bf16 ? 2 : 4) > page_bytes) return -12;
+        for (int j = 0; j < c; ++j) {
+          if (bf16) st(static_cast<__nv_bfloat16*>(pages) + off, j, fin[j]);
+          else st(static_cast<float*>(pages) + off, j, fin[j]);
+        }
+        continue;
+      }
+      const int rc = store_row(a, fin, off / (size_t)c, page_bytes, scale_bytes);
+      if (rc != 0) return rc;
+    }
+  return 0;
+}
