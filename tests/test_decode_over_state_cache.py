@@ -21,7 +21,9 @@ attention on those. Checks:
   - the output: the oracle's attention over the GPU's selection, within the bf16 output
     tolerance.
 The N_cap = 8192 case takes the decode top-k (histogram filled by the indexer), 1024 the
-row top-k. One case stores the KV entries as mixed-precision rows (e4m3 with a row scale,
+row top-k. In the prefill cases request 1 starts from a prefill chunk of 302 tokens handed
+over with csa_compress_paged / csa_compress + csa_encode_paged and csa_state_resume, and then
+decodes; the oracle takes every token one at a time. One case stores the KV entries as mixed-precision rows (e4m3 with a row scale,
 bf16 RoPE dims; 一(三)4): they must decode to within one step of each format of the
 oracle's entries, and the oracle attends its own mixed rows. The HCA case (m' = 128, pages
 of one entry, hca_dense_mqa_paged over the ring) attends every visible entry.
@@ -48,6 +50,7 @@ M, C, R, D_I, H, H_I, K, N_WIN = 4, 512, 64, 128, 64, 64, 64, 128
 BASE, EPS = 10000.0, 1e-6
 KV_ROWS, KEY_ROWS = 32, 128  # entries per page
 N_TOK = (1100, 517, 2051)    # tokens each request appends (129 visible keys: a page and one)
+PREFILL = 302                # with a prefill, request 1's first tokens come as one chunk
 
 
 class Stream:
@@ -124,8 +127,40 @@ def _up(x):
     return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).cuda()
 
 
-def run_gpu(st: Stream, bf16_scores: int, kv_fmt="bf16"):
-    """The appends and the forward call; returns host copies of the pools and the results."""
+def prefill_request(csa, torch, b, p_kv, p_key, kv_src, key_src, kv_desc, key_desc, kv_state,
+                    key_state, ring, mixed):
+    """Request b's first PREFILL tokens as a prefill chunk: the entries of its complete blocks
+    into the pages (bf16 KV: csa_compress_paged; mixed KV and MXFP4 keys: csa_compress in
+    fp32, then csa_encode_paged), then its raw tail and window into the state cache
+    (csa_state_resume)."""
+    n_full = PREFILL - PREFILL % M
+    f32 = lambda t: t.view(torch.bfloat16).float().contiguous()  # noqa: E731  (exact)
+    chunk = lambda src, k: src[k][b:b + 1, :n_full]  # noqa: E731
+    if not mixed:
+        csa.csa_compress_paged(p_kv, csa.CSA_BF16, 1, n_full, 0, chunk(kv_src, "Ca"),
+                               chunk(kv_src, "Cb"), chunk(kv_src, "Za"), chunk(kv_src, "Zb"),
+                               kv_src["bias"], None, None, None, 1, kv_desc)
+    for p, src, fin, desc, c, use in ((p_kv, kv_src, 1, kv_desc, C, mixed),
+                                      (p_key, key_src, 0, key_desc, D_I, True)):
+        if not use:
+            continue
+        tmp = torch.zeros((1, n_full // M, c), dtype=torch.float32, device="cuda")
+        csa.csa_compress(p, csa.CSA_F32, 1, n_full, 0, n_full // M, f32(chunk(src, "Ca")),
+                         f32(chunk(src, "Cb")), f32(chunk(src, "Za")), f32(chunk(src, "Zb")),
+                         f32(src["bias"]), None, None, None, fin, tmp)
+        csa.csa_encode_paged(p, csa.CSA_F32, 1, n_full // M, 0, tmp, desc)
+    tail = lambda src, k: src[k][b:b + 1, :PREFILL]  # noqa: E731
+    csa.csa_state_resume(p_kv, csa.CSA_BF16, 1, 0, PREFILL, tail(kv_src, "Ca"),
+                         tail(kv_src, "Cb"), tail(kv_src, "Za"), tail(kv_src, "Zb"),
+                         tail(kv_src, "win"), kv_state[b:b + 1], ring[b:b + 1])
+    csa.csa_state_resume(p_key, csa.CSA_BF16, 1, 0, PREFILL, tail(key_src, "Ca"),
+                         tail(key_src, "Cb"), tail(key_src, "Za"), tail(key_src, "Zb"), None,
+                         key_state[b:b + 1], None)
+
+
+def run_gpu(st: Stream, bf16_scores: int, kv_fmt="bf16", prefill=False):
+    """The appends (after a prefill chunk for request 1 when `prefill`) and the forward call;
+    returns host copies of the pools and the results."""
     import torch
     import long_context_sparse_08_b200 as csa
 
@@ -157,7 +192,16 @@ def run_gpu(st: Stream, bf16_scores: int, kv_fmt="bf16"):
         pos_all = torch.zeros((n, 2), dtype=torch.int64, device="cuda")
         pos_all[:, 0] = torch.arange(n, device="cuda")
         kv_tb, key_tb = up(st.kv_table[b:b + 1]), up(st.key_table[b:b + 1])
-        for t in range(n):
+        t0 = 0
+        if prefill and b == 1:
+            kv_desc = csa.paged_kv(kv_out, kv_pages, kv_scales, kv_tb, st.n_kv_pages, KV_ROWS,
+                                   kv_table.shape[1])
+            key_desc = csa.paged_kv(csa.CSA_MXFP4, key_pages, key_ex, key_tb, st.n_key_pages,
+                                    KEY_ROWS, key_table.shape[1])
+            prefill_request(csa, torch, b, p_kv, p_key, kv_src, key_src, kv_desc, key_desc,
+                            kv_state, key_state, ring, mixed)
+            t0 = PREFILL
+        for t in range(t0, n):
             pos = pos_all[t, :1]
             r = {k: v[b, t:t + 1] for k, v in kv_src.items() if k != "bias"}
             csa.csa_state_append(p_kv, csa.CSA_BF16, 1, pos, r["Ca"], r["Cb"], r["Za"], r["Zb"],
@@ -282,17 +326,20 @@ def check_selection_and_output(st, ora, got, off, bf16_scores):
         U.check_out(got["out"][b, 0], want, "bf16", f"request {b}: output")
 
 
-CASES = [(1024, 0, "bf16"), (1024, 1, "bf16"), (8192, 0, "bf16"), (8192, 1, "bf16"),
-         (8192, 0, "mixed")]
+CASES = [(1024, 0, "bf16", False), (1024, 1, "bf16", False), (8192, 0, "bf16", False),
+         (8192, 1, "bf16", False), (8192, 0, "mixed", False), (1024, 0, "bf16", True),
+         (8192, 1, "mixed", True)]
 
 
-@pytest.mark.parametrize("n_cap,bf16_scores,kv_fmt", CASES,
+@pytest.mark.parametrize("n_cap,bf16_scores,kv_fmt,prefill", CASES,
                          ids=[f"ncap{n}_{'bf16' if s else 'fp32'}_scores_{f}_kv"
-                              for n, s, f in CASES])
-def test_decode_step_over_the_state_cache(n_cap, bf16_scores, kv_fmt):
+                              f"{'_prefill' if pf else ''}" for n, s, f, pf in CASES])
+def test_decode_step_over_the_state_cache(n_cap, bf16_scores, kv_fmt, prefill):
+    """With `prefill`, request 1's first tokens are handed over from a prefill chunk; the
+    oracle still takes every token one at a time (its decode equals a whole prefill)."""
     st = Stream(n_cap)
     ora = oracle_caches(st, kv_fmt)
-    got = run_gpu(st, bf16_scores, kv_fmt)
+    got = run_gpu(st, bf16_scores, kv_fmt, prefill)
     off = check_pages(st, ora, got, kv_fmt)
     check_selection_and_output(st, ora, got, off, bf16_scores)
 
