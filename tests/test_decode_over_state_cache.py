@@ -225,11 +225,16 @@ def run_gpu(st: Stream, bf16_scores: int, kv_fmt="bf16", prefill=False):
     idx = torch.empty((B, 1, K), dtype=torch.int32, device="cuda")
     sc = torch.zeros((B, 1, st.n_cap), dtype=torch.int16 if bf16_scores else torch.float32,
                      device="cuda")
-    csa.csa_forward_paged(p_kv, B, 1, kv, keys, bf16_scores, up(st.qI), up(st.qI_scale),
-                          up(st.w), up(st.q), None, up(st.pos), ring, N_WIN, None, up(st.sink),
-                          idx, sc, out, ws, need)
+    args = (up(st.qI), up(st.qI_scale), up(st.w), up(st.q), None, up(st.pos), ring, N_WIN, None,
+            up(st.sink))
+    csa.csa_forward_paged(p_kv, B, 1, kv, keys, bf16_scores, *args, idx, sc, out, ws, need)
+    # a second run into fresh buffers must agree bit for bit (fixed-order combine, index
+    # tie-break: a race would show as a difference)
+    idx2, sc2, out2 = torch.empty_like(idx), torch.zeros_like(sc), torch.empty_like(out)
+    csa.csa_forward_paged(p_kv, B, 1, kv, keys, bf16_scores, *args, idx2, sc2, out2, ws, need)
     torch.cuda.synchronize()
     assert csa.device_error() == 0, "forward"
+    assert torch.equal(idx, idx2) and torch.equal(sc, sc2) and torch.equal(out, out2)
     scores = sc.cpu().numpy()
     scores = O.dec_bf16(scores.view(np.uint16)) if bf16_scores else scores.astype(np.float64)
     kvp = kv_pages.cpu().numpy()
