@@ -271,10 +271,6 @@ __device__ __forceinline__ float warp_reduce16(const float (&v)[16]) {
   const float other = __shfl_xor_sync(0xffffffffu, r, 1);
   return kMax ? fmaxf(r, other) : r + other;
 }
-// value index held by lane after warp_reduce16: j = 8*b4 + 4*b3 + 2*b2 + b1 (lane bits)
-__device__ __forceinline__ int reduce16_index(int lane) {
-  return ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
-}
 
 template <bool kMixed, bool kPaged>
 __global__ void __launch_bounds__(kThreads, 1)

@@ -28,7 +28,6 @@ namespace {
 constexpr int kBins = 4096;
 constexpr int kFThreads = 256;
 constexpr int kWarps = kFThreads / 32;
-constexpr int kBndCache = 2048;  // boundary entries kept in shared memory for the final pass
 constexpr int kDigitBits = 11;   // radix-select digit width
 constexpr int kDigits = 1 << kDigitBits;
 constexpr int kRankBnd = 2048;                 // boundary entries the rank path takes
