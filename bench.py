@@ -487,13 +487,14 @@ def _time_calls(fn, n_rep, warmup, steps):
 def check_part_workload(part, s):
     """Exit with a message when a part cannot run on the workload's caches (before any GPU
     work): the paged indexer and the BF16-score path take the tensor-core indexers' keys
-    (MXFP4, FP8 or bf16), the paged layer a CSA decode step, the layout comparison a decode
-    step."""
+    (MXFP4, FP8 or bf16), the paged layer and the layout comparison a decode step."""
     want = None
-    if part in ("bf16_scores", "forward_paged") and s.idx not in ("mxfp4", "fp8", "bf16"):
+    if part == "forward_paged" and s.kind == "hca_decode":
+        want = None  # the HCA layer: no indexer
+    elif part in ("bf16_scores", "forward_paged") and s.idx not in ("mxfp4", "fp8", "bf16"):
         want = "MXFP4, FP8 or bf16 indexer keys"
     elif part == "forward_paged" and s.kind != "csa_decode":
-        want = "a CSA decode step"
+        want = "a CSA or HCA decode step"
     elif part == "kv_layouts" and s.kind not in ("csa_decode", "hca_decode"):
         want = "a CSA or HCA decode step"
     if want:
@@ -510,7 +511,8 @@ def run_part(args, W):
     kv_layouts        the attention alone over bf16, mixed-precision and paged caches (CSA
                       or, on an HCA workload, the dense form);
     bf16_scores       index + top-k with fp32 and with BF16 scores;
-    forward_paged     the CSA layer over page pools and a window ring vs the contiguous one."""
+    forward_paged     the CSA (or HCA) layer over page pools and a window ring vs the
+                      contiguous one."""
     s = W.SHAPES[args.workload]
     check_part_workload(args.part, s)
     import torch
@@ -724,6 +726,43 @@ def run_part(args, W):
                     roofline={"bound": "tensor", "achieved": round(tf, 1), "peak": peak_tf,
                               "peak_source": peak_src, "unit": "TFLOP/s",
                               "frac": round(tf / peak_tf, 4), "flops_per_call": flops})
+    elif args.part == "forward_paged" and s.kind == "hca_decode":
+        # the HCA layer over a shuffled pool of one-entry pages with the window as a ring,
+        # against hca_dense_mqa on the contiguous cache and the linear window
+        inp = W.make_inputs(s)
+        dev = R.upload(inp, s)
+        p = R.params_for(s)
+        B, T, N = s.B, s.T, s.n_cap
+        g = torch.Generator(device="cpu").manual_seed(10)
+        perm = torch.randperm(B * N, generator=g).to(torch.int32).cuda()
+        table = perm.view(B, N)
+        pool = torch.empty((B * N, 1, s.c), dtype=dev["kv_cache"].dtype, device="cuda")
+        pool[perm.long()] = dev["kv_cache"].view(B * N, 1, s.c)
+        kv = csa.paged_kv(csa.CSA_BF16, pool, None, table, B * N, 1, N)
+        ring = torch.empty((B, s.n_win, s.c), dtype=dev["win_kv"].dtype, device="cuda")
+        for b in range(B):
+            t, p0 = int(inp["q_pos"][b, 0]), int(inp["win_pos0"][b])
+            for q0 in range(max(t - s.n_win + 1, 0), t + 1):
+                ring[b, q0 % s.n_win] = dev["win_kv"][b, q0 - p0]
+        need = csa.workspace_size(p, csa.CSA_WS_HCA_MQA, 0, B, T, N)
+        ws = torch.empty((max(need, 1),), dtype=torch.uint8, device="cuda")
+        out = torch.empty((B, T, s.n_heads, s.c), dtype=dev["q"].dtype, device="cuda")
+        L = dev["win_kv"].shape[1]
+        calls = {
+            "contiguous": lambda i: csa.hca_dense_mqa(
+                p, csa.CSA_BF16, B, T, dev["q"], dev["q_pos"], dev["kv_cache"], N, dev["win_kv"],
+                L, dev["win_pos0"], dev["sink"], None, out, ws, need),
+            "paged": lambda i: csa.hca_dense_mqa_paged(
+                p, B, T, dev["q"], dev["q_pos"], kv, ring, s.n_win, None, dev["sink"], None, out,
+                ws, need)}
+        res = {name: round(_time_calls(fn, 1, args.warmup, args.steps), 5)
+               for name, fn in calls.items()}
+        line.update(metric="HCA layer calls/s over the state cache's page pool",
+                    value=round(1e3 / res["paged"], 2), unit="calls/s (paged)",
+                    ms_per_call=res, config={"B": B, "T": T, "n_cap": N, "page_rows": 1,
+                                             "window": "ring"},
+                    roofline={"bound": "hbm (dense rows)", "peak": hbm, "peak_source": peak_src,
+                              "unit": "GB/s"})
     elif args.part == "forward_paged":
         # the CSA layer over page pools (KV pages of 32 entries, key pages of 128 keys, both
         # shuffled; the window as a ring) against csa_forward on the contiguous caches

@@ -102,11 +102,12 @@ def test_extension_bytes(bench):
 def test_parts_refuse_workloads_they_cannot_run(bench):
     # the checks run before any GPU work, so they can be exercised here
     for part in ("bf16_scores", "forward_paged"):
-        with pytest.raises(SystemExit, match="MXFP4, FP8 or bf16 indexer keys"):
-            bench.check_part_workload(part, W.SHAPES["hca_decode_1m"])
         bench.check_part_workload(part, W.SHAPES["flash_decode_131k"])
         bench.check_part_workload(part, W.SHAPES["pro_decode_1m"])
-    with pytest.raises(SystemExit, match="a CSA decode step"):
+    with pytest.raises(SystemExit, match="MXFP4, FP8 or bf16 indexer keys"):
+        bench.check_part_workload("bf16_scores", W.SHAPES["hca_decode_1m"])
+    bench.check_part_workload("forward_paged", W.SHAPES["hca_decode_1m"])  # the HCA layer
+    with pytest.raises(SystemExit, match="a CSA or HCA decode step"):
         bench.check_part_workload("forward_paged", W.SHAPES["flash_prefill_8k"])
     bench.check_part_workload("bf16_scores", W.SHAPES["flash_prefill_8k"])
     with pytest.raises(SystemExit, match="a CSA or HCA decode step"):
