@@ -64,7 +64,8 @@ def _mut_b_branch_same_block(Za, Zb, Ba, Bb, m, i, prev_Zb=None):
 
 def _mut_softmax_over_channels(logits):
     mx = logits.max(axis=1, keepdims=True)
-    e = np.exp(logits - mx)
+    with np.errstate(invalid="ignore"):  # rows of -inf (a sequence start) give NaN here
+        e = np.exp(logits - mx)
     return e / e.sum(axis=1, keepdims=True)
 
 
