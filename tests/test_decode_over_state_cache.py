@@ -375,17 +375,22 @@ class HcaStream:
             k += u
 
 
-def test_hca_decode_step_over_the_state_cache():
+@pytest.mark.parametrize("kv_fmt", ["bf16", "mixed"])
+def test_hca_decode_step_over_the_state_cache(kv_fmt):
     import torch
     import long_context_sparse_08_b200 as csa
 
     st = HcaStream()
+    mixed = kv_fmt == "mixed"
     B = st.B
     p = csa.make_params(m=HCA_M, overlap=0, c=C, rope_dims=R, rope_base=BASE, rms_eps=EPS,
                         n_heads=H, n_win=N_WIN)
     torch.cuda.synchronize()
     csa.device_error()
-    pages = torch.zeros((st.n_pages, 1, C), dtype=torch.int16, device="cuda")
+    pages = torch.zeros((st.n_pages, 1, C + R), dtype=torch.uint8, device="cuda") if mixed \
+        else torch.zeros((st.n_pages, 1, C), dtype=torch.int16, device="cuda")
+    scales = torch.zeros((st.n_pages, 1), dtype=torch.float32, device="cuda") if mixed else None
+    fmt = csa.CSA_MIXED_FP8_BF16 if mixed else csa.CSA_BF16
     state = torch.zeros((B, HCA_M, 2, C), dtype=torch.int16, device="cuda")
     ring = torch.zeros((B, N_WIN, C), dtype=torch.int16, device="cuda")
     src = {k: _up(st.kv[k]) for k in st.kv}
@@ -397,11 +402,11 @@ def test_hca_decode_step_over_the_state_cache():
             csa.csa_state_append(p, csa.CSA_BF16, 1, pos_all[t, :1], src["Ca"][b, t:t + 1], None,
                                  src["Za"][b, t:t + 1], None, src["win"][b, t:t + 1],
                                  src["bias"], None, 1, state[b:b + 1], ring[b:b + 1],
-                                 csa.CSA_BF16, pages, None, st.n_pages, 1, tb, HCA_N_CAP)
+                                 fmt, pages, scales, st.n_pages, 1, tb, HCA_N_CAP)
     torch.cuda.synchronize()
     assert csa.device_error() == 0, "appends"
     table = _up(st.table)
-    kv = csa.paged_kv(csa.CSA_BF16, pages, None, table, st.n_pages, 1, HCA_N_CAP)
+    kv = csa.paged_kv(fmt, pages, scales, table, st.n_pages, 1, HCA_N_CAP)
     need = csa.workspace_size(p, csa.CSA_WS_HCA_MQA, 0, B, 1, HCA_N_CAP)
     ws = torch.empty((max(need, 1),), dtype=torch.uint8, device="cuda")
     out = torch.empty((B, 1, H, C), dtype=torch.int16, device="cuda")
@@ -409,7 +414,9 @@ def test_hca_decode_step_over_the_state_cache():
                             _up(st.sink), None, out, ws, need)
     torch.cuda.synchronize()
     assert csa.device_error() == 0, "attention"
-    got_pages = pages.cpu().numpy().view(np.uint16)
+    got_pages = pages.cpu().numpy()
+    got_pages = got_pages if mixed else got_pages.view(np.uint16)
+    got_scales = scales.cpu().numpy() if mixed else None
     got = O.dec_bf16(out.cpu().numpy().view(np.uint16))
     for b, n in enumerate(HCA_N_TOK):
         pool = SC.PagePool(n // HCA_M + 1, 1, C)
@@ -419,10 +426,11 @@ def test_hca_decode_step_over_the_state_cache():
         for t in range(n):
             cs.append(r["Ca"][t], r["Za"][t], r["win"][t])
         ent = cs.entries()
-        U.check_rows(O.dec_bf16(got_pages[st.table[b, :len(ent)], 0]), ent, "bf16",
-                     f"HCA request {b}: entries")
+        pg = st.table[b, :len(ent)]
+        check_kv_rows(got_pages[pg, 0], None if got_scales is None else got_scales[pg, 0], ent,
+                      kv_fmt, f"HCA request {b}: entries")
         t = int(st.pos[b, 0])
-        want = O.hca_query(O.dec_bf16(st.q[b, 0]), t, stored_kv(ent, "bf16"),
+        want = O.hca_query(O.dec_bf16(st.q[b, 0]), t, stored_kv(ent, kv_fmt),
                            O.visible_entries(t, HCA_M, HCA_N_CAP), r["win"], 0, st.sink, r=R,
                            base=BASE, eps=EPS, scale=1.0 / math.sqrt(C), n_win=N_WIN)
         U.check_out(got[b, 0], want, "bf16", f"HCA request {b}: output")
