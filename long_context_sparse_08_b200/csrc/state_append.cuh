@@ -67,9 +67,13 @@ CSA_HD void st(__nv_bfloat16* p, size_t i, float v) { p[i] = __float2bfloat16_rn
 CSA_HD int slots(const Args& a) { return a.overlap ? 2 * a.m : a.m; }
 CSA_HD int rows(const Args& a) { return a.overlap ? 4 : 2; }
 
-// element (request b, token p, raw tensor r, channel j) of the state
+// element (request b, state slot, raw tensor r, channel j) of the state
+CSA_HD size_t slot_index(const Args& a, int64_t b, int slot, int r, int j) {
+  return (((size_t)b * slots(a) + (size_t)slot) * rows(a) + r) * (size_t)a.c + j;
+}
+// element (request b, token p, raw tensor r, channel j) of the state: token p in slot p mod S
 CSA_HD size_t state_index(const Args& a, int64_t b, int64_t p, int r, int j) {
-  return (((size_t)b * slots(a) + (size_t)(p % slots(a))) * rows(a) + r) * (size_t)a.c + j;
+  return slot_index(a, b, (int)(p % slots(a)), r, j);
 }
 
 // Element offset in `pages` of the row of entry i of request b, through the page table:
@@ -118,22 +122,29 @@ template <typename T>
 CSA_HD void resume_channel(const Args& a, int64_t b, int64_t first_tok, int64_t n_tok, int j) {
   T* s = static_cast<T*>(a.state);
   const int S = slots(a);
-  for (int64_t t = n_tok > S ? n_tok - S : 0; t < n_tok; ++t) {
+  // the slot (and ring row) of a token advance by one per token: one modulo per loop
+  const int64_t t0 = n_tok > S ? n_tok - S : 0;
+  int slot = (int)((first_tok + t0) % S);
+  for (int64_t t = t0; t < n_tok; ++t) {
     const size_t src = ((size_t)b * n_tok + t) * a.c + j;
-    const int64_t pabs = first_tok + t;
-    st(s, state_index(a, b, pabs, kRowCa, j), ld(static_cast<const T*>(a.Ca), src));
-    st(s, state_index(a, b, pabs, kRowZa, j), ld(static_cast<const T*>(a.Za), src));
+    st(s, slot_index(a, b, slot, kRowCa, j), ld(static_cast<const T*>(a.Ca), src));
+    st(s, slot_index(a, b, slot, kRowZa, j), ld(static_cast<const T*>(a.Za), src));
     if (a.overlap) {
-      st(s, state_index(a, b, pabs, kRowCb, j), ld(static_cast<const T*>(a.Cb), src));
-      st(s, state_index(a, b, pabs, kRowZb, j), ld(static_cast<const T*>(a.Zb), src));
+      st(s, slot_index(a, b, slot, kRowCb, j), ld(static_cast<const T*>(a.Cb), src));
+      st(s, slot_index(a, b, slot, kRowZb, j), ld(static_cast<const T*>(a.Zb), src));
+    }
+    slot = slot + 1 == S ? 0 : slot + 1;
+  }
+  if (a.win_ring != nullptr) {
+    const int64_t w0 = n_tok > a.n_win ? n_tok - a.n_win : 0;
+    int row = (int)((first_tok + w0) % a.n_win);
+    for (int64_t t = w0; t < n_tok; ++t) {
+      const size_t src = ((size_t)b * n_tok + t) * a.c + j;
+      const size_t dst = ((size_t)b * a.n_win + (size_t)row) * a.c + j;
+      st(static_cast<T*>(a.win_ring), dst, ld(static_cast<const T*>(a.win_row), src));
+      row = row + 1 == a.n_win ? 0 : row + 1;
     }
   }
-  if (a.win_ring != nullptr)
-    for (int64_t t = n_tok > a.n_win ? n_tok - a.n_win : 0; t < n_tok; ++t) {
-      const size_t src = ((size_t)b * n_tok + t) * a.c + j;
-      const size_t dst = ((size_t)b * a.n_win + (size_t)((first_tok + t) % a.n_win)) * a.c + j;
-      st(static_cast<T*>(a.win_ring), dst, ld(static_cast<const T*>(a.win_row), src));
-    }
 }
 
 // Channel j of entry i, pooled from the state: softmax over the block's logits plus biases
