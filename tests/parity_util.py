@@ -1,12 +1,14 @@
 """Comparison rules between the CUDA path and the float64 oracle.
 
 Tolerances (restated from the build's target):
-  - compressed entries and indexer scores agree to 1e-4 relative in fp32; for a score,
-    |dI| <= 1e-4 * A where A = sum_h |w_h| ReLU(q_h . k) >= |I| is the magnitude of the
-    terms summed (A = |I| when all w >= 0; with signed w it keeps the bound meaningful for
-    scores that cancel to near zero); a compressed row: ||d||/||ref|| <= 1e-4 and
-    |d| <= 1e-4 rms(ref);
-    a bf16 row is that fp32 bound plus one rounding to bf16 (half a bf16 ulp);
+  - compressed entries and indexer scores agree to 1e-4 relative in fp32. A score must
+    meet |dI| <= 1e-4 * max(|I|, 1e-3 * max_s |I|) (the "1e-4 relative" rule with a floor
+    at a thousandth of the row's largest score). The one exemption is a score that signed
+    head weights cancel: where |I| < A / 8, with A = sum_h |w_h| ReLU(q_h . k) >= |I| the
+    magnitude of the terms summed, fp32 rounding of the sum scales with A, not with |I|,
+    and such a score must instead meet |dI| <= 1e-4 * A. Every exemption is counted;
+  - a compressed row: ||d||/||ref|| <= 1e-4 and |d| <= 1e-4 rms(ref); a bf16 row is that
+    fp32 bound plus one rounding to bf16 (half a bf16 ulp);
   - top-k sets are identical except at near-ties: with tau the oracle's k-th largest score
     and tol = 1e-4 * max(|tau|, 1e-3 max|I|), every entry with I > tau + tol is selected and
     every selected entry has I >= tau - tol;
@@ -35,18 +37,47 @@ def dec_out(t, io: str) -> np.ndarray:
         t.cpu().numpy().astype(np.float64)
 
 
+# counts of the score checks in this process: scores checked, scores that meet the plain
+# relative rule, and cancellation exemptions (see the module docstring)
+SCORE_STATS = {"checked": 0, "relative": 0, "cancelled": 0}
+
+
+def score_limit(ref, scale):
+    """Per-score bound of the module docstring's rule: 1e-4 * max(|I|, 1e-3 * max|I|), and
+    for a cancelling score (|I| < A / 8) the larger of that and 1e-4 * A. Returns (bound,
+    mask of the scores where only the cancellation exemption can hold)."""
+    ref = np.asarray(ref, np.float64)
+    scale = np.asarray(scale, np.float64)
+    rel = 1e-4 * np.maximum(np.abs(ref), 1e-3 * np.abs(ref).max()) if ref.size else ref
+    cancel = np.abs(ref) < scale / 8
+    return np.where(cancel, np.maximum(rel, 1e-4 * scale), rel), cancel & (1e-4 * scale > rel)
+
+
 def check_scores(gpu: np.ndarray, ref: np.ndarray, scale: np.ndarray, what=""):
+    """Scores against the oracle under the rule of the module docstring. Returns
+    (n, n exempted as cancelling, worst error / the plain relative bound) and adds the
+    counts to SCORE_STATS."""
     ref = np.asarray(ref, np.float64)
     gpu = np.asarray(gpu, np.float64)
     scale = np.asarray(scale, np.float64)
     assert gpu.shape == ref.shape == scale.shape, what
     if ref.size == 0:
-        return
+        return 0, 0, 0.0
     assert np.all(scale >= np.abs(ref) * (1 - 1e-12)), f"{what}: scale below |I|"
     err = np.abs(gpu - ref)
-    bad = err > 1e-4 * scale
-    assert not bad.any(), (f"{what}: {bad.sum()} scores off; worst err/scale "
-                           f"{(err / np.maximum(scale, 1e-300)).max():.3e}")
+    rel = 1e-4 * np.maximum(np.abs(ref), 1e-3 * np.abs(ref).max())
+    lim, _ = score_limit(ref, scale)
+    bad = err > lim
+    assert not bad.any(), (f"{what}: {bad.sum()} scores off; worst err/bound "
+                           f"{(err / lim).max():.3e}")
+    n_c = int((err > rel).sum())  # passed only through the cancellation exemption
+    worst = float((err / rel).max())
+    SCORE_STATS["checked"] += ref.size
+    SCORE_STATS["relative"] += ref.size - n_c
+    SCORE_STATS["cancelled"] += n_c
+    print(f"[scores] {what}: n={ref.size} exempt(cancelling)={n_c} "
+          f"worst err/(1e-4 max(|I|,floor))={worst:.2e}")
+    return ref.size, n_c, worst
 
 
 def check_topk(gpu_idx: np.ndarray, ref_scores: np.ndarray, k: int, gpu_scores=None, what=""):

