@@ -439,7 +439,9 @@ csa_status csa_state_append(const csa_params* p, csa_dtype io, int32_t B, const 
               out_fmt == CSA_MIXED_FP8_BF16,
           "out_fmt must be the io dtype, CSA_FP8_E4M3_ROWSCALE, CSA_MXFP4 or CSA_MIXED_FP8_BF16");
   if (out_fmt == CSA_MIXED_FP8_BF16)
-    REQUIRE(p->rope_dims > 0 && p->rope_dims < p->c, "mixed rows need 0 < rope_dims < c");
+    REQUIRE(p->rope_dims > 0 && p->rope_dims < p->c && p->rope_dims % 16 == 0,
+            "mixed rows need 0 < rope_dims < c and rope_dims a multiple of 16 (16-byte "
+            "aligned rows, as the attention over mixed rows reads them)");
   if (out_fmt == CSA_MXFP4) {
     REQUIRE(p->c == 128, "MXFP4 rows are indexer keys of 128 values (c = %d)", p->c);
     REQUIRE(page_rows % 128 == 0, "MXFP4 pages hold whole 128-row exponent blocks");
@@ -501,7 +503,9 @@ csa_status csa_encode_paged(const csa_params* p, csa_dtype io, int32_t B, int64_
           "page format must be the io dtype, CSA_FP8_E4M3_ROWSCALE, CSA_MXFP4 or "
           "CSA_MIXED_FP8_BF16");
   if (fmt == CSA_MIXED_FP8_BF16)
-    REQUIRE(p->rope_dims > 0 && p->rope_dims < p->c, "mixed rows need 0 < rope_dims < c");
+    REQUIRE(p->rope_dims > 0 && p->rope_dims < p->c && p->rope_dims % 16 == 0,
+            "mixed rows need 0 < rope_dims < c and rope_dims a multiple of 16 (16-byte "
+            "aligned rows, as the attention over mixed rows reads them)");
   if (fmt == CSA_MXFP4) {
     REQUIRE(p->c == 128, "MXFP4 rows are indexer keys of 128 values (c = %d)", p->c);
     REQUIRE(out_pages->page_rows % 128 == 0, "MXFP4 pages hold whole 128-row exponent blocks");

@@ -208,10 +208,8 @@ cudaError_t launch_topk(const TopkArgs& a, void* ws, size_t ws_bytes, cudaStream
     return launch_topk_decode(topk_decode_args(a, ws), hist_ready, st);
   }
   if (a.scores16 != nullptr)
-    launch(false, k_topk_rows<__nv_bfloat16>, dim3(a.B * a.T), dim3(kThreads), 0, st, a);
-  else
-    launch(false, k_topk_rows<float>, dim3(a.B * a.T), dim3(kThreads), 0, st, a);
-  return cudaGetLastError();
+    return launch(false, k_topk_rows<__nv_bfloat16>, dim3(a.B * a.T), dim3(kThreads), 0, st, a);
+  return launch(false, k_topk_rows<float>, dim3(a.B * a.T), dim3(kThreads), 0, st, a);
 }
 
 }  // namespace csa

@@ -239,6 +239,11 @@ def test_state_append_checks():
     a = list(base)
     a[0], a[14], a[16] = ctypes.byref(norope), csa.CSA_MIXED_FP8_BF16, FAKE
     assert L.csa_state_append(*a) == csa.CSA_ERR_INVALID_ARG  # mixed rows need RoPE dims
+    for r in (8, 24, 40):  # the attention reads mixed rows in 16-byte pieces: r % 16 == 0
+        odd = _p(rope_dims=r)
+        a[0] = ctypes.byref(odd)
+        a[2] = 0  # even with nothing to append, a pool no reader accepts is refused
+        assert L.csa_state_append(*a) == csa.CSA_ERR_INVALID_ARG, r
     assert with_(out=csa.CSA_MIXED_FP8_BF16) == csa.CSA_ERR_INVALID_ARG  # no scales
     assert with_(out=csa.CSA_MIXED_FP8_BF16, scales=FAKE, B=0) == csa.CSA_OK
     hca = _p(overlap=0, m=128)

@@ -125,6 +125,11 @@ def test_checks_on_the_host():
     assert call(kv(csa.CSA_F32)) == csa.CSA_ERR_INVALID_ARG  # neither io nor a storage format
     assert call(kv(csa.CSA_MIXED_FP8_BF16), pp=csa.make_params(c=128, rope_dims=0)) == \
         csa.CSA_ERR_INVALID_ARG
+    for r in (8, 24, 40):  # mixed rows as the attention reads them: rope_dims % 16 == 0
+        assert call(kv(csa.CSA_MIXED_FP8_BF16), pp=csa.make_params(c=128, rope_dims=r)) == \
+            csa.CSA_ERR_INVALID_ARG, r
+    assert call(kv(csa.CSA_MIXED_FP8_BF16), n=0, pp=csa.make_params(c=128, rope_dims=32)) == \
+        csa.CSA_OK
     p512 = csa.make_params(c=512)
     assert L.csa_encode_paged(ctypes.byref(p512), csa.CSA_BF16, 2, 10, 0, F,
                               ctypes.byref(kv(csa.CSA_MXFP4)), None) == csa.CSA_ERR_INVALID_ARG
