@@ -363,9 +363,13 @@ def hca_dense_mqa_mixed_kv(p, B, T, q, q_pos, kv_rows, kv_scale, N_cap, win_kv, 
 
 
 def paged_kv(fmt, pages, scales, page_table, n_pages, page_rows, max_pages) -> CsaPagedKv:
-    """A csa_paged_kv over device tensors."""
-    return CsaPagedKv(int(fmt), _ptr(pages), _ptr(scales), _ptr(page_table), n_pages,
-                      page_rows, max_pages)
+    """A csa_paged_kv over device tensors. The descriptor holds only their addresses, so it
+    also keeps a reference to each tensor: a pool or page table passed as a temporary would
+    otherwise be freed at once, and its memory reused before the kernels read it."""
+    kv = CsaPagedKv(int(fmt), _ptr(pages), _ptr(scales), _ptr(page_table), n_pages,
+                    page_rows, max_pages)
+    kv._tensors = (pages, scales, page_table)
+    return kv
 
 
 def csa_sparse_mqa_paged(p, B, T, q, q_pos, kv: CsaPagedKv, idx, win_kv, L_raw, win_pos0, sink,

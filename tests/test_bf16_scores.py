@@ -9,14 +9,12 @@ values by (value desc, index asc). Checks:
     larger value selected, the smallest indices among the values equal to the last one,
     the list ordered, -1 past the visible count);
   - it differs from the oracle's own BF16 selection only at near-ties of the k-th value;
-  - its recall of the oracle's exact (unrounded) top-k is >= 0.99 (the pages report 99.7%
-    for their data; the synthetic scores give about the same).
-
-The kernels' bf16 store and selector instantiations have not yet run on a B200: the GPU
-tests run only with CSA_RUN_FIRST_GPU_CHECKS=1.
+  - its recall of the oracle's exact (unrounded) top-k equals that of the oracle's own BF16
+    selection up to the near-tie swaps, and averages >= 0.99 over a case's queries (the
+    pages report 99.7% for their data; the full-size Flash decode gives about 99.2% on the
+    synthetic N(0,1) scores, 98.4-99.6% per query).
 """
 import ctypes
-import os
 
 import numpy as np
 import pytest
@@ -27,7 +25,7 @@ from oracle import csa_oracle as O
 from oracle import pipeline as P
 import tests.parity_util as U
 
-CASES = ["edge_decode_fp8_tc", "edge_decode_bf16_tc", "mid_decode_fp8", "mid_prefill_bf16_tc",
+CASES = ["edge_decode_fp8_tc", "edge_decode_bf16_tc", "flash_decode_131k", "mid_prefill_bf16_tc",
          "edge_decode_mxfp4", "mid_decode_mxfp4"]
 
 
@@ -72,8 +70,6 @@ def _valid_selection(sel, R, k):
 
 
 @pytest.mark.gpu
-@pytest.mark.skipif(os.environ.get("CSA_RUN_FIRST_GPU_CHECKS") != "1",
-                    reason="awaiting its first run on a B200 (CSA_RUN_FIRST_GPU_CHECKS=1)")
 @pytest.mark.parametrize("name", CASES)
 def test_bf16_scores_and_selection(name):
     import torch
@@ -94,6 +90,7 @@ def test_bf16_scores_and_selection(name):
     assert csa.device_error() == 0
     got16 = sc16.cpu().numpy().view(np.uint16)
     idx = out_idx.cpu().numpy()
+    recalls = []
     for (b, ti), ref in res["scores"].items():
         n = ref.size
         g = O.dec_bf16(got16[b, ti, :n])
@@ -108,7 +105,16 @@ def test_bf16_scores_and_selection(name):
         theirs = O.topk_select_bf16(ref, s.topk)[:kk]
         tau = R_o[theirs[-1]]
         tol = U.bf16_ulp(np.array([tau]))[0] + 1e-4 * max(abs(tau), 1e-3 * np.abs(ref).max())
-        for i in mine.symmetric_difference(theirs.tolist()):
+        swaps = mine.symmetric_difference(theirs.tolist())
+        for i in swaps:
             assert abs(ref[i] - tau) <= tol, f"{name} b={b} t={ti}: {i} is not a near-tie"
+        # recall of the exact (unrounded) top-k: the GPU's equals the oracle's own BF16
+        # selection's up to the near-tie swaps, each of which moves it by at most 1/k
         exact = set(O.topk_select(ref, s.topk)[:kk].tolist())
-        assert len(mine & exact) / len(exact) >= 0.99
+        r_gpu, r_ora = len(mine & exact) / kk, len(set(theirs.tolist()) & exact) / kk
+        assert r_gpu >= r_ora - len(swaps) / (2 * kk) - 1e-12, f"{name} b={b} t={ti}: recall"
+        recalls.append(r_gpu)
+    if recalls:
+        print(f"[bf16 recall] {name}: mean {np.mean(recalls):.4f} min {np.min(recalls):.4f} "
+              f"over {len(recalls)} queries")
+        assert np.mean(recalls) >= 0.99, f"{name}: mean recall {np.mean(recalls):.4f}"

@@ -28,10 +28,8 @@ decodes; the oracle takes every token one at a time. One case stores the KV entr
 bf16 RoPE dims; 一(三)4): they must decode to within one step of each format of the
 oracle's entries, and the oracle attends its own mixed rows. The HCA case (m' = 128, pages
 of one entry, hca_dense_mqa_paged over the ring) attends every visible entry.
-Not yet run on a B200: the module runs only with CSA_RUN_FIRST_GPU_CHECKS=1.
 """
 import math
-import os
 
 import numpy as np
 import pytest
@@ -43,8 +41,6 @@ import tests.parity_util as U
 
 pytestmark = [
     pytest.mark.gpu,
-    pytest.mark.skipif(os.environ.get("CSA_RUN_FIRST_GPU_CHECKS") != "1",
-                       reason="awaiting its first run on a B200 (CSA_RUN_FIRST_GPU_CHECKS=1)"),
 ]
 
 M, C, R, D_I, H, H_I, K, N_WIN = 4, 512, 64, 128, 64, 64, 64, 128

@@ -9,10 +9,9 @@ mid-page and crossing pages; a page id outside the pool skips its entries (error
 leaves their rows untouched.
 
 The CPU tests run the kernel's arithmetic built for the host (tests/host_check); the device
-test runs the library's kernel (not yet on a B200: CSA_RUN_FIRST_GPU_CHECKS=1).
+test runs the library's kernel.
 """
 import ctypes
-import os
 import zlib
 
 import numpy as np
@@ -139,8 +138,6 @@ def test_checks_on_the_host():
 
 
 @pytest.mark.gpu
-@pytest.mark.skipif(os.environ.get("CSA_RUN_FIRST_GPU_CHECKS") != "1",
-                    reason="awaiting its first run on a B200 (CSA_RUN_FIRST_GPU_CHECKS=1)")
 @pytest.mark.parametrize("bad_page", [False, True], ids=["all_pages", "a_bad_page"])
 @pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
 def test_gpu_matches_the_encoders(case, bad_page):

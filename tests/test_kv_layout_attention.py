@@ -10,11 +10,7 @@ bytes exactly, and the kernel widens code * scale to bf16 before its tensor-core
 For paged caches the rows are scattered into a pool of pages through a shuffled page
 table, and the oracle reads the contiguous cache. The outputs must meet the bf16 output
 tolerance.
-
-These kernels have not yet run on a B200: the module runs only with
-CSA_RUN_FIRST_GPU_CHECKS=1, so a first run is a deliberate, separate step.
 """
-import os
 
 import numpy as np
 import pytest
@@ -28,8 +24,6 @@ import tests.parity_util as U
 
 pytestmark = [
     pytest.mark.gpu,
-    pytest.mark.skipif(os.environ.get("CSA_RUN_FIRST_GPU_CHECKS") != "1",
-                       reason="awaiting its first run on a B200 (CSA_RUN_FIRST_GPU_CHECKS=1)"),
 ]
 
 

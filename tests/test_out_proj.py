@@ -184,13 +184,11 @@ def test_gpu_decode_batch_of_forty_queries():
     _check(_run_gpu(inp, *shape), _oracle(inp, *shape), f"gpu {shape}")
 
 
-# prefill (tensor-core GEMMs): not yet run on a B200, so only with CSA_RUN_FIRST_GPU_CHECKS=1
+# prefill (tensor-core GEMMs)
 PREFILL = [(128, 8, 64, 2, 64, 128), (1000, 64, 512, 8, 1024, 4096)]
 
 
 @pytest.mark.gpu
-@pytest.mark.skipif(os.environ.get("CSA_RUN_FIRST_GPU_CHECKS") != "1",
-                    reason="awaiting its first run on a B200 (CSA_RUN_FIRST_GPU_CHECKS=1)")
 @pytest.mark.parametrize("shape", PREFILL, ids=["small", "flash_1000_queries"])
 def test_gpu_prefill_gemm_sampled(shape):
     Q, H, c, g, d_g, d = shape

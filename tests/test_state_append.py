@@ -517,15 +517,10 @@ def test_gpu_state_append_skips_requests_with_bad_pages():
 
 
 # ---------------------------------------------------------------------------
-# prefill -> decode hand-over on paged caches (not yet run on a B200: gated)
+# prefill -> decode hand-over on paged caches
 # ---------------------------------------------------------------------------
 
-_FIRST = pytest.mark.skipif(os.environ.get("CSA_RUN_FIRST_GPU_CHECKS") != "1",
-                            reason="awaiting its first run on a B200 (CSA_RUN_FIRST_GPU_CHECKS=1)")
-
-
 @pytest.mark.gpu
-@_FIRST
 def test_gpu_paged_compression_equals_contiguous():
     import torch
     import long_context_sparse_08_b200 as csa
@@ -552,7 +547,6 @@ def test_gpu_paged_compression_equals_contiguous():
 
 
 @pytest.mark.gpu
-@_FIRST
 @pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
 def test_gpu_resume_fills_the_state_of_a_prefill(case):
     import torch

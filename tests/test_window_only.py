@@ -3,12 +3,10 @@ DeepSeek-V4 三(二) 模型配置; the window of 一(三)3(3) with the sink of 3
 entries) is hca_dense_mqa with N_cap = 0: every query attends only its n_win most recent
 tokens. Checked against the oracle's HCA query with no visible entry, at positions before,
 at and past the first full window.
-
-Not yet run on a B200 (an empty cache with a NULL KV pointer takes the attention's window-only
-path for every request): runs only with CSA_RUN_FIRST_GPU_CHECKS=1.
+An empty cache with a NULL KV pointer takes the attention's window-only path for every
+request.
 """
 import math
-import os
 
 import numpy as np
 import pytest
@@ -19,8 +17,6 @@ import tests.parity_util as U
 
 pytestmark = [
     pytest.mark.gpu,
-    pytest.mark.skipif(os.environ.get("CSA_RUN_FIRST_GPU_CHECKS") != "1",
-                       reason="awaiting its first run on a B200 (CSA_RUN_FIRST_GPU_CHECKS=1)"),
 ]
 
 H, C, R, N_WIN, BASE, EPS = 64, 512, 64, 128, 10000.0, 1e-6
