@@ -165,8 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     Bf16IdxParams p) {
   using C = Cfg<kFp8, G>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* base = smem_align1024(smem_raw);
   uint8_t* opbase = base;                               // kOpN x 32 KB
   uint8_t* qbase = opbase + C::kOpN * kOpBytes;         // kQSlots x G x 16 KB
   uint8_t* stgbase = qbase + C::kQSlots * C::kQSlotBytes;  // fp8: kStg x 16 KB

@@ -135,8 +135,7 @@ __device__ __forceinline__ void index_mxf4_body(const CUtensorMap& tm_k, const C
                                                 const CUtensorMap& tm_q, const CUtensorMap& tm_qs,
                                                 const Mxf4Params& p, const Mxf4Ext& x) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* base = smem_align1024(smem_raw);
   uint8_t* qbase = base + kStages * kStageBytes;
   Smem& S = *reinterpret_cast<Smem*>(qbase + 2 * kQBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -278,8 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
              MqaTcParams P) {
   using Smem = SmemT<kMixed>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* base = smem_align1024(smem_raw);
   Smem& S = *reinterpret_cast<Smem*>(base + kOffEnd);
   const MqaArgs& a = P.a;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;

@@ -66,8 +66,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_out_proj_tc(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                   GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* base = smem_align1024(smem_raw);
   SmemG& S = *reinterpret_cast<SmemG*>(base + kStages * kStageBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int MT = (p.M + kBM - 1) / kBM, NT = (p.N + kBN - 1) / kBN, KB = (p.K + kBK - 1) / kBK;

@@ -23,6 +23,13 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
 
 __device__ __forceinline__ void set_error(int code) { atomicCAS(&g_device_error, 0, code); }
 
+// The first 1024-byte aligned byte of the dynamic shared memory `raw` (a pointer to the
+// kernel's extern __shared__ array), formed by an offset from `raw` so that the compiler
+// still knows every pointer derived from it addresses shared memory.
+__device__ __forceinline__ uint8_t* smem_align1024(uint8_t* raw) {
+  return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
+
 // ---------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------

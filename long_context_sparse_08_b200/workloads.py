@@ -177,6 +177,11 @@ class Shape:
     bias_std: float = 1.0
     overlap: int = 1
     q_pos_override: tuple = ()  # explicit per-request decode positions (edge cases)
+    # degenerate selections: requests whose indexer head weights are all zero (every score
+    # 0: the whole row ties), and a request whose indexer keys repeat with this period
+    # (groups of equal scores at distinct indices)
+    w_zero_requests: tuple = ()
+    dup_keys: tuple = ()  # (request, period)
 
 
 SHAPES: Dict[str, Shape] = {}
@@ -239,6 +244,17 @@ _reg(Shape("edge_decode_mxfp4", "csa_decode", "bf16", "mxfp4", B=5, T=1, m=4, c=
 _reg(Shape("edge_decode_mxfp4_long", "csa_decode", "bf16", "mxfp4", B=4, T=1, m=4, c=512,
            rope_dims=64, n_heads=128, n_idx_heads=64, d_idx=128, topk=1024, n_win=128,
            n_cap=16384, ctx=0, seed=19, q_pos_override=(4 * 16384 + 301, 48001, 13, 4100)))
+# MXFP4 decode cases on the decode selector path (N_cap >= 8192): many CTAs per request,
+# full visibility, exactly k and fewer than k visible entries, an empty request; and one
+# with heavy ties (a request whose head weights are zero, one whose keys repeat).
+_reg(Shape("mid_decode_mxfp4_sel", "csa_decode", "bf16", "mxfp4", B=6, T=1, m=4, c=512,
+           rope_dims=64, n_heads=128, n_idx_heads=64, d_idx=128, topk=1024, n_win=128,
+           n_cap=24576, ctx=0, seed=23,
+           q_pos_override=(4 * 24576 + 3, 80007, 4 * 1024 + 2, 4 * 1023 + 1, 3, 20001)))
+_reg(Shape("edge_decode_mxfp4_ties", "csa_decode", "bf16", "mxfp4", B=3, T=1, m=4, c=512,
+           rope_dims=64, n_heads=128, n_idx_heads=64, d_idx=128, topk=1024, n_win=128,
+           n_cap=12288, ctx=0, seed=24, q_pos_override=(4 * 12288, 4 * 12288 + 1, 30000),
+           w_zero_requests=(0,), dup_keys=(1, 64)))
 # Tensor-core indexer cases for fp8 and bf16 keys (cache capacity a multiple of 128): zero
 # tiles, a single partial tile, several tiles, and more positions than the cache holds.
 _reg(Shape("edge_decode_fp8_tc", "csa_decode", "bf16", "fp8", B=5, T=1, m=4, c=512,
@@ -373,6 +389,9 @@ def make_inputs(s: Shape, *, seed: Optional[int] = None) -> Dict[str, np.ndarray
     if s.kind == "csa_decode":
         qI = _normal(g, (B, T, s.n_idx_heads, s.d_idx))
         KI = _normal(g, (B, s.n_cap, s.d_idx))
+        if s.dup_keys:
+            rb, period = s.dup_keys
+            KI[rb] = np.tile(KI[rb, :period], (s.n_cap // period, 1))
         if s.idx == "bf16":
             out["qI"], out["KI"] = f32_to_bf16_bits(qI), f32_to_bf16_bits(KI)
         elif s.idx == "fp8":
@@ -387,6 +406,8 @@ def make_inputs(s: Shape, *, seed: Optional[int] = None) -> Dict[str, np.ndarray
         else:
             raise ValueError(s.idx)
         out["w"] = _normal(g, (B, T, s.n_idx_heads))
+        for rb in s.w_zero_requests:
+            out["w"][rb] = 0.0
     out["sink"] = _normal(g, (H,))
     return out
 

@@ -26,7 +26,7 @@ from oracle import pipeline as P
 import tests.parity_util as U
 
 CASES = ["edge_decode_fp8_tc", "edge_decode_bf16_tc", "flash_decode_131k", "mid_prefill_bf16_tc",
-         "edge_decode_mxfp4", "mid_decode_mxfp4"]
+         "edge_decode_mxfp4", "mid_decode_mxfp4", "mid_decode_mxfp4_sel"]
 
 
 def test_checks_on_the_host():

@@ -244,6 +244,10 @@ def _forward_parity(name, queries=None):
         U.check_scores(scores[b, ti, :ref.size], ref, res["scale"][(b, ti)],
                        f"{name} b={b} t={ti} scores")
         U.check_topk(idx[b, ti], ref, s.topk, scores[b, ti], f"{name} b={b} t={ti} top-k")
+        # the selector is exact: the GPU's selection is the top-k of the GPU's own scores
+        np.testing.assert_array_equal(
+            idx[b, ti], O.topk_select(scores[b, ti, :ref.size].astype(np.float64), s.topk),
+            err_msg=f"{name} b={b} t={ti}: selection of the GPU's own scores")
     if res["chunk"] is not None:
         first = s.ctx // s.m
         got_chunk = U.dec_out(dev["kv_cache"][0, first:first + s.n_tok // s.m], s.io)
@@ -290,7 +294,8 @@ def _mxfp4_recall_vs_fp32(s, inp, idx, res, what):
                                   "mid_decode_bf16", "edge_decode_bf16", "edge_decode_mxfp4",
                                   "edge_decode_mxfp4_long", "mid_prefill_bf16",
                                   "edge_decode_fp8_tc", "edge_decode_bf16_tc",
-                                  "mid_prefill_bf16_tc"])
+                                  "mid_prefill_bf16_tc", "mid_decode_mxfp4_sel",
+                                  "edge_decode_mxfp4_ties"])
 def test_forward_parity(name):
     s, inp, st, res = _forward_parity(name)
     if s.idx == "mxfp4":
@@ -333,8 +338,22 @@ def test_no_bounded_wait_gave_up():
     assert csa.device_error() == 0
 
 
-def test_forward_is_deterministic():
-    s, inp = U.inputs("mid_decode_mxfp4")
+def test_tied_scores_select_the_smallest_indices():
+    # every head weight of request 0 is zero, so all its scores are 0 and the selection is
+    # its k smallest indices; request 1's keys repeat every 64 rows, so its scores come in
+    # classes of equal values and the smallest indices of the last class taken win
+    s, inp, dev, st = _step("edge_decode_mxfp4_ties")
+    idx = st.out_idx.cpu().numpy()
+    np.testing.assert_array_equal(idx[0, 0], np.arange(s.topk))
+    sc = st.scores.cpu().numpy()[1, 0]
+    assert np.all(sc.reshape(-1, 64) == sc[:64][None, :]), "repeated keys must score alike"
+    np.testing.assert_array_equal(idx[1, 0], O.topk_select(sc.astype(np.float64), s.topk))
+    assert csa.device_error() == 0
+
+
+@pytest.mark.parametrize("name", ["mid_decode_mxfp4", "mid_decode_mxfp4_sel"])
+def test_forward_is_deterministic(name):
+    s, inp = U.inputs(name)
     dev = R.upload(inp, s)
     st = R.Step(s, dev, want_scores=True)
     st()

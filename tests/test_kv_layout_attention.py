@@ -183,7 +183,7 @@ def test_paged_cache_with_a_bad_page_id_reports_it():
 
 @pytest.mark.parametrize("name", ["edge_decode_fp8_tc", "edge_decode_bf16_tc",
                                   "mid_prefill_bf16_tc", "edge_decode_mxfp4",
-                                  "edge_decode_mxfp4_long"])
+                                  "edge_decode_mxfp4_long", "mid_decode_mxfp4_sel"])
 @pytest.mark.parametrize("bf16_scores", [0, 1])
 @pytest.mark.parametrize("holes", [False, True], ids=["all_pages", "unallocated_tail"])
 def test_index_topk_over_paged_keys_equals_contiguous(name, bf16_scores, holes):
@@ -271,7 +271,7 @@ def _paged_forward(s, inp, dev, kv_fmt, kv_rows, kv_scale, bf16_scores, ring=Non
 
 
 @pytest.mark.parametrize("name", ["edge_decode_fp8_tc", "edge_decode_bf16_tc",
-                                  "edge_decode_mxfp4"])
+                                  "edge_decode_mxfp4", "mid_decode_mxfp4_sel"])
 def test_forward_paged_equals_contiguous(name):
     s, inp = U.inputs(name)
     dev = R.upload(inp, s)
