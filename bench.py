@@ -42,6 +42,12 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--streams", type=int, default=1,
+                    help="CUDA streams the steps alternate over (independent batches in flight; "
+                         "1: one step after another)")
+    ap.add_argument("--concurrent", type=int, default=3,
+                    help="also time the steps over this many streams and report it as an extra "
+                         "key (0: skip); `value` stays that of --streams")
     ap.add_argument("--rounds", type=int, default=5,
                     help="timed rounds of K steps each; the median round gives the value")
     ap.add_argument("--workload", default="pro_decode_1m")
@@ -229,6 +235,9 @@ def run_ours(args, W, rank, world, local_rank):
         R_rep -= 1
     if args.replicas > 0:
         R_rep = args.replicas
+    S_str = max(1, args.streams)
+    S_all = max(S_str, args.concurrent if args.concurrent > 1 else 1)
+    R_rep = -(-R_rep // S_all) * S_all  # a multiple of the streams: a replica stays on one stream
     devs = [dev0] + [{k: v.clone() for k, v in dev0.items()} for _ in range(R_rep - 1)]
     for d in devs:  # per-query inputs side by side, so one copy uploads a step's inputs
         pack_query_inputs(d)
@@ -249,18 +258,37 @@ def run_ours(args, W, rank, world, local_rank):
     rounds = max(1, args.rounds)
     t0 = [torch.cuda.Event(enable_timing=True) for _ in range(rounds)]
     t1 = [torch.cuda.Event(enable_timing=True) for _ in range(rounds)]
+    side_all = [torch.cuda.Stream() for _ in range(S_all - 1)]
+
+    def timed_rounds(n_streams):
+        """ms of each round of K steps, the steps alternating over n_streams streams."""
+        side = side_all[:n_streams - 1]
+        strs = [stream] + side
+        for r in range(rounds):
+            t0[r].record(stream)
+            for sd in side:  # every stream starts after the round's start event
+                sd.wait_event(t0[r])
+            for i in range(K):
+                j = r * K + i
+                steps[j % R_rep](strs[j % n_streams])
+            for sd in side:  # and the round ends when every stream has drained
+                ev = torch.cuda.Event()
+                ev.record(sd)
+                stream.wait_event(ev)
+            t1[r].record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in zip(t0, t1)]
+
     launches0 = csa.kernel_launches()
-    for r in range(rounds):
-        t0[r].record(stream)
-        for i in range(K):
-            steps[(r * K + i) % R_rep]()
-        t1[r].record(stream)
+    ms_rounds = timed_rounds(S_str)
     launches = (csa.kernel_launches() - launches0) // rounds
-    torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
+    conc = None
+    if S_all > S_str:  # the same steps with more independent batches in flight
+        conc_rounds = timed_rounds(S_all)
+        conc = float(np.median(conc_rounds))
     clk = clocks.stop()
-    ms_rounds = [a.elapsed_time(b) for a, b in zip(t0, t1)]
     ms = float(np.median(ms_rounds))
     # The dominant kernel (the indexer) is timed by events around each of its launches over
     # a second pass of the same K steps: events between the kernels of a step would stop
@@ -279,6 +307,18 @@ def run_ours(args, W, rank, world, local_rank):
         torch.cuda.synchronize()
         idx_ms = sum(b.elapsed_time(a) for b, a in zip(ev_b, ev_a)) / K
         csa.set_index_timing_events([], [])
+    att_ms = None
+    if not has_index:
+        # HCA: the step is the dense attention call (attention kernel + split merge); events
+        # around each call, in a second pass of the same K steps
+        ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        for i in range(K):
+            ev_b[i].record(stream)
+            steps[i % R_rep]()
+            ev_a[i].record(stream)
+        torch.cuda.synchronize()
+        att_ms = sum(b.elapsed_time(a) for b, a in zip(ev_b, ev_a)) / K
     ms = max_over_ranks(ms, world, "cuda")
 
     # end to end through the public API: per-step query-side inputs from pinned host
@@ -305,6 +345,18 @@ def run_ours(args, W, rank, world, local_rank):
                 "traffic": traffic_from_profile(src, "k_index_bf16_tc", s.name),
                 "alg_flops_per_step": fl, "avg_ms_per_step": round(idx_ms, 5),
                 "peak_source": f"{peak_src} bf16_tflops_sustained (cuBLAS, seconds-long loop)"}
+    elif att_ms:
+        alg = queries * per_q["total"]
+        achieved = alg / (att_ms / 1e3) / 1e9
+        src = os.path.join(ROOT, "long_context_sparse_08_b200", "csrc", "mqa_tc.cu")
+        roof = {"kernel": "k_mqa_tc (dense) + k_mqa_combine", "bound": "hbm",
+                "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
+                "nominal_peak": NOMINAL_HBM_GBS,
+                "traffic": traffic_from_profile(src, "k_mqa_tc", s.name),
+                "alg_bytes_per_launch": alg, "avg_launch_ms": round(att_ms, 5),
+                "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)"}
     elif has_index and idx_ms:
         alg = queries * per_q["index"]
         achieved = alg / (idx_ms / 1e3) / 1e9
@@ -331,7 +383,7 @@ def run_ours(args, W, rank, world, local_rank):
         "metric": METRIC, "value": round(value, 2), "unit": "queries/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms / K, 5),
         "rounds": {"n": rounds, "ms_per_step": [round(x / K, 5) for x in ms_rounds],
-                   "value_from": "median round"},
+                   "value_from": "median round", "streams": S_str},
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": {"mxfp4": "mxfp4+bf16", "fp8": "e4m3+bf16", "bf16": "bf16",
                   "none": "bf16", "f32": "f32"}[s.idx],
@@ -340,12 +392,20 @@ def run_ours(args, W, rank, world, local_rank):
             s, l2=f"{R_rep} rotating input replicas ({R_rep * one_set / 1e9:.2f} GB); "
                   f"bytes touched per cycle {R_rep * step_bytes / 1e6:.0f} MB > L2",
             parallelism=f"replicas x{world} (independent requests)"),
-        "step_hbm_roofline": {"alg_bytes_per_step": step_bytes,
-                              "frac_of_peak": round(step_bytes / (ms / K / 1e3) / 1e9 /
-                                                    peaks["hbm_gbs"], 4),
-                              "frac_of_nominal": round(step_bytes / (ms / K / 1e3) / 1e9 /
-                                                       NOMINAL_HBM_GBS, 4)},
+        # decode steps are bounded by HBM; a prefill chunk is compared with the tensor peak
+        # instead (`tflops` below)
+        "step_hbm_roofline": None if s.kind == "csa_prefill" else {
+            "alg_bytes_per_step": step_bytes,
+            "frac_of_peak": round(step_bytes / (ms / K / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+            "frac_of_nominal": round(step_bytes / (ms / K / 1e3) / 1e9 / NOMINAL_HBM_GBS, 4)},
         "roofline": roof,
+        "concurrent_batches": None if conc is None else {
+            "streams": S_all, "batches_in_flight": S_all,
+            "value": round(whole_job_rate(world, queries, K, max_over_ranks(conc, world, "cuda")), 2),
+            "unit": "queries/s", "ms_per_step": round(conc / K, 5),
+            "note": "the same steps, each a whole csa_forward over its own batch, alternating "
+                    "over streams so that several independent batches are in flight; `value` "
+                    "is the one-batch-at-a-time figure"},
         "clocks": clk,
         "e2e": e2e,
         "gpu_launches": launches,
