@@ -48,18 +48,26 @@ namespace {
 using namespace tc;
 
 constexpr int kC = 512;          // head dim
-constexpr int kRows = 128;       // KV rows per chunk (MMA M of S^T)
 constexpr int kHg = 64;          // heads per CTA (MMA N)
 constexpr int kThreads = 160;    // warps 0-3: loads + softmax + epilogue; warp 4: MMA
 constexpr int kAtoms = kC / 64;  // 64-element (128 B) swizzle atoms along a row
 constexpr float kLazy = 8.f;     // rescale threshold (natural-log units)
 constexpr int kMaxPairs = 256;   // RoPE pairs (r / 2)
 
-// shared memory (offsets from a 1024-aligned base)
-constexpr int kOffKV = 0;                                // [atom][row][128 B]  128 KB
-constexpr int kOffQ = kOffKV + kAtoms * kRows * 128;     // [atom][head][128 B]  64 KB
-constexpr int kOffP = kOffQ + kAtoms * kHg * 128;        // [row][128 B]         16 KB
-constexpr int kOffEnd = kOffP + kRows * 128;
+// Shared memory (offsets from a 1024-aligned base) for chunks of kR KV rows: kR = 128 with
+// one KV buffer, or kR = 64 with two (the next chunk's rows arrive while this one's products
+// and softmax run). 208 KB either way; the KV area also stages the 64 raw query rows (64 KB)
+// before q_hat is built.
+template <int kR>
+struct Lay {
+  static constexpr int kBuf = kR == 64 ? 2 : 1;
+  static constexpr int kSlotKV = kAtoms * kR * 128;                   // [atom][row][128 B]
+  static constexpr int kOffKV = 0;
+  static constexpr int kOffQ = kOffKV + kBuf * kSlotKV;              // [atom][head][128 B]
+  static constexpr int kSlotP = kR * 128;                             // [row / 64][head][128 B]
+  static constexpr int kOffP = kOffQ + kAtoms * kHg * 128;
+  static constexpr int kOffEnd = kOffP + kBuf * kSlotP;
+};
 
 // TMEM columns
 constexpr uint32_t kTmemCols = 512;
@@ -68,16 +76,20 @@ constexpr uint32_t kColO = 256;   // O^T slice s: 256 + 64 s
 
 enum { kErrKvFull = 201, kErrSFull = 202, kErrPFull = 203, kErrKvFree = 204, kErrPageId = 205 };
 
-template <bool kMixed>
+template <bool kMixed, int kR>
 struct SmemT {
-  uint64_t kv_full, s_full, p_full, kv_free, done;
+  static constexpr int kBuf = Lay<kR>::kBuf;
+  uint64_t kv_full[kBuf], s_full[kBuf], p_full[kBuf], kv_free[kBuf], done;
   uint32_t tmem_slot;
-  uint32_t vmask[4];  // valid rows of the current chunk (bit j of word w: row 32w + j)
+  uint32_t vmask[kBuf][kR / 32];  // valid rows of a buffered chunk (bit j of word w: row 32w + j)
   float m_used[kHg], l_sum[kHg], alpha[kHg], fin[kHg];
   float cs[kMaxPairs], sn[kMaxPairs];  // RoPE table for pairs of the last r dims
   float wq[kC];                         // query RMSNorm weights
-  const __nv_bfloat16* src[kRows];  // source rows of the current chunk (nullptr: masked)
-  float rscale[kMixed ? kRows : 1];  // mixed rows: the row's FP8 scale; bf16 rows: -1
+  // per buffer: source rows of the chunk being gathered (nullptr: masked) and, for mixed
+  // rows, the row's FP8 scale (bf16 rows: -1); one set per buffer, since the next chunk's
+  // rows are resolved while other warps may still be copying this one's
+  const __nv_bfloat16* src[kBuf][kR];
+  float rscale[kBuf][kMixed ? kR : 1];
 };
 
 struct MqaTcParams {
@@ -272,11 +284,14 @@ __device__ __forceinline__ float warp_reduce16(const float (&v)[16]) {
   return kMax ? fmaxf(r, other) : r + other;
 }
 
-template <bool kMixed, bool kPaged>
+template <bool kMixed, bool kPaged, int kRows>
 __global__ void __launch_bounds__(kThreads, 1)
     k_mqa_tc(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_win,
              MqaTcParams P) {
-  using Smem = SmemT<kMixed>;
+  using Smem = SmemT<kMixed, kRows>;
+  using L = Lay<kRows>;
+  constexpr int kBuf = L::kBuf, kOffKV = L::kOffKV, kOffQ = L::kOffQ, kOffP = L::kOffP,
+                kOffEnd = L::kOffEnd;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_align1024(smem_raw);
   Smem& S = *reinterpret_cast<Smem*>(base + kOffEnd);
@@ -294,10 +309,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 4) {
     if (lane == 0) {
-      mbar_init(&S.kv_full, 129);  // the 128 loading threads + the TMA issue or its stand-in
-      mbar_init(&S.s_full, 1);
-      mbar_init(&S.p_full, 128);
-      mbar_init(&S.kv_free, 1);
+      for (int i = 0; i < kBuf; ++i) {
+        mbar_init(&S.kv_full[i], 129);  // the 128 loading threads + the TMA issue or its stand-in
+        mbar_init(&S.s_full[i], 1);
+        mbar_init(&S.p_full[i], 128);
+        mbar_init(&S.kv_free[i], 1);
+      }
       mbar_init(&S.done, 1);
       fence_barrier_init();
     }
@@ -391,36 +408,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int atom = d0 >> 6, chunk = (d0 & 63) >> 3;
         *reinterpret_cast<uint4*>(qs + atom * (kHg * 128) + sw128(qh, chunk)) = o;
       }
+      // the tile is read by the tensor cores, also when a chunk's rows come by TMA (whose
+      // arrival carries no fence of these stores)
+      fence_proxy_async_smem();
     }
 
     // the selected rows, the partials and the output belong to the previous kernels
     pdl_wait();
     pdl_trigger();
     bool ok = true;
-    const uint32_t kv_base = smem_u32(base + kOffKV);
     const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
     const bool head_thr = lane < 16;  // lanes 0-15: the softmax of head hh
     const int hh = 16 * warp + (lane & 15);
     float mu_h = -INFINITY, l_h = 0.f;  // running max used and running sum of this head
-#pragma unroll 1
-    for (int j = c0; j < c1 && ok; ++j) {
-      const uint32_t it = (uint32_t)(j - c0);
-      if (j > c0) ok = all_ok_softmax(mbar_wait(&S.kv_free, (it - 1) & 1, kErrKvFree));
-      if (!ok) break;
-      // ---- gather the chunk's 128 rows: thread r resolves row r, then warp w copies rows
-      //      w, w+4, ... with lane = 16-byte chunk (coalesced 512 B per instruction) ----
-      const __nv_bfloat16* my_src;
-      if constexpr (kMixed || kPaged) {
-        float sc;
-        my_src = static_cast<const __nv_bfloat16*>(
-            row_src_ext<kMixed, kPaged>(a, bt, b, rl, (int64_t)j * kRows + tid, &sc));
-        if constexpr (kMixed) S.rscale[tid] = sc;
-      } else {
-        my_src = row_src(a, bt, b, rl, (int64_t)j * kRows + tid);
+    // A chunk's rows are gathered in two steps: the issue (rows resolved, copies or TMA boxes
+    // started; returns whether TMA fills the slot) and the finish (cp.async copies: wait for
+    // this thread's, make them visible to the tensor cores; then arrive). With two buffers the
+    // next chunk is issued before this one's softmax and finished after it.
+    auto gather_issue = [&](int j, int slot) -> bool {
+      // ---- rows of chunk j into KV slot `slot`: thread r resolves row r, then warp w copies
+      //      rows w, w+4, ... with lane = 16-byte chunk (coalesced 512 B per instruction) ----
+      const uint32_t kv_base = smem_u32(base + kOffKV + slot * L::kSlotKV);
+      uint8_t* const kv_ptr = base + kOffKV + slot * L::kSlotKV;
+      const __nv_bfloat16* my_src = nullptr;
+      if (tid < kRows) {
+        if constexpr (kMixed || kPaged) {
+          float sc;
+          my_src = static_cast<const __nv_bfloat16*>(
+              row_src_ext<kMixed, kPaged>(a, bt, b, rl, (int64_t)j * kRows + tid, &sc));
+          if constexpr (kMixed) S.rscale[slot][tid] = sc;
+        } else {
+          my_src = row_src(a, bt, b, rl, (int64_t)j * kRows + tid);
+        }
+        S.src[slot][tid] = my_src;
       }
-      S.src[tid] = my_src;
       const uint32_t vb = __ballot_sync(0xffffffffu, my_src != nullptr);
-      if (lane == 0) S.vmask[warp] = vb;
+      if (lane == 0 && warp < kRows / 32) S.vmask[slot][warp] = vb;
       // a chunk of 128 contiguous rows (dense entries, or window rows) comes by TMA: eight
       // 128B-swizzled boxes issued by one thread instead of 64 cp.async per thread
       const int64_t r0 = (int64_t)j * kRows;
@@ -439,11 +462,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       bar_softmax();
       if (tmap != nullptr) {
         if (tid == 0) {
-          mbar_arrive_expect_tx(&S.kv_full, kRows * kC * 2);
+          mbar_arrive_expect_tx(&S.kv_full[slot], kRows * kC * 2);
 #pragma unroll
           for (int atom = 0; atom < kAtoms; ++atom)
-            tma_load_2d(base + kOffKV + atom * (kRows * 128), tmap, 64 * atom, trow, &S.kv_full);
+            tma_load_2d(kv_ptr + atom * (kRows * 128), tmap, 64 * atom, trow, &S.kv_full[slot]);
         }
+        return true;
       } else {
         if constexpr (kMixed) {
           // a warp takes rows w, w+4, ...: a mixed row's lanes 0..27 widen 16 codes each
@@ -453,8 +477,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int r = a.rope_dims, nope = kC - r;  // nope = 448 (c = 512, r = 64)
 #pragma unroll 1
           for (int rr = warp; rr < kRows; rr += 4) {
-            const __nv_bfloat16* src = S.src[rr];
-            const float sc = S.rscale[rr];
+            const __nv_bfloat16* src = S.src[slot][rr];
+            const float sc = S.rscale[slot][rr];
             if (src == nullptr || sc < 0.f) {
 #pragma unroll
               for (int hseg = 0; hseg < 2; ++hseg) {
@@ -475,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   o8[2 * q] = e4m3x2_scaled_bf16x2(w4[q] & 0xffffu, sc);
                   o8[2 * q + 1] = e4m3x2_scaled_bf16x2(w4[q] >> 16, sc);
                 }
-                uint8_t* at = base + kOffKV + (lane >> 2) * (kRows * 128);
+                uint8_t* at = kv_ptr + (lane >> 2) * (kRows * 128);
                 const int c8 = 2 * (lane & 3);
                 *reinterpret_cast<uint4*>(at + sw128(rr, c8)) = make_uint4(o8[0], o8[1], o8[2], o8[3]);
                 *reinterpret_cast<uint4*>(at + sw128(rr, c8 + 1)) =
@@ -497,7 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
 #pragma unroll 4
           for (int rr = warp; rr < kRows; rr += 4) {
-            const __nv_bfloat16* src = S.src[rr];
+            const __nv_bfloat16* src = S.src[slot][rr];
 #pragma unroll
             for (int hseg = 0; hseg < 2; ++hseg) {
               const int gch = lane + 32 * hseg;  // 16-byte chunk of the 1 KB row
@@ -508,36 +532,80 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
+        return false;
+      }
+    };
+    auto gather_finish = [&](int slot, bool tma) {
+      if (!tma) {
         cp_async_wait_all();
         fence_proxy_async_smem();
-        if (tid == 0) mbar_arrive(&S.kv_full);  // stands in for the TMA issue
+        if (tid == 0) mbar_arrive(&S.kv_full[slot]);  // stands in for the TMA issue
       }
-      mbar_arrive(&S.kv_full);
+      mbar_arrive(&S.kv_full[slot]);
+    };
+    int pend = -1;  // slot of a gather issued and not yet finished
+    bool pend_tma = false;
+    if (c0 < c1) {
+      pend_tma = gather_issue(c0, 0);
+      pend = 0;
+    }
+#pragma unroll 1
+    for (int j = c0; j < c1 && ok; ++j) {
+      const uint32_t it = (uint32_t)(j - c0);
+      const int slot = (int)(it % kBuf);
+      const uint32_t ph = (it / kBuf) & 1;
+      if constexpr (kBuf == 1) {
+        if (j > c0) {  // the previous chunk's O^T products are done: the buffer is free
+          ok = all_ok_softmax(mbar_wait(&S.kv_free[0], (it - 1) & 1, kErrKvFree));
+          if (!ok) break;
+          pend_tma = gather_issue(j, 0);
+          pend = 0;
+        }
+        gather_finish(0, pend_tma);
+        pend = -1;
+      } else {
+        if (j == c0) {
+          gather_finish(0, pend_tma);
+          pend = -1;
+        } else {  // O(j-1) done: its buffer may take chunk j+1, and O^T may be rescaled
+          ok = all_ok_softmax(mbar_wait(&S.kv_free[(it + 1) & 1], ((it - 1) >> 1) & 1, kErrKvFree));
+          if (!ok) break;
+        }
+        if (j + 1 < c1) {
+          pend_tma = gather_issue(j + 1, (int)((it + 1) & 1));
+          pend = (int)((it + 1) & 1);
+        }
+      }
 
       // ---- softmax: lanes 0-15 of warp w own heads 16w .. 16w+15 (the M = 64 accumulator
       //      puts row 16w + i in TMEM lane 32w + i); a thread holds its head's 128 row values ----
-      ok = all_ok_softmax(mbar_wait(&S.s_full, it & 1, kErrSFull));
+      ok = all_ok_softmax(mbar_wait(&S.s_full[slot], ph, kErrSFull));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sa[64], sb[64];
-      tmem_ld_32x32b_x64(lane_base + kColS, sa);
-      tmem_ld_32x32b_x64(lane_base + kColS + 64, sb);
+      constexpr int kHalves = kRows / 64;  // 64-row halves of a chunk
+      uint32_t sv[kHalves][64];
+#pragma unroll
+      for (int hv = 0; hv < kHalves; ++hv)
+        tmem_ld_32x32b_x64(lane_base + kColS + (kBuf == 2 ? 64 * slot : 0) + 64 * hv, sv[hv]);
       tmem_ld_wait();
-      const uint32_t vm0 = S.vmask[0], vm1 = S.vmask[1], vm2 = S.vmask[2], vm3 = S.vmask[3];
+      uint32_t vm[kRows / 32];
+#pragma unroll
+      for (int i = 0; i < kRows / 32; ++i) vm[i] = S.vmask[slot][i];
       // scaled logits in place (masked rows -> -inf); eight partial maxima keep the
       // dependency chains short (max is exact in any order)
       float cmx[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) cmx[i] = -INFINITY;
 #pragma unroll
-      for (int r = 0; r < 64; ++r) {
-        const uint32_t w0 = r < 32 ? vm0 : vm1, w1 = r < 32 ? vm2 : vm3;
-        const float x0 = ((w0 >> (r & 31)) & 1u) ? __uint_as_float(sa[r]) * a.scale : -INFINITY;
-        const float x1 = ((w1 >> (r & 31)) & 1u) ? __uint_as_float(sb[r]) * a.scale : -INFINITY;
-        sa[r] = __float_as_uint(x0);
-        sb[r] = __float_as_uint(x1);
-        cmx[r & 3] = fmaxf(cmx[r & 3], x0);
-        cmx[4 + (r & 3)] = fmaxf(cmx[4 + (r & 3)], x1);
+      for (int hv = 0; hv < kHalves; ++hv) {
+#pragma unroll
+        for (int r = 0; r < 64; ++r) {
+          const uint32_t w = vm[2 * hv + (r >> 5)];
+          const float x =
+              ((w >> (r & 31)) & 1u) ? __uint_as_float(sv[hv][r]) * a.scale : -INFINITY;
+          sv[hv][r] = __float_as_uint(x);
+          cmx[4 * hv + (r & 3)] = fmaxf(cmx[4 * hv + (r & 3)], x);
+        }
       }
       const float cm = fmaxf(fmaxf(fmaxf(cmx[0], cmx[1]), fmaxf(cmx[2], cmx[3])),
                              fmaxf(fmaxf(cmx[4], cmx[5]), fmaxf(cmx[6], cmx[7])));
@@ -566,17 +634,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // P row of this head (bf16) into the K-major B tile: [row / 64][head][128 B]
       if (head_thr) {
-        uint8_t* pt = base + kOffP;
+        uint8_t* pt = base + kOffP + slot * L::kSlotP;
         float lc[4] = {0.f, 0.f, 0.f, 0.f};  // partial sums (sum what the MMA multiplies)
         const float mref = mu_h == -INFINITY ? 0.f : mu_h;  // no valid row yet: every p is 0
 #pragma unroll
-        for (int c8 = 0; c8 < 16; ++c8) {  // rows 8*c8 .. 8*c8+7
+        for (int c8 = 0; c8 < kRows / 8; ++c8) {  // rows 8*c8 .. 8*c8+7
           uint32_t pk[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const int r = 8 * c8 + 2 * k;
-            const float s0 = __uint_as_float(r < 64 ? sa[r & 63] : sb[r & 63]);
-            const float s1 = __uint_as_float(r < 64 ? sa[(r + 1) & 63] : sb[(r + 1) & 63]);
+            const float s0 = __uint_as_float(sv[r >> 6][r & 63]);
+            const float s1 = __uint_as_float(sv[(r + 1) >> 6][(r + 1) & 63]);
             const __nv_bfloat16 b0 = __float2bfloat16_rn(__expf(s0 - mref));  // -inf -> 0
             const __nv_bfloat16 b1 = __float2bfloat16_rn(__expf(s1 - mref));
             lc[k] += __bfloat162float(b0) + __bfloat162float(b1);
@@ -589,15 +657,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&S.p_full);
+      mbar_arrive(&S.p_full[slot]);
+      if constexpr (kBuf == 2) {
+        if (pend >= 0) {  // the next chunk's rows: in flight during this softmax, landed now
+          gather_finish(pend, pend_tma);
+          pend = -1;
+        }
+      }
     }
+    if (pend >= 0) cp_async_wait_all();  // a wait gave up: no copy of this thread in flight
     if (head_thr) {
       S.m_used[hh] = mu_h;
       S.l_sum[hh] = l_h;
     }
     // ---- epilogue: wait for the last O^T, then finalise or write the partial ----
-    if (ok && c1 > c0)
-      ok = all_ok_softmax(mbar_wait(&S.kv_free, (uint32_t)(c1 - c0 - 1) & 1, kErrKvFree));
+    if (ok && c1 > c0) {
+      const uint32_t last = (uint32_t)(c1 - c0 - 1);
+      ok = all_ok_softmax(mbar_wait(&S.kv_free[last % kBuf], (last / kBuf) & 1, kErrKvFree));
+    }
     bar_softmax();
     const bool single = P.nsplit == 1;
     if (tid < kHg) {
@@ -657,14 +734,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------ MMA issuer (warp 4) ------------------------------
-    const uint32_t idS = idesc_f16(1, kHg, kRows);                 // M = 64, N = 128, K-major
-    const uint32_t idO = idesc_f16(1, kRows, kHg) | (1u << 15);    // A MN-major, B K-major
-    const uint32_t kv = smem_u32(base + kOffKV), qs = smem_u32(base + kOffQ),
-                   pt = smem_u32(base + kOffP);
+    const uint32_t idS = idesc_f16(1, kHg, kRows);              // M = 64, N = kRows, K-major
+    const uint32_t idO = idesc_f16(1, 128, kHg) | (1u << 15);   // M = 128 dims; A MN-major
+    const uint32_t qs = smem_u32(base + kOffQ);
     bool ok = true;
     for (int j = c0; j < c1 && ok; ++j) {
       const uint32_t it = (uint32_t)(j - c0);
-      ok = __all_sync(0xffffffffu, mbar_wait(&S.kv_full, it & 1, kErrKvFull));
+      const int slot = (int)(it % kBuf);
+      const uint32_t ph = (it / kBuf) & 1;
+      const uint32_t kv = smem_u32(base + kOffKV + slot * L::kSlotKV);
+      const uint32_t pt = smem_u32(base + kOffP + slot * L::kSlotP);
+      const uint32_t scol = kColS + (kBuf == 2 ? 64u * slot : 0u);
+      ok = __all_sync(0xffffffffu, mbar_wait(&S.kv_full[slot], ph, kErrKvFull));
       if (!ok) break;
       tc_fence_after();
       if (lane == 0) {
@@ -673,19 +754,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t atom = kk >> 2, koff = (kk & 3) * 32;
           const uint64_t ad = smem_desc(qs + atom * (kHg * 128) + koff, 16, 1024, kLayoutSw128);
           const uint64_t bd = smem_desc(kv + atom * (kRows * 128) + koff, 16, 1024, kLayoutSw128);
-          mma_f16(tmem + kColS, ad, bd, idS, kk > 0 ? 1u : 0u);
+          mma_f16(tmem + scol, ad, bd, idS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&S.s_full);
+        mma_commit(&S.s_full[slot]);
       }
       __syncwarp();
-      ok = __all_sync(0xffffffffu, mbar_wait(&S.p_full, it & 1, kErrPFull));
+      ok = __all_sync(0xffffffffu, mbar_wait(&S.p_full[slot], ph, kErrPFull));
       if (!ok) break;
       tc_fence_after();
       if (lane == 0) {
 #pragma unroll 1
         for (int sl = 0; sl < 4; ++sl) {
 #pragma unroll 1
-          for (int kk = 0; kk < kRows / 16; ++kk) {  // K = 128 rows in steps of 16
+          for (int kk = 0; kk < kRows / 16; ++kk) {  // K = kRows rows in steps of 16
             const uint64_t ad = smem_desc(kv + sl * 2 * (kRows * 128) + kk * 2048, kRows * 128,
                                           1024, kLayoutSw128);
             const uint64_t bd = smem_desc(pt + (kk >> 2) * (kHg * 128) + (kk & 3) * 32, 16, 1024,
@@ -693,7 +774,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_f16(tmem + kColO + 64 * sl, ad, bd, idO, (j > c0 || kk > 0) ? 1u : 0u);
           }
         }
-        mma_commit(&S.kv_free);
+        mma_commit(&S.kv_free[slot]);
       }
       __syncwarp();
     }
@@ -781,28 +862,41 @@ __global__ void __launch_bounds__(256) k_mqa_combine(MqaTcParams P) {
   *reinterpret_cast<__nv_bfloat162*>(out) = __floats2bfloat162_rn(y0, y1);
 }
 
-// bf16 rows of c = 512 values; box = one 128B swizzle atom (64 values) x 128 rows
-bool make_map_rows(CUtensorMap* m, const void* ptr, int64_t rows) {
+// bf16 rows of c = 512 values; box = one 128B swizzle atom (64 values) x box_rows rows
+bool make_map_rows(CUtensorMap* m, const void* ptr, int64_t rows, int box_rows) {
   auto fn = tensor_map_encoder();
-  if (!fn || ptr == nullptr || rows < kRows || rows >= (1ll << 31)) return false;
+  if (!fn || ptr == nullptr || rows < box_rows || rows >= (1ll << 31)) return false;
   cuuint64_t dims[2] = {(cuuint64_t)kC, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)kC * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)kRows};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t es[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// CTAs per stream: as many as fill the SMs, at most one per 128 rows of the longest list.
 int choose_nsplit(const MqaArgs& a) {
   const int64_t streams = (int64_t)a.B * a.T * (a.H / kHg);
   const int64_t rows_max = (a.k > 0 ? a.k : a.n_cap) + a.n_win;
-  const int64_t chunks_max = (rows_max + kRows - 1) / kRows;
+  const int64_t chunks_max = (rows_max + 127) / 128;
   int64_t ns = device_sm_count() / (streams > 0 ? streams : 1);
   if (ns < 1) ns = 1;
   if (ns > chunks_max) ns = chunks_max > 0 ? chunks_max : 1;
   if (ns > 32) ns = 32;
   return (int)ns;
+}
+
+// Rows per chunk: 64, with two buffers, when a stream's list is split over several CTAs
+// and each still walks two or more chunks of 128 (dense HCA lists: the next chunk's TMA boxes
+// land during this one's softmax); otherwise 128 with one buffer (sparse decode, where a CTA
+// takes one chunk, and prefill, where one CTA walks a whole list and 64-row chunks measured
+// slightly slower).
+int choose_rows(const MqaArgs& a) {
+  const int64_t rows_max = (a.k > 0 ? a.k : a.n_cap) + a.n_win;
+  const int64_t chunks = (rows_max + 127) / 128;
+  const int ns = choose_nsplit(a);
+  return ns > 1 && (chunks + ns - 1) / ns >= 2 ? 64 : 128;
 }
 
 }  // namespace
@@ -834,15 +928,25 @@ cudaError_t launch_mqa_tc(const MqaArgs& a, void* ws, size_t ws_bytes, cudaStrea
   memset(&tm_win, 0, sizeof(tm_win));
   const bool mixed = a.kv_scale != nullptr;    // mixed-precision cache rows
   const bool paged = a.page_table != nullptr;  // cache rows through the page table
+  const int rows = choose_rows(a);
   // cache rows come by TMA only when they are contiguous bf16 rows
-  P.tma_kv = !mixed && !paged && make_map_rows(&tm_kv, a.kv, (int64_t)a.B * a.n_cap) ? 1 : 0;
+  P.tma_kv =
+      !mixed && !paged && make_map_rows(&tm_kv, a.kv, (int64_t)a.B * a.n_cap, rows) ? 1 : 0;
   // window rows by TMA only from a linear window buffer (a ring wraps)
-  P.tma_win = a.win_pos0 != nullptr && make_map_rows(&tm_win, a.win, (int64_t)a.B * a.l_raw) ? 1 : 0;
+  P.tma_win =
+      a.win_pos0 != nullptr && make_map_rows(&tm_win, a.win, (int64_t)a.B * a.l_raw, rows) ? 1 : 0;
   if (P.nsplit > 1 && ws_bytes < mqa_tc_workspace_bytes(a)) return cudaErrorInvalidValue;
   const int64_t streams = (int64_t)a.B * a.T * P.G;
-  auto kern = mixed ? (paged ? k_mqa_tc<true, true> : k_mqa_tc<true, false>)
-                    : (paged ? k_mqa_tc<false, true> : k_mqa_tc<false, false>);
-  const size_t smem = 1024 + kOffEnd + (mixed ? sizeof(SmemT<true>) : sizeof(SmemT<false>));
+  auto kern = rows == 64
+                  ? (mixed ? (paged ? k_mqa_tc<true, true, 64> : k_mqa_tc<true, false, 64>)
+                           : (paged ? k_mqa_tc<false, true, 64> : k_mqa_tc<false, false, 64>))
+                  : (mixed ? (paged ? k_mqa_tc<true, true, 128> : k_mqa_tc<true, false, 128>)
+                           : (paged ? k_mqa_tc<false, true, 128> : k_mqa_tc<false, false, 128>));
+  const size_t smem =
+      1024 + (rows == 64 ? Lay<64>::kOffEnd +
+                               (mixed ? sizeof(SmemT<true, 64>) : sizeof(SmemT<false, 64>))
+                         : Lay<128>::kOffEnd +
+                               (mixed ? sizeof(SmemT<true, 128>) : sizeof(SmemT<false, 128>)));
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;

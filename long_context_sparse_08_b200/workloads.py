@@ -232,6 +232,11 @@ _reg(Shape("mid_prefill_bf16", "csa_prefill", "bf16", "bf16", B=1, T=384, m=4, c
 _reg(Shape("mid_hca_decode", "hca_decode", "bf16", "none", B=3, T=1, m=128, c=512, rope_dims=64,
            n_heads=64, n_idx_heads=0, d_idx=0, topk=0, n_win=128, n_cap=600, ctx=76900, seed=15,
            overlap=0))
+# Few streams over a long dense list: each stream is split over many CTAs that each walk
+# two or more chunks (the double-buffered 64-row form), with a ragged tail.
+_reg(Shape("long_hca_decode", "hca_decode", "bf16", "none", B=2, T=1, m=128, c=512,
+           rope_dims=64, n_heads=64, n_idx_heads=0, d_idx=0, topk=0, n_win=128, n_cap=4104,
+           ctx=525389, seed=41, overlap=0))
 # Degenerate decode cases: no visible entry (t < m), fewer visible entries than k,
 # exactly k, and a cache shorter than floor(t/m). Also an MXFP4 one for the tensor-core
 # indexer's edges (single partial tile, zero tiles, a request spanning many tiles).

@@ -323,7 +323,8 @@ def test_forward_parity_flash_prefill_8k_sampled():
     _forward_parity("flash_prefill_8k", [(0, t) for t in qs])
 
 
-@pytest.mark.parametrize("name", ["mid_hca_decode", "edge_hca_decode", "hca_decode_1m"])
+@pytest.mark.parametrize("name", ["mid_hca_decode", "edge_hca_decode", "long_hca_decode",
+                                  "hca_decode_1m"])
 def test_hca_dense_parity(name):
     s, inp, dev, st = _step(name, want_scores=False)
     res = P.run(s, inp)

@@ -61,7 +61,7 @@ def test_sparse_mqa_over_mixed_rows(name):
         U.check_out(got[b, ti], ref, "bf16", f"{name} mixed KV b={b} t={ti}")
 
 
-@pytest.mark.parametrize("name", ["mid_hca_decode", "edge_hca_decode"])
+@pytest.mark.parametrize("name", ["mid_hca_decode", "edge_hca_decode", "long_hca_decode"])
 def test_dense_mqa_over_mixed_rows(name):
     s, inp, inp2, rows, scale = _mixed(name)
     res = P.run(s, inp2)
@@ -139,9 +139,10 @@ def test_sparse_mqa_over_paged_cache(name, mixed, page_rows):
         U.check_out(got[b, ti], ref, "bf16", f"{name} paged b={b} t={ti}")
 
 
-@pytest.mark.parametrize("page_rows", [1, 8])
-def test_dense_mqa_over_paged_cache(page_rows):
-    s, inp = U.inputs("mid_hca_decode")
+@pytest.mark.parametrize("name,page_rows", [("mid_hca_decode", 1), ("mid_hca_decode", 8),
+                                            ("long_hca_decode", 8)])
+def test_dense_mqa_over_paged_cache(name, page_rows):
+    s, inp = U.inputs(name)
     res = P.run(s, inp)
     dev = R.upload(inp, s)
     pool, table = _paged(inp["kv_cache"], page_rows, 4)
@@ -158,7 +159,7 @@ def test_dense_mqa_over_paged_cache(page_rows):
     assert csa.device_error() == 0
     got = out.float().cpu().numpy()
     for (b, ti), ref in res["out"].items():
-        U.check_out(got[b, ti], ref, "bf16", f"mid_hca_decode paged({page_rows}) b={b}")
+        U.check_out(got[b, ti], ref, "bf16", f"{name} paged({page_rows}) b={b}")
 
 
 def test_paged_cache_with_a_bad_page_id_reports_it():
