@@ -7,8 +7,9 @@
 // softmax denominator.
 //
 // Work: a stream is (query, group of 64 heads); its KV row list (selected or visible
-// entries, then the window) is cut into chunks of 128 rows, and the chunks of a stream are
-// split over `nsplit` CTAs. Per chunk, with bf16 operands in 128B-swizzled shared memory
+// entries, then the window) is cut into chunks of 128 rows (one buffer) or, when a CTA walks
+// several, 64 rows (two buffers: the next chunk's rows arrive during this one's softmax),
+// and the chunks of a stream are split over `nsplit` CTAs. Per chunk, with bf16 operands in 128B-swizzled shared memory
 // and fp32 accumulators in TMEM:
 //   S[64 heads x 128 rows] = q_hat . K_chunk^T          (A = q_hat, M = 64; B = KV tile)
 //   P = exp(S * scale - m_h) in bf16                    (softmax: thread = head, its 128
@@ -306,6 +307,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int c0 = (int)(((int64_t)nchunks * split) / P.nsplit);
   const int c1 = (int)(((int64_t)nchunks * (split + 1)) / P.nsplit);
   const int r = a.rope_dims, r0 = kC - r;
+  // Without a programmatic launch every input is complete when the kernel starts, so with
+  // two KV buffers the first chunk's rows are requested before q_hat is built (the raw
+  // query rows are staged in the second buffer).
+  const bool early = kBuf == 2 && !a.chained && c0 < c1;
+  uint8_t* const q_stage = base + kOffKV + (kBuf == 2 ? L::kSlotKV : 0);
 
   if (warp == 4) {
     if (lane == 0) {
@@ -331,9 +337,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         cp_async16(qt + (d0 >> 6) * (kHg * 128) + sw128(h, (d0 & 63) >> 3), qg + i, true);
       }
     } else {
-      // the group's 64 raw query rows (64 KB, contiguous) into the KV tile area, which the
-      // first gather only overwrites after q_hat is built; one pass, one latency
-      const uint32_t stage = smem_u32(base + kOffKV);
+      // the group's 64 raw query rows (64 KB, contiguous) into a KV buffer that no gather
+      // overwrites before q_hat is built; one pass, one latency
+      const uint32_t stage = smem_u32(q_stage);
       const uint4* qg = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) +
                                                        ((size_t)bt * a.H + h0) * kC);
 #pragma unroll 4
@@ -351,76 +357,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = S.tmem_slot;
 
   if (warp < 4) {
-    if (a.qhat != nullptr) {
-      cp_async_wait_all();
-      fence_proxy_async_smem();  // the tile is read by the tensor cores
-    } else {
-      // ---- q_hat = RoPE_t(RMSNorm(q)) in bf16: two threads per head, 256 dims each. Thread
-      //      t reads its 32 chunks of 8 dims starting at chunk t % 32, so that a warp's reads
-      //      of one step spread over all banks. ----
-      uint8_t* qs = base + kOffQ;
-      const int qh = tid >> 1, qhalf = tid & 1;
-      const uint4* qrow = reinterpret_cast<const uint4*>(base + kOffKV + qh * (kC * 2)) + 32 * qhalf;
-      cp_async_wait_all();
-      bar_softmax();
-      float ss0 = 0.f, ss1 = 0.f;
-#pragma unroll 8
-      for (int i = 0; i < 32; ++i) {
-        const uint4 raw = qrow[(i + lane) & 31];
-        const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float lo = __uint_as_float(w4[k] << 16), hi = __uint_as_float(w4[k] & 0xffff0000u);
-          ss0 = fmaf(lo, lo, ss0);
-          ss1 = fmaf(hi, hi, ss1);
-        }
-      }
-      float ss = ss0 + ss1;
-      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-      const float rstd = rsqrtf(ss / (float)kC + a.eps);
-#pragma unroll 4
-      for (int i = 0; i < 32; ++i) {
-        const int c = (i + lane) & 31;
-        const uint4 raw = qrow[c];
-        const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-        const int d0 = 256 * qhalf + 8 * c;
-        float y[8];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          y[2 * k] = __uint_as_float(w4[k] << 16) * rstd * S.wq[d0 + 2 * k];
-          y[2 * k + 1] = __uint_as_float(w4[k] & 0xffff0000u) * rstd * S.wq[d0 + 2 * k + 1];
-        }
-        if (d0 >= r0) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int p = (d0 + 2 * k - r0) >> 1;
-            const float cs = S.cs[p], sn = S.sn[p], u = y[2 * k], v = y[2 * k + 1];
-            y[2 * k] = u * cs - v * sn;
-            y[2 * k + 1] = u * sn + v * cs;
-          }
-        }
-        uint4 o;
-        uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          ow[k] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * k])) |
-                  ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * k + 1])) << 16);
-        const int atom = d0 >> 6, chunk = (d0 & 63) >> 3;
-        *reinterpret_cast<uint4*>(qs + atom * (kHg * 128) + sw128(qh, chunk)) = o;
-      }
-      // the tile is read by the tensor cores, also when a chunk's rows come by TMA (whose
-      // arrival carries no fence of these stores)
-      fence_proxy_async_smem();
-    }
-
-    // the selected rows, the partials and the output belong to the previous kernels
-    pdl_wait();
-    pdl_trigger();
-    bool ok = true;
-    const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
-    const bool head_thr = lane < 16;  // lanes 0-15: the softmax of head hh
-    const int hh = 16 * warp + (lane & 15);
-    float mu_h = -INFINITY, l_h = 0.f;  // running max used and running sum of this head
     // A chunk's rows are gathered in two steps: the issue (rows resolved, copies or TMA boxes
     // started; returns whether TMA fills the slot) and the finish (cp.async copies: wait for
     // this thread's, make them visible to the tensor cores; then arrive). With two buffers the
@@ -545,7 +481,83 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     int pend = -1;  // slot of a gather issued and not yet finished
     bool pend_tma = false;
-    if (c0 < c1) {
+    if constexpr (kBuf == 2) {
+      if (early) {
+        pend_tma = gather_issue(c0, 0);
+        pend = 0;
+      }
+    }
+    if (a.qhat != nullptr) {
+      cp_async_wait_all();
+      fence_proxy_async_smem();  // the tile is read by the tensor cores
+    } else {
+      // ---- q_hat = RoPE_t(RMSNorm(q)) in bf16: two threads per head, 256 dims each. Thread
+      //      t reads its 32 chunks of 8 dims starting at chunk t % 32, so that a warp's reads
+      //      of one step spread over all banks. ----
+      uint8_t* qs = base + kOffQ;
+      const int qh = tid >> 1, qhalf = tid & 1;
+      const uint4* qrow = reinterpret_cast<const uint4*>(q_stage + qh * (kC * 2)) + 32 * qhalf;
+      cp_async_wait_all();
+      bar_softmax();
+      float ss0 = 0.f, ss1 = 0.f;
+#pragma unroll 8
+      for (int i = 0; i < 32; ++i) {
+        const uint4 raw = qrow[(i + lane) & 31];
+        const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float lo = __uint_as_float(w4[k] << 16), hi = __uint_as_float(w4[k] & 0xffff0000u);
+          ss0 = fmaf(lo, lo, ss0);
+          ss1 = fmaf(hi, hi, ss1);
+        }
+      }
+      float ss = ss0 + ss1;
+      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+      const float rstd = rsqrtf(ss / (float)kC + a.eps);
+#pragma unroll 4
+      for (int i = 0; i < 32; ++i) {
+        const int c = (i + lane) & 31;
+        const uint4 raw = qrow[c];
+        const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+        const int d0 = 256 * qhalf + 8 * c;
+        float y[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          y[2 * k] = __uint_as_float(w4[k] << 16) * rstd * S.wq[d0 + 2 * k];
+          y[2 * k + 1] = __uint_as_float(w4[k] & 0xffff0000u) * rstd * S.wq[d0 + 2 * k + 1];
+        }
+        if (d0 >= r0) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int p = (d0 + 2 * k - r0) >> 1;
+            const float cs = S.cs[p], sn = S.sn[p], u = y[2 * k], v = y[2 * k + 1];
+            y[2 * k] = u * cs - v * sn;
+            y[2 * k + 1] = u * sn + v * cs;
+          }
+        }
+        uint4 o;
+        uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          ow[k] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * k])) |
+                  ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y[2 * k + 1])) << 16);
+        const int atom = d0 >> 6, chunk = (d0 & 63) >> 3;
+        *reinterpret_cast<uint4*>(qs + atom * (kHg * 128) + sw128(qh, chunk)) = o;
+      }
+      // the tile is read by the tensor cores, also when a chunk's rows come by TMA (whose
+      // arrival carries no fence of these stores)
+      fence_proxy_async_smem();
+    }
+
+    // the selected rows, the partials and the output belong to the previous kernels
+    pdl_wait();
+    pdl_trigger();
+    bool ok = true;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+    const bool head_thr = lane < 16;  // lanes 0-15: the softmax of head hh
+    const int hh = 16 * warp + (lane & 15);
+    float mu_h = -INFINITY, l_h = 0.f;  // running max used and running sum of this head
+    if (c0 < c1 && pend < 0) {
       pend_tma = gather_issue(c0, 0);
       pend = 0;
     }
@@ -736,25 +748,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------ MMA issuer (warp 4) ------------------------------
     const uint32_t idS = idesc_f16(1, kHg, kRows);              // M = 64, N = kRows, K-major
     const uint32_t idO = idesc_f16(1, 128, kHg) | (1u << 15);   // M = 128 dims; A MN-major
-    const uint32_t qs = smem_u32(base + kOffQ);
+    // Descriptors are formed once; a step adds its operand's byte offset / 16 to the start
+    // address field (every operand lies below 256 KB, so the 14-bit field never carries), and
+    // the loops are unrolled, so issuing an MMA costs a few instructions.
+    const uint64_t dq = smem_desc(smem_u32(base + kOffQ), 16, 1024, kLayoutSw128);
     bool ok = true;
     for (int j = c0; j < c1 && ok; ++j) {
       const uint32_t it = (uint32_t)(j - c0);
       const int slot = (int)(it % kBuf);
       const uint32_t ph = (it / kBuf) & 1;
       const uint32_t kv = smem_u32(base + kOffKV + slot * L::kSlotKV);
-      const uint32_t pt = smem_u32(base + kOffP + slot * L::kSlotP);
-      const uint32_t scol = kColS + (kBuf == 2 ? 64u * slot : 0u);
+      const uint64_t dk = smem_desc(kv, 16, 1024, kLayoutSw128);           // K-major rows
+      const uint64_t dv = smem_desc(kv, kRows * 128, 1024, kLayoutSw128);  // the same, MN-major
+      const uint64_t dp = smem_desc(smem_u32(base + kOffP + slot * L::kSlotP), 16, 1024,
+                                    kLayoutSw128);
+      const uint32_t scol = tmem + kColS + (kBuf == 2 ? 64u * slot : 0u);
       ok = __all_sync(0xffffffffu, mbar_wait(&S.kv_full[slot], ph, kErrKvFull));
       if (!ok) break;
       tc_fence_after();
       if (lane == 0) {
-#pragma unroll 1
-        for (int kk = 0; kk < 32; ++kk) {  // K = 512 in steps of 16
-          const uint32_t atom = kk >> 2, koff = (kk & 3) * 32;
-          const uint64_t ad = smem_desc(qs + atom * (kHg * 128) + koff, 16, 1024, kLayoutSw128);
-          const uint64_t bd = smem_desc(kv + atom * (kRows * 128) + koff, 16, 1024, kLayoutSw128);
-          mma_f16(tmem + scol, ad, bd, idS, kk > 0 ? 1u : 0u);
+        // K = 512 in steps of 16: four steps per 64-dim atom. The atom loop is unrolled
+        // for 64-row chunks (a CTA walks many, so the code is warm) and kept rolled for
+        // 128-row chunks (typically one per CTA, where fetching a longer body costs more).
+#pragma unroll(kRows == 64 ? 8 : 1)
+        for (int atom = 0; atom < 8; ++atom) {
+#pragma unroll
+          for (int kq = 0; kq < 4; ++kq)
+            mma_f16(scol, dq + ((atom * (kHg * 128) + kq * 32) >> 4),
+                    dk + ((atom * (kRows * 128) + kq * 32) >> 4), idS,
+                    (atom | kq) != 0 ? 1u : 0u);
         }
         mma_commit(&S.s_full[slot]);
       }
@@ -763,16 +785,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       if (lane == 0) {
-#pragma unroll 1
-        for (int sl = 0; sl < 4; ++sl) {
-#pragma unroll 1
-          for (int kk = 0; kk < kRows / 16; ++kk) {  // K = kRows rows in steps of 16
-            const uint64_t ad = smem_desc(kv + sl * 2 * (kRows * 128) + kk * 2048, kRows * 128,
-                                          1024, kLayoutSw128);
-            const uint64_t bd = smem_desc(pt + (kk >> 2) * (kHg * 128) + (kk & 3) * 32, 16, 1024,
-                                          kLayoutSw128);
-            mma_f16(tmem + kColO + 64 * sl, ad, bd, idO, (j > c0 || kk > 0) ? 1u : 0u);
-          }
+        // K = kRows rows in steps of 16; the four O^T slices are independent accumulators,
+        // issued in turn
+#pragma unroll(kRows == 64 ? 4 : 1)
+        for (int kk = 0; kk < kRows / 16; ++kk) {
+#pragma unroll
+          for (int sl = 0; sl < 4; ++sl)
+            mma_f16(tmem + kColO + 64 * sl, dv + ((sl * 2 * (kRows * 128) + kk * 2048) >> 4),
+                    dp + (((kk >> 2) * (kHg * 128) + (kk & 3) * 32) >> 4), idO,
+                    (j > c0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&S.kv_free[slot]);
       }
@@ -887,16 +908,14 @@ int choose_nsplit(const MqaArgs& a) {
   return (int)ns;
 }
 
-// Rows per chunk: 64, with two buffers, when a stream's list is split over several CTAs
-// and each still walks two or more chunks of 128 (dense HCA lists: the next chunk's TMA boxes
-// land during this one's softmax); otherwise 128 with one buffer (sparse decode, where a CTA
-// takes one chunk, and prefill, where one CTA walks a whole list and 64-row chunks measured
-// slightly slower).
+// Rows per chunk: 64, with two buffers, when a CTA walks two or more chunks of 128 (dense
+// HCA lists, prefill: the next chunk's rows land during this one's softmax); 128 with one
+// buffer when it takes a single chunk (sparse decode).
 int choose_rows(const MqaArgs& a) {
   const int64_t rows_max = (a.k > 0 ? a.k : a.n_cap) + a.n_win;
   const int64_t chunks = (rows_max + 127) / 128;
   const int ns = choose_nsplit(a);
-  return ns > 1 && (chunks + ns - 1) / ns >= 2 ? 64 : 128;
+  return (chunks + ns - 1) / ns >= 2 ? 64 : 128;
 }
 
 }  // namespace
