@@ -9,10 +9,10 @@
 // Work: a stream is (query, group of 64 heads); its KV row list (selected or visible
 // entries, then the window) is cut into chunks of 128 rows (one buffer) or, when a CTA walks
 // several, 64 rows (two buffers: the next chunk's rows arrive during this one's softmax),
-// and the chunks of a stream are split over `nsplit` CTAs. Per chunk, with bf16 operands in 128B-swizzled shared memory
-// and fp32 accumulators in TMEM:
-//   S[64 heads x 128 rows] = q_hat . K_chunk^T          (A = q_hat, M = 64; B = KV tile)
-//   P = exp(S * scale - m_h) in bf16                    (softmax: thread = head, its 128
+// and the chunks of a stream are split over `nsplit` CTAs. Per chunk of R rows, with bf16
+// operands in 128B-swizzled shared memory and fp32 accumulators in TMEM:
+//   S[64 heads x R rows] = q_hat . K_chunk^T            (A = q_hat, M = 64; B = KV tile)
+//   P = exp(S * scale - m_h) in bf16                    (softmax: thread = head, its R
 //                                                        row values in registers)
 //   O^T[4 x 128 dims x 64 heads] += V_chunk^T . P^T     (A = the same KV tile read MN-major,
 //                                                        B = P, K-major)

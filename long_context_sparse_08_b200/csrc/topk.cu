@@ -4,10 +4,16 @@
 // among the top-k of I[t,:]. The result here is ordered by (score desc, index asc) and
 // padded with -1 when fewer than k entries are visible; it depends only on the scores.
 //
-// One CTA of 1024 threads per query row: an MSB-first radix select on order-preserving
-// 32-bit keys (4 passes of 8 bits, histograms in shared memory) finds the k-th largest
-// key T. Every entry with key >= T is then appended (warp-aggregated, any order) and a
-// bitonic sort of the (key, index) pairs orders them; its first k are the result. Only
+// Rows of up to 16384 entries (prefill chunks): one CTA of 512 threads per query row loads
+// the row's order-preserving 32-bit keys into shared memory once; an MSB-first radix
+// select over them (digits of 12, 12 and 8 bits, histograms in shared memory, stopping as
+// soon as the k-th key's digit bin is taken whole) finds the threshold T and how many keys
+// equal to T are needed. The keys above T and those ties are appended (warp-aggregated,
+// any order; ties in index order when only some are taken), and a bitonic sort of the
+// (key, index) pairs orders them.
+//
+// Longer rows: one CTA of 1024 threads per row re-reads the scores from global memory for
+// each of 4 radix passes of 8 bits, then appends every entry with key >= T and sorts; only
 // when ties at T overflow the 2048 shared slots does a block-wide scan in index order
 // gather the keys > T and the first (lowest-index) keys == T instead.
 #include "common.cuh"
@@ -193,6 +199,195 @@ __global__ void __launch_bounds__(kThreads) k_topk_rows(TopkArgs a) {
   for (int i = threadIdx.x; i < k; i += blockDim.x) out[i] = (int32_t)(pairs[i] & 0xffffffffu);
 }
 
+
+// ---------------------------------------------------------------------------
+// rows of up to kRowKeys entries: keys resident in shared memory
+// ---------------------------------------------------------------------------
+constexpr int kRThreads = 512;
+constexpr int kRowKeys = 16384;
+
+// Exclusive scan of one int per thread over the block (512 threads); *total = sum.
+__device__ __forceinline__ int block_excl_scan_int(int v, int* wsum, int* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) wsum[wid] = incl;
+  __syncthreads();
+  int base = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < kRThreads / 32; ++w) {
+    const int x = wsum[w];
+    base += w < wid ? x : 0;
+    tot += x;
+  }
+  *total = tot;
+  __syncthreads();  // wsum may be reused
+  return base + incl - v;
+}
+
+// The bin of a descending walk over hist[0..nbins) in which the count reaches `need`
+// (1 <= need <= sum): *bin, and *above = the count in the bins above it.
+__device__ __forceinline__ void find_bin(const int* hist, int nbins, int need, int* wsum,
+                                         int* s_bin, int* s_above) {
+  const int tid = threadIdx.x;
+  const int per = nbins >= kRThreads ? nbins / kRThreads : 1;
+  const int first = nbins - 1 - tid * per;  // this thread's bins: first, first-1, ...
+  int v[8], sum = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    v[j] = (j < per && first - j >= 0) ? hist[first - j] : 0;
+    sum += v[j];
+  }
+  int total;
+  int above = block_excl_scan_int(sum, wsum, &total);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j < per && first - j >= 0 && above < need && above + v[j] >= need) {
+      *s_bin = first - j;
+      *s_above = above;
+    }
+    above += v[j];
+  }
+  __syncthreads();
+}
+
+template <typename TS>
+__global__ void __launch_bounds__(kRThreads, 2) k_topk_rows_smem(TopkArgs a, int vec) {
+  extern __shared__ __align__(16) uint32_t kq[];  // the row's keys
+  __shared__ __align__(16) uint64_t s_u[kMaxTopk];  // histogram (ints), then (key, index) pairs
+  __shared__ int wsum[kRThreads / 32];
+  __shared__ int s_bin, s_above, s_cnt;
+  int* hist = reinterpret_cast<int*>(s_u);
+  uint64_t* pairs = s_u;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int bt = blockIdx.x;
+  const int64_t t = a.q_pos[bt];
+  if (a.qj.qhat != nullptr) {  // side job: this row's query heads for the attention
+    __shared__ float s_cs[256], s_sn[256];
+    qhat_rows(a.qj, bt, (double)t, 0, a.qj.H, s_cs, s_sn);
+  }
+  const int n = (int)(t < 0 ? 0 : (t / a.m < a.n_cap ? t / a.m : a.n_cap));
+  const TS* sc = (sizeof(TS) == 4 ? static_cast<const TS*>(static_cast<const void*>(a.scores))
+                                  : static_cast<const TS*>(a.scores16)) + (size_t)bt * a.n_cap;
+  int32_t* out = a.out_idx + (size_t)bt * a.k;
+  const int k = a.k;
+  int P = 1;
+  while (P < k) P <<= 1;
+
+  // ---- keys into shared memory (groups of 4 by vector loads when rows are 16-byte aligned) ----
+  if (vec) {
+    const int ng = (n + 3) >> 2;
+#pragma unroll 8
+    for (int g = tid; g < ng; g += kRThreads) {
+      float f[4];
+      if constexpr (sizeof(TS) == 4) {
+        const float4 x = reinterpret_cast<const float4*>(sc)[g];
+        f[0] = x.x; f[1] = x.y; f[2] = x.z; f[3] = x.w;
+      } else {
+        const uint2 x = reinterpret_cast<const uint2*>(sc)[g];
+        f[0] = __uint_as_float(x.x << 16); f[1] = __uint_as_float(x.x & 0xffff0000u);
+        f[2] = __uint_as_float(x.y << 16); f[3] = __uint_as_float(x.y & 0xffff0000u);
+      }
+      reinterpret_cast<uint4*>(kq)[g] =
+          make_uint4(float_key(f[0]), float_key(f[1]), float_key(f[2]), float_key(f[3]));
+    }
+  } else {
+    for (int i = tid; i < n; i += kRThreads) kq[i] = float_key(ld_score(sc, i));
+  }
+  for (int i = tid; i < 4096; i += kRThreads) hist[i] = 0;
+  __syncthreads();
+
+  if (n <= k) {  // everything visible is selected; just order it
+    for (int i = tid; i < P; i += kRThreads) pairs[i] = i < n ? pack_desc(kq[i], (uint32_t)i) : ~0ull;
+    __syncthreads();
+    bitonic_sort(pairs, P);
+    for (int i = tid; i < k; i += kRThreads)
+      out[i] = i < n ? (int32_t)(pairs[i] & 0xffffffffu) : -1;
+    return;
+  }
+
+  // ---- radix select of the k-th largest key: digits [31:20], [19:8], [7:0] ----
+  int kk = k;          // still to take among keys matching the prefix
+  uint32_t T = 0;      // threshold: every key >= T is taken ...
+  bool ties = false;   // ... unless only kk of the keys == T are (then in index order)
+  {
+    for (int i = tid; i < n; i += kRThreads) atomicAdd(&hist[kq[i] >> 20], 1);
+    __syncthreads();
+    find_bin(hist, 4096, kk, wsum, &s_bin, &s_above);
+    const uint32_t b1 = (uint32_t)s_bin;
+    kk -= s_above;
+    const int in1 = hist[b1];
+    __syncthreads();
+    if (in1 == kk) {
+      T = b1 << 20;
+    } else {
+      for (int i = tid; i < 4096; i += kRThreads) hist[i] = 0;
+      __syncthreads();
+      for (int i = tid; i < n; i += kRThreads) {
+        const uint32_t u = kq[i];
+        if ((u >> 20) == b1) atomicAdd(&hist[(u >> 8) & 0xfffu], 1);
+      }
+      __syncthreads();
+      find_bin(hist, 4096, kk, wsum, &s_bin, &s_above);
+      const uint32_t b2 = (b1 << 12) | (uint32_t)s_bin;
+      kk -= s_above;
+      const int in2 = hist[s_bin];
+      __syncthreads();
+      if (in2 == kk) {
+        T = b2 << 8;
+      } else {
+        for (int i = tid; i < 256; i += kRThreads) hist[i] = 0;
+        __syncthreads();
+        for (int i = tid; i < n; i += kRThreads) {
+          const uint32_t u = kq[i];
+          if ((u >> 8) == b2) atomicAdd(&hist[u & 0xffu], 1);
+        }
+        __syncthreads();
+        find_bin(hist, 256, kk, wsum, &s_bin, &s_above);
+        T = (b2 << 8) | (uint32_t)s_bin;
+        kk -= s_above;
+        ties = hist[s_bin] > kk;
+        __syncthreads();
+      }
+    }
+  }
+
+  // ---- append: keys > T (or >= T when the whole tie group is taken), any order ----
+  if (tid == 0) s_cnt = 0;
+  __syncthreads();
+  for (int base = 0; base < n; base += kRThreads) {
+    const int i = base + tid;
+    const uint32_t u = i < n ? kq[i] : 0u;
+    const bool take = i < n && (ties ? u > T : u >= T);
+    const unsigned bal = __ballot_sync(0xffffffffu, take);
+    if (bal == 0) continue;
+    int pos = 0;
+    if (lane == __ffs(bal) - 1) pos = atomicAdd(&s_cnt, __popc(bal));
+    pos = __shfl_sync(0xffffffffu, pos, __ffs(bal) - 1) + __popc(bal & ((1u << lane) - 1u));
+    if (take) pairs[pos] = pack_desc(u, (uint32_t)i);
+  }
+  if (ties) {  // the first kk keys == T in index order
+    const int n_gt = k - kk;
+    int run = 0;
+    for (int base = 0; base < n && run < kk; base += kRThreads) {
+      const int i = base + tid;
+      const bool eq = i < n && kq[i] == T;
+      int tot;
+      const int off = block_excl_scan_int(eq ? 1 : 0, wsum, &tot);
+      if (eq && run + off < kk) pairs[n_gt + run + off] = pack_desc(T, (uint32_t)i);
+      run += tot;
+    }
+  }
+  for (int i = k + tid; i < P; i += kRThreads) pairs[i] = ~0ull;
+  __syncthreads();
+  bitonic_sort(pairs, P);
+  for (int i = tid; i < k; i += kRThreads) out[i] = (int32_t)(pairs[i] & 0xffffffffu);
+}
+
 }  // namespace
 
 size_t topk_workspace_bytes(int B, int T, int64_t n_cap, int k) {
@@ -207,7 +402,19 @@ cudaError_t launch_topk(const TopkArgs& a, void* ws, size_t ws_bytes, cudaStream
       return cudaErrorInvalidValue;
     return launch_topk_decode(topk_decode_args(a, ws), hist_ready, st);
   }
-  if (a.scores16 != nullptr)
+  const bool b16 = a.scores16 != nullptr;
+  if (a.n_cap <= kRowKeys) {
+    // vector loads need every row start 16-byte (fp32) or 8-byte (bf16) aligned
+    const uintptr_t p = b16 ? (uintptr_t)a.scores16 : (uintptr_t)a.scores;
+    const int vec = (a.n_cap % 4 == 0 && p % 16 == 0) ? 1 : 0;
+    const size_t smem = (size_t)((a.n_cap + 3) / 4 * 4) * 4;
+    auto kern = b16 ? k_topk_rows_smem<__nv_bfloat16> : k_topk_rows_smem<float>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(kRowKeys * 4));
+    if (e != cudaSuccess) return e;
+    return launch(false, kern, dim3(a.B * a.T), dim3(kRThreads), smem, st, a, vec);
+  }
+  if (b16)
     return launch(false, k_topk_rows<__nv_bfloat16>, dim3(a.B * a.T), dim3(kThreads), 0, st, a);
   return launch(false, k_topk_rows<float>, dim3(a.B * a.T), dim3(kThreads), 0, st, a);
 }

@@ -131,15 +131,16 @@ def test_bf16_indexer_launch_batches_with_a_short_tail():
 # stage 3: top-k, exact on given fp32 scores
 # ---------------------------------------------------------------------------
 
+@pytest.mark.parametrize("N", [6000, 6001])  # rows of a multiple of 4 (vector loads) or not
 @pytest.mark.parametrize("k", [7, 512, 1000, 2048])
-def test_topk_exact_on_given_scores(k):
+def test_topk_exact_on_given_scores(k, N):
     g = np.random.default_rng(100 + k)
-    B, T, N = 2, 3, 6000
+    B, T = 2, 3
     sc = np.round(g.standard_normal((B, T, N)).astype(np.float32), 2)  # many exact ties
     sc[0, 1, :50] = -0.0
     sc[0, 1, 50:90] = 0.0
     sc[1, 2] = 1.5  # every score equal
-    pos = np.array([[0, 4 * 80, 4 * N + 3], [4 * 2000 + 1, 4 * 5999, 4 * N]], np.int64)
+    pos = np.array([[0, 4 * 80, 4 * N + 3], [4 * 2000 + 1, 4 * 5999 + 3, 4 * N]], np.int64)
     p = csa.make_params(topk=k)
     ws_bytes = csa.workspace_size(p, csa.CSA_WS_TOPK, 0, B, T, N)
     ws = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device="cuda")
@@ -152,6 +153,32 @@ def test_topk_exact_on_given_scores(k):
             nv = O.visible_entries(int(pos[b, t]), 4, N)
             ref = O.topk_select(sc[b, t, :nv].astype(np.float64), k)
             np.testing.assert_array_equal(got[b, t], ref, err_msg=f"b={b} t={t} k={k}")
+
+
+@pytest.mark.parametrize("N,k", [(16384, 512), (16384, 2048), (20000, 512)])
+def test_topk_exact_on_many_rows(N, k):
+    # more rows than the decode path takes: one CTA per row, with the row's keys in shared
+    # memory up to 16384 entries, re-read from global memory beyond
+    g = np.random.default_rng(300 + N + k)
+    B, T = 1, 72
+    sc = g.standard_normal((B, T, N)).astype(np.float32)
+    sc[0, :8] = np.round(sc[0, :8] * 4, 1)  # heavy ties
+    sc[0, 8] = 0.75  # every score equal
+    sc[0, 9, ::5] = -1e30
+    pos = (4 * np.linspace(0, N + 40, T)).astype(np.int64).reshape(B, T)
+    pos[0, :10] = 4 * N + 1
+    p = csa.make_params(topk=k)
+    ws_bytes = csa.workspace_size(p, csa.CSA_WS_TOPK, 0, B, T, N)
+    ws = torch.empty((max(ws_bytes, 1),), dtype=torch.uint8, device="cuda")
+    out = torch.empty((B, T, k), dtype=torch.int32, device="cuda")
+    csa.csa_topk(p, B, T, N, torch.from_numpy(sc).cuda(), torch.from_numpy(pos).cuda(), out, ws,
+                 ws_bytes)
+    got = out.cpu().numpy()
+    for t in range(T):
+        nv = O.visible_entries(int(pos[0, t]), 4, N)
+        ref = O.topk_select(sc[0, t, :nv].astype(np.float64), k)
+        np.testing.assert_array_equal(got[0, t], ref, err_msg=f"t={t} N={N} k={k}")
+    assert csa.device_error() == 0
 
 
 @pytest.mark.parametrize("k", [512, 1024, 2000])
