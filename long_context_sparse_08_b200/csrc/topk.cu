@@ -255,31 +255,86 @@ __device__ __forceinline__ void find_bin(const int* hist, int nbins, int need, i
   __syncthreads();
 }
 
+// Ascending bitonic sort of arr[0..512) with one element per thread (512 threads): partners
+// closer than a warp are exchanged by shuffles, farther ones through `buf` (512 entries, one
+// barrier per such stage), so only 10 of the 45 stages wait on the block. On return
+// arr[i] holds the i-th smallest.
+__device__ __forceinline__ void bitonic_sort512(uint64_t* arr, uint64_t* buf) {
+  const int tid = threadIdx.x;
+  uint64_t x = arr[tid];
+  uint64_t* cur = arr;  // exchange buffer of the next cross-warp stage (alternates)
+#pragma unroll
+  for (int size = 2; size <= 512; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      uint64_t y;
+      if (stride >= 32) {
+        uint64_t* b = cur;
+        cur = cur == arr ? buf : arr;
+        __syncthreads();  // the previous readers of b are done
+        b[tid] = x;
+        __syncthreads();
+        y = b[tid ^ stride];
+      } else {
+        const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)x, stride);
+        const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(x >> 32), stride);
+        y = ((uint64_t)hi << 32) | lo;
+      }
+      const bool asc = (tid & size) == 0, lower = (tid & stride) == 0;
+      x = (lower == asc) ? (x < y ? x : y) : (x < y ? y : x);
+    }
+  }
+  __syncthreads();
+  arr[tid] = x;
+  __syncthreads();
+}
+
 template <typename TS>
 __global__ void __launch_bounds__(kRThreads, 2) k_topk_rows_smem(TopkArgs a, int vec) {
   extern __shared__ __align__(16) uint32_t kq[];  // the row's keys
   __shared__ __align__(16) uint64_t s_u[kMaxTopk];  // histogram (ints), then (key, index) pairs
+  __shared__ uint64_t s_sortbuf[kRThreads];
   __shared__ int wsum[kRThreads / 32];
-  __shared__ int s_bin, s_above, s_cnt;
+  __shared__ int s_bin, s_above;
   int* hist = reinterpret_cast<int*>(s_u);
   uint64_t* pairs = s_u;
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x;
   const int bt = blockIdx.x;
   const int64_t t = a.q_pos[bt];
+  const int n = (int)(t < 0 ? 0 : (t / a.m < a.n_cap ? t / a.m : a.n_cap));
+  const TS* sc = (sizeof(TS) == 4 ? static_cast<const TS*>(static_cast<const void*>(a.scores))
+                                  : static_cast<const TS*>(a.scores16)) + (size_t)bt * a.n_cap;
+  // fp32 rows in groups of 4 straight into shared memory; they land during the side job
+  const bool async_row = sizeof(TS) == 4 && vec;
+  if (async_row) {
+    const int ng = (n + 3) >> 2;
+    const uint32_t dst = (uint32_t)__cvta_generic_to_shared(kq);
+    for (int g = tid; g < ng; g += kRThreads)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 16 * g),
+                   "l"(reinterpret_cast<const float4*>(sc) + g)
+                   : "memory");
+  }
   if (a.qj.qhat != nullptr) {  // side job: this row's query heads for the attention
     __shared__ float s_cs[256], s_sn[256];
     qhat_rows(a.qj, bt, (double)t, 0, a.qj.H, s_cs, s_sn);
   }
-  const int n = (int)(t < 0 ? 0 : (t / a.m < a.n_cap ? t / a.m : a.n_cap));
-  const TS* sc = (sizeof(TS) == 4 ? static_cast<const TS*>(static_cast<const void*>(a.scores))
-                                  : static_cast<const TS*>(a.scores16)) + (size_t)bt * a.n_cap;
   int32_t* out = a.out_idx + (size_t)bt * a.k;
   const int k = a.k;
   int P = 1;
   while (P < k) P <<= 1;
 
-  // ---- keys into shared memory (groups of 4 by vector loads when rows are 16-byte aligned) ----
-  if (vec) {
+  // ---- keys into shared memory (groups of 4 by vector loads when rows are 16-byte aligned;
+  //      each thread converts the groups it copied) ----
+  if (async_row) {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    const int ng = (n + 3) >> 2;
+    for (int g = tid; g < ng; g += kRThreads) {
+      const uint4 x = reinterpret_cast<const uint4*>(kq)[g];
+      reinterpret_cast<uint4*>(kq)[g] =
+          make_uint4(float_key(__uint_as_float(x.x)), float_key(__uint_as_float(x.y)),
+                     float_key(__uint_as_float(x.z)), float_key(__uint_as_float(x.w)));
+    }
+  } else if (vec) {
     const int ng = (n + 3) >> 2;
 #pragma unroll 8
     for (int g = tid; g < ng; g += kRThreads) {
@@ -356,19 +411,22 @@ __global__ void __launch_bounds__(kRThreads, 2) k_topk_rows_smem(TopkArgs a, int
     }
   }
 
-  // ---- append: keys > T (or >= T when the whole tie group is taken), any order ----
-  if (tid == 0) s_cnt = 0;
-  __syncthreads();
-  for (int base = 0; base < n; base += kRThreads) {
-    const int i = base + tid;
-    const uint32_t u = i < n ? kq[i] : 0u;
-    const bool take = i < n && (ties ? u > T : u >= T);
-    const unsigned bal = __ballot_sync(0xffffffffu, take);
-    if (bal == 0) continue;
-    int pos = 0;
-    if (lane == __ffs(bal) - 1) pos = atomicAdd(&s_cnt, __popc(bal));
-    pos = __shfl_sync(0xffffffffu, pos, __ffs(bal) - 1) + __popc(bal & ((1u << lane) - 1u));
-    if (take) pairs[pos] = pack_desc(u, (uint32_t)i);
+  // ---- append: keys > T (or >= T when the whole tie group is taken), any order: each
+  //      thread counts its own, one block scan places them ----
+  {
+    const uint32_t Tl = ties ? T + 1u : T;  // take u >= Tl
+    const bool none = ties && T == 0xffffffffu;  // no key above the largest
+    int mine = 0;
+    for (int i = tid; i < n && !none; i += kRThreads) mine += kq[i] >= Tl ? 1 : 0;
+    int tot;
+    int pos = block_excl_scan_int(mine, wsum, &tot);
+    for (int i = tid; i < n && mine > 0; i += kRThreads) {
+      const uint32_t u = kq[i];
+      if (u >= Tl) {
+        pairs[pos++] = pack_desc(u, (uint32_t)i);
+        --mine;
+      }
+    }
   }
   if (ties) {  // the first kk keys == T in index order
     const int n_gt = k - kk;
@@ -382,9 +440,11 @@ __global__ void __launch_bounds__(kRThreads, 2) k_topk_rows_smem(TopkArgs a, int
       run += tot;
     }
   }
+  if (P <= kRThreads) P = kRThreads;  // one element per thread: the shuffle network
   for (int i = k + tid; i < P; i += kRThreads) pairs[i] = ~0ull;
   __syncthreads();
-  bitonic_sort(pairs, P);
+  if (P == kRThreads) bitonic_sort512(pairs, s_sortbuf);
+  else bitonic_sort(pairs, P);
   for (int i = tid; i < k; i += kRThreads) out[i] = (int32_t)(pairs[i] & 0xffffffffu);
 }
 
