@@ -181,10 +181,12 @@ __device__ __forceinline__ const __nv_bfloat16* row_src(const MqaArgs& a, int bt
 
 // Source of list entry j for the mixed-precision and / or paged variants: a cache row (bf16,
 // or c + r mixed bytes with its scale in *scale) found through the page table when kPaged,
-// or a bf16 window row (*scale = -1); nullptr when masked.
+// or a bf16 window row (*scale = -1); nullptr when masked. pg_hint >= -1: the entry's page
+// id, read earlier.
 template <bool kMixed, bool kPaged>
 __device__ __forceinline__ const void* row_src_ext(const MqaArgs& a, int bt, int b,
-                                                   const RowList& rl, int64_t j, float* scale) {
+                                                   const RowList& rl, int64_t j, float* scale,
+                                                   int32_t pg_hint = -2) {
   *scale = -1.f;
   if (j < rl.n_sel) {
     int64_t e = j;
@@ -193,7 +195,8 @@ __device__ __forceinline__ const void* row_src_ext(const MqaArgs& a, int bt, int
     if (e < 0 || e >= a.n_cap) return nullptr;
     size_t row = (size_t)b * a.n_cap + e;
     if constexpr (kPaged) {
-      const int32_t pg = a.page_table[(size_t)b * a.max_pages + e / a.page_rows];
+      const int32_t pg =
+          pg_hint >= -1 ? pg_hint : a.page_table[(size_t)b * a.max_pages + e / a.page_rows];
       if (pg < 0 || pg >= a.n_pages) {
         set_error(kErrPageId);
         return nullptr;
@@ -361,6 +364,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // started; returns whether TMA fills the slot) and the finish (cp.async copies: wait for
     // this thread's, make them visible to the tensor cores; then arrive). With two buffers the
     // next chunk is issued before this one's softmax and finished after it.
+    // dense paged lists: the page ids of the next chunk's rows are read one chunk ahead, so
+    // that resolving a chunk's rows waits on no page-table load
+    int pf_j = -1;
+    int32_t pf_pg = -2;
     auto gather_issue = [&](int j, int slot) -> bool {
       // ---- rows of chunk j into KV slot `slot`: thread r resolves row r, then warp w copies
       //      rows w, w+4, ... with lane = 16-byte chunk (coalesced 512 B per instruction) ----
@@ -370,9 +377,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tid < kRows) {
         if constexpr (kMixed || kPaged) {
           float sc;
-          my_src = static_cast<const __nv_bfloat16*>(
-              row_src_ext<kMixed, kPaged>(a, bt, b, rl, (int64_t)j * kRows + tid, &sc));
+          my_src = static_cast<const __nv_bfloat16*>(row_src_ext<kMixed, kPaged>(
+              a, bt, b, rl, (int64_t)j * kRows + tid, &sc, pf_j == j ? pf_pg : -2));
           if constexpr (kMixed) S.rscale[slot][tid] = sc;
+          if constexpr (kPaged) {
+            const int64_t e1 = (int64_t)(j + 1) * kRows + tid;
+            pf_pg = -2;
+            if (a.k == 0 && j + 1 < c1 && e1 < rl.n_vis && e1 < a.n_cap)
+              pf_pg = a.page_table[(size_t)b * a.max_pages + e1 / a.page_rows];
+            pf_j = j + 1;
+          }
         } else {
           my_src = row_src(a, bt, b, rl, (int64_t)j * kRows + tid);
         }
@@ -409,46 +423,61 @@ __global__ void __launch_bounds__(kThreads, 1)
           // a warp takes rows w, w+4, ...: a mixed row's lanes 0..27 widen 16 codes each
           // (dims 16*lane ..: atom lane / 4, chunks 2*(lane % 4) and +1), lanes 28..31 copy
           // two 16-byte chunks of its bf16 RoPE values (dims 448 + 8*q: atom 7, chunk q);
-          // a bf16 window row (scale -1) or a masked row is copied as in the bf16 path
+          // a bf16 window row (scale -1) or a masked row is copied as in the bf16 path. Four
+          // rows at a time: their code loads are all issued before any is widened, so the
+          // warp waits for one round trip per four rows.
           const int r = a.rope_dims, nope = kC - r;  // nope = 448 (c = 512, r = 64)
 #pragma unroll 1
-          for (int rr = warp; rr < kRows; rr += 4) {
-            const __nv_bfloat16* src = S.src[slot][rr];
-            const float sc = S.rscale[slot][rr];
-            if (src == nullptr || sc < 0.f) {
+          for (int rb = warp; rb < kRows; rb += 16) {  // rows rb, rb + 4, rb + 8, rb + 12
+            uint4 raw[4];
 #pragma unroll
-              for (int hseg = 0; hseg < 2; ++hseg) {
-                const int gch = lane + 32 * hseg;
-                const int atom = gch >> 3, c = gch & 7;
-                const uint32_t dst = kv_base + atom * (kRows * 128) + sw128(rr, c);
-                cp_async16(dst, src ? src + 8 * gch : static_cast<const __nv_bfloat16*>(a.kv),
-                           src != nullptr);
-              }
-            } else {
-              const uint8_t* row = reinterpret_cast<const uint8_t*>(src);
-              if (lane < nope / 16) {
-                const uint4 raw = __ldg(reinterpret_cast<const uint4*>(row) + lane);
-                const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-                uint32_t o8[8];
+            for (int q = 0; q < 4; ++q) {
+              const __nv_bfloat16* src = S.src[slot][rb + 4 * q];
+              raw[q] = make_uint4(0u, 0u, 0u, 0u);
+              if (src != nullptr && S.rscale[slot][rb + 4 * q] >= 0.f && lane < nope / 16)
+                raw[q] = __ldg(reinterpret_cast<const uint4*>(src) + lane);
+            }
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  o8[2 * q] = e4m3x2_scaled_bf16x2(w4[q] & 0xffffu, sc);
-                  o8[2 * q + 1] = e4m3x2_scaled_bf16x2(w4[q] >> 16, sc);
+            for (int q = 0; q < 4; ++q) {
+              const int rr = rb + 4 * q;
+              const __nv_bfloat16* src = S.src[slot][rr];
+              const float sc = S.rscale[slot][rr];
+              if (src == nullptr || sc < 0.f) {
+#pragma unroll
+                for (int hseg = 0; hseg < 2; ++hseg) {
+                  const int gch = lane + 32 * hseg;
+                  const int atom = gch >> 3, c = gch & 7;
+                  const uint32_t dst = kv_base + atom * (kRows * 128) + sw128(rr, c);
+                  cp_async16(dst, src ? src + 8 * gch : static_cast<const __nv_bfloat16*>(a.kv),
+                             src != nullptr);
                 }
-                uint8_t* at = kv_ptr + (lane >> 2) * (kRows * 128);
-                const int c8 = 2 * (lane & 3);
-                *reinterpret_cast<uint4*>(at + sw128(rr, c8)) = make_uint4(o8[0], o8[1], o8[2], o8[3]);
-                *reinterpret_cast<uint4*>(at + sw128(rr, c8 + 1)) =
-                    make_uint4(o8[4], o8[5], o8[6], o8[7]);
               } else {
-                const int q0 = 2 * (lane - nope / 16);  // RoPE chunks q0, q0 + 1 of r / 8
+                const uint8_t* row = reinterpret_cast<const uint8_t*>(src);
+                if (lane < nope / 16) {
+                  const uint32_t w4[4] = {raw[q].x, raw[q].y, raw[q].z, raw[q].w};
+                  uint32_t o8[8];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                  const int q = q0 + h;
-                  if (q < r / 8) {
-                    const int d = nope + 8 * q;
-                    const uint32_t dst = kv_base + (d >> 6) * (kRows * 128) + sw128(rr, (d & 63) >> 3);
-                    cp_async16(dst, row + nope + 16 * q, true);
+                  for (int e = 0; e < 4; ++e) {
+                    o8[2 * e] = e4m3x2_scaled_bf16x2(w4[e] & 0xffffu, sc);
+                    o8[2 * e + 1] = e4m3x2_scaled_bf16x2(w4[e] >> 16, sc);
+                  }
+                  uint8_t* at = kv_ptr + (lane >> 2) * (kRows * 128);
+                  const int c8 = 2 * (lane & 3);
+                  *reinterpret_cast<uint4*>(at + sw128(rr, c8)) =
+                      make_uint4(o8[0], o8[1], o8[2], o8[3]);
+                  *reinterpret_cast<uint4*>(at + sw128(rr, c8 + 1)) =
+                      make_uint4(o8[4], o8[5], o8[6], o8[7]);
+                } else {
+                  const int q0 = 2 * (lane - nope / 16);  // RoPE chunks q0, q0 + 1 of r / 8
+#pragma unroll
+                  for (int h = 0; h < 2; ++h) {
+                    const int qq = q0 + h;
+                    if (qq < r / 8) {
+                      const int d = nope + 8 * qq;
+                      const uint32_t dst =
+                          kv_base + (d >> 6) * (kRows * 128) + sw128(rr, (d & 63) >> 3);
+                      cp_async16(dst, row + nope + 16 * qq, true);
+                    }
                   }
                 }
               }
