@@ -249,6 +249,24 @@ __device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t (&r)[
       : "memory");
 }
 
+// 16 TMEM lanes x 64 columns of 32-bit, two threads per lane: thread t of the warp gets lane
+// (quadrant base + t / 4 + 8 (t % 2)) and, in register i, column 2 i + (t / 2) % 2 (the
+// layout checked on the device by writing known values through the 32x32b shape).
+__device__ __forceinline__ void tmem_ld_16x64b_x32(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x64b.x32.b32"
+      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15,"
+      " %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31},"
+      " [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -583,8 +601,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_trigger();
     bool ok = true;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
-    const bool head_thr = lane < 16;  // lanes 0-15: the softmax of head hh
-    const int hh = 16 * warp + (lane & 15);
+    // the M = 64 accumulator puts head 16w + i in TMEM lane 32w + i (i < 16); threads t and
+    // t ^ 2 of warp w share head 16w + t / 4 + 8 (t % 2), each holding every other row of a
+    // chunk (rows 2i + par)
+    const int par = (lane >> 1) & 1;
+    const int hh = 16 * warp + (lane >> 2) + 8 * (lane & 1);
     float mu_h = -INFINITY, l_h = 0.f;  // running max used and running sum of this head
     if (c0 < c1 && pend < 0) {
       pend_tma = gather_issue(c0, 0);
@@ -618,16 +639,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
 
-      // ---- softmax: lanes 0-15 of warp w own heads 16w .. 16w+15 (the M = 64 accumulator
-      //      puts row 16w + i in TMEM lane 32w + i); a thread holds its head's 128 row values ----
+      // ---- softmax: the two threads of head hh hold its rows 2i + par (i < R / 2); each
+      //      reduction is the thread's own values and one exchange with its partner ----
       ok = all_ok_softmax(mbar_wait(&S.s_full[slot], ph, kErrSFull));
       if (!ok) break;
       tc_fence_after();
-      constexpr int kHalves = kRows / 64;  // 64-row halves of a chunk
-      uint32_t sv[kHalves][64];
+      constexpr int kV = kRows / 2;  // values per thread
+      uint32_t sv[kV];
 #pragma unroll
-      for (int hv = 0; hv < kHalves; ++hv)
-        tmem_ld_32x32b_x64(lane_base + kColS + (kBuf == 2 ? 64 * slot : 0) + 64 * hv, sv[hv]);
+      for (int h = 0; h < kRows / 64; ++h)
+        tmem_ld_16x64b_x32(lane_base + kColS + (kBuf == 2 ? 64 * slot : 0) + 64 * h, sv + 32 * h);
       tmem_ld_wait();
       uint32_t vm[kRows / 32];
 #pragma unroll
@@ -638,26 +659,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < 8; ++i) cmx[i] = -INFINITY;
 #pragma unroll
-      for (int hv = 0; hv < kHalves; ++hv) {
-#pragma unroll
-        for (int r = 0; r < 64; ++r) {
-          const uint32_t w = vm[2 * hv + (r >> 5)];
-          const float x =
-              ((w >> (r & 31)) & 1u) ? __uint_as_float(sv[hv][r]) * a.scale : -INFINITY;
-          sv[hv][r] = __float_as_uint(x);
-          cmx[4 * hv + (r & 3)] = fmaxf(cmx[4 * hv + (r & 3)], x);
-        }
+      for (int i = 0; i < kV; ++i) {
+        const int rr = 2 * i + par;
+        const float x =
+            ((vm[rr >> 5] >> (rr & 31)) & 1u) ? __uint_as_float(sv[i]) * a.scale : -INFINITY;
+        sv[i] = __float_as_uint(x);
+        cmx[i & 7] = fmaxf(cmx[i & 7], x);
       }
-      const float cm = fmaxf(fmaxf(fmaxf(cmx[0], cmx[1]), fmaxf(cmx[2], cmx[3])),
-                             fmaxf(fmaxf(cmx[4], cmx[5]), fmaxf(cmx[6], cmx[7])));
+      float cm = fmaxf(fmaxf(fmaxf(cmx[0], cmx[1]), fmaxf(cmx[2], cmx[3])),
+                       fmaxf(fmaxf(cmx[4], cmx[5]), fmaxf(cmx[6], cmx[7])));
+      cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, 2));
       float al = 1.f;
       if (cm > mu_h + kLazy || (mu_h == -INFINITY && cm != -INFINITY)) {
         al = (mu_h == -INFINITY) ? 0.f : expf(mu_h - cm);
         mu_h = cm;
       }
       l_h *= al;
-      if (head_thr) S.alpha[hh] = al;
-      if (any_softmax(head_thr && al != 1.f && j > c0)) {
+      if (par == 0) S.alpha[hh] = al;
+      if (any_softmax(al != 1.f && j > c0)) {
         // rare: scale O^T columns by alpha (the previous O^T MMAs are done)
 #pragma unroll 1
         for (int cgrp = 0; cgrp < 16; ++cgrp) {  // 4 slices x 4 groups of 16 heads
@@ -673,26 +692,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st_wait();
       }
-      // P row of this head (bf16) into the K-major B tile: [row / 64][head][128 B]
-      if (head_thr) {
+      // P row of this head (bf16) into the K-major B tile [row / 64][head][128 B]. Per 16
+      // rows the even thread writes rows 0-7 and the odd thread rows 8-15: each hands its
+      // partner the four values the partner's 16-byte chunk needs.
+      {
         uint8_t* pt = base + kOffP + slot * L::kSlotP;
         float lc[4] = {0.f, 0.f, 0.f, 0.f};  // partial sums (sum what the MMA multiplies)
         const float mref = mu_h == -INFINITY ? 0.f : mu_h;  // no valid row yet: every p is 0
 #pragma unroll
-        for (int c8 = 0; c8 < kRows / 8; ++c8) {  // rows 8*c8 .. 8*c8+7
-          uint32_t pk[4];
+        for (int g = 0; g < kRows / 16; ++g) {
+          uint32_t bb[8];  // bf16 bits of rows 16g + 2m + par
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const __nv_bfloat16 bv = __float2bfloat16_rn(__expf(__uint_as_float(sv[8 * g + m]) - mref));
+            lc[m & 3] += __bfloat162float(bv);
+            bb[m] = (uint32_t)__bfloat16_as_ushort(bv);
+          }
+          const uint32_t s0 = par ? (bb[0] | (bb[1] << 16)) : (bb[4] | (bb[5] << 16));
+          const uint32_t s1 = par ? (bb[2] | (bb[3] << 16)) : (bb[6] | (bb[7] << 16));
+          const uint32_t r0 = __shfl_xor_sync(0xffffffffu, s0, 2);
+          const uint32_t r1 = __shfl_xor_sync(0xffffffffu, s1, 2);
+          const uint32_t pk[4] = {r0 & 0xffffu, r0 >> 16, r1 & 0xffffu, r1 >> 16};
+          uint32_t w[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const int r = 8 * c8 + 2 * k;
-            const float s0 = __uint_as_float(sv[r >> 6][r & 63]);
-            const float s1 = __uint_as_float(sv[(r + 1) >> 6][(r + 1) & 63]);
-            const __nv_bfloat16 b0 = __float2bfloat16_rn(__expf(s0 - mref));  // -inf -> 0
-            const __nv_bfloat16 b1 = __float2bfloat16_rn(__expf(s1 - mref));
-            lc[k] += __bfloat162float(b0) + __bfloat162float(b1);
-            pk[k] = (uint32_t)__bfloat16_as_ushort(b0) | ((uint32_t)__bfloat16_as_ushort(b1) << 16);
+            const uint32_t own = par ? bb[4 + k] : bb[k];
+            w[k] = par ? (pk[k] | (own << 16)) : (own | (pk[k] << 16));
           }
+          const int c8 = 2 * g + par;  // 16-byte chunk: rows 8 c8 .. 8 c8 + 7
           *reinterpret_cast<uint4*>(pt + (c8 >> 3) * (kHg * 128) + sw128(hh, c8 & 7)) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              make_uint4(w[0], w[1], w[2], w[3]);
         }
         l_h += (lc[0] + lc[1]) + (lc[2] + lc[3]);
       }
@@ -707,7 +736,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (pend >= 0) cp_async_wait_all();  // a wait gave up: no copy of this thread in flight
-    if (head_thr) {
+    l_h += __shfl_xor_sync(0xffffffffu, l_h, 2);  // the two halves of the head's sum
+    if (par == 0) {
       S.m_used[hh] = mu_h;
       S.l_sum[hh] = l_h;
     }
