@@ -771,16 +771,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                        : P.part + ((size_t)stream * P.nsplit + split) * (kHg * (kC + 2)) + 2 * kHg;
     __nv_bfloat16* out =
         single ? static_cast<__nv_bfloat16*>(a.out) + ((size_t)bt * a.H + h0) * kC : nullptr;
+    // O^T slice by slice (dims 128 sl + tid), G heads per TMEM load: all 64 with 64-row
+    // chunks; 16 with 128-row chunks, where four smaller loads between the stores measured
+    // faster (the one-chunk CTAs of the sparse decodes)
+    constexpr int G = kRows == 64 ? 64 : 16;
 #pragma unroll 1
-    for (int cgrp = 0; cgrp < 16; ++cgrp) {  // slice = cgrp / 4, heads 16*(cgrp%4) ..
-      const int sl = cgrp >> 2, hb = 16 * (cgrp & 3);
-      uint32_t o[16];
+    for (int cg = 0; cg < 4 * (64 / G); ++cg) {
+      const int sl = cg / (64 / G), hb = G * (cg % (64 / G));
+      uint32_t o[G];
       if (have) {
-        tmem_ld_x16(lane_base + kColO + 64 * sl + hb, o);
+        if constexpr (G == 64) tmem_ld_32x32b_x64(lane_base + kColO + 64 * sl, o);
+        else tmem_ld_x16(lane_base + kColO + 64 * sl + hb, o);
         tmem_ld_wait();
       } else {
 #pragma unroll
-        for (int h = 0; h < 16; ++h) o[h] = 0u;
+        for (int h = 0; h < G; ++h) o[h] = 0u;
       }
       const int d = 128 * sl + tid;
       if (single) {
@@ -791,7 +796,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           sn = -S.sn[(d - r0) >> 1];  // rotation by -t
         }
 #pragma unroll
-        for (int h = 0; h < 16; ++h) {
+        for (int h = 0; h < G; ++h) {
           const float y = __uint_as_float(o[h]) * S.fin[hb + h];
           const float yp = __shfl_xor_sync(0xffffffffu, y, 1);
           float z = y;
@@ -800,7 +805,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
 #pragma unroll
-        for (int h = 0; h < 16; ++h) po[(size_t)(hb + h) * kC + d] = __uint_as_float(o[h]);
+        for (int h = 0; h < G; ++h) po[(size_t)(hb + h) * kC + d] = __uint_as_float(o[h]);
       }
     }
   } else {
