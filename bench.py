@@ -582,6 +582,8 @@ def check_part_workload(part, s):
         want = "a CSA or HCA decode step"
     elif part == "kv_layouts" and s.kind not in ("csa_decode", "hca_decode"):
         want = "a CSA or HCA decode step"
+    elif part == "stream" and s.kind != "csa_decode":
+        want = "a CSA decode step (its indexer's key stream)"
     if want:
         raise SystemExit(f"--part {part} wants a workload with {want} "
                          f"(e.g. --workload pro_decode_1m); {s.name} has "
@@ -597,7 +599,10 @@ def run_part(args, W):
                       or, on an HCA workload, the dense form);
     bf16_scores       index + top-k with fp32 and with BF16 scores;
     forward_paged     the CSA (or HCA) layer over page pools and a window ring vs the
-                      contiguous one."""
+                      contiguous one;
+    stream            the device's own rate for one read of the indexer's key bytes (a torch
+                      reduction and a torch copy of that many bytes, no library kernel): the
+                      short-stream ceiling the indexer is compared with."""
     s = W.SHAPES[args.workload]
     check_part_workload(args.part, s)
     import torch
@@ -925,6 +930,34 @@ def run_part(args, W):
                                              "window": "ring"},
                     roofline={"bound": "hbm (key stream)", "peak": hbm, "peak_source": peak_src,
                               "unit": "GB/s"})
+    elif args.part == "stream":
+        n_vis = min(s.ctx // s.m, s.n_cap)
+        nbytes = s.B * s.T * n_vis * indexer_key_bytes(s)
+        n = nbytes // 4
+        n_rep = max(2, int(np.ceil(3 * L2_BYTES / nbytes)))
+        src = [torch.rand(n, device="cuda") for _ in range(n_rep)]
+        dst = [torch.empty(n, device="cuda") for _ in range(n_rep)]
+        sink = torch.empty(n_rep, device="cuda")
+
+        def read(i):
+            torch.sum(src[i], dim=0, out=sink[i])
+
+        def copy(i):
+            dst[i].copy_(src[i])
+
+        ms_read = _time_calls(read, n_rep, args.warmup, args.steps)
+        ms_copy = _time_calls(copy, n_rep, args.warmup, args.steps)
+        rd, cp = nbytes / (ms_read / 1e3) / 1e9, 2 * nbytes / (ms_copy / 1e3) / 1e9
+        line.update(metric="HBM rate of one stream of the indexer's key bytes",
+                    value=round(rd, 1), unit="GB/s (read)",
+                    bytes_per_stream=nbytes, replicas=n_rep,
+                    ms_per_stream={"read": round(ms_read, 5), "copy": round(ms_copy, 5)},
+                    copy_gbs=round(cp, 1),
+                    roofline={"bound": "hbm", "peak": hbm, "peak_source": peak_src,
+                              "unit": "GB/s", "read_frac": round(rd / hbm, 4),
+                              "copy_frac": round(cp / hbm, 4)},
+                    note="torch kernels (a sum and a copy), each call a whole stream; the "
+                         "indexer reads the same bytes in one launch")
     line["gpu_launches"] = int(csa.kernel_launches() - before)
     line["clocks"] = clocks.stop()
     line["device_error"] = csa.device_error()
@@ -933,7 +966,7 @@ def run_part(args, W):
 
 
 PARTS = {"out_proj", "state_append", "kv_layouts", "bf16_scores", "out_proj_prefill",
-         "forward_paged"}
+         "forward_paged", "stream"}
 
 
 def main():

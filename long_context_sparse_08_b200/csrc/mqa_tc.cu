@@ -960,11 +960,12 @@ bool make_map_rows(CUtensorMap* m, const void* ptr, int64_t rows, int box_rows) 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// CTAs per stream: as many as fill the SMs, at most one per 128 rows of the longest list.
-int choose_nsplit(const MqaArgs& a) {
+// CTAs per stream for chunks of R rows: as many as fill the SMs, at most one per chunk of
+// the longest list, at most 32.
+int splits_for(const MqaArgs& a, int R) {
   const int64_t streams = (int64_t)a.B * a.T * (a.H / kHg);
   const int64_t rows_max = (a.k > 0 ? a.k : a.n_cap) + a.n_win;
-  const int64_t chunks_max = (rows_max + 127) / 128;
+  const int64_t chunks_max = (rows_max + R - 1) / R;
   int64_t ns = device_sm_count() / (streams > 0 ? streams : 1);
   if (ns < 1) ns = 1;
   if (ns > chunks_max) ns = chunks_max > 0 ? chunks_max : 1;
@@ -973,14 +974,21 @@ int choose_nsplit(const MqaArgs& a) {
 }
 
 // Rows per chunk: 64, with two buffers, when a CTA walks two or more chunks of 128 (dense
-// HCA lists, prefill: the next chunk's rows land during this one's softmax); 128 with one
-// buffer when it takes a single chunk (sparse decode).
+// HCA lists, prefill: the next chunk's rows land during this one's softmax), or when
+// 64-row chunks spread a short list over more CTAs and at most 12 partial states per
+// stream (Flash decode: 10 CTAs of one chunk each instead of 5); otherwise 128 with one
+// buffer (Pro decode, where 64-row chunks would make 18 partials per stream and the merge
+// measured slower than the shorter chain saves).
 int choose_rows(const MqaArgs& a) {
   const int64_t rows_max = (a.k > 0 ? a.k : a.n_cap) + a.n_win;
   const int64_t chunks = (rows_max + 127) / 128;
-  const int ns = choose_nsplit(a);
-  return (chunks + ns - 1) / ns >= 2 ? 64 : 128;
+  const int ns = splits_for(a, 128);
+  if ((chunks + ns - 1) / ns >= 2) return 64;
+  const int ns64 = splits_for(a, 64);
+  return ns64 > ns && ns64 <= 12 ? 64 : 128;
 }
+
+int choose_nsplit(const MqaArgs& a) { return splits_for(a, choose_rows(a)); }
 
 }  // namespace
 
